@@ -1,0 +1,450 @@
+"""Benchmark of paged split-KV decode attention on B200.
+
+One step = one decode-attention call (split kernel + combine kernel) over one
+batch of synthetic decode queries against a paged bf16 KV cache, through the
+C-ABI library.  Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|long|ragged|tiny]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host cores
+
+Metric: achieved HBM bandwidth over algorithmic bytes (KV bytes that must be read
++ q bytes + out bytes) per call, in GB/s, with the µs/call beside it.  Inputs
+are resident in HBM before the timed region.  Two independent instances of the
+workload (different seeds, each larger than L2 for the large workloads) are used
+in turn, so every call reads KV that the previous call did not touch.
+
+Several GPUs (one process each, under torchrun): every rank runs its own batch
+of the same shape (independent decode problems, no collective on the data path);
+the value is the bytes of all ranks divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention achieved HBM GB/s (algorithmic KV+q+out bytes per call / time)"
+UNIT = "GB/s"
+DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000}
+CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=sorted(workloads.NAMED), default="llama8b")
+    p.add_argument("--num-splits", type=int, default=0, help="0 = auto (the default launch configuration)")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    p.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks")
+    a = p.parse_args(argv)
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+# ---------------------------------------------------------------- ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return world, rank, local
+
+
+def init_group(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- inputs
+def make_instances(name: str, rank: int, count: int = 2):
+    """`count` independent instances of the named workload; seeds differ per rank and instance."""
+    gen = workloads.NAMED[name]
+    base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262}[name]
+    return [gen(seed=base + 1000003 * rank + i) for i in range(count)]
+
+
+class Resident:
+    """A workload's tensors resident on the device, plus its workspace."""
+
+    def __init__(self, w, device, num_splits, apd):
+        self.w = w
+        self.q = w.q.to(device)
+        self.k = w.k_cache.contiguous().to(device)
+        self.v = w.v_cache.contiguous().to(device)
+        self.page_table = w.page_table.to(device)
+        self.seq_lens = w.seq_lens.to(device)
+        self.out = torch.empty_like(self.q)
+        self.num_splits = num_splits
+        self.ws = apd.alloc_workspace(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, num_splits,
+                                      device=device)
+        self.bytes = w.algorithmic_bytes()
+
+    def call(self, apd, stream, **kw):
+        apd.attn_paged_decode(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, self.w.scale,
+                              self.num_splits, self.ws, stream=stream, **kw)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, enabled: bool = True):
+        self.proc = None
+        self.path = None
+        if not enabled:
+            return
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        import tempfile
+
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, r in rows:
+            for n, v in zip(names[1:], r[1:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- measurement legs
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(CSRC, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """dram read+write bytes per split-kernel launch from the committed ncu capture,
+    or None when the capture is missing, for another workload, or the kernel changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_sha") != kernel_source_sha() or t.get("workload") != workload:
+        return None
+    return t.get("dram_bytes_per_launch")
+
+
+def time_steps(insts, apd, stream, steps, split_events=False):
+    """Run `steps` calls rotating over the instances; returns (elapsed_s, mean split-kernel s or None)."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    per = []
+    if split_events:
+        per = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start.record(stream)
+    for i in range(steps):
+        inst = insts[i % len(insts)]
+        if split_events:
+            b, m = per[i]
+            b.record(stream)
+            inst.call(apd, stream, split_done_event=m)
+        else:
+            inst.call(apd, stream)
+    end.record(stream)
+    end.synchronize()
+    elapsed = start.elapsed_time(end) / 1e3
+    split = None
+    if split_events:
+        split = sum(b.elapsed_time(m) for b, m in per) / 1e3 / steps
+    return elapsed, split
+
+
+def e2e_steps(insts, apd, stream, steps):
+    """Per step: pinned-host -> device copies of q, page_table, seq_lens; the call;
+    device -> pinned-host copy of out.  Returns (elapsed_s, h2d bytes, d2h bytes) per step."""
+    hosts = []
+    for inst in insts:
+        hosts.append({
+            "q": inst.w.q.pin_memory(), "pt": inst.w.page_table.pin_memory(), "sl": inst.w.seq_lens.pin_memory(),
+            "out": torch.empty(inst.out.shape, dtype=inst.out.dtype).pin_memory(),
+        })
+    h2d = insts[0].q.nbytes + insts[0].page_table.nbytes + insts[0].seq_lens.nbytes
+    d2h = insts[0].out.nbytes
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(steps):
+            inst, h = insts[i % len(insts)], hosts[i % len(insts)]
+            inst.q.copy_(h["q"], non_blocking=True)
+            inst.page_table.copy_(h["pt"], non_blocking=True)
+            inst.seq_lens.copy_(h["sl"], non_blocking=True)
+            inst.call(apd, stream)
+            h["out"].copy_(inst.out, non_blocking=True)
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3, h2d, d2h
+
+
+def oracle_baseline(w, min_seconds: float = 10.0, max_calls: int = 50):
+    """The fp64 CPU oracle on the whole workload, repeated until about min_seconds."""
+    import oracle
+
+    oracle.paged_decode(w)  # loads the library and faults in the pages once
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        oracle.paged_decode(w)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or calls >= max_calls:
+            break
+    return {"value": w.algorithmic_bytes() * calls / el / 1e9, "unit": UNIT, "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"the whole {w.name} workload (all {w.batch * w.num_q_heads} query rows), {calls} calls, "
+                      f"{el:.1f} s, fp64, OpenMP over rows"}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(a):
+    """The reference arm: the fp64 CPU oracle, each step a bounded sample of the workload."""
+    world, rank, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    import oracle
+
+    w = make_instances(a.workload, 0, 1)[0]
+    B, Hq = w.batch, w.num_q_heads
+    row_tokens = w.seq_lens.to(torch.int64)
+    total_row_tokens = float(row_tokens.sum()) * Hq
+
+    def step(i):
+        b = i % B
+        rows = [(b, h) for h in range(Hq)]
+        oracle.paged_decode_rows(w, rows)
+        return w.algorithmic_bytes() * float(row_tokens[b]) * Hq / max(total_row_tokens, 1.0)
+
+    for i in range(a.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    done = 0.0
+    for i in range(a.steps):
+        done += step(a.warmup + i)
+    el = time.perf_counter() - t0
+    value = done / el / 1e9
+    cores = oracle.max_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": a.gpus, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, a),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the {Hq} query rows of one sequence of {w.name} (rotating over "
+                                   f"the {B} sequences), fp64 CPU oracle on {cores} threads"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, a):
+    d = w.describe()
+    d.pop("seed", None)
+    return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "page_size": w.page_size, "kv_tokens": w.kv_tokens(),
+            "num_splits": a.num_splits, "layout": w.layout,
+            "l2": "two independent instances used in turn (each call reads KV the previous call did not touch); "
+                  "large workloads are each larger than L2",
+            "algorithmic_bytes_per_call": w.algorithmic_bytes()}
+
+
+def run_ours(a):
+    world, rank, local = dist_env()
+    if a.gpus != world and world > 1:
+        print(f"--gpus {a.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
+    if a.gpus > 1 and world == 1:
+        print("--gpus N>1 needs torchrun (one process per GPU)", file=sys.stderr)
+        return 2
+    if not torch.cuda.is_available():
+        print("no CUDA device", file=sys.stderr)
+        return 2
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_group(world, "nccl")
+    import decode_attention_paged_split_b200 as apd
+
+    insts = [Resident(w, device, a.num_splits, apd) for w in make_instances(a.workload, rank, 2)]
+    w0 = insts[0].w
+    plan = apd.query_plan(w0.batch, w0.num_q_heads, w0.num_kv_heads, w0.head_dim, a.num_splits)
+    launches_per_step = 1 + (1 if plan.combine_ctas > 0 else 0)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+
+    # warm-up
+    time_steps(insts, apd, stream, a.warmup)
+
+    # main timed region
+    clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    elapsed, _ = time_steps(insts, apd, stream, a.steps)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    clock_info = clocks.stop()
+    bytes_rank = sum(insts[i % 2].bytes for i in range(a.steps))
+    t_max = max_over_ranks(elapsed, dist, device)
+    bytes_all = sum_over_ranks(float(bytes_rank), dist, device)
+    value = bytes_all / t_max / 1e9
+
+    # split-kernel duration: the same steps with an event between the two kernels
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    _, split_s = time_steps(insts, apd, stream, a.steps, split_events=True)
+    torch.cuda.synchronize(device)
+    split_s = max_over_ranks(split_s, dist, device)
+
+    # end to end through host buffers
+    e2e = None
+    if not a.no_e2e:
+        time_steps(insts, apd, stream, 3)
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        e_el, h2d, d2h = e2e_steps(insts, apd, stream, a.steps)
+        torch.cuda.synchronize(device)
+        e_max = max_over_ranks(e_el, dist, device)
+        e2e = {"value": bytes_all / e_max / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_max / a.steps * 1e3}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = oracle_baseline(w0)
+
+    if rank == 0:
+        peak, peak_src = peaks()
+        mean_bytes = bytes_rank / a.steps
+        achieved = mean_bytes / split_s / 1e9
+        traffic = committed_traffic(a.workload)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": t_max / a.steps * 1e3, "us_per_call": t_max / a.steps * 1e6,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": config_of(w0, a),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                         "kernel": "split_kernel", "kernel_us": split_s * 1e6,
+                         "call_frac_of_peak": value / world / peak},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * a.steps,
+            "clocks": clock_info,
+            "plan": {"mode": plan.mode, "workers": plan.num_workers, "ctas": plan.grid_ctas,
+                     "warps_per_cta": plan.warps_per_cta, "stages": plan.stages, "smem": plan.smem_bytes},
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    a = parse_args(argv)
+    if a.impl == "reference":
+        return run_reference(a)
+    return run_ours(a)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

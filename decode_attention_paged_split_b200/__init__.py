@@ -1,0 +1,261 @@
+"""Python binding of libattn_paged_decode.so: paged split-KV decode attention on B200.
+
+Argument marshalling only.  Every step of the computation runs in the library's
+CUDA kernels; PyTorch supplies device memory and the current stream.  There is
+no CPU fallback: if the library is missing or fails to load, every call raises.
+
+The operation (AstrAI commit d565d44c, ``csrc/kernels/attn_paged_decode.cu``,
+commit log): single-token decode attention over a paged bf16 KV cache with
+grouped-query attention, split-KV partials (o_part / ml_part) and one combine
+kernel.  The C declarations, with argument meaning, layout, ownership and error
+behaviour, are in ``include/attn_paged_decode.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "APDError",
+    "attn_paged_decode",
+    "workspace_size",
+    "alloc_workspace",
+    "workspace_init",
+    "read_device_flags",
+    "query_plan",
+    "status_string",
+    "library_path",
+    "FLAG_PAGE_OUT_OF_RANGE",
+    "FLAG_SEQ_LEN_CLAMPED",
+    "FLAG_SEQ_LEN_NEGATIVE",
+    "FLAG_WAIT_TIMEOUT",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libattn_paged_decode.so")
+
+DTYPE_BF16, DTYPE_INT32, DTYPE_FP32 = 1, 2, 3
+FLAG_PAGE_OUT_OF_RANGE = 0x1
+FLAG_SEQ_LEN_CLAMPED = 0x2
+FLAG_SEQ_LEN_NEGATIVE = 0x4
+FLAG_WAIT_TIMEOUT = 0x8
+
+_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.int32: DTYPE_INT32, torch.float32: DTYPE_FP32}
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("ndim", ctypes.c_int32),
+        ("shape", ctypes.c_int64 * 4),
+        ("stride", ctypes.c_int64 * 4),
+    ]
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [
+        ("mode", ctypes.c_int32),
+        ("num_workers", ctypes.c_int32),
+        ("grid_ctas", ctypes.c_int32),
+        ("warps_per_cta", ctypes.c_int32),
+        ("stages", ctypes.c_int32),
+        ("rows_per_unit", ctypes.c_int32),
+        ("head_blocks", ctypes.c_int32),
+        ("combine_ctas", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int64),
+        ("partial_slots", ctypes.c_int64),
+        ("workspace_bytes", ctypes.c_int64),
+    ]
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [
+        ("split_done_event", ctypes.c_void_p),
+        ("disable_pdl", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class APDError(RuntimeError):
+    """A non-zero apd_status returned by the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: status {status} ({status_string(status)})"
+        if status == 11:  # APD_ERR_CUDA
+            msg += f": {_load().apd_last_cuda_error().decode(errors='replace')}"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"{_LIB_PATH} is missing: build it with `python -m decode_attention_paged_split_b200.build` "
+            "(there is no fallback implementation)")
+    L = ctypes.CDLL(_LIB_PATH)
+    T = ctypes.POINTER(_Tensor)
+    L.apd_workspace_size.argtypes = [ctypes.c_int] * 5
+    L.apd_workspace_size.restype = ctypes.c_size_t
+    L.apd_workspace_init.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    L.apd_workspace_init.restype = ctypes.c_int
+    L.apd_attn_paged_decode.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_size_t, ctypes.c_void_p]
+    L.apd_attn_paged_decode.restype = ctypes.c_int
+    L.apd_attn_paged_decode_ex.argtypes = L.apd_attn_paged_decode.argtypes + [ctypes.POINTER(_Options)]
+    L.apd_attn_paged_decode_ex.restype = ctypes.c_int
+    L.apd_read_device_flags.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                        ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+    L.apd_read_device_flags.restype = ctypes.c_int
+    L.apd_query_plan.argtypes = [ctypes.c_int] * 5 + [ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_Plan)]
+    L.apd_query_plan.restype = ctypes.c_int
+    L.apd_status_string.argtypes = [ctypes.c_int]
+    L.apd_status_string.restype = ctypes.c_char_p
+    L.apd_last_cuda_error.argtypes = []
+    L.apd_last_cuda_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def lib():
+    """The loaded ctypes library (raises if it is missing)."""
+    return _load()
+
+
+def status_string(status: int) -> str:
+    return _load().apd_status_string(int(status)).decode()
+
+
+def _desc(t: torch.Tensor | None) -> _Tensor:
+    d = _Tensor()
+    if t is None:
+        return d
+    if t.dim() > 4:
+        raise ValueError("tensors passed to the library have at most 4 dimensions")
+    d.data = t.data_ptr() if t.numel() > 0 or t.data_ptr() else None
+    d.dtype = _DTYPES.get(t.dtype, 0)
+    d.ndim = t.dim()
+    for i in range(t.dim()):
+        d.shape[i] = t.shape[i]
+        d.stride[i] = t.stride(i)
+    return d
+
+
+def _stream_handle(stream, device) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream or None
+    return int(stream) or None
+
+
+def workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0) -> int:
+    """Bytes of workspace a call with these arguments needs (raises on invalid arguments)."""
+    n = _load().apd_workspace_size(batch, num_q_heads, num_kv_heads, head_dim, num_splits)
+    if n == 0:
+        raise ValueError("invalid arguments for apd_workspace_size "
+                         f"(batch={batch}, Hq={num_q_heads}, Hkv={num_kv_heads}, D={head_dim}, splits={num_splits})")
+    return int(n)
+
+
+def alloc_workspace(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,
+                    device="cuda") -> torch.Tensor:
+    """A zeroed uint8 device buffer of workspace_size(...) bytes (torch allocations are 256-byte aligned)."""
+    n = workspace_size(batch, num_q_heads, num_kv_heads, head_dim, num_splits)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    rc = _load().apd_workspace_init(workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                    _stream_handle(stream, workspace.device))
+    if rc:
+        raise APDError(rc, "apd_workspace_init")
+
+
+def attn_paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                      seq_lens: torch.Tensor, out: torch.Tensor, scale: float, num_splits: int = 0,
+                      workspace: torch.Tensor | None = None, stream=None, split_done_event=None,
+                      disable_pdl: bool = False) -> torch.Tensor:
+    """out[b, h, :] = softmax(scale * q[b, h] . K_b^T) V_b over the paged cache; returns ``out``.
+
+    q bf16 [B, Hq, D]; k_cache / v_cache bf16 [num_pages, page_size, Hkv, D] (any strides
+    with D contiguous); page_table int32 [B, max_pages]; seq_lens int32 [B]; out bf16 [B, Hq, D].
+    ``workspace``: a device buffer of at least workspace_size(...) bytes; preallocate it once
+    (allocating here, when it is None, makes the call not capturable in a CUDA graph).
+    ``split_done_event``: optional torch.cuda.Event recorded right after the split kernel.
+    """
+    L = _load()
+    if workspace is None:
+        workspace = alloc_workspace(q.shape[0], q.shape[1], k_cache.shape[2], q.shape[2], num_splits,
+                                    device=q.device)
+    descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+    ptrs = [ctypes.byref(d) for d in descs]
+    st = _stream_handle(stream, q.device)
+    ws_ptr = workspace.data_ptr()
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if split_done_event is None and not disable_pdl:
+        rc = L.apd_attn_paged_decode(*ptrs, ctypes.c_float(scale), int(num_splits), ws_ptr, ws_bytes, st)
+    else:
+        opts = _Options()
+        if split_done_event is not None:
+            if not split_done_event.cuda_event:  # torch creates its events lazily, at the first record
+                split_done_event.record(torch.cuda.current_stream(q.device) if stream is None else stream)
+            opts.split_done_event = split_done_event.cuda_event
+        opts.disable_pdl = 1 if disable_pdl else 0
+        rc = L.apd_attn_paged_decode_ex(*ptrs, ctypes.c_float(scale), int(num_splits), ws_ptr, ws_bytes, st,
+                                        ctypes.byref(opts))
+    if rc:
+        raise APDError(rc, "apd_attn_paged_decode")
+    return out
+
+
+def read_device_flags(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return the sticky APD_FLAG_* word of the workspace."""
+    flags = ctypes.c_uint32(0)
+    rc = _load().apd_read_device_flags(workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                       _stream_handle(stream, workspace.device), ctypes.byref(flags),
+                                       1 if clear else 0)
+    if rc:
+        raise APDError(rc, "apd_read_device_flags")
+    return int(flags.value)
+
+
+@dataclass
+class Plan:
+    mode: int
+    num_workers: int
+    grid_ctas: int
+    warps_per_cta: int
+    stages: int
+    rows_per_unit: int
+    head_blocks: int
+    combine_ctas: int
+    smem_bytes: int
+    partial_slots: int
+    workspace_bytes: int
+
+
+def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,
+               workspace_bytes: int | None = None, sm_count: int = 0) -> Plan:
+    """How the library would launch this problem (sm_count > 0: for a device with that
+    many SMs, computed on the host; 0: for the current CUDA device)."""
+    p = _Plan()
+    wb = ctypes.c_size_t(-1).value if workspace_bytes is None else int(workspace_bytes)
+    rc = _load().apd_query_plan(batch, num_q_heads, num_kv_heads, head_dim, num_splits, wb, int(sm_count),
+                                ctypes.byref(p))
+    if rc:
+        raise APDError(rc, "apd_query_plan")
+    return Plan(**{name: int(getattr(p, name)) for name, _ in _Plan._fields_})

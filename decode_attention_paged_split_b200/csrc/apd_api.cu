@@ -1,0 +1,553 @@
+// apd_api.cu -- the C ABI of libattn_paged_decode.so: argument validation,
+// launch planning, TMA descriptor encoding and the two kernel launches.
+//
+// The entry point and its checks follow the AstrAI commit log of
+// csrc/kernels/attn_paged_decode.cu: a thin binding that validates
+// q_head % kv_head == 0 and head-dim contiguity, checks the split-KV scratch
+// and output layout, runs on the caller's stream, and never allocates inside a
+// decode step (the partials live in a preallocated workspace, which is what lets
+// the decode step be captured in a CUDA graph).
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn_paged_decode.h"
+#include "apd_kernels.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[512] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", what, cudaGetErrorString(e));
+    return APD_ERR_CUDA;
+}
+
+int driver_fail(int code, const char* what) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: CUresult %d", what, code);
+    return APD_ERR_CUDA;
+}
+
+constexpr size_t kSmemLimit = 232448;  // sm_100a: 227 KB of opt-in shared memory per block
+constexpr size_t kWsAlign = 256;
+constexpr int kDefaultSmCount = 148;   // B200
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Traits {
+    int stages;
+    int max_warps;
+};
+
+Traits traits_for(int D) {
+    switch (D) {
+        case 32: return {4, 8};
+        case 64: return {4, 8};
+        case 128: return {3, 6};
+        default: return {2, 4};
+    }
+}
+
+bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
+
+struct Shape {
+    int B, Hq, Hkv, D, g, HB, rows_max;
+    int64_t units;  // B * Hkv * HB
+};
+
+int make_shape(int B, int Hq, int Hkv, int D, Shape* s) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0) return APD_ERR_SHAPE;
+    if (Hq % Hkv != 0) return APD_ERR_GQA;
+    if (!head_dim_ok(D)) return APD_ERR_HEAD_DIM;
+    if (B > APD_MAX_BATCH) return APD_ERR_TOO_LARGE;
+    s->B = B;
+    s->Hq = Hq;
+    s->Hkv = Hkv;
+    s->D = D;
+    s->g = Hq / Hkv;
+    s->HB = (s->g + apd::kMaxRows - 1) / apd::kMaxRows;
+    s->rows_max = s->g < apd::kMaxRows ? s->g : apd::kMaxRows;
+    s->units = static_cast<int64_t>(B) * Hkv * s->HB;
+    return APD_OK;
+}
+
+uint32_t q_tile_bytes(const Shape& s) { return static_cast<uint32_t>(align_up(static_cast<size_t>(s.rows_max) * s.D * 2, 1024)); }
+uint32_t stage_bytes(const Shape& s) { return 2u * apd::kTile * s.D * 2u + q_tile_bytes(s); }
+
+size_t smem_bytes(const Shape& s, int warps, int stages) {
+    const size_t meta = 8ull * warps * stages + 4ull * (2ull * s.B + 1);
+    return align_up(meta, 16) + 1024 + static_cast<size_t>(warps) * stages * stage_bytes(s);
+}
+
+int warps_for(const Shape& s) {
+    const Traits t = traits_for(s.D);
+    for (int w = t.max_warps; w >= 1; --w)
+        if (smem_bytes(s, w, t.stages) <= kSmemLimit) return w;
+    return 0;
+}
+
+// Workspace: [flags header 256 B][cum (B+1) int32][o_part][ml_part], each 256-aligned.
+size_t ws_head_bytes(const Shape& s) { return kWsAlign + align_up(4ull * (s.B + 1), kWsAlign); }
+size_t ws_bytes_for(const Shape& s, int64_t slots) {
+    return ws_head_bytes(s) + align_up(static_cast<size_t>(slots) * s.rows_max * s.D * 4, kWsAlign) +
+           align_up(static_cast<size_t>(slots) * s.rows_max * 2 * 4, kWsAlign);
+}
+int64_t slots_fitting(const Shape& s, size_t bytes) {
+    if (bytes < ws_head_bytes(s)) return -1;
+    const size_t per = static_cast<size_t>(s.rows_max) * (s.D + 2) * 4;
+    int64_t n = static_cast<int64_t>((bytes - ws_head_bytes(s)) / per);
+    while (n > 0 && ws_bytes_for(s, n) > bytes) --n;
+    return n;
+}
+
+struct Plan {
+    int mode, ksplit, workers, ctas, warps, stages, combine_ctas;
+    size_t smem;
+    int64_t slots;
+    size_t ws_needed;
+};
+
+// tiles_bound: an upper bound on the number of tiles (host-known), or -1.
+int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl) {
+    if (num_splits < 0) return APD_ERR_NUM_SPLITS;
+    const Traits t = traits_for(s.D);
+    pl->stages = t.stages;
+    pl->warps = warps_for(s);
+    if (pl->warps < 1) return APD_ERR_TOO_LARGE;
+    pl->smem = smem_bytes(s, pl->warps, pl->stages);
+    if (num_splits == 0) {
+        pl->mode = 0;
+        pl->ksplit = 0;
+        int64_t workers = static_cast<int64_t>(sm_count) * pl->warps;
+        if (tiles_bound >= 0 && workers > tiles_bound) workers = tiles_bound > 0 ? tiles_bound : 1;
+        if (ws_bytes != SIZE_MAX) {
+            const int64_t cap = slots_fitting(s, ws_bytes) / 2;
+            if (cap < 1) return APD_ERR_WORKSPACE;
+            if (workers > cap) workers = cap;
+        }
+        pl->workers = static_cast<int>(workers);
+        pl->slots = 2 * workers;
+        pl->combine_ctas = static_cast<int>(s.units);
+    } else {
+        pl->mode = 1;
+        pl->ksplit = num_splits;
+        const int64_t workers = s.units * num_splits;
+        if (workers > INT32_MAX / 2) return APD_ERR_TOO_LARGE;
+        pl->workers = static_cast<int>(workers);
+        pl->slots = num_splits >= 2 ? workers : 0;
+        pl->combine_ctas = num_splits >= 2 ? static_cast<int>(s.units) : 0;
+    }
+    pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
+    pl->ws_needed = ws_bytes_for(s, pl->slots);
+    if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
+    return APD_OK;
+}
+
+// ---------------------------------------------------------------- devices
+struct DeviceState {
+    bool init = false;
+    int sm_count = 0;
+    bool smem_attr_set[4] = {false, false, false, false};
+};
+std::mutex g_mu;
+DeviceState g_devices[128];
+
+int device_state(DeviceState** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 128) return APD_ERR_ARGUMENT;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& d = g_devices[dev];
+    if (!d.init) {
+        e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(MultiProcessorCount)");
+        d.init = true;
+    }
+    *out = &d;
+    return APD_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// ---------------------------------------------------------------- validation
+bool is_null(const apd_tensor* t) { return t == nullptr || t->data == nullptr; }
+
+// Strides with extent-1 dimensions replaced by the contiguous value, so that
+// any stride a framework reports for a broadcast / size-1 dim is accepted.
+void normalized_strides(const apd_tensor* t, int64_t* st) {
+    int64_t inner = 1;
+    for (int i = t->ndim - 1; i >= 0; --i) {
+        st[i] = (t->shape[i] == 1) ? inner : t->stride[i];
+        inner *= t->shape[i];
+    }
+}
+
+// Head dim contiguous, every other stride positive and a multiple of 8
+// elements (16 bytes), base 16-byte aligned.
+bool aligned_bf16_layout(const apd_tensor* t, int64_t* st) {
+    normalized_strides(t, st);
+    if (st[t->ndim - 1] != 1) return false;
+    for (int i = 0; i < t->ndim - 1; ++i)
+        if (st[i] <= 0 || st[i] % 8 != 0 || st[i] * 2 >= (1ll << 40)) return false;
+    return (reinterpret_cast<uintptr_t>(t->data) & 15u) == 0;
+}
+
+struct Validated {
+    Shape s;
+    int P, NP, MP;
+    int64_t qst[3], kst[4], vst[4], ost[3], pst[2];
+};
+
+int validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* pt,
+             const apd_tensor* sl, const apd_tensor* out, int num_splits, Validated* V) {
+    if (is_null(q) || is_null(k) || is_null(v) || is_null(pt) || is_null(sl) || is_null(out))
+        return APD_ERR_NULL_POINTER;
+    if (q->dtype != APD_DTYPE_BF16 || k->dtype != APD_DTYPE_BF16 || v->dtype != APD_DTYPE_BF16 ||
+        out->dtype != APD_DTYPE_BF16 || pt->dtype != APD_DTYPE_INT32 || sl->dtype != APD_DTYPE_INT32)
+        return APD_ERR_DTYPE;
+    if (q->ndim != 3 || out->ndim != 3 || k->ndim != 4 || v->ndim != 4 || pt->ndim != 2 || sl->ndim != 1)
+        return APD_ERR_SHAPE;
+    for (int i = 0; i < 4; ++i)
+        if (k->shape[i] != v->shape[i] || k->shape[i] <= 0) return APD_ERR_SHAPE;
+    for (int i = 0; i < 3; ++i)
+        if (q->shape[i] != out->shape[i] || q->shape[i] < 0) return APD_ERR_SHAPE;
+    const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+    const int64_t NP = k->shape[0], P = k->shape[1], Hkv = k->shape[2];
+    if (k->shape[3] != D || pt->shape[0] != B || sl->shape[0] != B || pt->shape[1] <= 0) return APD_ERR_SHAPE;
+    if (Hq <= 0 || D <= 0) return APD_ERR_SHAPE;
+    if (Hq > INT32_MAX || Hkv > INT32_MAX || NP > INT32_MAX || P > INT32_MAX || pt->shape[1] > INT32_MAX)
+        return APD_ERR_TOO_LARGE;
+    if (B > APD_MAX_BATCH) return APD_ERR_TOO_LARGE;
+    int rc = make_shape(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D), &V->s);
+    if (rc) return rc;
+    if (P % apd::kTile != 0) return APD_ERR_PAGE_SIZE;
+    if (num_splits < 0) return APD_ERR_NUM_SPLITS;
+    if (!aligned_bf16_layout(q, V->qst) || !aligned_bf16_layout(out, V->ost) || !aligned_bf16_layout(k, V->kst) ||
+        !aligned_bf16_layout(v, V->vst))
+        return APD_ERR_LAYOUT;
+    normalized_strides(pt, V->pst);
+    if (V->pst[0] < 0 || V->pst[1] < 0 || (reinterpret_cast<uintptr_t>(pt->data) & 3u)) return APD_ERR_LAYOUT;
+    int64_t sst[1];
+    normalized_strides(sl, sst);
+    if (sst[0] != 1 || (reinterpret_cast<uintptr_t>(sl->data) & 3u)) return APD_ERR_LAYOUT;
+    // flattened tile indices must fit in int32 on the device
+    const int64_t tiles_bound = V->s.units * pt->shape[1] * (P / apd::kTile);
+    if (tiles_bound >= INT32_MAX / 2) return APD_ERR_TOO_LARGE;
+    V->P = static_cast<int>(P);
+    V->NP = static_cast<int>(NP);
+    V->MP = static_cast<int>(pt->shape[1]);
+    return APD_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+// K/V: D >= 64 -> 5-D view {64, D/64, Hkv, P, NP}, box {64, D/64, 1, 32, 1},
+//      128-byte swizzle (one box = one [32 x D] tile, rows of 2*D bytes).
+//      D == 32 -> 4-D view {32, Hkv, P, NP}, box {32, 1, 32, 1}, 64-byte swizzle.
+int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D) {
+    auto fn = encode_fn();
+    if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
+    cuuint64_t dims[5], strides[4];
+    cuuint32_t box[5], estr[5] = {1, 1, 1, 1, 1};
+    cuuint32_t rank;
+    CUtensorMapSwizzle swz;
+    if (D >= 64) {
+        rank = 5;
+        dims[0] = 64; dims[1] = D / 64; dims[2] = t->shape[2]; dims[3] = t->shape[1]; dims[4] = t->shape[0];
+        strides[0] = 128; strides[1] = st[2] * 2; strides[2] = st[1] * 2; strides[3] = st[0] * 2;
+        box[0] = 64; box[1] = D / 64; box[2] = 1; box[3] = apd::kTile; box[4] = 1;
+        swz = CU_TENSOR_MAP_SWIZZLE_128B;
+    } else {
+        rank = 4;
+        dims[0] = 32; dims[1] = t->shape[2]; dims[2] = t->shape[1]; dims[3] = t->shape[0];
+        strides[0] = st[2] * 2; strides[1] = st[1] * 2; strides[2] = st[0] * 2;
+        box[0] = 32; box[1] = 1; box[2] = apd::kTile; box[3] = 1;
+        swz = CU_TENSOR_MAP_SWIZZLE_64B;
+    }
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, t->data, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return driver_fail(r, "cuTensorMapEncodeTiled(kv)");
+    return APD_OK;
+}
+
+// Q: D >= 64 -> 4-D view {64, D/64, Hq, B}, box {64, D/64, rows_max, 1};
+//    D == 32 -> 3-D view {32, Hq, B}, box {32, rows_max, 1}.
+int encode_q_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D, int rows_max) {
+    auto fn = encode_fn();
+    if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
+    cuuint64_t dims[4], strides[3];
+    cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
+    cuuint32_t rank;
+    CUtensorMapSwizzle swz;
+    if (D >= 64) {
+        rank = 4;
+        dims[0] = 64; dims[1] = D / 64; dims[2] = t->shape[1]; dims[3] = t->shape[0];
+        strides[0] = 128; strides[1] = st[1] * 2; strides[2] = st[0] * 2;
+        box[0] = 64; box[1] = D / 64; box[2] = rows_max; box[3] = 1;
+        swz = CU_TENSOR_MAP_SWIZZLE_128B;
+    } else {
+        rank = 3;
+        dims[0] = 32; dims[1] = t->shape[1]; dims[2] = t->shape[0];
+        strides[0] = st[1] * 2; strides[1] = st[0] * 2;
+        box[0] = 32; box[1] = rows_max; box[2] = 1;
+        swz = CU_TENSOR_MAP_SWIZZLE_64B;
+    }
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, t->data, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return driver_fail(r, "cuTensorMapEncodeTiled(q)");
+    return APD_OK;
+}
+
+// ---------------------------------------------------------------- launch
+template <int D>
+int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+           const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
+           void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
+    constexpr int kStagesD = (D == 32 || D == 64) ? 4 : (D == 128 ? 3 : 2);
+    auto kern = apd::split_kernel<D, kStagesD>;
+    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->smem_attr_set[kSlot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kSmemLimit));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(split_kernel)");
+            dev->smem_attr_set[kSlot] = true;
+        }
+    }
+    CUtensorMap kmap, vmap, qmap;
+    int rc = encode_kv_map(&kmap, k, V.kst, D);
+    if (!rc) rc = encode_kv_map(&vmap, v, V.vst, D);
+    if (!rc) rc = encode_q_map(&qmap, q, V.qst, D, V.s.rows_max);
+    if (rc) return rc;
+
+    const Shape& s = V.s;
+    char* ws = static_cast<char*>(workspace);
+    apd::SplitParams sp;
+    sp.page_table = static_cast<const int32_t*>(pt->data);
+    sp.pt_s0 = V.pst[0];
+    sp.pt_s1 = V.pst[1];
+    sp.seq_lens = static_cast<const int32_t*>(sl->data);
+    sp.out = static_cast<__nv_bfloat16*>(out->data);
+    sp.out_sb = V.ost[0];
+    sp.out_sh = V.ost[1];
+    sp.flags = reinterpret_cast<uint32_t*>(ws);
+    sp.cum_out = reinterpret_cast<int32_t*>(ws + kWsAlign);
+    sp.o_part = reinterpret_cast<float*>(ws + ws_head_bytes(s));
+    sp.ml_part = reinterpret_cast<float*>(ws + ws_head_bytes(s) +
+                                          align_up(static_cast<size_t>(pl.slots) * s.rows_max * s.D * 4, kWsAlign));
+    sp.B = s.B;
+    sp.Hq = s.Hq;
+    sp.Hkv = s.Hkv;
+    sp.g = s.g;
+    sp.HB = s.HB;
+    sp.rows_max = s.rows_max;
+    sp.P = V.P;
+    sp.NP = V.NP;
+    sp.MP = V.MP;
+    sp.mode = pl.mode;
+    sp.ksplit = pl.ksplit;
+    sp.num_workers = pl.workers;
+    sp.warps = pl.warps;
+    sp.stage_bytes = stage_bytes(s);
+    sp.q_box_bytes = static_cast<uint32_t>(s.rows_max) * s.D * 2u;
+    sp.scale_log2 = scale * 1.4426950408889634f;
+
+    kern<<<pl.ctas, pl.warps * 32, pl.smem, stream>>>(sp, kmap, vmap, qmap);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "split_kernel launch");
+    if (opts && opts->split_done_event) {
+        e = cudaEventRecord(static_cast<cudaEvent_t>(opts->split_done_event), stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(split_done_event)");
+    }
+    const bool use_pdl = !(opts && (opts->disable_pdl || opts->split_done_event));
+
+    if (pl.combine_ctas > 0) {
+        apd::CombineParams cp;
+        cp.cum = sp.cum_out;
+        cp.o_part = sp.o_part;
+        cp.ml_part = sp.ml_part;
+        cp.out = sp.out;
+        cp.out_sb = sp.out_sb;
+        cp.out_sh = sp.out_sh;
+        cp.B = s.B;
+        cp.Hkv = s.Hkv;
+        cp.g = s.g;
+        cp.HB = s.HB;
+        cp.rows_max = s.rows_max;
+        cp.mode = pl.mode;
+        cp.ksplit = pl.ksplit;
+        cp.num_workers = pl.workers;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(pl.combine_ctas));
+        cfg.blockDim = dim3(128);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = use_pdl ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, apd::combine_kernel<D>, cp);
+        if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+    }
+    return APD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t apd_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits) {
+    Shape s;
+    if (make_shape(batch, num_q_heads, num_kv_heads, head_dim, &s) != APD_OK) return 0;
+    if (num_splits < 0) return 0;
+    int sm_count = kDefaultSmCount;
+    int dev = 0;
+    if (num_splits == 0 && cudaGetDevice(&dev) == cudaSuccess) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) sm_count = n;
+    }
+    cudaGetLastError();  // a missing device is not an error of this query
+    Plan pl;
+    if (make_plan(s, num_splits, sm_count, SIZE_MAX, -1, &pl) != APD_OK) return 0;
+    return pl.ws_needed;
+}
+
+int apd_workspace_init(void* workspace, size_t workspace_bytes, apd_stream_t stream) {
+    if (!workspace) return APD_ERR_NULL_POINTER;
+    if (workspace_bytes < kWsAlign || (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)) return APD_ERR_WORKSPACE;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, kWsAlign, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace header)");
+    return APD_OK;
+}
+
+int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                             apd_stream_t stream, const apd_launch_options* options) {
+    if (options && options->reserved != 0) return APD_ERR_ARGUMENT;
+    Validated V;
+    int rc = validate(q, k_cache, v_cache, page_table, seq_lens, out, num_splits, &V);
+    if (rc) return rc;
+    if (!workspace) return APD_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return APD_ERR_WORKSPACE;
+    if (V.s.B == 0) return APD_OK;
+    Plan pl;
+    const int64_t tiles_bound = V.s.units * V.MP * (V.P / apd::kTile);
+    // A fixed split count does not depend on the device: check its workspace
+    // before any CUDA call.
+    if (num_splits > 0) {
+        rc = make_plan(V.s, num_splits, kDefaultSmCount, workspace_bytes, tiles_bound, &pl);
+        if (rc) return rc;
+    }
+    DeviceState* dev = nullptr;
+    rc = device_state(&dev);
+    if (rc) return rc;
+    rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (V.s.D) {
+        case 32: return launch<32>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
+        case 64: return launch<64>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
+        case 128: return launch<128>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
+        case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
+        default: return APD_ERR_HEAD_DIM;
+    }
+}
+
+int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                          const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                          float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                          apd_stream_t stream) {
+    return apd_attn_paged_decode_ex(q, k_cache, v_cache, page_table, seq_lens, out, scale, num_splits, workspace,
+                                    workspace_bytes, stream, nullptr);
+}
+
+int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_stream_t stream, uint32_t* flags,
+                          int clear) {
+    if (!workspace || !flags) return APD_ERR_NULL_POINTER;
+    if (workspace_bytes < kWsAlign) return APD_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    e = cudaMemcpy(flags, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(flags)");
+    if (clear) {
+        e = cudaMemset(const_cast<void*>(workspace), 0, sizeof(uint32_t));
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(flags)");
+    }
+    return APD_OK;
+}
+
+int apd_query_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
+                   size_t workspace_bytes, int sm_count, apd_plan* plan) {
+    if (!plan) return APD_ERR_NULL_POINTER;
+    Shape s;
+    int rc = make_shape(batch, num_q_heads, num_kv_heads, head_dim, &s);
+    if (rc) return rc;
+    if (sm_count <= 0) {
+        DeviceState* dev = nullptr;
+        rc = device_state(&dev);
+        if (rc) return rc;
+        sm_count = dev->sm_count;
+    }
+    Plan pl;
+    rc = make_plan(s, num_splits, sm_count, workspace_bytes, -1, &pl);
+    if (rc) return rc;
+    plan->mode = pl.mode;
+    plan->num_workers = pl.workers;
+    plan->grid_ctas = pl.ctas;
+    plan->warps_per_cta = pl.warps;
+    plan->stages = pl.stages;
+    plan->rows_per_unit = s.rows_max;
+    plan->head_blocks = s.HB;
+    plan->combine_ctas = pl.combine_ctas;
+    plan->smem_bytes = static_cast<int64_t>(pl.smem);
+    plan->partial_slots = pl.slots;
+    plan->workspace_bytes = static_cast<int64_t>(pl.ws_needed);
+    return APD_OK;
+}
+
+const char* apd_status_string(int status) {
+    switch (status) {
+        case APD_OK: return "ok";
+        case APD_ERR_NULL_POINTER: return "a tensor descriptor or its data pointer is NULL";
+        case APD_ERR_DTYPE: return "wrong dtype: q/k_cache/v_cache/out must be bf16, page_table/seq_lens int32";
+        case APD_ERR_SHAPE: return "tensor ranks or extents disagree";
+        case APD_ERR_GQA: return "num_q_heads must be a multiple of num_kv_heads";
+        case APD_ERR_HEAD_DIM: return "head_dim must be 32, 64, 128 or 256";
+        case APD_ERR_LAYOUT:
+            return "layout: the head dim must be contiguous and other strides / base pointers 16-byte aligned "
+                   "(seq_lens contiguous)";
+        case APD_ERR_PAGE_SIZE: return "page_size must be a positive multiple of 32";
+        case APD_ERR_NUM_SPLITS: return "num_splits must be >= 0";
+        case APD_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned, or smaller than apd_workspace_size()";
+        case APD_ERR_TOO_LARGE: return "problem too large (batch > APD_MAX_BATCH or index overflow)";
+        case APD_ERR_CUDA: return "a CUDA call failed (see apd_last_cuda_error)";
+        case APD_ERR_ARGUMENT: return "invalid argument";
+        default: return "unknown status";
+    }
+}
+
+const char* apd_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

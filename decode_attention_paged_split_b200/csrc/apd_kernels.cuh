@@ -1,0 +1,639 @@
+// apd_kernels.cuh -- sm_100a kernels of paged split-KV decode attention.
+//
+// The operation, and the pieces of the design taken from the pages, come from
+// the AstrAI commit log of csrc/kernels/attn_paged_decode.cu: decode attention
+// over a paged KV cache, head packing of the query heads that share a kv head
+// onto tensor-core tiles, one page-table lookup per 32-token tile (a tile never
+// straddles a page because page_size is a multiple of 32), split-KV partials
+// o_part / ml_part, and a single combine kernel.  The B200 design around them is
+// our own:
+//
+//  * The unit of work is a 32-token tile of one (sequence b, kv head, head
+//    block).  All tiles of all units are laid out in one flattened index space
+//    (b-major, then kv head / head block, then tile), found on the device from
+//    a prefix sum of the per-sequence tile counts.
+//  * Every warp is an independent worker that owns a contiguous run of that
+//    space: in balanced mode (num_splits == 0) the runs are equal shares of the
+//    whole space, one per resident warp of a persistent, SM-count-sized grid;
+//    in fixed mode (num_splits == k) the runs are the k page-aligned chunks of
+//    each unit.  A warp that covers a whole unit writes the final bf16 output;
+//    otherwise it writes an unnormalised fp32 partial plus (m, l), and the
+//    combine kernel merges the partials of each unit.
+//  * Each warp runs its own STAGES-deep ring in shared memory.  Lane 0 issues
+//    TMA tiled loads (cp.async.bulk.tensor, 128-byte swizzle) of the K and V
+//    tiles [32 tokens x D] of the next tiles straight from the paged cache,
+//    plus the unit's query rows when a unit starts; completion is tracked by
+//    mbarrier transaction bytes.  Page-table entries are fetched 32 tiles ahead,
+//    one coalesced load per warp.  Page indices outside the pool read as zeros
+//    (TMA bounds fill) instead of faulting.
+//  * QK^T and PV run on tensor cores (mma.sync m16n8k16, bf16 in, fp32
+//    accumulate) with the g query heads of a kv head on the M side (padded to
+//    16), so K/V are read once per kv head.  The softmax is the online form in
+//    fp32 with exp2 (logits pre-multiplied by scale * log2 e) and quad shuffles.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "apd_ptx.cuh"
+
+namespace apd {
+
+constexpr int kTile = 32;          // tokens per tile (= rows of one TMA box)
+constexpr int kMaxRows = 16;       // query heads per unit (mma M)
+constexpr int kMaxWarps = 8;       // warps per CTA, upper bound
+constexpr uint32_t kFlagPageOOR = 0x1u;
+constexpr uint32_t kFlagLenClamped = 0x2u;
+constexpr uint32_t kFlagLenNegative = 0x4u;
+constexpr uint32_t kFlagTimeout = 0x8u;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per async-copy wait
+
+struct SplitParams {
+    const int32_t* page_table;
+    int64_t pt_s0, pt_s1;
+    const int32_t* seq_lens;
+    __nv_bfloat16* out;
+    int64_t out_sb, out_sh;
+    float* o_part;      // [slots][rows_max][D]
+    float* ml_part;     // [slots][rows_max][2]
+    int32_t* cum_out;   // [B + 1] prefix sum of tiles per sequence (for the combine)
+    uint32_t* flags;
+    int32_t B, Hq, Hkv, g, HB, rows_max, P, NP, MP;
+    int32_t mode;       // 0 balanced, 1 fixed
+    int32_t ksplit;     // fixed mode: k
+    int32_t num_workers;
+    int32_t warps;      // warps per CTA
+    uint32_t stage_bytes, q_box_bytes;
+    float scale_log2;
+};
+
+struct CombineParams {
+    const int32_t* cum;  // [B + 1]
+    const float* o_part;
+    const float* ml_part;
+    __nv_bfloat16* out;
+    int64_t out_sb, out_sh;
+    int32_t B, Hkv, g, HB, rows_max;
+    int32_t mode, ksplit, num_workers;
+};
+
+template <int D>
+struct Geometry {
+    static_assert(D == 32 || D == 64 || D == 128 || D == 256, "head_dim");
+    static constexpr int kSteps = D / 16;              // k-steps of QK^T
+    static constexpr int kNTiles = D / 8;              // 8-wide n-tiles of PV
+    static constexpr int kChunks = D / 8;              // 16-byte chunks per row
+    static constexpr uint32_t kRowBytes = D * 2;
+    static constexpr uint32_t kKVTileBytes = kTile * D * 2;
+    // TMA swizzle applied to a byte offset from a 1024-aligned base:
+    // 128B mode XORs address bits [4:6] with [7:9]; 64B mode bits [4:5] with [7:8].
+    __device__ __forceinline__ static uint32_t swz(uint32_t off) {
+        if constexpr (D == 32) {
+            return off ^ (((off >> 7) & 3u) << 4);
+        } else {
+            return off ^ (((off >> 7) & 7u) << 4);
+        }
+    }
+};
+
+// Largest b in [0, B) with cum[b] <= x (cum non-decreasing, cum[0] = 0).
+__device__ __forceinline__ int find_seq(const int32_t* cum, int B, int x) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cum[mid] <= x) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Flattened tile index -> (sequence b, unit-in-sequence ul, tile j, tiles n).
+__device__ __forceinline__ void decode_tile(int64_t i, int units_per_seq, const int32_t* cum, int B, int& b,
+                                            int& ul, int& j, int& n) {
+    b = find_seq(cum, B, static_cast<int>(i / units_per_seq));
+    n = cum[b + 1] - cum[b];
+    const int rem = static_cast<int>(i - static_cast<int64_t>(units_per_seq) * cum[b]);
+    ul = rem / n;
+    j = rem - ul * n;
+}
+
+// Step a cursor to the next tile; only called when that tile exists.
+__device__ __forceinline__ void advance_tile(int units_per_seq, const int32_t* cum, int& b, int& ul, int& j,
+                                             int& n) {
+    if (++j == n) {
+        j = 0;
+        if (++ul == units_per_seq) {
+            ul = 0;
+            do {
+                ++b;
+                n = cum[b + 1] - cum[b];
+            } while (n == 0);
+        }
+    }
+}
+
+__device__ __forceinline__ int32_t fetch_page(const SplitParams& p, const int32_t* cum, int units_per_seq,
+                                              int64_t i, int64_t end) {
+    if (i >= end) return 0;
+    int b, ul, j, n;
+    decode_tile(i, units_per_seq, cum, p.B, b, ul, j, n);
+    const int pj = (j * kTile) / p.P;
+    return __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 + static_cast<int64_t>(pj) * p.pt_s1);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+template <int D>
+__device__ __forceinline__ void write_zero_rows(const SplitParams& p, int b, int head0, int rows, int lane) {
+    for (int idx = lane; idx < rows * (D / 2); idx += 32) {
+        const int r = idx / (D / 2), d2 = idx % (D / 2);
+        *reinterpret_cast<uint32_t*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 2 * d2) = 0u;
+    }
+}
+
+template <int D, int STAGES>
+__global__ void __launch_bounds__(32 * kMaxWarps, 1)
+    split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
+    using G = Geometry<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int B = p.B;
+
+    // ---- shared-memory carve-up: mbarriers, lengths, prefix sums, stage ring
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    int32_t* s_len = reinterpret_cast<int32_t*>(bars + p.warps * STAGES);
+    int32_t* s_cum = s_len + B;
+    const uint32_t meta_end = smem_u32(s_cum + B + 1);
+    const uint32_t ring = (meta_end + 1023u) & ~1023u;
+
+    if (tid == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+    }
+
+    // ---- per-sequence tile counts and their prefix sum (every CTA, from L2)
+    const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
+    uint32_t len_flags = 0;
+    for (int b = tid; b < B; b += blockDim.x) {
+        int L = __ldg(p.seq_lens + b);
+        if (L < 0) {
+            L = 0;
+            len_flags |= kFlagLenNegative;
+        }
+        if (L > cap) {
+            L = static_cast<int>(cap);
+            len_flags |= kFlagLenClamped;
+        }
+        s_len[b] = L;
+        s_cum[b + 1] = (L + kTile - 1) / kTile;
+    }
+    if (tid == 0) s_cum[0] = 0;
+    if (len_flags && blockIdx.x == 0) atomicOr(p.flags, len_flags);
+    __syncthreads();
+    if (warp == 0) {
+        const int per = (B + 31) / 32;
+        const int lo = 1 + lane * per;
+        const int hi = min(lo + per, B + 1);
+        int sum = 0;
+        for (int i = lo; i < hi; ++i) sum += s_cum[i];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int i = lo; i < hi; ++i) {
+            run += s_cum[i];
+            s_cum[i] = run;
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int i = tid; i <= B; i += blockDim.x) p.cum_out[i] = s_cum[i];
+    }
+    // The combine kernel may start its launch now; it waits (griddepcontrol.wait)
+    // for this whole grid to finish before it reads anything.
+    pdl_launch_dependents();
+    // No CTA-wide barrier after this point: warps are independent workers.
+
+    const int units_per_seq = p.Hkv * p.HB;
+    const int64_t total = static_cast<int64_t>(units_per_seq) * s_cum[B];
+    const int w = blockIdx.x * p.warps + warp;
+    if (w >= p.num_workers) return;
+
+    int64_t ws, we;
+    int fixed_slot = -1;
+    if (p.mode == 0) {
+        ws = static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / p.num_workers);
+        we = static_cast<int64_t>((static_cast<uint64_t>(w + 1) * static_cast<uint64_t>(total)) / p.num_workers);
+    } else {
+        const int u = w / p.ksplit;
+        const int s = w - u * p.ksplit;
+        const int b = u / units_per_seq;
+        const int ul = u - b * units_per_seq;
+        const int n = s_cum[b + 1] - s_cum[b];
+        if (n == 0) {
+            if (s == 0) {
+                const int kvh = ul / p.HB, hb = ul - (ul / p.HB) * p.HB;
+                write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
+            }
+            return;
+        }
+        const int S = min(p.ksplit, n);
+        const int c = (n + S - 1) / S;
+        const int t0 = s * c;
+        if (t0 >= n) return;
+        const int t1 = min(t0 + c, n);
+        const int64_t Tu = static_cast<int64_t>(units_per_seq) * s_cum[b] + static_cast<int64_t>(ul) * n;
+        ws = Tu + t0;
+        we = Tu + t1;
+        fixed_slot = u * p.ksplit + s;
+    }
+    if (ws >= we) return;
+
+    const uint32_t bar0 = smem_u32(bars + warp * STAGES);
+    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const uint64_t pol_stream = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
+
+    // ---- producer state: next tile to issue, its cursor, page-table window
+    int64_t pi = ws;
+    int pb, pul, pj, pn;
+    decode_tile(ws, units_per_seq, s_cum, B, pb, pul, pj, pn);
+    int64_t wbase = ws;
+    int32_t pg_cur = fetch_page(p, s_cum, units_per_seq, ws + lane, we);
+    int32_t pg_nxt = fetch_page(p, s_cum, units_per_seq, ws + 32 + lane, we);
+
+    auto issue_next = [&](int stage) {
+        if (pi >= we) return;
+        int off = static_cast<int>(pi - wbase);
+        if (off >= 32) {
+            pg_cur = pg_nxt;
+            wbase += 32;
+            off -= 32;
+            pg_nxt = fetch_page(p, s_cum, units_per_seq, wbase + 32 + lane, we);
+        }
+        const int32_t page = __shfl_sync(0xffffffffu, pg_cur, off);
+        const int kvh = pul / p.HB;
+        const int hb = pul - kvh * p.HB;
+        const int slot = (pj * kTile) % p.P;
+        const bool qload = (pj == 0) || (pi == ws);
+        if (lane == 0) {
+            if (page < 0 || page >= p.NP) atomicOr(p.flags, kFlagPageOOR);
+            const uint32_t bar = bar0 + 8 * stage;
+            const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+            mbar_arrive_expect_tx(bar, 2 * G::kKVTileBytes + (qload ? p.q_box_bytes : 0u));
+            if constexpr (D == 32) {
+                tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, page, pol_stream);
+                tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, pol_stream);
+                if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, kvh * p.g + kMaxRows * hb, pb,
+                                       pol_keep);
+            } else {
+                tma_load_5d(sbase, &kmap, bar, 0, 0, kvh, slot, page, pol_stream);
+                tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, 0, kvh, slot, page, pol_stream);
+                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, 0, kvh * p.g + kMaxRows * hb,
+                                       pb, pol_keep);
+            }
+        }
+        ++pi;
+        if (pi < we) advance_tile(units_per_seq, s_cum, pb, pul, pj, pn);
+    };
+
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) issue_next(s);
+
+    // ---- consumer state
+    const int tq = lane & 3;   // thread in quad: token / d pair
+    const int gq = lane >> 2;  // quad index: row within the 8-row half
+    int cb, cul, cj, cn;
+    decode_tile(ws, units_per_seq, s_cum, B, cb, cul, cj, cn);
+    int64_t seg_start = ws;
+    int j_start = cj;
+
+    uint32_t qf[G::kSteps][4];
+    float acc[G::kNTiles][4];
+    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+    int rows = 0;
+
+    for (int64_t i = ws; i < we; ++i) {
+        const int k = static_cast<int>(i - ws);
+        const int stage = k % STAGES;
+        const uint32_t parity = static_cast<uint32_t>(k / STAGES) & 1u;
+        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+        const bool unit_start = (cj == 0) || (i == ws);
+        const int kvh = cul / p.HB;
+        const int hb = cul - kvh * p.HB;
+
+        if (!mbar_wait_bounded(bar0 + 8 * stage, parity, kWaitTimeoutNs)) {
+            if (lane == 0) atomicOr(p.flags, kFlagTimeout);
+            // Give the other copies in flight a bounded chance to land, then stop.
+            for (int s = 0; s < STAGES; ++s) {
+                const int64_t t = i + s;
+                if (t < pi) {
+                    const int kk = static_cast<int>(t - ws);
+                    mbar_wait_bounded(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u,
+                                      kWaitTimeoutNs / 8);
+                }
+            }
+            return;
+        }
+
+        if (unit_start) {
+            seg_start = i;
+            j_start = cj;
+            rows = min(kMaxRows, p.g - kMaxRows * hb);
+            m_lo = m_hi = -INFINITY;
+            l_lo = l_hi = 0.f;
+#pragma unroll
+            for (int nd = 0; nd < G::kNTiles; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
+            // Q A-fragments: matrix m of ldmatrix.x4 = (rows 8*(m&1).., k chunk m>>1)
+            const uint32_t qbase = sbase + 2 * G::kKVTileBytes;
+            const int mi = lane >> 3;
+            int qrow = (mi & 1) * 8 + (lane & 7);
+            if (qrow >= p.rows_max) qrow = 0;  // stay inside the loaded box
+#pragma unroll
+            for (int ks = 0; ks < G::kSteps; ++ks) {
+                const uint32_t ch = 2 * ks + (mi >> 1);
+                ldsm_x4(qbase + G::swz(qrow * G::kRowBytes + ch * 16), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+                if (gq >= rows) qf[ks][0] = qf[ks][2] = 0u;
+                if (gq + 8 >= rows) qf[ks][1] = qf[ks][3] = 0u;
+            }
+        }
+
+        // ---- S = Q K^T over the 32 tokens of the tile: 4 n-tiles of 8 tokens
+        float s[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        {
+            const int mi = lane >> 3;
+#pragma unroll
+            for (int ks = 0; ks < G::kSteps; ++ks) {
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    const int row = 8 * (2 * np + (mi >> 1)) + (lane & 7);
+                    const uint32_t ch = 2 * ks + (mi & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(sbase + G::swz(row * G::kRowBytes + ch * 16), b0, b1, b2, b3);
+                    mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
+                    mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
+                }
+            }
+        }
+
+        // ---- mask tokens past the sequence end; tail V rows are zeroed so that
+        // 0 * (stale or NaN) never reaches the accumulator
+        const int valid = min(kTile, s_len[cb] - kTile * cj);
+        if (valid < kTile) {
+            const uint32_t vb = sbase + G::kKVTileBytes;
+            for (int idx = lane; idx < (kTile - valid) * G::kChunks; idx += 32) {
+                const int r = valid + idx / G::kChunks;
+                const int ch = idx % G::kChunks;
+                st_shared_zero16(vb + G::swz(r * G::kRowBytes + ch * 16));
+            }
+            __syncwarp();
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int t0 = 8 * nt + 2 * tq;
+            s[nt][0] = (t0 < valid) ? s[nt][0] * p.scale_log2 : -INFINITY;
+            s[nt][1] = (t0 + 1 < valid) ? s[nt][1] * p.scale_log2 : -INFINITY;
+            s[nt][2] = (t0 < valid) ? s[nt][2] * p.scale_log2 : -INFINITY;
+            s[nt][3] = (t0 + 1 < valid) ? s[nt][3] * p.scale_log2 : -INFINITY;
+        }
+
+        // ---- online softmax (rows gq and gq + 8 of the head tile)
+        float mx_lo = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        mx_lo = fmaxf(mx_lo, fmaxf(fmaxf(s[2][0], s[2][1]), fmaxf(s[3][0], s[3][1])));
+        float mx_hi = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        mx_hi = fmaxf(mx_hi, fmaxf(fmaxf(s[2][2], s[2][3]), fmaxf(s[3][2], s[3][3])));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 1));
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
+        const float mn_lo = fmaxf(m_lo, mx_lo);  // finite: every tile has >= 1 valid token
+        const float mn_hi = fmaxf(m_hi, mx_hi);
+        const float alpha_lo = exp2f(m_lo - mn_lo);
+        const float alpha_hi = exp2f(m_hi - mn_hi);
+        m_lo = mn_lo;
+        m_hi = mn_hi;
+
+        uint32_t pa[2][4];
+        float rs_lo = 0.f, rs_hi = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int nt = 2 * kk + h;
+                const uint32_t plo = pack_bf16x2(exp2f(s[nt][0] - mn_lo), exp2f(s[nt][1] - mn_lo));
+                const uint32_t phi = pack_bf16x2(exp2f(s[nt][2] - mn_hi), exp2f(s[nt][3] - mn_hi));
+                pa[kk][2 * h + 0] = plo;
+                pa[kk][2 * h + 1] = phi;
+                // the normaliser sums exactly the bf16 weights that enter PV
+                rs_lo += bf16_lo(plo) + bf16_hi(plo);
+                rs_hi += bf16_lo(phi) + bf16_hi(phi);
+            }
+        }
+        l_lo = l_lo * alpha_lo + rs_lo;
+        l_hi = l_hi * alpha_hi + rs_hi;
+#pragma unroll
+        for (int nd = 0; nd < G::kNTiles; ++nd) {
+            acc[nd][0] *= alpha_lo;
+            acc[nd][1] *= alpha_lo;
+            acc[nd][2] *= alpha_hi;
+            acc[nd][3] *= alpha_hi;
+        }
+
+        // ---- O += P V: k = 32 tokens (2 steps), n = D (8-wide tiles)
+        {
+            const uint32_t vb = sbase + G::kKVTileBytes;
+            const int mi = lane >> 3;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                for (int nd = 0; nd < G::kNTiles; nd += 2) {
+                    const int row = 16 * kk + 8 * (mi & 1) + (lane & 7);
+                    const uint32_t ch = nd + (mi >> 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_trans(vb + G::swz(row * G::kRowBytes + ch * 16), b0, b1, b2, b3);
+                    mma_bf16_16816(acc[nd], pa[kk], b0, b1);
+                    mma_bf16_16816(acc[nd + 1], pa[kk], b2, b3);
+                }
+            }
+        }
+
+        // ---- the stage is consumed: refill it with tile i + STAGES.  Each lane
+        // orders its own shared-memory accesses (the tail zeroing included)
+        // before the async-proxy write, then the warp syncs before lane 0 issues.
+        fence_proxy_async_smem();
+        __syncwarp();
+        issue_next(stage);
+
+        // ---- end of this unit's run in this worker: write output or a partial
+        const bool unit_end = (cj == cn - 1) || (i == we - 1);
+        if (unit_end) {
+            float ll = l_lo + __shfl_xor_sync(0xffffffffu, l_lo, 1);
+            ll += __shfl_xor_sync(0xffffffffu, ll, 2);
+            float lh = l_hi + __shfl_xor_sync(0xffffffffu, l_hi, 1);
+            lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+            const int head0 = kvh * p.g + kMaxRows * hb;
+            const bool direct = (j_start == 0) && (cj == cn - 1);
+            if (direct) {
+                const float il = 1.f / ll, ih = 1.f / lh;
+                __nv_bfloat16* o_lo = p.out + cb * p.out_sb + (head0 + gq) * p.out_sh;
+                __nv_bfloat16* o_hi = o_lo + 8 * p.out_sh;
+#pragma unroll
+                for (int nd = 0; nd < G::kNTiles; ++nd) {
+                    const int d = 8 * nd + 2 * tq;
+                    if (gq < rows)
+                        *reinterpret_cast<uint32_t*>(o_lo + d) = pack_bf16x2(acc[nd][0] * il, acc[nd][1] * il);
+                    if (gq + 8 < rows)
+                        *reinterpret_cast<uint32_t*>(o_hi + d) = pack_bf16x2(acc[nd][2] * ih, acc[nd][3] * ih);
+                }
+            } else {
+                const int64_t slot =
+                    (p.mode == 0) ? (2 * static_cast<int64_t>(w) + (seg_start == ws ? 0 : 1)) : fixed_slot;
+                float* op = p.o_part + slot * p.rows_max * D;
+                float* mp = p.ml_part + slot * p.rows_max * 2;
+#pragma unroll
+                for (int nd = 0; nd < G::kNTiles; ++nd) {
+                    const int d = 8 * nd + 2 * tq;
+                    if (gq < rows)
+                        *reinterpret_cast<float2*>(op + gq * D + d) = make_float2(acc[nd][0], acc[nd][1]);
+                    if (gq + 8 < rows)
+                        *reinterpret_cast<float2*>(op + (gq + 8) * D + d) = make_float2(acc[nd][2], acc[nd][3]);
+                }
+                if (tq == 0) {
+                    if (gq < rows) *reinterpret_cast<float2*>(mp + 2 * gq) = make_float2(m_lo, ll);
+                    if (gq + 8 < rows) *reinterpret_cast<float2*>(mp + 2 * (gq + 8)) = make_float2(m_hi, lh);
+                }
+            }
+        }
+        if (i + 1 < we) advance_tile(units_per_seq, s_cum, cb, cul, cj, cn);
+    }
+}
+
+// Balanced mode: the worker whose run contains flattened tile i.
+__device__ __forceinline__ int worker_of(int64_t i, int64_t total, int workers) {
+    return static_cast<int>((static_cast<uint64_t>(i + 1) * static_cast<uint64_t>(workers) - 1) /
+                            static_cast<uint64_t>(total));
+}
+
+__device__ __forceinline__ int64_t run_start(int w, int64_t total, int workers) {
+    return static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / workers);
+}
+
+// One CTA per unit (b, kv head, head block).  Merges the unit's partials:
+// M = max_s m_s over non-empty partials, out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// In balanced mode it also writes zeros for empty sequences.
+template <int D>
+__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ CombineParams p) {
+    const int u = blockIdx.x;
+    const int units_per_seq = p.Hkv * p.HB;
+    const int b = u / units_per_seq;
+    const int ul = u - b * units_per_seq;
+    const int kvh = ul / p.HB;
+    const int hb = ul - kvh * p.HB;
+    const int rows = min(kMaxRows, p.g - kMaxRows * hb);
+    const int head0 = kvh * p.g + kMaxRows * hb;
+    constexpr int kQuads = D / 4;
+
+    pdl_wait_prior_grid();
+    const int n = p.cum[b + 1] - p.cum[b];
+    if (n == 0) {
+        if (p.mode == 0) {
+            for (int it = threadIdx.x; it < rows * kQuads; it += blockDim.x) {
+                const int r = it / kQuads, q4 = it - (it / kQuads) * kQuads;
+                *reinterpret_cast<uint2*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 4 * q4) = make_uint2(0u, 0u);
+            }
+        }
+        return;
+    }
+
+    // slot list: (first, count) for fixed mode; worker range for balanced mode
+    int w_first = 0, w_last = -1, first_slot_fixed = 0, nslots_fixed = 0;
+    int64_t total = 0, Tu = 0;
+    if (p.mode == 0) {
+        total = static_cast<int64_t>(units_per_seq) * p.cum[p.B];
+        Tu = static_cast<int64_t>(units_per_seq) * p.cum[b] + static_cast<int64_t>(ul) * n;
+        w_first = worker_of(Tu, total, p.num_workers);
+        w_last = worker_of(Tu + n - 1, total, p.num_workers);
+        if (w_first == w_last) return;  // one worker covered it and wrote the output
+    } else {
+        const int S = min(p.ksplit, n);
+        const int c = (n + S - 1) / S;
+        nslots_fixed = (n + c - 1) / c;
+        if (nslots_fixed == 1) return;
+        first_slot_fixed = u * p.ksplit;
+    }
+
+    for (int it = threadIdx.x; it < rows * kQuads; it += blockDim.x) {
+        const int r = it / kQuads;
+        const int q4 = it - r * kQuads;
+        float M = -INFINITY;
+        // pass 1: the common max
+        if (p.mode == 0) {
+            for (int w = w_first; w <= w_last; ++w) {
+                const int64_t a = run_start(w, total, p.num_workers);
+                if (a == run_start(w + 1, total, p.num_workers)) continue;
+                const int64_t slot = 2 * static_cast<int64_t>(w) + ((w == w_first && a != Tu) ? 1 : 0);
+                const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
+                if (ml.y > 0.f) M = fmaxf(M, ml.x);
+            }
+        } else {
+            for (int s = 0; s < nslots_fixed; ++s) {
+                const int64_t slot = first_slot_fixed + s;
+                const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
+                if (ml.y > 0.f) M = fmaxf(M, ml.x);
+            }
+        }
+        // pass 2: weighted sums
+        float den = 0.f;
+        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto add = [&](int64_t slot) {
+            const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
+            if (!(ml.y > 0.f)) return;
+            const float wgt = exp2f(ml.x - M);
+            den += wgt * ml.y;
+            const float4 a = *reinterpret_cast<const float4*>(p.o_part + (slot * p.rows_max + r) * D + 4 * q4);
+            num.x += wgt * a.x;
+            num.y += wgt * a.y;
+            num.z += wgt * a.z;
+            num.w += wgt * a.w;
+        };
+        if (p.mode == 0) {
+            for (int w = w_first; w <= w_last; ++w) {
+                const int64_t a = run_start(w, total, p.num_workers);
+                if (a == run_start(w + 1, total, p.num_workers)) continue;
+                add(2 * static_cast<int64_t>(w) + ((w == w_first && a != Tu) ? 1 : 0));
+            }
+        } else {
+            for (int s = 0; s < nslots_fixed; ++s) add(first_slot_fixed + s);
+        }
+        const float inv = 1.f / den;
+        uint2 packed;
+        packed.x = pack_bf16x2(num.x * inv, num.y * inv);
+        packed.y = pack_bf16x2(num.z * inv, num.w * inv);
+        *reinterpret_cast<uint2*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 4 * q4) = packed;
+    }
+}
+
+}  // namespace apd

@@ -1,0 +1,236 @@
+/*
+ * attn_paged_decode.h -- C ABI of the B200 (sm_100a) paged split-KV decode
+ * attention library (libattn_paged_decode.so).
+ *
+ * Operation (AstrAI commit d565d44c, csrc/kernels/attn_paged_decode.cu, commit
+ * log: the attn_paged_decode entry, its scalar and MMA split-KV decode kernels,
+ * the o_part / ml_part partials and the single combine kernel):
+ *
+ *   single-token decode attention over a paged bf16 KV cache.  For every
+ *   sequence b and query head h, with g = Hq / Hkv, kv head kvh = h / g and
+ *   L = seq_lens[b]:
+ *       s_t   = scale * <q[b,h,:], K_t>          for t in [0, L)
+ *       out[b,h,:] = sum_t softmax(s)_t * V_t    (L == 0 -> zeros)
+ *   where K_t / V_t are row (page_table[b][t / P], t % P, kvh, :) of
+ *   k_cache / v_cache.  Decode is causal, so the one query token sees all L
+ *   stored positions.  The KV range of each (sequence, kv head) is split across
+ *   workers (split-KV); each split leaves a partial output with its running max
+ *   and sum, and one combine kernel merges them.  Query heads that share a kv
+ *   head are processed together, so K/V are read once per kv head.
+ *
+ * Ownership and threading.  The caller owns every buffer, including the
+ * workspace.  The library allocates nothing, never synchronises the stream and
+ * never reads device memory on the host, so a call can be captured in a CUDA
+ * graph once the workspace exists.  Work is enqueued on `stream` in stream
+ * order; a call returns as soon as the kernels are launched.  Calls may be made
+ * from several host threads; calls that share a workspace must be ordered on
+ * the device (same stream, or events).
+ *
+ * Errors.  Every entry point returns an apd_status.  Argument faults are found
+ * on the host before anything is launched; nothing is written then.  A failed
+ * CUDA launch returns APD_ERR_CUDA.  Device-side contract violations (see
+ * apd_attn_paged_decode) never fault: they are clamped or read as zeros and
+ * recorded as sticky bits in the workspace, which apd_read_device_flags reads.
+ * No C++ exception crosses this interface.
+ */
+#ifndef ATTN_PAGED_DECODE_H_
+#define ATTN_PAGED_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define APD_VERSION 1
+
+/* A CUDA stream handle; identical to cudaStream_t (NULL = legacy default stream). */
+typedef struct CUstream_st* apd_stream_t;
+
+typedef enum apd_dtype {
+    APD_DTYPE_BF16 = 1,
+    APD_DTYPE_INT32 = 2,
+    APD_DTYPE_FP32 = 3
+} apd_dtype;
+
+/* A strided view of device memory.  `stride` is in elements; only the first
+ * `ndim` entries of shape/stride are read.  Dimensions of extent 1 may carry
+ * any stride. */
+typedef struct apd_tensor {
+    void* data;
+    int32_t dtype;     /* apd_dtype */
+    int32_t ndim;
+    int64_t shape[4];
+    int64_t stride[4];
+} apd_tensor;
+
+typedef enum apd_status {
+    APD_OK = 0,
+    APD_ERR_NULL_POINTER = 1,     /* a descriptor or its data pointer is NULL            */
+    APD_ERR_DTYPE = 2,            /* q/k/v/out not bf16, page_table/seq_lens not int32    */
+    APD_ERR_SHAPE = 3,            /* ndim or extents disagree between the tensors         */
+    APD_ERR_GQA = 4,              /* num_q_heads is not a multiple of num_kv_heads        */
+    APD_ERR_HEAD_DIM = 5,         /* head_dim not in {32, 64, 128, 256}                   */
+    APD_ERR_LAYOUT = 6,           /* head dim not contiguous, or a stride / base pointer
+                                     not 16-byte aligned                                  */
+    APD_ERR_PAGE_SIZE = 7,        /* page_size not a positive multiple of 32              */
+    APD_ERR_NUM_SPLITS = 8,       /* num_splits < 0                                       */
+    APD_ERR_WORKSPACE = 9,        /* workspace NULL, not 256-byte aligned, or too small   */
+    APD_ERR_TOO_LARGE = 10,       /* batch > APD_MAX_BATCH or indices would overflow      */
+    APD_ERR_CUDA = 11,            /* a CUDA runtime call or a kernel launch failed        */
+    APD_ERR_ARGUMENT = 12         /* any other bad argument (e.g. a NULL output pointer)  */
+} apd_status;
+
+/* Largest batch one call accepts (the per-sequence lengths and their prefix
+ * sums are staged in shared memory). */
+#define APD_MAX_BATCH 4096
+
+/* Sticky device flags (apd_read_device_flags). */
+#define APD_FLAG_PAGE_OUT_OF_RANGE 0x1u /* a page-table entry outside [0, num_pages): read as zeros */
+#define APD_FLAG_SEQ_LEN_CLAMPED   0x2u /* seq_len > max_pages_per_seq * page_size: clamped         */
+#define APD_FLAG_SEQ_LEN_NEGATIVE  0x4u /* seq_len < 0: treated as 0                                */
+#define APD_FLAG_WAIT_TIMEOUT      0x8u /* an async copy did not complete in time: output invalid  */
+
+/*
+ * apd_workspace_size -- bytes of device workspace that apd_attn_paged_decode
+ * needs for this problem shape (workspace pattern of the AstrAI commit log:
+ * the decode partials are preallocated once and reused by every call, which is
+ * what makes the call capturable in a CUDA graph).
+ *
+ *   batch, num_q_heads, num_kv_heads, head_dim: as in apd_attn_paged_decode.
+ *   num_splits: the value that will be passed to apd_attn_paged_decode.
+ *     num_splits >= 1 needs room for batch * num_kv_heads * ceil(g/16) *
+ *     num_splits partial slots; num_splits == 0 ("auto") needs room for two
+ *     slots per hardware worker of the current CUDA device (148 SMs are assumed
+ *     when no device is visible).  A smaller auto workspace still works: the
+ *     call then uses fewer parallel workers.
+ *
+ * Returns 0 if the arguments are invalid.  Does not allocate.  The returned
+ * size is a multiple of 256; the workspace must be 256-byte aligned.
+ */
+size_t apd_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits);
+
+/*
+ * apd_workspace_init -- zero the workspace header (the sticky device flags).
+ * Enqueued on `stream`; call once after allocating a workspace (a workspace
+ * that is all zeros is already initialised).  Not needed for correct output.
+ */
+int apd_workspace_init(void* workspace, size_t workspace_bytes, apd_stream_t stream);
+
+/*
+ * apd_attn_paged_decode -- the decode attention call.
+ *
+ *   q          bf16 [B, Hq, D], stride(D) == 1, other strides multiples of 8
+ *              elements, base 16-byte aligned.
+ *   k_cache    bf16 [num_pages, page_size, Hkv, D] (logical "NHD" order); any
+ *   v_cache    strides that keep D contiguous and are multiples of 8 elements,
+ *              so "HND" storage [num_pages, Hkv, page_size, D] is passed as the
+ *              permuted view.  k_cache and v_cache have the same shape.
+ *   page_table int32 [B, max_pages_per_seq]; entry [b][j] is the physical page
+ *              holding tokens [j*P, (j+1)*P) of sequence b.  Entries at or past
+ *              ceil(seq_lens[b] / P) are never read.
+ *   seq_lens   int32 [B], on the device; read only by the kernels.
+ *   out        bf16 [B, Hq, D], stride(D) == 1, written for every (b, h).
+ *   scale      multiplies the q.K dot products (typically 1/sqrt(D)).
+ *   num_splits 0 = auto: the KV work of all sequences and kv heads is cut into
+ *              equal runs of 32-token tiles, one run per hardware worker, so
+ *              every SM gets the same number of tiles and longer sequences get
+ *              more splits (the ejkernel PageAttentionConfig convention that
+ *              num_splits = 0 means automatic).
+ *              k >= 1: sequence b is split into min(k, n_b) page-aligned chunks
+ *              of ceil(n_b / min(k, n_b)) 32-token tiles, n_b = ceil(L_b / 32);
+ *              k == 1 means no split-KV and a single kernel launch.
+ *   workspace  device memory of at least apd_workspace_size(...) bytes, 256-byte
+ *              aligned, owned by the caller; its contents between calls are
+ *              scratch except for the sticky flags word.
+ *   stream     CUDA stream the kernels are enqueued on.
+ *
+ * Requirements checked on the host (status codes above): Hq % Hkv == 0,
+ * D in {32, 64, 128, 256}, page_size % 32 == 0, 0 <= num_splits, B <= APD_MAX_BATCH,
+ * alignment of the strided layouts, workspace size.
+ *
+ * Device-side contract (not checked on the host, since seq_lens and page_table
+ * live on the device): 0 <= seq_lens[b] <= max_pages_per_seq * page_size and
+ * the first ceil(seq_lens[b] / page_size) page-table entries of sequence b lie in
+ * [0, num_pages).  Violations never fault: lengths are clamped, pages outside
+ * the pool read as zeros, and the matching APD_FLAG_* bit is set.
+ *
+ * Numerics: bf16 inputs, fp32 accumulation (tensor cores), softmax in fp32
+ * with exp2, probabilities rounded to bf16 for the PV product, output rounded
+ * to bf16 (nearest-even).  Results are deterministic for a given device, shape
+ * and num_splits.
+ */
+int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                          const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                          float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                          apd_stream_t stream);
+
+/*
+ * apd_attn_paged_decode_ex -- apd_attn_paged_decode with launch options.
+ *
+ * Same arguments, checks, results and errors as apd_attn_paged_decode, plus
+ * `options` (may be NULL, which makes the two calls identical):
+ *   split_done_event  a cudaEvent_t (created by the caller) that is recorded on
+ *                     `stream` right after the split kernel is enqueued, before
+ *                     the combine kernel; lets a caller time the split kernel
+ *                     alone with events.  Recording it between the kernels
+ *                     also turns off the programmatic (PDL) overlap of the
+ *                     combine kernel's launch for that call.
+ *   disable_pdl       nonzero: launch the combine kernel without programmatic
+ *                     dependent launch.
+ */
+typedef struct apd_launch_options {
+    void* split_done_event; /* cudaEvent_t or NULL */
+    int32_t disable_pdl;
+    int32_t reserved;       /* must be 0 */
+} apd_launch_options;
+
+int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                             apd_stream_t stream, const apd_launch_options* options);
+
+/*
+ * apd_read_device_flags -- synchronise `stream`, copy the sticky APD_FLAG_* word
+ * out of the workspace into *flags and, if `clear` is nonzero, reset it.  A
+ * debugging / testing aid: it blocks the host, so it does not belong in a
+ * captured or latency-critical loop.
+ */
+int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_stream_t stream, uint32_t* flags,
+                          int clear);
+
+/* apd_plan -- how a call with these arguments would be launched (for tests,
+ * benchmarks and profiling). */
+typedef struct apd_plan {
+    int32_t mode;              /* 0 = balanced (num_splits == 0), 1 = fixed splits */
+    int32_t num_workers;       /* warps that each own a run of tiles             */
+    int32_t grid_ctas;         /* CTAs of the split kernel                       */
+    int32_t warps_per_cta;
+    int32_t stages;            /* async-copy ring depth per warp                 */
+    int32_t rows_per_unit;     /* query heads packed per unit (<= 16)            */
+    int32_t head_blocks;       /* ceil(g / 16)                                   */
+    int32_t combine_ctas;      /* 0 when no combine kernel is launched           */
+    int64_t smem_bytes;        /* dynamic shared memory of the split kernel      */
+    int64_t partial_slots;
+    int64_t workspace_bytes;   /* bytes the call needs                           */
+} apd_plan;
+
+/* apd_query_plan -- fills *plan.  workspace_bytes: the size that will be passed
+ * (SIZE_MAX = unlimited).  sm_count > 0 plans for a device with that many SMs
+ * without touching CUDA (host-side planning, e.g. for tests); sm_count <= 0
+ * queries the current CUDA device. */
+int apd_query_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
+                   size_t workspace_bytes, int sm_count, apd_plan* plan);
+
+/* Human-readable text for an apd_status (never NULL). */
+const char* apd_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* apd_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_PAGED_DECODE_H_ */

@@ -1,0 +1,255 @@
+"""Host-only checks of the C-ABI library: it loads, exports every symbol its
+header declares, rejects bad arguments with the documented status codes before
+touching the GPU, and plans launches as documented.  No test here needs a GPU or
+launches a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import decode_attention_paged_split_b200 as apd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_paged_decode.h")
+
+OK, NULLP, DTYPE, SHAPE, GQA, HEADDIM, LAYOUT, PAGESIZE, NSPLIT, WS, TOOLARGE, CUDA, ARG = range(13)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w \*]*?\b(apd_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("apd_attn_paged_decode", "apd_workspace_size", "apd_status_string", "apd_attn_paged_decode_ex",
+                 "apd_query_plan", "apd_workspace_init", "apd_read_device_flags", "apd_last_cuda_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(apd.library_path())
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in range(13):
+        s = apd.status_string(code)
+        assert s and s != "unknown status"
+    assert apd.status_string(999) == "unknown status"
+
+
+# ---------------------------------------------------------------- fake descriptors
+FAKE = 1 << 32  # never dereferenced: every case below fails validation first
+
+
+def T(shape, dtype=apd.DTYPE_BF16, stride=None, data=FAKE):
+    d = apd._Tensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if stride is None:
+        stride, acc = [], 1
+        for s in reversed(shape):
+            stride.insert(0, acc)
+            acc *= s
+    for i, (s, st) in enumerate(zip(shape, stride)):
+        d.shape[i] = s
+        d.stride[i] = st
+    return d
+
+
+def problem(B=2, Hq=8, Hkv=2, D=64, P=32, NP=16, MP=4):
+    return dict(
+        q=T([B, Hq, D]), k=T([NP, P, Hkv, D]), v=T([NP, P, Hkv, D]),
+        pt=T([B, MP], apd.DTYPE_INT32), sl=T([B], apd.DTYPE_INT32), out=T([B, Hq, D]),
+    )
+
+
+def call(p, splits=0, ws=FAKE, ws_bytes=1 << 30, scale=0.125):
+    L = apd.lib()
+    return L.apd_attn_paged_decode(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]),
+                                   ctypes.byref(p["pt"]), ctypes.byref(p["sl"]), ctypes.byref(p["out"]),
+                                   ctypes.c_float(scale), splits, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "pt", "sl", "out"])
+def test_null_pointer(field):
+    p = problem()
+    p[field].data = None
+    assert call(p) == NULLP
+
+
+def test_null_descriptor():
+    p = problem()
+    L = apd.lib()
+    rc = L.apd_attn_paged_decode(None, ctypes.byref(p["k"]), ctypes.byref(p["v"]), ctypes.byref(p["pt"]),
+                                 ctypes.byref(p["sl"]), ctypes.byref(p["out"]), ctypes.c_float(1.0), 0, FAKE,
+                                 1 << 30, None)
+    assert rc == NULLP
+
+
+@pytest.mark.parametrize("field,dtype", [("q", apd.DTYPE_FP32), ("k", apd.DTYPE_INT32), ("v", apd.DTYPE_FP32),
+                                         ("out", apd.DTYPE_FP32), ("pt", apd.DTYPE_BF16), ("sl", apd.DTYPE_FP32)])
+def test_dtype(field, dtype):
+    p = problem()
+    p[field].dtype = dtype
+    assert call(p) == DTYPE
+
+
+def test_shape_errors():
+    p = problem()
+    p["q"] = T([2, 8, 64, 1])
+    assert call(p) == SHAPE
+    p = problem()
+    p["out"] = T([2, 8, 32])
+    assert call(p) == SHAPE
+    p = problem()
+    p["v"] = T([16, 32, 2, 32])
+    assert call(p) == SHAPE
+    p = problem()
+    p["pt"] = T([3, 4], apd.DTYPE_INT32)
+    assert call(p) == SHAPE
+    p = problem()
+    p["sl"] = T([3], apd.DTYPE_INT32)
+    assert call(p) == SHAPE
+
+
+def test_gqa_divisibility():
+    p = problem(Hq=6, Hkv=4)
+    assert call(p) == GQA
+
+
+@pytest.mark.parametrize("D", [16, 48, 96, 512])
+def test_head_dim(D):
+    assert call(problem(D=D)) == HEADDIM
+
+
+@pytest.mark.parametrize("P", [16, 48, 8])
+def test_page_size(P):
+    assert call(problem(P=P)) == PAGESIZE
+
+
+def test_layout_errors():
+    p = problem()
+    p["q"] = T([2, 8, 64], stride=[512, 1, 8])  # head dim not contiguous
+    assert call(p) == LAYOUT
+    p = problem()
+    p["k"] = T([16, 32, 2, 64], stride=[32 * 2 * 68, 2 * 68, 68, 1])  # 68 elements: not 16-byte aligned
+    assert call(p) == LAYOUT
+    p = problem()
+    p["out"].data = FAKE + 2  # misaligned base
+    assert call(p) == LAYOUT
+    p = problem()
+    p["sl"] = T([2], apd.DTYPE_INT32, stride=[2])
+    assert call(p) == LAYOUT
+
+
+def test_hnd_strides_are_accepted_by_validation():
+    """HND storage [NP, Hkv, P, D] passed as the NHD-ordered view passes the checks
+    (the call then needs a device, which this host does not have)."""
+    NP, P, Hkv, D = 16, 32, 2, 64
+    p = problem()
+    p["k"] = T([NP, P, Hkv, D], stride=[Hkv * P * D, D, P * D, 1])
+    p["v"] = T([NP, P, Hkv, D], stride=[Hkv * P * D, D, P * D, 1])
+    assert call(p, ws_bytes=1 << 30) in (OK, CUDA)
+
+
+def test_num_splits_negative():
+    assert call(problem(), splits=-1) == NSPLIT
+
+
+def test_workspace_errors():
+    assert call(problem(), ws=None) == WS
+    assert call(problem(), ws=FAKE + 128) == WS
+    assert call(problem(), splits=4, ws_bytes=1024) == WS
+
+
+def test_batch_too_large():
+    assert call(problem(B=5000)) == TOOLARGE
+
+
+def test_empty_batch_is_a_no_op():
+    assert call(problem(B=0)) == OK
+
+
+def test_ex_reserved_must_be_zero():
+    p = problem()
+    opts = apd._Options()
+    opts.reserved = 1
+    L = apd.lib()
+    rc = L.apd_attn_paged_decode_ex(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]),
+                                    ctypes.byref(p["pt"]), ctypes.byref(p["sl"]), ctypes.byref(p["out"]),
+                                    ctypes.c_float(1.0), 0, FAKE, 1 << 30, None, ctypes.byref(opts))
+    assert rc == ARG
+
+
+# ---------------------------------------------------------------- planning
+def test_workspace_size_invalid_is_zero():
+    L = apd.lib()
+    assert L.apd_workspace_size(2, 6, 4, 64, 0) == 0
+    assert L.apd_workspace_size(2, 8, 2, 80, 0) == 0
+    assert L.apd_workspace_size(2, 8, 2, 64, -1) == 0
+    with pytest.raises(ValueError):
+        apd.workspace_size(2, 6, 4, 64)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(16, 32, 8, 128), (2, 32, 8, 128), (128, 64, 8, 128), (4, 8, 8, 32),
+                                        (4, 32, 8, 256), (3, 40, 2, 64)])
+def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
+    pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
+    g = Hq // Hkv
+    assert pl.mode == 0
+    assert pl.grid_ctas == 148  # one persistent CTA per SM
+    assert pl.num_workers == 148 * pl.warps_per_cta
+    assert pl.partial_slots == 2 * pl.num_workers
+    assert pl.rows_per_unit == min(g, 16) and pl.head_blocks == -(-g // 16)
+    assert pl.combine_ctas == B * Hkv * pl.head_blocks
+    assert pl.smem_bytes <= 232448
+    assert pl.workspace_bytes % 256 == 0
+    assert pl.workspace_bytes == apd.lib().apd_workspace_size(B, Hq, Hkv, D, 0)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 4, 148])
+def test_plan_fixed(splits):
+    B, Hq, Hkv, D = 16, 32, 8, 128
+    pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=148)
+    units = B * Hkv
+    assert pl.mode == 1
+    assert pl.num_workers == units * splits
+    assert pl.grid_ctas == -(-pl.num_workers // pl.warps_per_cta)
+    assert pl.partial_slots == (units * splits if splits > 1 else 0)
+    assert pl.combine_ctas == (units if splits > 1 else 0)
+    assert pl.workspace_bytes == apd.workspace_size(B, Hq, Hkv, D, splits)
+
+
+def test_plan_small_workspace_uses_fewer_workers():
+    B, Hq, Hkv, D = 16, 32, 8, 128
+    full = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
+    half = apd.query_plan(B, Hq, Hkv, D, 0, workspace_bytes=full.workspace_bytes // 2, sm_count=148)
+    assert 0 < half.num_workers < full.num_workers
+    assert half.workspace_bytes <= full.workspace_bytes // 2
+
+
+def test_plan_workspace_too_small_for_fixed_splits():
+    need = apd.workspace_size(16, 32, 8, 128, 4)
+    with pytest.raises(apd.APDError) as e:
+        apd.query_plan(16, 32, 8, 128, 4, workspace_bytes=need - 256, sm_count=148)
+    assert e.value.status == WS
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    monkeypatch.setattr(apd, "_lib", None)
+    monkeypatch.setattr(apd, "_LIB_PATH", os.path.join(ROOT, "no_such_library.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        apd.workspace_size(1, 4, 1, 64)
+
+
+def test_binding_rejects_five_dim_tensors():
+    with pytest.raises(ValueError):
+        apd._desc(torch.zeros(1, 1, 1, 1, 1))

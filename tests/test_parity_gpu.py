@@ -1,0 +1,254 @@
+"""GPU parity: the CUDA path (through the C-ABI binding) against the fp64 CPU oracle.
+
+Every comparison is element by element on the same seeded inputs, with the
+per-element bound |gpu - ref| <= 1e-2 + 1e-2 |ref| (ref = fp64 oracle value).
+Covered: the tiny decode case, the full head-dim / GQA / split sweep, HND
+storage, NaN-poisoned slots that must never be read, ragged and empty
+sequences, head groups that span several 16-row blocks, larger pages, strided
+q / out, a side stream, CUDA-graph capture, determinism, the device-side
+contract flags, and the three large decode workloads at full size in the launch
+configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_paged_split_b200 as apd
+import oracle
+import workloads
+from gpu_util import DeviceProblem, check_close
+
+pytestmark = pytest.mark.gpu
+
+
+def small(seed, B, Hq, Hkv, D, lens, P=32, pool=None, **kw):
+    return workloads.make(name="case", seed=seed, batch=B, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                          page_size=P, seq_lens=list(lens), pool_pages=pool, **kw)
+
+
+# ---------------------------------------------------------------- named small workloads
+@pytest.mark.parametrize("splits", [1, 0, 4, 8])
+def test_tiny(splits):
+    w = workloads.tiny()
+    ref = oracle.paged_decode(w)
+    check_close(DeviceProblem(w).run(splits), ref, f"tiny splits={splits}")
+
+
+@pytest.mark.parametrize("D,Hq,Hkv,S", list(workloads.sweep_cases()))
+def test_sweep(D, Hq, Hkv, S):
+    w = workloads.sweep_case(D, Hq, Hkv, S)
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    check_close(dp.run(S), ref, w.name)
+    check_close(dp.run(0), ref, w.name + " auto")
+
+
+@pytest.mark.parametrize("D", workloads.SWEEP_HEAD_DIMS)
+@pytest.mark.parametrize("S", [1, 3, 0])
+def test_sweep_hnd_layout(D, S):
+    w = workloads.sweep_case(D, 32, 8, S, layout="HND", seed=99)
+    assert w.k_cache.stride(2) != D  # really strided
+    check_close(DeviceProblem(w).run(S), oracle.paged_decode(w), f"HND D={D} S={S}")
+
+
+@pytest.mark.parametrize("D", workloads.SWEEP_HEAD_DIMS)
+@pytest.mark.parametrize("S", [1, 4, 0])
+def test_poisoned_slots_are_never_read(D, S):
+    """Tail slots, unused pool pages and unused page-table entries hold NaN."""
+    w = small(7, B=5, Hq=16, Hkv=4, D=D, lens=(1, 31, 33, 200, 515), pool=40, poison=True,
+              max_pages_per_seq=20)
+    ref = oracle.paged_decode(w)
+    assert np.isfinite(ref).all()
+    check_close(DeviceProblem(w).run(S), ref, f"poison D={D} S={S}")
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [1, 3, 0, 148])
+def test_ragged_and_empty_sequences(D, S):
+    lens = (0, 1, 31, 32, 33, 64, 65, 1000, 0, 7)
+    w = small(21, B=len(lens), Hq=8, Hkv=2, D=D, lens=lens, pool=60, poison=True, max_pages_per_seq=32)
+    ref = oracle.paged_decode(w)
+    out = DeviceProblem(w).run(S)
+    check_close(out, ref, f"ragged D={D} S={S}")
+    assert torch.all(out[0] == 0) and torch.all(out[8] == 0)
+
+
+@pytest.mark.parametrize("S", [1, 0, 5])
+def test_all_sequences_empty(S):
+    w = small(22, B=3, Hq=4, Hkv=1, D=64, lens=(0, 0, 0), pool=2, max_pages_per_seq=4)
+    out = DeviceProblem(w).run(S)
+    assert torch.all(out == 0)
+
+
+def test_empty_batch():
+    w = small(23, B=1, Hq=4, Hkv=1, D=64, lens=(5,), pool=2)
+    dp = DeviceProblem(w)
+    q0 = dp.q[:0]
+    out0 = dp.out[:0]
+    ws = apd.alloc_workspace(0 + 1, 4, 1, 64, 0)
+    apd.attn_paged_decode(q0, dp.k, dp.v, dp.page_table[:0], dp.seq_lens[:0], out0, w.scale, 0, ws)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(12, 4), (40, 2), (64, 2), (16, 1), (7, 7), (48, 1)])
+@pytest.mark.parametrize("S", [1, 0, 4])
+def test_gqa_groups(Hq, Hkv, S):
+    """g = 3, 20 (a partial second 16-row head block), 32, 16, 1, 48."""
+    w = small(31, B=3, Hq=Hq, Hkv=Hkv, D=64, lens=(45, 300, 129), pool=30)
+    check_close(DeviceProblem(w).run(S), oracle.paged_decode(w), f"gqa {Hq}/{Hkv} S={S}")
+
+
+@pytest.mark.parametrize("P", [64, 128])
+@pytest.mark.parametrize("S", [1, 0, 3])
+def test_larger_pages(P, S):
+    w = small(41, B=4, Hq=8, Hkv=2, D=128, lens=(1, 100, 257, 640), P=P, pool=24, poison=True,
+              max_pages_per_seq=12)
+    check_close(DeviceProblem(w).run(S), oracle.paged_decode(w), f"P={P} S={S}")
+
+
+@pytest.mark.parametrize("D", [32, 256])
+def test_max_head_dim_and_group(D):
+    """D extremes with a full 16-row head block and a long sequence."""
+    w = small(43, B=2, Hq=32, Hkv=2, D=D, lens=(2049, 77), pool=70)
+    for S in (1, 0, 16):
+        check_close(DeviceProblem(w).run(S), oracle.paged_decode(w), f"D={D} S={S}")
+
+
+def test_strided_q_and_out():
+    w = small(51, B=3, Hq=8, Hkv=2, D=64, lens=(40, 90, 3), pool=8)
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    big_q = torch.zeros(3, 8, 192, dtype=torch.bfloat16, device="cuda")
+    big_q[:, :, 64:128] = dp.q
+    q = big_q[:, :, 64:128]
+    big_out = torch.full((3, 10, 72), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = big_out[:, 1:9, 8:]
+    ws = apd.alloc_workspace(3, 8, 2, 64, 0)
+    apd.attn_paged_decode(q, dp.k, dp.v, dp.page_table, dp.seq_lens, out, w.scale, 0, ws)
+    check_close(out, ref, "strided")
+    assert torch.isnan(big_out[:, 0]).all() and torch.isnan(big_out[:, 9]).all()
+    assert torch.isnan(big_out[:, :, :8]).all()
+
+
+def test_side_stream():
+    w = small(52, B=4, Hq=16, Hkv=4, D=128, lens=(500, 20, 1, 900), pool=50)
+    dp = DeviceProblem(w)
+    s = torch.cuda.Stream()
+    ws = apd.alloc_workspace(4, 16, 4, 128, 0)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    s.synchronize()
+    check_close(dp.out, oracle.paged_decode(w), "side stream")
+
+
+@pytest.mark.parametrize("S", [0, 1, 4])
+def test_cuda_graph_capture_and_replay(S):
+    w = small(53, B=4, Hq=32, Hkv=8, D=128, lens=(300, 1, 77, 1024), pool=60)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(4, 32, 8, 128, S)
+    eager = dp.run(S, workspace=ws).clone()
+    out = torch.full_like(dp.out, float("nan"))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, out, w.scale, S, ws)  # live first
+        with torch.cuda.graph(g, stream=s):
+            apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, out, w.scale, S, ws)
+    torch.cuda.current_stream().wait_stream(s)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    # new inputs in the same buffers are picked up by the replay
+    dp.q.mul_(-1)
+    g.replay()
+    torch.cuda.synchronize()
+    w.q.mul_(-1)
+    check_close(out, oracle.paged_decode(w), "graph replay with new q")
+
+
+def test_deterministic():
+    w = workloads.sweep_case(128, 32, 8, 0)
+    dp = DeviceProblem(w)
+    a = dp.run(0).clone()
+    b = dp.run(0).clone()
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- device-side contract
+def test_out_of_range_pages_set_a_flag_and_read_zeros():
+    w = small(61, B=3, Hq=8, Hkv=2, D=64, lens=(64, 64, 40), pool=8)
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    dp.page_table[1, 0] = w.num_pages + 3
+    dp.page_table[1, 1] = -2
+    ws = apd.alloc_workspace(3, 8, 2, 64, 0)
+    apd.workspace_init(ws)
+    apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    flags = apd.read_device_flags(ws)
+    assert flags & apd.FLAG_PAGE_OUT_OF_RANGE
+    out = dp.out.to(torch.float64).cpu().numpy()
+    assert np.isfinite(out).all()
+    # sequence 1 read only zero rows: every weight equal, V rows zero -> output 0
+    assert np.all(out[1] == 0)
+    check_close(dp.out[[0, 2]], ref[[0, 2]], "untouched sequences")
+    assert apd.read_device_flags(ws) == 0  # cleared by the previous read
+
+
+def test_seq_len_contract_flags():
+    w = small(62, B=3, Hq=4, Hkv=1, D=64, lens=(64, 10, 20), pool=6, max_pages_per_seq=2)
+    dp = DeviceProblem(w)
+    dp.seq_lens[1] = 5000   # > max_pages * page_size = 64: clamped to 64
+    dp.seq_lens[2] = -7     # treated as 0
+    ws = apd.alloc_workspace(3, 4, 1, 64, 0)
+    apd.workspace_init(ws)
+    apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    flags = apd.read_device_flags(ws)
+    assert flags & apd.FLAG_SEQ_LEN_CLAMPED and flags & apd.FLAG_SEQ_LEN_NEGATIVE
+    assert not flags & apd.FLAG_PAGE_OUT_OF_RANGE
+    assert torch.all(dp.out[2] == 0)
+    w.seq_lens[1] = 64
+    w.seq_lens[2] = 0
+    check_close(dp.out, oracle.paged_decode(w), "clamped lengths")
+
+
+def test_bad_arguments_raise_before_launch():
+    w = small(63, B=2, Hq=8, Hkv=2, D=64, lens=(10, 20), pool=2)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(2, 8, 2, 64, 4)
+    with pytest.raises(apd.APDError) as e:
+        apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 4, ws[:1024])
+    assert e.value.status == 9
+    with pytest.raises(apd.APDError) as e:
+        apd.attn_paged_decode(dp.q.float(), dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    assert e.value.status == 2
+
+
+# ---------------------------------------------------------------- full-size workloads
+@pytest.fixture(scope="module")
+def llama():
+    w = workloads.llama8b()
+    return w, oracle.paged_decode(w)
+
+
+@pytest.mark.parametrize("S", [0, 1, 4, 148])
+def test_llama8b_full_size(llama, S):
+    w, ref = llama
+    check_close(DeviceProblem(w).run(S), ref, f"llama8b S={S}")
+
+
+@pytest.mark.parametrize("S", [0, 148])
+def test_long_context_full_size(S):
+    w = workloads.long_context()
+    ref = oracle.paged_decode(w)
+    check_close(DeviceProblem(w).run(S), ref, f"long S={S}")
+
+
+def test_ragged_full_size():
+    w = workloads.ragged()
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    check_close(dp.run(0), ref, "ragged auto")
+    check_close(dp.run(16), ref, "ragged S=16")
