@@ -217,7 +217,9 @@ struct Validated {
 
 int validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* pt,
              const apd_tensor* sl, const apd_tensor* out, int num_splits, Validated* V) {
-    if (is_null(q) || is_null(k) || is_null(v) || is_null(pt) || is_null(sl) || is_null(out))
+    if (!q || !k || !v || !pt || !sl || !out || is_null(k) || is_null(v)) return APD_ERR_NULL_POINTER;
+    // The per-sequence tensors may be empty (and NULL) only when the batch is empty.
+    if ((is_null(q) || is_null(pt) || is_null(sl) || is_null(out)) && !(q->ndim >= 1 && q->shape[0] == 0))
         return APD_ERR_NULL_POINTER;
     if (q->dtype != APD_DTYPE_BF16 || k->dtype != APD_DTYPE_BF16 || v->dtype != APD_DTYPE_BF16 ||
         out->dtype != APD_DTYPE_BF16 || pt->dtype != APD_DTYPE_INT32 || sl->dtype != APD_DTYPE_INT32)

@@ -253,3 +253,13 @@ def test_binding_fails_loudly_without_the_library(monkeypatch):
 def test_binding_rejects_five_dim_tensors():
     with pytest.raises(ValueError):
         apd._desc(torch.zeros(1, 1, 1, 1, 1))
+
+
+def test_empty_batch_accepts_null_batch_tensors():
+    p = problem(B=0)
+    for f in ("q", "pt", "sl", "out"):
+        p[f].data = None
+    assert call(p) == OK
+    p = problem(B=0)
+    p["k"].data = None
+    assert call(p) == NULLP
