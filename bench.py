@@ -196,9 +196,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- measurement legs
 def kernel_source_sha() -> str:
+    """Hash of the device code (the kernel headers); the host-side API file is not included."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(CSRC)):
-        if name.endswith((".cu", ".cuh")):
+        if name.endswith(".cuh"):
             with open(os.path.join(CSRC, name), "rb") as f:
                 h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
