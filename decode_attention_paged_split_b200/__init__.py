@@ -21,6 +21,8 @@ import torch
 __all__ = [
     "APDError",
     "attn_paged_decode",
+    "attn_paged_decode_noalloc",
+    "NOALLOC_SCRATCH_BYTES",
     "workspace_size",
     "alloc_workspace",
     "workspace_init",
@@ -42,6 +44,7 @@ FLAG_PAGE_OUT_OF_RANGE = 0x1
 FLAG_SEQ_LEN_CLAMPED = 0x2
 FLAG_SEQ_LEN_NEGATIVE = 0x4
 FLAG_WAIT_TIMEOUT = 0x8
+NOALLOC_SCRATCH_BYTES = 8 << 20  # APD_NOALLOC_SCRATCH_BYTES
 
 _DTYPES = {torch.bfloat16: DTYPE_BF16, torch.int32: DTYPE_INT32, torch.float32: DTYPE_FP32}
 
@@ -117,6 +120,8 @@ def _load():
     L.apd_attn_paged_decode.restype = ctypes.c_int
     L.apd_attn_paged_decode_ex.argtypes = L.apd_attn_paged_decode.argtypes + [ctypes.POINTER(_Options)]
     L.apd_attn_paged_decode_ex.restype = ctypes.c_int
+    L.apd_attn_paged_decode_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+    L.apd_attn_paged_decode_noalloc.restype = ctypes.c_int
     L.apd_read_device_flags.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                         ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
     L.apd_read_device_flags.restype = ctypes.c_int
@@ -219,6 +224,20 @@ def attn_paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
                                         ctypes.byref(opts))
     if rc:
         raise APDError(rc, "apd_attn_paged_decode")
+    return out
+
+
+def attn_paged_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              page_table: torch.Tensor, seq_lens: torch.Tensor, out: torch.Tensor, scale: float,
+                              num_splits: int = 0, stream=None) -> torch.Tensor:
+    """attn_paged_decode for callers that cannot allocate device memory: no workspace
+    argument; the library's built-in static device scratch (NOALLOC_SCRATCH_BYTES per
+    device, shared by every call, so calls must be ordered on the GPU) is used instead."""
+    descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+    rc = _load().apd_attn_paged_decode_noalloc(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale),
+                                               int(num_splits), _stream_handle(stream, q.device))
+    if rc:
+        raise APDError(rc, "apd_attn_paged_decode_noalloc")
     return out
 
 

@@ -414,6 +414,31 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     return APD_OK;
 }
 
+// ---------------------------------------------------------------- built-in scratch
+// Scratch of apd_attn_paged_decode_noalloc: a static device array, so that entry
+// point allocates nothing.  Host code must not use its name as an address (on the
+// host it is only a stand-in); the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[APD_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_scratch_addr[128] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 128) return APD_ERR_ARGUMENT;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_noalloc_scratch_addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(noalloc scratch)");
+        g_noalloc_scratch_addr[dev] = ptr;
+    }
+    *out = g_noalloc_scratch_addr[dev];
+    return APD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -484,6 +509,40 @@ int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const 
                                     workspace_bytes, stream, nullptr);
 }
 
+int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                                  const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                                  float scale, int num_splits, apd_stream_t stream) {
+    Validated V;
+    int rc = validate(q, k_cache, v_cache, page_table, seq_lens, out, num_splits, &V);
+    if (rc) return rc;
+    if (V.s.B == 0) return APD_OK;
+    constexpr size_t kScratch = APD_NOALLOC_SCRATCH_BYTES;
+    Plan pl;
+    const int64_t tiles_bound = V.s.units * V.MP * (V.P / apd::kTile);
+    if (num_splits > 0) {
+        rc = make_plan(V.s, num_splits, kDefaultSmCount, kScratch, tiles_bound, &pl);
+        if (rc == APD_ERR_WORKSPACE) return APD_ERR_SCRATCH_LIMIT;
+        if (rc) return rc;
+    }
+    DeviceState* dev = nullptr;
+    rc = device_state(&dev);
+    if (rc) return rc;
+    rc = make_plan(V.s, num_splits, dev->sm_count, kScratch, tiles_bound, &pl);
+    if (rc == APD_ERR_WORKSPACE) return APD_ERR_SCRATCH_LIMIT;
+    if (rc) return rc;
+    void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (V.s.D) {
+        case 32: return launch<32>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
+        case 64: return launch<64>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
+        case 128: return launch<128>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
+        case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
+        default: return APD_ERR_HEAD_DIM;
+    }
+}
+
 int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_stream_t stream, uint32_t* flags,
                           int clear) {
     if (!workspace || !flags) return APD_ERR_NULL_POINTER;
@@ -546,6 +605,9 @@ const char* apd_status_string(int status) {
         case APD_ERR_TOO_LARGE: return "problem too large (batch > APD_MAX_BATCH or index overflow)";
         case APD_ERR_CUDA: return "a CUDA call failed (see apd_last_cuda_error)";
         case APD_ERR_ARGUMENT: return "invalid argument";
+        case APD_ERR_SCRATCH_LIMIT:
+            return "the problem needs more scratch than apd_attn_paged_decode_noalloc's built-in "
+                   "APD_NOALLOC_SCRATCH_BYTES (use apd_attn_paged_decode with a workspace, or fewer splits)";
         default: return "unknown status";
     }
 }

@@ -79,7 +79,9 @@ typedef enum apd_status {
     APD_ERR_WORKSPACE = 9,        /* workspace NULL, not 256-byte aligned, or too small   */
     APD_ERR_TOO_LARGE = 10,       /* batch > APD_MAX_BATCH or indices would overflow      */
     APD_ERR_CUDA = 11,            /* a CUDA runtime call or a kernel launch failed        */
-    APD_ERR_ARGUMENT = 12         /* any other bad argument (e.g. a NULL output pointer)  */
+    APD_ERR_ARGUMENT = 12,        /* any other bad argument (e.g. a NULL output pointer)  */
+    APD_ERR_SCRATCH_LIMIT = 13    /* apd_attn_paged_decode_noalloc: the problem needs more
+                                     scratch than APD_NOALLOC_SCRATCH_BYTES               */
 } apd_status;
 
 /* Largest batch one call accepts (the per-sequence lengths and their prefix
@@ -190,6 +192,46 @@ int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, con
                              const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
                              float scale, int num_splits, void* workspace, size_t workspace_bytes,
                              apd_stream_t stream, const apd_launch_options* options);
+
+/*
+ * apd_attn_paged_decode_noalloc -- the same decode call for callers that cannot
+ * allocate device memory.  The pages have no counterpart of this entry point.
+ *
+ * Some callers have no way to obtain a workspace: a plugin handed only its input
+ * and output tensors by a host framework that owns every device allocation; code
+ * that runs under a fixed device-memory budget where a side allocation is not
+ * allowed; or code on a latency path where cudaMalloc, which can synchronise the
+ * device, is not acceptable.  This entry point needs no workspace: its scratch
+ * (the split partials, their running max and sum, and the per-sequence tile
+ * prefix sums) lives in one file-scope static device array of
+ * APD_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds until
+ * the process exits.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *
+ *   Arguments, layouts, checks, numerics and errors are those of
+ *   apd_attn_paged_decode, without `workspace` / `workspace_bytes`.
+ *   num_splits 0 (auto) plans as many parallel workers as the scratch holds
+ *              partials for (all of them for common shapes); num_splits >= 1
+ *              needs apd_workspace_size(...) <= APD_NOALLOC_SCRATCH_BYTES.
+ *   Returns APD_ERR_SCRATCH_LIMIT, before anything is launched, when the
+ *   problem needs more scratch than the array holds.
+ *
+ * Set-up: the first call on each device (with that device current) looks up the
+ * array's device address with cudaGetSymbolAddress, which can load the library's
+ * device code; make that first call before any stream capture.
+ *
+ * Sharing: every call in the process uses the same array on a given device, and
+ * the array keeps whatever the last call left in it.  No part of it has to start
+ * at zero (each call writes every partial and prefix sum it later reads).  Calls
+ * that can overlap on the GPU (unordered streams) race on the array and may
+ * return wrong results; order them on one stream or with events.  The sticky
+ * device flags of this entry point go to the array and are not reported.
+ */
+#define APD_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB per device */
+
+int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                                  const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                                  float scale, int num_splits, apd_stream_t stream);
 
 /*
  * apd_read_device_flags -- synchronise `stream`, copy the sticky APD_FLAG_* word

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(13):
+    for code in range(14):
         s = apd.status_string(code)
         assert s and s != "unknown status"
     assert apd.status_string(999) == "unknown status"
