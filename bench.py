@@ -113,25 +113,45 @@ def make_instances(name: str, rank: int, count: int = 2):
     return [gen(seed=base + 1000003 * rank + i) for i in range(count)]
 
 
+def _align(n: int, a: int) -> int:
+    return (n + a - 1) // a * a
+
+
 class Resident:
-    """A workload's tensors resident on the device, plus its workspace."""
+    """A workload resident on the device: KV cache, a packed [q | page_table | seq_lens]
+    buffer (so the end-to-end leg moves a step's inputs in one copy), out, workspace and
+    the prepared library call."""
 
     def __init__(self, w, device, num_splits, apd):
         self.w = w
-        self.q = w.q.to(device)
         self.k = w.k_cache.contiguous().to(device)
         self.v = w.v_cache.contiguous().to(device)
-        self.page_table = w.page_table.to(device)
-        self.seq_lens = w.seq_lens.to(device)
+        qb, pb, sb = w.q.numel() * 2, w.page_table.numel() * 4, w.seq_lens.numel() * 4
+        self.offsets = (0, _align(qb, 256), _align(qb, 256) + _align(pb, 256))
+        self.packed_bytes = self.offsets[2] + sb
+        host = torch.zeros(self.packed_bytes, dtype=torch.uint8)
+        self._views(host)[0].copy_(w.q)
+        self._views(host)[1].copy_(w.page_table)
+        self._views(host)[2].copy_(w.seq_lens)
+        self.host_packed = host.pin_memory()
+        self.dev_packed = self.host_packed.to(device)
+        self.q, self.page_table, self.seq_lens = self._views(self.dev_packed)
         self.out = torch.empty_like(self.q)
+        self.host_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
         self.num_splits = num_splits
         self.ws = apd.alloc_workspace(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, num_splits,
                                       device=device)
+        self.call = apd.DecodeCall(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, w.scale,
+                                   num_splits, self.ws)
         self.bytes = w.algorithmic_bytes()
 
-    def call(self, apd, stream, **kw):
-        apd.attn_paged_decode(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, self.w.scale,
-                              self.num_splits, self.ws, stream=stream, **kw)
+    def _views(self, buf):
+        w = self.w
+        o = self.offsets
+        q = buf[o[0]:o[0] + w.q.numel() * 2].view(torch.bfloat16).view(w.q.shape)
+        pt = buf[o[1]:o[1] + w.page_table.numel() * 4].view(torch.int32).view(w.page_table.shape)
+        sl = buf[o[2]:o[2] + w.seq_lens.numel() * 4].view(torch.int32).view(w.seq_lens.shape)
+        return q, pt, sl
 
 
 # ---------------------------------------------------------------- clocks
@@ -218,8 +238,8 @@ def committed_traffic(workload: str):
     return t.get("dram_bytes_per_launch")
 
 
-def time_steps(insts, apd, stream, steps, split_events=False):
-    """Run `steps` calls rotating over the instances; returns (elapsed_s, mean split-kernel s or None)."""
+def time_steps(insts, stream, steps, split_events=False):
+    """Eager calls rotating over the instances; returns (elapsed_s, mean split-kernel s or None)."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     per = []
@@ -231,9 +251,9 @@ def time_steps(insts, apd, stream, steps, split_events=False):
         if split_events:
             b, m = per[i]
             b.record(stream)
-            inst.call(apd, stream, split_done_event=m)
+            inst.call(stream, split_done_event=m)
         else:
-            inst.call(apd, stream)
+            inst.call(stream)
     end.record(stream)
     end.synchronize()
     elapsed = start.elapsed_time(end) / 1e3
@@ -243,29 +263,89 @@ def time_steps(insts, apd, stream, steps, split_events=False):
     return elapsed, split
 
 
-def e2e_steps(insts, apd, stream, steps):
-    """Per step: pinned-host -> device copies of q, page_table, seq_lens; the call;
-    device -> pinned-host copy of out.  Returns (elapsed_s, h2d bytes, d2h bytes) per step."""
-    hosts = []
-    for inst in insts:
-        hosts.append({
-            "q": inst.w.q.pin_memory(), "pt": inst.w.page_table.pin_memory(), "sl": inst.w.seq_lens.pin_memory(),
-            "out": torch.empty(inst.out.shape, dtype=inst.out.dtype).pin_memory(),
-        })
-    h2d = insts[0].q.nbytes + insts[0].page_table.nbytes + insts[0].seq_lens.nbytes
+GRAPH_CHUNK = 100
+
+
+class GraphSteps:
+    """CUDA graphs of consecutive calls (rotating over the instances): `steps` calls in
+    all, as steps // GRAPH_CHUNK replays of a GRAPH_CHUNK-call graph plus one graph of
+    the remainder."""
+
+    def __init__(self, insts, stream, steps):
+        self.plan = []
+        full, rest = divmod(steps, GRAPH_CHUNK)
+        if full:
+            self.plan.append((self._capture(insts, stream, GRAPH_CHUNK), full))
+        if rest:
+            self.plan.append((self._capture(insts, stream, rest), 1))
+
+    @staticmethod
+    def _capture(insts, stream, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    insts[i % len(insts)].call(stream)
+        return g
+
+    def run(self, stream):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for g, reps in self.plan:
+                for _ in range(reps):
+                    g.replay()
+            end.record(stream)
+        end.synchronize()
+        return start.elapsed_time(end) / 1e3
+
+    def release(self):
+        self.plan = []
+
+
+def e2e_steps(insts, stream, steps):
+    """End to end through the public API with host buffers.  Per step: one pinned-host
+    -> device copy of the packed [q | page_table | seq_lens] inputs, the call, and one
+    device -> pinned-host copy of out.  Copies run on two copy streams so that step
+    i+1's inputs and step i-1's output move while step i computes; events keep every
+    buffer's reuse ordered (instance j is used by steps j, j+2, ...).
+    Returns (elapsed_s, h2d bytes, d2h bytes) per step."""
+    dev = insts[0].q.device
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = len(insts)
+    computed = [torch.cuda.Event() for _ in range(n)]
+    out_copied = [torch.cuda.Event() for _ in range(n)]
+    in_ready = [torch.cuda.Event() for _ in range(n)]
+    used = [False] * n
+    h2d = insts[0].packed_bytes
     d2h = insts[0].out.nbytes
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for i in range(steps):
-            inst, h = insts[i % len(insts)], hosts[i % len(insts)]
-            inst.q.copy_(h["q"], non_blocking=True)
-            inst.page_table.copy_(h["pt"], non_blocking=True)
-            inst.seq_lens.copy_(h["sl"], non_blocking=True)
-            inst.call(apd, stream)
-            h["out"].copy_(inst.out, non_blocking=True)
-        end.record(stream)
+    start.record(stream)
+    h2d_s.wait_stream(stream)
+    d2h_s.wait_stream(stream)
+    for i in range(steps):
+        j = i % n
+        inst = insts[j]
+        with torch.cuda.stream(h2d_s):
+            if used[j]:
+                h2d_s.wait_event(computed[j])  # the previous call on these buffers has read its inputs
+            inst.dev_packed.copy_(inst.host_packed, non_blocking=True)
+            in_ready[j].record(h2d_s)
+        stream.wait_event(in_ready[j])
+        if used[j]:
+            stream.wait_event(out_copied[j])  # the previous output of these buffers has left the device
+        inst.call(stream)
+        computed[j].record(stream)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(computed[j])
+            inst.host_out.copy_(inst.out, non_blocking=True)
+            out_copied[j].record(d2h_s)
+        used[j] = True
+    stream.wait_stream(d2h_s)
+    stream.wait_stream(h2d_s)
+    end.record(stream)
     end.synchronize()
     return start.elapsed_time(end) / 1e3, h2d, d2h
 
@@ -341,14 +421,13 @@ def run_reference(a):
 
 
 def config_of(w, a):
-    d = w.describe()
-    d.pop("seed", None)
     return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "page_size": w.page_size, "kv_tokens": w.kv_tokens(),
             "num_splits": a.num_splits, "layout": w.layout,
             "l2": "two independent instances used in turn (each call reads KV the previous call did not touch); "
                   "large workloads are each larger than L2",
-            "algorithmic_bytes_per_call": w.algorithmic_bytes()}
+            "algorithmic_bytes_per_call": w.algorithmic_bytes(),
+            "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"}
 
 
 def run_ours(a):
@@ -374,40 +453,52 @@ def run_ours(a):
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize(device)
 
-    # warm-up
-    time_steps(insts, apd, stream, a.warmup)
+    # warm-up (eager), then capture the timed calls as CUDA graphs and run them once untimed
+    time_steps(insts, stream, a.warmup)
+    graphs = GraphSteps(insts, stream, a.steps)
+    graphs.run(stream)
 
-    # main timed region
+    # main timed region: exactly `steps` calls, replayed from the graphs
     clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
     barrier(dist, device)
     torch.cuda.synchronize(device)
-    elapsed, _ = time_steps(insts, apd, stream, a.steps)
+    elapsed = graphs.run(stream)
     torch.cuda.synchronize(device)
     barrier(dist, device)
     clock_info = clocks.stop()
+    graphs.release()
     bytes_rank = sum(insts[i % 2].bytes for i in range(a.steps))
     t_max = max_over_ranks(elapsed, dist, device)
     bytes_all = sum_over_ranks(float(bytes_rank), dist, device)
     value = bytes_all / t_max / 1e9
 
+    # the same steps launched eagerly from Python, for reference
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    eager_el, _ = time_steps(insts, stream, a.steps)
+    eager_max = max_over_ranks(eager_el, dist, device)
+
     # split-kernel duration: the same steps with an event between the two kernels
     barrier(dist, device)
     torch.cuda.synchronize(device)
-    _, split_s = time_steps(insts, apd, stream, a.steps, split_events=True)
+    _, split_s = time_steps(insts, stream, a.steps, split_events=True)
     torch.cuda.synchronize(device)
     split_s = max_over_ranks(split_s, dist, device)
 
     # end to end through host buffers
     e2e = None
     if not a.no_e2e:
-        time_steps(insts, apd, stream, 3)
+        time_steps(insts, stream, 3)
         barrier(dist, device)
         torch.cuda.synchronize(device)
-        e_el, h2d, d2h = e2e_steps(insts, apd, stream, a.steps)
+        e_el, h2d, d2h = e2e_steps(insts, stream, a.steps)
         torch.cuda.synchronize(device)
         e_max = max_over_ranks(e_el, dist, device)
         e2e = {"value": bytes_all / e_max / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e_max / a.steps * 1e3}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_max / a.steps * 1e3,
+               "how": "per step, eager through the public Python API: one pinned-host->device copy of the "
+                      "packed q|page_table|seq_lens, the call, one device->pinned-host copy of out; copies on "
+                      "two copy streams overlap the neighbouring steps' compute"}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -421,6 +512,7 @@ def run_ours(a):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
             "ms_per_step": t_max / a.steps * 1e3, "us_per_call": t_max / a.steps * 1e6,
+            "eager_us_per_call": eager_max / a.steps * 1e6,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": config_of(w0, a),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,

@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "APDError",
     "attn_paged_decode",
+    "DecodeCall",
     "attn_paged_decode_noalloc",
     "NOALLOC_SCRATCH_BYTES",
     "workspace_size",
@@ -144,19 +145,18 @@ def status_string(status: int) -> str:
     return _load().apd_status_string(int(status)).decode()
 
 
+_I64x4 = ctypes.c_int64 * 4
+
+
 def _desc(t: torch.Tensor | None) -> _Tensor:
-    d = _Tensor()
     if t is None:
-        return d
-    if t.dim() > 4:
+        return _Tensor()
+    n = t.dim()
+    if n > 4:
         raise ValueError("tensors passed to the library have at most 4 dimensions")
-    d.data = t.data_ptr() if t.numel() > 0 or t.data_ptr() else None
-    d.dtype = _DTYPES.get(t.dtype, 0)
-    d.ndim = t.dim()
-    for i in range(t.dim()):
-        d.shape[i] = t.shape[i]
-        d.stride[i] = t.stride(i)
-    return d
+    pad = (0,) * (4 - n)
+    return _Tensor(t.data_ptr() or None, _DTYPES.get(t.dtype, 0), n, _I64x4(*t.shape, *pad),
+                   _I64x4(*t.stride(), *pad))
 
 
 def _stream_handle(stream, device) -> int | None:
@@ -239,6 +239,47 @@ def attn_paged_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     if rc:
         raise APDError(rc, "apd_attn_paged_decode_noalloc")
     return out
+
+
+class DecodeCall:
+    """apd_attn_paged_decode with its arguments marshalled once, for repeated calls on
+    the same buffers (a decode loop, a benchmark, a CUDA-graph capture).  Calling the
+    object enqueues one decode call; the tensors' contents may change between calls,
+    their storage, shapes and strides may not."""
+
+    def __init__(self, q, k_cache, v_cache, page_table, seq_lens, out, scale: float, num_splits: int = 0,
+                 workspace: torch.Tensor | None = None):
+        if workspace is None:
+            workspace = alloc_workspace(q.shape[0], q.shape[1], k_cache.shape[2], q.shape[2], num_splits,
+                                        device=q.device)
+        self.tensors = (q, k_cache, v_cache, page_table, seq_lens, out, workspace)
+        self.device = q.device
+        self._descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+        self._head = tuple(ctypes.byref(d) for d in self._descs) + (
+            ctypes.c_float(scale), int(num_splits), workspace.data_ptr(), workspace.numel() * workspace.element_size())
+        self._opts = _Options()
+        self._opts_ref = ctypes.byref(self._opts)
+        self._lib = _load()
+
+    @property
+    def out(self) -> torch.Tensor:
+        return self.tensors[5]
+
+    @property
+    def workspace(self) -> torch.Tensor:
+        return self.tensors[6]
+
+    def __call__(self, stream=None, split_done_event=None) -> None:
+        st = _stream_handle(stream, self.device)
+        if split_done_event is None:
+            rc = self._lib.apd_attn_paged_decode(*self._head, st)
+        else:
+            if not split_done_event.cuda_event:  # torch creates its events lazily, at the first record
+                split_done_event.record(torch.cuda.current_stream(self.device) if stream is None else stream)
+            self._opts.split_done_event = split_done_event.cuda_event
+            rc = self._lib.apd_attn_paged_decode_ex(*self._head, st, self._opts_ref)
+        if rc:
+            raise APDError(rc, "apd_attn_paged_decode")
 
 
 def read_device_flags(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:

@@ -131,7 +131,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         }
         pl->workers = static_cast<int>(workers);
         pl->slots = 2 * workers;
-        pl->combine_ctas = static_cast<int>(s.units);
+        pl->combine_ctas = static_cast<int>(s.units * s.rows_max);
     } else {
         pl->mode = 1;
         pl->ksplit = num_splits;
@@ -139,7 +139,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         if (workers > INT32_MAX / 2) return APD_ERR_TOO_LARGE;
         pl->workers = static_cast<int>(workers);
         pl->slots = num_splits >= 2 ? workers : 0;
-        pl->combine_ctas = num_splits >= 2 ? static_cast<int>(s.units) : 0;
+        pl->combine_ctas = num_splits >= 2 ? static_cast<int>(s.units * s.rows_max) : 0;
     }
     pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
     pl->ws_needed = ws_bytes_for(s, pl->slots);
@@ -373,14 +373,29 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     sp.q_box_bytes = static_cast<uint32_t>(s.rows_max) * s.D * 2u;
     sp.scale_log2 = scale * 1.4426950408889634f;
 
-    kern<<<pl.ctas, pl.warps * 32, pl.smem, stream>>>(sp, kmap, vmap, qmap);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "split_kernel launch");
+    // Both kernels are launched with programmatic dependent launch (PDL): each
+    // begins launching while the previous kernel in the stream drains, and waits
+    // (griddepcontrol.wait) for it before touching global memory.
+    const bool use_pdl = !(opts && opts->disable_pdl);
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(pl.ctas));
+        cfg.blockDim = dim3(static_cast<unsigned>(pl.warps * 32));
+        cfg.dynamicSmemBytes = pl.smem;
+        cfg.stream = stream;
+        cfg.attrs = pdl_attr;
+        cfg.numAttrs = use_pdl ? 1 : 0;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, kern, sp, kmap, vmap, qmap);
+        if (e != cudaSuccess) return cuda_fail(e, "split_kernel launch");
+    }
+    cudaError_t e = cudaSuccess;
     if (opts && opts->split_done_event) {
         e = cudaEventRecord(static_cast<cudaEvent_t>(opts->split_done_event), stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(split_done_event)");
     }
-    const bool use_pdl = !(opts && (opts->disable_pdl || opts->split_done_event));
 
     if (pl.combine_ctas > 0) {
         apd::CombineParams cp;
@@ -399,15 +414,12 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
         cp.ksplit = pl.ksplit;
         cp.num_workers = pl.workers;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(pl.combine_ctas));
-        cfg.blockDim = dim3(128);
+        cfg.gridDim = dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
+        cfg.blockDim = dim3(32 * apd::kCombineWarps);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = use_pdl ? 1 : 0;
+        cfg.attrs = pdl_attr;
+        cfg.numAttrs = (use_pdl && !(opts && opts->split_done_event)) ? 1 : 0;
         e = cudaLaunchKernelEx(&cfg, apd::combine_kernel<D>, cp);
         if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
     }

@@ -139,7 +139,7 @@ __device__ __forceinline__ int32_t fetch_page(const SplitParams& p, const int32_
     int b, ul, j, n;
     decode_tile(i, units_per_seq, cum, p.B, b, ul, j, n);
     const int pj = (j * kTile) / p.P;
-    return __ldg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 + static_cast<int64_t>(pj) * p.pt_s1);
+    return __ldcg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 + static_cast<int64_t>(pj) * p.pt_s1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -181,12 +181,17 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
+    // Launched with programmatic dependent launch: this CTA may start while the
+    // previous kernel in the stream is still running.  Nothing above touches
+    // global memory; from here on, that kernel has finished and its writes are
+    // visible.
+    pdl_wait_prior_grid();
 
     // ---- per-sequence tile counts and their prefix sum (every CTA, from L2)
     const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
     uint32_t len_flags = 0;
     for (int b = tid; b < B; b += blockDim.x) {
-        int L = __ldg(p.seq_lens + b);
+        int L = __ldcg(p.seq_lens + b);
         if (L < 0) {
             L = 0;
             len_flags |= kFlagLenNegative;
@@ -541,98 +546,160 @@ __device__ __forceinline__ int64_t run_start(int w, int64_t total, int workers) 
     return static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / workers);
 }
 
-// One CTA per unit (b, kv head, head block).  Merges the unit's partials:
-// M = max_s m_s over non-empty partials, out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
-// In balanced mode it also writes zeros for empty sequences.
+constexpr int kCombineWarps = 4;
+constexpr int kCombineBatch = 4;  // partial slots whose loads a warp issues together
+
+// One CTA per (unit, head row).  Merges the row's partials:
+//   M = max_s m_s over non-empty partials,
+//   out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// The CTA's warps split the unit's partial slots and each keeps a running
+// (max, sum, acc) over its share, loading kCombineBatch slots at a time; each
+// lane owns float4 columns of the row.  The warps' states are merged through
+// shared memory.  In balanced mode it also writes zeros for empty sequences.
 template <int D>
-__global__ void __launch_bounds__(128) combine_kernel(const __grid_constant__ CombineParams p) {
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __grid_constant__ CombineParams p) {
+    constexpr int kCols = D / 4;                 // float4 columns of a row
+    constexpr int kPerLane = (kCols + 31) / 32;  // float4 columns per lane
+    __shared__ float4 s_acc[kCombineWarps][kCols];
+    __shared__ float s_m[kCombineWarps], s_den[kCombineWarps];
+
+    // Every CTA of this grid is resident once it gets here, so the next kernel in
+    // the stream may begin launching (it waits for this grid before reading).
+    pdl_launch_dependents();
+
     const int u = blockIdx.x;
+    const int r = blockIdx.y;
     const int units_per_seq = p.Hkv * p.HB;
     const int b = u / units_per_seq;
     const int ul = u - b * units_per_seq;
     const int kvh = ul / p.HB;
     const int hb = ul - kvh * p.HB;
     const int rows = min(kMaxRows, p.g - kMaxRows * hb);
-    const int head0 = kvh * p.g + kMaxRows * hb;
-    constexpr int kQuads = D / 4;
+    if (r >= rows) return;
+    const int head = kvh * p.g + kMaxRows * hb + r;
+    __nv_bfloat16* orow = p.out + b * p.out_sb + head * p.out_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     pdl_wait_prior_grid();
     const int n = p.cum[b + 1] - p.cum[b];
     if (n == 0) {
-        if (p.mode == 0) {
-            for (int it = threadIdx.x; it < rows * kQuads; it += blockDim.x) {
-                const int r = it / kQuads, q4 = it - (it / kQuads) * kQuads;
-                *reinterpret_cast<uint2*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 4 * q4) = make_uint2(0u, 0u);
-            }
-        }
+        if (p.mode == 0)
+            for (int c = tid; c < kCols; c += blockDim.x) *reinterpret_cast<uint2*>(orow + 4 * c) = make_uint2(0u, 0u);
         return;
     }
 
-    // slot list: (first, count) for fixed mode; worker range for balanced mode
-    int w_first = 0, w_last = -1, first_slot_fixed = 0, nslots_fixed = 0;
+    // The unit's partial slots, numbered k = 0 .. nk-1.
+    int nk, w_first = 0, first_slot_fixed = 0;
     int64_t total = 0, Tu = 0;
     if (p.mode == 0) {
         total = static_cast<int64_t>(units_per_seq) * p.cum[p.B];
         Tu = static_cast<int64_t>(units_per_seq) * p.cum[b] + static_cast<int64_t>(ul) * n;
         w_first = worker_of(Tu, total, p.num_workers);
-        w_last = worker_of(Tu + n - 1, total, p.num_workers);
+        const int w_last = worker_of(Tu + n - 1, total, p.num_workers);
         if (w_first == w_last) return;  // one worker covered it and wrote the output
+        nk = w_last - w_first + 1;
     } else {
         const int S = min(p.ksplit, n);
         const int c = (n + S - 1) / S;
-        nslots_fixed = (n + c - 1) / c;
-        if (nslots_fixed == 1) return;
+        nk = (n + c - 1) / c;
+        if (nk == 1) return;
         first_slot_fixed = u * p.ksplit;
     }
+    // slot of partial k, or -1 for a worker whose run is empty (it wrote nothing)
+    auto slot_of = [&](int k) -> int64_t {
+        if (p.mode != 0) return first_slot_fixed + k;
+        const int w = w_first + k;
+        const int64_t a = run_start(w, total, p.num_workers);
+        if (a == run_start(w + 1, total, p.num_workers)) return -1;
+        return 2 * static_cast<int64_t>(w) + ((k == 0 && a != Tu) ? 1 : 0);
+    };
 
-    for (int it = threadIdx.x; it < rows * kQuads; it += blockDim.x) {
-        const int r = it / kQuads;
-        const int q4 = it - r * kQuads;
-        float M = -INFINITY;
-        // pass 1: the common max
-        if (p.mode == 0) {
-            for (int w = w_first; w <= w_last; ++w) {
-                const int64_t a = run_start(w, total, p.num_workers);
-                if (a == run_start(w + 1, total, p.num_workers)) continue;
-                const int64_t slot = 2 * static_cast<int64_t>(w) + ((w == w_first && a != Tu) ? 1 : 0);
-                const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
-                if (ml.y > 0.f) M = fmaxf(M, ml.x);
-            }
-        } else {
-            for (int s = 0; s < nslots_fixed; ++s) {
-                const int64_t slot = first_slot_fixed + s;
-                const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
-                if (ml.y > 0.f) M = fmaxf(M, ml.x);
+    float M = -INFINITY, den = 0.f;
+    float4 acc[kPerLane];
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k0 = warp; k0 < nk; k0 += kCombineBatch * kCombineWarps) {
+        float2 ml[kCombineBatch];
+        float4 o[kCombineBatch][kPerLane];
+#pragma unroll
+        for (int t = 0; t < kCombineBatch; ++t) {
+            const int k = k0 + t * kCombineWarps;
+            const int64_t slot = k < nk ? slot_of(k) : -1;
+            ml[t] = make_float2(-INFINITY, 0.f);
+            if (slot >= 0) {
+                ml[t] = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
+                const float4* src = reinterpret_cast<const float4*>(p.o_part + (slot * p.rows_max + r) * D);
+#pragma unroll
+                for (int j = 0; j < kPerLane; ++j) {
+                    const int c = lane + 32 * j;
+                    o[t][j] = c < kCols ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
             }
         }
-        // pass 2: weighted sums
-        float den = 0.f;
-        float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-        auto add = [&](int64_t slot) {
-            const float2 ml = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
-            if (!(ml.y > 0.f)) return;
-            const float wgt = exp2f(ml.x - M);
-            den += wgt * ml.y;
-            const float4 a = *reinterpret_cast<const float4*>(p.o_part + (slot * p.rows_max + r) * D + 4 * q4);
-            num.x += wgt * a.x;
-            num.y += wgt * a.y;
-            num.z += wgt * a.z;
-            num.w += wgt * a.w;
-        };
-        if (p.mode == 0) {
-            for (int w = w_first; w <= w_last; ++w) {
-                const int64_t a = run_start(w, total, p.num_workers);
-                if (a == run_start(w + 1, total, p.num_workers)) continue;
-                add(2 * static_cast<int64_t>(w) + ((w == w_first && a != Tu) ? 1 : 0));
+#pragma unroll
+        for (int t = 0; t < kCombineBatch; ++t) {
+            if (!(ml[t].y > 0.f)) continue;  // empty split or no slot
+            if (ml[t].x > M) {
+                const float sc = exp2f(M - ml[t].x);  // 0 while M is -inf (acc and den are 0 then)
+                den *= sc;
+#pragma unroll
+                for (int j = 0; j < kPerLane; ++j) {
+                    acc[j].x *= sc;
+                    acc[j].y *= sc;
+                    acc[j].z *= sc;
+                    acc[j].w *= sc;
+                }
+                M = ml[t].x;
             }
-        } else {
-            for (int s = 0; s < nslots_fixed; ++s) add(first_slot_fixed + s);
+            const float wgt = exp2f(ml[t].x - M);
+            den += wgt * ml[t].y;
+#pragma unroll
+            for (int j = 0; j < kPerLane; ++j) {
+                acc[j].x += wgt * o[t][j].x;
+                acc[j].y += wgt * o[t][j].y;
+                acc[j].z += wgt * o[t][j].z;
+                acc[j].w += wgt * o[t][j].w;
+            }
         }
-        const float inv = 1.f / den;
+    }
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+        const int c = lane + 32 * j;
+        if (c < kCols) s_acc[warp][c] = acc[j];
+    }
+    if (lane == 0) {
+        s_m[warp] = M;
+        s_den[warp] = den;
+    }
+    __syncthreads();
+
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w)
+        if (s_den[w] > 0.f) Mt = fmaxf(Mt, s_m[w]);
+    float wt[kCombineWarps];
+    float dsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+        wt[w] = s_den[w] > 0.f ? exp2f(s_m[w] - Mt) : 0.f;
+        dsum += wt[w] * s_den[w];
+    }
+    const float inv = 1.f / dsum;
+    for (int c = tid; c < kCols; c += blockDim.x) {
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) {
+            if (wt[w] == 0.f) continue;
+            const float4 a = s_acc[w][c];
+            t.x += wt[w] * a.x;
+            t.y += wt[w] * a.y;
+            t.z += wt[w] * a.z;
+            t.w += wt[w] * a.w;
+        }
         uint2 packed;
-        packed.x = pack_bf16x2(num.x * inv, num.y * inv);
-        packed.y = pack_bf16x2(num.z * inv, num.w * inv);
-        *reinterpret_cast<uint2*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 4 * q4) = packed;
+        packed.x = pack_bf16x2(t.x * inv, t.y * inv);
+        packed.y = pack_bf16x2(t.z * inv, t.w * inv);
+        *reinterpret_cast<uint2*>(orow + 4 * c) = packed;
     }
 }
 

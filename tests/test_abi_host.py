@@ -209,7 +209,7 @@ def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     assert pl.num_workers == 148 * pl.warps_per_cta
     assert pl.partial_slots == 2 * pl.num_workers
     assert pl.rows_per_unit == min(g, 16) and pl.head_blocks == -(-g // 16)
-    assert pl.combine_ctas == B * Hkv * pl.head_blocks
+    assert pl.combine_ctas == B * Hkv * pl.head_blocks * pl.rows_per_unit
     assert pl.smem_bytes <= 232448
     assert pl.workspace_bytes % 256 == 0
     assert pl.workspace_bytes == apd.lib().apd_workspace_size(B, Hq, Hkv, D, 0)
@@ -224,7 +224,7 @@ def test_plan_fixed(splits):
     assert pl.num_workers == units * splits
     assert pl.grid_ctas == -(-pl.num_workers // pl.warps_per_cta)
     assert pl.partial_slots == (units * splits if splits > 1 else 0)
-    assert pl.combine_ctas == (units if splits > 1 else 0)
+    assert pl.combine_ctas == (units * pl.rows_per_unit if splits > 1 else 0)
     assert pl.workspace_bytes == apd.workspace_size(B, Hq, Hkv, D, splits)
 
 
