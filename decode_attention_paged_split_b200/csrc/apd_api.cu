@@ -259,8 +259,9 @@ int validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, cons
 }
 
 // ---------------------------------------------------------------- TMA maps
-// K/V: D >= 64 -> 5-D view {64, D/64, Hkv, P, NP}, box {64, D/64, 1, 32, 1},
-//      128-byte swizzle (one box = one [32 x D] tile, rows of 2*D bytes).
+// K/V: D >= 64 -> 5-D view {64, Hkv, P, NP, D/64}, box {64, 1, 32, 1, D/64},
+//      128-byte swizzle: one box = one [32 x D] tile of one kv head, landing in
+//      shared memory as D/64 blocks of [32 tokens][64 elements].
 //      D == 32 -> 4-D view {32, Hkv, P, NP}, box {32, 1, 32, 1}, 64-byte swizzle.
 int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D) {
     auto fn = encode_fn();
@@ -271,9 +272,9 @@ int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int 
     CUtensorMapSwizzle swz;
     if (D >= 64) {
         rank = 5;
-        dims[0] = 64; dims[1] = D / 64; dims[2] = t->shape[2]; dims[3] = t->shape[1]; dims[4] = t->shape[0];
-        strides[0] = 128; strides[1] = st[2] * 2; strides[2] = st[1] * 2; strides[3] = st[0] * 2;
-        box[0] = 64; box[1] = D / 64; box[2] = 1; box[3] = apd::kTile; box[4] = 1;
+        dims[0] = 64; dims[1] = t->shape[2]; dims[2] = t->shape[1]; dims[3] = t->shape[0]; dims[4] = D / 64;
+        strides[0] = st[2] * 2; strides[1] = st[1] * 2; strides[2] = st[0] * 2; strides[3] = 128;
+        box[0] = 64; box[1] = 1; box[2] = apd::kTile; box[3] = 1; box[4] = D / 64;
         swz = CU_TENSOR_MAP_SWIZZLE_128B;
     } else {
         rank = 4;
@@ -289,7 +290,8 @@ int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int 
     return APD_OK;
 }
 
-// Q: D >= 64 -> 4-D view {64, D/64, Hq, B}, box {64, D/64, rows_max, 1};
+// Q: D >= 64 -> 4-D view {64, Hq, B, D/64}, box {64, rows_max, 1, D/64}
+//    (D/64 blocks of [rows_max][64] in shared memory);
 //    D == 32 -> 3-D view {32, Hq, B}, box {32, rows_max, 1}.
 int encode_q_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D, int rows_max) {
     auto fn = encode_fn();
@@ -300,9 +302,9 @@ int encode_q_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D
     CUtensorMapSwizzle swz;
     if (D >= 64) {
         rank = 4;
-        dims[0] = 64; dims[1] = D / 64; dims[2] = t->shape[1]; dims[3] = t->shape[0];
-        strides[0] = 128; strides[1] = st[1] * 2; strides[2] = st[0] * 2;
-        box[0] = 64; box[1] = D / 64; box[2] = rows_max; box[3] = 1;
+        dims[0] = 64; dims[1] = t->shape[1]; dims[2] = t->shape[0]; dims[3] = D / 64;
+        strides[0] = st[1] * 2; strides[1] = st[0] * 2; strides[2] = 128;
+        box[0] = 64; box[1] = rows_max; box[2] = 1; box[3] = D / 64;
         swz = CU_TENSOR_MAP_SWIZZLE_128B;
     } else {
         rank = 3;

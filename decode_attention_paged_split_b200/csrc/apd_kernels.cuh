@@ -21,7 +21,8 @@
 //    combine kernel merges the partials of each unit.
 //  * Each warp runs its own STAGES-deep ring in shared memory.  Lane 0 issues
 //    TMA tiled loads (cp.async.bulk.tensor, 128-byte swizzle) of the K and V
-//    tiles [32 tokens x D] of the next tiles straight from the paged cache,
+//    tiles [32 tokens x D] of the next tiles straight from the paged cache
+//    (stored as D/64 blocks of [32 tokens][64], conflict-free for ldmatrix),
 //    plus the unit's query rows when a unit starts; completion is tracked by
 //    mbarrier transaction bytes.  Page-table entries are fetched 32 tiles ahead,
 //    one coalesced load per warp.  Page indices outside the pool read as zeros
@@ -84,7 +85,6 @@ struct Geometry {
     static constexpr int kSteps = D / 16;              // k-steps of QK^T
     static constexpr int kNTiles = D / 8;              // 8-wide n-tiles of PV
     static constexpr int kChunks = D / 8;              // 16-byte chunks per row
-    static constexpr uint32_t kRowBytes = D * 2;
     static constexpr uint32_t kKVTileBytes = kTile * D * 2;
     // TMA swizzle applied to a byte offset from a 1024-aligned base:
     // 128B mode XORs address bits [4:6] with [7:9]; 64B mode bits [4:5] with [7:8].
@@ -93,6 +93,18 @@ struct Geometry {
             return off ^ (((off >> 7) & 3u) << 4);
         } else {
             return off ^ (((off >> 7) & 7u) << 4);
+        }
+    }
+    // Byte offset of 16-byte chunk `ch` (8 elements of the head dim) of row `row`
+    // in a staged tile of `rows` rows.  D >= 64: the tile is stored as D/64 blocks
+    // of [rows][64 elements], so each 128-byte swizzle row is one token (or query
+    // head) and the 8 rows an ldmatrix reads fall in 8 distinct swizzle phases
+    // (no bank conflicts).  D == 32: [rows][32 elements] with the 64-byte swizzle.
+    __device__ __forceinline__ static uint32_t chunk_off(int row, int ch, int rows) {
+        if constexpr (D == 32) {
+            return swz(static_cast<uint32_t>(row * 64 + ch * 16));
+        } else {
+            return swz(static_cast<uint32_t>((ch >> 3) * rows * 128 + row * 128 + (ch & 7) * 16));
         }
     }
 };
@@ -313,10 +325,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
                 if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, kvh * p.g + kMaxRows * hb, pb,
                                        pol_keep);
             } else {
-                tma_load_5d(sbase, &kmap, bar, 0, 0, kvh, slot, page, pol_stream);
-                tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, 0, kvh, slot, page, pol_stream);
-                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, 0, kvh * p.g + kMaxRows * hb,
-                                       pb, pol_keep);
+                tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, page, 0, pol_stream);
+                tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, 0, pol_stream);
+                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, kvh * p.g + kMaxRows * hb, pb, 0,
+                                       pol_keep);
             }
         }
         ++pi;
@@ -378,7 +390,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 #pragma unroll
             for (int ks = 0; ks < G::kSteps; ++ks) {
                 const uint32_t ch = 2 * ks + (mi >> 1);
-                ldsm_x4(qbase + G::swz(qrow * G::kRowBytes + ch * 16), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+                ldsm_x4(qbase + G::chunk_off(qrow, ch, p.rows_max), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
                 if (gq >= rows) qf[ks][0] = qf[ks][2] = 0u;
                 if (gq + 8 >= rows) qf[ks][1] = qf[ks][3] = 0u;
             }
@@ -397,7 +409,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
                     const int row = 8 * (2 * np + (mi >> 1)) + (lane & 7);
                     const uint32_t ch = 2 * ks + (mi & 1);
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4(sbase + G::swz(row * G::kRowBytes + ch * 16), b0, b1, b2, b3);
+                    ldsm_x4(sbase + G::chunk_off(row, ch, kTile), b0, b1, b2, b3);
                     mma_bf16_16816(s[2 * np], qf[ks], b0, b1);
                     mma_bf16_16816(s[2 * np + 1], qf[ks], b2, b3);
                 }
@@ -412,7 +424,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             for (int idx = lane; idx < (kTile - valid) * G::kChunks; idx += 32) {
                 const int r = valid + idx / G::kChunks;
                 const int ch = idx % G::kChunks;
-                st_shared_zero16(vb + G::swz(r * G::kRowBytes + ch * 16));
+                st_shared_zero16(vb + G::chunk_off(r, ch, kTile));
             }
             __syncwarp();
         }
@@ -478,7 +490,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
                     const int row = 16 * kk + 8 * (mi & 1) + (lane & 7);
                     const uint32_t ch = nd + (mi >> 1);
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_trans(vb + G::swz(row * G::kRowBytes + ch * 16), b0, b1, b2, b3);
+                    ldsm_x4_trans(vb + G::chunk_off(row, ch, kTile), b0, b1, b2, b3);
                     mma_bf16_16816(acc[nd], pa[kk], b0, b1);
                     mma_bf16_16816(acc[nd + 1], pa[kk], b2, b3);
                 }
