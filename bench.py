@@ -107,10 +107,11 @@ def barrier(dist, device=None):
 
 # ---------------------------------------------------------------- inputs
 def make_instances(name: str, rank: int, count: int = 2):
-    """`count` independent instances of the named workload; seeds differ per rank and instance."""
+    """`count` instances of the named workload with the same structure (lengths, page
+    table) and independent values; the seed of the values differs per rank and instance."""
     gen = workloads.NAMED[name]
     base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262}[name]
-    return [gen(seed=base + 1000003 * rank + i) for i in range(count)]
+    return [gen(seed=base, value_seed=base + 1000003 * rank + i) for i in range(count)]
 
 
 def _align(n: int, a: int) -> int:

@@ -71,6 +71,9 @@ def test_instances_differ_per_rank_and_instance():
     b0, = bench.make_instances("tiny", 1, 1)
     assert not torch.equal(a0.q, a1.q) and not torch.equal(a0.q, b0.q)
     assert a0.q.shape == b0.q.shape and a0.algorithmic_bytes() == b0.algorithmic_bytes()
+    r0, r1 = bench.make_instances("ragged", 0, 2)
+    assert torch.equal(r0.seq_lens, r1.seq_lens) and torch.equal(r0.page_table, r1.page_table)
+    assert r0.algorithmic_bytes() == r1.algorithmic_bytes() and not torch.equal(r0.q, r1.q)
 
 
 def test_reference_arm_prints_one_json_line():

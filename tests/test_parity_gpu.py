@@ -169,6 +169,33 @@ def test_cuda_graph_capture_and_replay(S):
     check_close(out, oracle.paged_decode(w), "graph replay with new q")
 
 
+def test_inputs_written_by_the_preceding_kernel_are_seen():
+    """The split kernel may start launching before the previous kernel in the stream
+    ends (programmatic dependent launch); it must still read q, page_table and
+    seq_lens only after that kernel's writes.  Each call here follows torch kernels
+    that rewrite those inputs in place."""
+    ws_len = (700, 64, 1500)
+    w = small(54, B=3, Hq=16, Hkv=4, D=128, lens=ws_len, pool=80, max_pages_per_seq=48)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(3, 16, 4, 128, 0)
+    call = apd.DecodeCall(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    qs = [torch.randn(3, 16, 128, generator=torch.Generator().manual_seed(i)).to(torch.bfloat16) for i in range(4)]
+    lens = [torch.tensor(x, dtype=torch.int32) for x in ((700, 64, 1500), (1, 1200, 33), (0, 1536, 640), (95, 5, 1))]
+    outs = []
+    qs_dev = [q.cuda() for q in qs]
+    lens_dev = [l.cuda() for l in lens]
+    for i in range(4):
+        dp.q.copy_(qs_dev[i])
+        dp.seq_lens.copy_(lens_dev[i])
+        call()
+        outs.append(dp.out.clone())
+    torch.cuda.synchronize()
+    for i in range(4):
+        w.q.copy_(qs[i])
+        w.seq_lens.copy_(lens[i])
+        check_close(outs[i], oracle.paged_decode(w), f"step {i}")
+
+
 def test_deterministic():
     w = workloads.sweep_case(128, 32, 8, 0)
     dp = DeviceProblem(w)

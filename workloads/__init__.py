@@ -182,8 +182,11 @@ def make(
     layout: str = "NHD",
     poison: bool = False,
     meta: dict | None = None,
+    value_seed: int | None = None,
 ) -> Workload:
-    """Build one seeded problem.  ``seq_lens`` is a list/array of B ints."""
+    """Build one seeded problem.  ``seq_lens`` is a list/array of B ints.  ``seed`` drives
+    the structure (page permutation); ``value_seed`` (default: ``seed``) drives the bf16
+    values, so two problems can share their structure and differ in their data."""
     lens = np.asarray(seq_lens, dtype=np.int64).reshape(-1)
     assert lens.shape[0] == batch and (lens >= 0).all()
     P = page_size
@@ -206,7 +209,8 @@ def make(
         pt[b, :n] = perm[cursor:cursor + n]
         cursor += n
 
-    q = seeded_randn_bf16(batch * num_q_heads * head_dim, seed, _S_Q).view(batch, num_q_heads, head_dim)
+    vseed = seed if value_seed is None else value_seed
+    q = seeded_randn_bf16(batch * num_q_heads * head_dim, vseed, _S_Q).view(batch, num_q_heads, head_dim)
     kv_numel = total_pages * P * num_kv_heads * head_dim
     if layout == "NHD":
         shape_store = (total_pages, P, num_kv_heads, head_dim)
@@ -216,10 +220,10 @@ def make(
         to_nhd = (0, 2, 1, 3)
     else:
         raise ValueError(f"unknown layout {layout!r}")
-    k_store = seeded_randn_bf16(kv_numel, seed, _S_K).view(*shape_store)
-    v_store = seeded_randn_bf16(kv_numel, seed, _S_V).view(*shape_store)
+    k_store = seeded_randn_bf16(kv_numel, vseed, _S_K).view(*shape_store)
+    v_store = seeded_randn_bf16(kv_numel, vseed, _S_V).view(*shape_store)
     if k_outlier_frac > 0.0:
-        mask = seeded_bernoulli(kv_numel, k_outlier_frac, seed, _S_KMASK).view(*shape_store)
+        mask = seeded_bernoulli(kv_numel, k_outlier_frac, vseed, _S_KMASK).view(*shape_store)
         k_store[mask] = k_store[mask] * k_outlier_mult  # x8 is exact in bf16
     k_cache = k_store.permute(*to_nhd)
     v_cache = v_store.permute(*to_nhd)
