@@ -39,7 +39,8 @@ import workloads  # noqa: E402
 
 METRIC = "paged decode attention achieved HBM GB/s (algorithmic KV+q+out bytes per call / time)"
 UNIT = "GB/s"
-DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000}
+DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000, "llama8b_contig": 20000,
+                 "long_contig": 5000}
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
 
@@ -110,7 +111,8 @@ def make_instances(name: str, rank: int, count: int = 2):
     """`count` instances of the named workload with the same structure (lengths, page
     table) and independent values; the seed of the values differs per rank and instance."""
     gen = workloads.NAMED[name]
-    base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262}[name]
+    base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262, "llama8b_contig": 8,
+            "long_contig": 131072}[name]
     return [gen(seed=base, value_seed=base + 1000003 * rank + i) for i in range(count)]
 
 
@@ -142,8 +144,9 @@ class Resident:
         self.num_splits = num_splits
         self.ws = apd.alloc_workspace(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, num_splits,
                                       device=device)
-        self.call = apd.DecodeCall(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, w.scale,
-                                   num_splits, self.ws)
+        self.contig = w.meta.get("kv_policy") == "contig"
+        self.call = apd.DecodeCall(self.q, self.k, self.v, None if self.contig else self.page_table, self.seq_lens,
+                                   self.out, w.scale, num_splits, self.ws)
         self.bytes = w.algorithmic_bytes()
 
     def _views(self, buf):
@@ -424,7 +427,7 @@ def run_reference(a):
 def config_of(w, a):
     return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "page_size": w.page_size, "kv_tokens": w.kv_tokens(),
-            "num_splits": a.num_splits, "layout": w.layout,
+            "num_splits": a.num_splits, "layout": w.layout, "kv_policy": w.meta.get("kv_policy", "paged"),
             "l2": "two independent instances used in turn (each call reads KV the previous call did not touch); "
                   "large workloads are each larger than L2",
             "algorithmic_bytes_per_call": w.algorithmic_bytes(),

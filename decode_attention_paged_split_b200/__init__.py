@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "APDError",
     "attn_paged_decode",
+    "attn_contig_decode",
     "DecodeCall",
     "attn_paged_decode_noalloc",
     "NOALLOC_SCRATCH_BYTES",
@@ -120,6 +121,11 @@ def _load():
                                         ctypes.c_size_t, ctypes.c_void_p]
     L.apd_attn_paged_decode.restype = ctypes.c_int
     L.apd_attn_paged_decode_ex.argtypes = L.apd_attn_paged_decode.argtypes + [ctypes.POINTER(_Options)]
+    L.apd_attn_contig_decode.argtypes = [T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_size_t, ctypes.c_void_p]
+    L.apd_attn_contig_decode.restype = ctypes.c_int
+    L.apd_attn_contig_decode_ex.argtypes = L.apd_attn_contig_decode.argtypes + [ctypes.POINTER(_Options)]
+    L.apd_attn_contig_decode_ex.restype = ctypes.c_int
     L.apd_attn_paged_decode_ex.restype = ctypes.c_int
     L.apd_attn_paged_decode_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
     L.apd_attn_paged_decode_noalloc.restype = ctypes.c_int
@@ -241,11 +247,30 @@ def attn_paged_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
     return out
 
 
+def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
+                       out: torch.Tensor, scale: float, num_splits: int = 0, workspace: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Decode attention over a contiguous KV cache: k / v bf16 [B, Lmax, Hkv, D] ("blhd"
+    order; "bhld" storage is passed as the permuted view), token t of sequence b at
+    k[b, t].  Same arguments and results as attn_paged_decode otherwise."""
+    L = _load()
+    if workspace is None:
+        workspace = alloc_workspace(q.shape[0], q.shape[1], k.shape[2], q.shape[2], num_splits, device=q.device)
+    descs = [_desc(t) for t in (q, k, v, seq_lens, out)]
+    rc = L.apd_attn_contig_decode(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale), int(num_splits),
+                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                  _stream_handle(stream, q.device))
+    if rc:
+        raise APDError(rc, "apd_attn_contig_decode")
+    return out
+
+
 class DecodeCall:
     """apd_attn_paged_decode with its arguments marshalled once, for repeated calls on
     the same buffers (a decode loop, a benchmark, a CUDA-graph capture).  Calling the
     object enqueues one decode call; the tensors' contents may change between calls,
-    their storage, shapes and strides may not."""
+    their storage, shapes and strides may not.  page_table=None selects the
+    contiguous-KV call (apd_attn_contig_decode)."""
 
     def __init__(self, q, k_cache, v_cache, page_table, seq_lens, out, scale: float, num_splits: int = 0,
                  workspace: torch.Tensor | None = None):
@@ -254,7 +279,9 @@ class DecodeCall:
                                         device=q.device)
         self.tensors = (q, k_cache, v_cache, page_table, seq_lens, out, workspace)
         self.device = q.device
-        self._descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+        self.contig = page_table is None
+        args = (q, k_cache, v_cache, seq_lens, out) if self.contig else (q, k_cache, v_cache, page_table, seq_lens, out)
+        self._descs = [_desc(t) for t in args]
         self._head = tuple(ctypes.byref(d) for d in self._descs) + (
             ctypes.c_float(scale), int(num_splits), workspace.data_ptr(), workspace.numel() * workspace.element_size())
         self._opts = _Options()
@@ -272,12 +299,14 @@ class DecodeCall:
     def __call__(self, stream=None, split_done_event=None) -> None:
         st = _stream_handle(stream, self.device)
         if split_done_event is None:
-            rc = self._lib.apd_attn_paged_decode(*self._head, st)
+            fn = self._lib.apd_attn_contig_decode if self.contig else self._lib.apd_attn_paged_decode
+            rc = fn(*self._head, st)
         else:
             if not split_done_event.cuda_event:  # torch creates its events lazily, at the first record
                 split_done_event.record(torch.cuda.current_stream(self.device) if stream is None else stream)
             self._opts.split_done_event = split_done_event.cuda_event
-            rc = self._lib.apd_attn_paged_decode_ex(*self._head, st, self._opts_ref)
+            fn = self._lib.apd_attn_contig_decode_ex if self.contig else self._lib.apd_attn_paged_decode_ex
+            rc = fn(*self._head, st, self._opts_ref)
         if rc:
             raise APDError(rc, "apd_attn_paged_decode")
 

@@ -215,46 +215,60 @@ struct Validated {
     int64_t qst[3], kst[4], vst[4], ost[3], pst[2];
 };
 
+// Checks the call's descriptors.  pt == nullptr selects the contiguous-KV form:
+// k/v are [B, Lmax, Hkv, D] (one "page" of Lmax tokens per sequence, page b for
+// sequence b), and Lmax need not be a multiple of 32.
 int validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* pt,
              const apd_tensor* sl, const apd_tensor* out, int num_splits, Validated* V) {
-    if (!q || !k || !v || !pt || !sl || !out || is_null(k) || is_null(v)) return APD_ERR_NULL_POINTER;
+    const bool contig = (pt == nullptr);
+    if (!q || !k || !v || !sl || !out) return APD_ERR_NULL_POINTER;
+    const bool empty_batch = (q->ndim >= 1 && q->shape[0] == 0);
+    if ((is_null(k) || is_null(v)) && !(contig && empty_batch)) return APD_ERR_NULL_POINTER;
     // The per-sequence tensors may be empty (and NULL) only when the batch is empty.
-    if ((is_null(q) || is_null(pt) || is_null(sl) || is_null(out)) && !(q->ndim >= 1 && q->shape[0] == 0))
+    if ((is_null(q) || (!contig && is_null(pt)) || is_null(sl) || is_null(out)) && !empty_batch)
         return APD_ERR_NULL_POINTER;
     if (q->dtype != APD_DTYPE_BF16 || k->dtype != APD_DTYPE_BF16 || v->dtype != APD_DTYPE_BF16 ||
-        out->dtype != APD_DTYPE_BF16 || pt->dtype != APD_DTYPE_INT32 || sl->dtype != APD_DTYPE_INT32)
+        out->dtype != APD_DTYPE_BF16 || (!contig && pt->dtype != APD_DTYPE_INT32) || sl->dtype != APD_DTYPE_INT32)
         return APD_ERR_DTYPE;
-    if (q->ndim != 3 || out->ndim != 3 || k->ndim != 4 || v->ndim != 4 || pt->ndim != 2 || sl->ndim != 1)
+    if (q->ndim != 3 || out->ndim != 3 || k->ndim != 4 || v->ndim != 4 || (!contig && pt->ndim != 2) ||
+        sl->ndim != 1)
         return APD_ERR_SHAPE;
-    for (int i = 0; i < 4; ++i)
-        if (k->shape[i] != v->shape[i] || k->shape[i] <= 0) return APD_ERR_SHAPE;
     for (int i = 0; i < 3; ++i)
         if (q->shape[i] != out->shape[i] || q->shape[i] < 0) return APD_ERR_SHAPE;
     const int64_t B = q->shape[0], Hq = q->shape[1], D = q->shape[2];
+    for (int i = 0; i < 4; ++i)
+        if (k->shape[i] != v->shape[i] || (k->shape[i] <= 0 && !(contig && i == 0 && B == 0))) return APD_ERR_SHAPE;
     const int64_t NP = k->shape[0], P = k->shape[1], Hkv = k->shape[2];
-    if (k->shape[3] != D || pt->shape[0] != B || sl->shape[0] != B || pt->shape[1] <= 0) return APD_ERR_SHAPE;
+    const int64_t MP = contig ? 1 : pt->shape[1];
+    if (k->shape[3] != D || sl->shape[0] != B) return APD_ERR_SHAPE;
+    if (contig ? (NP != B) : (pt->shape[0] != B || MP <= 0)) return APD_ERR_SHAPE;
     if (Hq <= 0 || D <= 0) return APD_ERR_SHAPE;
-    if (Hq > INT32_MAX || Hkv > INT32_MAX || NP > INT32_MAX || P > INT32_MAX || pt->shape[1] > INT32_MAX)
+    if (Hq > INT32_MAX || Hkv > INT32_MAX || NP > INT32_MAX || P > INT32_MAX || MP > INT32_MAX)
         return APD_ERR_TOO_LARGE;
     if (B > APD_MAX_BATCH) return APD_ERR_TOO_LARGE;
     int rc = make_shape(static_cast<int>(B), static_cast<int>(Hq), static_cast<int>(Hkv), static_cast<int>(D), &V->s);
     if (rc) return rc;
-    if (P % apd::kTile != 0) return APD_ERR_PAGE_SIZE;
+    // A 32-token tile must not straddle two pages (one page-table lookup per tile).
+    if (!contig && P % apd::kTile != 0) return APD_ERR_PAGE_SIZE;
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
     if (!aligned_bf16_layout(q, V->qst) || !aligned_bf16_layout(out, V->ost) || !aligned_bf16_layout(k, V->kst) ||
         !aligned_bf16_layout(v, V->vst))
         return APD_ERR_LAYOUT;
-    normalized_strides(pt, V->pst);
-    if (V->pst[0] < 0 || V->pst[1] < 0 || (reinterpret_cast<uintptr_t>(pt->data) & 3u)) return APD_ERR_LAYOUT;
+    if (contig) {
+        V->pst[0] = V->pst[1] = 0;
+    } else {
+        normalized_strides(pt, V->pst);
+        if (V->pst[0] < 0 || V->pst[1] < 0 || (reinterpret_cast<uintptr_t>(pt->data) & 3u)) return APD_ERR_LAYOUT;
+    }
     int64_t sst[1];
     normalized_strides(sl, sst);
     if (sst[0] != 1 || (reinterpret_cast<uintptr_t>(sl->data) & 3u)) return APD_ERR_LAYOUT;
     // flattened tile indices must fit in int32 on the device
-    const int64_t tiles_bound = V->s.units * pt->shape[1] * (P / apd::kTile);
+    const int64_t tiles_bound = V->s.units * MP * ((P + apd::kTile - 1) / apd::kTile);
     if (tiles_bound >= INT32_MAX / 2) return APD_ERR_TOO_LARGE;
     V->P = static_cast<int>(P);
     V->NP = static_cast<int>(NP);
-    V->MP = static_cast<int>(pt->shape[1]);
+    V->MP = static_cast<int>(MP);
     return APD_OK;
 }
 
@@ -346,7 +360,7 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     const Shape& s = V.s;
     char* ws = static_cast<char*>(workspace);
     apd::SplitParams sp;
-    sp.page_table = static_cast<const int32_t*>(pt->data);
+    sp.page_table = pt ? static_cast<const int32_t*>(pt->data) : nullptr;
     sp.pt_s0 = V.pst[0];
     sp.pt_s1 = V.pst[1];
     sp.seq_lens = static_cast<const int32_t*>(sl->data);
@@ -481,10 +495,16 @@ int apd_workspace_init(void* workspace, size_t workspace_bytes, apd_stream_t str
     return APD_OK;
 }
 
-int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
-                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
-                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
-                             apd_stream_t stream, const apd_launch_options* options) {
+}  // extern "C"
+
+namespace {
+
+// The decode call behind every workspace entry point; page_table == nullptr is the
+// contiguous-KV form (see validate).
+int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out, float scale,
+                int num_splits, void* workspace, size_t workspace_bytes, apd_stream_t stream,
+                const apd_launch_options* options) {
     if (options && options->reserved != 0) return APD_ERR_ARGUMENT;
     Validated V;
     int rc = validate(q, k_cache, v_cache, page_table, seq_lens, out, num_splits, &V);
@@ -493,7 +513,7 @@ int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, con
     if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return APD_ERR_WORKSPACE;
     if (V.s.B == 0) return APD_OK;
     Plan pl;
-    const int64_t tiles_bound = V.s.units * V.MP * (V.P / apd::kTile);
+    const int64_t tiles_bound = V.s.units * V.MP * ((V.P + apd::kTile - 1) / apd::kTile);
     // A fixed split count does not depend on the device: check its workspace
     // before any CUDA call.
     if (num_splits > 0) {
@@ -515,6 +535,19 @@ int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, con
     }
 }
 
+}  // namespace
+
+extern "C" {
+
+int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                             apd_stream_t stream, const apd_launch_options* options) {
+    if (!page_table) return APD_ERR_NULL_POINTER;
+    return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, scale, num_splits, workspace, workspace_bytes,
+                       stream, options);
+}
+
 int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
                           const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
                           float scale, int num_splits, void* workspace, size_t workspace_bytes,
@@ -523,16 +556,32 @@ int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const 
                                     workspace_bytes, stream, nullptr);
 }
 
+int apd_attn_contig_decode_ex(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                              const apd_tensor* seq_lens, const apd_tensor* out, float scale, int num_splits,
+                              void* workspace, size_t workspace_bytes, apd_stream_t stream,
+                              const apd_launch_options* options) {
+    return decode_impl(q, k, v, nullptr, seq_lens, out, scale, num_splits, workspace, workspace_bytes, stream,
+                       options);
+}
+
+int apd_attn_contig_decode(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* seq_lens,
+                           const apd_tensor* out, float scale, int num_splits, void* workspace,
+                           size_t workspace_bytes, apd_stream_t stream) {
+    return decode_impl(q, k, v, nullptr, seq_lens, out, scale, num_splits, workspace, workspace_bytes, stream,
+                       nullptr);
+}
+
 int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
                                   const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
                                   float scale, int num_splits, apd_stream_t stream) {
+    if (!page_table) return APD_ERR_NULL_POINTER;
     Validated V;
     int rc = validate(q, k_cache, v_cache, page_table, seq_lens, out, num_splits, &V);
     if (rc) return rc;
     if (V.s.B == 0) return APD_OK;
     constexpr size_t kScratch = APD_NOALLOC_SCRATCH_BYTES;
     Plan pl;
-    const int64_t tiles_bound = V.s.units * V.MP * (V.P / apd::kTile);
+    const int64_t tiles_bound = V.s.units * V.MP * ((V.P + apd::kTile - 1) / apd::kTile);
     if (num_splits > 0) {
         rc = make_plan(V.s, num_splits, kDefaultSmCount, kScratch, tiles_bound, &pl);
         if (rc == APD_ERR_WORKSPACE) return APD_ERR_SCRATCH_LIMIT;

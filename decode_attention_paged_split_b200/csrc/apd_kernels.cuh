@@ -51,7 +51,7 @@ constexpr uint32_t kFlagTimeout = 0x8u;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per async-copy wait
 
 struct SplitParams {
-    const int32_t* page_table;
+    const int32_t* page_table;  // NULL: contiguous KV, sequence b is page b
     int64_t pt_s0, pt_s1;
     const int32_t* seq_lens;
     __nv_bfloat16* out;
@@ -150,6 +150,7 @@ __device__ __forceinline__ int32_t fetch_page(const SplitParams& p, const int32_
     if (i >= end) return 0;
     int b, ul, j, n;
     decode_tile(i, units_per_seq, cum, p.B, b, ul, j, n);
+    if (p.page_table == nullptr) return b;  // contiguous KV: sequence b is "page" b of Lmax tokens
     const int pj = (j * kTile) / p.P;
     return __ldcg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 + static_cast<int64_t>(pj) * p.pt_s1);
 }

@@ -194,6 +194,35 @@ int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, con
                              apd_stream_t stream, const apd_launch_options* options);
 
 /*
+ * apd_attn_contig_decode -- the same decode attention over a contiguous (not
+ * paged) KV cache: the ContigKV addressing policy next to PagedKV in the AstrAI
+ * commit log of csrc/kernels/attn_paged_decode.cu (attn_kv_source.cuh with
+ * ContigKV/PagedKV, kernels templated on the KV policy, stride-based addressing
+ * for the "bhld" / "blhd" layouts).
+ *
+ *   k, v       bf16 [B, Lmax, Hkv, D] in logical "blhd" order, D contiguous, other
+ *              strides multiples of 8 elements: "bhld" storage [B, Hkv, Lmax, D] is
+ *              passed as the permuted view.  Lmax is any positive length (not
+ *              necessarily a multiple of 32).  Token t of sequence b is
+ *              k[b, t, kvh, :].
+ *   q, seq_lens, out, scale, num_splits, workspace, stream: as in
+ *              apd_attn_paged_decode (same workspace size).  Device contract:
+ *              0 <= seq_lens[b] <= Lmax (larger values are clamped and flagged).
+ *
+ * It runs the paged kernels with one Lmax-token page per sequence (page b), so a
+ * paged and a contiguous cache holding the same tokens give identical results.
+ */
+int apd_attn_contig_decode(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* seq_lens,
+                           const apd_tensor* out, float scale, int num_splits, void* workspace,
+                           size_t workspace_bytes, apd_stream_t stream);
+
+/* apd_attn_contig_decode with launch options (see apd_attn_paged_decode_ex). */
+int apd_attn_contig_decode_ex(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                              const apd_tensor* seq_lens, const apd_tensor* out, float scale, int num_splits,
+                              void* workspace, size_t workspace_bytes, apd_stream_t stream,
+                              const apd_launch_options* options);
+
+/*
  * apd_attn_paged_decode_noalloc -- the same decode call for callers that cannot
  * allocate device memory.  The pages have no counterpart of this entry point.
  *

@@ -18,13 +18,15 @@ class DeviceProblem:
     def __init__(self, w, device="cuda"):
         self.w = w
         self.q = w.q.to(device)
-        # keep the storage order (NHD or HND) of the host cache
-        ks = w.k_cache.permute(0, 2, 1, 3) if w.layout == "HND" else w.k_cache
-        vs = w.v_cache.permute(0, 2, 1, 3) if w.layout == "HND" else w.v_cache
+        # keep the storage order (NHD/blhd, or HND/bhld) of the host cache
+        heads_outer = w.layout in ("HND", "bhld")
+        ks = w.k_cache.permute(0, 2, 1, 3) if heads_outer else w.k_cache
+        vs = w.v_cache.permute(0, 2, 1, 3) if heads_outer else w.v_cache
         ks = ks.contiguous().to(device)
         vs = vs.contiguous().to(device)
-        self.k = ks.permute(0, 2, 1, 3) if w.layout == "HND" else ks
-        self.v = vs.permute(0, 2, 1, 3) if w.layout == "HND" else vs
+        self.k = ks.permute(0, 2, 1, 3) if heads_outer else ks
+        self.v = vs.permute(0, 2, 1, 3) if heads_outer else vs
+        self.contig = w.meta.get("kv_policy") == "contig"
         self.page_table = w.page_table.to(device)
         self.seq_lens = w.seq_lens.to(device)
         self.out = torch.full_like(self.q, float("nan"))
@@ -35,8 +37,12 @@ class DeviceProblem:
         if workspace is None:
             workspace = apd.alloc_workspace(self.q.shape[0], self.q.shape[1], self.k.shape[2], self.q.shape[2], s)
         self.workspace = workspace
-        apd.attn_paged_decode(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, self.w.scale, s,
-                              workspace, stream=stream)
+        if self.contig:
+            apd.attn_contig_decode(self.q, self.k, self.v, self.seq_lens, self.out, self.w.scale, s, workspace,
+                                   stream=stream)
+        else:
+            apd.attn_paged_decode(self.q, self.k, self.v, self.page_table, self.seq_lens, self.out, self.w.scale, s,
+                                  workspace, stream=stream)
         return self.out
 
 

@@ -27,6 +27,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("apd_attn_paged_decode", "apd_workspace_size", "apd_status_string", "apd_attn_paged_decode_ex",
+                 "apd_attn_contig_decode",
                  "apd_query_plan", "apd_workspace_init", "apd_read_device_flags", "apd_last_cuda_error"):
         assert must in names
 
@@ -263,3 +264,44 @@ def test_empty_batch_accepts_null_batch_tensors():
     p = problem(B=0)
     p["k"].data = None
     assert call(p) == NULLP
+
+
+# ---------------------------------------------------------------- contiguous KV
+def contig_call(p, splits=0, ws=FAKE, ws_bytes=1 << 30):
+    return apd.lib().apd_attn_contig_decode(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]),
+                                            ctypes.byref(p["sl"]), ctypes.byref(p["out"]), ctypes.c_float(0.1),
+                                            splits, ws, ws_bytes, None)
+
+
+def contig_problem(B=2, Hq=8, Hkv=2, D=64, Lmax=1000):
+    return dict(q=T([B, Hq, D]), k=T([B, Lmax, Hkv, D]), v=T([B, Lmax, Hkv, D]), sl=T([B], apd.DTYPE_INT32),
+                out=T([B, Hq, D]))
+
+
+def test_contig_validation():
+    # any Lmax is accepted (the call then needs a device, which this host does not have)
+    assert contig_call(contig_problem(Lmax=1000)) in (OK, CUDA)
+    assert contig_call(contig_problem(Lmax=7)) in (OK, CUDA)
+    p = contig_problem()
+    p["k"] = T([3, 1000, 2, 64])  # one KV row per sequence: leading extent must be B
+    p["v"] = T([3, 1000, 2, 64])
+    assert contig_call(p) == SHAPE
+    assert contig_call(contig_problem(Hq=6, Hkv=4)) == GQA
+    assert contig_call(contig_problem(D=96)) == HEADDIM
+    assert contig_call(contig_problem(), splits=4, ws_bytes=1024) == WS
+    p = contig_problem()
+    p["k"].data = None
+    assert contig_call(p) == NULLP
+    assert contig_call(contig_problem(B=0)) == OK
+
+
+def test_paged_entry_still_rejects_a_null_page_table_descriptor():
+    p = problem()
+    L = apd.lib()
+    rc = L.apd_attn_paged_decode(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]), None,
+                                 ctypes.byref(p["sl"]), ctypes.byref(p["out"]), ctypes.c_float(1.0), 0, FAKE, 1 << 30,
+                                 None)
+    assert rc == NULLP
+    rc = L.apd_attn_paged_decode_noalloc(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]), None,
+                                         ctypes.byref(p["sl"]), ctypes.byref(p["out"]), ctypes.c_float(1.0), 0, None)
+    assert rc == NULLP

@@ -264,6 +264,84 @@ def make(
     )
 
 
+def make_contig(
+    *,
+    name: str,
+    seed: int,
+    batch: int,
+    num_q_heads: int,
+    num_kv_heads: int,
+    head_dim: int,
+    seq_lens,
+    lmax: int | None = None,
+    layout: str = "blhd",
+    scale: float | None = None,
+    value_seed: int | None = None,
+    poison: bool = True,
+    k_outlier_frac: float = 0.0,
+) -> Workload:
+    """A contiguous KV cache: k / v bf16 [B, Lmax, Hkv, D] ("blhd"), or "bhld" storage
+    [B, Hkv, Lmax, D] returned as the [B, Lmax, Hkv, D]-ordered view.  Slots at or past a
+    sequence's length hold NaN when ``poison`` (they must never be read).  The returned
+    Workload describes the same cache as a paged one with one Lmax-token page per
+    sequence (page_table[b] = [b]), which is how the oracle reads it."""
+    lens = np.asarray(seq_lens, dtype=np.int64).reshape(-1)
+    assert lens.shape[0] == batch and (lens >= 0).all()
+    lmax = int(lmax if lmax is not None else max(1, int(lens.max(initial=0))))
+    assert lmax >= int(lens.max(initial=0))
+    vseed = seed if value_seed is None else value_seed
+    q = seeded_randn_bf16(batch * num_q_heads * head_dim, vseed, _S_Q).view(batch, num_q_heads, head_dim)
+    numel = batch * lmax * num_kv_heads * head_dim
+    if layout == "blhd":
+        shape_store, to_blhd = (batch, lmax, num_kv_heads, head_dim), (0, 1, 2, 3)
+    elif layout == "bhld":
+        shape_store, to_blhd = (batch, num_kv_heads, lmax, head_dim), (0, 2, 1, 3)
+    else:
+        raise ValueError(f"unknown layout {layout!r}")
+    k = seeded_randn_bf16(numel, vseed, _S_K).view(*shape_store).permute(*to_blhd)
+    v = seeded_randn_bf16(numel, vseed, _S_V).view(*shape_store).permute(*to_blhd)
+    if k_outlier_frac > 0.0:
+        mask = seeded_bernoulli(numel, k_outlier_frac, vseed, _S_KMASK).view(*shape_store).permute(*to_blhd)
+        k[mask] = k[mask] * 8.0
+    if poison:
+        for b in range(batch):
+            k[b, int(lens[b]):] = float("nan")
+            v[b, int(lens[b]):] = float("nan")
+    if scale is None:
+        scale = 1.0 / math.sqrt(head_dim)
+    return Workload(name=name, seed=seed, q=q, k_cache=k, v_cache=v,
+                    page_table=torch.arange(batch, dtype=torch.int32).view(batch, 1),
+                    seq_lens=torch.from_numpy(lens.astype(np.int32)), scale=float(scale), layout=layout,
+                    meta={"kv_policy": "contig", "lmax": lmax})
+
+
+def paged_from_contig(w: Workload, page_size: int = 32, seed: int = 0, poison: bool = True) -> Workload:
+    """The same tokens as a contiguous workload, placed page by page into a shuffled pool
+    of ``page_size``-token pages (the pages' paged-versus-contiguous agreement case)."""
+    B, Hkv, D = w.batch, w.num_kv_heads, w.head_dim
+    lens = w.seq_lens.to(torch.int64).tolist()
+    P = page_size
+    npages = [(L + P - 1) // P for L in lens]
+    pool = sum(npages)
+    mp = max(1, max(npages, default=1))
+    perm = np.random.default_rng([seed, 5]).permutation(max(pool, 1))
+    fill = float("nan") if poison else 0.0
+    k = torch.full((max(pool, 1), P, Hkv, D), fill, dtype=torch.bfloat16)
+    v = torch.full((max(pool, 1), P, Hkv, D), fill, dtype=torch.bfloat16)
+    pt = torch.zeros(B, mp, dtype=torch.int32)
+    cursor = 0
+    for b in range(B):
+        for j in range(npages[b]):
+            page = int(perm[cursor])
+            cursor += 1
+            pt[b, j] = page
+            t0, t1 = j * P, min((j + 1) * P, lens[b])
+            k[page, : t1 - t0] = w.k_cache[b, t0:t1]
+            v[page, : t1 - t0] = w.v_cache[b, t0:t1]
+    return Workload(name=w.name + "_paged", seed=w.seed, q=w.q, k_cache=k, v_cache=v, page_table=pt,
+                    seq_lens=w.seq_lens, scale=w.scale, meta={"kv_policy": "paged"})
+
+
 # ----------------------------------------------------------------------------
 # The named decode workloads
 # ----------------------------------------------------------------------------
@@ -340,9 +418,27 @@ def ragged(seed: int = 4262, **kw) -> Workload:
     return make(**args)
 
 
+def llama8b_contig(seed: int = 8, **kw) -> Workload:
+    """The llama8b-shaped decode over a contiguous [16, 4096, 8, 128] KV cache."""
+    args = dict(name="llama8b_contig_b16_h32x8_d128_l4096", seed=seed, batch=16, num_q_heads=32, num_kv_heads=8,
+                head_dim=128, seq_lens=[4096] * 16, lmax=4096, k_outlier_frac=0.01, poison=False)
+    args.update(kw)
+    return make_contig(**args)
+
+
+def long_contig(seed: int = 131072, **kw) -> Workload:
+    """The long-context decode over a contiguous [2, 131072, 8, 128] KV cache."""
+    args = dict(name="long_contig_b2_h32x8_d128_l131072", seed=seed, batch=2, num_q_heads=32, num_kv_heads=8,
+                head_dim=128, seq_lens=[131072] * 2, lmax=131072, poison=False)
+    args.update(kw)
+    return make_contig(**args)
+
+
 NAMED = {
     "tiny": tiny,
     "llama8b": llama8b,
     "long": long_context,
     "ragged": ragged,
+    "llama8b_contig": llama8b_contig,
+    "long_contig": long_contig,
 }
