@@ -64,6 +64,7 @@ struct SplitParams {
     int32_t mode;       // 0 balanced, 1 fixed
     int32_t ksplit;     // fixed mode: k
     int32_t num_workers;
+    int32_t groups;     // balanced mode: worker groups (num_workers = groups * Hkv * HB)
     int32_t warps;      // warps per CTA
     uint32_t stage_bytes, q_box_bytes;
     float scale_log2;
@@ -76,7 +77,7 @@ struct CombineParams {
     __nv_bfloat16* out;
     int64_t out_sb, out_sh;
     int32_t B, Hkv, g, HB, rows_max;
-    int32_t mode, ksplit, num_workers;
+    int32_t mode, ksplit, num_workers, groups;
 };
 
 template <int D>
@@ -109,6 +110,17 @@ struct Geometry {
     }
 };
 
+// Equal shares of [0, total) among `parts`: part w owns [run_start(w), run_start(w + 1)).
+__device__ __forceinline__ int64_t run_start(int w, int64_t total, int parts) {
+    return static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / parts);
+}
+
+// The part whose share contains position i.
+__device__ __forceinline__ int worker_of(int64_t i, int64_t total, int parts) {
+    return static_cast<int>((static_cast<uint64_t>(i + 1) * static_cast<uint64_t>(parts) - 1) /
+                            static_cast<uint64_t>(total));
+}
+
 // Largest b in [0, B) with cum[b] <= x (cum non-decreasing, cum[0] = 0).
 __device__ __forceinline__ int find_seq(const int32_t* cum, int B, int x) {
     int lo = 0, hi = B - 1;
@@ -120,36 +132,30 @@ __device__ __forceinline__ int find_seq(const int32_t* cum, int B, int x) {
     return lo;
 }
 
-// Flattened tile index -> (sequence b, unit-in-sequence ul, tile j, tiles n).
-__device__ __forceinline__ void decode_tile(int64_t i, int units_per_seq, const int32_t* cum, int B, int& b,
-                                            int& ul, int& j, int& n) {
-    b = find_seq(cum, B, static_cast<int>(i / units_per_seq));
+// Position s of the sequence-tile space (s = cum[b] + j, all sequences' tiles in
+// sequence order) -> (sequence b, tile j, tiles of that sequence n).
+__device__ __forceinline__ void decode_pos(int s, const int32_t* cum, int B, int& b, int& j, int& n) {
+    b = find_seq(cum, B, s);
     n = cum[b + 1] - cum[b];
-    const int rem = static_cast<int>(i - static_cast<int64_t>(units_per_seq) * cum[b]);
-    ul = rem / n;
-    j = rem - ul * n;
+    j = s - cum[b];
 }
 
-// Step a cursor to the next tile; only called when that tile exists.
-__device__ __forceinline__ void advance_tile(int units_per_seq, const int32_t* cum, int& b, int& ul, int& j,
-                                             int& n) {
+// Step a cursor to the next position; only called when that position exists.
+__device__ __forceinline__ void advance_pos(const int32_t* cum, int& b, int& j, int& n) {
     if (++j == n) {
         j = 0;
-        if (++ul == units_per_seq) {
-            ul = 0;
-            do {
-                ++b;
-                n = cum[b + 1] - cum[b];
-            } while (n == 0);
-        }
+        do {
+            ++b;
+            n = cum[b + 1] - cum[b];
+        } while (n == 0);
     }
 }
 
-__device__ __forceinline__ int32_t fetch_page(const SplitParams& p, const int32_t* cum, int units_per_seq,
-                                              int64_t i, int64_t end) {
-    if (i >= end) return 0;
-    int b, ul, j, n;
-    decode_tile(i, units_per_seq, cum, p.B, b, ul, j, n);
+// Page of the tile at position s (0 past `end`).
+__device__ __forceinline__ int32_t fetch_page(const SplitParams& p, const int32_t* cum, int s, int end) {
+    if (s >= end) return 0;
+    int b, j, n;
+    decode_pos(s, cum, p.B, b, j, n);
     if (p.page_table == nullptr) return b;  // contiguous KV: sequence b is "page" b of Lmax tokens
     const int pj = (j * kTile) / p.P;
     return __ldcg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 + static_cast<int64_t>(pj) * p.pt_s1);
@@ -247,20 +253,27 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // No CTA-wide barrier after this point: warps are independent workers.
 
     const int units_per_seq = p.Hkv * p.HB;
-    const int64_t total = static_cast<int64_t>(units_per_seq) * s_cum[B];
     const int w = blockIdx.x * p.warps + warp;
     if (w >= p.num_workers) return;
 
-    int64_t ws, we;
+    // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-
+    // sequence ul (kv head and head block).
+    int ws, we, ul;
     int fixed_slot = -1;
     if (p.mode == 0) {
-        ws = static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / p.num_workers);
-        we = static_cast<int64_t>((static_cast<uint64_t>(w + 1) * static_cast<uint64_t>(total)) / p.num_workers);
+        // Workers form groups of units_per_seq warps, one per (kv head, head block);
+        // group grp owns an equal share of the positions of all sequences.  The warps
+        // of a group walk the same pages together, so the kv heads of a page are read
+        // at about the same time.
+        const int grp = w / units_per_seq;
+        ul = w - grp * units_per_seq;
+        ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
+        we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
     } else {
         const int u = w / p.ksplit;
         const int s = w - u * p.ksplit;
         const int b = u / units_per_seq;
-        const int ul = u - b * units_per_seq;
+        ul = u - b * units_per_seq;
         const int n = s_cum[b + 1] - s_cum[b];
         if (n == 0) {
             if (s == 0) {
@@ -274,9 +287,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         const int t0 = s * c;
         if (t0 >= n) return;
         const int t1 = min(t0 + c, n);
-        const int64_t Tu = static_cast<int64_t>(units_per_seq) * s_cum[b] + static_cast<int64_t>(ul) * n;
-        ws = Tu + t0;
-        we = Tu + t1;
+        ws = s_cum[b] + t0;
+        we = s_cum[b] + t1;
         fixed_slot = u * p.ksplit + s;
     }
     if (ws >= we) return;
@@ -293,26 +305,29 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     const uint64_t pol_stream = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
 
-    // ---- producer state: next tile to issue, its cursor, page-table window
-    int64_t pi = ws;
-    int pb, pul, pj, pn;
-    decode_tile(ws, units_per_seq, s_cum, B, pb, pul, pj, pn);
-    int64_t wbase = ws;
-    int32_t pg_cur = fetch_page(p, s_cum, units_per_seq, ws + lane, we);
-    int32_t pg_nxt = fetch_page(p, s_cum, units_per_seq, ws + 32 + lane, we);
+    const int kvh = ul / p.HB;
+    const int hb = ul - kvh * p.HB;
+    const int head0 = kvh * p.g + kMaxRows * hb;
+    const int rows = min(kMaxRows, p.g - kMaxRows * hb);
+
+    // ---- producer state: next position to issue, its cursor, page-table window
+    int pi = ws;
+    int pb, pj, pn;
+    decode_pos(ws, s_cum, B, pb, pj, pn);
+    int wbase = ws;
+    int32_t pg_cur = fetch_page(p, s_cum, ws + lane, we);
+    int32_t pg_nxt = fetch_page(p, s_cum, ws + 32 + lane, we);
 
     auto issue_next = [&](int stage) {
         if (pi >= we) return;
-        int off = static_cast<int>(pi - wbase);
+        int off = pi - wbase;
         if (off >= 32) {
             pg_cur = pg_nxt;
             wbase += 32;
             off -= 32;
-            pg_nxt = fetch_page(p, s_cum, units_per_seq, wbase + 32 + lane, we);
+            pg_nxt = fetch_page(p, s_cum, wbase + 32 + lane, we);
         }
         const int32_t page = __shfl_sync(0xffffffffu, pg_cur, off);
-        const int kvh = pul / p.HB;
-        const int hb = pul - kvh * p.HB;
         const int slot = (pj * kTile) % p.P;
         const bool qload = (pj == 0) || (pi == ws);
         if (lane == 0) {
@@ -323,17 +338,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             if constexpr (D == 32) {
                 tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, page, pol_stream);
                 tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, pol_stream);
-                if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, kvh * p.g + kMaxRows * hb, pb,
-                                       pol_keep);
+                if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, pb, pol_keep);
             } else {
                 tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, page, 0, pol_stream);
                 tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, 0, pol_stream);
-                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, kvh * p.g + kMaxRows * hb, pb, 0,
-                                       pol_keep);
+                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, pb, 0, pol_keep);
             }
         }
         ++pi;
-        if (pi < we) advance_tile(units_per_seq, s_cum, pb, pul, pj, pn);
+        if (pi < we) advance_pos(s_cum, pb, pj, pn);
     };
 
 #pragma unroll
@@ -342,32 +355,29 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // ---- consumer state
     const int tq = lane & 3;   // thread in quad: token / d pair
     const int gq = lane >> 2;  // quad index: row within the 8-row half
-    int cb, cul, cj, cn;
-    decode_tile(ws, units_per_seq, s_cum, B, cb, cul, cj, cn);
-    int64_t seg_start = ws;
+    int cb, cj, cn;
+    decode_pos(ws, s_cum, B, cb, cj, cn);
+    int seg_start = ws;
     int j_start = cj;
 
     uint32_t qf[G::kSteps][4];
     float acc[G::kNTiles][4];
     float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-    int rows = 0;
 
-    for (int64_t i = ws; i < we; ++i) {
-        const int k = static_cast<int>(i - ws);
+    for (int i = ws; i < we; ++i) {
+        const int k = i - ws;
         const int stage = k % STAGES;
         const uint32_t parity = static_cast<uint32_t>(k / STAGES) & 1u;
         const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
         const bool unit_start = (cj == 0) || (i == ws);
-        const int kvh = cul / p.HB;
-        const int hb = cul - kvh * p.HB;
 
         if (!mbar_wait_bounded(bar0 + 8 * stage, parity, kWaitTimeoutNs)) {
             if (lane == 0) atomicOr(p.flags, kFlagTimeout);
             // Give the other copies in flight a bounded chance to land, then stop.
             for (int s = 0; s < STAGES; ++s) {
-                const int64_t t = i + s;
+                const int t = i + s;
                 if (t < pi) {
-                    const int kk = static_cast<int>(t - ws);
+                    const int kk = t - ws;
                     mbar_wait_bounded(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u,
                                       kWaitTimeoutNs / 8);
                 }
@@ -378,7 +388,6 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         if (unit_start) {
             seg_start = i;
             j_start = cj;
-            rows = min(kMaxRows, p.g - kMaxRows * hb);
             m_lo = m_hi = -INFINITY;
             l_lo = l_hi = 0.f;
 #pragma unroll
@@ -512,7 +521,6 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             ll += __shfl_xor_sync(0xffffffffu, ll, 2);
             float lh = l_hi + __shfl_xor_sync(0xffffffffu, l_hi, 1);
             lh += __shfl_xor_sync(0xffffffffu, lh, 2);
-            const int head0 = kvh * p.g + kMaxRows * hb;
             const bool direct = (j_start == 0) && (cj == cn - 1);
             if (direct) {
                 const float il = 1.f / ll, ih = 1.f / lh;
@@ -545,18 +553,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
                 }
             }
         }
-        if (i + 1 < we) advance_tile(units_per_seq, s_cum, cb, cul, cj, cn);
+        if (i + 1 < we) advance_pos(s_cum, cb, cj, cn);
     }
-}
-
-// Balanced mode: the worker whose run contains flattened tile i.
-__device__ __forceinline__ int worker_of(int64_t i, int64_t total, int workers) {
-    return static_cast<int>((static_cast<uint64_t>(i + 1) * static_cast<uint64_t>(workers) - 1) /
-                            static_cast<uint64_t>(total));
-}
-
-__device__ __forceinline__ int64_t run_start(int w, int64_t total, int workers) {
-    return static_cast<int64_t>((static_cast<uint64_t>(w) * static_cast<uint64_t>(total)) / workers);
 }
 
 constexpr int kCombineWarps = 4;
@@ -601,16 +599,18 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __gri
         return;
     }
 
-    // The unit's partial slots, numbered k = 0 .. nk-1.
-    int nk, w_first = 0, first_slot_fixed = 0;
-    int64_t total = 0, Tu = 0;
+    // The unit's partial slots, numbered k = 0 .. nk-1.  Balanced mode: the groups
+    // whose shares of the sequence-tile positions meet sequence b; group g's warp
+    // for this unit is g * units_per_seq + ul.
+    int nk, g_first = 0, first_slot_fixed = 0;
+    int64_t total = 0, Sb = 0;
     if (p.mode == 0) {
-        total = static_cast<int64_t>(units_per_seq) * p.cum[p.B];
-        Tu = static_cast<int64_t>(units_per_seq) * p.cum[b] + static_cast<int64_t>(ul) * n;
-        w_first = worker_of(Tu, total, p.num_workers);
-        const int w_last = worker_of(Tu + n - 1, total, p.num_workers);
-        if (w_first == w_last) return;  // one worker covered it and wrote the output
-        nk = w_last - w_first + 1;
+        total = p.cum[p.B];
+        Sb = p.cum[b];
+        g_first = worker_of(Sb, total, p.groups);
+        const int g_last = worker_of(Sb + n - 1, total, p.groups);
+        if (g_first == g_last) return;  // one warp covered it and wrote the output
+        nk = g_last - g_first + 1;
     } else {
         const int S = min(p.ksplit, n);
         const int c = (n + S - 1) / S;
@@ -618,13 +618,14 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __gri
         if (nk == 1) return;
         first_slot_fixed = u * p.ksplit;
     }
-    // slot of partial k, or -1 for a worker whose run is empty (it wrote nothing)
+    // slot of partial k, or -1 for a group whose share is empty (it wrote nothing)
     auto slot_of = [&](int k) -> int64_t {
         if (p.mode != 0) return first_slot_fixed + k;
-        const int w = w_first + k;
-        const int64_t a = run_start(w, total, p.num_workers);
-        if (a == run_start(w + 1, total, p.num_workers)) return -1;
-        return 2 * static_cast<int64_t>(w) + ((k == 0 && a != Tu) ? 1 : 0);
+        const int g = g_first + k;
+        const int64_t a = run_start(g, total, p.groups);
+        if (a == run_start(g + 1, total, p.groups)) return -1;
+        const int64_t w = static_cast<int64_t>(g) * units_per_seq + ul;
+        return 2 * w + ((k == 0 && a != Sb) ? 1 : 0);
     };
 
     float M = -INFINITY, den = 0.f;

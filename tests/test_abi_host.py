@@ -205,9 +205,14 @@ def test_workspace_size_invalid_is_zero():
 def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
     g = Hq // Hkv
+    ups = Hkv * -(-g // 16)  # warps per group: one per (kv head, 16-row head block)
     assert pl.mode == 0
-    assert pl.grid_ctas == 148  # one persistent CTA per SM
-    assert pl.num_workers == 148 * pl.warps_per_cta
+    # as many whole groups as the warp budget holds (7/8 of the resident warps for
+    # D = 128, all of them otherwise): at most one CTA per SM
+    budget = 148 * pl.warps_per_cta * 7 // 8 if D == 128 else 148 * pl.warps_per_cta
+    assert pl.num_workers == (budget // ups) * ups
+    assert pl.grid_ctas == -(-pl.num_workers // pl.warps_per_cta) <= 148
+    assert budget - pl.num_workers < ups
     assert pl.partial_slots == 2 * pl.num_workers
     assert pl.rows_per_unit == min(g, 16) and pl.head_blocks == -(-g // 16)
     assert pl.combine_ctas == B * Hkv * pl.head_blocks * pl.rows_per_unit
