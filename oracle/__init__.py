@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for paged decode attention (ctypes front end of paged_decode_oracle.c).
+"""fp64 CPU oracles: paged decode attention (paged_decode_oracle.c) and the decode
+projection GEMV (gemv_oracle.c), through ctypes.
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
 baseline / reference leg of ``bench.py`` import this package.  The CUDA library
@@ -165,3 +166,31 @@ def max_threads() -> int:
 
 def num_host_cores() -> int:
     return os.cpu_count() or 1
+
+
+_gemv_lib = None
+
+
+def _gemv():
+    global _gemv_lib
+    if _gemv_lib is None:
+        L = ctypes.CDLL(_build.build_gemv())
+        dp = ctypes.POINTER(ctypes.c_double)
+        L.oracle_gemv.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int, dp, dp, ctypes.c_int]
+        _gemv_lib = L
+    return _gemv_lib
+
+
+def gemv(x: torch.Tensor, w: torch.Tensor, nthreads: int = 0):
+    """y = x W^T in fp64 for bf16 x [M, K] and W [N, K] (rows contiguous); returns
+    (y, absy), both float64 [M, N], absy[m, n] = sum_k |x[m, k] W[n, k]|."""
+    assert x.dtype == torch.bfloat16 and w.dtype == torch.bfloat16 and x.device.type == "cpu"
+    assert x.stride(1) == 1 and w.stride(1) == 1 and x.shape[1] == w.shape[1]
+    M, K = x.shape
+    N = w.shape[0]
+    y = np.zeros((M, N), dtype=np.float64)
+    a = np.zeros((M, N), dtype=np.float64)
+    _check(_gemv().oracle_gemv(x.data_ptr(), x.stride(0), w.data_ptr(), w.stride(0), M, N, K, _dptr(y), _dptr(a),
+                               nthreads), "gemv")
+    return y, a

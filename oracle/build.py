@@ -11,20 +11,32 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "paged_decode_oracle.c")
 LIB = os.path.join(HERE, "liboracle_paged_decode.so")
+GEMV_SRC = os.path.join(HERE, "gemv_oracle.c")
+GEMV_LIB = os.path.join(HERE, "liboracle_gemv.so")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
-        return LIB
+def _build_one(src: str, lib: str, force: bool, verbose: bool) -> str:
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= os.path.getmtime(src):
+        return lib
     # -O2 without -ffast-math: IEEE double arithmetic in program order.
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC",
-           "-shared", "-Wall", "-Wextra", "-o", tmp, SRC, "-lm"]
+           "-shared", "-Wall", "-Wextra", "-o", tmp, src, "-lm"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Build both oracle libraries; returns the decode-attention one."""
+    _build_one(GEMV_SRC, GEMV_LIB, force, verbose)
+    return _build_one(SRC, LIB, force, verbose)
+
+
+def build_gemv(force: bool = False, verbose: bool = False) -> str:
+    return _build_one(GEMV_SRC, GEMV_LIB, force, verbose)
 
 
 if __name__ == "__main__":

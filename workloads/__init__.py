@@ -442,3 +442,49 @@ NAMED = {
     "llama8b_contig": llama8b_contig,
     "long_contig": long_contig,
 }
+
+
+# ----------------------------------------------------------------------------
+# Decode projection (GEMV) inputs: x [M, K] and W [N, K] bf16, iid N(0, 1)
+# ----------------------------------------------------------------------------
+_S_GX, _S_GW = 11, 12
+
+# (N, K) of the projections of the AstrAI 1B decode benchmark (hidden 1536,
+# intermediate 6912, vocabulary 100000, kv width 256), named after their layers.
+GEMV_SHAPES = {
+    "q": (1536, 1536),
+    "kv": (256, 1536),
+    "gate_up": (6912, 1536),
+    "down": (1536, 6912),
+    "lm_head": (100000, 1536),
+}
+
+
+@dataclass
+class GemvCase:
+    name: str
+    seed: int
+    x: torch.Tensor  # bf16 [M, K]
+    w: torch.Tensor  # bf16 [N, K]
+
+    def algorithmic_bytes(self) -> int:
+        """Weight bytes + x bytes + y bytes (bf16)."""
+        M, K = self.x.shape
+        N = self.w.shape[0]
+        return 2 * (N * K + M * K + M * N)
+
+    def algorithmic_flops(self) -> int:
+        M, K = self.x.shape
+        return 2 * M * K * self.w.shape[0]
+
+
+def gemv_case(M: int, N: int, K: int, seed: int = 7, name: str | None = None, value_seed: int | None = None) -> GemvCase:
+    vs = seed if value_seed is None else value_seed
+    x = seeded_randn_bf16(M * K, vs, _S_GX).view(M, K)
+    w = seeded_randn_bf16(N * K, vs, _S_GW).view(N, K)
+    return GemvCase(name=name or f"gemv_m{M}_n{N}_k{K}", seed=seed, x=x, w=w)
+
+
+def gemv_named(layer: str, M: int, seed: int = 7, **kw) -> GemvCase:
+    N, K = GEMV_SHAPES[layer]
+    return gemv_case(M, N, K, seed=seed, name=f"gemv_{layer}_m{M}_n{N}_k{K}", **kw)
