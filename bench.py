@@ -42,6 +42,8 @@ UNIT = "GB/s"
 DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000, "llama8b_contig": 20000,
                  "long_contig": 5000}
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
+GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes per call / time)"
+GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
 
 
@@ -51,14 +53,15 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(workloads.NAMED), default="llama8b")
+    p.add_argument("--workload", choices=sorted(workloads.NAMED) + GEMV_WORKLOADS, default="llama8b",
+                   help="a decode-attention workload, or gemv_<layer>_m<M> for the decode projection")
     p.add_argument("--num-splits", type=int, default=0, help="0 = auto (the default launch configuration)")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     p.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks")
     a = p.parse_args(argv)
     if a.steps is None:
-        a.steps = DEFAULT_STEPS[a.workload]
+        a.steps = DEFAULT_STEPS.get(a.workload, 2000)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
     return a
@@ -536,10 +539,164 @@ def run_ours(a):
     return 0
 
 
+# ---------------------------------------------------------------- decode projection (GEMV)
+def gemv_spec(name: str):
+    layer, m = name[len("gemv_"):].rsplit("_m", 1)
+    return layer, int(m)
+
+
+def run_gemv(a):
+    """The decode projection y = x W^T on one GPU: CUDA-graph replays of the call,
+    rotating over enough weight copies that every call reads weights from HBM."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        print("no CUDA device", file=sys.stderr)
+        return 2
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_group(world, "nccl")
+    import decode_attention_paged_split_b200 as apd
+
+    layer, M = gemv_spec(a.workload)
+    N, K = workloads.GEMV_SHAPES[layer]
+    case = workloads.gemv_named(layer, M, value_seed=7 + 1000003 * rank)
+    copies = max(2, -(-400_000_000 // (N * K * 2)))
+    x = case.x.to(device)
+    ws = torch.zeros(apd.gemv_workspace_size(M, N, K), dtype=torch.uint8, device=device)
+    ys = [torch.empty(M, N, dtype=torch.bfloat16, device=device) for _ in range(copies)]
+    wdev = case.w.to(device)
+    weights = [wdev] + [wdev.clone() for _ in range(copies - 1)]
+    stream = torch.cuda.Stream(device)
+    per_call = case.algorithmic_bytes()
+
+    def call(i, st):
+        apd.gemv(x, weights[i % copies], ys[i % copies], ws, stream=st)
+
+    for i in range(a.warmup):
+        call(i, stream)
+    torch.cuda.synchronize(device)
+    plan = []
+    full, rest = divmod(a.steps, GRAPH_CHUNK)
+    for n, reps in ((GRAPH_CHUNK, full), (rest, 1 if rest else 0)):
+        if reps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n):
+                        call(i, stream)
+            plan.append((g, reps))
+
+    def replay():
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for g, reps in plan:
+                for _ in range(reps):
+                    g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    replay()
+    clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    el = replay()
+    barrier(dist, device)
+    clock_info = clocks.stop()
+    plan = []
+    t_max = max_over_ranks(el, dist, device)
+    bytes_all = sum_over_ranks(float(per_call * a.steps), dist, device)
+    value = bytes_all / t_max / 1e9
+
+    e2e = None
+    if not a.no_e2e:
+        # per step: x in (pinned host -> device), the call, y out (device -> pinned host); the copies run on
+        # two copy streams so they overlap the neighbouring steps' compute; buffers rotate over the copies
+        hx = case.x.pin_memory()
+        hys = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for _ in range(copies)]
+        xs = [x] + [x.clone() for _ in range(copies - 1)]
+        h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        computed = [torch.cuda.Event() for _ in range(copies)]
+        copied = [torch.cuda.Event() for _ in range(copies)]
+        ready = [torch.cuda.Event() for _ in range(copies)]
+        used = [False] * copies
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d_s.wait_stream(stream)
+        d2h_s.wait_stream(stream)
+        for i in range(a.steps):
+            j = i % copies
+            with torch.cuda.stream(h2d_s):
+                if used[j]:
+                    h2d_s.wait_event(computed[j])
+                xs[j].copy_(hx, non_blocking=True)
+                ready[j].record(h2d_s)
+            stream.wait_event(ready[j])
+            if used[j]:
+                stream.wait_event(copied[j])
+            apd.gemv(xs[j], weights[j], ys[j], ws, stream=stream)
+            computed[j].record(stream)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(computed[j])
+                hys[j].copy_(ys[j], non_blocking=True)
+                copied[j].record(d2h_s)
+            used[j] = True
+        stream.wait_stream(d2h_s)
+        stream.wait_stream(h2d_s)
+        e1.record(stream)
+        e1.synchronize()
+        e_max = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
+        e2e = {"value": bytes_all / e_max / 1e9, "unit": UNIT, "h2d_bytes_per_step": x.nbytes,
+               "d2h_bytes_per_step": ys[0].nbytes, "ms_per_step": e_max / a.steps * 1e3,
+               "how": "per step, eager through the public Python API: pinned-host->device copy of x, the call, "
+                      "device->pinned-host copy of y (weights resident); copies on two copy streams overlap the "
+                      "neighbouring steps' compute"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import oracle
+
+        oracle.gemv(case.x, case.w)
+        t0, calls = time.perf_counter(), 0
+        while time.perf_counter() - t0 < 10.0 and calls < 200:
+            oracle.gemv(case.x, case.w)
+            calls += 1
+        el_cpu = time.perf_counter() - t0
+        cpu = {"value": per_call * calls / el_cpu / 1e9, "unit": UNIT, "cores": oracle.max_threads(),
+               "kind": "oracle", "sample": f"the whole {case.name} product, {calls} calls, {el_cpu:.1f} s, fp64"}
+
+    if rank == 0:
+        peak, peak_src = peaks()
+        us = t_max / a.steps * 1e6
+        line = {
+            "metric": GEMV_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": us / 1e3, "us_per_call": us, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": case.name, "M": M, "N": N, "K": K, "algorithmic_bytes_per_call": per_call,
+                       "l2": f"{copies} weight copies used in turn ({copies * N * K * 2 / 1e6:.0f} MB > L2)",
+                       "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
+            "roofline": {"bound": "hbm", "achieved": per_call / (t_max / a.steps) / 1e9, "peak": peak, "unit": UNIT,
+                         "frac": per_call / (t_max / a.steps) / 1e9 / peak, "traffic": None, "peak_source": peak_src,
+                         "kernel": "gemv_kernel + gemv_sum_kernel (whole call)"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * a.steps, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     a = parse_args(argv)
     if a.impl == "reference":
+        if a.workload.startswith("gemv_"):
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the decode-attention "
+                                                                  "workloads; use the gemv workloads' cpu_baseline"}))
+            return 0
         return run_reference(a)
+    if a.workload.startswith("gemv_"):
+        return run_gemv(a)
     return run_ours(a)
 
 

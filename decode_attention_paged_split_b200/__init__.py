@@ -22,6 +22,8 @@ __all__ = [
     "APDError",
     "attn_paged_decode",
     "attn_contig_decode",
+    "gemv",
+    "gemv_workspace_size",
     "DecodeCall",
     "attn_paged_decode_noalloc",
     "NOALLOC_SCRATCH_BYTES",
@@ -129,6 +131,10 @@ def _load():
     L.apd_attn_paged_decode_ex.restype = ctypes.c_int
     L.apd_attn_paged_decode_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
     L.apd_attn_paged_decode_noalloc.restype = ctypes.c_int
+    L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
+    L.apd_gemv_workspace_size.restype = ctypes.c_size_t
+    L.apd_gemv_bf16.argtypes = [T, T, T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    L.apd_gemv_bf16.restype = ctypes.c_int
     L.apd_read_device_flags.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                         ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
     L.apd_read_device_flags.restype = ctypes.c_int
@@ -263,6 +269,29 @@ def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
     if rc:
         raise APDError(rc, "apd_attn_contig_decode")
     return out
+
+
+def gemv_workspace_size(m: int, n: int, k: int) -> int:
+    nb = _load().apd_gemv_workspace_size(m, n, k)
+    if nb == 0:
+        raise ValueError(f"invalid GEMV shape M={m}, N={n}, K={k}")
+    return int(nb)
+
+
+def gemv(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+         stream=None) -> torch.Tensor:
+    """Decode projection y = x W^T: x bf16 [M, K] (M <= 8), w bf16 [N, K] -> y bf16 [M, N]."""
+    if y is None:
+        y = torch.empty(x.shape[0], w.shape[0], dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(gemv_workspace_size(x.shape[0], w.shape[0], x.shape[1]), dtype=torch.uint8,
+                                device=x.device)
+    d = [_desc(t) for t in (x, w, y)]
+    rc = _load().apd_gemv_bf16(*[ctypes.byref(t) for t in d], workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream_handle(stream, x.device))
+    if rc:
+        raise APDError(rc, "apd_gemv_bf16")
+    return y
 
 
 class DecodeCall:

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "../../include/attn_paged_decode.h"
+#include "apd_gemv.cuh"
 #include "apd_kernels.cuh"
 
 namespace {
@@ -169,6 +170,7 @@ struct DeviceState {
     bool init = false;
     int sm_count = 0;
     bool smem_attr_set[4] = {false, false, false, false};
+    bool gemv_attr_set = false;
 };
 std::mutex g_mu;
 DeviceState g_devices[128];
@@ -461,6 +463,77 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     return APD_OK;
 }
 
+// ---------------------------------------------------------------- decode projection (GEMV)
+constexpr int kGemvWarps = 4;
+constexpr int kGemvStages = 4;
+
+size_t gemv_smem_bytes() { return 8ull * kGemvWarps * kGemvStages + 1024 + static_cast<size_t>(kGemvWarps) * kGemvStages * apd::kGemvStageBytes; }
+
+int64_t gemv_workers(int sm_count, int64_t units) {
+    int64_t w = static_cast<int64_t>(sm_count) * kGemvWarps;
+    return std::max<int64_t>(1, std::min(w, units));
+}
+
+// Workspace: [flags 256 B][fp32 partials, 2 per worker].
+size_t gemv_ws_bytes(int64_t workers) {
+    return kWsAlign + align_up(static_cast<size_t>(2 * workers) * apd::kGemvRows * apd::kGemvXRows * 4, kWsAlign);
+}
+
+// A bf16 row-major matrix [rows, K]: K contiguous, row stride a multiple of 8
+// elements, base 16-byte aligned (the TMA rules for the tiled loads).
+bool gemv_matrix_ok(const apd_tensor* t, int64_t* ld) {
+    int64_t st[2];
+    normalized_strides(t, st);
+    if (st[1] != 1 || st[0] <= 0 || st[0] % 8 != 0 || st[0] * 2 >= (1ll << 40)) return false;
+    if (reinterpret_cast<uintptr_t>(t->data) & 15u) return false;
+    *ld = st[0];
+    return true;
+}
+
+int encode_gemv_map(CUtensorMap* map, const apd_tensor* t, int64_t ld, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(t->shape[1]), static_cast<cuuint64_t>(t->shape[0])};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, t->data, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return driver_fail(r, "cuTensorMapEncodeTiled(gemv)");
+    return APD_OK;
+}
+
+struct GemvShape {
+    int M, N, K;
+    int64_t ldx, ldw, ysm, ysn, units, mtiles, ktiles;
+};
+
+int gemv_validate(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, GemvShape* g) {
+    if (!x || !w || !y) return APD_ERR_NULL_POINTER;
+    if (x->dtype != APD_DTYPE_BF16 || w->dtype != APD_DTYPE_BF16 || y->dtype != APD_DTYPE_BF16) return APD_ERR_DTYPE;
+    if (x->ndim != 2 || w->ndim != 2 || y->ndim != 2) return APD_ERR_SHAPE;
+    const int64_t M = x->shape[0], K = x->shape[1], N = w->shape[0];
+    if (w->shape[1] != K || y->shape[0] != M || y->shape[1] != N) return APD_ERR_SHAPE;
+    if (M < 1 || M > APD_GEMV_MAX_M || N < 1 || K < 1) return APD_ERR_SHAPE;
+    if (N > INT32_MAX / 2 || K > INT32_MAX / 2) return APD_ERR_TOO_LARGE;
+    if (is_null(x) || is_null(w) || is_null(y)) return APD_ERR_NULL_POINTER;
+    if (K % 8 != 0) return APD_ERR_LAYOUT;
+    if (!gemv_matrix_ok(x, &g->ldx) || !gemv_matrix_ok(w, &g->ldw)) return APD_ERR_LAYOUT;
+    int64_t yst[2];
+    normalized_strides(y, yst);
+    if (yst[0] < 0 || yst[1] < 0 || (reinterpret_cast<uintptr_t>(y->data) & 1u)) return APD_ERR_LAYOUT;
+    g->M = static_cast<int>(M);
+    g->N = static_cast<int>(N);
+    g->K = static_cast<int>(K);
+    g->ysm = yst[0];
+    g->ysn = yst[1];
+    g->mtiles = (N + apd::kGemvRows - 1) / apd::kGemvRows;
+    g->ktiles = (K + apd::kGemvCols - 1) / apd::kGemvCols;
+    g->units = g->mtiles * g->ktiles;
+    return APD_OK;
+}
+
 // ---------------------------------------------------------------- built-in scratch
 // Scratch of apd_attn_paged_decode_noalloc: a static device array, so that entry
 // point allocates nothing.  Host code must not use its name as an address (on the
@@ -509,8 +582,8 @@ size_t apd_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head
 int apd_workspace_init(void* workspace, size_t workspace_bytes, apd_stream_t stream) {
     if (!workspace) return APD_ERR_NULL_POINTER;
     if (workspace_bytes < kWsAlign || (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)) return APD_ERR_WORKSPACE;
-    cudaError_t e = cudaMemsetAsync(workspace, 0, kWsAlign, reinterpret_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace header)");
+    cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
     return APD_OK;
 }
 
@@ -623,6 +696,82 @@ int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache
         case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
         default: return APD_ERR_HEAD_DIM;
     }
+}
+
+size_t apd_gemv_workspace_size(int m, int n, int k) {
+    if (m < 1 || m > APD_GEMV_MAX_M || n < 1 || k < 1) return 0;
+    int sm_count = kDefaultSmCount;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int c = 0;
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && c > 0) sm_count = c;
+    }
+    cudaGetLastError();
+    const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
+    const int64_t units = mtiles * ((static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols);
+    return gemv_ws_bytes(gemv_workers(sm_count, units));
+}
+
+int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, void* workspace,
+                  size_t workspace_bytes, apd_stream_t stream) {
+    GemvShape g;
+    int rc = gemv_validate(x, w, y, &g);
+    if (rc) return rc;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)) return APD_ERR_WORKSPACE;
+    DeviceState* dev = nullptr;
+    rc = device_state(&dev);
+    if (rc) return rc;
+    const int64_t workers = gemv_workers(dev->sm_count, g.units);
+    if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
+    auto kern = apd::gemv_kernel<kGemvStages>;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->gemv_attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(gemv_smem_bytes()));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv_kernel)");
+            dev->gemv_attr_set = true;
+        }
+    }
+    CUtensorMap wmap, xmap;
+    rc = encode_gemv_map(&wmap, w, g.ldw, apd::kGemvRows);
+    if (!rc) rc = encode_gemv_map(&xmap, x, g.ldx, apd::kGemvXRows);
+    if (rc) return rc;
+    apd::GemvParams gp;
+    gp.y = static_cast<__nv_bfloat16*>(y->data);
+    gp.y_sm = g.ysm;
+    gp.y_sn = g.ysn;
+    gp.flags = static_cast<uint32_t*>(workspace);
+    gp.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + kWsAlign);
+    gp.M = g.M;
+    gp.N = g.N;
+    gp.K = g.K;
+    gp.mtiles = static_cast<int32_t>(g.mtiles);
+    gp.ktiles = static_cast<int32_t>(g.ktiles);
+    gp.num_workers = static_cast<int32_t>(workers);
+    gp.warps = kGemvWarps;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((workers + kGemvWarps - 1) / kGemvWarps));
+    cfg.blockDim = dim3(32 * kGemvWarps);
+    cfg.dynamicSmemBytes = gemv_smem_bytes();
+    cfg.stream = st;
+    cfg.attrs = pdl_attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, gp, wmap, xmap);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv_kernel launch");
+    cudaLaunchConfig_t cfg2 = {};
+    cfg2.gridDim = dim3(static_cast<unsigned>((g.mtiles + 3) / 4));
+    cfg2.blockDim = dim3(128);
+    cfg2.stream = st;
+    cfg2.attrs = pdl_attr;
+    cfg2.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg2, apd::gemv_sum_kernel, gp);
+    if (e != cudaSuccess) return cuda_fail(e, "gemv_sum_kernel launch");
+    return APD_OK;
 }
 
 int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_stream_t stream, uint32_t* flags,

@@ -114,9 +114,9 @@ typedef enum apd_status {
 size_t apd_workspace_size(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits);
 
 /*
- * apd_workspace_init -- zero the workspace header (the sticky device flags).
- * Enqueued on `stream`; call once after allocating a workspace (a workspace
- * that is all zeros is already initialised).  Not needed for correct output.
+ * apd_workspace_init -- zero a workspace (all workspace_bytes of it), enqueued on
+ * `stream`, which clears the sticky device flags.  Optional: correct output does
+ * not depend on the workspace's contents.
  */
 int apd_workspace_init(void* workspace, size_t workspace_bytes, apd_stream_t stream);
 
@@ -261,6 +261,34 @@ int apd_attn_contig_decode_ex(const apd_tensor* q, const apd_tensor* k, const ap
 int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
                                   const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
                                   float scale, int num_splits, apd_stream_t stream);
+
+/*
+ * apd_gemv_bf16 -- the decode projection y = x W^T of a bf16 linear layer with a
+ * few activation rows (AstrAI commit logs of astrai/extension/ops/gemv.py and
+ * docs/developer/decode_linear_benchmark.md: the bf16 GEMV that decode-time
+ * linear layers use for M = 1..8, weights [out_features, in_features]).
+ *
+ *   x          bf16 [M, K], 1 <= M <= APD_GEMV_MAX_M, K a multiple of 8, K
+ *              contiguous, row stride a multiple of 8 elements, base 16-byte
+ *              aligned.
+ *   w          bf16 [N, K] with the same layout rules (a linear layer's weight).
+ *   y          bf16 [M, N], any strides (2-byte aligned); y[m][n] =
+ *              sum_k x[m][k] * w[n][k], accumulated in fp32 on tensor cores and
+ *              rounded to bf16 (nearest-even).
+ *   workspace  at least apd_gemv_workspace_size(M, N, K) bytes, 256-byte aligned,
+ *              caller-owned; scratch between calls (calls sharing a workspace must
+ *              be ordered on the device).
+ *
+ * Same conventions as apd_attn_paged_decode: no allocation, no synchronisation,
+ * stream-ordered, capturable in a CUDA graph; argument faults are returned
+ * before anything is launched.
+ */
+#define APD_GEMV_MAX_M 8
+
+size_t apd_gemv_workspace_size(int m, int n, int k);
+
+int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, void* workspace,
+                  size_t workspace_bytes, apd_stream_t stream);
 
 /*
  * apd_read_device_flags -- synchronise `stream`, copy the sticky APD_FLAG_* word

@@ -310,3 +310,22 @@ def test_paged_entry_still_rejects_a_null_page_table_descriptor():
     rc = L.apd_attn_paged_decode_noalloc(ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]), None,
                                          ctypes.byref(p["sl"]), ctypes.byref(p["out"]), ctypes.c_float(1.0), 0, None)
     assert rc == NULLP
+
+
+# ---------------------------------------------------------------- GEMV
+def gemv_call(x, w, y, ws=FAKE, ws_bytes=1 << 30):
+    return apd.lib().apd_gemv_bf16(ctypes.byref(x), ctypes.byref(w), ctypes.byref(y), ws, ws_bytes, None)
+
+
+def test_gemv_validation():
+    assert gemv_call(T([9, 64]), T([16, 64]), T([9, 16])) == SHAPE      # M > 8
+    assert gemv_call(T([2, 64]), T([16, 32]), T([2, 16])) == SHAPE      # K mismatch
+    assert gemv_call(T([2, 64]), T([16, 64]), T([2, 15])) == SHAPE      # y shape
+    assert gemv_call(T([2, 60]), T([16, 60]), T([2, 16])) == LAYOUT     # K % 8
+    assert gemv_call(T([2, 64], stride=[68, 1]), T([16, 64]), T([2, 16])) == LAYOUT  # row stride not 16-B
+    assert gemv_call(T([2, 64], apd.DTYPE_FP32), T([16, 64]), T([2, 16])) == DTYPE
+    x = T([2, 64]); x.data = None
+    assert gemv_call(x, T([16, 64]), T([2, 16])) == NULLP
+    assert gemv_call(T([2, 64]), T([16, 64]), T([2, 16]), ws=None) == WS
+    assert apd.lib().apd_gemv_workspace_size(9, 16, 64) == 0
+    assert apd.gemv_workspace_size(8, 100000, 1536) % 256 == 0

@@ -1,0 +1,82 @@
+"""GPU parity of the decode projection GEMV (apd_gemv_bf16) against the fp64 oracle.
+
+Per element: |gpu - ref| <= 2^-8 |ref| + 2^-13 sum_k |x w|, i.e. the bf16 rounding
+of the output (at most one ulp allowed) plus fp32 accumulation error scaled by the
+magnitude of the terms.  Shapes cover every M in 1..8, N and K tails, strided
+operands, tiny and very wide layers, and the AstrAI-1B projection shapes at full
+size."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_paged_split_b200 as apd
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def check(y, x, w, what=""):
+    ref, absref = oracle.gemv(x, w)
+    got = y.to(torch.float64).cpu().numpy()
+    assert np.isfinite(got).all(), what
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -13 * absref
+    assert (err <= bound).all(), f"{what}: max err {err.max():.3e}, worst ratio {(err / bound).max():.2f}"
+
+
+@pytest.mark.parametrize("M", range(1, 9))
+@pytest.mark.parametrize("N,K", [(64, 256), (37, 1000), (1, 8), (300, 4104), (16, 264)])
+def test_gemv_shapes(M, N, K):
+    c = workloads.gemv_case(M, N, K, seed=M * 7 + N)
+    y = apd.gemv(c.x.cuda(), c.w.cuda())
+    check(y, c.x, c.w, f"M={M} N={N} K={K}")
+
+
+def test_gemv_strided_operands():
+    c = workloads.gemv_case(5, 200, 512, seed=3)
+    xb = torch.zeros(5, 640, dtype=torch.bfloat16, device="cuda")
+    xb[:, 64:576] = c.x.cuda()
+    wb = torch.zeros(200, 528, dtype=torch.bfloat16, device="cuda")
+    wb[:, 8:520] = c.w.cuda()
+    yt = torch.full((200, 5), float("nan"), dtype=torch.bfloat16, device="cuda")  # y as a transposed view
+    apd.gemv(xb[:, 64:576], wb[:, 8:520], yt.t())
+    check(yt.t(), c.x, c.w, "strided")
+
+
+@pytest.mark.parametrize("layer", list(workloads.GEMV_SHAPES))
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_gemv_projection_shapes(layer, M):
+    c = workloads.gemv_named(layer, M)
+    check(apd.gemv(c.x.cuda(), c.w.cuda()), c.x, c.w, f"{layer} M={M}")
+
+
+def test_gemv_graph_capture_and_repeat():
+    c = workloads.gemv_case(4, 1000, 2048, seed=9)
+    x, w = c.x.cuda(), c.w.cuda()
+    ws = torch.zeros(apd.gemv_workspace_size(4, 1000, 2048), dtype=torch.uint8, device="cuda")
+    y = torch.empty(4, 1000, dtype=torch.bfloat16, device="cuda")
+    apd.gemv(x, w, y, ws)
+    first = y.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            apd.gemv(x, w, y, ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    y.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, first)  # deterministic
+
+
+def test_gemv_rejects_bad_arguments():
+    x = torch.zeros(9, 64, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(16, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(Exception):
+        apd.gemv(x, w)  # M > 8
+    with pytest.raises(apd.APDError):
+        apd.gemv(torch.zeros(2, 60, dtype=torch.bfloat16, device="cuda"),
+                 torch.zeros(16, 60, dtype=torch.bfloat16, device="cuda"),
+                 workspace=torch.zeros(1 << 20, dtype=torch.uint8, device="cuda"))  # K % 8 != 0
