@@ -194,3 +194,73 @@ def gemv(x: torch.Tensor, w: torch.Tensor, nthreads: int = 0):
     _check(_gemv().oracle_gemv(x.data_ptr(), x.stride(0), w.data_ptr(), w.stride(0), M, N, K, _dptr(y), _dptr(a),
                                nthreads), "gemv")
     return y, a
+
+
+class _PrefillProblem(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p),
+        ("q_stride", ctypes.c_int64 * 4),
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("kv_stride", ctypes.c_int64 * 4),
+        ("page_table", ctypes.c_void_p),
+        ("pt_stride", ctypes.c_int64 * 2),
+        ("seq_lens", ctypes.c_void_p),
+        ("mask", ctypes.c_void_p),
+        ("mask_stride", ctypes.c_int64 * 3),
+        ("mask_kv_len", ctypes.c_int64),
+        ("batch", ctypes.c_int32),
+        ("q_len", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
+        ("causal_offset", ctypes.c_int32),
+        ("scale", ctypes.c_double),
+    ]
+
+
+_prefill_lib = None
+
+
+def _prefill():
+    global _prefill_lib
+    if _prefill_lib is None:
+        L = ctypes.CDLL(_build.build_prefill())
+        L.oracle_paged_prefill.argtypes = [ctypes.POINTER(_PrefillProblem), ctypes.POINTER(ctypes.c_double),
+                                           ctypes.c_int]
+        _prefill_lib = L
+    return _prefill_lib
+
+
+def paged_prefill(w, nthreads: int = 0) -> np.ndarray:
+    """Multi-query attention of a ``workloads.PrefillWorkload``: float64 [B, Lq, Hq, D]."""
+    q, k, v = w.q, w.k_cache, w.v_cache
+    pt = w.page_table.to(torch.int32)
+    sl = w.seq_lens.to(torch.int32).contiguous()
+    mask = w.mask
+    keep = [q, k, v, pt, sl, mask]
+    s = _PrefillProblem()
+    s.q = q.data_ptr()
+    s.q_stride = (ctypes.c_int64 * 4)(*q.stride())
+    s.k, s.v = k.data_ptr(), v.data_ptr()
+    s.kv_stride = (ctypes.c_int64 * 4)(*k.stride())
+    s.page_table = pt.data_ptr()
+    s.pt_stride = (ctypes.c_int64 * 2)(*pt.stride())
+    s.seq_lens = sl.data_ptr()
+    if mask is not None:
+        assert mask.dtype == torch.uint8
+        ms = mask.stride()
+        s.mask = mask.data_ptr()
+        s.mask_stride = (ctypes.c_int64 * 3)(ms[0], 0, ms[1]) if mask.dim() == 2 else (ctypes.c_int64 * 3)(*ms)
+        s.mask_kv_len = mask.shape[-1]
+    s.batch, s.q_len, s.num_q_heads, s.head_dim = q.shape[0], q.shape[1], q.shape[2], q.shape[3]
+    s.num_kv_heads, s.page_size, s.num_pages, s.max_pages = k.shape[2], k.shape[1], k.shape[0], pt.shape[1]
+    s.causal_offset = int(w.causal_offset)
+    s.scale = float(w.scale)
+    out = np.zeros(tuple(q.shape), dtype=np.float64)
+    _check(_prefill().oracle_paged_prefill(ctypes.byref(s), _dptr(out), nthreads), "paged_prefill")
+    del keep
+    return out

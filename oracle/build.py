@@ -13,6 +13,8 @@ SRC = os.path.join(HERE, "paged_decode_oracle.c")
 LIB = os.path.join(HERE, "liboracle_paged_decode.so")
 GEMV_SRC = os.path.join(HERE, "gemv_oracle.c")
 GEMV_LIB = os.path.join(HERE, "liboracle_gemv.so")
+PREFILL_SRC = os.path.join(HERE, "paged_prefill_oracle.c")
+PREFILL_LIB = os.path.join(HERE, "liboracle_paged_prefill.so")
 
 
 def _build_one(src: str, lib: str, force: bool, verbose: bool) -> str:
@@ -30,13 +32,18 @@ def _build_one(src: str, lib: str, force: bool, verbose: bool) -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Build both oracle libraries; returns the decode-attention one."""
+    """Build every oracle library; returns the decode-attention one."""
     _build_one(GEMV_SRC, GEMV_LIB, force, verbose)
+    _build_one(PREFILL_SRC, PREFILL_LIB, force, verbose)
     return _build_one(SRC, LIB, force, verbose)
 
 
 def build_gemv(force: bool = False, verbose: bool = False) -> str:
     return _build_one(GEMV_SRC, GEMV_LIB, force, verbose)
+
+
+def build_prefill(force: bool = False, verbose: bool = False) -> str:
+    return _build_one(PREFILL_SRC, PREFILL_LIB, force, verbose)
 
 
 if __name__ == "__main__":

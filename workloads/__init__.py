@@ -488,3 +488,78 @@ def gemv_case(M: int, N: int, K: int, seed: int = 7, name: str | None = None, va
 def gemv_named(layer: str, M: int, seed: int = 7, **kw) -> GemvCase:
     N, K = GEMV_SHAPES[layer]
     return gemv_case(M, N, K, seed=seed, name=f"gemv_{layer}_m{M}_n{N}_k{K}", **kw)
+
+
+# ----------------------------------------------------------------------------
+# Multi-query (chunked prefill) inputs over the same paged cache
+# ----------------------------------------------------------------------------
+_S_PQ, _S_MASK = 13, 14
+
+
+@dataclass
+class PrefillWorkload:
+    """Lq query tokens per sequence against a paged cache (all host tensors)."""
+
+    name: str
+    seed: int
+    q: torch.Tensor            # bf16 [B, Lq, Hq, D]
+    k_cache: torch.Tensor      # bf16 [NP, P, Hkv, D]
+    v_cache: torch.Tensor
+    page_table: torch.Tensor   # int32 [B, MP]
+    seq_lens: torch.Tensor     # int32 [B]
+    scale: float
+    causal_offset: int = -1    # -1: no causal mask; c >= 0: query i sits at position c + i
+    mask: torch.Tensor | None = None  # uint8 [B, kv_len] or [B, Lq, kv_len]; nonzero = visible
+
+    @property
+    def batch(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def q_len(self) -> int:
+        return self.q.shape[1]
+
+    def algorithmic_bytes(self) -> int:
+        """KV bytes of the visible range of every sequence + q + out (bf16)."""
+        B, Lq, Hq, D = self.q.shape
+        Hkv = self.k_cache.shape[2]
+        kv = 0
+        for b in range(B):
+            L = int(self.seq_lens[b])
+            if self.causal_offset >= 0:
+                L = min(L, self.causal_offset + Lq)
+            kv += L
+        return kv * Hkv * D * 4 + 2 * B * Lq * Hq * D * 2
+
+    def algorithmic_flops(self) -> int:
+        """QK^T + PV over the (query, key) pairs each query sees without a mask."""
+        B, Lq, Hq, D = self.q.shape
+        pairs = 0
+        for b in range(B):
+            L = int(self.seq_lens[b])
+            for i in range(Lq):
+                pairs += L if self.causal_offset < 0 else max(0, min(L, self.causal_offset + i + 1))
+        return 4 * D * Hq * pairs
+
+
+def make_prefill(*, name: str, seed: int, batch: int, q_len: int, num_q_heads: int, num_kv_heads: int,
+                 head_dim: int, seq_lens, page_size: int = 32, causal_offset: int = -1, mask: str | None = None,
+                 mask_keep: float = 0.9, layout: str = "NHD", poison: bool = False, pool_pages: int | None = None,
+                 max_pages_per_seq: int | None = None, scale: float | None = None) -> PrefillWorkload:
+    """``mask``: None, "2d" ([B, kv_len]) or "3d" ([B, Lq, kv_len]), each entry visible
+    with probability ``mask_keep`` (seeded), kv_len = max_pages_per_seq * page_size."""
+    base = make(name=name, seed=seed, batch=batch, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                head_dim=head_dim, page_size=page_size, seq_lens=seq_lens, pool_pages=pool_pages,
+                max_pages_per_seq=max_pages_per_seq, scale=scale, layout=layout, poison=poison)
+    q = seeded_randn_bf16(batch * q_len * num_q_heads * head_dim, seed, _S_PQ).view(
+        batch, q_len, num_q_heads, head_dim)
+    m = None
+    if mask is not None:
+        kv_len = base.page_table.shape[1] * page_size
+        shape = (batch, kv_len) if mask == "2d" else (batch, q_len, kv_len)
+        n = int(np.prod(shape))
+        keep = seeded_bernoulli(n, mask_keep, seed, _S_MASK).view(*shape)
+        m = keep.to(torch.uint8)
+    return PrefillWorkload(name=name, seed=seed, q=q, k_cache=base.k_cache, v_cache=base.v_cache,
+                           page_table=base.page_table, seq_lens=base.seq_lens, scale=base.scale,
+                           causal_offset=causal_offset, mask=m)
