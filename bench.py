@@ -44,6 +44,8 @@ DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000, 
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
 GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes per call / time)"
 GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
+PREFILL_METRIC = "paged multi-query (prefill chunk) attention achieved TFLOP/s and HBM GB/s"
+PREFILL_WORKLOADS = ["prefill_llama8b_chunk"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
 
 
@@ -53,7 +55,8 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(workloads.NAMED) + GEMV_WORKLOADS, default="llama8b",
+    p.add_argument("--workload", choices=sorted(workloads.NAMED) + GEMV_WORKLOADS + PREFILL_WORKLOADS,
+                   default="llama8b",
                    help="a decode-attention workload, or gemv_<layer>_m<M> for the decode projection")
     p.add_argument("--num-splits", type=int, default=0, help="0 = auto (the default launch configuration)")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
@@ -687,16 +690,126 @@ def run_gemv(a):
     return 0
 
 
+# ---------------------------------------------------------------- multi-query (prefill chunk)
+def peak_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 1590.0, "fallback"
+
+
+def run_prefill(a):
+    """The prefill chunk on one GPU: CUDA-graph replays of the call over two cache
+    instances used in turn (each larger than L2)."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        print("no CUDA device", file=sys.stderr)
+        return 2
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_group(world, "nccl")
+    import decode_attention_paged_split_b200 as apd
+
+    ws = [workloads.prefill_llama8b_chunk(seed=8 + 1000003 * rank + i) for i in range(2)]
+    dev = [dict(q=w.q.to(device), k=w.k_cache.contiguous().to(device), v=w.v_cache.contiguous().to(device),
+                pt=w.page_table.to(device), sl=w.seq_lens.to(device), out=torch.empty_like(w.q, device=device))
+           for w in ws]
+    w0 = ws[0]
+    per_bytes, per_flops = w0.algorithmic_bytes(), w0.algorithmic_flops()
+    stream = torch.cuda.Stream(device)
+
+    def call(i):
+        d, w = dev[i % 2], ws[i % 2]
+        apd.attn_paged_prefill(d["q"], d["k"], d["v"], d["pt"], d["sl"], w.scale, w.causal_offset, None, d["out"],
+                               stream=stream)
+
+    for i in range(a.warmup):
+        call(i)
+    torch.cuda.synchronize(device)
+    plan = []
+    full, rest = divmod(a.steps, GRAPH_CHUNK)
+    for n, reps in ((GRAPH_CHUNK, full), (rest, 1 if rest else 0)):
+        if reps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(n):
+                        call(i)
+            plan.append((g, reps))
+
+    def replay():
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for g, reps in plan:
+                for _ in range(reps):
+                    g.replay()
+            e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    replay()
+    clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    el = replay()
+    barrier(dist, device)
+    clock_info = clocks.stop()
+    plan = []
+    t_max = max_over_ranks(el, dist, device)
+    bytes_all = sum_over_ranks(float(per_bytes * a.steps), dist, device)
+    flops_all = sum_over_ranks(float(per_flops * a.steps), dist, device)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import oracle
+
+        sample = workloads.prefill_llama8b_chunk(batch=1, seq_lens=[4096])
+        t0 = time.perf_counter()
+        oracle.paged_prefill(sample)
+        el_cpu = time.perf_counter() - t0
+        cpu = {"value": sample.algorithmic_flops() / el_cpu / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(),
+               "kind": "oracle", "sample": f"sequence 0 only (1 of 16) of the chunk, fp64, {el_cpu:.1f} s"}
+
+    if rank == 0:
+        us = t_max / a.steps * 1e6
+        tpeak, tsrc = peak_tflops()
+        hpeak, hsrc = peaks()
+        tf = per_flops / (t_max / a.steps) / 1e12
+        gbs = per_bytes / (t_max / a.steps) / 1e9
+        line = {
+            "metric": PREFILL_METRIC, "value": flops_all / t_max / 1e12, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": us / 1e3, "us_per_call": us, "hbm_gbs": gbs,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w0.name, "batch": w0.batch, "q_len": w0.q_len, "num_q_heads": 32,
+                       "num_kv_heads": 8, "head_dim": 128, "seq_len": 4096, "causal_offset": w0.causal_offset,
+                       "algorithmic_bytes_per_call": per_bytes, "algorithmic_flops_per_call": per_flops,
+                       "l2": "two cache instances used in turn, each larger than L2",
+                       "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
+                         "traffic": None, "peak_source": tsrc, "kernel": "prefill_kernel",
+                         "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hpeak},
+            "cpu_baseline": cpu, "e2e": None, "gpu_launches": a.steps, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     a = parse_args(argv)
     if a.impl == "reference":
-        if a.workload.startswith("gemv_"):
+        if a.workload.startswith(("gemv_", "prefill_")):
             print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the decode-attention "
                                                                   "workloads; use the gemv workloads' cpu_baseline"}))
             return 0
         return run_reference(a)
     if a.workload.startswith("gemv_"):
         return run_gemv(a)
+    if a.workload.startswith("prefill_"):
+        return run_prefill(a)
     return run_ours(a)
 
 

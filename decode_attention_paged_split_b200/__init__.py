@@ -22,6 +22,7 @@ __all__ = [
     "APDError",
     "attn_paged_decode",
     "attn_contig_decode",
+    "attn_paged_prefill",
     "gemv",
     "gemv_workspace_size",
     "DecodeCall",
@@ -50,7 +51,9 @@ FLAG_SEQ_LEN_NEGATIVE = 0x4
 FLAG_WAIT_TIMEOUT = 0x8
 NOALLOC_SCRATCH_BYTES = 8 << 20  # APD_NOALLOC_SCRATCH_BYTES
 
-_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.int32: DTYPE_INT32, torch.float32: DTYPE_FP32}
+DTYPE_UINT8 = 4
+_DTYPES = {torch.bfloat16: DTYPE_BF16, torch.int32: DTYPE_INT32, torch.float32: DTYPE_FP32,
+           torch.uint8: DTYPE_UINT8, torch.bool: DTYPE_UINT8}
 
 
 class _Tensor(ctypes.Structure):
@@ -131,6 +134,8 @@ def _load():
     L.apd_attn_paged_decode_ex.restype = ctypes.c_int
     L.apd_attn_paged_decode_noalloc.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
     L.apd_attn_paged_decode_noalloc.restype = ctypes.c_int
+    L.apd_attn_paged_prefill.argtypes = [T, T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
+    L.apd_attn_paged_prefill.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
     L.apd_gemv_bf16.argtypes = [T, T, T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
@@ -268,6 +273,29 @@ def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
                                   _stream_handle(stream, q.device))
     if rc:
         raise APDError(rc, "apd_attn_contig_decode")
+    return out
+
+
+def attn_paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
+                       seq_lens: torch.Tensor, scale: float, causal_offset: int = -1,
+                       mask: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Multi-query attention of q [B, Lq, Hq, D] over the paged cache; returns out [B, Lq, Hq, D].
+
+    causal_offset -1: no causal mask; c >= 0: query i sits at position c + i.  mask: None,
+    uint8/bool [B, kv_len] or [B, Lq, kv_len] (nonzero = visible)."""
+    if out is None:
+        out = torch.empty_like(q)
+    if mask is not None and mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    L = _load()
+    descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens)]
+    md = _desc(mask) if mask is not None else None
+    od = _desc(out)
+    rc = L.apd_attn_paged_prefill(*[ctypes.byref(d) for d in descs], ctypes.byref(md) if md is not None else None,
+                                  ctypes.byref(od), ctypes.c_float(scale), int(causal_offset),
+                                  _stream_handle(stream, q.device))
+    if rc:
+        raise APDError(rc, "apd_attn_paged_prefill")
     return out
 
 

@@ -19,6 +19,7 @@
 #include "../../include/attn_paged_decode.h"
 #include "apd_gemv.cuh"
 #include "apd_kernels.cuh"
+#include "apd_prefill.cuh"
 
 namespace {
 
@@ -171,6 +172,7 @@ struct DeviceState {
     int sm_count = 0;
     bool smem_attr_set[4] = {false, false, false, false};
     bool gemv_attr_set = false;
+    bool prefill_attr_set[4] = {false, false, false, false};
 };
 std::mutex g_mu;
 DeviceState g_devices[128];
@@ -534,6 +536,136 @@ int gemv_validate(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     return APD_OK;
 }
 
+// ---------------------------------------------------------------- multi-query (prefill)
+int prefill_stages(int D) { return D == 32 ? 8 : D == 64 ? 6 : D == 128 ? 4 : 3; }
+
+size_t prefill_smem_bytes(int D) {
+    return 16ull * prefill_stages(D) + 1024 + static_cast<size_t>(prefill_stages(D)) * 2 * apd::kTile * D * 2;
+}
+
+struct PrefillCheck {
+    Validated V;  // the KV side, checked as for decode (q's role taken by a [B, Hq, D] view)
+    int Lq;
+    int64_t qst[4], ost[4], mst[3];
+    int mask_dims;
+};
+
+int prefill_validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, const apd_tensor* pt,
+                     const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out, int causal_offset,
+                     PrefillCheck* C) {
+    if (!q || !out || !pt) return APD_ERR_NULL_POINTER;
+    if (q->dtype != APD_DTYPE_BF16 || out->dtype != APD_DTYPE_BF16) return APD_ERR_DTYPE;
+    if (q->ndim != 4 || out->ndim != 4) return APD_ERR_SHAPE;
+    for (int i = 0; i < 4; ++i)
+        if (q->shape[i] != out->shape[i] || q->shape[i] < 0) return APD_ERR_SHAPE;
+    if (q->shape[1] < 1 || q->shape[1] > (1 << 20)) return APD_ERR_SHAPE;
+    if (causal_offset < -1) return APD_ERR_ARGUMENT;
+    // the KV side and the per-sequence tensors: reuse the decode checks on [B, Hq, D] views
+    apd_tensor q3 = *q, o3 = *out;
+    q3.ndim = o3.ndim = 3;
+    q3.shape[1] = q->shape[2];
+    q3.shape[2] = q->shape[3];
+    q3.stride[1] = q->stride[2];
+    q3.stride[2] = q->stride[3];
+    o3.shape[1] = out->shape[2];
+    o3.shape[2] = out->shape[3];
+    o3.stride[1] = out->stride[2];
+    o3.stride[2] = out->stride[3];
+    int rc = validate(&q3, k, v, pt, sl, &o3, 0, &C->V);
+    if (rc) return rc;
+    C->Lq = static_cast<int>(q->shape[1]);
+    if (static_cast<int64_t>(C->Lq) * C->V.s.g > (1 << 26)) return APD_ERR_TOO_LARGE;
+    if (C->V.s.B > 0 && (!aligned_bf16_layout(q, C->qst) || !aligned_bf16_layout(out, C->ost))) return APD_ERR_LAYOUT;
+    C->mask_dims = 0;
+    C->mst[0] = C->mst[1] = C->mst[2] = 0;
+    if (mask) {
+        if (mask->dtype != APD_DTYPE_UINT8) return APD_ERR_DTYPE;
+        if (mask->ndim != 2 && mask->ndim != 3) return APD_ERR_SHAPE;
+        if (mask->shape[0] != q->shape[0]) return APD_ERR_SHAPE;
+        if (mask->ndim == 3 && mask->shape[1] != q->shape[1]) return APD_ERR_SHAPE;
+        // every key index below the page-table capacity must be inside the mask
+        if (mask->shape[mask->ndim - 1] < static_cast<int64_t>(C->V.MP) * C->V.P) return APD_ERR_SHAPE;
+        if (C->V.s.B > 0 && is_null(mask)) return APD_ERR_NULL_POINTER;
+        int64_t st[3];
+        normalized_strides(mask, st);
+        for (int i = 0; i < mask->ndim; ++i)
+            if (st[i] < 0) return APD_ERR_LAYOUT;
+        C->mst[0] = st[0];
+        C->mst[1] = mask->ndim == 3 ? st[1] : 0;
+        C->mst[2] = st[mask->ndim - 1];
+        C->mask_dims = mask->ndim;
+    }
+    return APD_OK;
+}
+
+template <int D>
+int launch_prefill(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                   const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
+                   float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
+    constexpr int kStages = (D == 32) ? 8 : (D == 64) ? 6 : (D == 128) ? 4 : 3;
+    auto kern = apd::prefill_kernel<D, kStages>;
+    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->prefill_attr_set[kSlot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(prefill_smem_bytes(D)));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_kernel)");
+            dev->prefill_attr_set[kSlot] = true;
+        }
+    }
+    CUtensorMap kmap, vmap;
+    int rc = encode_kv_map(&kmap, k, C.V.kst, D);
+    if (!rc) rc = encode_kv_map(&vmap, v, C.V.vst, D);
+    if (rc) return rc;
+    const Shape& s = C.V.s;
+    apd::PrefillParams pp;
+    pp.q = static_cast<const __nv_bfloat16*>(q->data);
+    pp.q_sb = C.qst[0];
+    pp.q_si = C.qst[1];
+    pp.q_sh = C.qst[2];
+    pp.out = static_cast<__nv_bfloat16*>(out->data);
+    pp.o_sb = C.ost[0];
+    pp.o_si = C.ost[1];
+    pp.o_sh = C.ost[2];
+    pp.page_table = static_cast<const int32_t*>(pt->data);
+    pp.pt_s0 = C.V.pst[0];
+    pp.pt_s1 = C.V.pst[1];
+    pp.seq_lens = static_cast<const int32_t*>(sl->data);
+    pp.mask = mask ? static_cast<const uint8_t*>(mask->data) : nullptr;
+    pp.m_sb = C.mst[0];
+    pp.m_si = C.mst[1];
+    pp.m_st = C.mst[2];
+    pp.flags = nullptr;
+    pp.B = s.B;
+    pp.Lq = C.Lq;
+    pp.Hq = s.Hq;
+    pp.Hkv = s.Hkv;
+    pp.g = s.g;
+    pp.P = C.V.P;
+    pp.NP = C.V.NP;
+    pp.MP = C.V.MP;
+    constexpr int kRows = apd::PrefillShape<D>::kRows;
+    pp.blocks_per_head = static_cast<int32_t>((static_cast<int64_t>(C.Lq) * s.g + kRows - 1) / kRows);
+    pp.causal_offset = causal_offset;
+    pp.scale_log2 = scale * 1.4426950408889634f;
+    const int64_t grid = static_cast<int64_t>(s.B) * s.Hkv * pp.blocks_per_head;
+    if (grid > INT32_MAX) return APD_ERR_TOO_LARGE;
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(apd::PrefillShape<D>::kThreads);
+    cfg.dynamicSmemBytes = prefill_smem_bytes(D);
+    cfg.stream = stream;
+    cfg.attrs = pdl_attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill_kernel launch");
+    return APD_OK;
+}
+
 // ---------------------------------------------------------------- built-in scratch
 // Scratch of apd_attn_paged_decode_noalloc: a static device array, so that entry
 // point allocates nothing.  Host code must not use its name as an address (on the
@@ -694,6 +826,26 @@ int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache
         case 64: return launch<64>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
         case 128: return launch<128>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
         case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, scratch, dev, st, nullptr);
+        default: return APD_ERR_HEAD_DIM;
+    }
+}
+
+int apd_attn_paged_prefill(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                           const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* mask,
+                           const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream) {
+    PrefillCheck C;
+    int rc = prefill_validate(q, k_cache, v_cache, page_table, seq_lens, mask, out, causal_offset, &C);
+    if (rc) return rc;
+    if (C.V.s.B == 0) return APD_OK;
+    DeviceState* dev = nullptr;
+    rc = device_state(&dev);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    switch (C.V.s.D) {
+        case 32: return launch_prefill<32>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+        case 64: return launch_prefill<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+        case 128: return launch_prefill<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+        case 256: return launch_prefill<256>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
         default: return APD_ERR_HEAD_DIM;
     }
 }

@@ -51,7 +51,8 @@ typedef struct CUstream_st* apd_stream_t;
 typedef enum apd_dtype {
     APD_DTYPE_BF16 = 1,
     APD_DTYPE_INT32 = 2,
-    APD_DTYPE_FP32 = 3
+    APD_DTYPE_FP32 = 3,
+    APD_DTYPE_UINT8 = 4
 } apd_dtype;
 
 /* A strided view of device memory.  `stride` is in elements; only the first
@@ -221,6 +222,34 @@ int apd_attn_contig_decode_ex(const apd_tensor* q, const apd_tensor* k, const ap
                               const apd_tensor* seq_lens, const apd_tensor* out, float scale, int num_splits,
                               void* workspace, size_t workspace_bytes, apd_stream_t stream,
                               const apd_launch_options* options);
+
+/*
+ * apd_attn_paged_prefill -- multi-query (chunked prefill) attention over the same
+ * paged cache (AstrAI commit log of csrc/kernels/attn_paged_decode.cu: prefill
+ * kernels templated on the paged KV policy, the unified causal_offset, and 2-D /
+ * 3-D masks that may be combined with causal).
+ *
+ *   q          bf16 [B, Lq, Hq, D] (Lq >= 1 new query tokens per sequence), D
+ *              contiguous, other strides multiples of 8 elements, base 16-byte
+ *              aligned.
+ *   k_cache, v_cache, page_table, seq_lens, scale: as in apd_attn_paged_decode;
+ *              seq_lens[b] keys are stored for sequence b.
+ *   mask       NULL, or uint8 [B, kv_len] (one row per sequence) or [B, Lq, kv_len]
+ *              (one row per query), nonzero = visible, kv_len >=
+ *              max_pages_per_seq * page_size, any non-negative strides.
+ *   out        bf16 [B, Lq, Hq, D], same layout rules as q.
+ *   causal_offset  -1: no causal mask; c >= 0: query i sits at position c + i and
+ *              sees keys t <= c + i.
+ *
+ * Query i of sequence b sees key t when t < seq_lens[b], the causal rule allows it
+ * and the mask (if any) is nonzero at t; the output is the softmax-weighted sum of
+ * the visible V rows, or zeros when no key is visible.  One kernel launch, no
+ * workspace, no split of the key range (each CTA streams its rows' whole range).
+ * Same threading, error and device-contract conventions as apd_attn_paged_decode.
+ */
+int apd_attn_paged_prefill(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                           const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* mask,
+                           const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream);
 
 /*
  * apd_attn_paged_decode_noalloc -- the same decode call for callers that cannot

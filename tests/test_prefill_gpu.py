@@ -1,0 +1,111 @@
+"""GPU parity of the multi-query (chunked prefill) call against the fp64 oracle.
+
+Per element |gpu - ref| <= 1e-2 + 1e-2 |ref|, as for decode.  Covered: every head
+dim, GQA groups 1/4/8/20, query counts from 1 to 70 (several 64-row blocks and a
+ragged last block), no causal mask, causal offsets that cut the key range, 2-D and
+3-D masks, rows that see no key (zeros), NaN-poisoned slots that must not be read,
+larger pages, HND storage and a graph capture."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_paged_split_b200 as apd
+import oracle
+import workloads
+from gpu_util import check_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run(w, stream=None):
+    heads_outer = w.k_cache.stride(1) < w.k_cache.stride(2)  # HND storage passed as a view
+    def dev(t):
+        if heads_outer:
+            return t.permute(0, 2, 1, 3).contiguous().cuda().permute(0, 2, 1, 3)
+        return t.contiguous().cuda()
+    q = w.q.cuda()
+    mask = w.mask.cuda() if w.mask is not None else None
+    out = torch.full_like(q, float("nan"))
+    apd.attn_paged_prefill(q, dev(w.k_cache), dev(w.v_cache), w.page_table.cuda(), w.seq_lens.cuda(), w.scale,
+                           w.causal_offset, mask, out, stream=stream)
+    torch.cuda.synchronize()
+    return out
+
+
+def case(seed, D=64, Hq=8, Hkv=2, Lq=5, lens=(40, 9, 100), causal=-1, mask=None, P=32, **kw):
+    mp = max(1, -(-max(lens) // P))
+    return workloads.make_prefill(name="pf", seed=seed, batch=len(lens), q_len=Lq, num_q_heads=Hq,
+                                  num_kv_heads=Hkv, head_dim=D, seq_lens=list(lens), page_size=P, causal_offset=causal,
+                                  mask=mask, max_pages_per_seq=mp, **kw)
+
+
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
+@pytest.mark.parametrize("causal", [-1, 60])
+@pytest.mark.parametrize("mask", [None, "2d", "3d"])
+def test_prefill_head_dims_causal_masks(D, causal, mask):
+    w = case(3, D=D, causal=causal, mask=mask, poison=True)
+    check_close(run(w), oracle.paged_prefill(w), f"D={D} causal={causal} mask={mask}")
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (40, 2)])
+@pytest.mark.parametrize("Lq", [1, 16, 17, 70])
+def test_prefill_groups_and_query_counts(Hq, Hkv, Lq):
+    w = case(5, D=128, Hq=Hq, Hkv=Hkv, Lq=Lq, lens=(300, 77), causal=300 - Lq)
+    check_close(run(w), oracle.paged_prefill(w), f"{Hq}/{Hkv} Lq={Lq}")
+
+
+def test_prefill_rows_that_see_nothing_are_zero():
+    w = case(6, D=64, Lq=4, lens=(50, 0, 20), mask="3d", mask_keep=0.5)
+    w.mask[0, 2] = 0  # query 2 of sequence 0 sees no key
+    out = run(w)
+    ref = oracle.paged_prefill(w)
+    check_close(out, ref, "zero rows")
+    assert torch.all(out[1] == 0) and torch.all(out[0, 2] == 0)
+
+
+def test_prefill_causal_offset_zero():
+    w = case(7, D=128, Lq=33, lens=(40, 100), causal=0, poison=True)
+    check_close(run(w), oracle.paged_prefill(w), "causal 0")
+
+
+@pytest.mark.parametrize("P", [64, 128])
+def test_prefill_larger_pages_hnd(P):
+    w = case(8, D=128, Hq=16, Hkv=4, Lq=9, lens=(257, 31), causal=250, P=P, layout="HND", poison=True)
+    check_close(run(w), oracle.paged_prefill(w), f"P={P} HND")
+
+
+def test_prefill_side_stream_and_graph():
+    w = case(9, D=64, Hq=32, Hkv=8, Lq=12, lens=(200, 500), causal=480, mask="2d")
+    q = w.q.cuda()
+    k, v, pt, sl = w.k_cache.cuda(), w.v_cache.cuda(), w.page_table.cuda(), w.seq_lens.cuda()
+    mask = w.mask.cuda()
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s)
+        with torch.cuda.graph(g, stream=s):
+            apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    check_close(out, oracle.paged_prefill(w), "graph replay")
+
+
+def test_prefill_chunk_at_scale():
+    """A 128-token chunk of 4 sequences of 1024 keys, 32/8 heads, D = 128, causal."""
+    w = case(10, D=128, Hq=32, Hkv=8, Lq=128, lens=(1024, 1024, 1000, 640), causal=None or 0)
+    w.causal_offset = 1024 - 128
+    check_close(run(w), oracle.paged_prefill(w), "chunk at scale")
+
+
+def test_prefill_rejects_bad_arguments():
+    w = case(11, D=64, Lq=3, lens=(10, 20, 30), mask="2d")
+    q = w.q.cuda()
+    args = (w.k_cache.cuda(), w.v_cache.cuda(), w.page_table.cuda(), w.seq_lens.cuda(), w.scale)
+    with pytest.raises(apd.APDError):  # causal offset below -1
+        apd.attn_paged_prefill(q, *args, causal_offset=-5)
+    with pytest.raises(apd.APDError):  # mask shorter than the page-table capacity
+        apd.attn_paged_prefill(q, *args, mask=w.mask[:, :5].cuda())

@@ -563,3 +563,13 @@ def make_prefill(*, name: str, seed: int, batch: int, q_len: int, num_q_heads: i
     return PrefillWorkload(name=name, seed=seed, q=q, k_cache=base.k_cache, v_cache=base.v_cache,
                            page_table=base.page_table, seq_lens=base.seq_lens, scale=base.scale,
                            causal_offset=causal_offset, mask=m)
+
+
+def prefill_llama8b_chunk(seed: int = 8, **kw) -> PrefillWorkload:
+    """A 128-token prefill chunk at the end of 16 sequences of 4096 keys, 32/8 heads,
+    D = 128, causal (queries at positions 3968..4095), over a shuffled 2048-page pool."""
+    args = dict(name="prefill_llama8b_b16_q128_h32x8_d128_l4096", seed=seed, batch=16, q_len=128, num_q_heads=32,
+                num_kv_heads=8, head_dim=128, seq_lens=[4096] * 16, page_size=32, causal_offset=4096 - 128,
+                pool_pages=2048)
+    args.update(kw)
+    return make_prefill(**args)
