@@ -59,6 +59,8 @@ def parse_args(argv=None):
                    default="llama8b",
                    help="a decode-attention workload, or gemv_<layer>_m<M> for the decode projection")
     p.add_argument("--num-splits", type=int, default=0, help="0 = auto (the default launch configuration)")
+    p.add_argument("--prefill-kernel", choices=["auto", "mma_sync", "tcgen05"], default="auto",
+                   help="kernel of the prefill workload (auto = what attn_paged_prefill picks)")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     p.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks")
@@ -699,6 +701,15 @@ def peak_tflops():
         return 1590.0, "fallback"
 
 
+def prefill_kernel_name(choice):
+    """The kernel the prefill workload (D = 128) runs for a --prefill-kernel choice."""
+    import decode_attention_paged_split_b200 as apd
+
+    if choice == "auto":
+        choice = apd.prefill_auto_kernel(128)
+    return "prefill_tc_kernel" if choice == "tcgen05" else "prefill_kernel"
+
+
 def run_prefill(a):
     """The prefill chunk on one GPU: CUDA-graph replays of the call over two cache
     instances used in turn (each larger than L2)."""
@@ -722,7 +733,7 @@ def run_prefill(a):
     def call(i):
         d, w = dev[i % 2], ws[i % 2]
         apd.attn_paged_prefill(d["q"], d["k"], d["v"], d["pt"], d["sl"], w.scale, w.causal_offset, None, d["out"],
-                               stream=stream)
+                               stream=stream, kernel=a.prefill_kernel)
 
     for i in range(a.warmup):
         call(i)
@@ -788,7 +799,7 @@ def run_prefill(a):
                        "l2": "two cache instances used in turn, each larger than L2",
                        "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                         "traffic": None, "peak_source": tsrc, "kernel": "prefill_kernel",
+                         "traffic": None, "peak_source": tsrc, "kernel": prefill_kernel_name(a.prefill_kernel),
                          "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hpeak},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": a.steps, "clocks": clock_info,
         }

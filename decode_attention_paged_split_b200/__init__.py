@@ -136,6 +136,9 @@ def _load():
     L.apd_attn_paged_decode_noalloc.restype = ctypes.c_int
     L.apd_attn_paged_prefill.argtypes = [T, T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
     L.apd_attn_paged_prefill.restype = ctypes.c_int
+    L.apd_attn_paged_prefill_ex.argtypes = [T, T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                            ctypes.c_int]
+    L.apd_attn_paged_prefill_ex.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
     L.apd_gemv_bf16.argtypes = [T, T, T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
@@ -276,13 +279,28 @@ def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
     return out
 
 
+PREFILL_KERNELS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
+
+
+def prefill_auto_kernel(head_dim: int) -> str:
+    """The kernel attn_paged_prefill(kernel="auto") runs for a head dim."""
+    return "tcgen05" if PREFILL_AUTO_TC and head_dim != 32 else "mma_sync"
+
+
+PREFILL_AUTO_TC = True  # mirrors the library's default choice
+
+
 def attn_paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
                        seq_lens: torch.Tensor, scale: float, causal_offset: int = -1,
-                       mask: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                       mask: torch.Tensor | None = None, out: torch.Tensor | None = None, stream=None,
+                       kernel: str = "auto") -> torch.Tensor:
     """Multi-query attention of q [B, Lq, Hq, D] over the paged cache; returns out [B, Lq, Hq, D].
 
     causal_offset -1: no causal mask; c >= 0: query i sits at position c + i.  mask: None,
-    uint8/bool [B, kv_len] or [B, Lq, kv_len] (nonzero = visible)."""
+    uint8/bool [B, kv_len] or [B, Lq, kv_len] (nonzero = visible).  kernel: "auto",
+    "mma_sync" (every head dim) or "tcgen05" (D = 64, 128, 256)."""
+    if kernel not in PREFILL_KERNELS:
+        raise ValueError(f"kernel must be one of {sorted(PREFILL_KERNELS)}")
     if out is None:
         out = torch.empty_like(q)
     if mask is not None and mask.dtype == torch.bool:
@@ -291,9 +309,9 @@ def attn_paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Te
     descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens)]
     md = _desc(mask) if mask is not None else None
     od = _desc(out)
-    rc = L.apd_attn_paged_prefill(*[ctypes.byref(d) for d in descs], ctypes.byref(md) if md is not None else None,
-                                  ctypes.byref(od), ctypes.c_float(scale), int(causal_offset),
-                                  _stream_handle(stream, q.device))
+    rc = L.apd_attn_paged_prefill_ex(*[ctypes.byref(d) for d in descs], ctypes.byref(md) if md is not None else None,
+                                     ctypes.byref(od), ctypes.c_float(scale), int(causal_offset),
+                                     _stream_handle(stream, q.device), PREFILL_KERNELS[kernel])
     if rc:
         raise APDError(rc, "apd_attn_paged_prefill")
     return out

@@ -19,6 +19,7 @@
 #include "../../include/attn_paged_decode.h"
 #include "apd_gemv.cuh"
 #include "apd_kernels.cuh"
+#include "apd_prefill_tc.cuh"
 #include "apd_prefill.cuh"
 
 namespace {
@@ -173,6 +174,8 @@ struct DeviceState {
     bool smem_attr_set[4] = {false, false, false, false};
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
+    bool prefill_tc_attr_set[4] = {false, false, false, false};
+    bool prefill_tc2_attr_set[4] = {false, false, false, false};
 };
 std::mutex g_mu;
 DeviceState g_devices[128];
@@ -298,7 +301,10 @@ int validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor* v, cons
 //      128-byte swizzle: one box = one [32 x D] tile of one kv head, landing in
 //      shared memory as D/64 blocks of [32 tokens][64 elements].
 //      D == 32 -> 4-D view {32, Hkv, P, NP}, box {32, 1, 32, 1}, 64-byte swizzle.
-int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D) {
+// box_blocks < D/64 (D >= 64): a box holds that many 64-dim blocks instead (the
+// tensor-core prefill loads one block per box so the tile's rows of one block are
+// contiguous).
+int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D, int box_blocks = 0) {
     auto fn = encode_fn();
     if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
     cuuint64_t dims[5], strides[4];
@@ -309,7 +315,7 @@ int encode_kv_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int 
         rank = 5;
         dims[0] = 64; dims[1] = t->shape[2]; dims[2] = t->shape[1]; dims[3] = t->shape[0]; dims[4] = D / 64;
         strides[0] = st[2] * 2; strides[1] = st[1] * 2; strides[2] = st[0] * 2; strides[3] = 128;
-        box[0] = 64; box[1] = 1; box[2] = apd::kTile; box[3] = 1; box[4] = D / 64;
+        box[0] = 64; box[1] = 1; box[2] = apd::kTile; box[3] = 1; box[4] = box_blocks > 0 ? box_blocks : D / 64;
         swz = CU_TENSOR_MAP_SWIZZLE_128B;
     } else {
         rank = 4;
@@ -539,6 +545,9 @@ int gemv_validate(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
 // ---------------------------------------------------------------- multi-query (prefill)
 int prefill_stages(int D) { return D == 32 ? 8 : D == 64 ? 6 : D == 128 ? 4 : 3; }
 
+// Default prefill kernel for D >= 64: the tcgen05 one (mma.sync stays selectable, and serves D = 32).
+constexpr bool kPrefillAutoTc = true;
+
 size_t prefill_smem_bytes(int D) {
     return 16ull * prefill_stages(D) + 1024 + static_cast<size_t>(prefill_stages(D)) * 2 * apd::kTile * D * 2;
 }
@@ -598,26 +607,9 @@ int prefill_validate(const apd_tensor* q, const apd_tensor* k, const apd_tensor*
     return APD_OK;
 }
 
-template <int D>
-int launch_prefill(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
-                   const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
-                   float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
-    constexpr int kStages = (D == 32) ? 8 : (D == 64) ? 6 : (D == 128) ? 4 : 3;
-    auto kern = apd::prefill_kernel<D, kStages>;
-    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!dev->prefill_attr_set[kSlot]) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(prefill_smem_bytes(D)));
-            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_kernel)");
-            dev->prefill_attr_set[kSlot] = true;
-        }
-    }
-    CUtensorMap kmap, vmap;
-    int rc = encode_kv_map(&kmap, k, C.V.kst, D);
-    if (!rc) rc = encode_kv_map(&vmap, v, C.V.vst, D);
-    if (rc) return rc;
+apd::PrefillParams prefill_params(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* pt,
+                                  const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out, float scale,
+                                  int causal_offset, int rows_per_cta) {
     const Shape& s = C.V.s;
     apd::PrefillParams pp;
     pp.q = static_cast<const __nv_bfloat16*>(q->data);
@@ -645,25 +637,108 @@ int launch_prefill(const PrefillCheck& C, const apd_tensor* q, const apd_tensor*
     pp.P = C.V.P;
     pp.NP = C.V.NP;
     pp.MP = C.V.MP;
-    constexpr int kRows = apd::PrefillShape<D>::kRows;
-    pp.blocks_per_head = static_cast<int32_t>((static_cast<int64_t>(C.Lq) * s.g + kRows - 1) / kRows);
+    pp.blocks_per_head =
+        static_cast<int32_t>((static_cast<int64_t>(C.Lq) * s.g + rows_per_cta - 1) / rows_per_cta);
     pp.causal_offset = causal_offset;
     pp.scale_log2 = scale * 1.4426950408889634f;
-    const int64_t grid = static_cast<int64_t>(s.B) * s.Hkv * pp.blocks_per_head;
+    return pp;
+}
+
+template <typename Kernel>
+int launch_prefill_grid(Kernel kern, const apd::PrefillParams& pp, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                        int threads, size_t smem, cudaStream_t stream, const char* what) {
+    const int64_t grid = static_cast<int64_t>(pp.B) * pp.Hkv * pp.blocks_per_head;
     if (grid > INT32_MAX) return APD_ERR_TOO_LARGE;
     cudaLaunchAttribute pdl_attr[1];
     pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(apd::PrefillShape<D>::kThreads);
-    cfg.dynamicSmemBytes = prefill_smem_bytes(D);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cfg.attrs = pdl_attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, pp, kmap, vmap);
-    if (e != cudaSuccess) return cuda_fail(e, "prefill_kernel launch");
+    if (e != cudaSuccess) return cuda_fail(e, what);
     return APD_OK;
+}
+
+// mma.sync kernel (every head dim)
+template <int D>
+int launch_prefill(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                   const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
+                   float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
+    constexpr int kStages = (D == 32) ? 8 : (D == 64) ? 6 : (D == 128) ? 4 : 3;
+    auto kern = apd::prefill_kernel<D, kStages>;
+    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->prefill_attr_set[kSlot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(prefill_smem_bytes(D)));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_kernel)");
+            dev->prefill_attr_set[kSlot] = true;
+        }
+    }
+    CUtensorMap kmap, vmap;
+    int rc = encode_kv_map(&kmap, k, C.V.kst, D);
+    if (!rc) rc = encode_kv_map(&vmap, v, C.V.vst, D);
+    if (rc) return rc;
+    const apd::PrefillParams pp =
+        prefill_params(C, q, pt, sl, mask, out, scale, causal_offset, apd::PrefillShape<D>::kRows);
+    return launch_prefill_grid(kern, pp, kmap, vmap, apd::PrefillShape<D>::kThreads, prefill_smem_bytes(D), stream,
+                               "prefill_kernel launch");
+}
+
+// tcgen05 kernel with two 128-row Q tiles per CTA (D = 64, 128)
+template <int D>
+int launch_prefill_tc2(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                       const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
+                       float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
+    using T = apd::Tc2Shape<D>;
+    auto kern = apd::prefill_tc2_kernel<D>;
+    constexpr int kSlot = (D == 64) ? 1 : 2;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->prefill_tc2_attr_set[kSlot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(T::kSmemBytes));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc2_kernel)");
+            dev->prefill_tc2_attr_set[kSlot] = true;
+        }
+    }
+    CUtensorMap kmap, vmap;
+    int rc = encode_kv_map(&kmap, k, C.V.kst, D, 1);
+    if (!rc) rc = encode_kv_map(&vmap, v, C.V.vst, D, 1);
+    if (rc) return rc;
+    const apd::PrefillParams pp = prefill_params(C, q, pt, sl, mask, out, scale, causal_offset, 2 * T::kM);
+    return launch_prefill_grid(kern, pp, kmap, vmap, T::kThreads, T::kSmemBytes, stream, "prefill_tc2_kernel launch");
+}
+
+// tcgen05 kernel, one 128-row Q tile per CTA (D = 64, 128, 256)
+template <int D>
+int launch_prefill_tc(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                      const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
+                      float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
+    using T = apd::TcShape<D>;
+    auto kern = apd::prefill_tc_kernel<D>;
+    constexpr int kSlot = (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->prefill_tc_attr_set[kSlot]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(T::kSmemBytes));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill_tc_kernel)");
+            dev->prefill_tc_attr_set[kSlot] = true;
+        }
+    }
+    CUtensorMap kmap, vmap;
+    int rc = encode_kv_map(&kmap, k, C.V.kst, D, 1);
+    if (!rc) rc = encode_kv_map(&vmap, v, C.V.vst, D, 1);
+    if (rc) return rc;
+    const apd::PrefillParams pp = prefill_params(C, q, pt, sl, mask, out, scale, causal_offset, T::kM);
+    return launch_prefill_grid(kern, pp, kmap, vmap, T::kThreads, T::kSmemBytes, stream, "prefill_tc_kernel launch");
 }
 
 // ---------------------------------------------------------------- built-in scratch
@@ -833,15 +908,42 @@ int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache
 int apd_attn_paged_prefill(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
                            const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* mask,
                            const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream) {
+    return apd_attn_paged_prefill_ex(q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset,
+                                     stream, APD_PREFILL_AUTO);
+}
+
+int apd_attn_paged_prefill_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                              const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* mask,
+                              const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream,
+                              int kernel) {
+    if (kernel != APD_PREFILL_AUTO && kernel != APD_PREFILL_MMA_SYNC && kernel != APD_PREFILL_TCGEN05)
+        return APD_ERR_ARGUMENT;
     PrefillCheck C;
     int rc = prefill_validate(q, k_cache, v_cache, page_table, seq_lens, mask, out, causal_offset, &C);
     if (rc) return rc;
+    const int D = C.V.s.D;
+    if (kernel == APD_PREFILL_TCGEN05 && D == 32) return APD_ERR_HEAD_DIM;
+    const bool tc = kernel == APD_PREFILL_TCGEN05 || (kernel == APD_PREFILL_AUTO && kPrefillAutoTc && D != 32);
     if (C.V.s.B == 0) return APD_OK;
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    switch (C.V.s.D) {
+    // two Q tiles per CTA when a kv head has more than one tile of query rows
+    const bool two_tiles = static_cast<int64_t>(C.Lq) * C.V.s.g > 128;
+    if (tc && two_tiles && D == 64)
+        return launch_prefill_tc2<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+    if (tc && two_tiles && D == 128)
+        return launch_prefill_tc2<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+    if (tc) {
+        switch (D) {
+            case 64: return launch_prefill_tc<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+            case 128: return launch_prefill_tc<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+            case 256: return launch_prefill_tc<256>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
+            default: return APD_ERR_HEAD_DIM;
+        }
+    }
+    switch (D) {
         case 32: return launch_prefill<32>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
         case 64: return launch_prefill<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
         case 128: return launch_prefill<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);

@@ -252,6 +252,25 @@ int apd_attn_paged_prefill(const apd_tensor* q, const apd_tensor* k_cache, const
                            const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream);
 
 /*
+ * apd_attn_paged_prefill_ex -- apd_attn_paged_prefill with the kernel chosen by
+ * the caller (same result within the tolerance; for A/B measurement and tests).
+ *
+ *   kernel  APD_PREFILL_AUTO (0): what apd_attn_paged_prefill uses;
+ *           APD_PREFILL_MMA_SYNC (1): warp-level mma.sync tiles, every head dim;
+ *           APD_PREFILL_TCGEN05 (2): fifth-generation tensor cores (tcgen05.mma
+ *           with TMEM accumulators, 128 query rows x 128 keys per step, 64 keys
+ *           for D = 256); D = 64, 128, 256 only (D = 32 -> APD_ERR_HEAD_DIM).
+ *   Any other value -> APD_ERR_ARGUMENT, before any launch.
+ */
+#define APD_PREFILL_AUTO 0
+#define APD_PREFILL_MMA_SYNC 1
+#define APD_PREFILL_TCGEN05 2
+int apd_attn_paged_prefill_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                              const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* mask,
+                              const apd_tensor* out, float scale, int causal_offset, apd_stream_t stream,
+                              int kernel);
+
+/*
  * apd_attn_paged_decode_noalloc -- the same decode call for callers that cannot
  * allocate device memory.  The pages have no counterpart of this entry point.
  *

@@ -329,3 +329,37 @@ def test_gemv_validation():
     assert gemv_call(T([2, 64]), T([16, 64]), T([2, 16]), ws=None) == WS
     assert apd.lib().apd_gemv_workspace_size(9, 16, 64) == 0
     assert apd.gemv_workspace_size(8, 100000, 1536) % 256 == 0
+
+
+# ---------------------------------------------------------------- multi-query (prefill)
+def prefill_call(p, kernel=0, causal=-1, mask=None):
+    return apd.lib().apd_attn_paged_prefill_ex(
+        ctypes.byref(p["q"]), ctypes.byref(p["k"]), ctypes.byref(p["v"]), ctypes.byref(p["pt"]),
+        ctypes.byref(p["sl"]), ctypes.byref(mask) if mask is not None else None, ctypes.byref(p["out"]),
+        ctypes.c_float(0.1), causal, None, kernel)
+
+
+def prefill_problem(B=2, Lq=5, Hq=8, Hkv=2, D=64, P=32, NP=16, MP=4):
+    return dict(q=T([B, Lq, Hq, D]), k=T([NP, P, Hkv, D]), v=T([NP, P, Hkv, D]),
+                pt=T([B, MP], apd.DTYPE_INT32), sl=T([B], apd.DTYPE_INT32), out=T([B, Lq, Hq, D]))
+
+
+def test_prefill_kernel_choice_is_validated_before_any_launch():
+    for bad in (-1, 3, 99):
+        assert prefill_call(prefill_problem(), kernel=bad) == ARG
+    # the tensor-core kernel has no D = 32 variant; the mma.sync one has
+    assert prefill_call(prefill_problem(D=32), kernel=apd.PREFILL_KERNELS["tcgen05"]) == HEADDIM
+    for k in apd.PREFILL_KERNELS.values():
+        assert prefill_call(prefill_problem(D=32), kernel=k) in (OK, CUDA) or k == 2
+        assert prefill_call(prefill_problem(B=0), kernel=k) == OK
+        assert prefill_call(prefill_problem(Hq=6, Hkv=4), kernel=k) == GQA
+        assert prefill_call(prefill_problem(), kernel=k, causal=-2) == ARG
+    mask = T([2, 100], apd.DTYPE_UINT8)  # shorter than MP * P = 128
+    assert prefill_call(prefill_problem(), mask=mask) == SHAPE
+
+
+def test_prefill_binding_rejects_unknown_kernel_names():
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        apd.attn_paged_prefill(q, q, q, torch.zeros(1, 1, dtype=torch.int32), torch.zeros(1, dtype=torch.int32),
+                               0.1, kernel="wgmma")

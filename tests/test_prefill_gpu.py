@@ -17,7 +17,15 @@ from gpu_util import check_close
 pytestmark = pytest.mark.gpu
 
 
-def run(w, stream=None):
+@pytest.fixture(params=["mma_sync", "tcgen05"])
+def kernel(request):
+    """Every case runs on both kernels (the tensor-core one has no D = 32 variant)."""
+    return request.param
+
+
+def run(w, stream=None, kernel="auto"):
+    if kernel == "tcgen05" and w.q.shape[-1] == 32:
+        pytest.skip("no tcgen05 kernel for D = 32")
     heads_outer = w.k_cache.stride(1) < w.k_cache.stride(2)  # HND storage passed as a view
     def dev(t):
         if heads_outer:
@@ -27,7 +35,7 @@ def run(w, stream=None):
     mask = w.mask.cuda() if w.mask is not None else None
     out = torch.full_like(q, float("nan"))
     apd.attn_paged_prefill(q, dev(w.k_cache), dev(w.v_cache), w.page_table.cuda(), w.seq_lens.cuda(), w.scale,
-                           w.causal_offset, mask, out, stream=stream)
+                           w.causal_offset, mask, out, stream=stream, kernel=kernel)
     torch.cuda.synchronize()
     return out
 
@@ -42,39 +50,45 @@ def case(seed, D=64, Hq=8, Hkv=2, Lq=5, lens=(40, 9, 100), causal=-1, mask=None,
 @pytest.mark.parametrize("D", [32, 64, 128, 256])
 @pytest.mark.parametrize("causal", [-1, 60])
 @pytest.mark.parametrize("mask", [None, "2d", "3d"])
-def test_prefill_head_dims_causal_masks(D, causal, mask):
-    w = case(3, D=D, causal=causal, mask=mask, poison=True)
-    check_close(run(w), oracle.paged_prefill(w), f"D={D} causal={causal} mask={mask}")
+@pytest.mark.parametrize("Lq", [5, 45])
+def test_prefill_head_dims_causal_masks(D, causal, mask, Lq, kernel):
+    """Lq = 5 gives 20 rows per kv head (one 128-row tile), Lq = 45 gives 180 rows
+    (the two-tile tensor-core kernel for D = 64 and 128, second tile partly empty)."""
+    w = case(3, D=D, Lq=Lq, causal=causal, mask=mask, poison=True)
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), f"D={D} Lq={Lq} causal={causal} mask={mask}")
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (32, 8), (64, 8), (40, 2)])
 @pytest.mark.parametrize("Lq", [1, 16, 17, 70])
-def test_prefill_groups_and_query_counts(Hq, Hkv, Lq):
-    w = case(5, D=128, Hq=Hq, Hkv=Hkv, Lq=Lq, lens=(300, 77), causal=300 - Lq)
-    check_close(run(w), oracle.paged_prefill(w), f"{Hq}/{Hkv} Lq={Lq}")
+def test_prefill_groups_and_query_counts(D, Hq, Hkv, Lq, kernel):
+    """Rows per kv head from 1 to 1400: one tile, two tiles, several CTAs per head and a
+    ragged last CTA; g = 20 packs queries unevenly into the 128-row tiles."""
+    w = case(5, D=D, Hq=Hq, Hkv=Hkv, Lq=Lq, lens=(300, 77), causal=300 - Lq)
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), f"D={D} {Hq}/{Hkv} Lq={Lq}")
 
 
-def test_prefill_rows_that_see_nothing_are_zero():
+def test_prefill_rows_that_see_nothing_are_zero(kernel):
     w = case(6, D=64, Lq=4, lens=(50, 0, 20), mask="3d", mask_keep=0.5)
     w.mask[0, 2] = 0  # query 2 of sequence 0 sees no key
-    out = run(w)
+    out = run(w, kernel=kernel)
     ref = oracle.paged_prefill(w)
     check_close(out, ref, "zero rows")
     assert torch.all(out[1] == 0) and torch.all(out[0, 2] == 0)
 
 
-def test_prefill_causal_offset_zero():
+def test_prefill_causal_offset_zero(kernel):
     w = case(7, D=128, Lq=33, lens=(40, 100), causal=0, poison=True)
-    check_close(run(w), oracle.paged_prefill(w), "causal 0")
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), "causal 0")
 
 
 @pytest.mark.parametrize("P", [64, 128])
-def test_prefill_larger_pages_hnd(P):
+def test_prefill_larger_pages_hnd(P, kernel):
     w = case(8, D=128, Hq=16, Hkv=4, Lq=9, lens=(257, 31), causal=250, P=P, layout="HND", poison=True)
-    check_close(run(w), oracle.paged_prefill(w), f"P={P} HND")
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), f"P={P} HND")
 
 
-def test_prefill_side_stream_and_graph():
+def test_prefill_side_stream_and_graph(kernel):
     w = case(9, D=64, Hq=32, Hkv=8, Lq=12, lens=(200, 500), causal=480, mask="2d")
     q = w.q.cuda()
     k, v, pt, sl = w.k_cache.cuda(), w.v_cache.cuda(), w.page_table.cuda(), w.seq_lens.cuda()
@@ -84,9 +98,9 @@ def test_prefill_side_stream_and_graph():
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(s):
-        apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s)
+        apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s, kernel=kernel)
         with torch.cuda.graph(g, stream=s):
-            apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s)
+            apd.attn_paged_prefill(q, k, v, pt, sl, w.scale, w.causal_offset, mask, out, stream=s, kernel=kernel)
     torch.cuda.current_stream().wait_stream(s)
     out.fill_(float("nan"))
     g.replay()
@@ -94,11 +108,11 @@ def test_prefill_side_stream_and_graph():
     check_close(out, oracle.paged_prefill(w), "graph replay")
 
 
-def test_prefill_chunk_at_scale():
+def test_prefill_chunk_at_scale(kernel):
     """A 128-token chunk of 4 sequences of 1024 keys, 32/8 heads, D = 128, causal."""
     w = case(10, D=128, Hq=32, Hkv=8, Lq=128, lens=(1024, 1024, 1000, 640), causal=None or 0)
     w.causal_offset = 1024 - 128
-    check_close(run(w), oracle.paged_prefill(w), "chunk at scale")
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), "chunk at scale")
 
 
 def test_prefill_rejects_bad_arguments():
@@ -109,3 +123,21 @@ def test_prefill_rejects_bad_arguments():
         apd.attn_paged_prefill(q, *args, causal_offset=-5)
     with pytest.raises(apd.APDError):  # mask shorter than the page-table capacity
         apd.attn_paged_prefill(q, *args, mask=w.mask[:, :5].cuda())
+
+
+@pytest.mark.parametrize("Lq", [20, 50])
+@pytest.mark.parametrize("grow", [True, False])
+def test_prefill_running_max_moves_across_tiles(grow, Lq, kernel):
+    """Keys past position 300 scaled by 6 (exact in bf16): the logits of later tiles
+    exceed the earlier maximum by far more than 2^8 (grow) or fall far below it; the
+    tensor-core kernel rescales O in TMEM only in the first case."""
+    w = case(12, D=128, Hq=8, Hkv=2, Lq=Lq, lens=(900, 700), causal=-1)
+    P = w.k_cache.shape[1]
+    for b, L in enumerate(w.seq_lens.tolist()):
+        for t in range(300, L):
+            page = int(w.page_table[b, t // P])
+            if grow:
+                w.k_cache[page, t % P] *= 6
+            else:
+                w.k_cache[page, t % P] /= 8
+    check_close(run(w, kernel=kernel), oracle.paged_prefill(w), f"grow={grow}")
