@@ -74,6 +74,14 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -133,6 +141,64 @@ __device__ __forceinline__ float ex2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+// ---- packed fp32 pairs (sm_100a f32x2 arithmetic) and a 3-input maximum
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair on the FMA pipe, so that part of the exponentials leave the MUFU
+// unit (which bounds the softmax otherwise).  Cody-Waite style: x = j + f with j =
+// round(x) taken from the low mantissa bits of x + 1.5 * 2^23 and f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial whose coefficients come from exp2_poly.py (maximum
+// relative error 1.0e-4, far below bf16's 2^-9); j is added to the exponent field.
+// x is clamped to >= -125 so that the exponent field stays positive (2^-125 is
+// negligible next to the row's maximum weight, which is >= 2^-8 ... 2^8).
+__device__ __forceinline__ void exp2_fma2(uint64_t x2, float& p0, float& p1) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
+    const uint64_t jf = f2_add(t, f2_pack(-kRound, -kRound));
+    const uint64_t fr = f2_fma(jf, f2_pack(-1.f, -1.f), xc);
+    uint64_t q = f2_fma(fr, f2_pack(0.0550354384f, 0.0550354384f), f2_pack(0.242211014f, 0.242211014f));
+    q = f2_fma(q, fr, f2_pack(0.693277419f, 0.693277419f));
+    q = f2_fma(q, fr, f2_pack(1.f, 1.f));
+    float t0, t1, q0, q1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(q, q0, q1);
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Which pairs of each group of 8 take exp2_fma2 instead of MUFU ex2 (bit c of the mask
+// for pair c mod 8).  Measured on the 128-token chunk workload (D = 128): none 188.6 us,
+// 2/8 195.0 us, 3/8 199.5 us, 4/8 200.2 us -- the MUFU pipe is not what bounds the
+// softmax of the two-tile kernel, so the default sends every exponential to MUFU.
+#ifndef APD_EXP2_FMA_MASK
+#define APD_EXP2_FMA_MASK 0x00u
+#endif
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
@@ -899,9 +965,12 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
 #pragma unroll
-            for (int c = 8; c < N; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * cs;
+            for (int c = 8; c < N; c += 16) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    mx[e] = fmax3(mx[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e < N ? c + 8 + e : c + e]));
+            }
+            const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * cs;
             // ---- lazy rescale (S_t(j) full implies P_t(j-1) V_{j-1} has finished)
             float alpha = 1.f;
             bool grow = false;
@@ -926,23 +995,33 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
             }
             // ---- P = 2^(s * cs - reference) as bf16 pairs over the first half of S_t
             const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
-            float rs[8];
+            const uint64_t cs2 = f2_pack(cs, cs), nref2 = f2_pack(nref, nref);
+            uint64_t rs2[2] = {0ull, 0ull};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) rs[e] = 0.f;
+            for (int hh = 0; hh < N / 32; ++hh) {  // 32 keys -> 16 TMEM columns of bf16 pairs
+                uint32_t pw[16];
 #pragma unroll
-            for (int hh = 0; hh < N / 64; ++hh) {
-                uint32_t pw[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sr[64 * hh + 2 * c]), cs, nref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sr[64 * hh + 2 * c + 1]), cs, nref));
-                    rs[(2 * c) & 7] += p0;
-                    rs[(2 * c + 1) & 7] += p1;
+                for (int c = 0; c < 16; ++c) {
+                    const uint64_t x2 = f2_fma(
+                        f2_pack(__uint_as_float(sr[32 * hh + 2 * c]), __uint_as_float(sr[32 * hh + 2 * c + 1])), cs2,
+                        nref2);
+                    float p0, p1;
+                    if ((APD_EXP2_FMA_MASK >> (c & 7)) & 1u) {
+                        exp2_fma2(x2, p0, p1);
+                    } else {
+                        float x0, x1;
+                        f2_unpack(x2, x0, x1);
+                        p0 = ex2_approx(x0);
+                        p1 = ex2_approx(x1);
+                    }
+                    rs2[c & 1] = f2_add(rs2[c & 1], f2_pack(p0, p1));
                     pw[c] = pack_bf16x2(p0, p1);
                 }
-                tc_st32(tmem + t_lane + s_col + static_cast<uint32_t>(32 * hh), pw);
+                tc_st16(tmem + t_lane + s_col + static_cast<uint32_t>(16 * hh), pw);
             }
-            l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+            float ra, rb;
+            f2_unpack(f2_add(rs2[0], rs2[1]), ra, rb);
+            l = l * alpha + (ra + rb);
             // ---- last tile: V rows past the last visible key hold anything (NaN
             // included, or nothing loaded): tile 0's warpgroup zeroes them before
             // either tile multiplies them by a zero weight
@@ -971,7 +1050,9 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
         }
         __syncwarp();
         if (ok) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            // a row that saw no visible key outputs zeros (its emulated exponentials of
+            // -inf are tiny, not 0, so test the running maximum rather than l)
+            const float inv = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
             __nv_bfloat16* orow = p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
