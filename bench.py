@@ -47,6 +47,7 @@ GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m 
 PREFILL_METRIC = "paged multi-query (prefill chunk) attention achieved TFLOP/s and HBM GB/s"
 PREFILL_WORKLOADS = ["prefill_llama8b_chunk"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
+PREFILL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_tc2_kernel_traffic.json")
 
 
 def parse_args(argv=None):
@@ -227,25 +228,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- measurement legs
-def kernel_source_sha() -> str:
-    """Hash of the device code (the kernel headers); the host-side API file is not included."""
+DECODE_KERNEL_SOURCES = ("apd_kernels.cuh", "apd_ptx.cuh")  # the split and combine kernels' device code
+
+
+def kernel_source_sha(sources=DECODE_KERNEL_SOURCES) -> str:
+    """Hash of the decode kernels' device code (the headers they are compiled from); the
+    host-side API file and the other kernels' headers are not included."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
-        if name.endswith(".cuh"):
-            with open(os.path.join(CSRC, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in sorted(sources):
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(workload: str):
-    """dram read+write bytes per split-kernel launch from the committed ncu capture,
-    or None when the capture is missing, for another workload, or the kernel changed since."""
+PREFILL_KERNEL_SOURCES = ("apd_kernels.cuh", "apd_prefill.cuh", "apd_prefill_tc.cuh", "apd_ptx.cuh")
+
+
+def committed_traffic(workload: str, path=None, sources=DECODE_KERNEL_SOURCES):
+    """dram read+write bytes per launch of the dominant kernel from a committed ncu capture
+    (default: the decode split kernel), or None when the capture is missing, for another
+    workload, or the kernel's device code changed since."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(path or TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_sha") != kernel_source_sha() or t.get("workload") != workload:
+    if t.get("kernel_source_sha") != kernel_source_sha(sources) or t.get("workload") != workload:
         return None
     return t.get("dram_bytes_per_launch")
 
@@ -702,12 +710,13 @@ def peak_tflops():
 
 
 def prefill_kernel_name(choice):
-    """The kernel the prefill workload (D = 128) runs for a --prefill-kernel choice."""
+    """The kernel the prefill workload (D = 128, 512 query rows per kv head) runs for a
+    --prefill-kernel choice."""
     import decode_attention_paged_split_b200 as apd
 
     if choice == "auto":
         choice = apd.prefill_auto_kernel(128)
-    return "prefill_tc_kernel" if choice == "tcgen05" else "prefill_kernel"
+    return "prefill_tc2_kernel" if choice == "tcgen05" else "prefill_kernel"
 
 
 def run_prefill(a):
@@ -799,7 +808,9 @@ def run_prefill(a):
                        "l2": "two cache instances used in turn, each larger than L2",
                        "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                         "traffic": None, "peak_source": tsrc, "kernel": prefill_kernel_name(a.prefill_kernel),
+                         "traffic": (committed_traffic(w0.name, PREFILL_TRAFFIC_FILE, PREFILL_KERNEL_SOURCES)
+                                     if prefill_kernel_name(a.prefill_kernel) == "prefill_tc2_kernel" else None),
+                         "peak_source": tsrc, "kernel": prefill_kernel_name(a.prefill_kernel),
                          "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hpeak},
             "cpu_baseline": cpu, "e2e": None, "gpu_launches": a.steps, "clocks": clock_info,
         }
