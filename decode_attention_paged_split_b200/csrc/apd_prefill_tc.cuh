@@ -527,9 +527,12 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx[e] = __uint_as_float(sr[e]);
 #pragma unroll
-            for (int c = 8; c < NH; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c]));
-            const float mr = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            for (int c = 8; c < NH; c += 16) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    mx[e] = fmax3(mx[e], __uint_as_float(sr[c + e]), __uint_as_float(sr[c + 8 + e < NH ? c + 8 + e : c + e]));
+            }
+            const float mr = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
             // ---- the row's maximum over both halves (exchange phase j of this quadrant)
             xmax[((j & 1) * 2 + h) * M + r] = mr;
             mbar_arrive(xbar);
@@ -550,18 +553,21 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
             // ---- P = 2^(s * cs - reference) into registers while P_{j-1} V_{j-1} runs
             const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
             uint32_t pw[NH / 2];
-            float rs[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) rs[e] = 0.f;
+            const uint64_t cs2 = f2_pack(cs, cs), nref2 = f2_pack(nref, nref);
+            uint64_t rs2[2] = {0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < NH / 2; ++c) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), cs, nref));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), cs, nref));
-                rs[(2 * c) & 7] += p0;
-                rs[(2 * c + 1) & 7] += p1;
+                const uint64_t x2 =
+                    f2_fma(f2_pack(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), cs2, nref2);
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                rs2[c & 1] = f2_add(rs2[c & 1], f2_pack(p0, p1));
                 pw[c] = pack_bf16x2(p0, p1);
             }
-            l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
+            float ra, rb;
+            f2_unpack(f2_add(rs2[0], rs2[1]), ra, rb);
+            l = l * alpha + (ra + rb);
             // ---- O and the P buffer are free once P_{j-1} V_{j-1} has completed
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, tc_wait(bar(kPVDone), static_cast<uint32_t>(j - 1) & 1u, abort_flag,
