@@ -286,6 +286,36 @@ def time_steps(insts, stream, steps, split_events=False):
 GRAPH_CHUNK = 100
 
 
+def graph_split_times(insts, stream, replays):
+    """Split-kernel duration inside CUDA-graph replays: a graph of GRAPH_CHUNK calls (rotating
+    over the instances) with an external event recorded before each call and the call's
+    split_done_event right after its split kernel (both become event-record nodes), replayed
+    `replays` times.  The event between the kernels turns off the programmatic overlap of
+    those two launches, so this is the kernel's own start-to-end time.  Returns the mean in s."""
+    ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+          for _ in range(GRAPH_CHUNK)]
+    for b, m in ev:  # create the events before capture
+        b.record(stream)
+        m.record(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i, (b, m) in enumerate(ev):
+                b.record(stream)
+                insts[i % len(insts)].call(stream, split_done_event=m)
+    g.replay()
+    torch.cuda.synchronize()
+    tot, n = 0.0, 0
+    for _ in range(replays):
+        g.replay()
+        torch.cuda.synchronize()
+        tot += sum(b.elapsed_time(m) for b, m in ev) / 1e3
+        n += len(ev)
+    del g
+    return tot / n
+
+
 class GraphSteps:
     """CUDA graphs of consecutive calls (rotating over the instances): `steps` calls in
     all, as steps // GRAPH_CHUNK replays of a GRAPH_CHUNK-call graph plus one graph of
@@ -498,11 +528,19 @@ def run_ours(a):
     eager_el, _ = time_steps(insts, stream, a.steps)
     eager_max = max_over_ranks(eager_el, dist, device)
 
-    # split-kernel duration: the same steps with an event between the two kernels
+    # split-kernel duration: events around each split kernel inside graph replays (the
+    # launch configuration of the timed region); eager event pairs, which also count the
+    # launch latency of every kernel, are kept for reference
     barrier(dist, device)
     torch.cuda.synchronize(device)
-    _, split_s = time_steps(insts, stream, a.steps, split_events=True)
+    _, split_eager_s = time_steps(insts, stream, a.steps, split_events=True)
     torch.cuda.synchronize(device)
+    split_eager_s = max_over_ranks(split_eager_s, dist, device)
+    try:
+        split_s = graph_split_times(insts, stream, replays=max(1, min(20, a.steps // GRAPH_CHUNK)))
+    except RuntimeError as err:  # event-record nodes unavailable: fall back to the eager pairs
+        print(f"graph split timing unavailable ({err}); using eager event pairs", file=sys.stderr)
+        split_s = split_eager_s
     split_s = max_over_ranks(split_s, dist, device)
 
     # end to end through host buffers
@@ -538,6 +576,9 @@ def run_ours(a):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "kernel": "split_kernel", "kernel_us": split_s * 1e6,
+                         "kernel_us_eager_events": split_eager_s * 1e6,
+                         "kernel_timing": "CUDA events recorded around each split kernel inside replays of a "
+                                          f"{GRAPH_CHUNK}-call graph (event-record nodes)",
                          "call_frac_of_peak": value / world / peak},
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -709,6 +750,39 @@ def peak_tflops():
         return 1590.0, "fallback"
 
 
+class PrefillInst:
+    """One prefill-chunk instance on the device.  q, page_table and seq_lens are views into
+    one packed device buffer (with a pinned host twin) so the end-to-end leg moves the
+    step's inputs in one copy; the KV cache stays resident."""
+
+    def __init__(self, w, device, kernel):
+        import decode_attention_paged_split_b200 as apd
+
+        self.apd, self.w, self.kernel = apd, w, kernel
+        qb, ptb, slb = w.q.numel() * 2, w.page_table.numel() * 4, w.seq_lens.numel() * 4
+        off_pt = (qb + 15) // 16 * 16
+        off_sl = (off_pt + ptb + 15) // 16 * 16
+        self.packed_bytes = off_sl + slb
+
+        def views(buf):
+            return (buf[:qb].view(torch.bfloat16).view(w.q.shape),
+                    buf[off_pt:off_pt + ptb].view(torch.int32).view(w.page_table.shape),
+                    buf[off_sl:off_sl + slb].view(torch.int32))
+
+        self.host_packed = torch.empty(self.packed_bytes, dtype=torch.uint8, pin_memory=True)
+        for dst, src in zip(views(self.host_packed), (w.q, w.page_table, w.seq_lens)):
+            dst.copy_(src)
+        self.dev_packed = self.host_packed.to(device)
+        self.q, self.pt, self.sl = views(self.dev_packed)
+        self.k, self.v = w.k_cache.contiguous().to(device), w.v_cache.contiguous().to(device)
+        self.out = torch.empty_like(self.q)
+        self.host_out = torch.empty(self.out.shape, dtype=self.out.dtype, pin_memory=True)
+
+    def call(self, stream):
+        self.apd.attn_paged_prefill(self.q, self.k, self.v, self.pt, self.sl, self.w.scale, self.w.causal_offset,
+                                    None, self.out, stream=stream, kernel=self.kernel)
+
+
 def prefill_kernel_name(choice):
     """The kernel the prefill workload (D = 128, 512 query rows per kv head) runs for a
     --prefill-kernel choice."""
@@ -732,17 +806,13 @@ def run_prefill(a):
     import decode_attention_paged_split_b200 as apd
 
     ws = [workloads.prefill_llama8b_chunk(seed=8 + 1000003 * rank + i) for i in range(2)]
-    dev = [dict(q=w.q.to(device), k=w.k_cache.contiguous().to(device), v=w.v_cache.contiguous().to(device),
-                pt=w.page_table.to(device), sl=w.seq_lens.to(device), out=torch.empty_like(w.q, device=device))
-           for w in ws]
+    insts = [PrefillInst(w, device, a.prefill_kernel) for w in ws]
     w0 = ws[0]
     per_bytes, per_flops = w0.algorithmic_bytes(), w0.algorithmic_flops()
     stream = torch.cuda.Stream(device)
 
     def call(i):
-        d, w = dev[i % 2], ws[i % 2]
-        apd.attn_paged_prefill(d["q"], d["k"], d["v"], d["pt"], d["sl"], w.scale, w.causal_offset, None, d["out"],
-                               stream=stream, kernel=a.prefill_kernel)
+        insts[i % 2].call(stream)
 
     for i in range(a.warmup):
         call(i)
@@ -781,6 +851,21 @@ def run_prefill(a):
     bytes_all = sum_over_ranks(float(per_bytes * a.steps), dist, device)
     flops_all = sum_over_ranks(float(per_flops * a.steps), dist, device)
 
+    # end to end through host buffers (PCIe-bound: the chunk's q and out are 16.8 MB each)
+    e2e = None
+    if not a.no_e2e:
+        e2e_n = max(4, min(a.steps, 200))
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        e2e_el, h2d, d2h = e2e_steps(insts, stream, e2e_n)
+        e2e_max = max_over_ranks(e2e_el, dist, device)
+        e2e_flops = sum_over_ranks(float(per_flops * e2e_n), dist, device)
+        e2e = {"value": e2e_flops / e2e_max / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_max / e2e_n * 1e3, "steps": e2e_n,
+               "how": "per step, eager through the public Python API: one pinned-host->device copy of the packed "
+                      "q|page_table|seq_lens, the call, one device->pinned-host copy of out; copies on two copy "
+                      "streams overlap the neighbouring steps' compute"}
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         import oracle
@@ -812,7 +897,7 @@ def run_prefill(a):
                                      if prefill_kernel_name(a.prefill_kernel) == "prefill_tc2_kernel" else None),
                          "peak_source": tsrc, "kernel": prefill_kernel_name(a.prefill_kernel),
                          "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hpeak},
-            "cpu_baseline": cpu, "e2e": None, "gpu_launches": a.steps, "clocks": clock_info,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": a.steps, "clocks": clock_info,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

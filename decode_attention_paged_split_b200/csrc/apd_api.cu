@@ -437,7 +437,13 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     }
     cudaError_t e = cudaSuccess;
     if (opts && opts->split_done_event) {
-        e = cudaEventRecord(static_cast<cudaEvent_t>(opts->split_done_event), stream);
+        // while the stream is being captured into a CUDA graph the record becomes an
+        // event-record node (external), so the event still times the replayed kernel
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        e = cudaStreamIsCapturing(stream, &cap);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+        e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(opts->split_done_event), stream,
+                                     cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(split_done_event)");
     }
 

@@ -196,6 +196,13 @@ __device__ __forceinline__ void exp2_fma2(uint64_t x2, float& p0, float& p1) {
 // for pair c mod 8).  Measured on the 128-token chunk workload (D = 128): none 188.6 us,
 // 2/8 195.0 us, 3/8 199.5 us, 4/8 200.2 us -- the MUFU pipe is not what bounds the
 // softmax of the two-tile kernel, so the default sends every exponential to MUFU.
+// Parts in which a softmax warpgroup of the two-tile kernel hands P over to the MMA
+// issuer (the first parts' P V runs while the later parts' exponentials are computed).
+// Chunk workload (D = 128): 1 part 185.2 us, 2 parts 183.6 us, 4 parts 181.7 us.
+#ifndef APD_PREFILL_P_PARTS
+#define APD_PREFILL_P_PARTS 4
+#endif
+
 #ifndef APD_EXP2_FMA_MASK
 #define APD_EXP2_FMA_MASK 0x00u
 #endif
@@ -725,8 +732,11 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
     constexpr uint32_t kIdescQK = bf16_idesc(M, N, false);
     constexpr uint32_t kIdescPV = bf16_idesc(M, D, true);
     // mbarrier indices
+    // P full per (Q tile t, key part h): index kParts t + h (P is handed over N / kParts keys at a time)
+    constexpr int kParts = APD_PREFILL_P_PARTS;
+    static_assert(kParts == 1 || kParts == 2 || kParts == 4, "P hand-over parts");
     constexpr int kQFull = 0, kFull = 1, kEmpty = 1 + NS, kSFull = 1 + 2 * NS, kPFull = 3 + 2 * NS;
-    constexpr int kPVDone = 5 + 2 * NS, kDrain = 7 + 2 * NS, kBars = 8 + 2 * NS;
+    constexpr int kPVDone = kPFull + 2 * kParts, kDrain = kPVDone + 2, kBars = kDrain + 1;
     static_assert(8 * kBars + 8 <= T::kHeaderBytes, "header");
 
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -755,7 +765,8 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(kSFull + t), 1);
-            mbar_init(bar(kPFull + t), 128);
+#pragma unroll
+            for (int h = 0; h < kParts; ++h) mbar_init(bar(kPFull + kParts * t + h), 128);
             mbar_init(bar(kPVDone + t), 1);
         }
         mbar_init(bar(kDrain), 1);
@@ -862,15 +873,28 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                 }
                 tc_commit(bar(kSFull + t));
             };
-            // O_t += P_t V_j, P_t from TMEM (8 columns per 16 keys)
-            auto pv = [&](int t, int j) {
+            // O_t += P_t V_j over part h of the keys, P_t from TMEM (8 columns per 16 keys)
+            auto pv = [&](int t, int j, int h) {
                 const uint32_t vb = ring + static_cast<uint32_t>((2 * j + 1) % NS) * T::kSlotBytes;
 #pragma unroll
-                for (int k = 0; k < N / 16; ++k)
+                for (int kk = 0; kk < N / 16 / kParts; ++kk) {
+                    const int k = (N / 16 / kParts) * h + kk;
                     tc_mma_bf16_ts(tmem + T::kColO + static_cast<uint32_t>(D * t), tmem + T::kColS + 128u * t + 8u * k,
                                    sw128_desc(vb + static_cast<uint32_t>(k) * 2048u, N * 128, 1024), kIdescPV,
                                    (j > 0 || k > 0) ? 1u : 0u);
-                tc_commit(bar(kPVDone + t));
+                }
+                if (h == kParts - 1) tc_commit(bar(kPVDone + t));
+            };
+            // the parts of P_t(j) V_j, each as soon as the softmax warpgroup hands it over
+            auto pv_halves = [&](int t, int j) -> bool {
+#pragma unroll
+                for (int h = 0; h < kParts; ++h) {
+                    if (!tc_wait(bar(kPFull + kParts * t + h), static_cast<uint32_t>(j) & 1u, abort_flag, p.flags))
+                        return false;
+                    tc_fence_after();
+                    pv(t, j, h);
+                }
+                return true;
             };
             ok = tc_wait(bar(kQFull), 0, abort_flag, p.flags) && wait_load(0);
             if (ok) {
@@ -881,20 +905,16 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                 issued = true;
             }
             for (int j = 0; ok && j < ntiles; ++j) {
-                ok = tc_wait(bar(kPFull + 0), static_cast<uint32_t>(j) & 1u, abort_flag, p.flags) && wait_load(2 * j + 1);
+                ok = wait_load(2 * j + 1) && pv_halves(0, j);
                 if (!ok) break;
-                tc_fence_after();
-                pv(0, j);
                 if (j + 1 < ntiles) {
                     ok = wait_load(2 * j + 2);
                     if (!ok) break;
                     tc_fence_after();
                     qk(0, j + 1);
                 }
-                ok = tc_wait(bar(kPFull + 1), static_cast<uint32_t>(j) & 1u, abort_flag, p.flags);
+                ok = pv_halves(1, j);
                 if (!ok) break;
-                tc_fence_after();
-                pv(1, j);
                 tc_commit(bar(kEmpty + (2 * j + 1) % NS));  // V_j read by both tiles
                 if (j + 1 < ntiles) {
                     qk(1, j + 1);
@@ -999,7 +1019,24 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                     tc_st32(ta, o);
                 }
             }
-            // ---- P = 2^(s * cs - reference) as bf16 pairs over the first half of S_t
+            // ---- last tile: V rows past the last visible key hold anything (NaN
+            // included, or nothing loaded): tile 0's warpgroup zeroes them before
+            // either tile multiplies them by a zero weight
+            if (t == 0 && j == ntiles - 1 && j * N + N > kv_end) {
+                const int nv = 2 * j + 1;
+                ok = __all_sync(0xffffffffu, tc_wait(bar(kFull + nv % NS), static_cast<uint32_t>(nv / NS) & 1u,
+                                                     abort_flag, p.flags));
+                if (!ok) break;
+                const int v0 = kv_end - j * N;
+                const uint32_t vb = ring + static_cast<uint32_t>(nv % NS) * T::kSlotBytes;
+                for (int idx = wt; idx < (N - v0) * kBlk * 8; idx += 128) {
+                    const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
+                    st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
+                }
+                fence_proxy_async_smem();  // before the first half of P is handed over
+            }
+            // ---- P = 2^(s * cs - reference) as bf16 pairs over the first half of S_t,
+            // handed to the MMA issuer N / kParts keys at a time
             const float nref = (m_used == -INFINITY) ? 0.f : -m_used;
             const uint64_t cs2 = f2_pack(cs, cs), nref2 = f2_pack(nref, nref);
             uint64_t rs2[2] = {0ull, 0ull};
@@ -1024,29 +1061,17 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                     pw[c] = pack_bf16x2(p0, p1);
                 }
                 tc_st16(tmem + t_lane + s_col + static_cast<uint32_t>(16 * hh), pw);
+                constexpr int kPer = (N / 32) / kParts;  // 32-key chunks per part
+                if (hh % kPer == kPer - 1) {
+                    tc_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(kPFull + kParts * t + hh / kPer));
+                }
             }
             float ra, rb;
             f2_unpack(f2_add(rs2[0], rs2[1]), ra, rb);
             l = l * alpha + (ra + rb);
-            // ---- last tile: V rows past the last visible key hold anything (NaN
-            // included, or nothing loaded): tile 0's warpgroup zeroes them before
-            // either tile multiplies them by a zero weight
-            if (t == 0 && j == ntiles - 1 && j * N + N > kv_end) {
-                const int nv = 2 * j + 1;
-                ok = __all_sync(0xffffffffu, tc_wait(bar(kFull + nv % NS), static_cast<uint32_t>(nv / NS) & 1u,
-                                                     abort_flag, p.flags));
-                if (!ok) break;
-                const int v0 = kv_end - j * N;
-                const uint32_t vb = ring + static_cast<uint32_t>(nv % NS) * T::kSlotBytes;
-                for (int idx = wt; idx < (N - v0) * kBlk * 8; idx += 128) {
-                    const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
-                    st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
-                }
-                fence_proxy_async_smem();
-            }
-            tc_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(kPFull + t));
+
         }
         // ---- epilogue: out = O_t / l (zeros for a row that saw no key)
         if (ok && ntiles > 0) {

@@ -179,7 +179,10 @@ int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const 
  *                     the combine kernel; lets a caller time the split kernel
  *                     alone with events.  Recording it between the kernels
  *                     also turns off the programmatic (PDL) overlap of the
- *                     combine kernel's launch for that call.
+ *                     combine kernel's launch for that call.  While `stream`
+ *                     is being captured into a CUDA graph the event is recorded
+ *                     as an external event-record node, so it also times the
+ *                     kernel in every replay of the graph.
  *   disable_pdl       nonzero: launch the combine kernel without programmatic
  *                     dependent launch.
  */

@@ -169,6 +169,35 @@ def test_cuda_graph_capture_and_replay(S):
     check_close(out, oracle.paged_decode(w), "graph replay with new q")
 
 
+def test_split_done_event_inside_a_graph_times_the_split_kernel():
+    """Recorded while the stream is captured, the split-done event becomes an event-record
+    node: each replay stamps it between the two kernels, and the result is unchanged."""
+    w = small(54, B=4, Hq=32, Hkv=8, D=128, lens=(3000, 1, 777, 4096), pool=300)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(4, 32, 8, 128, 0)
+    eager = dp.run(0, workspace=ws).clone()
+    b = torch.cuda.Event(enable_timing=True, external=True)
+    m = torch.cuda.Event(enable_timing=True, external=True)
+    e = torch.cuda.Event(enable_timing=True, external=True)
+    s = torch.cuda.Stream()
+    for ev in (b, m, e):
+        ev.record(s)
+    s.synchronize()
+    out = torch.full_like(dp.out, float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            b.record(s)
+            apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, out, w.scale, 0, ws, stream=s,
+                                  split_done_event=m)
+            e.record(s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)
+    split_ms, call_ms = b.elapsed_time(m), b.elapsed_time(e)
+    assert 0 < split_ms <= call_ms, (split_ms, call_ms)
+
+
 def test_inputs_written_by_the_preceding_kernel_are_seen():
     """The split kernel may start launching before the previous kernel in the stream
     ends (programmatic dependent launch); it must still read q, page_table and
