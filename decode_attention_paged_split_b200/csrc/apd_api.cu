@@ -481,7 +481,23 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
 constexpr int kGemvWarps = 4;
 constexpr int kGemvStages = 4;
 
-size_t gemv_smem_bytes() { return 8ull * kGemvWarps * kGemvStages + 1024 + static_cast<size_t>(kGemvWarps) * kGemvStages * apd::kGemvStageBytes; }
+// Shared memory of the GEMV kernel: mbarriers, the staged x rows (xs) with a zero chunk,
+// alignment, the ring.  x is staged once per CTA when it fits with at least 2 stages.
+int gemv_x_pitch(int K) { return 16 * ((K / 8) | 1); }
+size_t gemv_smem_bytes(int M, int K, int stages, bool xs) {
+    const size_t x = xs ? static_cast<size_t>(M) * gemv_x_pitch(K) + 16 + 16 : 0;
+    return 8ull * kGemvWarps * stages + x + 1024 +
+           static_cast<size_t>(kGemvWarps) * stages * (xs ? apd::kGemvWBytes : apd::kGemvStageBytes);
+}
+// x is staged once per CTA for long weight streams (W >= 64 MB) when it is at most 32 KB
+// (every CTA copies it from L2) and the full ring still fits.  Graph-timed on the
+// AstrAI-1B shapes: lm_head (100000 x 1536) 59.3 -> 56.7 us at M = 1, 60.1 -> 58.0 at
+// M = 3, 59.7 -> 59.1 at M = 8; the 21 MB layers, which are latency-bound, lose up to
+// 3 us to the copy that precedes their first MMA (gate_up M = 8: 8.5 -> 11.8 us).
+bool gemv_stage_x(int M, int N, int K) {
+    return static_cast<int64_t>(N) * K * 2 >= (64ll << 20) && static_cast<int64_t>(M) * gemv_x_pitch(K) <= 32768 &&
+           gemv_smem_bytes(M, K, kGemvStages, true) <= 232448;
+}
 
 int64_t gemv_workers(int sm_count, int64_t units) {
     int64_t w = static_cast<int64_t>(sm_count) * kGemvWarps;
@@ -983,13 +999,16 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     if (rc) return rc;
     const int64_t workers = gemv_workers(dev->sm_count, g.units);
     if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
-    auto kern = apd::gemv_kernel<kGemvStages>;
+    const bool xs = gemv_stage_x(g.M, g.N, g.K);
+    auto kern = xs ? apd::gemv_kernel<kGemvStages, true> : apd::gemv_kernel<kGemvStages, false>;
+    const size_t smem = gemv_smem_bytes(g.M, g.K, kGemvStages, xs);
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!dev->gemv_attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(gemv_smem_bytes()));
-            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv_kernel)");
+        if (!dev->gemv_attr_set) {  // the largest either variant uses, for both
+            for (auto k : {apd::gemv_kernel<kGemvStages, true>, apd::gemv_kernel<kGemvStages, false>}) {
+                cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemv_kernel)");
+            }
             dev->gemv_attr_set = true;
         }
     }
@@ -998,6 +1017,9 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     if (!rc) rc = encode_gemv_map(&xmap, x, g.ldx, apd::kGemvXRows);
     if (rc) return rc;
     apd::GemvParams gp;
+    gp.x = static_cast<const __nv_bfloat16*>(x->data);
+    gp.ldx = g.ldx;
+    gp.x_pitch = gemv_x_pitch(g.K);
     gp.y = static_cast<__nv_bfloat16*>(y->data);
     gp.y_sm = g.ysm;
     gp.y_sn = g.ysn;
@@ -1017,7 +1039,7 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((workers + kGemvWarps - 1) / kGemvWarps));
     cfg.blockDim = dim3(32 * kGemvWarps);
-    cfg.dynamicSmemBytes = gemv_smem_bytes();
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = pdl_attr;
     cfg.numAttrs = 1;

@@ -16,8 +16,13 @@
 //    the end of each warp's share cost more than the second launch.
 //  * Each warp runs its own ring of STAGES stages.  Lane 0 issues TMA tiled loads
 //    (cp.async.bulk.tensor, 128-byte swizzle, bounds-filled with zeros past N and
-//    K) of the W unit as 4 boxes of [16 rows][64] and of the matching x columns as
-//    4 boxes of [8 rows][64] (rows >= M are zero); completion by mbarrier bytes.
+//    K) of the W unit as 4 boxes of [16 rows][64]; completion by mbarrier bytes.
+//  * x: when its M rows fit in shared memory beside the ring (XS), the CTA copies
+//    them once, with rows padded to an odd number of 16-byte chunks so the 8-row
+//    ldmatrix reads hit distinct banks; lanes whose x row is >= M or whose column
+//    is >= K read a 16-byte zero chunk instead.  Otherwise each stage also loads
+//    the unit's x columns as 4 TMA boxes of [8 rows][64] (rows >= M zero-filled),
+//    which costs the TMA engine half again the W bytes.
 //  * The product runs on tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate)
 //    with 16 W rows on M and the <= 8 rows of x on N.  At M = 8 a scalar FMA loop
 //    would need about as many issue slots as the SMs have at full HBM bandwidth;
@@ -41,6 +46,9 @@ constexpr uint32_t kGemvXBytes = kGemvXRows * kGemvCols * 2;  // 4 KB
 constexpr uint32_t kGemvStageBytes = kGemvWBytes + kGemvXBytes;
 
 struct GemvParams {
+    const __nv_bfloat16* x;  // [M, K], row stride ldx (used when x is staged once per CTA)
+    int64_t ldx;
+    int32_t x_pitch;         // bytes per staged x row: 16 * (K / 8 | 1)
     __nv_bfloat16* y;
     int64_t y_sm, y_sn;  // element strides of y [M, N]
     float* part;         // [2 * workers][16][8] fp32 partials
@@ -67,33 +75,36 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
-template <int STAGES>
+template <int STAGES, bool XS>
 __global__ void __launch_bounds__(32 * 8, 1)
     gemv_kernel(const __grid_constant__ GemvParams p, const __grid_constant__ CUtensorMap wmap,
                 const __grid_constant__ CUtensorMap xmap) {
+    constexpr uint32_t kStage = XS ? kGemvWBytes : kGemvStageBytes;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int w = blockIdx.x * p.warps + warp;
 
+    // shared memory: mbarriers | x rows (XS) | 16-byte zero chunk (XS) | stage ring
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    const uint32_t ring = (smem_u32(bars + p.warps * STAGES) + 1023u) & ~1023u;
+    const uint32_t xs = (smem_u32(bars + p.warps * STAGES) + 15u) & ~15u;
+    const uint32_t xz = xs + (XS ? static_cast<uint32_t>(p.M * p.x_pitch) : 0u);
+    const uint32_t ring = ((XS ? xz + 16u : xs) + 1023u) & ~1023u;
     if (threadIdx.x == 0) {
         prefetch_tensormap(&wmap);
-        prefetch_tensormap(&xmap);
+        if (!XS) prefetch_tensormap(&xmap);
     }
     // x and W may be written by the previous kernel in the stream (PDL launch).
     pdl_wait_prior_grid();
     pdl_launch_dependents();
-    if (w >= p.num_workers) return;
 
     const int64_t total = static_cast<int64_t>(p.mtiles) * p.ktiles;
-    const int64_t ws = static_cast<int64_t>((static_cast<uint64_t>(w) * total) / p.num_workers);
-    const int64_t we = static_cast<int64_t>((static_cast<uint64_t>(w + 1) * total) / p.num_workers);
-    if (ws >= we) return;
+    const int64_t ws = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w) * total) / p.num_workers) : 0;
+    const int64_t we = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w + 1) * total) / p.num_workers) : 0;
+    const bool active = ws < we;
 
     const uint32_t bar0 = smem_u32(bars + warp * STAGES);
-    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * kGemvStageBytes;
+    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * kStage;
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -110,19 +121,35 @@ __global__ void __launch_bounds__(32 * 8, 1)
         const int kt = static_cast<int>(pi - static_cast<int64_t>(mt) * p.ktiles);
         if (lane == 0) {
             const uint32_t bar = bar0 + 8 * stage;
-            const uint32_t sbase = wring + static_cast<uint32_t>(stage) * kGemvStageBytes;
-            mbar_arrive_expect_tx(bar, kGemvStageBytes);
+            const uint32_t sbase = wring + static_cast<uint32_t>(stage) * kStage;
+            mbar_arrive_expect_tx(bar, kStage);
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb) {
                 const int k0 = kt * kGemvCols + 64 * kb;
                 tma_load_2d(sbase + kb * kGemvRows * 128, &wmap, bar, k0, mt * kGemvRows, pol_stream);
-                tma_load_2d(sbase + kGemvWBytes + kb * kGemvXRows * 128, &xmap, bar, k0, 0, pol_keep);
+                if (!XS) tma_load_2d(sbase + kGemvWBytes + kb * kGemvXRows * 128, &xmap, bar, k0, 0, pol_keep);
             }
         }
         ++pi;
     };
+    // the first W loads go out before the CTA copies x, so the copy overlaps them
+    if (active) {
 #pragma unroll
-    for (int s = 0; s < STAGES; ++s) issue_next(s);
+        for (int s = 0; s < STAGES; ++s) issue_next(s);
+    }
+    if constexpr (XS) {
+        const int kch = p.K / 8;
+        for (int idx = threadIdx.x; idx < p.M * kch; idx += blockDim.x) {
+            const int r = idx / kch, c = idx - r * kch;
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + r * p.ldx) + c);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xs + static_cast<uint32_t>(r * p.x_pitch + 16 * c)),
+                         "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                         : "memory");
+        }
+        if (threadIdx.x == 0) st_shared_zero16(xz);
+        __syncthreads();
+    }
+    if (!active) return;
 
     const int tq = lane & 3, gq = lane >> 2, mi = lane >> 3;
     float acc[2][4];  // two accumulators per k-step parity, summed at the end
@@ -152,13 +179,20 @@ __global__ void __launch_bounds__(32 * 8, 1)
             }
             return;
         }
-        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * kGemvStageBytes;
+        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * kStage;
         const uint32_t xbase = sbase + kGemvWBytes;
         // 16 k-steps of 16 columns: A = W rows (ldmatrix.x4), B = x rows (ldmatrix.x4 covers 2 k-steps)
 #pragma unroll
         for (int ks2 = 0; ks2 < kGemvCols / 32; ++ks2) {
             uint32_t b[4];
-            ldsm_x4(xbase + gemv_off(lane & 7, 4 * ks2 + mi, kGemvXRows), b[0], b[1], b[2], b[3]);
+            if constexpr (XS) {
+                const int xr = lane & 7;
+                const int kel = kt * kGemvCols + 8 * (4 * ks2 + mi);  // first column of this lane's chunk
+                ldsm_x4((xr < p.M && kel < p.K) ? xs + static_cast<uint32_t>(xr * p.x_pitch + 2 * kel) : xz, b[0], b[1],
+                        b[2], b[3]);
+            } else {
+                ldsm_x4(xbase + gemv_off(lane & 7, 4 * ks2 + mi, kGemvXRows), b[0], b[1], b[2], b[3]);
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int ks = 2 * ks2 + h;

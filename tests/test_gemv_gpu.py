@@ -26,7 +26,7 @@ def check(y, x, w, what=""):
 
 
 @pytest.mark.parametrize("M", range(1, 9))
-@pytest.mark.parametrize("N,K", [(64, 256), (37, 1000), (1, 8), (300, 4104), (16, 264)])
+@pytest.mark.parametrize("N,K", [(64, 256), (37, 1000), (1, 8), (300, 4104), (16, 264), (50, 1040)])
 def test_gemv_shapes(M, N, K):
     c = workloads.gemv_case(M, N, K, seed=M * 7 + N)
     y = apd.gemv(c.x.cuda(), c.w.cuda())
@@ -49,6 +49,18 @@ def test_gemv_strided_operands():
 def test_gemv_projection_shapes(layer, M):
     c = workloads.gemv_named(layer, M)
     check(apd.gemv(c.x.cuda(), c.w.cuda()), c.x, c.w, f"{layer} M={M}")
+
+
+@pytest.mark.parametrize("M,N,K,pad", [(5, 22000, 1544, 8), (8, 21000, 1600, 0), (1, 22000, 1544, 0)])
+def test_gemv_x_staged_once_per_cta(M, N, K, pad):
+    """Weights of 64 MB and more take the path that copies x into shared memory once per
+    CTA: an odd number of 16-byte chunks per row with a partial last 256-column tile
+    (K = 1544), an even number that needs the padded row pitch (K = 1600), a strided x."""
+    c = workloads.gemv_case(M, N, K, seed=21)
+    xb = torch.zeros(M, K + pad, dtype=torch.bfloat16, device="cuda")
+    xb[:, :K] = c.x.cuda()
+    y = apd.gemv(xb[:, :K], c.w.cuda())
+    check(y, c.x, c.w, f"staged x M={M} N={N} K={K} pad={pad}")
 
 
 def test_gemv_graph_capture_and_repeat():
