@@ -23,6 +23,7 @@ __all__ = [
     "attn_paged_decode",
     "attn_contig_decode",
     "attn_paged_prefill",
+    "selftest_bounded_wait",
     "gemv",
     "gemv_workspace_size",
     "DecodeCall",
@@ -139,6 +140,8 @@ def _load():
     L.apd_attn_paged_prefill_ex.argtypes = [T, T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                             ctypes.c_int]
     L.apd_attn_paged_prefill_ex.restype = ctypes.c_int
+    L.apd_selftest_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p]
+    L.apd_selftest_bounded_wait.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
     L.apd_gemv_bf16.argtypes = [T, T, T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
@@ -280,6 +283,18 @@ def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
 
 
 PREFILL_KERNELS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
+
+
+def selftest_bounded_wait(short_timeout_ns: int = 1_000_000, device="cuda") -> list[int]:
+    """Runs the library's bounded-wait self-test on the GPU and returns [first wait gave up,
+    second wait gave up (through the abort flag), second wait's duration in us, flag word]."""
+    out = torch.zeros(4, dtype=torch.int32, device=device)
+    L = _load()
+    rc = L.apd_selftest_bounded_wait(out.data_ptr(), int(short_timeout_ns), _stream_handle(None, out.device))
+    if rc:
+        raise APDError(rc, "apd_selftest_bounded_wait")
+    torch.cuda.synchronize(out.device)
+    return [int(v) & 0xFFFFFFFF for v in out.cpu().tolist()]
 
 
 def prefill_auto_kernel(head_dim: int) -> str:

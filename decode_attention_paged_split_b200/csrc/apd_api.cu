@@ -1128,3 +1128,15 @@ const char* apd_status_string(int status) {
 const char* apd_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
+
+int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stream_t stream) {
+    if (!out) return APD_ERR_NULL_POINTER;
+    if (short_timeout_ns == 0 || short_timeout_ns > 1000000000ull) return APD_ERR_ARGUMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(out, 0, 4 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(selftest)");
+    apd::wait_selftest_kernel<<<1, 64, 0, st>>>(out, short_timeout_ns);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "wait_selftest_kernel launch");
+    return APD_OK;
+}

@@ -245,17 +245,44 @@ struct TcShape {
 
 // Bounded mbarrier wait that also gives up when another role raised the abort flag.
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                        uint32_t* flags) {
+                                        uint32_t* flags, uint64_t timeout_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if ((it & 63u) == 0 && global_timer_ns() - t0 > kWaitTimeoutNs) {
+        if ((it & 63u) == 0 && global_timer_ns() - t0 > timeout_ns) {
             *abort_flag = 1u;
             if (flags) atomicOr(flags, kFlagTimeout);
             return false;
         }
+    }
+}
+
+// Self-test of the bounded waits, on mbarriers that nothing ever completes (no copy,
+// no MMA, no fault): thread 0 waits with a short limit and must give up, record the
+// timeout flag and raise the abort flag; thread 32 waits with the kernels' full limit and
+// must give up early through that abort flag.  out[0..3]: thread 0 gave up, thread 32 gave
+// up, thread 32's wait in microseconds, the flag word.
+__global__ void __launch_bounds__(64) wait_selftest_kernel(uint32_t* out, uint64_t short_ns) {
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ uint32_t abort_word;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        abort_word = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    volatile uint32_t* abort_flag = &abort_word;
+    if (threadIdx.x == 0) {
+        const bool done = tc_wait(smem_u32(&bars[0]), 0u, abort_flag, out + 3, short_ns);
+        out[0] = done ? 0u : 1u;
+    } else if (threadIdx.x == 32) {
+        const uint64_t t0 = global_timer_ns();
+        const bool done = tc_wait(smem_u32(&bars[1]), 0u, abort_flag, nullptr);
+        out[2] = static_cast<uint32_t>((global_timer_ns() - t0) / 1000u);
+        out[1] = done ? 0u : 1u;
     }
 }
 

@@ -350,6 +350,22 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
 int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_stream_t stream, uint32_t* flags,
                           int clear);
 
+/*
+ * apd_selftest_bounded_wait -- exercises, on the GPU, the bounded waits every kernel
+ * here uses on its mbarriers, without any copy, MMA or fault: one thread waits on an
+ * mbarrier that nothing completes, with a limit of `short_timeout_ns` (1 .. 1e9 ns),
+ * and must give up, set APD_FLAG_WAIT_TIMEOUT and raise the CTA's abort flag; a second
+ * thread waits on another such mbarrier with the kernels' full limit (2 s) and must give
+ * up early because of that abort flag.
+ *
+ *   out      device uint32[4] (caller-owned): out[0] = 1 if the first wait gave up,
+ *            out[1] = 1 if the second gave up, out[2] = the second wait's duration in
+ *            microseconds, out[3] = the flag word written by the first wait.
+ *   Returns APD_ERR_NULL_POINTER / APD_ERR_ARGUMENT before any launch, APD_ERR_CUDA on a
+ *   launch failure, else APD_OK (asynchronous: read `out` after synchronising `stream`).
+ */
+int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stream_t stream);
+
 /* apd_plan -- how a call with these arguments would be launched (for tests,
  * benchmarks and profiling). */
 typedef struct apd_plan {

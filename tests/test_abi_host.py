@@ -363,3 +363,10 @@ def test_prefill_binding_rejects_unknown_kernel_names():
     with pytest.raises(ValueError):
         apd.attn_paged_prefill(q, q, q, torch.zeros(1, 1, dtype=torch.int32), torch.zeros(1, dtype=torch.int32),
                                0.1, kernel="wgmma")
+
+
+def test_selftest_arguments_are_checked_before_any_launch():
+    L = apd.lib()
+    assert L.apd_selftest_bounded_wait(None, 1000, None) == NULLP
+    assert L.apd_selftest_bounded_wait(FAKE, 0, None) == ARG
+    assert L.apd_selftest_bounded_wait(FAKE, 2_000_000_000, None) == ARG
