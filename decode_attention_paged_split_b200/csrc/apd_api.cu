@@ -571,7 +571,7 @@ int prefill_stages(int D) { return D == 32 ? 8 : D == 64 ? 6 : D == 128 ? 4 : 3;
 constexpr bool kPrefillAutoTc = true;
 
 size_t prefill_smem_bytes(int D) {
-    return 16ull * prefill_stages(D) + 1024 + static_cast<size_t>(prefill_stages(D)) * 2 * apd::kTile * D * 2;
+    return 16ull * prefill_stages(D) + 8 + 1024 + static_cast<size_t>(prefill_stages(D)) * 2 * apd::kTile * D * 2;
 }
 
 struct PrefillCheck {

@@ -79,7 +79,8 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
     const int warp = threadIdx.x >> 5;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + STAGES;
-    const uint32_t ring = (smem_u32(empty + STAGES) + 1023u) & ~1023u;
+    uint64_t* vzero = empty + STAGES;  // consumers meet here after zeroing the V tail (at most once)
+    const uint32_t ring = (smem_u32(vzero + 1) + 1023u) & ~1023u;
 
     // ---- work item: (sequence b, kv head, block of kPrefillRows query rows)
     const int rb = blockIdx.x % p.blocks_per_head;
@@ -94,6 +95,9 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(full + s), 1);
             mbar_init(smem_u32(empty + s), kPrefillConsumers);
+        }
+        {
+            mbar_init(smem_u32(vzero), 32 * kPrefillConsumers);
         }
         fence_mbar_init();
         prefetch_tensormap(&kmap);
@@ -212,7 +216,13 @@ __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)
             for (int idx = warp * 32 + lane; idx < (kTile - valid) * G::kChunks; idx += 32 * kPrefillConsumers) {
                 st_shared_zero16(vb + G::chunk_off(valid + idx / G::kChunks, idx % G::kChunks, kTile));
             }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kPrefillConsumers) : "memory");
+            // an mbarrier with a bounded wait rather than a named barrier: a consumer that
+            // gave up on an earlier wait cannot leave the others blocked here
+            mbar_arrive(smem_u32(vzero));
+            if (!mbar_wait_bounded(smem_u32(vzero), 0u, kWaitTimeoutNs)) {
+                if (lane == 0 && p.flags) atomicOr(p.flags, kFlagTimeout);
+                return;
+            }
         }
 
         // ---- S = Q K^T over the tile's 32 keys
