@@ -212,6 +212,70 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
+// ---- pieces shared by the tensor-core prefill kernels
+
+// Q rows [row_first, row_first + 128) of (sequence b, kv head kvh), the (query, head-in-
+// group) pairs row = i * g + hh, into the 128-byte-swizzled K-major A layout
+// [D/64][128][64] at q_s; rows >= R are zeros.  Threads tid (of nthreads) share the copy.
+template <int D>
+__device__ __forceinline__ void stage_q_tile(uint32_t q_s, const PrefillParams& p, int b, int kvh, int row_first,
+                                             int R, int tid, int nthreads) {
+    constexpr int M = 128;
+    for (int idx = tid; idx < M * (D / 8); idx += nthreads) {
+        const int row = idx / (D / 8), ch = idx % (D / 8);
+        const int rq = row_first + row;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (rq < R) {
+            const int i = rq / p.g, hh = rq - i * p.g;
+            v = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
+                                                     ch * 8));
+        }
+        st_shared_v4(q_s + static_cast<uint32_t>((ch >> 3) * (M * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4)),
+                     v.x, v.y, v.z, v.w);
+    }
+}
+
+// Zeroes rows [v0, N) of a V tile staged as [D/64][N][64] with 128-byte rows (the swizzle
+// only permutes 16-byte chunks within a row, so whole rows are cleared in place).
+template <int D, int N>
+__device__ __forceinline__ void zero_v_rows(uint32_t vb, int v0, int tid, int nthreads) {
+    constexpr int kBlk = D / 64;
+    for (int idx = tid; idx < (N - v0) * kBlk * 8; idx += nthreads) {
+        const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
+        st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
+    }
+}
+
+// Epilogue of one row: NC columns of O from TMEM at taddr (this thread's lane), times inv,
+// as bf16 to orow.  The TMEM loads are warp-collective, so every lane loads; only rows
+// that exist store.  With no tile processed (have_o false) the row is zeros.
+template <int NC>
+__device__ __forceinline__ void store_o_row(uint32_t taddr, bool have_o, float inv, bool row_ok,
+                                            __nv_bfloat16* orow) {
+#pragma unroll 1
+    for (int c = 0; c < NC / 32; ++c) {
+        uint32_t o[32];
+        if (have_o) {
+            tc_ld32(taddr + static_cast<uint32_t>(32 * c), o);
+            tc_wait_ld();
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+                *reinterpret_cast<uint4*>(orow + 32 * c + 8 * e) = w;
+            }
+        }
+    }
+}
+
 // Tile shape and shared-memory / TMEM layout per head dim.
 template <int D>
 struct TcShape {
@@ -497,19 +561,7 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
         const int cb = h * NH;  // this warp's first column of S (and key of the tile)
         const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t xbar = bar(kXchg + quad);
-        // Q tile into the swizzled K-major A layout, zeros past the last row
-        for (int idx = threadIdx.x; idx < M * (D / 8); idx += SW) {
-            const int row = idx / (D / 8), ch = idx % (D / 8);
-            const int rg = row0 + row;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (rg < R) {
-                const int i = rg / p.g, hh = rg - i * p.g;
-                v = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
-                                                         ch * 8));
-            }
-            st_shared_v4(q_s + static_cast<uint32_t>((ch >> 3) * (M * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4)),
-                         v.x, v.y, v.z, v.w);
-        }
+        stage_q_tile<D>(q_s, p, b, kvh, row0, R, threadIdx.x, SW);
         fence_proxy_async_smem();
         mbar_arrive(bar(kQFull));
 
@@ -638,10 +690,7 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                 if (!ok) break;
                 const int v0 = kv_end - j * N;
                 const uint32_t vb = tb + T::kVOff + static_cast<uint32_t>(stage) * T::kKVBytes;
-                for (int idx = threadIdx.x; idx < (N - v0) * kBlk * 8; idx += SW) {
-                    const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
-                    st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
-                }
+                zero_v_rows<D, N>(vb, v0, threadIdx.x, SW);
             }
             fence_proxy_async_smem();  // P (and the zeroed V rows) -> tensor core
             tc_fence_before();
@@ -663,29 +712,8 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
         if (ok) {
             const float lt = l + xsum[(h ^ 1) * M + r];
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            __nv_bfloat16* orow = p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh + h * DH;
-#pragma unroll 1
-            for (int c = 0; c < DH / 32; ++c) {
-                uint32_t o[32];
-                if (ntiles > 0) {
-                    tc_ld32(tmem + t_lane + T::kColO + static_cast<uint32_t>(h * DH + 32 * c), o);
-                    tc_wait_ld();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0u;
-                }
-                if (row_ok) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + 32 * c + 8 * e) = w;
-                    }
-                }
-            }
+            store_o_row<DH>(tmem + t_lane + T::kColO + static_cast<uint32_t>(h * DH), ntiles > 0, inv, row_ok,
+                            p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh + h * DH);
         }
     }
     // ---- all roles meet before the TMEM columns are freed
@@ -962,19 +990,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
         const uint32_t s_col = T::kColS + 128u * t;
         const uint32_t o_col = T::kColO + static_cast<uint32_t>(D * t);
         const uint32_t q_s = tb + static_cast<uint32_t>(t) * T::kQBytes;
-        // Q tile t into the swizzled K-major A layout, zeros past the last row
-        for (int idx = wt; idx < M * (D / 8); idx += 128) {
-            const int row = idx / (D / 8), ch = idx % (D / 8);
-            const int rq = row0 + M * t + row;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (rq < R) {
-                const int i = rq / p.g, hh = rq - i * p.g;
-                v = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
-                                                         ch * 8));
-            }
-            st_shared_v4(q_s + static_cast<uint32_t>((ch >> 3) * (M * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4)),
-                         v.x, v.y, v.z, v.w);
-        }
+        stage_q_tile<D>(q_s, p, b, kvh, row0 + M * t, R, wt, 128);
         fence_proxy_async_smem();
         mbar_arrive(bar(kQFull));
 
@@ -1056,10 +1072,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                 if (!ok) break;
                 const int v0 = kv_end - j * N;
                 const uint32_t vb = ring + static_cast<uint32_t>(nv % NS) * T::kSlotBytes;
-                for (int idx = wt; idx < (N - v0) * kBlk * 8; idx += 128) {
-                    const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
-                    st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
-                }
+                zero_v_rows<D, N>(vb, v0, wt, 128);
                 fence_proxy_async_smem();  // before the first half of P is handed over
             }
             // ---- P = 2^(s * cs - reference) as bf16 pairs over the first half of S_t,
@@ -1111,29 +1124,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
             // a row that saw no visible key outputs zeros (its emulated exponentials of
             // -inf are tiny, not 0, so test the running maximum rather than l)
             const float inv = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                if (ntiles > 0) {
-                    tc_ld32(tmem + t_lane + o_col + static_cast<uint32_t>(32 * c), o);
-                    tc_wait_ld();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0u;
-                }
-                if (row_ok) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + 32 * c + 8 * e) = w;
-                    }
-                }
-            }
+            store_o_row<D>(tmem + t_lane + o_col, ntiles > 0, inv, row_ok, p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh);
         }
     }
     // ---- all roles meet before the TMEM columns are freed
