@@ -299,7 +299,7 @@ def selftest_bounded_wait(short_timeout_ns: int = 1_000_000, device="cuda") -> l
 
 def prefill_auto_kernel(head_dim: int) -> str:
     """The kernel attn_paged_prefill(kernel="auto") runs for a head dim."""
-    return "tcgen05" if PREFILL_AUTO_TC and head_dim != 32 else "mma_sync"
+    return "tcgen05" if PREFILL_AUTO_TC else "mma_sync"
 
 
 PREFILL_AUTO_TC = True  # mirrors the library's default choice
@@ -313,7 +313,7 @@ def attn_paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Te
 
     causal_offset -1: no causal mask; c >= 0: query i sits at position c + i.  mask: None,
     uint8/bool [B, kv_len] or [B, Lq, kv_len] (nonzero = visible).  kernel: "auto",
-    "mma_sync" (every head dim) or "tcgen05" (D = 64, 128, 256)."""
+    "mma_sync" or "tcgen05" (both: every head dim)."""
     if kernel not in PREFILL_KERNELS:
         raise ValueError(f"kernel must be one of {sorted(PREFILL_KERNELS)}")
     if out is None:

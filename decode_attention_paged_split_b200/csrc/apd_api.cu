@@ -567,7 +567,7 @@ int gemv_validate(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
 // ---------------------------------------------------------------- multi-query (prefill)
 int prefill_stages(int D) { return D == 32 ? 8 : D == 64 ? 6 : D == 128 ? 4 : 3; }
 
-// Default prefill kernel for D >= 64: the tcgen05 one (mma.sync stays selectable, and serves D = 32).
+// Default prefill kernel: the tcgen05 one for every head dim (mma.sync stays selectable).
 constexpr bool kPrefillAutoTc = true;
 
 size_t prefill_smem_bytes(int D) {
@@ -713,14 +713,14 @@ int launch_prefill(const PrefillCheck& C, const apd_tensor* q, const apd_tensor*
                                "prefill_kernel launch");
 }
 
-// tcgen05 kernel with two 128-row Q tiles per CTA (D = 64, 128)
+// tcgen05 kernel with two 128-row Q tiles per CTA (D = 32, 64, 128)
 template <int D>
 int launch_prefill_tc2(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
                        const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
                        float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
     using T = apd::Tc2Shape<D>;
     auto kern = apd::prefill_tc2_kernel<D>;
-    constexpr int kSlot = (D == 64) ? 1 : 2;
+    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : 2;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!dev->prefill_tc2_attr_set[kSlot]) {
@@ -738,14 +738,14 @@ int launch_prefill_tc2(const PrefillCheck& C, const apd_tensor* q, const apd_ten
     return launch_prefill_grid(kern, pp, kmap, vmap, T::kThreads, T::kSmemBytes, stream, "prefill_tc2_kernel launch");
 }
 
-// tcgen05 kernel, one 128-row Q tile per CTA (D = 64, 128, 256)
+// tcgen05 kernel, one 128-row Q tile per CTA (every D)
 template <int D>
 int launch_prefill_tc(const PrefillCheck& C, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
                       const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* mask, const apd_tensor* out,
                       float scale, int causal_offset, DeviceState* dev, cudaStream_t stream) {
     using T = apd::TcShape<D>;
     auto kern = apd::prefill_tc_kernel<D>;
-    constexpr int kSlot = (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!dev->prefill_tc_attr_set[kSlot]) {
@@ -944,8 +944,7 @@ int apd_attn_paged_prefill_ex(const apd_tensor* q, const apd_tensor* k_cache, co
     int rc = prefill_validate(q, k_cache, v_cache, page_table, seq_lens, mask, out, causal_offset, &C);
     if (rc) return rc;
     const int D = C.V.s.D;
-    if (kernel == APD_PREFILL_TCGEN05 && D == 32) return APD_ERR_HEAD_DIM;
-    const bool tc = kernel == APD_PREFILL_TCGEN05 || (kernel == APD_PREFILL_AUTO && kPrefillAutoTc && D != 32);
+    const bool tc = kernel == APD_PREFILL_TCGEN05 || (kernel == APD_PREFILL_AUTO && kPrefillAutoTc);
     if (C.V.s.B == 0) return APD_OK;
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
@@ -953,12 +952,15 @@ int apd_attn_paged_prefill_ex(const apd_tensor* q, const apd_tensor* k_cache, co
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // two Q tiles per CTA when a kv head has more than one tile of query rows
     const bool two_tiles = static_cast<int64_t>(C.Lq) * C.V.s.g > 128;
+    if (tc && two_tiles && D == 32)
+        return launch_prefill_tc2<32>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
     if (tc && two_tiles && D == 64)
         return launch_prefill_tc2<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
     if (tc && two_tiles && D == 128)
         return launch_prefill_tc2<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
     if (tc) {
         switch (D) {
+            case 32: return launch_prefill_tc<32>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
             case 64: return launch_prefill_tc<64>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
             case 128: return launch_prefill_tc<128>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);
             case 256: return launch_prefill_tc<256>(C, q, k_cache, v_cache, page_table, seq_lens, mask, out, scale, causal_offset, dev, st);

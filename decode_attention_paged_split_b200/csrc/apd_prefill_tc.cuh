@@ -123,6 +123,37 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same for the 64-byte swizzle (mode 4), whose atoms are 8 rows of 64 bytes: the
+// layout of operands with 32-element rows (head dim 32).
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+
+// Staging geometry of a [rows][D] bf16 operand: column blocks of kCols elements
+// (64 with the 128-byte swizzle; the whole row, 32, with the 64-byte swizzle for
+// D = 32), each block [rows][kCols] with kRowBytes-byte rows.
+template <int D>
+struct OperandGeom {
+    static constexpr int kCols = D >= 64 ? 64 : D;
+    static constexpr int kRowBytes = 2 * kCols;
+    static constexpr int kBlk = D / kCols;
+    static constexpr int kChunks = kRowBytes / 16;  // 16-byte chunks per row of a block
+    static constexpr uint32_t kSbo = 8 * kRowBytes;  // 8-row groups
+    static_assert(D == 32 || D % 64 == 0, "head dim");
+    // physical 16-byte chunk of logical chunk c in row `row` of a block
+    __device__ static constexpr int swz(int row, int c) { return D >= 64 ? (c ^ (row & 7)) : (c ^ ((row >> 1) & 3)); }
+    __device__ static uint64_t desc(uint32_t saddr, uint32_t lbo) {
+        if constexpr (D >= 64) return sw128_desc(saddr, lbo, kSbo);
+        else return sw64_desc(saddr, lbo, kSbo);
+    }
+    // K-major operand [rows][D] staged as kBlk blocks of [rows][kCols]: start of the 16-
+    // element K step ks
+    __device__ static constexpr uint32_t kstep(int ks, int rows) {
+        return static_cast<uint32_t>((ks / (kCols / 16)) * rows * kRowBytes + (ks % (kCols / 16)) * 32);
+    }
+};
+
 // Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B, fp32 D,
 // A K-major, B K-major or MN-major, shape M x N (N % 16 == 0 for M = 128).
 constexpr uint32_t bf16_idesc(int M, int N, bool b_mn_major) {
@@ -220,6 +251,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <int D>
 __device__ __forceinline__ void stage_q_tile(uint32_t q_s, const PrefillParams& p, int b, int kvh, int row_first,
                                              int R, int tid, int nthreads) {
+    using O = OperandGeom<D>;
     constexpr int M = 128;
     for (int idx = tid; idx < M * (D / 8); idx += nthreads) {
         const int row = idx / (D / 8), ch = idx % (D / 8);
@@ -230,19 +262,22 @@ __device__ __forceinline__ void stage_q_tile(uint32_t q_s, const PrefillParams& 
             v = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
                                                      ch * 8));
         }
-        st_shared_v4(q_s + static_cast<uint32_t>((ch >> 3) * (M * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4)),
+        st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (M * O::kRowBytes) + row * O::kRowBytes +
+                                                 (O::swz(row, ch % O::kChunks) << 4)),
                      v.x, v.y, v.z, v.w);
     }
 }
 
-// Zeroes rows [v0, N) of a V tile staged as [D/64][N][64] with 128-byte rows (the swizzle
-// only permutes 16-byte chunks within a row, so whole rows are cleared in place).
+// Zeroes rows [v0, N) of a V tile staged as OperandGeom blocks (the swizzle only permutes
+// 16-byte chunks within a row, so whole rows are cleared in place).
 template <int D, int N>
 __device__ __forceinline__ void zero_v_rows(uint32_t vb, int v0, int tid, int nthreads) {
-    constexpr int kBlk = D / 64;
-    for (int idx = tid; idx < (N - v0) * kBlk * 8; idx += nthreads) {
-        const int row = v0 + idx / (kBlk * 8), rest = idx % (kBlk * 8);
-        st_shared_zero16(vb + static_cast<uint32_t>((rest >> 3) * (N * 128) + row * 128 + ((rest & 7) << 4)));
+    using O = OperandGeom<D>;
+    constexpr int kPerRow = O::kBlk * O::kChunks;
+    for (int idx = tid; idx < (N - v0) * kPerRow; idx += nthreads) {
+        const int row = v0 + idx / kPerRow, rest = idx % kPerRow;
+        st_shared_zero16(vb + static_cast<uint32_t>((rest / O::kChunks) * (N * O::kRowBytes) + row * O::kRowBytes +
+                                                    ((rest % O::kChunks) << 4)));
     }
 }
 
@@ -281,7 +316,7 @@ template <int D>
 struct TcShape {
     static constexpr int kM = 128;                    // query rows per CTA (TMEM lanes)
     static constexpr int kN = (D == 256) ? 64 : 128;  // keys per tile
-    static constexpr int kStages = (D == 64) ? 4 : 2;
+    static constexpr int kStages = (D == 32) ? 6 : (D == 64) ? 4 : 2;
     static constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quadrant, half a row's columns each
     static constexpr int kSoftmaxThreads = 32 * kSoftmaxWarps;
     static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
@@ -356,7 +391,7 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                       const __grid_constant__ CUtensorMap vmap) {
     using T = TcShape<D>;
     constexpr int M = T::kM, N = T::kN, ST = T::kStages;
-    constexpr int kBlk = D / 64;    // 64-dim column blocks of Q, K and V
+    using O = OperandGeom<D>;  // staging of Q, K and V: O::kBlk blocks of [rows][O::kCols]
     constexpr int kGroups = N / 32; // 32-token boxes per tile
     constexpr uint32_t kIdescQK = bf16_idesc(M, N, false);
     constexpr uint32_t kIdescPV = bf16_idesc(M, D, true);
@@ -476,10 +511,15 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                         const int page = pages[q];
                         if ((page < 0 || page >= p.NP) && p.flags) atomicOr(p.flags, kFlagPageOOR);
                         const int slot = (j * N + 32 * q) % p.P;
+                        if constexpr (D == 32) {
+                            tma_load_4d(dst + static_cast<uint32_t>(q * 32 * O::kRowBytes), kv ? &vmap : &kmap, full,
+                                        0, kvh, slot, page, pol);
+                        } else {
 #pragma unroll
-                        for (int c = 0; c < kBlk; ++c)
-                            tma_load_5d(dst + static_cast<uint32_t>(c * N * 128 + q * 4096), kv ? &vmap : &kmap,
-                                        full, 0, kvh, slot, page, c, pol);
+                            for (int c = 0; c < O::kBlk; ++c)
+                                tma_load_5d(dst + static_cast<uint32_t>(c * N * O::kRowBytes + q * 32 * O::kRowBytes),
+                                            kv ? &vmap : &kmap, full, 0, kvh, slot, page, c, pol);
+                        }
                     }
                 }
                 __syncwarp();
@@ -515,7 +555,7 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                 for (int k = 0; k < N / 16; ++k) {
                     const uint32_t po = static_cast<uint32_t>((k >> 2) * (M * 128) + (k & 3) * 32);
                     tc_mma_bf16(tmem + T::kColO, sw128_desc(p_s + po, 16, 1024),
-                                sw128_desc(vb + static_cast<uint32_t>(k) * 2048u, N * 128, 1024), kIdescPV,
+                                O::desc(vb + static_cast<uint32_t>(k * 16 * O::kRowBytes), N * O::kRowBytes), kIdescPV,
                                 (jj > 0 || k > 0) ? 1u : 0u);
                 }
                 tc_commit(bar(kPVDone));
@@ -535,9 +575,7 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                 const uint32_t d = tmem + T::kColS + static_cast<uint32_t>((j & 1) * N);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t qo = static_cast<uint32_t>((k >> 2) * (M * 128) + (k & 3) * 32);
-                    const uint32_t ko = static_cast<uint32_t>((k >> 2) * (N * 128) + (k & 3) * 32);
-                    tc_mma_bf16(d, sw128_desc(q_s + qo, 16, 1024), sw128_desc(kb + ko, 16, 1024), kIdescQK,
+                    tc_mma_bf16(d, O::desc(q_s + O::kstep(k, M), 16), O::desc(kb + O::kstep(k, N), 16), kIdescQK,
                                 k > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(kSFull + (j & 1)));
@@ -555,8 +593,11 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
     } else {
         // ================= softmax warps: warps w and w + 4 share TMEM lane quadrant w
         // (rows 32w .. 32w + 31, one per thread) and take half of each row's columns
-        constexpr int NH = N / 2, DH = D / 2;
+        // O columns per warp: half of them each, or (D = 32, one 32-column load) all of
+        // them for the first half and none for the second
+        constexpr int NH = N / 2, DH = D >= 64 ? D / 2 : D;
         const int quad = warp & 3, h = warp >> 2;
+        const bool o_owner = D >= 64 || h == 0;
         const int r = 32 * quad + lane;
         const int cb = h * NH;  // this warp's first column of S (and key of the tile)
         const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
@@ -661,9 +702,9 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
             }
-            if (__any_sync(0xffffffffu, grow)) {
+            if (o_owner && __any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-                for (int c = 0; c < DH / 32; ++c) {  // this warp's half of the O columns
+                for (int c = 0; c < DH / 32; ++c) {  // this warp's O columns
                     uint32_t o[32];
                     const uint32_t ta = tmem + t_lane + T::kColO + static_cast<uint32_t>(h * DH + 32 * c);
                     tc_ld32(ta, o);
@@ -712,8 +753,9 @@ __global__ void __launch_bounds__(TcShape<D>::kThreads, 1)
         if (ok) {
             const float lt = l + xsum[(h ^ 1) * M + r];
             const float inv = lt > 0.f ? 1.f / lt : 0.f;
-            store_o_row<DH>(tmem + t_lane + T::kColO + static_cast<uint32_t>(h * DH), ntiles > 0, inv, row_ok,
-                            p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh + h * DH);
+            if (o_owner)
+                store_o_row<DH>(tmem + t_lane + T::kColO + static_cast<uint32_t>(h * DH), ntiles > 0, inv, row_ok,
+                                p.out + b * p.o_sb + qi * p.o_si + qh * p.o_sh + h * DH);
         }
     }
     // ---- all roles meet before the TMEM columns are freed
@@ -758,7 +800,7 @@ template <int D>
 struct Tc2Shape {
     static constexpr int kM = 128;  // rows per Q tile (TMEM lanes); two tiles per CTA
     static constexpr int kN = 128;  // keys per tile
-    static constexpr int kSlots = (D == 64) ? 8 : 4;
+    static constexpr int kSlots = (D == 32) ? 16 : (D == 64) ? 8 : 4;
     static constexpr int kThreads = 320;  // warps 0-7 softmax, 8 producer, 9 MMA issuer
     static constexpr int kProducerWarp = 8, kMmaWarp = 9;
     static constexpr uint32_t kQBytes = kM * D * 2;  // one Q tile
@@ -771,7 +813,7 @@ struct Tc2Shape {
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;    // S_t at 128 t
     static constexpr uint32_t kColO = 256;  // O_t at 256 + D t
-    static_assert(D == 64 || D == 128, "two-tile kernel: D = 64 or 128");
+    static_assert(D == 32 || D == 64 || D == 128, "two-tile kernel: D = 32, 64 or 128");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the 512 TMEM columns are always free");
 };
@@ -782,7 +824,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                        const __grid_constant__ CUtensorMap vmap) {
     using T = Tc2Shape<D>;
     constexpr int M = T::kM, N = T::kN, NS = T::kSlots;
-    constexpr int kBlk = D / 64;
+    using O = OperandGeom<D>;
     constexpr int kGroups = N / 32;
     constexpr uint32_t kIdescQK = bf16_idesc(M, N, false);
     constexpr uint32_t kIdescPV = bf16_idesc(M, D, true);
@@ -891,10 +933,15 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                     const int page = pages[q];
                     if ((page < 0 || page >= p.NP) && p.flags) atomicOr(p.flags, kFlagPageOOR);
                     const int sl = (j * N + 32 * q) % p.P;
+                    if constexpr (D == 32) {
+                        tma_load_4d(dst + static_cast<uint32_t>(q * 32 * O::kRowBytes), kv ? &vmap : &kmap, full, 0,
+                                    kvh, sl, page, pol);
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < kBlk; ++c)
-                        tma_load_5d(dst + static_cast<uint32_t>(c * N * 128 + q * 4096), kv ? &vmap : &kmap, full, 0,
-                                    kvh, sl, page, c, pol);
+                        for (int c = 0; c < O::kBlk; ++c)
+                            tma_load_5d(dst + static_cast<uint32_t>(c * N * O::kRowBytes + q * 32 * O::kRowBytes),
+                                        kv ? &vmap : &kmap, full, 0, kvh, sl, page, c, pol);
+                    }
                 }
             }
             __syncwarp();
@@ -921,9 +968,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                 const uint32_t qb = tb + static_cast<uint32_t>(t) * T::kQBytes;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
-                    const uint32_t qo = static_cast<uint32_t>((k >> 2) * (M * 128) + (k & 3) * 32);
-                    const uint32_t ko = static_cast<uint32_t>((k >> 2) * (N * 128) + (k & 3) * 32);
-                    tc_mma_bf16(tmem + T::kColS + 128u * t, sw128_desc(qb + qo, 16, 1024), sw128_desc(kb + ko, 16, 1024),
+                    tc_mma_bf16(tmem + T::kColS + 128u * t, O::desc(qb + O::kstep(k, M), 16), O::desc(kb + O::kstep(k, N), 16),
                                 kIdescQK, k > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(kSFull + t));
@@ -935,7 +980,7 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                 for (int kk = 0; kk < N / 16 / kParts; ++kk) {
                     const int k = (N / 16 / kParts) * h + kk;
                     tc_mma_bf16_ts(tmem + T::kColO + static_cast<uint32_t>(D * t), tmem + T::kColS + 128u * t + 8u * k,
-                                   sw128_desc(vb + static_cast<uint32_t>(k) * 2048u, N * 128, 1024), kIdescPV,
+                                   O::desc(vb + static_cast<uint32_t>(k * 16 * O::kRowBytes), N * O::kRowBytes), kIdescPV,
                                    (j > 0 || k > 0) ? 1u : 0u);
                 }
                 if (h == kParts - 1) tc_commit(bar(kPVDone + t));

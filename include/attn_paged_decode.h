@@ -262,7 +262,7 @@ int apd_attn_paged_prefill(const apd_tensor* q, const apd_tensor* k_cache, const
  *           APD_PREFILL_MMA_SYNC (1): warp-level mma.sync tiles, every head dim;
  *           APD_PREFILL_TCGEN05 (2): fifth-generation tensor cores (tcgen05.mma
  *           with TMEM accumulators, 128 query rows x 128 keys per step, 64 keys
- *           for D = 256); D = 64, 128, 256 only (D = 32 -> APD_ERR_HEAD_DIM).
+ *           for D = 256); every head dim.
  *   Any other value -> APD_ERR_ARGUMENT, before any launch.
  */
 #define APD_PREFILL_AUTO 0

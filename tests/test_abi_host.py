@@ -347,10 +347,10 @@ def prefill_problem(B=2, Lq=5, Hq=8, Hkv=2, D=64, P=32, NP=16, MP=4):
 def test_prefill_kernel_choice_is_validated_before_any_launch():
     for bad in (-1, 3, 99):
         assert prefill_call(prefill_problem(), kernel=bad) == ARG
-    # the tensor-core kernel has no D = 32 variant; the mma.sync one has
-    assert prefill_call(prefill_problem(D=32), kernel=apd.PREFILL_KERNELS["tcgen05"]) == HEADDIM
     for k in apd.PREFILL_KERNELS.values():
-        assert prefill_call(prefill_problem(D=32), kernel=k) in (OK, CUDA) or k == 2
+        for D in (32, 64, 128, 256):  # every head dim on every kernel (the call then needs a device)
+            assert prefill_call(prefill_problem(D=D), kernel=k) in (OK, CUDA)
+        assert prefill_call(prefill_problem(D=96), kernel=k) == HEADDIM
         assert prefill_call(prefill_problem(B=0), kernel=k) == OK
         assert prefill_call(prefill_problem(Hq=6, Hkv=4), kernel=k) == GQA
         assert prefill_call(prefill_problem(), kernel=k, causal=-2) == ARG

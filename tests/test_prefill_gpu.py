@@ -19,13 +19,11 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture(params=["mma_sync", "tcgen05"])
 def kernel(request):
-    """Every case runs on both kernels (the tensor-core one has no D = 32 variant)."""
+    """Every case runs on both kernels."""
     return request.param
 
 
 def run(w, stream=None, kernel="auto"):
-    if kernel == "tcgen05" and w.q.shape[-1] == 32:
-        pytest.skip("no tcgen05 kernel for D = 32")
     heads_outer = w.k_cache.stride(1) < w.k_cache.stride(2)  # HND storage passed as a view
     def dev(t):
         if heads_outer:
