@@ -450,6 +450,9 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     if (pl.combine_ctas > 0) {
         apd::CombineParams cp;
         cp.cum = sp.cum_out;
+        cp.seq_lens = sp.seq_lens;
+        cp.MP = sp.MP;
+        cp.P = sp.P;
         cp.o_part = sp.o_part;
         cp.ml_part = sp.ml_part;
         cp.out = sp.out;

@@ -71,7 +71,9 @@ struct SplitParams {
 };
 
 struct CombineParams {
-    const int32_t* cum;  // [B + 1]
+    const int32_t* cum;       // [B + 1] (written by the split kernel; unused by the combine itself)
+    const int32_t* seq_lens;  // [B]: the combine recomputes its prefix sums from these
+    int32_t MP, P;            // page-table capacity MP * P, for the same clamp as the split kernel
     const float* o_part;
     const float* ml_part;
     __nv_bfloat16* out;
@@ -591,8 +593,43 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __gri
     __nv_bfloat16* orow = p.out + b * p.out_sb + head * p.out_sh;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    // Tile counts of the sequences, clamped as the split kernel clamps them, and their
+    // prefix sums at b and over all B.  This runs before the wait on the split grid:
+    // seq_lens is not written by it, and this grid cannot start before every split CTA
+    // has passed its own wait on the kernel before it, so seq_lens is final here.  It
+    // takes one dependent load off the path that follows the split grid's end.
+    __shared__ int s_pre[kCombineWarps], s_tot[kCombineWarps], s_nb;
+    {
+        const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
+        int pre = 0, tot = 0;
+        for (int i = tid; i < p.B; i += blockDim.x) {
+            int L = __ldcg(p.seq_lens + i);
+            L = L < 0 ? 0 : (L > cap ? static_cast<int>(cap) : L);
+            const int t = (L + kTile - 1) / kTile;
+            tot += t;
+            if (i < b) pre += t;
+            if (i == b) s_nb = t;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            pre += __shfl_xor_sync(0xffffffffu, pre, o);
+            tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        }
+        if (lane == 0) {
+            s_pre[warp] = pre;
+            s_tot[warp] = tot;
+        }
+        __syncthreads();
+    }
+    int cum_b = 0, cum_B = 0;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+        cum_b += s_pre[w];
+        cum_B += s_tot[w];
+    }
+    const int n = s_nb;
+
     pdl_wait_prior_grid();
-    const int n = p.cum[b + 1] - p.cum[b];
     if (n == 0) {
         if (p.mode == 0)
             for (int c = tid; c < kCols; c += blockDim.x) *reinterpret_cast<uint2*>(orow + 4 * c) = make_uint2(0u, 0u);
@@ -605,8 +642,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __gri
     int nk, g_first = 0, first_slot_fixed = 0;
     int64_t total = 0, Sb = 0;
     if (p.mode == 0) {
-        total = p.cum[p.B];
-        Sb = p.cum[b];
+        total = cum_B;
+        Sb = cum_b;
         g_first = worker_of(Sb, total, p.groups);
         const int g_last = worker_of(Sb + n - 1, total, p.groups);
         if (g_first == g_last) return;  // one warp covered it and wrote the output
