@@ -139,3 +139,24 @@ def test_prefill_running_max_moves_across_tiles(grow, Lq, kernel):
             else:
                 w.k_cache[page, t % P] /= 8
     check_close(run(w, kernel=kernel), oracle.paged_prefill(w), f"grow={grow}")
+
+
+# ---------------------------------------------------------------- full size
+@pytest.mark.parametrize("kernel_name", ["tcgen05", "mma_sync"])
+def test_prefill_chunk_workload_full_size_sampled(kernel_name):
+    """The bench's prefill workload at full size (16 sequences x 4096 keys, 128 causal
+    queries, 32/8 heads, D = 128, shuffled 2048-page pool) in the bench's launch; three
+    sequences are checked in full against the oracle, run on one-sequence slices of the
+    same inputs (same pool, same page-table rows)."""
+    w = workloads.prefill_llama8b_chunk()
+    q = w.q.cuda()
+    out = torch.full_like(q, float("nan"))
+    apd.attn_paged_prefill(q, w.k_cache.cuda(), w.v_cache.cuda(), w.page_table.cuda(), w.seq_lens.cuda(), w.scale,
+                           w.causal_offset, None, out, kernel=kernel_name)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+    for b in (0, 7, 15):
+        one = workloads.PrefillWorkload(name=f"{w.name}[{b}]", seed=w.seed, q=w.q[b:b + 1], k_cache=w.k_cache,
+                                        v_cache=w.v_cache, page_table=w.page_table[b:b + 1],
+                                        seq_lens=w.seq_lens[b:b + 1], scale=w.scale, causal_offset=w.causal_offset)
+        check_close(out[b:b + 1], oracle.paged_prefill(one), f"{kernel_name} sequence {b}")
