@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -231,13 +232,22 @@ class ClockSampler:
 DECODE_KERNEL_SOURCES = ("apd_kernels.cuh", "apd_ptx.cuh")  # the split and combine kernels' device code
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and with whitespace collapsed, so that editing a comment
+    does not change the hash of the code."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_sha(sources=DECODE_KERNEL_SOURCES) -> str:
-    """Hash of the decode kernels' device code (the headers they are compiled from); the
-    host-side API file and the other kernels' headers are not included."""
+    """Hash of the decode kernels' device code (the headers they are compiled from, comments
+    and whitespace ignored); the host-side API file and the other kernels' headers are not
+    included."""
     h = hashlib.sha256()
     for name in sorted(sources):
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

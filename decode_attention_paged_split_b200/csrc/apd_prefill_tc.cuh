@@ -4,22 +4,27 @@
 // Same operation as apd_prefill.cuh (AstrAI commit log of
 // csrc/kernels/attn_paged_decode.cu: prefill over the paged KV policy with the
 // unified causal_offset and 2-D / 3-D masks); this is the dense-contraction
-// design for B200:
+// design for B200.  Two kernels:
 //
-//  * A CTA owns M = 128 query rows of one (sequence b, kv head), the
+//  * prefill_tc2_kernel -- two 128-row Q tiles per CTA (used when a kv head has
+//    more than 128 query rows, D = 32, 64, 128); described with its code below.
+//  * prefill_tc_kernel -- one 128-row Q tile per CTA (D = 256, and fewer rows):
+//
+//  - A CTA owns M = 128 query rows of one (sequence b, kv head), the
 //    (query i, head-in-group hh) pairs in query-major order (row = i * g + hh),
 //    so the g heads of the kv head share every K/V tile.
-//  * Warp 8 (producer) resolves the pages of each tile of N keys and issues the
-//    TMA loads of the K and V tiles, 32 tokens x 64 dims per box, into two
-//    STAGES-deep rings laid out as the 128-byte-swizzled canonical operand
-//    layouts of the tensor core ([D/64][N][64] for both).
-//  * Warp 9 lane 0 (MMA issuer) runs S_j = Q K_j^T (M=128, N keys, K=D; both
+//  - Warp 8 (producer) resolves the pages of each tile of N keys and issues the
+//    TMA loads of the K and V tiles, 32 tokens per box, into two STAGES-deep
+//    rings laid out as the swizzled canonical operand layouts of the tensor core
+//    (OperandGeom: [D/64][N][64] blocks with the 128-byte swizzle, or for
+//    D = 32 one block of 64-byte rows with the 64-byte swizzle).
+//  - Warp 9 lane 0 (MMA issuer) runs S_j = Q K_j^T (M=128, N keys, K=D; both
 //    operands K-major) into one of two TMEM S buffers and O += P_j V_j
 //    (M=128, N=D, K=N keys; V is the MN-major B operand) into a TMEM O
 //    accumulator; tcgen05.commit arrives on the mbarriers that free the K/V
 //    stages and hand S and O to the softmax warps.  The next tile's Q K^T runs
 //    while the softmax warps work on the current one.
-//  * Warps 0-7 (softmax): TMEM lane r is query row r; warps w and w + 4 both
+//  - Warps 0-7 (softmax): TMEM lane r is query row r; warps w and w + 4 both
 //    read lane quadrant w (a warp may only reach the quadrant of its warp index
 //    mod 4) and each takes half of the row's columns, so every SM sub-partition
 //    runs two softmax warps.  A thread owns one row half: row maximum and sum
@@ -30,10 +35,11 @@
 //    2^8), write P = 2^(s * scale * log2 e - max) (MUFU ex2, the scale folded
 //    into one FFMA) as bf16 into shared memory in the swizzled A layout, and in
 //    the epilogue read O from TMEM, divide by the row sum and store bf16.
-//  * Every mbarrier wait is bounded; a wait that runs out raises a shared abort
-//    flag that every role polls, the producer and the MMA issuer then wait
-//    (bounded) for their own copies and MMAs in flight, and all warps meet
-//    before the TMEM columns are freed.
+//
+// In both, every mbarrier wait is bounded; a wait that runs out raises a shared
+// abort flag that every role polls, the producer and the MMA issuer then wait
+// (bounded) for their own copies and MMAs in flight, and all warps meet before
+// the TMEM columns are freed.
 #pragma once
 
 #include <cuda.h>
