@@ -150,7 +150,9 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         const int64_t workers = groups * ups;
         pl->workers = static_cast<int>(workers);
         pl->slots = 2 * workers;
-        pl->combine_ctas = static_cast<int>(s.units * s.rows_max);
+        // one group covers every position: no unit is split, every warp writes its
+        // output directly, and the call is a single launch (the unsplit path)
+        pl->combine_ctas = groups > 1 ? static_cast<int>(s.units * s.rows_max) : 0;
     } else {
         pl->mode = 1;
         pl->ksplit = num_splits;
