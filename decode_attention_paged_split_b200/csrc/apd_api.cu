@@ -504,9 +504,20 @@ bool gemv_stage_x(int M, int N, int K) {
            gemv_smem_bytes(M, K, kGemvStages, true) <= 232448;
 }
 
-int64_t gemv_workers(int sm_count, int64_t units) {
-    int64_t w = static_cast<int64_t>(sm_count) * kGemvWarps;
-    return std::max<int64_t>(1, std::min(w, units));
+// Whole m-tiles per warp when there are between one and four per SM and each is short
+// (K <= 2048, at most 64 KB of W per warp): no m-tile is split, every warp writes its
+// rows of y directly, and the sum kernel is not launched.  Graph-timed on the AstrAI-1B
+// shapes: gate_up (432 m-tiles) 8.5 -> 6.8 us; kv (16 m-tiles, too few warps) went
+// 5.9 -> 6.7 us and q (96) was even, so fewer m-tiles than SMs keep the split of units
+// over all warps, as do longer rows.
+bool gemv_whole_mtiles(int sm_count, int64_t mtiles, int64_t ktiles) {
+    return mtiles >= sm_count && mtiles <= static_cast<int64_t>(sm_count) * kGemvWarps && ktiles <= 8;
+}
+
+int64_t gemv_workers(int sm_count, int64_t mtiles, int64_t ktiles) {
+    if (gemv_whole_mtiles(sm_count, mtiles, ktiles)) return mtiles;
+    const int64_t w = static_cast<int64_t>(sm_count) * kGemvWarps;
+    return std::max<int64_t>(1, std::min(w, mtiles * ktiles));
 }
 
 // Workspace: [flags 256 B][fp32 partials, 2 per worker].
@@ -991,8 +1002,8 @@ size_t apd_gemv_workspace_size(int m, int n, int k) {
     }
     cudaGetLastError();
     const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
-    const int64_t units = mtiles * ((static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols);
-    return gemv_ws_bytes(gemv_workers(sm_count, units));
+    const int64_t ktiles = (static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols;
+    return gemv_ws_bytes(gemv_workers(sm_count, mtiles, ktiles));
 }
 
 int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, void* workspace,
@@ -1004,7 +1015,8 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    const int64_t workers = gemv_workers(dev->sm_count, g.units);
+    const int64_t workers = gemv_workers(dev->sm_count, g.mtiles, g.ktiles);
+    const bool whole = gemv_whole_mtiles(dev->sm_count, g.mtiles, g.ktiles);
     if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
     const bool xs = gemv_stage_x(g.M, g.N, g.K);
     auto kern = xs ? apd::gemv_kernel<kGemvStages, true> : apd::gemv_kernel<kGemvStages, false>;
@@ -1058,8 +1070,10 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     cfg2.stream = st;
     cfg2.attrs = pdl_attr;
     cfg2.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg2, apd::gemv_sum_kernel, gp);
-    if (e != cudaSuccess) return cuda_fail(e, "gemv_sum_kernel launch");
+    if (!whole) {  // some m-tiles are shared by two or more warps: add their partials
+        e = cudaLaunchKernelEx(&cfg2, apd::gemv_sum_kernel, gp);
+        if (e != cudaSuccess) return cuda_fail(e, "gemv_sum_kernel launch");
+    }
     return APD_OK;
 }
 

@@ -26,7 +26,8 @@ def check(y, x, w, what=""):
 
 
 @pytest.mark.parametrize("M", range(1, 9))
-@pytest.mark.parametrize("N,K", [(64, 256), (37, 1000), (1, 8), (300, 4104), (16, 264), (50, 1040)])
+@pytest.mark.parametrize("N,K", [(64, 256), (37, 1000), (1, 8), (300, 4104), (16, 264), (50, 1040), (3000, 1000),
+                                 (9470, 2048)])
 def test_gemv_shapes(M, N, K):
     c = workloads.gemv_case(M, N, K, seed=M * 7 + N)
     y = apd.gemv(c.x.cuda(), c.w.cuda())
