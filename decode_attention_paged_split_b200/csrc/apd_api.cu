@@ -398,6 +398,7 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     sp.out_sh = V.ost[1];
     sp.flags = reinterpret_cast<uint32_t*>(ws);
     sp.cum_out = reinterpret_cast<int32_t*>(ws + kWsAlign);
+    sp.zero_empty = (pl.mode == 0 && pl.combine_ctas == 0) ? 1 : 0;
     sp.o_part = reinterpret_cast<float*>(ws + ws_head_bytes(s));
     sp.ml_part = reinterpret_cast<float*>(ws + ws_head_bytes(s) +
                                           align_up(static_cast<size_t>(pl.slots) * s.rows_max * s.D * 4, kWsAlign));

@@ -59,6 +59,7 @@ struct SplitParams {
     float* o_part;      // [slots][rows_max][D]
     float* ml_part;     // [slots][rows_max][2]
     int32_t* cum_out;   // [B + 1] prefix sum of tiles per sequence (for the combine)
+    int32_t zero_empty;  // balanced mode with no combine kernel: write the rows of empty sequences
     uint32_t* flags;
     int32_t B, Hq, Hkv, g, HB, rows_max, P, NP, MP;
     int32_t mode;       // 0 balanced, 1 fixed
@@ -257,6 +258,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     const int units_per_seq = p.Hkv * p.HB;
     const int w = blockIdx.x * p.warps + warp;
     if (w >= p.num_workers) return;
+    if (p.zero_empty) {
+        // no combine kernel follows: the workers write the zero rows of empty sequences
+        for (int u = w; u < p.B * units_per_seq; u += p.num_workers) {
+            const int b = u / units_per_seq;
+            if (s_cum[b + 1] != s_cum[b]) continue;
+            const int ulz = u - b * units_per_seq, kvh = ulz / p.HB, hb = ulz - (ulz / p.HB) * p.HB;
+            write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
+        }
+    }
 
     // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-
     // sequence ul (kv head and head block).

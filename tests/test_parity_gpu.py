@@ -81,6 +81,37 @@ def test_all_sequences_empty(S):
     assert torch.all(out == 0)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_empty_sequence_when_one_group_covers_every_position(D):
+    """At most one tile per unit: a single worker group, no combine kernel; the
+    empty sequence's rows are still written (zeros)."""
+    w = small(24, B=1, Hq=8, Hkv=2, D=D, lens=(0,), P=32, pool=2, max_pages_per_seq=1)
+    out = DeviceProblem(w).run(0)
+    assert torch.all(out == 0)
+
+
+def test_small_workspace_one_group_with_empty_sequences():
+    """A workspace with room for one worker group only: every unit runs unsplit in
+    one launch, and empty sequences still come out as zeros."""
+    lens = (0, 100, 0, 37, 0)
+    w = small(25, B=len(lens), Hq=8, Hkv=2, D=64, lens=lens, pool=12, max_pages_per_seq=4)
+    dims = (w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim)
+    lo, hi = 256, apd.workspace_size(*dims, 0)
+    while lo < hi:  # the smallest workspace the balanced plan accepts
+        mid = (lo + hi) // 512 * 256
+        try:
+            apd.query_plan(*dims, 0, workspace_bytes=mid)
+            hi = mid
+        except apd.APDError:
+            lo = mid + 256
+    plan = apd.query_plan(*dims, 0, workspace_bytes=hi)
+    assert plan.num_workers == w.num_kv_heads and plan.combine_ctas == 0
+    ws = torch.zeros(hi, dtype=torch.uint8, device="cuda")
+    out = DeviceProblem(w).run(0, workspace=ws)
+    check_close(out, oracle.paged_decode(w), "one group, small workspace")
+    assert torch.all(out[0] == 0) and torch.all(out[2] == 0) and torch.all(out[4] == 0)
+
+
 def test_empty_batch():
     w = small(23, B=1, Hq=4, Hkv=1, D=64, lens=(5,), pool=2)
     dp = DeviceProblem(w)
