@@ -88,7 +88,19 @@ class _Options(ctypes.Structure):
         ("split_done_event", ctypes.c_void_p),
         ("disable_pdl", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+        ("host_seq_lens", ctypes.c_void_p),
     ]
+
+
+def _host_lens(host_seq_lens, batch: int):
+    """The host_seq_lens hint as a contiguous int32 CPU tensor of `batch` entries (kept
+    alive by the caller for the duration of the call), or None."""
+    if host_seq_lens is None:
+        return None
+    t = torch.as_tensor(host_seq_lens, dtype=torch.int32, device="cpu").contiguous()
+    if t.dim() != 1 or t.numel() != batch:
+        raise ValueError(f"host_seq_lens must hold {batch} lengths, got shape {tuple(t.shape)}")
+    return t
 
 
 class APDError(RuntimeError):
@@ -151,6 +163,9 @@ def _load():
     L.apd_read_device_flags.restype = ctypes.c_int
     L.apd_query_plan.argtypes = [ctypes.c_int] * 5 + [ctypes.c_size_t, ctypes.c_int, ctypes.POINTER(_Plan)]
     L.apd_query_plan.restype = ctypes.c_int
+    L.apd_query_plan_ex.argtypes = [ctypes.c_int] * 5 + [ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p,
+                                                         ctypes.c_int64, ctypes.POINTER(_Plan)]
+    L.apd_query_plan_ex.restype = ctypes.c_int
     L.apd_status_string.argtypes = [ctypes.c_int]
     L.apd_status_string.restype = ctypes.c_char_p
     L.apd_last_cuda_error.argtypes = []
@@ -216,7 +231,7 @@ def workspace_init(workspace: torch.Tensor, stream=None) -> None:
 def attn_paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, page_table: torch.Tensor,
                       seq_lens: torch.Tensor, out: torch.Tensor, scale: float, num_splits: int = 0,
                       workspace: torch.Tensor | None = None, stream=None, split_done_event=None,
-                      disable_pdl: bool = False) -> torch.Tensor:
+                      disable_pdl: bool = False, host_seq_lens=None) -> torch.Tensor:
     """out[b, h, :] = softmax(scale * q[b, h] . K_b^T) V_b over the paged cache; returns ``out``.
 
     q bf16 [B, Hq, D]; k_cache / v_cache bf16 [num_pages, page_size, Hkv, D] (any strides
@@ -224,8 +239,11 @@ def attn_paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
     ``workspace``: a device buffer of at least workspace_size(...) bytes; preallocate it once
     (allocating here, when it is None, makes the call not capturable in a CUDA graph).
     ``split_done_event``: optional torch.cuda.Event recorded right after the split kernel.
+    ``host_seq_lens``: optional host copy of the lengths (a planning hint with num_splits = 0;
+    see apd_launch_options.host_seq_lens: it changes the launch, never the result).
     """
     L = _load()
+    hl = _host_lens(host_seq_lens, q.shape[0])
     if workspace is None:
         workspace = alloc_workspace(q.shape[0], q.shape[1], k_cache.shape[2], q.shape[2], num_splits,
                                     device=q.device)
@@ -234,10 +252,11 @@ def attn_paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Ten
     st = _stream_handle(stream, q.device)
     ws_ptr = workspace.data_ptr()
     ws_bytes = workspace.numel() * workspace.element_size()
-    if split_done_event is None and not disable_pdl:
+    if split_done_event is None and not disable_pdl and hl is None:
         rc = L.apd_attn_paged_decode(*ptrs, ctypes.c_float(scale), int(num_splits), ws_ptr, ws_bytes, st)
     else:
         opts = _Options()
+        opts.host_seq_lens = hl.data_ptr() if hl is not None else None
         if split_done_event is not None:
             if not split_done_event.cuda_event:  # torch creates its events lazily, at the first record
                 split_done_event.record(torch.cuda.current_stream(q.device) if stream is None else stream)
@@ -266,7 +285,7 @@ def attn_paged_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: t
 
 def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
                        out: torch.Tensor, scale: float, num_splits: int = 0, workspace: torch.Tensor | None = None,
-                       stream=None) -> torch.Tensor:
+                       stream=None, host_seq_lens=None) -> torch.Tensor:
     """Decode attention over a contiguous KV cache: k / v bf16 [B, Lmax, Hkv, D] ("blhd"
     order; "bhld" storage is passed as the permuted view), token t of sequence b at
     k[b, t].  Same arguments and results as attn_paged_decode otherwise."""
@@ -274,9 +293,12 @@ def attn_contig_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_le
     if workspace is None:
         workspace = alloc_workspace(q.shape[0], q.shape[1], k.shape[2], q.shape[2], num_splits, device=q.device)
     descs = [_desc(t) for t in (q, k, v, seq_lens, out)]
-    rc = L.apd_attn_contig_decode(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale), int(num_splits),
-                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                                  _stream_handle(stream, q.device))
+    hl = _host_lens(host_seq_lens, q.shape[0])
+    opts = _Options()
+    opts.host_seq_lens = hl.data_ptr() if hl is not None else None
+    rc = L.apd_attn_contig_decode_ex(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale), int(num_splits),
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_handle(stream, q.device), ctypes.byref(opts))
     if rc:
         raise APDError(rc, "apd_attn_contig_decode")
     return out
@@ -360,10 +382,11 @@ class DecodeCall:
     the same buffers (a decode loop, a benchmark, a CUDA-graph capture).  Calling the
     object enqueues one decode call; the tensors' contents may change between calls,
     their storage, shapes and strides may not.  page_table=None selects the
-    contiguous-KV call (apd_attn_contig_decode)."""
+    contiguous-KV call (apd_attn_contig_decode).  ``host_seq_lens``: the planning hint of
+    attn_paged_decode, copied here and passed on every call."""
 
     def __init__(self, q, k_cache, v_cache, page_table, seq_lens, out, scale: float, num_splits: int = 0,
-                 workspace: torch.Tensor | None = None):
+                 workspace: torch.Tensor | None = None, host_seq_lens=None):
         if workspace is None:
             workspace = alloc_workspace(q.shape[0], q.shape[1], k_cache.shape[2], q.shape[2], num_splits,
                                         device=q.device)
@@ -375,6 +398,8 @@ class DecodeCall:
         self._head = tuple(ctypes.byref(d) for d in self._descs) + (
             ctypes.c_float(scale), int(num_splits), workspace.data_ptr(), workspace.numel() * workspace.element_size())
         self._opts = _Options()
+        self._host_lens = _host_lens(host_seq_lens, q.shape[0])
+        self._opts.host_seq_lens = self._host_lens.data_ptr() if self._host_lens is not None else None
         self._opts_ref = ctypes.byref(self._opts)
         self._lib = _load()
 
@@ -388,13 +413,14 @@ class DecodeCall:
 
     def __call__(self, stream=None, split_done_event=None) -> None:
         st = _stream_handle(stream, self.device)
-        if split_done_event is None:
+        if split_done_event is None and self._host_lens is None:
             fn = self._lib.apd_attn_contig_decode if self.contig else self._lib.apd_attn_paged_decode
             rc = fn(*self._head, st)
         else:
-            if not split_done_event.cuda_event:  # torch creates its events lazily, at the first record
+            if split_done_event is not None and not split_done_event.cuda_event:
+                # torch creates its events lazily, at the first record
                 split_done_event.record(torch.cuda.current_stream(self.device) if stream is None else stream)
-            self._opts.split_done_event = split_done_event.cuda_event
+            self._opts.split_done_event = split_done_event.cuda_event if split_done_event is not None else None
             fn = self._lib.apd_attn_contig_decode_ex if self.contig else self._lib.apd_attn_paged_decode_ex
             rc = fn(*self._head, st, self._opts_ref)
         if rc:
@@ -428,13 +454,17 @@ class Plan:
 
 
 def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,
-               workspace_bytes: int | None = None, sm_count: int = 0) -> Plan:
+               workspace_bytes: int | None = None, sm_count: int = 0, host_seq_lens=None,
+               max_seq_len: int = 0) -> Plan:
     """How the library would launch this problem (sm_count > 0: for a device with that
-    many SMs, computed on the host; 0: for the current CUDA device)."""
+    many SMs, computed on the host; 0: for the current CUDA device).  With
+    ``host_seq_lens`` (and ``max_seq_len`` = max_pages_per_seq * page_size, the clamp):
+    the plan of a call given that hint."""
     p = _Plan()
     wb = ctypes.c_size_t(-1).value if workspace_bytes is None else int(workspace_bytes)
-    rc = _load().apd_query_plan(batch, num_q_heads, num_kv_heads, head_dim, num_splits, wb, int(sm_count),
-                                ctypes.byref(p))
+    hl = _host_lens(host_seq_lens, batch)
+    rc = _load().apd_query_plan_ex(batch, num_q_heads, num_kv_heads, head_dim, num_splits, wb, int(sm_count),
+                                   hl.data_ptr() if hl is not None else None, int(max_seq_len), ctypes.byref(p))
     if rc:
         raise APDError(rc, "apd_query_plan")
     return Plan(**{name: int(getattr(p, name)) for name, _ in _Plan._fields_})

@@ -83,7 +83,7 @@ uint32_t q_tile_bytes(const Shape& s) { return static_cast<uint32_t>(align_up(st
 uint32_t stage_bytes(const Shape& s) { return 2u * apd::kTile * s.D * 2u + q_tile_bytes(s); }
 
 size_t smem_bytes(const Shape& s, int warps, int stages) {
-    const size_t meta = 8ull * warps * stages + 4ull * (2ull * s.B + 1);
+    const size_t meta = 8ull * warps * stages + 8 + 4ull * (2ull * s.B + 1);
     return align_up(meta, 16) + 1024 + static_cast<size_t>(warps) * stages * stage_bytes(s);
 }
 
@@ -115,8 +115,43 @@ struct Plan {
     size_t ws_needed;
 };
 
+// CTA-local plan (mode 2): CTA u owns unit u and its warps take equal parts of the unit's
+// tiles, merged in shared memory; a single launch, no partials in the workspace.
+void cta_local_plan(const Shape& s, Plan* pl) {
+    pl->mode = 2;
+    pl->ksplit = pl->warps;
+    pl->groups = 0;
+    pl->workers = static_cast<int>(s.units * pl->warps);
+    pl->ctas = static_cast<int>(s.units);
+    pl->slots = 0;
+    pl->combine_ctas = 0;
+}
+
+// Whether the CTA-local plan beats the balanced plan `pl` for these host-known lengths
+// (clamped to [0, len_cap] as the kernels clamp them).  Only when every unit gets a CTA
+// of its own on a distinct SM, and the longest unit is at most the balanced plan's
+// share per CTA plus about what the combine kernel costs: 3% and 1024 / D tiles.
+bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t* host_lens, int64_t len_cap) {
+    if (s.units > sm_count || pl.ctas < 1) return false;
+    // a part's (m, l) and accumulator rows go to its warp's ring once the stream ends
+    if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(pl.stages) * stage_bytes(s)) return false;
+    const int64_t ups = static_cast<int64_t>(s.Hkv) * s.HB;
+    int64_t total = 0, longest = 0;
+    for (int b = 0; b < s.B; ++b) {
+        const int64_t L = std::min<int64_t>(std::max<int32_t>(host_lens[b], 0), len_cap);
+        const int64_t n = (L + apd::kTile - 1) / apd::kTile;
+        total += n * ups;
+        longest = std::max(longest, n);
+    }
+    const int64_t share = (total + pl.ctas - 1) / pl.ctas;
+    return 32 * longest <= 33 * share + 32 * (1024 / s.D);
+}
+
 // tiles_bound: an upper bound on the number of tiles (host-known), or -1.
-int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl) {
+// host_lens: NULL, or the B sequence lengths as the host knows them (a planning hint;
+// the kernels read the device lengths), clamped to len_cap.
+int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl,
+              const int32_t* host_lens = nullptr, int64_t len_cap = 0) {
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
     const Traits t = traits_for(s.D);
     pl->stages = t.stages;
@@ -153,6 +188,9 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         // one group covers every position: no unit is split, every warp writes its
         // output directly, and the call is a single launch (the unsplit path)
         pl->combine_ctas = groups > 1 ? static_cast<int>(s.units * s.rows_max) : 0;
+        pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
+        if (host_lens && pl->combine_ctas > 0 && cta_local_wins(s, *pl, sm_count, host_lens, len_cap))
+            cta_local_plan(s, pl);
     } else {
         pl->mode = 1;
         pl->ksplit = num_splits;
@@ -163,7 +201,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         pl->slots = num_splits >= 2 ? workers : 0;
         pl->combine_ctas = num_splits >= 2 ? static_cast<int>(s.units * s.rows_max) : 0;
     }
-    pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
+    if (pl->mode != 2) pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
     pl->ws_needed = ws_bytes_for(s, pl->slots);
     if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
     return APD_OK;
@@ -861,7 +899,8 @@ int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl);
+    rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl,
+                   options ? options->host_seq_lens : nullptr, static_cast<int64_t>(V.MP) * V.P);
     if (rc) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (V.s.D) {
@@ -1096,7 +1135,15 @@ int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_str
 
 int apd_query_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
                    size_t workspace_bytes, int sm_count, apd_plan* plan) {
+    return apd_query_plan_ex(batch, num_q_heads, num_kv_heads, head_dim, num_splits, workspace_bytes, sm_count,
+                             nullptr, 0, plan);
+}
+
+int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
+                      size_t workspace_bytes, int sm_count, const int32_t* host_seq_lens, int64_t max_seq_len,
+                      apd_plan* plan) {
     if (!plan) return APD_ERR_NULL_POINTER;
+    if (host_seq_lens && max_seq_len < 0) return APD_ERR_ARGUMENT;
     Shape s;
     int rc = make_shape(batch, num_q_heads, num_kv_heads, head_dim, &s);
     if (rc) return rc;
@@ -1107,7 +1154,7 @@ int apd_query_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, i
         sm_count = dev->sm_count;
     }
     Plan pl;
-    rc = make_plan(s, num_splits, sm_count, workspace_bytes, -1, &pl);
+    rc = make_plan(s, num_splits, sm_count, workspace_bytes, -1, &pl, host_seq_lens, max_seq_len);
     if (rc) return rc;
     plan->mode = pl.mode;
     plan->num_workers = pl.workers;

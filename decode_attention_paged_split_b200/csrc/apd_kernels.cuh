@@ -180,6 +180,72 @@ __device__ __forceinline__ void write_zero_rows(const SplitParams& p, int b, int
     }
 }
 
+// CTA-local mode: CTA u owns unit u (sequence u / (Hkv * HB)); its warps take equal
+// parts of the unit's tiles, as fixed splits do, and merge them through shared memory.
+__device__ __forceinline__ int cta_local_tiles(const SplitParams& p, const int32_t* s_cum, int u) {
+    const int b = u / (p.Hkv * p.HB);
+    return s_cum[b + 1] - s_cum[b];
+}
+// Non-empty parts when n tiles are cut into at most W parts of ceil(n / min(W, n)) tiles.
+__device__ __forceinline__ int cta_local_parts(int n, int W) {
+    const int S = min(W, n);
+    const int c = (n + S - 1) / S;
+    return (n + c - 1) / c;
+}
+
+// Row stride (floats) of a CTA-local part's accumulator rows in shared memory: 8 floats of
+// padding put the 8 rows one warp store touches on different banks.
+template <int D>
+constexpr int kPartStride = D + 8;
+
+// Merge of the CTA-local parts of one unit: part k's (m, l) rows at ml_k = the start of
+// warp k's first ring stage, its accumulator rows [kMaxRows][kPartStride] (fp32) 128
+// bytes later.
+// Warp `part` of `nparts` merges rows part, part + nparts, ...:
+//   M = max_k m_k over parts with l_k > 0, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+template <int D>
+__device__ __noinline__ void cta_local_merge(const SplitParams& p, const uint8_t* ring0, uint32_t warp_bytes,
+                                                int b, int head0, int rows, int part, int nparts, int lane) {
+    constexpr int kVec = D / 32;  // consecutive columns per lane
+    for (int r = part; r < rows; r += nparts) {
+        float M = -INFINITY;
+        for (int k = 0; k < nparts; ++k) {
+            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
+            if (ml[2 * r + 1] > 0.f) M = fmaxf(M, ml[2 * r]);
+        }
+        float den = 0.f, acc[kVec];
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
+        for (int k = 0; k < nparts; ++k) {
+            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
+            if (!(ml[2 * r + 1] > 0.f)) continue;
+            const float wk = exp2f(ml[2 * r] - M);
+            den += wk * ml[2 * r + 1];
+            const float* a = ml + 2 * kMaxRows + r * kPartStride<D> + kVec * lane;
+            float v[kVec];  // this lane's kVec consecutive columns, in 16- (or 8-) byte loads
+            if constexpr (kVec % 4 == 0) {
+#pragma unroll
+                for (int e = 0; e < kVec; e += 4) *reinterpret_cast<float4*>(v + e) = *reinterpret_cast<const float4*>(a + e);
+            } else if constexpr (kVec == 2) {
+                *reinterpret_cast<float2*>(v) = *reinterpret_cast<const float2*>(a);
+            } else {
+                v[0] = a[0];
+            }
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) acc[e] += wk * v[e];
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        __nv_bfloat16* o = p.out + b * p.out_sb + (head0 + r) * p.out_sh + kVec * lane;
+        if constexpr (kVec == 1) {
+            o[0] = __float2bfloat16_rn(acc[0] * inv);
+        } else {
+#pragma unroll
+            for (int e = 0; e < kVec; e += 2)
+                *reinterpret_cast<uint32_t*>(o + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+        }
+    }
+}
+
 template <int D, int STAGES>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
@@ -193,7 +259,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 
     // ---- shared-memory carve-up: mbarriers, lengths, prefix sums, stage ring
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    int32_t* s_len = reinterpret_cast<int32_t*>(bars + p.warps * STAGES);
+    uint64_t* merge_bar = bars + p.warps * STAGES;  // CTA-local mode: the parts of the CTA's unit are in
+    int32_t* s_len = reinterpret_cast<int32_t*>(merge_bar + 1);
     int32_t* s_cum = s_len + B;
     const uint32_t meta_end = smem_u32(s_cum + B + 1);
     const uint32_t ring = (meta_end + 1023u) & ~1023u;
@@ -245,6 +312,13 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             run += s_cum[i];
             s_cum[i] = run;
         }
+        __syncwarp();
+        if (p.mode == 2 && lane == 0) {
+            // one arrival per non-empty part of this CTA's unit
+            const int n = cta_local_tiles(p, s_cum, blockIdx.x);
+            mbar_init(smem_u32(merge_bar), static_cast<uint32_t>(32 * (n >= 2 ? cta_local_parts(n, p.ksplit) : 1)));
+            fence_mbar_init();
+        }
     }
     __syncthreads();
     if (blockIdx.x == 0) {
@@ -253,7 +327,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // The combine kernel may start its launch now; it waits (griddepcontrol.wait)
     // for this whole grid to finish before it reads anything.
     pdl_launch_dependents();
-    // No CTA-wide barrier after this point: warps are independent workers.
+    // No CTA-wide barrier after this point: warps are independent workers (in the
+    // CTA-local mode the parts of the CTA's unit meet on an mbarrier, with a bounded wait).
 
     const int units_per_seq = p.Hkv * p.HB;
     const int w = blockIdx.x * p.warps + warp;
@@ -282,6 +357,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
         we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
     } else {
+        // fixed splits (mode 1), or the CTA-local mode (2: ksplit = warps, so unit u is
+        // CTA u and its parts are the CTA's warps)
         const int u = w / p.ksplit;
         const int s = w - u * p.ksplit;
         const int b = u / units_per_seq;
@@ -549,15 +626,19 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             } else {
                 const int64_t slot =
                     (p.mode == 0) ? (2 * static_cast<int64_t>(w) + (seg_start == ws ? 0 : 1)) : fixed_slot;
-                float* op = p.o_part + slot * p.rows_max * D;
-                float* mp = p.ml_part + slot * p.rows_max * 2;
+                // CTA-local mode: the part goes to this warp's (now idle) ring, as (m, l) rows
+                // then accumulator rows
+                float* const own = reinterpret_cast<float*>(smem + (wring - smem_u32(smem)));
+                float* op = (p.mode == 2) ? own + 2 * kMaxRows : p.o_part + slot * p.rows_max * D;
+                float* mp = (p.mode == 2) ? own : p.ml_part + slot * p.rows_max * 2;
+                const int ost = (p.mode == 2) ? kPartStride<D> : D;
 #pragma unroll
                 for (int nd = 0; nd < G::kNTiles; ++nd) {
                     const int d = 8 * nd + 2 * tq;
                     if (gq < rows)
-                        *reinterpret_cast<float2*>(op + gq * D + d) = make_float2(acc[nd][0], acc[nd][1]);
+                        *reinterpret_cast<float2*>(op + gq * ost + d) = make_float2(acc[nd][0], acc[nd][1]);
                     if (gq + 8 < rows)
-                        *reinterpret_cast<float2*>(op + (gq + 8) * D + d) = make_float2(acc[nd][2], acc[nd][3]);
+                        *reinterpret_cast<float2*>(op + (gq + 8) * ost + d) = make_float2(acc[nd][2], acc[nd][3]);
                 }
                 if (tq == 0) {
                     if (gq < rows) *reinterpret_cast<float2*>(mp + 2 * gq) = make_float2(m_lo, ll);
@@ -566,6 +647,20 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             }
         }
         if (i + 1 < we) advance_pos(s_cum, cb, cj, cn);
+    }
+    // CTA-local mode: part `warp` of the CTA's unit (recomputed here rather than kept
+    // live through the loop)
+    const int nparts = (p.mode == 2) ? cta_local_parts(cta_local_tiles(p, s_cum, blockIdx.x), p.ksplit) : 1;
+    if (nparts >= 2) {
+        // every lane's part rows are written: arrive, wait (bounded) for the other parts,
+        // and merge this warp's share of the rows
+        mbar_arrive(smem_u32(merge_bar));
+        if (!mbar_wait_bounded(smem_u32(merge_bar), 0u, kWaitTimeoutNs)) {
+            if (lane == 0) atomicOr(p.flags, kFlagTimeout);
+            return;
+        }
+        cta_local_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, cb,
+                           head0, rows, warp, nparts, lane);
     }
 }
 

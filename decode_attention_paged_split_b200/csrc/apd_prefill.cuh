@@ -62,9 +62,6 @@ struct PrefillParams {
     float scale_log2;
 };
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 
 template <int D, int STAGES>
 __global__ void __launch_bounds__(PrefillShape<D>::kThreads, 1)

@@ -185,11 +185,25 @@ int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const 
  *                     kernel in every replay of the graph.
  *   disable_pdl       nonzero: launch the combine kernel without programmatic
  *                     dependent launch.
+ *   host_seq_lens     NULL, or host memory holding the B sequence lengths as the
+ *                     caller knows them on the host (the values seq_lens holds on
+ *                     the device).  A planning hint for num_splits == 0, read during
+ *                     the call (and baked into a CUDA graph captured around it):
+ *                     when every (sequence, kv head, head block) unit can have a CTA
+ *                     of its own on a distinct SM and the longest unit is no longer
+ *                     than the balanced plan's share per CTA (within 3% plus about
+ *                     the combine kernel's cost), the call runs one kernel whose
+ *                     CTAs each own one unit and merge its parts in shared memory
+ *                     (plan mode 2), with no partials and no combine kernel.
+ *                     Otherwise the plan is the one without the hint.  The kernels
+ *                     always read the lengths from the device seq_lens, so a hint
+ *                     that differs from them changes the speed, never the result.
  */
 typedef struct apd_launch_options {
-    void* split_done_event; /* cudaEvent_t or NULL */
+    void* split_done_event;       /* cudaEvent_t or NULL */
     int32_t disable_pdl;
-    int32_t reserved;       /* must be 0 */
+    int32_t reserved;             /* must be 0 */
+    const int32_t* host_seq_lens; /* NULL or int32[B] in host memory */
 } apd_launch_options;
 
 int apd_attn_paged_decode_ex(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
@@ -369,7 +383,10 @@ int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stre
 /* apd_plan -- how a call with these arguments would be launched (for tests,
  * benchmarks and profiling). */
 typedef struct apd_plan {
-    int32_t mode;              /* 0 = balanced (num_splits == 0), 1 = fixed splits */
+    int32_t mode;              /* 0 = balanced (num_splits == 0), 1 = fixed splits,
+                                  2 = one CTA per unit, parts merged in shared memory
+                                  (num_splits == 0 with host lengths, see
+                                  apd_launch_options.host_seq_lens) */
     int32_t num_workers;       /* warps that each own a run of tiles             */
     int32_t grid_ctas;         /* CTAs of the split kernel                       */
     int32_t warps_per_cta;
@@ -388,6 +405,14 @@ typedef struct apd_plan {
  * queries the current CUDA device. */
 int apd_query_plan(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
                    size_t workspace_bytes, int sm_count, apd_plan* plan);
+
+/* apd_query_plan_ex -- apd_query_plan for a call given host_seq_lens (int32[batch] in
+ * host memory, or NULL) and the longest length the cache holds, max_seq_len =
+ * max_pages_per_seq * page_size (Lmax for a contiguous cache); lengths are clamped
+ * to [0, max_seq_len] as the kernels clamp them. */
+int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim, int num_splits,
+                      size_t workspace_bytes, int sm_count, const int32_t* host_seq_lens, int64_t max_seq_len,
+                      apd_plan* plan);
 
 /* Human-readable text for an apd_status (never NULL). */
 const char* apd_status_string(int status);

@@ -242,6 +242,61 @@ def test_plan_small_workspace_uses_fewer_workers():
     assert half.workspace_bytes <= full.workspace_bytes // 2
 
 
+def cta_local_expected(B, Hq, Hkv, D, lens, cap, sm=148):
+    """The CTA-local choice restated from its rule: every unit on its own SM, and the
+    longest unit within 3% plus 1024 / D tiles of the balanced plan's share per CTA."""
+    base = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
+    units = B * Hkv * base.head_blocks
+    tiles = [-(-min(max(L, 0), cap) // 32) for L in lens]
+    total = sum(tiles) * Hkv * base.head_blocks
+    share = -(-total // base.grid_ctas)
+    return units <= sm and base.combine_ctas > 0 and 32 * max(tiles) <= 33 * share + 32 * (1024 // D)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,lens,cap,want", [
+    (16, 32, 8, 128, [4096] * 16, 4096, 2),            # the LLaMA-8B-shaped batch: 128 units, one per CTA
+    (16, 32, 8, 128, [4000] * 15 + [4096], 4096, 2),   # within the slack
+    (16, 32, 8, 128, [2048] * 15 + [4096], 4096, 0),   # one long sequence: balanced
+    (2, 32, 8, 128, [131072] * 2, 131072, 0),          # 16 units on 128 CTAs: balanced
+    (128, 64, 8, 128, [1000] * 128, 1024, 0),          # 1024 units > SMs: balanced
+    (18, 32, 8, 128, [4096] * 18, 4096, 2),            # 144 units: 128 tiles each, under the 144-tile share
+    (20, 32, 8, 128, [4096] * 20, 4096, 0),            # 160 units > 148 SMs: balanced
+    (16, 32, 8, 128, [9000] * 16, 4096, 2),            # clamped to the cache: still uniform
+    (16, 32, 8, 128, [-5] * 8 + [4096] * 8, 4096, 0),  # negative lengths count as empty
+    (36, 32, 8, 64, [3000] * 36, 3008, 0),             # 288 units
+    (18, 16, 8, 64, [3000] * 18, 3008, 2),             # 144 units on 148 SMs (D = 64 uses every SM)
+    (4, 40, 2, 64, [1500] * 4, 1536, 0),               # 16 units: balanced spreads them wider
+    (1, 4, 1, 64, [256], 256, 2),                      # the tiny case: one unit, one launch
+])
+def test_plan_cta_local_from_host_lengths(B, Hq, Hkv, D, lens, cap, want):
+    pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=lens, max_seq_len=cap)
+    assert pl.mode == want
+    assert (want == 2) == cta_local_expected(B, Hq, Hkv, D, lens, cap)
+    if want == 2:
+        units = B * Hkv * pl.head_blocks
+        assert pl.grid_ctas == units and pl.num_workers == units * pl.warps_per_cta
+        assert pl.combine_ctas == 0 and pl.partial_slots == 0
+        assert pl.workspace_bytes <= apd.workspace_size(B, Hq, Hkv, D, 0)
+    else:
+        assert pl == apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
+
+
+def test_plan_host_lengths_do_not_change_fixed_splits():
+    lens = [4096] * 16
+    for splits in (1, 4):
+        assert apd.query_plan(16, 32, 8, 128, splits, sm_count=148, host_seq_lens=lens, max_seq_len=4096) == \
+            apd.query_plan(16, 32, 8, 128, splits, sm_count=148)
+
+
+def test_plan_host_lengths_checked():
+    with pytest.raises(ValueError):
+        apd.query_plan(16, 32, 8, 128, 0, sm_count=148, host_seq_lens=[4096] * 15, max_seq_len=4096)
+    p = apd._Plan()
+    lens = (ctypes.c_int32 * 2)(10, 10)
+    assert apd.lib().apd_query_plan_ex(2, 8, 2, 64, 0, ctypes.c_size_t(-1).value, 148, ctypes.cast(lens, ctypes.c_void_p),
+                                       -1, ctypes.byref(p)) == ARG
+
+
 def test_plan_workspace_too_small_for_fixed_splits():
     need = apd.workspace_size(16, 32, 8, 128, 4)
     with pytest.raises(apd.APDError) as e:

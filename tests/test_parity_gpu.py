@@ -339,3 +339,89 @@ def test_ragged_full_size():
     dp = DeviceProblem(w)
     check_close(dp.run(0), ref, "ragged auto")
     check_close(dp.run(16), ref, "ragged S=16")
+
+
+def test_llama8b_full_size_host_hint(llama):
+    """The benchmark's launch: the host lengths select one CTA per (sequence, kv head),
+    four parts merged in shared memory, one kernel."""
+    w, ref = llama
+    lens = w.seq_lens.tolist()
+    assert apd.query_plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, 0, host_seq_lens=lens,
+                          max_seq_len=w.page_table.shape[1] * w.page_size).mode == 2
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, 0)
+    apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws, host_seq_lens=lens)
+    check_close(dp.out, ref, "llama8b host hint")
+    assert apd.read_device_flags(ws) == 0
+
+
+# ---------------------------------------------------------------- host-length hint (CTA-local plan)
+def run_hinted(w, hint, stream=None):
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, 0)
+    if dp.contig:
+        apd.attn_contig_decode(dp.q, dp.k, dp.v, dp.seq_lens, dp.out, w.scale, 0, ws, stream=stream,
+                               host_seq_lens=hint)
+    else:
+        apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws, stream=stream,
+                              host_seq_lens=hint)
+    return dp.out, ws
+
+
+# Per head dim, a length whose tiles fit the CTA-local slack (1024 / D tiles) and cut into
+# every warp of the CTA (a ragged last tile included).
+HINT_LEN = {32: 1000, 64: 500, 128: 250, 256: 120}
+
+
+@pytest.mark.parametrize("D", workloads.SWEEP_HEAD_DIMS)
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (40, 2), (8, 8), (48, 1)])
+def test_host_hint_cta_local_matches_oracle(D, Hq, Hkv):
+    """Equal lengths: the hint selects the one-kernel plan (mode 2); g = 4, 20 (two head
+    blocks, the second partial), 1 and 48 (three)."""
+    L = HINT_LEN[D]
+    lens = [L] * 5
+    mp = -(-L // 32)
+    w = small(71, B=5, Hq=Hq, Hkv=Hkv, D=D, lens=lens, pool=5 * mp + 4, poison=True, max_pages_per_seq=mp)
+    pl = apd.query_plan(5, Hq, Hkv, D, 0, host_seq_lens=lens, max_seq_len=mp * 32)
+    assert pl.mode == 2 and pl.combine_ctas == 0
+    out, ws = run_hinted(w, lens)
+    check_close(out, oracle.paged_decode(w), f"hint D={D} {Hq}/{Hkv}")
+    assert apd.read_device_flags(ws) == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_host_hint_that_disagrees_with_the_device_lengths(D):
+    """The hint promises equal short lengths; the device lengths are ragged, empty and
+    long.  The plan follows the hint (mode 2), the result follows the device lengths."""
+    lens = (0, 1, 1000, 31, 257, 0, 640)
+    w = small(72, B=len(lens), Hq=16, Hkv=4, D=D, lens=lens, pool=80, poison=True, max_pages_per_seq=32)
+    hint = [HINT_LEN[D]] * len(lens)
+    assert apd.query_plan(len(lens), 16, 4, D, 0, host_seq_lens=hint, max_seq_len=32 * 32).mode == 2
+    out, ws = run_hinted(w, hint)
+    check_close(out, oracle.paged_decode(w), f"lying hint D={D}")
+    assert torch.all(out[0] == 0) and torch.all(out[5] == 0)
+
+
+def test_host_hint_contig_and_graph_replay():
+    lens = [250] * 6
+    w = workloads.make_contig(name="hint", seed=73, batch=6, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                              seq_lens=lens, lmax=256, layout="bhld")
+    ref = oracle.paged_decode(w)
+    out, _ = run_hinted(w, lens)
+    check_close(out, ref, "contig hint")
+    # the same call captured in a graph (the plan is baked in at capture) and replayed
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(6, 32, 8, 128, 0)
+    call = apd.DecodeCall(dp.q, dp.k, dp.v, None, dp.seq_lens, dp.out, w.scale, 0, ws, host_seq_lens=lens)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        call(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            call(s)
+    dp.out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    check_close(dp.out, ref, "contig hint graph")
