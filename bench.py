@@ -49,6 +49,7 @@ PREFILL_METRIC = "paged multi-query (prefill chunk) attention achieved TFLOP/s a
 PREFILL_WORKLOADS = ["prefill_llama8b_chunk"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
 PREFILL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_tc2_kernel_traffic.json")
+GEMV_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_kernel_traffic.json")
 
 
 def parse_args(argv=None):
@@ -256,6 +257,7 @@ def kernel_source_sha(sources=DECODE_KERNEL_SOURCES) -> str:
 
 
 PREFILL_KERNEL_SOURCES = ("apd_kernels.cuh", "apd_prefill.cuh", "apd_prefill_tc.cuh", "apd_ptx.cuh")
+GEMV_KERNEL_SOURCES = ("apd_gemv.cuh", "apd_kernels.cuh", "apd_ptx.cuh")
 
 
 def committed_traffic(workload: str, path=None, sources=DECODE_KERNEL_SOURCES):
@@ -755,6 +757,7 @@ def run_gemv(a):
 
     if rank == 0:
         peak, peak_src = peaks()
+        gplan = apd.gemv_query_plan(M, N, K)
         us = t_max / a.steps * 1e6
         line = {
             "metric": GEMV_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -764,9 +767,13 @@ def run_gemv(a):
                        "l2": f"{copies} weight copies used in turn ({copies * N * K * 2 / 1e6:.0f} MB > L2)",
                        "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
             "roofline": {"bound": "hbm", "achieved": per_call / (t_max / a.steps) / 1e9, "peak": peak, "unit": UNIT,
-                         "frac": per_call / (t_max / a.steps) / 1e9 / peak, "traffic": None, "peak_source": peak_src,
-                         "kernel": "gemv_kernel + gemv_sum_kernel (whole call)"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * a.steps, "clocks": clock_info,
+                         "frac": per_call / (t_max / a.steps) / 1e9 / peak,
+                         "traffic": committed_traffic(case.name, GEMV_TRAFFIC_FILE, GEMV_KERNEL_SOURCES),
+                         "peak_source": peak_src,
+                         "kernel": "gemv_kernel + gemv_sum_kernel (whole call)" if gplan["sum_ctas"]
+                         else "gemv_kernel (the whole call)"},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (2 if gplan["sum_ctas"] else 1) * a.steps,
+            "clocks": clock_info, "plan": gplan,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

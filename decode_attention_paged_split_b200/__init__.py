@@ -103,6 +103,18 @@ def _host_lens(host_seq_lens, batch: int):
     return t
 
 
+class _GemvPlan(ctypes.Structure):
+    _fields_ = [
+        ("workers", ctypes.c_int32),
+        ("grid_ctas", ctypes.c_int32),
+        ("warps_per_cta", ctypes.c_int32),
+        ("stages", ctypes.c_int32),
+        ("x_staged", ctypes.c_int32),
+        ("sum_ctas", ctypes.c_int32),
+        ("workspace_bytes", ctypes.c_int64),
+    ]
+
+
 class APDError(RuntimeError):
     """A non-zero apd_status returned by the library."""
 
@@ -156,6 +168,8 @@ def _load():
     L.apd_selftest_bounded_wait.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
+    L.apd_gemv_query_plan.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(_GemvPlan)]
+    L.apd_gemv_query_plan.restype = ctypes.c_int
     L.apd_gemv_bf16.argtypes = [T, T, T, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
     L.apd_gemv_bf16.restype = ctypes.c_int
     L.apd_read_device_flags.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
@@ -359,6 +373,16 @@ def gemv_workspace_size(m: int, n: int, k: int) -> int:
     if nb == 0:
         raise ValueError(f"invalid GEMV shape M={m}, N={n}, K={k}")
     return int(nb)
+
+
+def gemv_query_plan(m: int, n: int, k: int, sm_count: int = 0) -> dict:
+    """How apd_gemv_bf16 launches this shape (sm_count > 0: for a device with that many
+    SMs, on the host; 0: the current device)."""
+    p = _GemvPlan()
+    rc = _load().apd_gemv_query_plan(m, n, k, int(sm_count), ctypes.byref(p))
+    if rc:
+        raise APDError(rc, "apd_gemv_query_plan")
+    return {name: int(getattr(p, name)) for name, _ in _GemvPlan._fields_}
 
 
 def gemv(x: torch.Tensor, w: torch.Tensor, y: torch.Tensor | None = None, workspace: torch.Tensor | None = None,

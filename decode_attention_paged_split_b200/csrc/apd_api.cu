@@ -522,16 +522,23 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
 }
 
 // ---------------------------------------------------------------- decode projection (GEMV)
-constexpr int kGemvWarps = 4;
 constexpr int kGemvStages = 4;
+// Warps per CTA, and eighths of the SMs that get a CTA, for the two x paths.  With x staged
+// once per CTA (long weight streams), lm_head 100000 x 1536, graph-timed over M = 1..8
+// (4 warps on every SM -> 6 warps on 7/8 of them): 56.6 -> 50.1 us at M = 1, 57.6 -> 50.5
+// at M = 2, 58.5 -> 51.6 at M = 4, 58.9 -> 52.2 at M = 8; 5 warps on all SMs, 5 warps x 5
+// stages, 8 warps x 3 stages all measured between the two.  The shorter streams that load x
+// with every stage keep 4 warps on every SM (their stages are 12 KB).
+constexpr int gemv_warps(bool xs) { return xs ? 6 : 4; }
+constexpr int gemv_sm_eighths(bool xs) { return xs ? 7 : 8; }
 
 // Shared memory of the GEMV kernel: mbarriers, the staged x rows (xs) with a zero chunk,
 // alignment, the ring.  x is staged once per CTA when it fits with at least 2 stages.
 int gemv_x_pitch(int K) { return 16 * ((K / 8) | 1); }
 size_t gemv_smem_bytes(int M, int K, int stages, bool xs) {
     const size_t x = xs ? static_cast<size_t>(M) * gemv_x_pitch(K) + 16 + 16 : 0;
-    return 8ull * kGemvWarps * stages + x + 1024 +
-           static_cast<size_t>(kGemvWarps) * stages * (xs ? apd::kGemvWBytes : apd::kGemvStageBytes);
+    return 8ull * gemv_warps(xs) * stages + x + 1024 +
+           static_cast<size_t>(gemv_warps(xs)) * stages * (xs ? apd::kGemvWBytes : apd::kGemvStageBytes);
 }
 // x is staged once per CTA for long weight streams (W >= 64 MB) when it is at most 32 KB
 // (every CTA copies it from L2) and the full ring still fits.  Graph-timed on the
@@ -549,13 +556,13 @@ bool gemv_stage_x(int M, int N, int K) {
 // shapes: gate_up (432 m-tiles) 8.5 -> 6.8 us; kv (16 m-tiles, too few warps) went
 // 5.9 -> 6.7 us and q (96) was even, so fewer m-tiles than SMs keep the split of units
 // over all warps, as do longer rows.
-bool gemv_whole_mtiles(int sm_count, int64_t mtiles, int64_t ktiles) {
-    return mtiles >= sm_count && mtiles <= static_cast<int64_t>(sm_count) * kGemvWarps && ktiles <= 8;
+bool gemv_whole_mtiles(int sm_count, int64_t mtiles, int64_t ktiles, bool xs) {
+    return mtiles >= sm_count && mtiles <= static_cast<int64_t>(sm_count) * gemv_warps(xs) && ktiles <= 8;
 }
 
-int64_t gemv_workers(int sm_count, int64_t mtiles, int64_t ktiles) {
-    if (gemv_whole_mtiles(sm_count, mtiles, ktiles)) return mtiles;
-    const int64_t w = static_cast<int64_t>(sm_count) * kGemvWarps;
+int64_t gemv_workers(int sm_count, int64_t mtiles, int64_t ktiles, bool xs) {
+    if (gemv_whole_mtiles(sm_count, mtiles, ktiles, xs)) return mtiles;
+    const int64_t w = static_cast<int64_t>(sm_count) * gemv_sm_eighths(xs) / 8 * gemv_warps(xs);
     return std::max<int64_t>(1, std::min(w, mtiles * ktiles));
 }
 
@@ -1032,6 +1039,30 @@ int apd_attn_paged_prefill_ex(const apd_tensor* q, const apd_tensor* k_cache, co
     }
 }
 
+int apd_gemv_query_plan(int m, int n, int k, int sm_count, apd_gemv_plan* plan) {
+    if (!plan) return APD_ERR_NULL_POINTER;
+    if (m < 1 || m > APD_GEMV_MAX_M || n < 1 || k < 1) return APD_ERR_ARGUMENT;
+    if (sm_count <= 0) {
+        DeviceState* dev = nullptr;
+        const int rc = device_state(&dev);
+        if (rc) return rc;
+        sm_count = dev->sm_count;
+    }
+    const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
+    const int64_t ktiles = (static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols;
+    const bool xs = gemv_stage_x(m, n, k);
+    const int warps = gemv_warps(xs);
+    const int64_t workers = gemv_workers(sm_count, mtiles, ktiles, xs);
+    plan->workers = static_cast<int32_t>(workers);
+    plan->grid_ctas = static_cast<int32_t>((workers + warps - 1) / warps);
+    plan->warps_per_cta = warps;
+    plan->stages = kGemvStages;
+    plan->x_staged = xs ? 1 : 0;
+    plan->sum_ctas = gemv_whole_mtiles(sm_count, mtiles, ktiles, xs) ? 0 : static_cast<int32_t>((mtiles + 3) / 4);
+    plan->workspace_bytes = static_cast<int64_t>(gemv_ws_bytes(workers));
+    return APD_OK;
+}
+
 size_t apd_gemv_workspace_size(int m, int n, int k) {
     if (m < 1 || m > APD_GEMV_MAX_M || n < 1 || k < 1) return 0;
     int sm_count = kDefaultSmCount;
@@ -1043,7 +1074,7 @@ size_t apd_gemv_workspace_size(int m, int n, int k) {
     cudaGetLastError();
     const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
     const int64_t ktiles = (static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols;
-    return gemv_ws_bytes(gemv_workers(sm_count, mtiles, ktiles));
+    return gemv_ws_bytes(gemv_workers(sm_count, mtiles, ktiles, gemv_stage_x(m, n, k)));
 }
 
 int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, void* workspace,
@@ -1055,10 +1086,11 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    const int64_t workers = gemv_workers(dev->sm_count, g.mtiles, g.ktiles);
-    const bool whole = gemv_whole_mtiles(dev->sm_count, g.mtiles, g.ktiles);
-    if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
     const bool xs = gemv_stage_x(g.M, g.N, g.K);
+    const int warps = gemv_warps(xs);
+    const int64_t workers = gemv_workers(dev->sm_count, g.mtiles, g.ktiles, xs);
+    const bool whole = gemv_whole_mtiles(dev->sm_count, g.mtiles, g.ktiles, xs);
+    if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
     auto kern = xs ? apd::gemv_kernel<kGemvStages, true> : apd::gemv_kernel<kGemvStages, false>;
     const size_t smem = gemv_smem_bytes(g.M, g.K, kGemvStages, xs);
     {
@@ -1090,14 +1122,14 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     gp.mtiles = static_cast<int32_t>(g.mtiles);
     gp.ktiles = static_cast<int32_t>(g.ktiles);
     gp.num_workers = static_cast<int32_t>(workers);
-    gp.warps = kGemvWarps;
+    gp.warps = warps;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute pdl_attr[1];
     pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((workers + kGemvWarps - 1) / kGemvWarps));
-    cfg.blockDim = dim3(32 * kGemvWarps);
+    cfg.gridDim = dim3(static_cast<unsigned>((workers + warps - 1) / warps));
+    cfg.blockDim = dim3(32 * warps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = pdl_attr;

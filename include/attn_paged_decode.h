@@ -356,6 +356,26 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
                   size_t workspace_bytes, apd_stream_t stream);
 
 /*
+ * apd_gemv_query_plan -- how apd_gemv_bf16 launches an [M, K] x [N, K]^T product:
+ * the weight matrix is cut into units of 16 rows x 256 columns that `workers` warps
+ * share equally (or, with one to four 16-row tiles per SM and rows of at most 2048
+ * columns, each warp takes whole 16-row tiles).  sm_count > 0 plans for a device with
+ * that many SMs without touching CUDA; sm_count <= 0 queries the current device.
+ * Returns APD_ERR_ARGUMENT for M outside 1..APD_GEMV_MAX_M or N, K < 1.
+ */
+typedef struct apd_gemv_plan {
+    int32_t workers;        /* warps sharing the weight stream                          */
+    int32_t grid_ctas;      /* CTAs of the GEMV kernel                                  */
+    int32_t warps_per_cta;
+    int32_t stages;         /* async-copy ring depth per warp                           */
+    int32_t x_staged;       /* 1: x is copied once per CTA into shared memory            */
+    int32_t sum_ctas;       /* CTAs of the partial-sum kernel; 0 when it is not launched */
+    int64_t workspace_bytes;
+} apd_gemv_plan;
+
+int apd_gemv_query_plan(int m, int n, int k, int sm_count, apd_gemv_plan* plan);
+
+/*
  * apd_read_device_flags -- synchronise `stream`, copy the sticky APD_FLAG_* word
  * out of the workspace into *flags and, if `clear` is nonzero, reset it.  A
  * debugging / testing aid: it blocks the host, so it does not belong in a

@@ -425,3 +425,30 @@ def test_selftest_arguments_are_checked_before_any_launch():
     assert L.apd_selftest_bounded_wait(None, 1000, None) == NULLP
     assert L.apd_selftest_bounded_wait(FAKE, 0, None) == ARG
     assert L.apd_selftest_bounded_wait(FAKE, 2_000_000_000, None) == ARG
+
+
+# ---------------------------------------------------------------- GEMV planning
+@pytest.mark.parametrize("M,N,K", [(1, 100000, 1536), (8, 100000, 1536), (1, 6912, 1536), (3, 1536, 1536),
+                                   (1, 256, 1536), (8, 1536, 6912), (5, 50, 1040)])
+def test_gemv_plan(M, N, K):
+    p = apd.gemv_query_plan(M, N, K, 148)
+    mtiles, ktiles = -(-N // 16), -(-K // 256)
+    # x is staged once per CTA for weight streams of at least 64 MB; those run 6 warps on
+    # 7/8 of the SMs, the rest 4 warps on every SM
+    xs = N * K * 2 >= (64 << 20)
+    assert p["x_staged"] == int(xs)
+    assert p["warps_per_cta"] == (6 if xs else 4) and p["stages"] == 4
+    whole = mtiles >= 148 and mtiles <= 148 * p["warps_per_cta"] and ktiles <= 8
+    if whole:
+        assert p["workers"] == mtiles and p["sum_ctas"] == 0
+    else:
+        assert p["workers"] == min(148 * (7 if xs else 8) // 8 * p["warps_per_cta"], mtiles * ktiles)
+        assert p["sum_ctas"] == -(-mtiles // 4)
+    assert p["grid_ctas"] == -(-p["workers"] // p["warps_per_cta"])
+    assert p["workspace_bytes"] == 256 + -(-(2 * p["workers"] * 16 * 8 * 4) // 256) * 256
+
+
+def test_gemv_plan_rejects_bad_shapes():
+    for m, n, k in ((0, 16, 64), (9, 16, 64), (1, 0, 64), (1, 16, 0)):
+        with pytest.raises(apd.APDError):
+            apd.gemv_query_plan(m, n, k, 148)
