@@ -259,18 +259,33 @@ __device__ __forceinline__ void stage_q_tile(uint32_t q_s, const PrefillParams& 
                                              int R, int tid, int nthreads) {
     using O = OperandGeom<D>;
     constexpr int M = 128;
-    for (int idx = tid; idx < M * (D / 8); idx += nthreads) {
-        const int row = idx / (D / 8), ch = idx % (D / 8);
-        const int rq = row_first + row;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (rq < R) {
-            const int i = rq / p.g, hh = rq - i * p.g;
-            v = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
-                                                     ch * 8));
+    // Loads issued together before their stores: one round trip per batch rather than per
+    // 16-byte chunk (the shared store's memory clobber keeps the compiler from hoisting the
+    // next load).  Chunk workload, D = 128: 180.4 -> 170.8 us with 8; 16 measured 179 us.
+    constexpr int kBatch = 8;
+    for (int idx0 = tid; idx0 < M * (D / 8); idx0 += kBatch * nthreads) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int idx = idx0 + u * nthreads;
+            const int row = idx / (D / 8), ch = idx % (D / 8);
+            const int rq = row_first + row;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (idx < M * (D / 8) && rq < R) {
+                const int i = rq / p.g, hh = rq - i * p.g;
+                v[u] = __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + i * p.q_si + (kvh * p.g + hh) * p.q_sh +
+                                                            ch * 8));
+            }
         }
-        st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (M * O::kRowBytes) + row * O::kRowBytes +
-                                                 (O::swz(row, ch % O::kChunks) << 4)),
-                     v.x, v.y, v.z, v.w);
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int idx = idx0 + u * nthreads;
+            if (idx >= M * (D / 8)) break;
+            const int row = idx / (D / 8), ch = idx % (D / 8);
+            st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (M * O::kRowBytes) + row * O::kRowBytes +
+                                                     (O::swz(row, ch % O::kChunks) << 4)),
+                         v[u].x, v[u].y, v[u].z, v[u].w);
+        }
     }
 }
 
