@@ -111,6 +111,7 @@ class _GemvPlan(ctypes.Structure):
         ("stages", ctypes.c_int32),
         ("x_staged", ctypes.c_int32),
         ("sum_ctas", ctypes.c_int32),
+        ("cta_per_mtile", ctypes.c_int32),
         ("workspace_bytes", ctypes.c_int64),
     ]
 

@@ -535,10 +535,10 @@ constexpr int gemv_sm_eighths(bool xs) { return xs ? 7 : 8; }
 // Shared memory of the GEMV kernel: mbarriers, the staged x rows (xs) with a zero chunk,
 // alignment, the ring.  x is staged once per CTA when it fits with at least 2 stages.
 int gemv_x_pitch(int K) { return 16 * ((K / 8) | 1); }
-size_t gemv_smem_bytes(int M, int K, int stages, bool xs) {
+size_t gemv_smem_bytes(int M, int K, int stages, bool xs, int warps) {
     const size_t x = xs ? static_cast<size_t>(M) * gemv_x_pitch(K) + 16 + 16 : 0;
-    return 8ull * gemv_warps(xs) * stages + x + 1024 +
-           static_cast<size_t>(gemv_warps(xs)) * stages * (xs ? apd::kGemvWBytes : apd::kGemvStageBytes);
+    return 8ull * warps * stages + 8 + 16 + x + 1024 +
+           static_cast<size_t>(warps) * stages * (xs ? apd::kGemvWBytes : apd::kGemvStageBytes);
 }
 // x is staged once per CTA for long weight streams (W >= 64 MB) when it is at most 32 KB
 // (every CTA copies it from L2) and the full ring still fits.  Graph-timed on the
@@ -547,7 +547,7 @@ size_t gemv_smem_bytes(int M, int K, int stages, bool xs) {
 // 3 us to the copy that precedes their first MMA (gate_up M = 8: 8.5 -> 11.8 us).
 bool gemv_stage_x(int M, int N, int K) {
     return static_cast<int64_t>(N) * K * 2 >= (64ll << 20) && static_cast<int64_t>(M) * gemv_x_pitch(K) <= 32768 &&
-           gemv_smem_bytes(M, K, kGemvStages, true) <= 232448;
+           gemv_smem_bytes(M, K, kGemvStages, true, gemv_warps(true)) <= 232448;
 }
 
 // Whole m-tiles per warp when there are between one and four per SM and each is short
@@ -569,6 +569,46 @@ int64_t gemv_workers(int sm_count, int64_t mtiles, int64_t ktiles, bool xs) {
 // Workspace: [flags 256 B][fp32 partials, 2 per worker].
 size_t gemv_ws_bytes(int64_t workers) {
     return kWsAlign + align_up(static_cast<size_t>(2 * workers) * apd::kGemvRows * apd::kGemvXRows * 4, kWsAlign);
+}
+
+// One CTA per m-tile for short weight streams (at most 32 MB) with fewer m-tiles than SMs
+// and at least two k-tiles: up to 4 warps split the m-tile's k-tiles and add their parts
+// in shared memory, so the call is one kernel with no partials in global memory.
+bool gemv_cta_per_mtile(int sm_count, int M, int N, int K, int64_t mtiles, int64_t ktiles) {
+    return !gemv_stage_x(M, N, K) && mtiles <= sm_count && ktiles >= 2 &&
+           static_cast<int64_t>(N) * K * 2 <= (32ll << 20);
+}
+
+// The launch of one GEMV shape, as apd_gemv_bf16 makes it.
+struct GemvLaunch {
+    bool xs, whole, cta;
+    int warps;
+    int64_t workers, ctas, sum_ctas;
+    size_t smem, ws_bytes;
+};
+GemvLaunch gemv_launch(int sm_count, int M, int N, int K) {
+    GemvLaunch L;
+    const int64_t mtiles = (static_cast<int64_t>(N) + apd::kGemvRows - 1) / apd::kGemvRows;
+    const int64_t ktiles = (static_cast<int64_t>(K) + apd::kGemvCols - 1) / apd::kGemvCols;
+    L.xs = gemv_stage_x(M, N, K);
+    L.cta = gemv_cta_per_mtile(sm_count, M, N, K, mtiles, ktiles);
+    if (L.cta) {
+        L.whole = false;
+        L.warps = static_cast<int>(std::min<int64_t>(4, ktiles));
+        L.workers = mtiles * L.warps;
+        L.ctas = mtiles;
+        L.sum_ctas = 0;
+        L.ws_bytes = gemv_ws_bytes(0);
+    } else {
+        L.warps = gemv_warps(L.xs);
+        L.whole = gemv_whole_mtiles(sm_count, mtiles, ktiles, L.xs);
+        L.workers = gemv_workers(sm_count, mtiles, ktiles, L.xs);
+        L.ctas = (L.workers + L.warps - 1) / L.warps;
+        L.sum_ctas = L.whole ? 0 : (mtiles + 3) / 4;
+        L.ws_bytes = gemv_ws_bytes(L.workers);
+    }
+    L.smem = gemv_smem_bytes(M, K, kGemvStages, L.xs, L.warps);
+    return L;
 }
 
 // A bf16 row-major matrix [rows, K]: K contiguous, row stride a multiple of 8
@@ -1048,18 +1088,15 @@ int apd_gemv_query_plan(int m, int n, int k, int sm_count, apd_gemv_plan* plan) 
         if (rc) return rc;
         sm_count = dev->sm_count;
     }
-    const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
-    const int64_t ktiles = (static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols;
-    const bool xs = gemv_stage_x(m, n, k);
-    const int warps = gemv_warps(xs);
-    const int64_t workers = gemv_workers(sm_count, mtiles, ktiles, xs);
-    plan->workers = static_cast<int32_t>(workers);
-    plan->grid_ctas = static_cast<int32_t>((workers + warps - 1) / warps);
-    plan->warps_per_cta = warps;
+    const GemvLaunch L = gemv_launch(sm_count, m, n, k);
+    plan->workers = static_cast<int32_t>(L.workers);
+    plan->grid_ctas = static_cast<int32_t>(L.ctas);
+    plan->warps_per_cta = L.warps;
     plan->stages = kGemvStages;
-    plan->x_staged = xs ? 1 : 0;
-    plan->sum_ctas = gemv_whole_mtiles(sm_count, mtiles, ktiles, xs) ? 0 : static_cast<int32_t>((mtiles + 3) / 4);
-    plan->workspace_bytes = static_cast<int64_t>(gemv_ws_bytes(workers));
+    plan->x_staged = L.xs ? 1 : 0;
+    plan->sum_ctas = static_cast<int32_t>(L.sum_ctas);
+    plan->cta_per_mtile = L.cta ? 1 : 0;
+    plan->workspace_bytes = static_cast<int64_t>(L.ws_bytes);
     return APD_OK;
 }
 
@@ -1072,9 +1109,7 @@ size_t apd_gemv_workspace_size(int m, int n, int k) {
         if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && c > 0) sm_count = c;
     }
     cudaGetLastError();
-    const int64_t mtiles = (static_cast<int64_t>(n) + apd::kGemvRows - 1) / apd::kGemvRows;
-    const int64_t ktiles = (static_cast<int64_t>(k) + apd::kGemvCols - 1) / apd::kGemvCols;
-    return gemv_ws_bytes(gemv_workers(sm_count, mtiles, ktiles, gemv_stage_x(m, n, k)));
+    return gemv_launch(sm_count, m, n, k).ws_bytes;
 }
 
 int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y, void* workspace,
@@ -1086,13 +1121,9 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    const bool xs = gemv_stage_x(g.M, g.N, g.K);
-    const int warps = gemv_warps(xs);
-    const int64_t workers = gemv_workers(dev->sm_count, g.mtiles, g.ktiles, xs);
-    const bool whole = gemv_whole_mtiles(dev->sm_count, g.mtiles, g.ktiles, xs);
-    if (workspace_bytes < gemv_ws_bytes(workers)) return APD_ERR_WORKSPACE;
-    auto kern = xs ? apd::gemv_kernel<kGemvStages, true> : apd::gemv_kernel<kGemvStages, false>;
-    const size_t smem = gemv_smem_bytes(g.M, g.K, kGemvStages, xs);
+    const GemvLaunch L = gemv_launch(dev->sm_count, g.M, g.N, g.K);
+    if (workspace_bytes < L.ws_bytes) return APD_ERR_WORKSPACE;
+    auto kern = L.xs ? apd::gemv_kernel<kGemvStages, true> : apd::gemv_kernel<kGemvStages, false>;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!dev->gemv_attr_set) {  // the largest either variant uses, for both
@@ -1121,28 +1152,29 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
     gp.K = g.K;
     gp.mtiles = static_cast<int32_t>(g.mtiles);
     gp.ktiles = static_cast<int32_t>(g.ktiles);
-    gp.num_workers = static_cast<int32_t>(workers);
-    gp.warps = warps;
+    gp.num_workers = static_cast<int32_t>(L.workers);
+    gp.warps = L.warps;
+    gp.cta_per_mtile = L.cta ? 1 : 0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute pdl_attr[1];
     pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((workers + warps - 1) / warps));
-    cfg.blockDim = dim3(32 * warps);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(static_cast<unsigned>(L.ctas));
+    cfg.blockDim = dim3(32 * L.warps);
+    cfg.dynamicSmemBytes = L.smem;
     cfg.stream = st;
     cfg.attrs = pdl_attr;
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, gp, wmap, xmap);
     if (e != cudaSuccess) return cuda_fail(e, "gemv_kernel launch");
     cudaLaunchConfig_t cfg2 = {};
-    cfg2.gridDim = dim3(static_cast<unsigned>((g.mtiles + 3) / 4));
+    cfg2.gridDim = dim3(static_cast<unsigned>(L.sum_ctas));
     cfg2.blockDim = dim3(128);
     cfg2.stream = st;
     cfg2.attrs = pdl_attr;
     cfg2.numAttrs = 1;
-    if (!whole) {  // some m-tiles are shared by two or more warps: add their partials
+    if (L.sum_ctas > 0) {  // some m-tiles are shared by warps of different CTAs: add their partials
         e = cudaLaunchKernelEx(&cfg2, apd::gemv_sum_kernel, gp);
         if (e != cudaSuccess) return cuda_fail(e, "gemv_sum_kernel launch");
     }

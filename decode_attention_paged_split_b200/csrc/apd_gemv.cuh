@@ -57,6 +57,7 @@ struct GemvParams {
     int32_t mtiles;      // ceil(N / 16)
     int32_t ktiles;      // ceil(K / 256)
     int32_t num_workers, warps;
+    int32_t cta_per_mtile;  // 1: CTA b owns m-tile b, its warps split the k-tiles and add their parts in shared memory
 };
 
 // Byte offset of 16-byte chunk `ch` (8 columns) of row `row` in a unit staged as
@@ -85,9 +86,10 @@ __global__ void __launch_bounds__(32 * 8, 1)
     const int warp = threadIdx.x >> 5;
     const int w = blockIdx.x * p.warps + warp;
 
-    // shared memory: mbarriers | x rows (XS) | 16-byte zero chunk (XS) | stage ring
+    // shared memory: mbarriers | merge mbarrier | x rows (XS) | 16-byte zero chunk (XS) | stage ring
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    const uint32_t xs = (smem_u32(bars + p.warps * STAGES) + 15u) & ~15u;
+    const uint32_t merge_bar = smem_u32(bars + p.warps * STAGES);
+    const uint32_t xs = (merge_bar + 8u + 15u) & ~15u;
     const uint32_t xz = xs + (XS ? static_cast<uint32_t>(p.M * p.x_pitch) : 0u);
     const uint32_t ring = ((XS ? xz + 16u : xs) + 1023u) & ~1023u;
     if (threadIdx.x == 0) {
@@ -99,8 +101,23 @@ __global__ void __launch_bounds__(32 * 8, 1)
     pdl_launch_dependents();
 
     const int64_t total = static_cast<int64_t>(p.mtiles) * p.ktiles;
-    const int64_t ws = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w) * total) / p.num_workers) : 0;
-    const int64_t we = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w + 1) * total) / p.num_workers) : 0;
+    int64_t ws, we;
+    int nparts = 1;  // CTA-per-m-tile mode: warps with k-tiles (those that add their parts)
+    if (p.cta_per_mtile) {
+        // m-tile blockIdx.x; warp `warp` takes k-tiles [warp K / W, (warp + 1) K / W)
+        const int64_t t0 = static_cast<int64_t>(blockIdx.x) * p.ktiles;
+        ws = t0 + (static_cast<int64_t>(warp) * p.ktiles) / p.warps;
+        we = t0 + (static_cast<int64_t>(warp + 1) * p.ktiles) / p.warps;
+        nparts = p.ktiles < p.warps ? p.ktiles : p.warps;
+        if (threadIdx.x == 0) {
+            mbar_init(merge_bar, static_cast<uint32_t>(32 * nparts));
+            fence_mbar_init();
+        }
+        __syncthreads();
+    } else {
+        ws = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w) * total) / p.num_workers) : 0;
+        we = w < p.num_workers ? static_cast<int64_t>((static_cast<uint64_t>(w + 1) * total) / p.num_workers) : 0;
+    }
     const bool active = ws < we;
 
     const uint32_t bar0 = smem_u32(bars + warp * STAGES);
@@ -138,13 +155,27 @@ __global__ void __launch_bounds__(32 * 8, 1)
         for (int s = 0; s < STAGES; ++s) issue_next(s);
     }
     if constexpr (XS) {
+        // 8 loads in flight per thread before their stores (the store's memory clobber
+        // would otherwise hold each load until the previous chunk is stored)
         const int kch = p.K / 8;
-        for (int idx = threadIdx.x; idx < p.M * kch; idx += blockDim.x) {
-            const int r = idx / kch, c = idx - r * kch;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + r * p.ldx) + c);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xs + static_cast<uint32_t>(r * p.x_pitch + 16 * c)),
-                         "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                         : "memory");
+        constexpr int kBatch = 8;
+        for (int idx0 = threadIdx.x; idx0 < p.M * kch; idx0 += kBatch * blockDim.x) {
+            uint4 v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int idx = idx0 + u * static_cast<int>(blockDim.x);
+                const int r = idx / kch, c = idx - r * kch;
+                if (idx < p.M * kch) v[u] = __ldg(reinterpret_cast<const uint4*>(p.x + r * p.ldx) + c);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int idx = idx0 + u * static_cast<int>(blockDim.x);
+                if (idx >= p.M * kch) break;
+                const int r = idx / kch, c = idx - r * kch;
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(xs + static_cast<uint32_t>(r * p.x_pitch + 16 * c)),
+                             "r"(v[u].x), "r"(v[u].y), "r"(v[u].z), "r"(v[u].w)
+                             : "memory");
+            }
         }
         if (threadIdx.x == 0) st_shared_zero16(xz);
         __syncthreads();
@@ -224,6 +255,11 @@ __global__ void __launch_bounds__(32 * 8, 1)
                     if (m0 < p.M) p.y[m0 * p.y_sm + n_hi * p.y_sn] = __float2bfloat16_rn(c[2]);
                     if (m1 < p.M) p.y[m1 * p.y_sm + n_hi * p.y_sn] = __float2bfloat16_rn(c[3]);
                 }
+            } else if (p.cta_per_mtile) {
+                // this warp's part of the m-tile, [16 rows][8 m] fp32, into its ring (idle now)
+                float* dst = reinterpret_cast<float*>(smem + (wring - smem_u32(smem)));
+                *reinterpret_cast<float2*>(dst + gq * kGemvXRows + m0) = make_float2(c[0], c[1]);
+                *reinterpret_cast<float2*>(dst + (gq + 8) * kGemvXRows + m0) = make_float2(c[2], c[3]);
             } else {
                 const int64_t slot = 2 * static_cast<int64_t>(w) + (seg_first ? 0 : 1);
                 float* dst = p.part + slot * (kGemvRows * kGemvXRows);
@@ -231,6 +267,34 @@ __global__ void __launch_bounds__(32 * 8, 1)
                 *reinterpret_cast<float2*>(dst + (gq + 8) * kGemvXRows + m0) = make_float2(c[2], c[3]);
             }
             seg_first = false;
+        }
+    }
+    if (p.cta_per_mtile && nparts >= 2) {
+        // every lane's part is in shared memory: arrive; the last warp (never empty) waits,
+        // bounded, for the other parts and writes the m-tile's rows of y
+        mbar_arrive(merge_bar);
+        if (warp != p.warps - 1) return;
+        if (!mbar_wait_bounded(merge_bar, 0u, kWaitTimeoutNs)) {
+            if (lane == 0) atomicOr(p.flags, kFlagTimeout);
+            return;
+        }
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);  // lane -> 4 of the m-tile's 128 (row, m) values
+        for (int k = 0; k < p.warps; ++k) {
+            if ((k * p.ktiles) / p.warps == ((k + 1) * p.ktiles) / p.warps) continue;  // no k-tiles: no part
+            const float4 v = *reinterpret_cast<const float4*>(smem + (ring - smem_u32(smem)) +
+                                                              static_cast<uint32_t>(k) * STAGES * kStage + 16 * lane);
+            a.x += v.x;
+            a.y += v.y;
+            a.z += v.z;
+            a.w += v.w;
+        }
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int idx = 4 * lane + e;
+            const int row = idx / kGemvXRows, m = idx % kGemvXRows;
+            const int n = static_cast<int>(blockIdx.x) * kGemvRows + row;
+            if (n < p.N && m < p.M) p.y[m * p.y_sm + n * p.y_sn] = __float2bfloat16_rn(av[e]);
         }
     }
 }

@@ -359,7 +359,8 @@ int apd_gemv_bf16(const apd_tensor* x, const apd_tensor* w, const apd_tensor* y,
  * apd_gemv_query_plan -- how apd_gemv_bf16 launches an [M, K] x [N, K]^T product:
  * the weight matrix is cut into units of 16 rows x 256 columns that `workers` warps
  * share equally (or, with one to four 16-row tiles per SM and rows of at most 2048
- * columns, each warp takes whole 16-row tiles).  sm_count > 0 plans for a device with
+ * columns, each warp takes whole 16-row tiles; or, for weights of at most 32 MB with
+ * fewer 16-row tiles than SMs, each CTA takes one tile and splits its columns).  sm_count > 0 plans for a device with
  * that many SMs without touching CUDA; sm_count <= 0 queries the current device.
  * Returns APD_ERR_ARGUMENT for M outside 1..APD_GEMV_MAX_M or N, K < 1.
  */
@@ -370,6 +371,8 @@ typedef struct apd_gemv_plan {
     int32_t stages;         /* async-copy ring depth per warp                           */
     int32_t x_staged;       /* 1: x is copied once per CTA into shared memory            */
     int32_t sum_ctas;       /* CTAs of the partial-sum kernel; 0 when it is not launched */
+    int32_t cta_per_mtile;  /* 1: CTA b owns 16-row tile b; its warps split K and add their
+                               parts in shared memory (one kernel, no partials)        */
     int64_t workspace_bytes;
 } apd_gemv_plan;
 

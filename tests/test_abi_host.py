@@ -429,14 +429,27 @@ def test_selftest_arguments_are_checked_before_any_launch():
 
 # ---------------------------------------------------------------- GEMV planning
 @pytest.mark.parametrize("M,N,K", [(1, 100000, 1536), (8, 100000, 1536), (1, 6912, 1536), (3, 1536, 1536),
-                                   (1, 256, 1536), (8, 1536, 6912), (5, 50, 1040)])
+                                   (1, 256, 1536), (8, 1536, 6912), (5, 50, 1040), (2, 3000, 1000), (1, 64, 200),
+                                   (4, 2048, 16384), (1, 2360, 520)])
 def test_gemv_plan(M, N, K):
     p = apd.gemv_query_plan(M, N, K, 148)
     mtiles, ktiles = -(-N // 16), -(-K // 256)
     # x is staged once per CTA for weight streams of at least 64 MB; those run 6 warps on
     # 7/8 of the SMs, the rest 4 warps on every SM
-    xs = N * K * 2 >= (64 << 20)
+    # x is staged once per CTA for weight streams of at least 64 MB when its padded rows
+    # (16-byte chunks, an odd number per row) take at most 32 KB and fit beside the ring
+    x_bytes = M * 16 * ((K // 8) | 1)
+    xs = N * K * 2 >= (64 << 20) and x_bytes <= 32768 and 8 * 6 * 4 + 8 + 16 + x_bytes + 32 + 1024 + 6 * 4 * 8192 <= 232448
     assert p["x_staged"] == int(xs)
+    # short weight streams with fewer 16-row tiles than SMs: one CTA per tile, up to 4
+    # warps splitting its k-tiles, parts added in shared memory, one kernel
+    cta = not xs and mtiles <= 148 and ktiles >= 2 and N * K * 2 <= (32 << 20)
+    assert p["cta_per_mtile"] == int(cta)
+    if cta:
+        assert p["warps_per_cta"] == min(4, ktiles) and p["grid_ctas"] == mtiles
+        assert p["workers"] == mtiles * p["warps_per_cta"] and p["sum_ctas"] == 0
+        assert p["workspace_bytes"] == 256
+        return
     assert p["warps_per_cta"] == (6 if xs else 4) and p["stages"] == 4
     whole = mtiles >= 148 and mtiles <= 148 * p["warps_per_cta"] and ktiles <= 8
     if whole:

@@ -34,6 +34,22 @@ def test_gemv_shapes(M, N, K):
     check(y, c.x, c.w, f"M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 64, 520), (8, 1000, 6920), (3, 2360, 1040), (2, 16, 512), (5, 33, 8200),
+                                   (7, 1536, 6912)])
+def test_gemv_one_cta_per_mtile(M, N, K):
+    """Short weight streams with fewer 16-row tiles than SMs: one CTA per tile, whose warps
+    split its k-tiles (3 k-tiles on 3 warps, 28 with a K tail, 5, 2, 33 on 4 warps) and add
+    their parts in shared memory; N tails (1000, 33) and the full 148 tiles (2360)."""
+    plan = apd.gemv_query_plan(M, N, K)
+    assert plan["cta_per_mtile"] == 1 and plan["sum_ctas"] == 0
+    c = workloads.gemv_case(M, N, K, seed=N + K)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(apd.gemv_workspace_size(M, N, K), dtype=torch.uint8, device="cuda")
+    apd.gemv(c.x.cuda(), c.w.cuda(), y, ws)
+    check(y, c.x, c.w, f"cta per m-tile M={M} N={N} K={K}")
+    assert apd.read_device_flags(ws) == 0
+
+
 def test_gemv_strided_operands():
     c = workloads.gemv_case(5, 200, 512, seed=3)
     xb = torch.zeros(5, 640, dtype=torch.bfloat16, device="cuda")
