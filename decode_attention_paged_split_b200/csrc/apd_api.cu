@@ -603,6 +603,9 @@ GemvLaunch gemv_launch(int sm_count, int M, int N, int K) {
         L.warps = gemv_warps(L.xs);
         L.whole = gemv_whole_mtiles(sm_count, mtiles, ktiles, L.xs);
         L.workers = gemv_workers(sm_count, mtiles, ktiles, L.xs);
+        // whole m-tiles per warp: as few warps per CTA as put every SM to work (gate_up,
+        // 432 m-tiles: 3 warps on 144 SMs instead of 4 on 108, 6.82 -> 6.59 us)
+        if (L.whole) L.warps = static_cast<int>(std::min<int64_t>(L.warps, (mtiles + sm_count - 1) / sm_count));
         L.ctas = (L.workers + L.warps - 1) / L.warps;
         L.sum_ctas = L.whole ? 0 : (mtiles + 3) / 4;
         L.ws_bytes = gemv_ws_bytes(L.workers);

@@ -450,11 +450,14 @@ def test_gemv_plan(M, N, K):
         assert p["workers"] == mtiles * p["warps_per_cta"] and p["sum_ctas"] == 0
         assert p["workspace_bytes"] == 256
         return
-    assert p["warps_per_cta"] == (6 if xs else 4) and p["stages"] == 4
-    whole = mtiles >= 148 and mtiles <= 148 * p["warps_per_cta"] and ktiles <= 8
+    assert p["stages"] == 4
+    whole = mtiles >= 148 and mtiles <= 148 * (6 if xs else 4) and ktiles <= 8
     if whole:
+        # one warp per m-tile, as few warps per CTA as put every SM to work
+        assert p["warps_per_cta"] == min(6 if xs else 4, -(-mtiles // 148))
         assert p["workers"] == mtiles and p["sum_ctas"] == 0
     else:
+        assert p["warps_per_cta"] == (6 if xs else 4)
         assert p["workers"] == min(148 * (7 if xs else 8) // 8 * p["warps_per_cta"], mtiles * ktiles)
         assert p["sum_ctas"] == -(-mtiles // 4)
     assert p["grid_ctas"] == -(-p["workers"] // p["warps_per_cta"])
