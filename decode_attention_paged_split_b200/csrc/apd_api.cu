@@ -147,6 +147,18 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
     return 32 * longest <= 33 * share + 32 * (1024 / s.D);
 }
 
+// Warps of a combine CTA: enough for one batch of kCombineBatch partial slots per warp,
+// 4 to 16.  A unit has about groups / B partials in the balanced mode (each sequence's
+// share of the groups, plus the one it starts in) and num_splits in the fixed mode.
+// Measured (llama8b-shaped, L = 4096, graph-timed): 8 warps at 4 partials per unit cost
+// llama8b 45.9 -> 48.2 us and ragged 332 -> 345-353 us, so 4 stays the floor.
+int combine_warps(const Shape& s, const Plan& pl) {
+    const int64_t per_unit = pl.mode == 0 ? pl.groups / std::max(1, s.B) + 1 : pl.ksplit;
+    int w = 4;
+    while (w < 16 && static_cast<int64_t>(w) * apd::kCombineBatch < per_unit) w *= 2;
+    return w;
+}
+
 // tiles_bound: an upper bound on the number of tiles (host-known), or -1.
 // host_lens: NULL, or the B sequence lengths as the host knows them (a planning hint;
 // the kernels read the device lengths), clamped to len_cap.
@@ -508,14 +520,17 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
         cp.ksplit = pl.ksplit;
         cp.num_workers = pl.workers;
         cp.groups = pl.groups;
+        const int cw = combine_warps(s, pl);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
-        cfg.blockDim = dim3(32 * apd::kCombineWarps);
+        cfg.blockDim = dim3(32 * cw);
         cfg.dynamicSmemBytes = 0;
         cfg.stream = stream;
         cfg.attrs = pdl_attr;
         cfg.numAttrs = (use_pdl && !(opts && opts->split_done_event)) ? 1 : 0;
-        e = cudaLaunchKernelEx(&cfg, apd::combine_kernel<D>, cp);
+        e = cw == 16 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 16>, cp)
+            : cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 8>, cp)
+                      : cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 4>, cp);
         if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
     }
     return APD_OK;

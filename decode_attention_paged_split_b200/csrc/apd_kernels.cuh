@@ -664,7 +664,6 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     }
 }
 
-constexpr int kCombineWarps = 4;  // 8 measured slower (llama8b 45.9 -> 48.2 us, ragged 332 -> 345-353 us)
 constexpr int kCombineBatch = 4;  // partial slots whose loads a warp issues together
 
 // One CTA per (unit, head row).  Merges the row's partials:
@@ -673,9 +672,11 @@ constexpr int kCombineBatch = 4;  // partial slots whose loads a warp issues tog
 // The CTA's warps split the unit's partial slots and each keeps a running
 // (max, sum, acc) over its share, loading kCombineBatch slots at a time; each
 // lane owns float4 columns of the row.  The warps' states are merged through
-// shared memory.  In balanced mode it also writes zeros for empty sequences.
-template <int D>
-__global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(const __grid_constant__ CombineParams p) {
+// shared memory.  In balanced mode it also writes zeros for empty sequences.  W warps
+// (4, 8 or 16, from the partials a unit is expected to have: one batch per warp).
+template <int D, int W>
+__global__ void __launch_bounds__(32 * W) combine_kernel(const __grid_constant__ CombineParams p) {
+    constexpr int kCombineWarps = W;
     constexpr int kCols = D / 4;                 // float4 columns of a row
     constexpr int kPerLane = (kCols + 31) / 32;  // float4 columns per lane
     __shared__ float4 s_acc[kCombineWarps][kCols];
