@@ -4,7 +4,7 @@ One step = one decode-attention call (split kernel + combine kernel) over one
 batch of synthetic decode queries against a paged bf16 KV cache, through the
 C-ABI library.  Prints ONE JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|long|ragged|tiny]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|long|ragged|gqa32|tiny|...]
     python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host cores
 
 Metric: achieved HBM bandwidth over algorithmic bytes (KV bytes that must be read
@@ -41,7 +41,7 @@ import workloads  # noqa: E402
 METRIC = "paged decode attention achieved HBM GB/s (algorithmic KV+q+out bytes per call / time)"
 UNIT = "GB/s"
 DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000, "llama8b_contig": 20000,
-                 "long_contig": 5000}
+                 "long_contig": 5000, "gqa32": 10000}
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
 GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes per call / time)"
 GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
@@ -125,7 +125,7 @@ def make_instances(name: str, rank: int, count: int = 2):
     table) and independent values; the seed of the values differs per rank and instance."""
     gen = workloads.NAMED[name]
     base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262, "llama8b_contig": 8,
-            "long_contig": 131072}[name]
+            "long_contig": 131072, "gqa32": 32}[name]
     return [gen(seed=base, value_seed=base + 1000003 * rank + i) for i in range(count)]
 
 
@@ -620,7 +620,8 @@ def run_ours(a):
                      "mode_name": {0: "balanced + combine", 1: "fixed splits", 2: "one CTA per unit, single kernel"}
                      [plan.mode],
                      "workers": plan.num_workers, "ctas": plan.grid_ctas,
-                     "warps_per_cta": plan.warps_per_cta, "stages": plan.stages, "smem": plan.smem_bytes},
+                     "warps_per_cta": plan.warps_per_cta, "stages": plan.stages, "smem": plan.smem_bytes,
+                     "shared_kv_ring": bool(plan.shared_kv_ring)},
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

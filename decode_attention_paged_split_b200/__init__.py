@@ -80,6 +80,8 @@ class _Plan(ctypes.Structure):
         ("smem_bytes", ctypes.c_int64),
         ("partial_slots", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_int64),
+        ("shared_kv_ring", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
     ]
 
 
@@ -476,6 +478,7 @@ class Plan:
     smem_bytes: int
     partial_slots: int
     workspace_bytes: int
+    shared_kv_ring: int  # 1: a kv head's head-block warps read one K/V ring (balanced, g > 16)
 
 
 def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,
@@ -492,4 +495,4 @@ def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, n
                                    hl.data_ptr() if hl is not None else None, int(max_seq_len), ctypes.byref(p))
     if rc:
         raise APDError(rc, "apd_query_plan")
-    return Plan(**{name: int(getattr(p, name)) for name, _ in _Plan._fields_})
+    return Plan(**{name: int(getattr(p, name)) for name, _ in _Plan._fields_ if not name.startswith("reserved")})

@@ -56,6 +56,23 @@ Traits traits_for(int D) {
     }
 }
 
+// The shared-ring layout (balanced mode, g > 16): K/V stages per kv head and the most
+// warps per CTA; {0, 0} = not used for this head dim.  Measured on B200 (B = 16,
+// 268 MB of K/V, graph-timed): these warps per SM are latency-bound, so more warps beat
+// deeper rings.  D = 128, g = 32: 8 warps x 2 stages 64.3 us, 6 x 3 75.3 us, 4 x 3 or 4 x 4
+// 84-85 us, one ring per warp 97.8 us.  D = 32 keeps one ring per warp (71.6 us against
+// 77.1 shared): its short tiles leave a warp pair with too little work per wait.
+Traits share_traits_for(int D) {
+    switch (D) {
+        case 32: return {0, 0};
+        case 64: return {4, 8};
+        case 128: return {2, 8};
+        default: return {2, 4};
+    }
+}
+template <int D>
+constexpr int kShareStages = (D == 64) ? 4 : (D == 128) ? 2 : (D == 256) ? 2 : 0;
+
 bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
 
 struct Shape {
@@ -82,15 +99,22 @@ int make_shape(int B, int Hq, int Hkv, int D, Shape* s) {
 uint32_t q_tile_bytes(const Shape& s) { return static_cast<uint32_t>(align_up(static_cast<size_t>(s.rows_max) * s.D * 2, 1024)); }
 uint32_t stage_bytes(const Shape& s) { return 2u * apd::kTile * s.D * 2u + q_tile_bytes(s); }
 
-size_t smem_bytes(const Shape& s, int warps, int stages) {
-    const size_t meta = 8ull * warps * stages + 8 + 4ull * (2ull * s.B + 1);
-    return align_up(meta, 16) + 1024 + static_cast<size_t>(warps) * stages * stage_bytes(s);
+// share: the layout where the HB warps of a kv head share one K/V ring (the balanced mode
+// when g > 16): warps / HB K/V rings and `warps` Q rings, and an `empty` mbarrier per stage.
+size_t smem_bytes(const Shape& s, int warps, int stages, bool share = false) {
+    const size_t meta = 8ull * warps * stages * (share ? 2 : 1) + 8 + 4ull * (2ull * s.B + 1);
+    const size_t rings = share ? static_cast<size_t>(warps / s.HB) * stages * (2ull * apd::kTile * s.D * 2) +
+                                     static_cast<size_t>(warps) * stages * q_tile_bytes(s)
+                               : static_cast<size_t>(warps) * stages * stage_bytes(s);
+    return align_up(meta, 16) + 1024 + rings;
 }
 
-int warps_for(const Shape& s) {
-    const Traits t = traits_for(s.D);
+// The most warps per CTA that fit (a multiple of HB in the shared layout), or 0.
+int warps_for(const Shape& s, bool share = false) {
+    const Traits t = share ? share_traits_for(s.D) : traits_for(s.D);
+    if (t.stages < 1) return 0;
     for (int w = t.max_warps; w >= 1; --w)
-        if (smem_bytes(s, w, t.stages) <= kSmemLimit) return w;
+        if ((!share || w % s.HB == 0) && smem_bytes(s, w, t.stages, share) <= kSmemLimit) return w;
     return 0;
 }
 
@@ -110,6 +134,7 @@ int64_t slots_fitting(const Shape& s, size_t bytes) {
 
 struct Plan {
     int mode, ksplit, workers, groups, ctas, warps, stages, combine_ctas;
+    bool share;  // balanced mode, g > 16: a kv head's HB warps share one K/V ring
     size_t smem;
     int64_t slots;
     size_t ws_needed;
@@ -119,6 +144,10 @@ struct Plan {
 // tiles, merged in shared memory; a single launch, no partials in the workspace.
 void cta_local_plan(const Shape& s, Plan* pl) {
     pl->mode = 2;
+    pl->share = false;
+    pl->stages = traits_for(s.D).stages;
+    pl->warps = warps_for(s);
+    pl->smem = smem_bytes(s, pl->warps, pl->stages);
     pl->ksplit = pl->warps;
     pl->groups = 0;
     pl->workers = static_cast<int>(s.units * pl->warps);
@@ -134,7 +163,8 @@ void cta_local_plan(const Shape& s, Plan* pl) {
 bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t* host_lens, int64_t len_cap) {
     if (s.units > sm_count || pl.ctas < 1) return false;
     // a part's (m, l) and accumulator rows go to its warp's ring once the stream ends
-    if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(pl.stages) * stage_bytes(s)) return false;
+    if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(traits_for(s.D).stages) * stage_bytes(s))
+        return false;
     const int64_t ups = static_cast<int64_t>(s.Hkv) * s.HB;
     int64_t total = 0, longest = 0;
     for (int b = 0; b < s.B; ++b) {
@@ -170,12 +200,20 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
     pl->warps = warps_for(s);
     if (pl->warps < 1) return APD_ERR_TOO_LARGE;
     pl->smem = smem_bytes(s, pl->warps, pl->stages);
+    pl->share = false;
     if (num_splits == 0) {
         // Balanced mode: groups of Hkv * HB warps (one per kv head and head block)
         // share the sequence-tile positions equally; as many groups as fit the
         // device's resident warps, the known tile bound and the workspace.
         pl->mode = 0;
         pl->ksplit = 0;
+        if (s.HB > 1 && warps_for(s, true) > 0) {
+            // the HB warps of a kv head walk the same positions: one K/V stream for them
+            pl->share = true;
+            pl->stages = share_traits_for(s.D).stages;
+            pl->warps = warps_for(s, true);
+            pl->smem = smem_bytes(s, pl->warps, pl->stages, true);
+        }
         const int64_t ups = static_cast<int64_t>(s.Hkv) * s.HB;
         // D = 128 streams HBM with spare per-SM issue capacity: it runs fastest on
         // 7/8 of the SMs (measured on B200: 128 of 148 CTAs is 5-9% faster than 148
@@ -223,7 +261,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
-    bool smem_attr_set[4] = {false, false, false, false};
+    bool smem_attr_set[8] = {false, false, false, false, false, false, false, false};
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -419,8 +457,11 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
     constexpr int kStagesD = (D == 32 || D == 64) ? 4 : (D == 128 ? 3 : 2);
-    auto kern = apd::split_kernel<D, kStagesD>;
-    constexpr int kSlot = (D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3;
+    auto kern = apd::split_kernel<D, kStagesD, false>;
+    if constexpr (kShareStages<D> > 0) {
+        if (pl.share) kern = apd::split_kernel<D, kShareStages<D>, true>;
+    }
+    const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + (pl.share ? 4 : 0);
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!dev->smem_attr_set[kSlot]) {
@@ -1249,6 +1290,8 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
     plan->smem_bytes = static_cast<int64_t>(pl.smem);
     plan->partial_slots = pl.slots;
     plan->workspace_bytes = static_cast<int64_t>(pl.ws_needed);
+    plan->shared_kv_ring = pl.share ? 1 : 0;
+    plan->reserved0 = 0;
     return APD_OK;
 }
 

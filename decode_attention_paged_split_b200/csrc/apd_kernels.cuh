@@ -246,7 +246,14 @@ __device__ __noinline__ void cta_local_merge(const SplitParams& p, const uint8_t
     }
 }
 
-template <int D, int STAGES>
+// SHARE (balanced mode with g > 16, so HB = ceil(g / 16) head blocks per kv head): the HB
+// warps of one kv head, which walk the same positions in one CTA, share one K/V ring, which
+// the first of them (the leader) fills.  Before refilling a stage the leader waits on that
+// stage's `empty` mbarrier, on which the other HB - 1 warps arrive once they have read the
+// tile.  Each warp loads its own Q rows into a Q ring of its own.  Shared-memory layout:
+// [K/V rings, one per kv head of the CTA][Q rings, one per warp], so a CTA of HB warps
+// holds one K/V ring instead of HB.
+template <int D, int STAGES, bool SHARE>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
@@ -259,7 +266,8 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 
     // ---- shared-memory carve-up: mbarriers, lengths, prefix sums, stage ring
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* merge_bar = bars + p.warps * STAGES;  // CTA-local mode: the parts of the CTA's unit are in
+    uint64_t* empties = bars + p.warps * STAGES;  // SHARE: stage released by the followers
+    uint64_t* merge_bar = empties + (SHARE ? p.warps * STAGES : 0);  // CTA-local mode: the parts of the CTA's unit are in
     int32_t* s_len = reinterpret_cast<int32_t*>(merge_bar + 1);
     int32_t* s_cum = s_len + B;
     const uint32_t meta_end = smem_u32(s_cum + B + 1);
@@ -295,6 +303,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     if (tid == 0) s_cum[0] = 0;
     if (len_flags && blockIdx.x == 0) atomicOr(p.flags, len_flags);
     __syncthreads();
+    if (SHARE && warp == 1) {
+        // every warp's ring barriers, before any warp waits on another warp's
+        for (int i = lane; i < p.warps * STAGES; i += 32) {
+            mbar_init(smem_u32(bars + i), 1);
+            mbar_init(smem_u32(empties + i), static_cast<uint32_t>(p.HB - 1));
+        }
+        fence_mbar_init();
+    }
     if (warp == 0) {
         const int per = (B + 31) / 32;
         const int lo = 1 + lane * per;
@@ -383,19 +399,33 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     if (ws >= we) return;
 
     const uint32_t bar0 = smem_u32(bars + warp * STAGES);
-    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;
-    if (lane == 0) {
+    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;  // unshared layout
+    if constexpr (!SHARE) {
+        if (lane == 0) {
 #pragma unroll
-        for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
-        fence_mbar_init();
+            for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
     }
-    __syncwarp();
 
     const uint64_t pol_stream = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
 
     const int kvh = ul / p.HB;
     const int hb = ul - kvh * p.HB;
+    // Stage addresses.  Unshared: stage t of this warp is [K | V | Q] at wring + t * stage_bytes.
+    // SHARE: the K/V ring of this warp's kv head (its leader is hb warps lower in the same
+    // CTA: the host makes the warps per CTA a multiple of HB), and a Q ring of its own.
+    const bool follower = SHARE && hb > 0;
+    const uint32_t kv_step = SHARE ? 2 * G::kKVTileBytes : p.stage_bytes;
+    const uint32_t q_step = SHARE ? ((p.q_box_bytes + 1023u) & ~1023u) : p.stage_bytes;
+    const uint32_t kv_ring = SHARE ? ring + static_cast<uint32_t>(warp / p.HB) * STAGES * kv_step : wring;
+    const uint32_t q_ring = SHARE ? ring + static_cast<uint32_t>(p.warps / p.HB) * STAGES * kv_step +
+                                        static_cast<uint32_t>(warp) * STAGES * q_step
+                                  : wring + 2 * G::kKVTileBytes;
+    const uint32_t kv_bar0 = SHARE ? smem_u32(bars + (warp - hb) * STAGES) : bar0;
+    const uint32_t empty0 = smem_u32(empties + (warp - hb) * STAGES);
     const int head0 = kvh * p.g + kMaxRows * hb;
     const int rows = min(kMaxRows, p.g - kMaxRows * hb);
 
@@ -404,11 +434,34 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     int pb, pj, pn;
     decode_pos(ws, s_cum, B, pb, pj, pn);
     int wbase = ws;
-    int32_t pg_cur = fetch_page(p, s_cum, ws + lane, we);
-    int32_t pg_nxt = fetch_page(p, s_cum, ws + 32 + lane, we);
+    int32_t pg_cur = follower ? 0 : fetch_page(p, s_cum, ws + lane, we);
+    int32_t pg_nxt = follower ? 0 : fetch_page(p, s_cum, ws + 32 + lane, we);
 
     auto issue_next = [&](int stage) {
         if (pi >= we) return;
+        if (follower) {
+            // this warp's Q rows only; an expect of 0 bytes keeps one phase per tile
+            const bool qload = (pj == 0) || (pi == ws);
+            if (lane == 0) {
+                const uint32_t bar = bar0 + 8 * stage;
+                const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
+                mbar_arrive_expect_tx(bar, qload ? p.q_box_bytes : 0u);
+                if (qload) {
+                    if constexpr (D == 32) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
+                    else tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
+                }
+            }
+            ++pi;
+            if (pi < we) advance_pos(s_cum, pb, pj, pn);
+            return;
+        }
+        if (SHARE && pi - ws >= STAGES) {
+            // the followers have read the tile this stage held, STAGES tiles back
+            const int kk = pi - ws - STAGES;
+            if (!mbar_wait_bounded(empty0 + 8 * stage, static_cast<uint32_t>(kk / STAGES) & 1u, kWaitTimeoutNs) &&
+                lane == 0)
+                atomicOr(p.flags, kFlagTimeout);
+        }
         int off = pi - wbase;
         if (off >= 32) {
             pg_cur = pg_nxt;
@@ -422,16 +475,17 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         if (lane == 0) {
             if (page < 0 || page >= p.NP) atomicOr(p.flags, kFlagPageOOR);
             const uint32_t bar = bar0 + 8 * stage;
-            const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+            const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;
+            const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
             mbar_arrive_expect_tx(bar, 2 * G::kKVTileBytes + (qload ? p.q_box_bytes : 0u));
             if constexpr (D == 32) {
                 tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, page, pol_stream);
                 tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, pol_stream);
-                if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, pb, pol_keep);
+                if (qload) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
             } else {
                 tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, page, 0, pol_stream);
                 tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, 0, pol_stream);
-                if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, pb, 0, pol_keep);
+                if (qload) tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
             }
         }
         ++pi;
@@ -457,10 +511,12 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         const int k = i - ws;
         const int stage = k % STAGES;
         const uint32_t parity = static_cast<uint32_t>(k / STAGES) & 1u;
-        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+        const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;  // K, V
+        const uint32_t qbase_t = q_ring + static_cast<uint32_t>(stage) * q_step;  // this warp's Q
         const bool unit_start = (cj == 0) || (i == ws);
 
-        if (!mbar_wait_bounded(bar0 + 8 * stage, parity, kWaitTimeoutNs)) {
+        if (!mbar_wait_bounded(kv_bar0 + 8 * stage, parity, kWaitTimeoutNs) ||
+            (follower && !mbar_wait_bounded(bar0 + 8 * stage, parity, kWaitTimeoutNs))) {
             if (lane == 0) atomicOr(p.flags, kFlagTimeout);
             // Give the other copies in flight a bounded chance to land, then stop.
             for (int s = 0; s < STAGES; ++s) {
@@ -482,7 +538,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 #pragma unroll
             for (int nd = 0; nd < G::kNTiles; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
             // Q A-fragments: matrix m of ldmatrix.x4 = (rows 8*(m&1).., k chunk m>>1)
-            const uint32_t qbase = sbase + 2 * G::kKVTileBytes;
+            const uint32_t qbase = qbase_t;
             const int mi = lane >> 3;
             int qrow = (mi & 1) * 8 + (lane & 7);
             if (qrow >= p.rows_max) qrow = 0;  // stay inside the loaded box
@@ -601,6 +657,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         // before the async-proxy write, then the warp syncs before lane 0 issues.
         fence_proxy_async_smem();
         __syncwarp();
+        if (follower && lane == 0) mbar_arrive(empty0 + 8 * stage);  // the leader may refill it
         issue_next(stage);
 
         // ---- end of this unit's run in this worker: write output or a partial
@@ -650,7 +707,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     }
     // CTA-local mode: part `warp` of the CTA's unit (recomputed here rather than kept
     // live through the loop)
-    const int nparts = (p.mode == 2) ? cta_local_parts(cta_local_tiles(p, s_cum, blockIdx.x), p.ksplit) : 1;
+    const int nparts = (!SHARE && p.mode == 2) ? cta_local_parts(cta_local_tiles(p, s_cum, blockIdx.x), p.ksplit) : 1;
     if (nparts >= 2) {
         // every lane's part rows are written: arrive, wait (bounded) for the other parts,
         // and merge this warp's share of the rows

@@ -420,6 +420,12 @@ typedef struct apd_plan {
     int64_t smem_bytes;        /* dynamic shared memory of the split kernel      */
     int64_t partial_slots;
     int64_t workspace_bytes;   /* bytes the call needs                           */
+    int32_t shared_kv_ring;    /* 1: balanced mode with g > 16; the head_blocks
+                                  warps of a kv head sit in one CTA and read K/V
+                                  from one ring that the first of them fills, so
+                                  each K/V tile leaves HBM once (warps_per_cta is
+                                  then a multiple of head_blocks)               */
+    int32_t reserved0;
 } apd_plan;
 
 /* apd_query_plan -- fills *plan.  workspace_bytes: the size that will be passed

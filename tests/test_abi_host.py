@@ -201,7 +201,7 @@ def test_workspace_size_invalid_is_zero():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,D", [(16, 32, 8, 128), (2, 32, 8, 128), (128, 64, 8, 128), (4, 8, 8, 32),
-                                        (4, 32, 8, 256), (3, 40, 2, 64)])
+                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 128), (8, 96, 2, 128)])
 def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
     g = Hq // Hkv
@@ -219,6 +219,54 @@ def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     assert pl.smem_bytes <= 232448
     assert pl.workspace_bytes % 256 == 0
     assert pl.workspace_bytes == apd.lib().apd_workspace_size(B, Hq, Hkv, D, 0)
+
+
+# per head dim: async-copy stages and the most warps a CTA may have, with one ring per
+# warp and with a K/V ring shared by the head blocks of a kv head (None: not shared)
+_TRAITS = {32: (4, 8), 64: (4, 8), 128: (3, 6), 256: (2, 4)}
+_SHARE_TRAITS = {32: None, 64: (4, 8), 128: (2, 8), 256: (2, 4)}
+
+
+def _smem(B, D, rows, warps, stages, hb, shared):
+    """Dynamic shared memory of the split kernel: mbarriers (full, plus empty when the K/V
+    ring is shared), the merge barrier, lengths and prefix sums, 1 KB of alignment slack,
+    then the rings: per warp [K | V | Q] stages, or, shared, one K/V ring per kv head and
+    one Q ring per warp (K and V tiles are 32 tokens x D bf16, Q tiles 1 KB aligned)."""
+    meta = 8 * warps * stages * (2 if shared else 1) + 8 + 4 * (2 * B + 1)
+    kv = 2 * 32 * D * 2
+    q = -(-rows * D * 2 // 1024) * 1024
+    rings = (warps // hb * stages * kv + warps * stages * q) if shared else warps * stages * (kv + q)
+    return -(-meta // 16) * 16 + 1024 + rings
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 64, 2, 128), (4, 96, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
+                                        (4, 64, 2, 256), (4, 32, 8, 128), (4, 16, 1, 64)])
+def test_plan_shared_kv_ring(B, Hq, Hkv, D):
+    # balanced mode with g > 16: the head blocks of a kv head share one K/V ring, so the
+    # warps per CTA are the most that fit which are a multiple of the head blocks
+    g = Hq // Hkv
+    hb, rows = -(-g // 16), min(g, 16)
+
+    def fits(shared):
+        stages, max_warps = _SHARE_TRAITS[D] if shared else _TRAITS[D]
+        return stages, [w for w in range(max_warps, 0, -1)
+                        if (not shared or w % hb == 0) and _smem(B, D, rows, w, stages, hb, shared) <= 232448]
+
+    shared = hb > 1 and _SHARE_TRAITS[D] is not None and bool(fits(True)[1])
+    stages, ws = fits(shared)
+    pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
+    assert pl.shared_kv_ring == int(shared)
+    assert pl.warps_per_cta == ws[0] and pl.stages == stages
+    assert pl.smem_bytes == _smem(B, D, rows, ws[0], stages, hb, shared)
+    # fixed splits and the one-CTA-per-unit plan keep one ring per warp
+    stages, ws = fits(False)
+    fixed = apd.query_plan(B, Hq, Hkv, D, 2, sm_count=148)
+    assert fixed.shared_kv_ring == 0 and fixed.stages == stages and fixed.warps_per_cta == ws[0]
+    assert fixed.smem_bytes == _smem(B, D, rows, ws[0], stages, hb, False)
+    local = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=[4096] * B, max_seq_len=4096)
+    if local.mode == 2:
+        assert local.shared_kv_ring == 0 and local.stages == stages
+        assert local.smem_bytes == _smem(B, D, rows, local.warps_per_cta, stages, hb, False)
 
 
 @pytest.mark.parametrize("splits", [1, 2, 4, 148])

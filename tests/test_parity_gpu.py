@@ -129,6 +129,30 @@ def test_gqa_groups(Hq, Hkv, S):
     check_close(DeviceProblem(w).run(S), oracle.paged_decode(w), f"gqa {Hq}/{Hkv} S={S}")
 
 
+@pytest.mark.parametrize("D", [32, 64, 128, 256])
+@pytest.mark.parametrize("Hq,Hkv", [(40, 2), (64, 2), (48, 1), (80, 1)])
+@pytest.mark.parametrize("ws_div", [1, 16])
+def test_shared_kv_ring(D, Hq, Hkv, ws_div):
+    """Balanced mode with g = 20, 32, 48, 80 (2 to 5 head blocks per kv head): the head
+    blocks of a kv head read one K/V ring (except D = 32, and D = 256 with 5 head blocks).  Ragged lengths with an empty sequence and a
+    partial last tile, NaN-poisoned unused slots; ws_div = 16 gives a workspace a sixteenth
+    of the default, so fewer groups and runs of many tiles per warp (every stage's release
+    barrier goes through many phases)."""
+    lens = (1500, 0, 33, 777)
+    w = small(71, B=4, Hq=Hq, Hkv=Hkv, D=D, lens=lens, pool=90, poison=True)
+    dp = DeviceProblem(w)
+    default = apd.workspace_size(4, Hq, Hkv, D, 0)
+    ws = torch.zeros(default // ws_div // 256 * 256, dtype=torch.uint8, device="cuda")  # flags start clear
+    pl = apd.query_plan(4, Hq, Hkv, D, 0, workspace_bytes=ws.numel())
+    # D = 32 keeps one ring per warp; D = 256 takes at most 4 warps per CTA, so 5 head
+    # blocks keep one ring per warp too
+    shared = D != 32 and not (D == 256 and pl.head_blocks > 4)
+    assert pl.mode == 0 and pl.shared_kv_ring == int(shared)
+    assert pl.warps_per_cta % pl.head_blocks == 0 or not shared
+    check_close(dp.run(0, workspace=ws), oracle.paged_decode(w), f"shared ring D={D} {Hq}/{Hkv} ws/{ws_div}")
+    assert apd.read_device_flags(ws) == 0
+
+
 @pytest.mark.parametrize("P", [64, 128])
 @pytest.mark.parametrize("S", [1, 0, 3])
 def test_larger_pages(P, S):

@@ -434,11 +434,22 @@ def long_contig(seed: int = 131072, **kw) -> Workload:
     return make_contig(**args)
 
 
+def gqa32(seed: int = 32, **kw) -> Workload:
+    """B=16, 64 q heads / 2 kv heads (32 q heads per kv head: two 16-row head blocks),
+    D=128, L=16384 each (268 MB of K/V, the llama8b byte count), shuffled pool."""
+    args = dict(name="gqa32_b16_h64x2_d128_l16384", seed=seed, batch=16, num_q_heads=64,
+                num_kv_heads=2, head_dim=128, page_size=32, seq_lens=[16384] * 16, pool_pages=8192,
+                num_splits=0)
+    args.update(kw)
+    return make(**args)
+
+
 NAMED = {
     "tiny": tiny,
     "llama8b": llama8b,
     "long": long_context,
     "ragged": ragged,
+    "gqa32": gqa32,
     "llama8b_contig": llama8b_contig,
     "long_contig": long_contig,
 }
