@@ -262,16 +262,19 @@ GEMV_KERNEL_SOURCES = ("apd_gemv.cuh", "apd_kernels.cuh", "apd_ptx.cuh")
 
 def committed_traffic(workload: str, path=None, sources=DECODE_KERNEL_SOURCES):
     """dram read+write bytes per launch of the dominant kernel from a committed ncu capture
-    (default: the decode split kernel), or None when the capture is missing, for another
-    workload, or the kernel's device code changed since."""
+    (default: the decode split kernel), or None when no capture of this workload is
+    recorded or the kernel's device code changed since.  The file holds one record or a
+    list of records (one per workload)."""
     try:
         with open(path or TRAFFIC_FILE) as f:
-            t = json.load(f)
+            recs = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("kernel_source_sha") != kernel_source_sha(sources) or t.get("workload") != workload:
-        return None
-    return t.get("dram_bytes_per_launch")
+    sha = kernel_source_sha(sources)
+    for t in recs if isinstance(recs, list) else [recs]:
+        if t.get("kernel_source_sha") == sha and t.get("workload") == workload:
+            return t.get("dram_bytes_per_launch")
+    return None
 
 
 def time_steps(insts, stream, steps, split_events=False):

@@ -109,3 +109,10 @@ def test_traffic_lookup_is_tied_to_the_kernel_source(tmp_path, monkeypatch):
     assert bench.committed_traffic("long") is None
     f.write_text(json.dumps({"kernel_source_sha": "0" * 16, "workload": "llama8b", "dram_bytes_per_launch": 123}))
     assert bench.committed_traffic("llama8b") is None
+    # one record per workload in a list
+    sha = bench.kernel_source_sha()
+    f.write_text(json.dumps([{"kernel_source_sha": sha, "workload": "llama8b", "dram_bytes_per_launch": 5},
+                             {"kernel_source_sha": "0" * 16, "workload": "gqa32", "dram_bytes_per_launch": 6},
+                             {"kernel_source_sha": sha, "workload": "long", "dram_bytes_per_launch": 7}]))
+    assert bench.committed_traffic("llama8b") == 5 and bench.committed_traffic("long") == 7
+    assert bench.committed_traffic("gqa32") is None and bench.committed_traffic("ragged") is None
