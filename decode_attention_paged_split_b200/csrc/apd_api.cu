@@ -261,7 +261,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
-    bool smem_attr_set[8] = {false, false, false, false, false, false, false, false};
+    bool smem_attr_set[12] = {};  // split kernel: head dim x {plain ring, shared ring, CTA-local at D = 128}
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -457,11 +457,24 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
     constexpr int kStagesD = (D == 32 || D == 64) ? 4 : (D == 128 ? 3 : 2);
-    auto kern = apd::split_kernel<D, kStagesD, false>;
+    // the lean per-tile form everywhere but D = 256 and the CTA-local plan at D = 128
+    // (the kernel's LEAN parameter lists the measurements)
+    constexpr bool kLeanD = D != 256;
+    auto kern = apd::split_kernel<D, kStagesD, false, kLeanD>;
+    int variant = 0;
     if constexpr (kShareStages<D> > 0) {
-        if (pl.share) kern = apd::split_kernel<D, kShareStages<D>, true>;
+        if (pl.share) {
+            kern = apd::split_kernel<D, kShareStages<D>, true, kLeanD>;
+            variant = 1;
+        }
     }
-    const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + (pl.share ? 4 : 0);
+    if constexpr (D == 128) {
+        if (pl.mode == 2) {
+            kern = apd::split_kernel<D, kStagesD, false, false>;
+            variant = 2;
+        }
+    }
+    const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + 4 * variant;
     {
         std::lock_guard<std::mutex> lock(g_mu);
         if (!dev->smem_attr_set[kSlot]) {

@@ -253,7 +253,7 @@ __device__ __noinline__ void cta_local_merge(const SplitParams& p, const uint8_t
 // tile.  Each warp loads its own Q rows into a Q ring of its own.  Shared-memory layout:
 // [K/V rings, one per kv head of the CTA][Q rings, one per warp], so a CTA of HB warps
 // holds one K/V ring instead of HB.
-template <int D, int STAGES, bool SHARE>
+template <int D, int STAGES, bool SHARE, bool LEAN>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
@@ -429,10 +429,29 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     const int head0 = kvh * p.g + kMaxRows * hb;
     const int rows = min(kMaxRows, p.g - kMaxRows * hb);
 
+    // LEAN: the lean per-tile form, which trims the instructions of a tile:
+    // - the row sums of the bf16 weights come from an mma against a B of ones;
+    // - 2^x is the SFU instruction;
+    // - full tiles skip the masking selects;
+    // - the rescale of the accumulators is skipped while no row's max grows;
+    // - the page slot is a running cursor.
+    // The plain form instead keeps:
+    // - per-thread row sums, with the quad's partial sums added at the unit's end;
+    // - exp2f;
+    // - masking and rescale on every tile.
+    // The host picks the form by measurement (B200, 268 MB of K/V, CUDA-graph replays):
+    // - lean: D = 32 and 64, and D = 128 in the balanced and fixed plans (7-15% faster
+    //   where per-tile latency binds);
+    // - plain: D = 256, which sits at the 255-register cap (the lean form measured 2-3%
+    //   slower there), and the CTA-local plan at D = 128 (the lean form measured 1% slower
+    //   on the llama8b shape).
+    constexpr bool kLean = LEAN;
+
     // ---- producer state: next position to issue, its cursor, page-table window
     int pi = ws;
     int pb, pj, pn;
     decode_pos(ws, s_cum, B, pb, pj, pn);
+    int pslot = (pj * kTile) % p.P;  // token slot of tile pj in its page (lean: stepped below)
     int wbase = ws;
     int32_t pg_cur = follower ? 0 : fetch_page(p, s_cum, ws + lane, we);
     int32_t pg_nxt = follower ? 0 : fetch_page(p, s_cum, ws + 32 + lane, we);
@@ -470,7 +489,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             pg_nxt = fetch_page(p, s_cum, wbase + 32 + lane, we);
         }
         const int32_t page = __shfl_sync(0xffffffffu, pg_cur, off);
-        const int slot = (pj * kTile) % p.P;
+        const int slot = kLean ? pslot : (pj * kTile) % p.P;
         const bool qload = (pj == 0) || (pi == ws);
         if (lane == 0) {
             if (page < 0 || page >= p.NP) atomicOr(p.flags, kFlagPageOOR);
@@ -489,7 +508,10 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             }
         }
         ++pi;
-        if (pi < we) advance_pos(s_cum, pb, pj, pn);
+        if (pi < we) {
+            advance_pos(s_cum, pb, pj, pn);
+            if constexpr (kLean) pslot = (pj == 0 || pslot + kTile == p.P) ? 0 : pslot + kTile;
+        }
     };
 
 #pragma unroll
@@ -505,7 +527,9 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
 
     uint32_t qf[G::kSteps][4];
     float acc[G::kNTiles][4];
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+    float accl[4];  // row sums: rows gq in [0], [1] and gq + 8 in [2], [3]
+    float m_lo = -INFINITY, m_hi = -INFINITY;
+    constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
 
     for (int i = ws; i < we; ++i) {
         const int k = i - ws;
@@ -534,7 +558,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
             seg_start = i;
             j_start = cj;
             m_lo = m_hi = -INFINITY;
-            l_lo = l_hi = 0.f;
+            accl[0] = accl[1] = accl[2] = accl[3] = 0.f;
 #pragma unroll
             for (int nd = 0; nd < G::kNTiles; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
             // Q A-fragments: matrix m of ldmatrix.x4 = (rows 8*(m&1).., k chunk m>>1)
@@ -574,6 +598,16 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         // ---- mask tokens past the sequence end; tail V rows are zeroed so that
         // 0 * (stale or NaN) never reaches the accumulator
         const int valid = min(kTile, s_len[cb] - kTile * cj);
+        auto mask_and_scale = [&]() {
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const int t0 = 8 * nt + 2 * tq;
+                s[nt][0] = (t0 < valid) ? s[nt][0] * p.scale_log2 : -INFINITY;
+                s[nt][1] = (t0 + 1 < valid) ? s[nt][1] * p.scale_log2 : -INFINITY;
+                s[nt][2] = (t0 < valid) ? s[nt][2] * p.scale_log2 : -INFINITY;
+                s[nt][3] = (t0 + 1 < valid) ? s[nt][3] * p.scale_log2 : -INFINITY;
+            }
+        };
         if (valid < kTile) {
             const uint32_t vb = sbase + G::kKVTileBytes;
             for (int idx = lane; idx < (kTile - valid) * G::kChunks; idx += 32) {
@@ -582,15 +616,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
                 st_shared_zero16(vb + G::chunk_off(r, ch, kTile));
             }
             __syncwarp();
-        }
+            if constexpr (kLean) mask_and_scale();
+        } else if constexpr (kLean) {
+            // a full tile: no token to mask
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int t0 = 8 * nt + 2 * tq;
-            s[nt][0] = (t0 < valid) ? s[nt][0] * p.scale_log2 : -INFINITY;
-            s[nt][1] = (t0 + 1 < valid) ? s[nt][1] * p.scale_log2 : -INFINITY;
-            s[nt][2] = (t0 < valid) ? s[nt][2] * p.scale_log2 : -INFINITY;
-            s[nt][3] = (t0 + 1 < valid) ? s[nt][3] * p.scale_log2 : -INFINITY;
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
         }
+        if constexpr (!kLean) mask_and_scale();
 
         // ---- online softmax (rows gq and gq + 8 of the head tile)
         float mx_lo = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
@@ -603,35 +637,68 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
         const float mn_lo = fmaxf(m_lo, mx_lo);  // finite: every tile has >= 1 valid token
         const float mn_hi = fmaxf(m_hi, mx_hi);
-        const float alpha_lo = exp2f(m_lo - mn_lo);
-        const float alpha_hi = exp2f(m_hi - mn_hi);
-        m_lo = mn_lo;
-        m_hi = mn_hi;
-
         uint32_t pa[2][4];
-        float rs_lo = 0.f, rs_hi = 0.f;
+        if constexpr (kLean) {
+            // Rescale only when some row's running max grew.  Otherwise alpha would be
+            // 2^0 = 1 exactly, so skipping is exact, and after a sequence's first tiles the
+            // maxima rarely move.
+            if (__any_sync(0xffffffffu, (mn_lo != m_lo) || (mn_hi != m_hi))) {
+                const float alpha_lo = ex2_approx(m_lo - mn_lo);  // 0 on the unit's first tile
+                const float alpha_hi = ex2_approx(m_hi - mn_hi);
+                m_lo = mn_lo;
+                m_hi = mn_hi;
+                accl[0] *= alpha_lo;
+                accl[1] *= alpha_lo;
+                accl[2] *= alpha_hi;
+                accl[3] *= alpha_hi;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int nt = 2 * kk + h;
-                const uint32_t plo = pack_bf16x2(exp2f(s[nt][0] - mn_lo), exp2f(s[nt][1] - mn_lo));
-                const uint32_t phi = pack_bf16x2(exp2f(s[nt][2] - mn_hi), exp2f(s[nt][3] - mn_hi));
-                pa[kk][2 * h + 0] = plo;
-                pa[kk][2 * h + 1] = phi;
-                // the normaliser sums exactly the bf16 weights that enter PV
-                rs_lo += bf16_lo(plo) + bf16_hi(plo);
-                rs_hi += bf16_lo(phi) + bf16_hi(phi);
+                for (int nd = 0; nd < G::kNTiles; ++nd) {
+                    acc[nd][0] *= alpha_lo;
+                    acc[nd][1] *= alpha_lo;
+                    acc[nd][2] *= alpha_hi;
+                    acc[nd][3] *= alpha_hi;
+                }
             }
-        }
-        l_lo = l_lo * alpha_lo + rs_lo;
-        l_hi = l_hi * alpha_hi + rs_hi;
 #pragma unroll
-        for (int nd = 0; nd < G::kNTiles; ++nd) {
-            acc[nd][0] *= alpha_lo;
-            acc[nd][1] *= alpha_lo;
-            acc[nd][2] *= alpha_hi;
-            acc[nd][3] *= alpha_hi;
+            for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int nt = 2 * kk + h;
+                    pa[kk][2 * h + 0] = pack_bf16x2(ex2_approx(s[nt][0] - mn_lo), ex2_approx(s[nt][1] - mn_lo));
+                    pa[kk][2 * h + 1] = pack_bf16x2(ex2_approx(s[nt][2] - mn_hi), ex2_approx(s[nt][3] - mn_hi));
+                }
+                // the normaliser sums exactly the bf16 weights that enter PV
+                mma_bf16_16816(accl, pa[kk], kOnesBf16x2, kOnesBf16x2);
+            }
+        } else {
+            const float alpha_lo = exp2f(m_lo - mn_lo);
+            const float alpha_hi = exp2f(m_hi - mn_hi);
+            m_lo = mn_lo;
+            m_hi = mn_hi;
+            float rs_lo = 0.f, rs_hi = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int nt = 2 * kk + h;
+                    const uint32_t plo = pack_bf16x2(exp2f(s[nt][0] - mn_lo), exp2f(s[nt][1] - mn_lo));
+                    const uint32_t phi = pack_bf16x2(exp2f(s[nt][2] - mn_hi), exp2f(s[nt][3] - mn_hi));
+                    pa[kk][2 * h + 0] = plo;
+                    pa[kk][2 * h + 1] = phi;
+                    // the normaliser sums exactly the bf16 weights that enter PV
+                    rs_lo += bf16_lo(plo) + bf16_hi(plo);
+                    rs_hi += bf16_lo(phi) + bf16_hi(phi);
+                }
+            }
+            accl[0] = accl[0] * alpha_lo + rs_lo;
+            accl[2] = accl[2] * alpha_hi + rs_hi;
+#pragma unroll
+            for (int nd = 0; nd < G::kNTiles; ++nd) {
+                acc[nd][0] *= alpha_lo;
+                acc[nd][1] *= alpha_lo;
+                acc[nd][2] *= alpha_hi;
+                acc[nd][3] *= alpha_hi;
+            }
         }
 
         // ---- O += P V: k = 32 tokens (2 steps), n = D (8-wide tiles)
@@ -663,10 +730,13 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
         // ---- end of this unit's run in this worker: write output or a partial
         const bool unit_end = (cj == cn - 1) || (i == we - 1);
         if (unit_end) {
-            float ll = l_lo + __shfl_xor_sync(0xffffffffu, l_lo, 1);
-            ll += __shfl_xor_sync(0xffffffffu, ll, 2);
-            float lh = l_hi + __shfl_xor_sync(0xffffffffu, l_hi, 1);
-            lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+            float ll = accl[0], lh = accl[2];
+            if constexpr (!kLean) {
+                ll += __shfl_xor_sync(0xffffffffu, ll, 1);
+                ll += __shfl_xor_sync(0xffffffffu, ll, 2);
+                lh += __shfl_xor_sync(0xffffffffu, lh, 1);
+                lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+            }
             const bool direct = (j_start == 0) && (cj == cn - 1);
             if (direct) {
                 const float il = 1.f / ll, ih = 1.f / lh;

@@ -171,14 +171,6 @@ constexpr uint32_t bf16_idesc(int M, int N, bool b_mn_major) {
            | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
-// 2^x by the MUFU instruction (inputs here are <= 8 or -inf; results below the
-// normal range flush to zero, which only drops weights under 2^-126).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // ---- packed fp32 pairs (sm_100a f32x2 arithmetic) and a 3-input maximum
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
