@@ -47,10 +47,14 @@ struct Traits {
     int max_warps;
 };
 
+// One ring per warp.  D = 32 and 64 are latency-bound per warp, so more warps beat deeper
+// rings (B200, 268 MB of K/V, graph-timed): D = 32, g = 4: 8 warps x 4 stages 55.3 us,
+// 12 x 3 52.9 us; g = 32: 62.8 -> 52.4 us.  D = 64, g = 4: 8 x 4 (6 fit) 50.4 us, 10 x 2
+// 48.7 us; g = 1: 50.0 -> 46.1 us.
 Traits traits_for(int D) {
     switch (D) {
-        case 32: return {4, 8};
-        case 64: return {4, 8};
+        case 32: return {3, 12};
+        case 64: return {2, 10};
         case 128: return {3, 6};
         default: return {2, 4};
     }
@@ -456,7 +460,7 @@ template <int D>
 int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
-    constexpr int kStagesD = (D == 32 || D == 64) ? 4 : (D == 128 ? 3 : 2);
+    constexpr int kStagesD = (D == 32) ? 3 : (D == 64) ? 2 : (D == 128 ? 3 : 2);
     // the lean per-tile form everywhere but D = 256 and the CTA-local plan at D = 128
     // (the kernel's LEAN parameter lists the measurements)
     constexpr bool kLeanD = D != 256;

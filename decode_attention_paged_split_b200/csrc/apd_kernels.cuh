@@ -43,7 +43,12 @@ namespace apd {
 
 constexpr int kTile = 32;          // tokens per tile (= rows of one TMA box)
 constexpr int kMaxRows = 16;       // query heads per unit (mma M)
-constexpr int kMaxWarps = 8;       // warps per CTA, upper bound
+constexpr int kMaxWarps = 8;       // warps per CTA, upper bound (D >= 128, shared K/V rings)
+// Warps per CTA, upper bound of the split kernel.  Small tiles leave a warp latency-bound,
+// and their register footprint leaves room for more warps: 12 at D = 32 and 10 at D = 64
+// with one ring per warp (the launch bound caps registers at 170 and 204).
+template <int D, bool SHARE>
+constexpr int kMaxWarpsD = SHARE ? kMaxWarps : (D == 32 ? 12 : (D == 64 ? 10 : kMaxWarps));
 constexpr uint32_t kFlagPageOOR = 0x1u;
 constexpr uint32_t kFlagLenClamped = 0x2u;
 constexpr uint32_t kFlagLenNegative = 0x4u;
@@ -254,7 +259,7 @@ __device__ __noinline__ void cta_local_merge(const SplitParams& p, const uint8_t
 // [K/V rings, one per kv head of the CTA][Q rings, one per warp], so a CTA of HB warps
 // holds one K/V ring instead of HB.
 template <int D, int STAGES, bool SHARE, bool LEAN>
-__global__ void __launch_bounds__(32 * kMaxWarps, 1)
+__global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
     split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
     using G = Geometry<D>;

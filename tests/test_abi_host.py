@@ -223,7 +223,7 @@ def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
 
 # per head dim: async-copy stages and the most warps a CTA may have, with one ring per
 # warp and with a K/V ring shared by the head blocks of a kv head (None: not shared)
-_TRAITS = {32: (4, 8), 64: (4, 8), 128: (3, 6), 256: (2, 4)}
+_TRAITS = {32: (3, 12), 64: (2, 10), 128: (3, 6), 256: (2, 4)}
 _SHARE_TRAITS = {32: None, 64: (4, 8), 128: (2, 8), 256: (2, 4)}
 
 

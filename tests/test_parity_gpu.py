@@ -392,9 +392,10 @@ def run_hinted(w, hint, stream=None):
     return dp.out, ws
 
 
-# Per head dim, a length whose tiles fit the CTA-local slack (1024 / D tiles) and cut into
-# every warp of the CTA (a ragged last tile included).
-HINT_LEN = {32: 1000, 64: 500, 128: 250, 256: 120}
+# Per head dim, a length whose tiles fit the CTA-local slack (1024 / D tiles) for every
+# head shape below and cut into all, or all but one, of the CTA's warps (a ragged last tile
+# included): 36 tiles in 12 parts at D = 32, 18 in 9 of 10 warps at D = 64.
+HINT_LEN = {32: 1140, 64: 564, 128: 250, 256: 120}
 
 
 @pytest.mark.parametrize("D", workloads.SWEEP_HEAD_DIMS)
