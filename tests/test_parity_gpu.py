@@ -153,6 +153,34 @@ def test_shared_kv_ring(D, Hq, Hkv, ws_div):
     assert apd.read_device_flags(ws) == 0
 
 
+@pytest.mark.parametrize("D,Hq,Hkv", [(128, 64, 2), (64, 48, 1)])
+def test_shared_kv_ring_one_group(D, Hq, Hkv):
+    """The shared K/V ring with a workspace that holds one worker group only: every warp
+    streams all positions, units are written directly (no combine kernel), and the
+    workers write the zero rows of the empty sequences.  Pages of 64 tokens put two tiles
+    in a page, so the page-slot cursor steps within pages too."""
+    lens = (0, 700, 0, 65, 1)
+    w = small(73, B=len(lens), Hq=Hq, Hkv=Hkv, D=D, lens=lens, P=64, pool=20, poison=True,
+              max_pages_per_seq=12)
+    dims = (w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim)
+    lo, hi = 256, apd.workspace_size(*dims, 0)
+    while lo < hi:  # the smallest workspace the balanced plan accepts
+        mid = (lo + hi) // 512 * 256
+        try:
+            apd.query_plan(*dims, 0, workspace_bytes=mid)
+            hi = mid
+        except apd.APDError:
+            lo = mid + 256
+    plan = apd.query_plan(*dims, 0, workspace_bytes=hi)
+    hb = -(-(Hq // Hkv) // 16)
+    assert plan.shared_kv_ring == 1 and plan.num_workers == Hkv * hb and plan.combine_ctas == 0
+    ws = torch.zeros(hi, dtype=torch.uint8, device="cuda")
+    out = DeviceProblem(w).run(0, workspace=ws)
+    check_close(out, oracle.paged_decode(w), f"shared ring, one group, D={D} {Hq}/{Hkv}")
+    assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
+    assert apd.read_device_flags(ws) == 0
+
+
 @pytest.mark.parametrize("P", [64, 128])
 @pytest.mark.parametrize("S", [1, 0, 3])
 def test_larger_pages(P, S):
