@@ -50,14 +50,10 @@ struct Traits {
 // One ring per warp.  D = 32 and 64 are latency-bound per warp, so more warps beat deeper
 // rings (B200, 268 MB of K/V, graph-timed): D = 32, g = 4: 8 warps x 4 stages 55.3 us,
 // 12 x 3 52.9 us; g = 32: 62.8 -> 52.4 us.  D = 64, g = 4: 8 x 4 (6 fit) 50.4 us, 10 x 2
-// 48.7 us; g = 1: 50.0 -> 46.1 us.
-Traits traits_for(int D) {
-    switch (D) {
-        case 32: return {3, 12};
-        case 64: return {2, 10};
-        case 128: return {3, 6};
-        default: return {2, 4};
-    }
+// 48.7 us; g = 1: 50.0 -> 46.1 us.  The kernels are instantiated with these stages, so
+// this table is their single source.
+constexpr Traits traits_for(int D) {
+    return D == 32 ? Traits{3, 12} : D == 64 ? Traits{2, 10} : D == 128 ? Traits{3, 6} : Traits{2, 4};
 }
 
 // The shared-ring layout (balanced mode, g > 16): K/V stages per kv head and the most
@@ -66,16 +62,24 @@ Traits traits_for(int D) {
 // deeper rings.  D = 128, g = 32: 8 warps x 2 stages 64.3 us, 6 x 3 75.3 us, 4 x 3 or 4 x 4
 // 84-85 us, one ring per warp 97.8 us.  D = 32 keeps one ring per warp (71.6 us against
 // 77.1 shared): its short tiles leave a warp pair with too little work per wait.
-Traits share_traits_for(int D) {
-    switch (D) {
-        case 32: return {0, 0};
-        case 64: return {4, 8};
-        case 128: return {2, 8};
-        default: return {2, 4};
-    }
+constexpr Traits share_traits_for(int D) {
+    return D == 32 ? Traits{0, 0} : D == 64 ? Traits{4, 8} : D == 128 ? Traits{2, 8} : Traits{2, 4};
 }
 template <int D>
-constexpr int kShareStages = (D == 64) ? 4 : (D == 128) ? 2 : (D == 256) ? 2 : 0;
+constexpr int kStages = traits_for(D).stages;
+template <int D>
+constexpr int kShareStages = share_traits_for(D).stages;
+
+// A plan never asks for more warps than the kernel's launch bound allows.
+static_assert(traits_for(32).max_warps <= apd::kMaxWarpsD<32, false> &&
+                  traits_for(64).max_warps <= apd::kMaxWarpsD<64, false> &&
+                  traits_for(128).max_warps <= apd::kMaxWarpsD<128, false> &&
+                  traits_for(256).max_warps <= apd::kMaxWarpsD<256, false>,
+              "warps per CTA above the split kernel's launch bound");
+static_assert(share_traits_for(64).max_warps <= apd::kMaxWarpsD<64, true> &&
+                  share_traits_for(128).max_warps <= apd::kMaxWarpsD<128, true> &&
+                  share_traits_for(256).max_warps <= apd::kMaxWarpsD<256, true>,
+              "warps per CTA above the shared-ring kernel's launch bound");
 
 bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
 
@@ -460,7 +464,7 @@ template <int D>
 int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
-    constexpr int kStagesD = (D == 32) ? 3 : (D == 64) ? 2 : (D == 128 ? 3 : 2);
+    constexpr int kStagesD = kStages<D>;
     // the lean per-tile form everywhere but D = 256 and the CTA-local plan at D = 128
     // (the kernel's LEAN parameter lists the measurements)
     constexpr bool kLeanD = D != 256;
