@@ -516,3 +516,42 @@ def test_gemv_plan_rejects_bad_shapes():
     for m, n, k in ((0, 16, 64), (9, 16, 64), (1, 0, 64), (1, 16, 0)):
         with pytest.raises(apd.APDError):
             apd.gemv_query_plan(m, n, k, 148)
+
+
+# ---------------------------------------------------------------- plan invariants
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=300, deadline=None)
+@given(B=st.integers(1, 300), Hkv=st.sampled_from([1, 2, 4, 8, 16]), g=st.integers(1, 80),
+       D=st.sampled_from([32, 64, 128, 256]), sm=st.sampled_from([1, 8, 132, 148]),
+       splits=st.sampled_from([0, 0, 1, 3]), L=st.integers(0, 70000))
+def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
+    """Whatever the shape, SM count or hint, a plan is one the kernels can run:
+    - its shared memory fits a CTA;
+    - every CTA's warps are within the launch bound;
+    - the grid covers the workers;
+    - with a shared K/V ring, the head blocks of a kv head share a CTA;
+    - with the CTA-local plan, each unit gets its own SM and no combine runs."""
+    Hq = Hkv * g
+    hb = -(-g // 16)
+    pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=sm, host_seq_lens=[L] * B, max_seq_len=70000)
+    bound = {32: 12, 64: 10}.get(D, 8) if not pl.shared_kv_ring else 8
+    assert pl.smem_bytes <= 232448
+    assert 1 <= pl.warps_per_cta <= bound
+    assert pl.grid_ctas * pl.warps_per_cta >= pl.num_workers > 0
+    assert pl.head_blocks == hb and pl.rows_per_unit == min(g, 16)
+    units = B * Hkv * hb
+    if pl.shared_kv_ring:
+        assert pl.mode == 0 and hb > 1 and D != 32
+        assert pl.warps_per_cta % hb == 0 and pl.num_workers % (Hkv * hb) == 0
+    if pl.mode == 0:
+        # at most one CTA per SM, unless one worker group alone needs more CTAs (the CTAs
+        # never wait on one another, so they may also run in waves)
+        assert splits == 0 and pl.num_workers % (Hkv * hb) == 0
+        assert pl.grid_ctas <= max(sm, -(-(Hkv * hb) // pl.warps_per_cta))
+    elif pl.mode == 1:
+        assert splits > 0 and pl.num_workers == units * splits
+    else:
+        assert splits == 0 and pl.mode == 2 and units <= sm
+        assert pl.grid_ctas == units and pl.combine_ctas == 0 and pl.partial_slots == 0
