@@ -31,6 +31,12 @@
 //    accumulate) with the g query heads of a kv head on the M side (padded to
 //    16), so K/V are read once per kv head.  The softmax is the online form in
 //    fp32 with exp2 (logits pre-multiplied by scale * log2 e) and quad shuffles.
+//  * g > 16 takes ceil(g / 16) head blocks, one warp each.  In balanced mode they
+//    share one K/V ring in their CTA (SHARE): the first fills it, the others
+//    release each stage on an mbarrier, and every K/V tile leaves HBM once.
+//  * LEAN selects the trimmed per-tile code: row sums from an mma against ones,
+//    2^x from the SFU, no masking on full tiles, and no rescale while no row's
+//    max grows.
 #pragma once
 
 #include <cuda.h>
