@@ -9,6 +9,7 @@ import re
 
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 import decode_attention_paged_split_b200 as apd
 
@@ -480,10 +481,12 @@ def test_selftest_arguments_are_checked_before_any_launch():
                                    (1, 256, 1536), (8, 1536, 6912), (5, 50, 1040), (2, 3000, 1000), (1, 64, 200),
                                    (4, 2048, 16384), (1, 2360, 520)])
 def test_gemv_plan(M, N, K):
+    _check_gemv_plan(M, N, K)
+
+
+def _check_gemv_plan(M, N, K):
     p = apd.gemv_query_plan(M, N, K, 148)
     mtiles, ktiles = -(-N // 16), -(-K // 256)
-    # x is staged once per CTA for weight streams of at least 64 MB; those run 6 warps on
-    # 7/8 of the SMs, the rest 4 warps on every SM
     # x is staged once per CTA for weight streams of at least 64 MB when its padded rows
     # (16-byte chunks, an odd number per row) take at most 32 KB and fit beside the ring
     x_bytes = M * 16 * ((K // 8) | 1)
@@ -512,6 +515,14 @@ def test_gemv_plan(M, N, K):
     assert p["workspace_bytes"] == 256 + -(-(2 * p["workers"] * 16 * 8 * 4) // 256) * 256
 
 
+@settings(max_examples=300, deadline=None)
+@given(M=st.integers(1, 8), N=st.integers(1, 200000), K8=st.integers(1, 2048))
+def test_gemv_plan_random_shapes(M, N, K8):
+    """The restated GEMV launch rule over random shapes (K a multiple of 8, as the call
+    requires)."""
+    _check_gemv_plan(M, N, 8 * K8)
+
+
 def test_gemv_plan_rejects_bad_shapes():
     for m, n, k in ((0, 16, 64), (9, 16, 64), (1, 0, 64), (1, 16, 0)):
         with pytest.raises(apd.APDError):
@@ -519,7 +530,6 @@ def test_gemv_plan_rejects_bad_shapes():
 
 
 # ---------------------------------------------------------------- plan invariants
-from hypothesis import given, settings, strategies as st  # noqa: E402
 
 
 @settings(max_examples=300, deadline=None)
