@@ -413,7 +413,8 @@ typedef struct apd_plan {
     int32_t num_workers;       /* warps that each own a run of tiles             */
     int32_t grid_ctas;         /* CTAs of the split kernel                       */
     int32_t warps_per_cta;
-    int32_t stages;            /* async-copy ring depth per warp                 */
+    int32_t stages;            /* async-copy ring depth per warp (per kv head
+                                  when shared_kv_ring = 1)                      */
     int32_t rows_per_unit;     /* query heads packed per unit (<= 16)            */
     int32_t head_blocks;       /* ceil(g / 16)                                   */
     int32_t combine_ctas;      /* 0 when no combine kernel is launched           */
