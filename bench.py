@@ -40,8 +40,12 @@ import workloads  # noqa: E402
 
 METRIC = "paged decode attention achieved HBM GB/s (algorithmic KV+q+out bytes per call / time)"
 UNIT = "GB/s"
-DEFAULT_STEPS = {"llama8b": 20000, "long": 5000, "ragged": 2000, "tiny": 20000, "llama8b_contig": 20000,
-                 "long_contig": 5000, "gqa32": 10000}
+DEFAULT_STEPS = {"llama8b": 200, "long": 100, "ragged": 50, "tiny": 200, "llama8b_contig": 200,
+                 "long_contig": 100, "gqa32": 200}
+DEFAULT_REFERENCE_STEPS = 20
+# measured beside the headline decode workload, in the same run (the other configurations with a
+# 70% target or a reported number)
+PER_CONFIG = ("long", "ragged")
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
 GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes per call / time)"
 GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
@@ -69,9 +73,19 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     p.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi clocks")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="decode: do not also measure the long-context and ragged configurations")
+    p.add_argument("--instances", type=int, default=2,
+                   help="independent copies of the workload used in turn (1 keeps the device footprint small "
+                        "for profiling; every large workload is bigger than L2 on its own)")
+    p.add_argument("--min-seconds", type=float, default=2.0,
+                   help="repeat the timed K-step region until about this long (at least 3 repetitions)")
     a = p.parse_args(argv)
+    a.steps_given = a.steps is not None
     if a.steps is None:
-        a.steps = DEFAULT_STEPS.get(a.workload, 2000)
+        a.steps = (DEFAULT_REFERENCE_STEPS if a.impl == "reference" else DEFAULT_STEPS.get(a.workload, 2000))
+    if a.instances < 1:
+        p.error("--instances must be >= 1")
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
     return a
@@ -336,41 +350,85 @@ def graph_split_times(insts, stream, replays):
 
 
 class GraphSteps:
-    """CUDA graphs of consecutive calls (rotating over the instances): `steps` calls in
-    all, as steps // GRAPH_CHUNK replays of a GRAPH_CHUNK-call graph plus one graph of
-    the remainder."""
+    """Exactly `steps` consecutive calls `call(i, stream)` (i = 0 .. steps-1; the calls repeat
+    with `period`, e.g. instances used in turn) captured as CUDA graphs of up to GRAPH_CHUNK
+    calls, with event-record nodes before the first call and after the last: the interval
+    between them is the calls' time on the device, without the host's launch of the graphs.
+    Longer runs chain a first graph (with the start event), a middle graph replayed as often
+    as needed and a last graph (with the end event)."""
 
-    def __init__(self, insts, stream, steps):
-        self.plan = []
-        full, rest = divmod(steps, GRAPH_CHUNK)
-        if full:
-            self.plan.append((self._capture(insts, stream, GRAPH_CHUNK), full))
-        if rest:
-            self.plan.append((self._capture(insts, stream, rest), 1))
+    def __init__(self, call, stream, steps, period=1):
+        self.start = torch.cuda.Event(enable_timing=True, external=True)
+        self.end = torch.cuda.Event(enable_timing=True, external=True)
+        self.start.record(stream)  # create the events before capture
+        self.end.record(stream)
+        torch.cuda.synchronize()
+        # a graph that is replayed more than once holds a whole number of periods
+        chunk = max(period, GRAPH_CHUNK - GRAPH_CHUNK % period)
+        if steps <= chunk:
+            self.plan = [(self._capture(call, stream, steps, True, True), 1)]
+        else:
+            mid_reps, last = divmod(steps - chunk, chunk)
+            if last == 0:
+                mid_reps, last = mid_reps - 1, chunk
+            self.plan = [(self._capture(call, stream, chunk, True, False), 1)]
+            if mid_reps:
+                self.plan.append((self._capture(call, stream, chunk, False, False), mid_reps))
+            self.plan.append((self._capture(call, stream, last, False, True), 1))
+        self.steps = steps
 
-    @staticmethod
-    def _capture(insts, stream, n):
+    def _capture(self, call, stream, count, with_start, with_end):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             with torch.cuda.graph(g, stream=stream):
-                for i in range(n):
-                    insts[i % len(insts)].call(stream)
+                if with_start:
+                    self.start.record(stream)
+                for i in range(count):
+                    call(i, stream)
+                if with_end:
+                    self.end.record(stream)
         return g
 
     def run(self, stream):
-        start = torch.cuda.Event(enable_timing=True)
-        end = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            start.record(stream)
             for g, reps in self.plan:
                 for _ in range(reps):
                     g.replay()
-            end.record(stream)
-        end.synchronize()
-        return start.elapsed_time(end) / 1e3
+        self.end.synchronize()
+        return self.start.elapsed_time(self.end) / 1e3
 
     def release(self):
         self.plan = []
+
+
+def timed_reps(run, dist, device, min_seconds: float, max_reps: int = 20000):
+    """Repetitions of one timed region (`run()` returns its device seconds), each bracketed by
+    a barrier and a device synchronisation: one untimed, then as many as last about
+    min_seconds (at least 3; the same count on every rank).  Returns the per-repetition
+    seconds, each the max over ranks."""
+    run()
+    t1 = run()
+    reps = max(3, min(max_reps, math.ceil(min_seconds / max(t1, 1e-9))))
+    reps = int(max_over_ranks(float(reps), dist, device))
+    times = []
+    for _ in range(reps):
+        barrier(dist, device)
+        if device.type == "cuda":
+            torch.cuda.synchronize(device)
+        times.append(run())
+    if dist is not None:
+        t = torch.tensor(times, dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        times = t.cpu().tolist()
+    return times
+
+
+def timing_summary(times, steps):
+    med = statistics.median(times)
+    return {"reps": len(times), "steps_per_rep": steps, "median_us_per_call": med / steps * 1e6,
+            "min_us_per_call": min(times) / steps * 1e6, "max_us_per_call": max(times) / steps * 1e6,
+            "timed_s": sum(times),
+            "stat": "median over repetitions of the K-call region (each the max over ranks)"}
 
 
 def e2e_steps(insts, stream, steps):
@@ -419,22 +477,32 @@ def e2e_steps(insts, stream, steps):
     return start.elapsed_time(end) / 1e3, h2d, d2h
 
 
-def oracle_baseline(w, min_seconds: float = 10.0, max_calls: int = 50):
-    """The fp64 CPU oracle on the whole workload, repeated until about min_seconds."""
+def oracle_baseline(w, min_seconds: float = 10.0, max_calls: int = 50, single_core_seconds: float = 5.0):
+    """The fp64 CPU oracle on the whole workload, as it stands: on all host threads (OpenMP
+    over query rows), repeated until about min_seconds, then on one thread for about
+    single_core_seconds."""
     import oracle
 
+    def timed(nthreads, seconds, cap):
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            oracle.paged_decode(w, nthreads=nthreads)
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or calls >= cap:
+                return calls, el
+
     oracle.paged_decode(w)  # loads the library and faults in the pages once
-    calls, t0 = 0, time.perf_counter()
-    while True:
-        oracle.paged_decode(w)
-        calls += 1
-        el = time.perf_counter() - t0
-        if el >= min_seconds or calls >= max_calls:
-            break
-    return {"value": w.algorithmic_bytes() * calls / el / 1e9, "unit": UNIT, "cores": oracle.max_threads(),
-            "kind": "oracle",
-            "sample": f"the whole {w.name} workload (all {w.batch * w.num_q_heads} query rows), {calls} calls, "
-                      f"{el:.1f} s, fp64, OpenMP over rows"}
+    threads = oracle.max_threads()
+    calls, el = timed(0, min_seconds, max_calls)
+    calls1, el1 = timed(1, single_core_seconds, max_calls)
+    rows = w.batch * w.num_q_heads
+    return {"value": w.algorithmic_bytes() * calls / el / 1e9, "unit": UNIT, "cores": threads,
+            "kind": "oracle", "nproc": os.cpu_count(), "omp_threads": threads,
+            "sample": f"the whole {w.name} workload (all {rows} query rows), {calls} calls, {el:.1f} s, fp64, "
+                      f"OpenMP over rows on {threads} threads",
+            "single_core": {"value": w.algorithmic_bytes() * calls1 / el1 / 1e9, "unit": UNIT, "cores": 1,
+                            "sample": f"the whole workload, {calls1} calls, {el1:.1f} s, one thread"}}
 
 
 def peaks():
@@ -449,7 +517,9 @@ def peaks():
 
 # ---------------------------------------------------------------- arms
 def run_reference(a):
-    """The reference arm: the fp64 CPU oracle, each step a bounded sample of the workload."""
+    """The reference arm: the fp64 CPU oracle on all host threads, each step the whole
+    workload (the cpu_baseline leg's sample), or an equal share of its query rows when K
+    whole calls would not end within a few minutes."""
     world, rank, _ = dist_env()
     if world > 1 and rank != 0:
         return 0
@@ -457,14 +527,32 @@ def run_reference(a):
 
     w = make_instances(a.workload, 0, 1)[0]
     B, Hq = w.batch, w.num_q_heads
-    row_tokens = w.seq_lens.to(torch.int64)
-    total_row_tokens = float(row_tokens.sum()) * Hq
+    total_bytes = w.algorithmic_bytes()
+    oracle.paged_decode(w)  # loads the library and faults in the pages once
+    t0 = time.perf_counter()
+    oracle.paged_decode(w)
+    t_whole = time.perf_counter() - t0
+    budget = 150.0  # seconds for the warm-up and timed steps together
+    rows_all = [(b, h) for b in range(B) for h in range(Hq)]
+    per_row = w.seq_lens.to(torch.float64)
+    row_weight = [float(per_row[b]) for b, _ in rows_all]
+    total_weight = max(sum(row_weight), 1.0)
+    if t_whole * (a.steps + a.warmup) <= budget:
+        nrows = len(rows_all)
+        sample = f"each step: the whole {w.name} workload (all {nrows} query rows)"
+    else:
+        nrows = max(1, int(len(rows_all) * budget / (t_whole * (a.steps + a.warmup))))
+        sample = (f"each step: {nrows} of the {len(rows_all)} query rows of {w.name} (a window rotating over "
+                  f"them; bytes counted in proportion to the rows' tokens)")
 
     def step(i):
-        b = i % B
-        rows = [(b, h) for h in range(Hq)]
-        oracle.paged_decode_rows(w, rows)
-        return w.algorithmic_bytes() * float(row_tokens[b]) * Hq / max(total_row_tokens, 1.0)
+        if nrows == len(rows_all):
+            oracle.paged_decode(w)
+            return float(total_bytes)
+        lo = (i * nrows) % len(rows_all)
+        idx = [(lo + j) % len(rows_all) for j in range(nrows)]
+        oracle.paged_decode_rows(w, [rows_all[j] for j in idx])
+        return total_bytes * sum(row_weight[j] for j in idx) / total_weight
 
     for i in range(a.warmup):
         step(i)
@@ -480,9 +568,8 @@ def run_reference(a):
         "warmup": a.warmup, "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, a),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"each step: the {Hq} query rows of one sequence of {w.name} (rotating over "
-                                   f"the {B} sequences), fp64 CPU oracle on {cores} threads"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "nproc": os.cpu_count(),
+                         "omp_threads": cores, "sample": f"{sample}, fp64 CPU oracle on {cores} threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -490,14 +577,85 @@ def run_reference(a):
 
 
 def config_of(w, a):
+    n = getattr(a, "instances", 2)
     return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
             "head_dim": w.head_dim, "page_size": w.page_size, "kv_tokens": w.kv_tokens(),
             "num_splits": a.num_splits, "layout": w.layout, "kv_policy": w.meta.get("kv_policy", "paged"),
-            "l2": "two independent instances used in turn (each call reads KV the previous call did not touch); "
-                  "large workloads are each larger than L2",
+            "l2": (f"{n} independent instances used in turn (each call reads KV the previous call did not touch); "
+                   "large workloads are each larger than L2") if n > 1 else
+                  "one instance (large workloads are larger than L2 on their own)",
             "algorithmic_bytes_per_call": w.algorithmic_bytes(),
             "host_seq_lens_hint": not getattr(a, "no_host_lens", False),
-            "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"}
+            "launch": f"CUDA graphs of up to {GRAPH_CHUNK} consecutive calls with event-record nodes around "
+                      f"the K calls; the K-call region repeated for about {getattr(a, 'min_seconds', 2.0):g} s"}
+
+
+def measure_decode(a, name, apd, device, dist, rank, local, min_seconds, want_clocks, extras=False):
+    """Times `a.steps` consecutive calls of a decode workload (graph replays, repeated, see
+    timed_reps) on this rank's instances.  Returns a dict of the numbers, and the instances
+    when `extras` (for the headline's eager, end-to-end and oracle legs)."""
+    insts = [Resident(w, device, a.num_splits, apd, host_hint=not a.no_host_lens)
+             for w in make_instances(name, rank, a.instances)]
+    w0 = insts[0].w
+    max_len = w0.k_cache.shape[1] if insts[0].contig else w0.page_table.shape[1] * w0.page_size
+    plan = apd.query_plan(w0.batch, w0.num_q_heads, w0.num_kv_heads, w0.head_dim, a.num_splits,
+                          host_seq_lens=insts[0].host_lens, max_seq_len=max_len)
+    launches_per_step = 1 + (1 if plan.combine_ctas > 0 else 0)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize(device)
+
+    time_steps(insts, stream, a.warmup)  # warm-up (eager)
+    graphs = GraphSteps(lambda i, st: insts[i % len(insts)].call(st), stream, a.steps, period=len(insts))
+    clocks = ClockSampler(local, enabled=want_clocks)
+    times = timed_reps(lambda: graphs.run(stream), dist, device, min_seconds)
+    clock_info = clocks.stop()
+    graphs.release()
+    t_med = statistics.median(times)
+    bytes_rank = sum(insts[i % len(insts)].bytes for i in range(a.steps))
+    bytes_all = sum_over_ranks(float(bytes_rank), dist, device)
+    if launches_per_step == 1:
+        # The call is this one kernel: its average launch duration is the timed region over
+        # the launches in it.
+        split_s = t_med / a.steps
+        kernel_timing = ("the call is this one kernel: the median K-call region (event-record nodes around "
+                         "the graph-replayed calls) over the K launches in it")
+    else:
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        try:
+            split_s = graph_split_times(insts, stream, replays=10)
+        except RuntimeError as err:  # event-record nodes unavailable: fall back to eager event pairs
+            print(f"graph split timing unavailable ({err}); using eager event pairs", file=sys.stderr)
+            _, split_s = time_steps(insts, stream, a.steps, split_events=True)
+        split_s = max_over_ranks(split_s, dist, device)
+        kernel_timing = ("CUDA events recorded around each split kernel inside replays of a "
+                         f"{GRAPH_CHUNK}-call graph (event-record nodes)")
+    peak, peak_src = peaks()
+    mean_bytes = bytes_rank / a.steps
+    achieved = mean_bytes / split_s / 1e9
+    res = {
+        "workload": w0.name, "us_per_call": t_med / a.steps * 1e6, "value": bytes_all / t_med / 1e9,
+        "timing": timing_summary(times, a.steps),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "traffic": committed_traffic(name), "peak_source": peak_src, "kernel": "split_kernel",
+                     "kernel_us": split_s * 1e6, "kernel_timing": kernel_timing,
+                     "call_frac_of_peak": bytes_all / t_med / 1e9 / max(1, (dist.get_world_size() if dist else 1))
+                     / peak},
+        "gpu_launches": launches_per_step * a.steps * len(times),
+        "clocks": clock_info,
+        "plan": {"mode": plan.mode,
+                 "mode_name": {0: "balanced + combine", 1: "fixed splits", 2: "one CTA per unit, single kernel"}
+                 [plan.mode],
+                 "workers": plan.num_workers, "ctas": plan.grid_ctas, "warps_per_cta": plan.warps_per_cta,
+                 "stages": plan.stages, "smem": plan.smem_bytes, "shared_kv_ring": bool(plan.shared_kv_ring),
+                 "combine_ctas": plan.combine_ctas},
+        "config": config_of(w0, a),
+    }
+    if extras:
+        res.update(_insts=insts, _stream=stream, _t_med=t_med, _bytes_all=bytes_all)
+    else:
+        del insts
+    return res
 
 
 def run_ours(a):
@@ -516,67 +674,15 @@ def run_ours(a):
     dist = init_group(world, "nccl")
     import decode_attention_paged_split_b200 as apd
 
-    insts = [Resident(w, device, a.num_splits, apd, host_hint=not a.no_host_lens)
-             for w in make_instances(a.workload, rank, 2)]
-    w0 = insts[0].w
-    max_len = w0.k_cache.shape[1] if insts[0].contig else w0.page_table.shape[1] * w0.page_size
-    plan = apd.query_plan(w0.batch, w0.num_q_heads, w0.num_kv_heads, w0.head_dim, a.num_splits,
-                          host_seq_lens=insts[0].host_lens, max_seq_len=max_len)
-    launches_per_step = 1 + (1 if plan.combine_ctas > 0 else 0)
-    stream = torch.cuda.Stream(device)
-    torch.cuda.synchronize(device)
-
-    # warm-up (eager), then capture the timed calls as CUDA graphs and run them once untimed
-    time_steps(insts, stream, a.warmup)
-    graphs = GraphSteps(insts, stream, a.steps)
-    graphs.run(stream)
-
-    # main timed region: exactly `steps` calls, replayed from the graphs
-    clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
-    elapsed = graphs.run(stream)
-    torch.cuda.synchronize(device)
-    barrier(dist, device)
-    clock_info = clocks.stop()
-    graphs.release()
-    bytes_rank = sum(insts[i % 2].bytes for i in range(a.steps))
-    t_max = max_over_ranks(elapsed, dist, device)
-    bytes_all = sum_over_ranks(float(bytes_rank), dist, device)
-    value = bytes_all / t_max / 1e9
+    want_clocks = not a.no_clocks and rank == 0
+    head = measure_decode(a, a.workload, apd, device, dist, rank, local, a.min_seconds, want_clocks, extras=True)
+    insts, stream, t_med, bytes_all = head["_insts"], head["_stream"], head["_t_med"], head["_bytes_all"]
 
     # the same steps launched eagerly from Python, for reference
     barrier(dist, device)
     torch.cuda.synchronize(device)
     eager_el, _ = time_steps(insts, stream, a.steps)
     eager_max = max_over_ranks(eager_el, dist, device)
-
-    # split-kernel duration: events around each split kernel inside graph replays (the
-    # launch configuration of the timed region); eager event pairs, which also count the
-    # launch latency of every kernel, are kept for reference
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
-    _, split_eager_s = time_steps(insts, stream, a.steps, split_events=True)
-    torch.cuda.synchronize(device)
-    split_eager_s = max_over_ranks(split_eager_s, dist, device)
-    try:
-        split_s = graph_split_times(insts, stream, replays=max(1, min(20, a.steps // GRAPH_CHUNK)))
-    except RuntimeError as err:  # event-record nodes unavailable: fall back to the eager pairs
-        print(f"graph split timing unavailable ({err}); using eager event pairs", file=sys.stderr)
-        split_s = split_eager_s
-    split_s = max_over_ranks(split_s, dist, device)
-    split_bracketed_s = split_s
-    if launches_per_step == 1:
-        # The call is this one kernel: its average launch duration is the timed region
-        # (events around the graph replays) over the launches in it.  Events recorded
-        # around each launch inside the graph also stop one launch from overlapping the
-        # next (programmatic dependent launch), so they overstate it; kept for reference.
-        split_s = t_max / a.steps
-        kernel_timing = ("the call is this one kernel: CUDA events around the timed region of graph replays, "
-                         "divided by the launches in it")
-    else:
-        kernel_timing = ("CUDA events recorded around each split kernel inside replays of a "
-                         f"{GRAPH_CHUNK}-call graph (event-record nodes)")
 
     # end to end through host buffers
     e2e = None
@@ -592,40 +698,36 @@ def run_ours(a):
                "how": "per step, eager through the public Python API: one pinned-host->device copy of the "
                       "packed q|page_table|seq_lens, the call, one device->pinned-host copy of out; copies on "
                       "two copy streams overlap the neighbouring steps' compute"}
+    w0 = insts[0].w
+    del insts, head["_insts"]
+    torch.cuda.empty_cache()
+
+    # the other configurations with a target or a reported number, in the same run
+    per_config = {}
+    if a.workload == "llama8b" and not a.no_per_config:
+        for name in PER_CONFIG:
+            r = measure_decode(a, name, apd, device, dist, rank, local, max(0.5, a.min_seconds / 2), want_clocks)
+            per_config[r["workload"]] = {k2: r[k2] for k2 in ("us_per_call", "value", "timing", "roofline", "clocks",
+                                                             "plan", "gpu_launches")}
+            per_config[r["workload"]]["unit"] = UNIT
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         cpu = oracle_baseline(w0)
 
     if rank == 0:
-        peak, peak_src = peaks()
-        mean_bytes = bytes_rank / a.steps
-        achieved = mean_bytes / split_s / 1e9
-        traffic = committed_traffic(a.workload)
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": t_max / a.steps * 1e3, "us_per_call": t_max / a.steps * 1e6,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": t_med / a.steps * 1e3, "us_per_call": head["us_per_call"],
             "eager_us_per_call": eager_max / a.steps * 1e6,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_of(w0, a),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT,
-                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "kernel": "split_kernel", "kernel_us": split_s * 1e6,
-                         "kernel_us_event_bracketed": split_bracketed_s * 1e6,
-                         "kernel_us_eager_events": split_eager_s * 1e6,
-                         "kernel_timing": kernel_timing,
-                         "call_frac_of_peak": value / world / peak},
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches_per_step * a.steps,
-            "clocks": clock_info,
-            "plan": {"mode": plan.mode,
-                     "mode_name": {0: "balanced + combine", 1: "fixed splits", 2: "one CTA per unit, single kernel"}
-                     [plan.mode],
-                     "workers": plan.num_workers, "ctas": plan.grid_ctas,
-                     "warps_per_cta": plan.warps_per_cta, "stages": plan.stages, "smem": plan.smem_bytes,
-                     "shared_kv_ring": bool(plan.shared_kv_ring)},
+            "data": "synthetic", "config": head["config"], "timing": head["timing"],
+            "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"], "plan": head["plan"],
         }
+        if per_config:
+            line["per_config"] = per_config
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -668,37 +770,12 @@ def run_gemv(a):
     for i in range(a.warmup):
         call(i, stream)
     torch.cuda.synchronize(device)
-    plan = []
-    full, rest = divmod(a.steps, GRAPH_CHUNK)
-    for n, reps in ((GRAPH_CHUNK, full), (rest, 1 if rest else 0)):
-        if reps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(stream):
-                with torch.cuda.graph(g, stream=stream):
-                    for i in range(n):
-                        call(i, stream)
-            plan.append((g, reps))
-
-    def replay():
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for g, reps in plan:
-                for _ in range(reps):
-                    g.replay()
-            e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1) / 1e3
-
-    replay()
+    graphs = GraphSteps(call, stream, a.steps, period=copies)
     clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
-    el = replay()
-    barrier(dist, device)
+    times = timed_reps(lambda: graphs.run(stream), dist, device, a.min_seconds)
     clock_info = clocks.stop()
-    plan = []
-    t_max = max_over_ranks(el, dist, device)
+    graphs.release()
+    t_max = statistics.median(times)
     bytes_all = sum_over_ranks(float(per_call * a.steps), dist, device)
     value = bytes_all / t_max / 1e9
 
@@ -769,14 +846,16 @@ def run_gemv(a):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": case.name, "M": M, "N": N, "K": K, "algorithmic_bytes_per_call": per_call,
                        "l2": f"{copies} weight copies used in turn ({copies * N * K * 2 / 1e6:.0f} MB > L2)",
-                       "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
+                       "launch": f"CUDA graphs of up to {GRAPH_CHUNK} consecutive calls with event-record nodes "
+                                 f"around the K calls; the K-call region repeated for about {a.min_seconds:g} s"},
             "roofline": {"bound": "hbm", "achieved": per_call / (t_max / a.steps) / 1e9, "peak": peak, "unit": UNIT,
                          "frac": per_call / (t_max / a.steps) / 1e9 / peak,
                          "traffic": committed_traffic(case.name, GEMV_TRAFFIC_FILE, GEMV_KERNEL_SOURCES),
                          "peak_source": peak_src,
                          "kernel": "gemv_kernel + gemv_sum_kernel (whole call)" if gplan["sum_ctas"]
                          else "gemv_kernel (the whole call)"},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (2 if gplan["sum_ctas"] else 1) * a.steps,
+            "timing": timing_summary(times, a.steps),
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (2 if gplan["sum_ctas"] else 1) * a.steps * len(times),
             "clocks": clock_info, "plan": gplan,
         }
         print(json.dumps(line), flush=True)
@@ -861,37 +940,12 @@ def run_prefill(a):
     for i in range(a.warmup):
         call(i)
     torch.cuda.synchronize(device)
-    plan = []
-    full, rest = divmod(a.steps, GRAPH_CHUNK)
-    for n, reps in ((GRAPH_CHUNK, full), (rest, 1 if rest else 0)):
-        if reps:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(stream):
-                with torch.cuda.graph(g, stream=stream):
-                    for i in range(n):
-                        call(i)
-            plan.append((g, reps))
-
-    def replay():
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for g, reps in plan:
-                for _ in range(reps):
-                    g.replay()
-            e1.record(stream)
-        e1.synchronize()
-        return e0.elapsed_time(e1) / 1e3
-
-    replay()
+    graphs = GraphSteps(lambda i, st: call(i), stream, a.steps, period=2)
     clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
-    barrier(dist, device)
-    torch.cuda.synchronize(device)
-    el = replay()
-    barrier(dist, device)
+    times = timed_reps(lambda: graphs.run(stream), dist, device, a.min_seconds)
     clock_info = clocks.stop()
-    plan = []
-    t_max = max_over_ranks(el, dist, device)
+    graphs.release()
+    t_max = statistics.median(times)
     bytes_all = sum_over_ranks(float(per_bytes * a.steps), dist, device)
     flops_all = sum_over_ranks(float(per_flops * a.steps), dist, device)
 
@@ -935,13 +989,15 @@ def run_prefill(a):
                        "num_kv_heads": 8, "head_dim": 128, "seq_len": 4096, "causal_offset": w0.causal_offset,
                        "algorithmic_bytes_per_call": per_bytes, "algorithmic_flops_per_call": per_flops,
                        "l2": "two cache instances used in turn, each larger than L2",
-                       "launch": f"CUDA graphs of {GRAPH_CHUNK} consecutive calls, replayed"},
+                       "launch": f"CUDA graphs of up to {GRAPH_CHUNK} consecutive calls with event-record nodes "
+                                 f"around the K calls; the K-call region repeated for about {a.min_seconds:g} s"},
             "roofline": {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
                          "traffic": (committed_traffic(w0.name, PREFILL_TRAFFIC_FILE, PREFILL_KERNEL_SOURCES)
                                      if prefill_kernel_name(a.prefill_kernel) == "prefill_tc2_kernel" else None),
                          "peak_source": tsrc, "kernel": prefill_kernel_name(a.prefill_kernel),
                          "hbm_achieved_gbs": gbs, "hbm_frac": gbs / hpeak},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": a.steps, "clocks": clock_info,
+            "timing": timing_summary(times, a.steps),
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": a.steps * len(times), "clocks": clock_info,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

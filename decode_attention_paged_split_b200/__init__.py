@@ -24,6 +24,7 @@ __all__ = [
     "attn_contig_decode",
     "attn_paged_prefill",
     "selftest_bounded_wait",
+    "selftest_shared_ring_release",
     "gemv",
     "gemv_workspace_size",
     "DecodeCall",
@@ -169,6 +170,9 @@ def _load():
     L.apd_attn_paged_prefill_ex.restype = ctypes.c_int
     L.apd_selftest_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p]
     L.apd_selftest_bounded_wait.restype = ctypes.c_int
+    L.apd_selftest_shared_ring_release.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
+                                                   ctypes.c_uint64, ctypes.c_void_p]
+    L.apd_selftest_shared_ring_release.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
     L.apd_gemv_query_plan.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(_GemvPlan)]
@@ -334,6 +338,20 @@ def selftest_bounded_wait(short_timeout_ns: int = 1_000_000, device="cuda") -> l
         raise APDError(rc, "apd_selftest_bounded_wait")
     torch.cuda.synchronize(out.device)
     return [int(v) & 0xFFFFFFFF for v in out.cpu().tolist()]
+
+
+def selftest_shared_ring_release(q, k_cache, v_cache, page_table, seq_lens, out, scale: float,
+                                 workspace: torch.Tensor, short_timeout_ns: int = 1_000_000, stream=None) -> None:
+    """Enqueues the shared K/V ring's release self-test (apd_selftest_shared_ring_release) on
+    a problem with more than 16 q heads per kv head: the followers never release a stage
+    and every wait gives up after short_timeout_ns.  Read the outcome with
+    read_device_flags(workspace)."""
+    descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+    rc = _load().apd_selftest_shared_ring_release(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale),
+                                                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                                  int(short_timeout_ns), _stream_handle(stream, q.device))
+    if rc:
+        raise APDError(rc, "apd_selftest_shared_ring_release")
 
 
 def prefill_auto_kernel(head_dim: int) -> str:

@@ -110,7 +110,9 @@ uint32_t stage_bytes(const Shape& s) { return 2u * apd::kTile * s.D * 2u + q_til
 // share: the layout where the HB warps of a kv head share one K/V ring (the balanced mode
 // when g > 16): warps / HB K/V rings and `warps` Q rings, and an `empty` mbarrier per stage.
 size_t smem_bytes(const Shape& s, int warps, int stages, bool share = false) {
-    const size_t meta = 8ull * warps * stages * (share ? 2 : 1) + 8 + 4ull * (2ull * s.B + 1);
+    // mbarriers (full, and empty in the shared layout), the merge mbarrier, the abort word
+    // (8 bytes), lengths and prefix sums
+    const size_t meta = 8ull * warps * stages * (share ? 2 : 1) + 8 + 8 + 4ull * (2ull * s.B + 1);
     const size_t rings = share ? static_cast<size_t>(warps / s.HB) * stages * (2ull * apd::kTile * s.D * 2) +
                                      static_cast<size_t>(warps) * stages * q_tile_bytes(s)
                                : static_cast<size_t>(warps) * stages * stage_bytes(s);
@@ -460,10 +462,17 @@ int encode_q_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D
 }
 
 // ---------------------------------------------------------------- launch
+// Self-test settings of the split kernel (the defaults are the product's).
+struct SplitTestHooks {
+    uint64_t wait_ns = apd::kWaitTimeoutNs;
+    int skip_release = 0;
+};
+
 template <int D>
 int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
-           void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
+           void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts,
+           const SplitTestHooks& hooks = SplitTestHooks()) {
     constexpr int kStagesD = kStages<D>;
     // the lean per-tile form everywhere but D = 256 and the CTA-local plan at D = 128
     // (the kernel's LEAN parameter lists the measurements)
@@ -531,6 +540,8 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     sp.stage_bytes = stage_bytes(s);
     sp.q_box_bytes = static_cast<uint32_t>(s.rows_max) * s.D * 2u;
     sp.scale_log2 = scale * 1.4426950408889634f;
+    sp.wait_ns = hooks.wait_ns;
+    sp.test_skip_release = hooks.skip_release;
 
     // Both kernels are launched with programmatic dependent launch (PDL): each
     // begins launching while the previous kernel in the stream drains, and waits
@@ -1007,7 +1018,7 @@ namespace {
 int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
                 const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out, float scale,
                 int num_splits, void* workspace, size_t workspace_bytes, apd_stream_t stream,
-                const apd_launch_options* options) {
+                const apd_launch_options* options, const SplitTestHooks* hooks = nullptr) {
     if (options && options->reserved != 0) return APD_ERR_ARGUMENT;
     Validated V;
     int rc = validate(q, k_cache, v_cache, page_table, seq_lens, out, num_splits, &V);
@@ -1029,12 +1040,15 @@ int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor
     rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl,
                    options ? options->host_seq_lens : nullptr, static_cast<int64_t>(V.MP) * V.P);
     if (rc) return rc;
+    const SplitTestHooks h = hooks ? *hooks : SplitTestHooks();
+    // the release self-test needs the shared K/V ring (auto splits, more than 16 q heads per kv head)
+    if (h.skip_release && !pl.share) return APD_ERR_ARGUMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (V.s.D) {
-        case 32: return launch<32>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
-        case 64: return launch<64>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
-        case 128: return launch<128>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
-        case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options);
+        case 32: return launch<32>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options, h);
+        case 64: return launch<64>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options, h);
+        case 128: return launch<128>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options, h);
+        case 256: return launch<256>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options, h);
         default: return APD_ERR_HEAD_DIM;
     }
 }
@@ -1343,6 +1357,19 @@ const char* apd_status_string(int status) {
 const char* apd_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"
+
+int apd_selftest_shared_ring_release(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                                     const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     uint64_t short_timeout_ns, apd_stream_t stream) {
+    if (!page_table) return APD_ERR_NULL_POINTER;
+    if (short_timeout_ns == 0 || short_timeout_ns > 1000000000ull) return APD_ERR_ARGUMENT;
+    SplitTestHooks h;
+    h.wait_ns = short_timeout_ns;
+    h.skip_release = 1;
+    return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, scale, 0, workspace, workspace_bytes, stream,
+                       nullptr, &h);
+}
 
 int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stream_t stream) {
     if (!out) return APD_ERR_NULL_POINTER;

@@ -61,6 +61,37 @@ constexpr uint32_t kFlagLenNegative = 0x4u;
 constexpr uint32_t kFlagTimeout = 0x8u;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per async-copy wait
 
+// Wait, as one warp, for phase `parity` of an mbarrier.  Every lane polls, and lane 0
+// decides for the whole warp when to give up, so the lanes never part ways: once
+// `abort_word` (if given) has been raised by another warp of the CTA, or after about
+// timeout_ns, when lane 0 raises `abort_word` and sets kFlagTimeout in `flags` (each if
+// given).  Returns false when it gave up.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                          volatile uint32_t* abort_word, uint32_t* flags) {
+    bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (!done) done = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if ((it & 15u) == 0) {
+            int give_up = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (abort_word && *abort_word) give_up = 1;
+                else if (global_timer_ns() - t0 > timeout_ns) give_up = 2;
+            }
+            give_up = __shfl_sync(0xffffffffu, give_up, 0);
+            if (give_up) {
+                if (give_up == 2 && (threadIdx.x & 31) == 0) {
+                    if (abort_word) *abort_word = 1u;
+                    if (flags) atomicOr(flags, kFlagTimeout);
+                }
+                return false;
+            }
+        }
+    }
+}
+
 struct SplitParams {
     const int32_t* page_table;  // NULL: contiguous KV, sequence b is page b
     int64_t pt_s0, pt_s1;
@@ -80,6 +111,8 @@ struct SplitParams {
     int32_t warps;      // warps per CTA
     uint32_t stage_bytes, q_box_bytes;
     float scale_log2;
+    uint64_t wait_ns;           // limit of each mbarrier wait (kWaitTimeoutNs; shorter in the self-test)
+    int32_t test_skip_release;  // self-test only: followers never release a shared stage (0 otherwise)
 };
 
 struct CombineParams {
@@ -279,7 +312,9 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empties = bars + p.warps * STAGES;  // SHARE: stage released by the followers
     uint64_t* merge_bar = empties + (SHARE ? p.warps * STAGES : 0);  // CTA-local mode: the parts of the CTA's unit are in
-    int32_t* s_len = reinterpret_cast<int32_t*>(merge_bar + 1);
+    // raised by a warp that gave up on a wait: the CTA's other waits then give up too
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(merge_bar + 1);
+    int32_t* s_len = reinterpret_cast<int32_t*>(merge_bar + 2);
     int32_t* s_cum = s_len + B;
     const uint32_t meta_end = smem_u32(s_cum + B + 1);
     const uint32_t ring = (meta_end + 1023u) & ~1023u;
@@ -311,7 +346,10 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         s_len[b] = L;
         s_cum[b + 1] = (L + kTile - 1) / kTile;
     }
-    if (tid == 0) s_cum[0] = 0;
+    if (tid == 0) {
+        s_cum[0] = 0;
+        *s_abort = 0u;
+    }
     if (len_flags && blockIdx.x == 0) atomicOr(p.flags, len_flags);
     __syncthreads();
     if (SHARE && warp == 1) {
@@ -467,8 +505,9 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
     int32_t pg_cur = follower ? 0 : fetch_page(p, s_cum, ws + lane, we);
     int32_t pg_nxt = follower ? 0 : fetch_page(p, s_cum, ws + 32 + lane, we);
 
+    bool stopped = false;  // the leader of a shared ring gave up on a release: no further issues
     auto issue_next = [&](int stage) {
-        if (pi >= we) return;
+        if (pi >= we || stopped) return;
         if (follower) {
             // this warp's Q rows only; an expect of 0 bytes keeps one phase per tile
             const bool qload = (pj == 0) || (pi == ws);
@@ -486,11 +525,14 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
             return;
         }
         if (SHARE && pi - ws >= STAGES) {
-            // the followers have read the tile this stage held, STAGES tiles back
+            // the followers have read the tile this stage held, STAGES tiles back.  If they
+            // never release it (a follower gave up), issue nothing more: the stage may still
+            // be read, and the consumer loop below stops at the first tile not issued.
             const int kk = pi - ws - STAGES;
-            if (!mbar_wait_bounded(empty0 + 8 * stage, static_cast<uint32_t>(kk / STAGES) & 1u, kWaitTimeoutNs) &&
-                lane == 0)
-                atomicOr(p.flags, kFlagTimeout);
+            if (!warp_wait(empty0 + 8 * stage, static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns, s_abort, p.flags)) {
+                stopped = true;
+                return;
+            }
         }
         int off = pi - wbase;
         if (off >= 32) {
@@ -550,16 +592,18 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         const uint32_t qbase_t = q_ring + static_cast<uint32_t>(stage) * q_step;  // this warp's Q
         const bool unit_start = (cj == 0) || (i == ws);
 
-        if (!mbar_wait_bounded(kv_bar0 + 8 * stage, parity, kWaitTimeoutNs) ||
-            (follower && !mbar_wait_bounded(bar0 + 8 * stage, parity, kWaitTimeoutNs))) {
-            if (lane == 0) atomicOr(p.flags, kFlagTimeout);
-            // Give the other copies in flight a bounded chance to land, then stop.
+        if (i >= pi || !warp_wait(kv_bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags) ||
+            (follower && !warp_wait(bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags))) {
+            // Gave up (this warp timed out, another warp of the CTA did, or this warp, as the
+            // leader of a shared ring, stopped issuing): let this warp's own copies in flight
+            // land, each wait bounded, then stop.
+            *s_abort = 1u;
             for (int s = 0; s < STAGES; ++s) {
                 const int t = i + s;
                 if (t < pi) {
                     const int kk = t - ws;
-                    mbar_wait_bounded(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u,
-                                      kWaitTimeoutNs / 8);
+                    warp_wait(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns / 8,
+                              nullptr, nullptr);
                 }
             }
             return;
@@ -735,7 +779,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         // before the async-proxy write, then the warp syncs before lane 0 issues.
         fence_proxy_async_smem();
         __syncwarp();
-        if (follower && lane == 0) mbar_arrive(empty0 + 8 * stage);  // the leader may refill it
+        if (follower && lane == 0 && !p.test_skip_release) mbar_arrive(empty0 + 8 * stage);  // the leader may refill it
         issue_next(stage);
 
         // ---- end of this unit's run in this worker: write output or a partial
@@ -793,10 +837,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         // every lane's part rows are written: arrive, wait (bounded) for the other parts,
         // and merge this warp's share of the rows
         mbar_arrive(smem_u32(merge_bar));
-        if (!mbar_wait_bounded(smem_u32(merge_bar), 0u, kWaitTimeoutNs)) {
-            if (lane == 0) atomicOr(p.flags, kFlagTimeout);
-            return;
-        }
+        if (!warp_wait(smem_u32(merge_bar), 0u, p.wait_ns, s_abort, p.flags)) return;
         cta_local_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, cb,
                            head0, rows, warp, nparts, lane);
     }

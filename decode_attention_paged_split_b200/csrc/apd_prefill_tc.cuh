@@ -196,44 +196,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return d;
 }
 
-// 2^x for a pair on the FMA pipe, so that part of the exponentials leave the MUFU
-// unit (which bounds the softmax otherwise).  Cody-Waite style: x = j + f with j =
-// round(x) taken from the low mantissa bits of x + 1.5 * 2^23 and f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial whose coefficients come from exp2_poly.py (maximum
-// relative error 1.0e-4, far below bf16's 2^-9); j is added to the exponent field.
-// x is clamped to >= -125 so that the exponent field stays positive (2^-125 is
-// negligible next to the row's maximum weight, which is >= 2^-8 ... 2^8).
-__device__ __forceinline__ void exp2_fma2(uint64_t x2, float& p0, float& p1) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    float x0, x1;
-    f2_unpack(x2, x0, x1);
-    const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = f2_add(xc, f2_pack(kRound, kRound));
-    const uint64_t jf = f2_add(t, f2_pack(-kRound, -kRound));
-    const uint64_t fr = f2_fma(jf, f2_pack(-1.f, -1.f), xc);
-    uint64_t q = f2_fma(fr, f2_pack(0.0550354384f, 0.0550354384f), f2_pack(0.242211014f, 0.242211014f));
-    q = f2_fma(q, fr, f2_pack(0.693277419f, 0.693277419f));
-    q = f2_fma(q, fr, f2_pack(1.f, 1.f));
-    float t0, t1, q0, q1;
-    f2_unpack(t, t0, t1);
-    f2_unpack(q, q0, q1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
-// Which pairs of each group of 8 take exp2_fma2 instead of MUFU ex2 (bit c of the mask
-// for pair c mod 8).  Measured on the 128-token chunk workload (D = 128): none 188.6 us,
-// 2/8 195.0 us, 3/8 199.5 us, 4/8 200.2 us -- the MUFU pipe is not what bounds the
-// softmax of the two-tile kernel, so the default sends every exponential to MUFU.
 // Parts in which a softmax warpgroup of the two-tile kernel hands P over to the MMA
 // issuer (the first parts' P V runs while the later parts' exponentials are computed).
 // Chunk workload (D = 128): 1 part 185.2 us, 2 parts 183.6 us, 4 parts 181.7 us.
 #ifndef APD_PREFILL_P_PARTS
 #define APD_PREFILL_P_PARTS 4
-#endif
-
-#ifndef APD_EXP2_FMA_MASK
-#define APD_EXP2_FMA_MASK 0x00u
 #endif
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -1146,15 +1113,9 @@ __global__ void __launch_bounds__(Tc2Shape<D>::kThreads, 1)
                     const uint64_t x2 = f2_fma(
                         f2_pack(__uint_as_float(sr[32 * hh + 2 * c]), __uint_as_float(sr[32 * hh + 2 * c + 1])), cs2,
                         nref2);
-                    float p0, p1;
-                    if ((APD_EXP2_FMA_MASK >> (c & 7)) & 1u) {
-                        exp2_fma2(x2, p0, p1);
-                    } else {
-                        float x0, x1;
-                        f2_unpack(x2, x0, x1);
-                        p0 = ex2_approx(x0);
-                        p1 = ex2_approx(x1);
-                    }
+                    float x0, x1;
+                    f2_unpack(x2, x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     rs2[c & 1] = f2_add(rs2[c & 1], f2_pack(p0, p1));
                     pw[c] = pack_bf16x2(p0, p1);
                 }

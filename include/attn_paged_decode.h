@@ -403,6 +403,27 @@ int apd_read_device_flags(const void* workspace, size_t workspace_bytes, apd_str
  */
 int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stream_t stream);
 
+/*
+ * apd_selftest_shared_ring_release -- exercises, on the GPU and without any fault, the
+ * error path of the shared K/V ring (auto splits with more than 16 query heads per kv
+ * head, where the head blocks of a kv head share one ring that the first of them fills
+ * and the others release stage by stage).  It runs apd_attn_paged_decode(num_splits = 0)
+ * on the given problem with two differences: the followers never release a stage, and
+ * every mbarrier wait gives up after `short_timeout_ns` (1 .. 1e9 ns) instead of 2 s.
+ * Each ring's leader must then give up on its first refill, stop issuing copies, wait
+ * (bounded) for its copies in flight and return; its followers must give up on their
+ * next wait through the CTA's abort word.  The call ends within a few limits, the flag
+ * word in the workspace gets APD_FLAG_WAIT_TIMEOUT, and `out` is undefined.
+ *
+ *   Arguments as apd_attn_paged_decode with num_splits = 0.  Returns APD_ERR_ARGUMENT
+ *   before any launch when the problem does not take the shared ring (16 or fewer q
+ *   heads per kv head) or the limit is out of range; otherwise as that call.
+ */
+int apd_selftest_shared_ring_release(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                                     const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     uint64_t short_timeout_ns, apd_stream_t stream);
+
 /* apd_plan -- how a call with these arguments would be launched (for tests,
  * benchmarks and profiling). */
 typedef struct apd_plan {
@@ -444,7 +465,12 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
                       size_t workspace_bytes, int sm_count, const int32_t* host_seq_lens, int64_t max_seq_len,
                       apd_plan* plan);
 
-/* Human-readable text for an apd_status (never NULL). */
+/* apd_status_string -- human-readable text for an apd_status (never NULL; unknown codes
+ * give "unknown status").  The statuses are the argument checks that the AstrAI commit
+ * log of csrc/kernels/attn_paged_decode.cu lists for the decode entry (q_head divisible
+ * by kv_head, head-dim contiguity, the split-KV scratch and output layout), plus this
+ * library's own size, workspace and CUDA failures.  The returned string is static: do
+ * not free it. */
 const char* apd_status_string(int status);
 
 /* Text of the last CUDA error seen by this thread inside the library ("" if none). */

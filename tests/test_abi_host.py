@@ -230,10 +230,11 @@ _SHARE_TRAITS = {32: None, 64: (4, 8), 128: (2, 8), 256: (2, 4)}
 
 def _smem(B, D, rows, warps, stages, hb, shared):
     """Dynamic shared memory of the split kernel: mbarriers (full, plus empty when the K/V
-    ring is shared), the merge barrier, lengths and prefix sums, 1 KB of alignment slack,
-    then the rings: per warp [K | V | Q] stages, or, shared, one K/V ring per kv head and
-    one Q ring per warp (K and V tiles are 32 tokens x D bf16, Q tiles 1 KB aligned)."""
-    meta = 8 * warps * stages * (2 if shared else 1) + 8 + 4 * (2 * B + 1)
+    ring is shared), the merge barrier, the CTA's abort word (8 bytes), lengths and prefix
+    sums, 1 KB of alignment slack, then the rings: per warp [K | V | Q] stages, or, shared,
+    one K/V ring per kv head and one Q ring per warp (K and V tiles are 32 tokens x D bf16,
+    Q tiles 1 KB aligned)."""
+    meta = 8 * warps * stages * (2 if shared else 1) + 8 + 8 + 4 * (2 * B + 1)
     kv = 2 * 32 * D * 2
     q = -(-rows * D * 2 // 1024) * 1024
     rings = (warps // hb * stages * kv + warps * stages * q) if shared else warps * stages * (kv + q)
@@ -474,6 +475,25 @@ def test_selftest_arguments_are_checked_before_any_launch():
     assert L.apd_selftest_bounded_wait(None, 1000, None) == NULLP
     assert L.apd_selftest_bounded_wait(FAKE, 0, None) == ARG
     assert L.apd_selftest_bounded_wait(FAKE, 2_000_000_000, None) == ARG
+
+
+def test_release_selftest_arguments_are_checked_before_any_launch():
+    """The shared-ring release self-test: a NULL page table, a limit outside 1 ns .. 1 s, and a
+    problem that does not take the shared ring (g <= 16) are refused without a launch."""
+    L = apd.lib()
+
+    def call(p, limit=1_000_000, pt=True):
+        a = [ctypes.byref(p[n]) for n in ("q", "k", "v")] + [ctypes.byref(p["pt"]) if pt else None] + \
+            [ctypes.byref(p[n]) for n in ("sl", "out")]
+        return L.apd_selftest_shared_ring_release(*a, ctypes.c_float(0.1), FAKE, 1 << 30, limit, None)
+
+    g32 = dict(q=T([2, 64, 128]), out=T([2, 64, 128]), k=T([16, 32, 2, 128]), v=T([16, 32, 2, 128]),
+               pt=T([2, 4], apd.DTYPE_INT32), sl=T([2], apd.DTYPE_INT32))
+    assert call(g32, pt=False) == NULLP
+    assert call(g32, limit=0) == ARG
+    assert call(g32, limit=2_000_000_000) == ARG
+    g4 = dict(g32, q=T([2, 8, 128]), out=T([2, 8, 128]))
+    assert call(g4) in (ARG, CUDA)  # ARG once the plan is made (it needs the device's SM count)
 
 
 # ---------------------------------------------------------------- GEMV planning

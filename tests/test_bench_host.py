@@ -53,6 +53,47 @@ def test_max_and_sum_over_two_gloo_ranks():
         assert b == 30.0  # bytes of all ranks
 
 
+def _reps_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist = bench.init_group(world, "gloo")
+    dev = torch.device("cpu")
+    calls = [0]
+
+    def run():  # rank 1 is twice as slow, and its first (untimed) region looks very long
+        calls[0] += 1
+        return (5.0 if calls[0] == 1 and rank == 1 else 0.01 * (rank + 1))
+
+    times = bench.timed_reps(run, dist, dev, min_seconds=0.05)
+    q.put((rank, times))
+    dist.destroy_process_group()
+
+
+def test_timed_repetitions_agree_over_two_gloo_ranks():
+    """Every rank runs the same number of repetitions (the most any rank asked for) and each
+    repetition's time is the max over ranks."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_reps_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=10) for _ in range(2))
+    assert got[0] == got[1]
+    assert len(got[0]) == 5  # rank 0: 0.05 s / 0.01 s per region
+    assert all(t == 0.02 for t in got[0])
+
+
+def test_timing_summary():
+    s = bench.timing_summary([0.004, 0.002, 0.003], 20)
+    assert s["reps"] == 3 and s["steps_per_rep"] == 20
+    assert abs(s["median_us_per_call"] - 150.0) < 1e-9
+    assert abs(s["min_us_per_call"] - 100.0) < 1e-9 and abs(s["max_us_per_call"] - 200.0) < 1e-9
+
+
 def test_single_process_reductions_are_identity():
     assert bench.max_over_ranks(3.5, None, torch.device("cpu")) == 3.5
     assert bench.sum_over_ranks(7.0, None, torch.device("cpu")) == 7.0

@@ -28,3 +28,39 @@ def test_context_is_usable_after_a_wait_gave_up():
                        seq_lens=[100, 7, 64], page_size=32)
     dp = DeviceProblem(w)
     check_close(dp.run(0), oracle.paged_decode(w), "decode after the self-test")
+
+
+def test_shared_ring_leader_stops_when_a_release_never_comes():
+    """The shared K/V ring's error path (more than 16 q heads per kv head, auto splits): the
+    self-test runs the real decode with followers that never release a stage and a 1 ms
+    limit per wait.  Each ring's leader must give up at its first refill, stop issuing and
+    return, and its followers must stop through the CTA's abort word, so the call ends
+    within a few limits (a leader that kept refilling would wait out one limit per tile:
+    over 100 ms here) with APD_FLAG_WAIT_TIMEOUT set.  A normal call afterwards is correct."""
+    w = workloads.make(name="ring_release", seed=83, batch=4, num_q_heads=64, num_kv_heads=2, head_dim=128,
+                       seq_lens=[16384, 16000, 12000, 16384], page_size=32)
+    dp = DeviceProblem(w)
+    default = apd.workspace_size(4, 64, 2, 128, 0)
+    ws = torch.zeros(default // 16 // 256 * 256, dtype=torch.uint8, device="cuda")  # long runs per warp
+    plan = apd.query_plan(4, 64, 2, 128, 0, workspace_bytes=ws.numel())
+    assert plan.shared_kv_ring == 1 and plan.mode == 0
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    apd.selftest_shared_ring_release(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, ws, 1_000_000)
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert apd.read_device_flags(ws) & apd.FLAG_WAIT_TIMEOUT
+    assert ms < 30.0, f"the self-test call took {ms:.1f} ms"
+    check_close(dp.run(0, workspace=ws), oracle.paged_decode(w), "decode after the release self-test")
+    assert apd.read_device_flags(ws) == 0
+
+
+def test_release_selftest_needs_the_shared_ring():
+    w = workloads.make(name="no_ring", seed=84, batch=2, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                       seq_lens=[64, 96], page_size=32)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(2, 32, 8, 128, 0)
+    with pytest.raises(apd.APDError):
+        apd.selftest_shared_ring_release(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, ws)

@@ -6,8 +6,9 @@ library's built-in static device scratch instead.
 
 The GPU test calls it through the C ABI (ctypes, no binding helper) twice in a row,
 so the second call runs on scratch the first one left behind. Each time it
-compares the output with the workspace entry point's, within the tolerance of the
-parity tests.  This file is named so that pytest collects it last.
+compares the output with the workspace entry point's and with the fp64 oracle,
+within the tolerance of the parity tests.  This file is named so that pytest
+collects it last.
 """
 import ctypes
 
@@ -16,7 +17,9 @@ import pytest
 import torch
 
 import decode_attention_paged_split_b200 as apd
+import oracle
 import workloads
+from gpu_util import check_close
 
 SCRATCH_LIMIT = 13  # APD_ERR_SCRATCH_LIMIT
 ATOL = RTOL = 1e-2  # the parity tests' per-element bound
@@ -74,6 +77,7 @@ def test_noalloc_matches_workspace_entry_twice(name, make, splits):
     apd.attn_paged_decode(q, k, v, pt, sl, ref_out, w.scale, splits, ws)
     ref = ref_out.to(torch.float64).cpu().numpy()
     assert np.isfinite(ref).all()
+    oref = oracle.paged_decode(w)
     stream = torch.cuda.current_stream().cuda_stream or None
     for call in range(2):
         out = torch.full_like(q, float("nan"))
@@ -84,3 +88,4 @@ def test_noalloc_matches_workspace_entry_twice(name, make, splits):
         assert np.isfinite(got).all(), f"{name} call {call}: non-finite output"
         err = np.abs(got - ref)
         assert (err <= ATOL + RTOL * np.abs(ref)).all(), f"{name} call {call}: max err {err.max():.3e}"
+        check_close(out, oref, f"{name} call {call} against the oracle")
