@@ -110,13 +110,20 @@ uint32_t stage_bytes(const Shape& s) { return 2u * apd::kTile * s.D * 2u + q_til
 // share: the layout where the HB warps of a kv head share one K/V ring (the balanced mode
 // when g > 16): warps / HB K/V rings and `warps` Q rings, and an `empty` mbarrier per stage.
 size_t smem_bytes(const Shape& s, int warps, int stages, bool share = false) {
-    // mbarriers (full, and empty in the shared layout), the merge mbarrier, the abort word
-    // (8 bytes), lengths and prefix sums
-    const size_t meta = 8ull * warps * stages * (share ? 2 : 1) + 8 + 8 + 4ull * (2ull * s.B + 1);
+    // mbarriers (full, and empty in the shared layout), the abort word (8 bytes), lengths and
+    // prefix sums
+    const size_t meta = 8ull * warps * stages * (share ? 2 : 1) + 8 + 4ull * (2ull * s.B + 1);
     const size_t rings = share ? static_cast<size_t>(warps / s.HB) * stages * (2ull * apd::kTile * s.D * 2) +
                                      static_cast<size_t>(warps) * stages * q_tile_bytes(s)
                                : static_cast<size_t>(warps) * stages * stage_bytes(s);
     return align_up(meta, 16) + 1024 + rings;
+}
+
+// The one-CTA-per-unit kernel (unit_kernel): full mbarriers, the merge mbarrier, the abort
+// word and tile counter (8 bytes), the claimed tile of each stage, then the per-warp rings.
+size_t unit_smem_bytes(const Shape& s, int warps, int stages) {
+    const size_t meta = 8ull * warps * stages + 8 + 8 + 4ull * warps * stages;
+    return align_up(meta, 16) + 1024 + static_cast<size_t>(warps) * stages * stage_bytes(s);
 }
 
 // The most warps per CTA that fit (a multiple of HB in the shared layout), or 0.
@@ -150,14 +157,16 @@ struct Plan {
     size_t ws_needed;
 };
 
-// CTA-local plan (mode 2): CTA u owns unit u and its warps take equal parts of the unit's
-// tiles, merged in shared memory; a single launch, no partials in the workspace.
+// One-CTA-per-unit plan (mode 2, unit_kernel): CTA u owns unit u, its warps claim the
+// unit's tiles from a shared counter and merge their parts in shared memory; a single
+// launch, no partials in the workspace.
 void cta_local_plan(const Shape& s, Plan* pl) {
     pl->mode = 2;
     pl->share = false;
     pl->stages = traits_for(s.D).stages;
-    pl->warps = warps_for(s);
-    pl->smem = smem_bytes(s, pl->warps, pl->stages);
+    pl->warps = traits_for(s.D).max_warps;
+    while (pl->warps > 1 && unit_smem_bytes(s, pl->warps, pl->stages) > kSmemLimit) --pl->warps;
+    pl->smem = unit_smem_bytes(s, pl->warps, pl->stages);
     pl->ksplit = pl->warps;
     pl->groups = 0;
     pl->workers = static_cast<int>(s.units * pl->warps);
@@ -166,7 +175,7 @@ void cta_local_plan(const Shape& s, Plan* pl) {
     pl->combine_ctas = 0;
 }
 
-// Whether the CTA-local plan beats the balanced plan `pl` for these host-known lengths
+// Whether the one-CTA-per-unit plan beats the balanced plan `pl` for these host-known lengths
 // (clamped to [0, len_cap] as the kernels clamp them).  Only when every unit gets a CTA
 // of its own on a distinct SM, and the longest unit is at most the balanced plan's
 // share per CTA plus about what the combine kernel costs: 3% and 1024 / D tiles.
@@ -271,7 +280,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
-    bool smem_attr_set[12] = {};  // split kernel: head dim x {plain ring, shared ring, CTA-local at D = 128}
+    bool smem_attr_set[12] = {};  // head dim x {split kernel, split kernel with shared rings, unit kernel}
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -474,8 +483,8 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts,
            const SplitTestHooks& hooks = SplitTestHooks()) {
     constexpr int kStagesD = kStages<D>;
-    // the lean per-tile form everywhere but D = 256 and the CTA-local plan at D = 128
-    // (the kernel's LEAN parameter lists the measurements)
+    // the lean per-tile form everywhere but D = 256 (the split kernel's LEAN parameter lists
+    // the measurements)
     constexpr bool kLeanD = D != 256;
     auto kern = apd::split_kernel<D, kStagesD, false, kLeanD>;
     int variant = 0;
@@ -485,11 +494,11 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
             variant = 1;
         }
     }
-    if constexpr (D == 128) {
-        if (pl.mode == 2) {
-            kern = apd::split_kernel<D, kStagesD, false, false>;
-            variant = 2;
-        }
+    if (pl.mode == 2) {
+        // one CTA per unit: the lean per-tile form at D = 32 and 64 only (the plain form
+        // measured 1% faster for the llama8b shape at D = 128)
+        kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64)>;
+        variant = 2;
     }
     const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + 4 * variant;
     {

@@ -104,7 +104,7 @@ struct SplitParams {
     int32_t zero_empty;  // balanced mode with no combine kernel: write the rows of empty sequences
     uint32_t* flags;
     int32_t B, Hq, Hkv, g, HB, rows_max, P, NP, MP;
-    int32_t mode;       // 0 balanced, 1 fixed
+    int32_t mode;       // 0 balanced, 1 fixed (split_kernel); 2 one CTA per unit (unit_kernel)
     int32_t ksplit;     // fixed mode: k
     int32_t num_workers;
     int32_t groups;     // balanced mode: worker groups (num_workers = groups * Hkv * HB)
@@ -224,411 +224,50 @@ __device__ __forceinline__ void write_zero_rows(const SplitParams& p, int b, int
     }
 }
 
-// CTA-local mode: CTA u owns unit u (sequence u / (Hkv * HB)); its warps take equal
-// parts of the unit's tiles, as fixed splits do, and merge them through shared memory.
-__device__ __forceinline__ int cta_local_tiles(const SplitParams& p, const int32_t* s_cum, int u) {
-    const int b = u / (p.Hkv * p.HB);
-    return s_cum[b + 1] - s_cum[b];
-}
-// Non-empty parts when n tiles are cut into at most W parts of ceil(n / min(W, n)) tiles.
-__device__ __forceinline__ int cta_local_parts(int n, int W) {
-    const int S = min(W, n);
-    const int c = (n + S - 1) / S;
-    return (n + c - 1) / c;
-}
-
-// Row stride (floats) of a CTA-local part's accumulator rows in shared memory: 8 floats of
-// padding put the 8 rows one warp store touches on different banks.
-template <int D>
-constexpr int kPartStride = D + 8;
-
-// Merge of the CTA-local parts of one unit: part k's (m, l) rows at ml_k = the start of
-// warp k's first ring stage, its accumulator rows [kMaxRows][kPartStride] (fp32) 128
-// bytes later.
-// Warp `part` of `nparts` merges rows part, part + nparts, ...:
-//   M = max_k m_k over parts with l_k > 0, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
-template <int D>
-__device__ __noinline__ void cta_local_merge(const SplitParams& p, const uint8_t* ring0, uint32_t warp_bytes,
-                                                int b, int head0, int rows, int part, int nparts, int lane) {
-    constexpr int kVec = D / 32;  // consecutive columns per lane
-    for (int r = part; r < rows; r += nparts) {
-        float M = -INFINITY;
-        for (int k = 0; k < nparts; ++k) {
-            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
-            if (ml[2 * r + 1] > 0.f) M = fmaxf(M, ml[2 * r]);
-        }
-        float den = 0.f, acc[kVec];
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
-        for (int k = 0; k < nparts; ++k) {
-            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
-            if (!(ml[2 * r + 1] > 0.f)) continue;
-            const float wk = exp2f(ml[2 * r] - M);
-            den += wk * ml[2 * r + 1];
-            const float* a = ml + 2 * kMaxRows + r * kPartStride<D> + kVec * lane;
-            float v[kVec];  // this lane's kVec consecutive columns, in 16- (or 8-) byte loads
-            if constexpr (kVec % 4 == 0) {
-#pragma unroll
-                for (int e = 0; e < kVec; e += 4) *reinterpret_cast<float4*>(v + e) = *reinterpret_cast<const float4*>(a + e);
-            } else if constexpr (kVec == 2) {
-                *reinterpret_cast<float2*>(v) = *reinterpret_cast<const float2*>(a);
-            } else {
-                v[0] = a[0];
-            }
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) acc[e] += wk * v[e];
-        }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        __nv_bfloat16* o = p.out + b * p.out_sb + (head0 + r) * p.out_sh + kVec * lane;
-        if constexpr (kVec == 1) {
-            o[0] = __float2bfloat16_rn(acc[0] * inv);
-        } else {
-#pragma unroll
-            for (int e = 0; e < kVec; e += 2)
-                *reinterpret_cast<uint32_t*>(o + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
-        }
-    }
-}
-
-// SHARE (balanced mode with g > 16, so HB = ceil(g / 16) head blocks per kv head): the HB
-// warps of one kv head, which walk the same positions in one CTA, share one K/V ring, which
-// the first of them (the leader) fills.  Before refilling a stage the leader waits on that
-// stage's `empty` mbarrier, on which the other HB - 1 warps arrive once they have read the
-// tile.  Each warp loads its own Q rows into a Q ring of its own.  Shared-memory layout:
-// [K/V rings, one per kv head of the CTA][Q rings, one per warp], so a CTA of HB warps
-// holds one K/V ring instead of HB.
-template <int D, int STAGES, bool SHARE, bool LEAN>
-__global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
-    split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
-                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
+// The running state of one warp over the tiles of one unit: the query rows' mma A-fragments,
+// the fp32 accumulators of O (rows gq and gq + 8 of the 16-row head tile, columns 8 nd +
+// 2 tq, + 1), the row sums and the row maxima (in log2 units).  step() consumes one staged
+// 32-token K/V tile.
+template <int D, bool LEAN>
+struct TileAcc {
     using G = Geometry<D>;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int warp = tid >> 5;
-    const int B = p.B;
-
-    // ---- shared-memory carve-up: mbarriers, lengths, prefix sums, stage ring
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* empties = bars + p.warps * STAGES;  // SHARE: stage released by the followers
-    uint64_t* merge_bar = empties + (SHARE ? p.warps * STAGES : 0);  // CTA-local mode: the parts of the CTA's unit are in
-    // raised by a warp that gave up on a wait: the CTA's other waits then give up too
-    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(merge_bar + 1);
-    int32_t* s_len = reinterpret_cast<int32_t*>(merge_bar + 2);
-    int32_t* s_cum = s_len + B;
-    const uint32_t meta_end = smem_u32(s_cum + B + 1);
-    const uint32_t ring = (meta_end + 1023u) & ~1023u;
-
-    if (tid == 0) {
-        prefetch_tensormap(&kmap);
-        prefetch_tensormap(&vmap);
-        prefetch_tensormap(&qmap);
-    }
-    // Launched with programmatic dependent launch: this CTA may start while the
-    // previous kernel in the stream is still running.  Nothing above touches
-    // global memory; from here on, that kernel has finished and its writes are
-    // visible.
-    pdl_wait_prior_grid();
-
-    // ---- per-sequence tile counts and their prefix sum (every CTA, from L2)
-    const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
-    uint32_t len_flags = 0;
-    for (int b = tid; b < B; b += blockDim.x) {
-        int L = __ldcg(p.seq_lens + b);
-        if (L < 0) {
-            L = 0;
-            len_flags |= kFlagLenNegative;
-        }
-        if (L > cap) {
-            L = static_cast<int>(cap);
-            len_flags |= kFlagLenClamped;
-        }
-        s_len[b] = L;
-        s_cum[b + 1] = (L + kTile - 1) / kTile;
-    }
-    if (tid == 0) {
-        s_cum[0] = 0;
-        *s_abort = 0u;
-    }
-    if (len_flags && blockIdx.x == 0) atomicOr(p.flags, len_flags);
-    __syncthreads();
-    if (SHARE && warp == 1) {
-        // every warp's ring barriers, before any warp waits on another warp's
-        for (int i = lane; i < p.warps * STAGES; i += 32) {
-            mbar_init(smem_u32(bars + i), 1);
-            mbar_init(smem_u32(empties + i), static_cast<uint32_t>(p.HB - 1));
-        }
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        const int per = (B + 31) / 32;
-        const int lo = 1 + lane * per;
-        const int hi = min(lo + per, B + 1);
-        int sum = 0;
-        for (int i = lo; i < hi; ++i) sum += s_cum[i];
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-        for (int i = lo; i < hi; ++i) {
-            run += s_cum[i];
-            s_cum[i] = run;
-        }
-        __syncwarp();
-        if (p.mode == 2 && lane == 0) {
-            // one arrival per non-empty part of this CTA's unit
-            const int n = cta_local_tiles(p, s_cum, blockIdx.x);
-            mbar_init(smem_u32(merge_bar), static_cast<uint32_t>(32 * (n >= 2 ? cta_local_parts(n, p.ksplit) : 1)));
-            fence_mbar_init();
-        }
-    }
-    __syncthreads();
-    if (blockIdx.x == 0) {
-        for (int i = tid; i <= B; i += blockDim.x) p.cum_out[i] = s_cum[i];
-    }
-    // The combine kernel may start its launch now; it waits (griddepcontrol.wait)
-    // for this whole grid to finish before it reads anything.
-    pdl_launch_dependents();
-    // No CTA-wide barrier after this point: warps are independent workers (in the
-    // CTA-local mode the parts of the CTA's unit meet on an mbarrier, with a bounded wait).
-
-    const int units_per_seq = p.Hkv * p.HB;
-    const int w = blockIdx.x * p.warps + warp;
-    if (w >= p.num_workers) return;
-    if (p.zero_empty) {
-        // no combine kernel follows: the workers write the zero rows of empty sequences
-        for (int u = w; u < p.B * units_per_seq; u += p.num_workers) {
-            const int b = u / units_per_seq;
-            if (s_cum[b + 1] != s_cum[b]) continue;
-            const int ulz = u - b * units_per_seq, kvh = ulz / p.HB, hb = ulz - (ulz / p.HB) * p.HB;
-            write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
-        }
-    }
-
-    // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-
-    // sequence ul (kv head and head block).
-    int ws, we, ul;
-    int fixed_slot = -1;
-    if (p.mode == 0) {
-        // Workers form groups of units_per_seq warps, one per (kv head, head block);
-        // group grp owns an equal share of the positions of all sequences.  The warps
-        // of a group walk the same pages together, so the kv heads of a page are read
-        // at about the same time.
-        const int grp = w / units_per_seq;
-        ul = w - grp * units_per_seq;
-        ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
-        we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
-    } else {
-        // fixed splits (mode 1), or the CTA-local mode (2: ksplit = warps, so unit u is
-        // CTA u and its parts are the CTA's warps)
-        const int u = w / p.ksplit;
-        const int s = w - u * p.ksplit;
-        const int b = u / units_per_seq;
-        ul = u - b * units_per_seq;
-        const int n = s_cum[b + 1] - s_cum[b];
-        if (n == 0) {
-            if (s == 0) {
-                const int kvh = ul / p.HB, hb = ul - (ul / p.HB) * p.HB;
-                write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
-            }
-            return;
-        }
-        const int S = min(p.ksplit, n);
-        const int c = (n + S - 1) / S;
-        const int t0 = s * c;
-        if (t0 >= n) return;
-        const int t1 = min(t0 + c, n);
-        ws = s_cum[b] + t0;
-        we = s_cum[b] + t1;
-        fixed_slot = u * p.ksplit + s;
-    }
-    if (ws >= we) return;
-
-    const uint32_t bar0 = smem_u32(bars + warp * STAGES);
-    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;  // unshared layout
-    if constexpr (!SHARE) {
-        if (lane == 0) {
-#pragma unroll
-            for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
-            fence_mbar_init();
-        }
-        __syncwarp();
-    }
-
-    const uint64_t pol_stream = l2_policy_evict_first();
-    const uint64_t pol_keep = l2_policy_evict_last();
-
-    const int kvh = ul / p.HB;
-    const int hb = ul - kvh * p.HB;
-    // Stage addresses.  Unshared: stage t of this warp is [K | V | Q] at wring + t * stage_bytes.
-    // SHARE: the K/V ring of this warp's kv head (its leader is hb warps lower in the same
-    // CTA: the host makes the warps per CTA a multiple of HB), and a Q ring of its own.
-    const bool follower = SHARE && hb > 0;
-    const uint32_t kv_step = SHARE ? 2 * G::kKVTileBytes : p.stage_bytes;
-    const uint32_t q_step = SHARE ? ((p.q_box_bytes + 1023u) & ~1023u) : p.stage_bytes;
-    const uint32_t kv_ring = SHARE ? ring + static_cast<uint32_t>(warp / p.HB) * STAGES * kv_step : wring;
-    const uint32_t q_ring = SHARE ? ring + static_cast<uint32_t>(p.warps / p.HB) * STAGES * kv_step +
-                                        static_cast<uint32_t>(warp) * STAGES * q_step
-                                  : wring + 2 * G::kKVTileBytes;
-    const uint32_t kv_bar0 = SHARE ? smem_u32(bars + (warp - hb) * STAGES) : bar0;
-    const uint32_t empty0 = smem_u32(empties + (warp - hb) * STAGES);
-    const int head0 = kvh * p.g + kMaxRows * hb;
-    const int rows = min(kMaxRows, p.g - kMaxRows * hb);
-
-    // LEAN: the lean per-tile form, which trims the instructions of a tile:
-    // - the row sums of the bf16 weights come from an mma against a B of ones;
-    // - 2^x is the SFU instruction;
-    // - full tiles skip the masking selects;
-    // - the rescale of the accumulators is skipped while no row's max grows;
-    // - the page slot is a running cursor.
-    // The plain form instead keeps:
-    // - per-thread row sums, with the quad's partial sums added at the unit's end;
-    // - exp2f;
-    // - masking and rescale on every tile.
-    // The host picks the form by measurement (B200, 268 MB of K/V, CUDA-graph replays):
-    // - lean: D = 32 and 64, and D = 128 in the balanced and fixed plans (7-15% faster
-    //   where per-tile latency binds);
-    // - plain: D = 256, which sits at the 255-register cap (the lean form measured 2-3%
-    //   slower there), and the CTA-local plan at D = 128 (the lean form measured 1% slower
-    //   on the llama8b shape).
-    constexpr bool kLean = LEAN;
-
-    // ---- producer state: next position to issue, its cursor, page-table window
-    int pi = ws;
-    int pb, pj, pn;
-    decode_pos(ws, s_cum, B, pb, pj, pn);
-    int pslot = (pj * kTile) % p.P;  // token slot of tile pj in its page (lean: stepped below)
-    int wbase = ws;
-    int32_t pg_cur = follower ? 0 : fetch_page(p, s_cum, ws + lane, we);
-    int32_t pg_nxt = follower ? 0 : fetch_page(p, s_cum, ws + 32 + lane, we);
-
-    bool stopped = false;  // the leader of a shared ring gave up on a release: no further issues
-    auto issue_next = [&](int stage) {
-        if (pi >= we || stopped) return;
-        if (follower) {
-            // this warp's Q rows only; an expect of 0 bytes keeps one phase per tile
-            const bool qload = (pj == 0) || (pi == ws);
-            if (lane == 0) {
-                const uint32_t bar = bar0 + 8 * stage;
-                const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
-                mbar_arrive_expect_tx(bar, qload ? p.q_box_bytes : 0u);
-                if (qload) {
-                    if constexpr (D == 32) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
-                    else tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
-                }
-            }
-            ++pi;
-            if (pi < we) advance_pos(s_cum, pb, pj, pn);
-            return;
-        }
-        if (SHARE && pi - ws >= STAGES) {
-            // the followers have read the tile this stage held, STAGES tiles back.  If they
-            // never release it (a follower gave up), issue nothing more: the stage may still
-            // be read, and the consumer loop below stops at the first tile not issued.
-            const int kk = pi - ws - STAGES;
-            if (!warp_wait(empty0 + 8 * stage, static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns, s_abort, p.flags)) {
-                stopped = true;
-                return;
-            }
-        }
-        int off = pi - wbase;
-        if (off >= 32) {
-            pg_cur = pg_nxt;
-            wbase += 32;
-            off -= 32;
-            pg_nxt = fetch_page(p, s_cum, wbase + 32 + lane, we);
-        }
-        const int32_t page = __shfl_sync(0xffffffffu, pg_cur, off);
-        const int slot = kLean ? pslot : (pj * kTile) % p.P;
-        const bool qload = (pj == 0) || (pi == ws);
-        if (lane == 0) {
-            if (page < 0 || page >= p.NP) atomicOr(p.flags, kFlagPageOOR);
-            const uint32_t bar = bar0 + 8 * stage;
-            const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;
-            const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
-            mbar_arrive_expect_tx(bar, 2 * G::kKVTileBytes + (qload ? p.q_box_bytes : 0u));
-            if constexpr (D == 32) {
-                tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, page, pol_stream);
-                tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, pol_stream);
-                if (qload) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
-            } else {
-                tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, page, 0, pol_stream);
-                tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, 0, pol_stream);
-                if (qload) tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
-            }
-        }
-        ++pi;
-        if (pi < we) {
-            advance_pos(s_cum, pb, pj, pn);
-            if constexpr (kLean) pslot = (pj == 0 || pslot + kTile == p.P) ? 0 : pslot + kTile;
-        }
-    };
-
-#pragma unroll
-    for (int s = 0; s < STAGES; ++s) issue_next(s);
-
-    // ---- consumer state
-    const int tq = lane & 3;   // thread in quad: token / d pair
-    const int gq = lane >> 2;  // quad index: row within the 8-row half
-    int cb, cj, cn;
-    decode_pos(ws, s_cum, B, cb, cj, cn);
-    int seg_start = ws;
-    int j_start = cj;
-
     uint32_t qf[G::kSteps][4];
     float acc[G::kNTiles][4];
     float accl[4];  // row sums: rows gq in [0], [1] and gq + 8 in [2], [3]
-    float m_lo = -INFINITY, m_hi = -INFINITY;
-    constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
+    float m_lo, m_hi;
 
-    for (int i = ws; i < we; ++i) {
-        const int k = i - ws;
-        const int stage = k % STAGES;
-        const uint32_t parity = static_cast<uint32_t>(k / STAGES) & 1u;
-        const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;  // K, V
-        const uint32_t qbase_t = q_ring + static_cast<uint32_t>(stage) * q_step;  // this warp's Q
-        const bool unit_start = (cj == 0) || (i == ws);
-
-        if (i >= pi || !warp_wait(kv_bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags) ||
-            (follower && !warp_wait(bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags))) {
-            // Gave up (this warp timed out, another warp of the CTA did, or this warp, as the
-            // leader of a shared ring, stopped issuing): let this warp's own copies in flight
-            // land, each wait bounded, then stop.
-            *s_abort = 1u;
-            for (int s = 0; s < STAGES; ++s) {
-                const int t = i + s;
-                if (t < pi) {
-                    const int kk = t - ws;
-                    warp_wait(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns / 8,
-                              nullptr, nullptr);
-                }
-            }
-            return;
-        }
-
-        if (unit_start) {
-            seg_start = i;
-            j_start = cj;
-            m_lo = m_hi = -INFINITY;
-            accl[0] = accl[1] = accl[2] = accl[3] = 0.f;
+    __device__ __forceinline__ void reset() {
+        m_lo = m_hi = -INFINITY;
+        accl[0] = accl[1] = accl[2] = accl[3] = 0.f;
 #pragma unroll
-            for (int nd = 0; nd < G::kNTiles; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
-            // Q A-fragments: matrix m of ldmatrix.x4 = (rows 8*(m&1).., k chunk m>>1)
-            const uint32_t qbase = qbase_t;
-            const int mi = lane >> 3;
-            int qrow = (mi & 1) * 8 + (lane & 7);
-            if (qrow >= p.rows_max) qrow = 0;  // stay inside the loaded box
+        for (int nd = 0; nd < G::kNTiles; ++nd) acc[nd][0] = acc[nd][1] = acc[nd][2] = acc[nd][3] = 0.f;
+    }
+
+    // Q A-fragments from a staged [rows_max x D] tile: matrix m of ldmatrix.x4 = (rows
+    // 8*(m&1).., k chunk m>>1); rows at and past `rows` are zero.
+    __device__ __forceinline__ void load_q(uint32_t qbase, int rows_max, int rows, int lane) {
+        const int gq = lane >> 2;
+        const int mi = lane >> 3;
+        int qrow = (mi & 1) * 8 + (lane & 7);
+        if (qrow >= rows_max) qrow = 0;  // stay inside the loaded box
 #pragma unroll
-            for (int ks = 0; ks < G::kSteps; ++ks) {
-                const uint32_t ch = 2 * ks + (mi >> 1);
-                ldsm_x4(qbase + G::chunk_off(qrow, ch, p.rows_max), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
-                if (gq >= rows) qf[ks][0] = qf[ks][2] = 0u;
-                if (gq + 8 >= rows) qf[ks][1] = qf[ks][3] = 0u;
-            }
+        for (int ks = 0; ks < G::kSteps; ++ks) {
+            const uint32_t ch = 2 * ks + (mi >> 1);
+            ldsm_x4(qbase + G::chunk_off(qrow, ch, rows_max), qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
+            if (gq >= rows) qf[ks][0] = qf[ks][2] = 0u;
+            if (gq + 8 >= rows) qf[ks][1] = qf[ks][3] = 0u;
         }
+    }
+
+    // One tile at `sbase` ([K | V], each 32 tokens x D): S = Q K^T, tokens at and past `valid`
+    // masked (and their V rows zeroed, so that 0 * (stale or NaN) never reaches the
+    // accumulator), online softmax in log2 units, O += P V.
+    __device__ __forceinline__ void step(uint32_t sbase, int valid, float scale_log2, int lane) {
+        const int tq = lane & 3;   // thread in quad: token / d pair
+        const int gq = lane >> 2;  // quad index: row within the 8-row half
+        constexpr uint32_t kOnesBf16x2 = 0x3F803F80u;
+        constexpr bool kLean = LEAN;
+        (void)gq;
 
         // ---- S = Q K^T over the 32 tokens of the tile: 4 n-tiles of 8 tokens
         float s[4][4];
@@ -650,17 +289,15 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
             }
         }
 
-        // ---- mask tokens past the sequence end; tail V rows are zeroed so that
-        // 0 * (stale or NaN) never reaches the accumulator
-        const int valid = min(kTile, s_len[cb] - kTile * cj);
+        // ---- mask tokens past the sequence end; zero their V rows
         auto mask_and_scale = [&]() {
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int t0 = 8 * nt + 2 * tq;
-                s[nt][0] = (t0 < valid) ? s[nt][0] * p.scale_log2 : -INFINITY;
-                s[nt][1] = (t0 + 1 < valid) ? s[nt][1] * p.scale_log2 : -INFINITY;
-                s[nt][2] = (t0 < valid) ? s[nt][2] * p.scale_log2 : -INFINITY;
-                s[nt][3] = (t0 + 1 < valid) ? s[nt][3] * p.scale_log2 : -INFINITY;
+                s[nt][0] = (t0 < valid) ? s[nt][0] * scale_log2 : -INFINITY;
+                s[nt][1] = (t0 + 1 < valid) ? s[nt][1] * scale_log2 : -INFINITY;
+                s[nt][2] = (t0 < valid) ? s[nt][2] * scale_log2 : -INFINITY;
+                s[nt][3] = (t0 + 1 < valid) ? s[nt][3] * scale_log2 : -INFINITY;
             }
         };
         if (valid < kTile) {
@@ -677,7 +314,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) s[nt][e] *= p.scale_log2;
+                for (int e = 0; e < 4; ++e) s[nt][e] *= scale_log2;
         }
         if constexpr (!kLean) mask_and_scale();
 
@@ -773,6 +410,416 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
                 }
             }
         }
+    }
+
+    // The rows' sums of weights (rows gq and gq + 8), complete in every lane of the quad.
+    __device__ __forceinline__ void row_sums(float& ll, float& lh) const {
+        ll = accl[0];
+        lh = accl[2];
+        if constexpr (!LEAN) {
+            ll += __shfl_xor_sync(0xffffffffu, ll, 1);
+            ll += __shfl_xor_sync(0xffffffffu, ll, 2);
+            lh += __shfl_xor_sync(0xffffffffu, lh, 1);
+            lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+        }
+    }
+
+    // out rows (normalised, bf16): row r of the head tile at o_row0 + r * out_sh.
+    __device__ __forceinline__ void write_out(__nv_bfloat16* o_row0, int64_t out_sh, int rows, int lane) const {
+        const int tq = lane & 3, gq = lane >> 2;
+        float ll, lh;
+        row_sums(ll, lh);
+        const float il = 1.f / ll, ih = 1.f / lh;
+        __nv_bfloat16* o_lo = o_row0 + gq * out_sh;
+        __nv_bfloat16* o_hi = o_lo + 8 * out_sh;
+#pragma unroll
+        for (int nd = 0; nd < G::kNTiles; ++nd) {
+            const int d = 8 * nd + 2 * tq;
+            if (gq < rows) *reinterpret_cast<uint32_t*>(o_lo + d) = pack_bf16x2(acc[nd][0] * il, acc[nd][1] * il);
+            if (gq + 8 < rows) *reinterpret_cast<uint32_t*>(o_hi + d) = pack_bf16x2(acc[nd][2] * ih, acc[nd][3] * ih);
+        }
+    }
+
+    // An unnormalised part: accumulator rows at op + r * ost (fp32) and (m, l) pairs at mp + 2 r.
+    __device__ __forceinline__ void write_part(float* op, int ost, float* mp, int rows, int lane) const {
+        const int tq = lane & 3, gq = lane >> 2;
+        float ll, lh;
+        row_sums(ll, lh);
+#pragma unroll
+        for (int nd = 0; nd < G::kNTiles; ++nd) {
+            const int d = 8 * nd + 2 * tq;
+            if (gq < rows) *reinterpret_cast<float2*>(op + gq * ost + d) = make_float2(acc[nd][0], acc[nd][1]);
+            if (gq + 8 < rows)
+                *reinterpret_cast<float2*>(op + (gq + 8) * ost + d) = make_float2(acc[nd][2], acc[nd][3]);
+        }
+        if (tq == 0) {
+            if (gq < rows) *reinterpret_cast<float2*>(mp + 2 * gq) = make_float2(m_lo, ll);
+            if (gq + 8 < rows) *reinterpret_cast<float2*>(mp + 2 * (gq + 8)) = make_float2(m_hi, lh);
+        }
+    }
+};
+
+// Row stride (floats) of a unit part's accumulator rows in shared memory: 8 floats of
+// padding put the 8 rows one warp store touches on different banks.
+template <int D>
+constexpr int kPartStride = D + 8;
+
+// Merge of the parts of one unit in unit_kernel: part k's (m, l) rows at ml_k = the start of
+// warp k's first ring stage, its accumulator rows [kMaxRows][kPartStride] (fp32) 128
+// bytes later.
+// Warp `part` of `nparts` merges rows part, part + nparts, ...:
+//   M = max_k m_k over parts with l_k > 0, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+template <int D>
+__device__ __noinline__ void unit_merge(const SplitParams& p, const uint8_t* ring0, uint32_t warp_bytes,
+                                                int b, int head0, int rows, int part, int nparts, int lane) {
+    constexpr int kVec = D / 32;  // consecutive columns per lane
+    for (int r = part; r < rows; r += nparts) {
+        float M = -INFINITY;
+        for (int k = 0; k < nparts; ++k) {
+            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
+            if (ml[2 * r + 1] > 0.f) M = fmaxf(M, ml[2 * r]);
+        }
+        float den = 0.f, acc[kVec];
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) acc[e] = 0.f;
+        for (int k = 0; k < nparts; ++k) {
+            const float* ml = reinterpret_cast<const float*>(ring0 + static_cast<size_t>(k) * warp_bytes);
+            if (!(ml[2 * r + 1] > 0.f)) continue;
+            const float wk = exp2f(ml[2 * r] - M);
+            den += wk * ml[2 * r + 1];
+            const float* a = ml + 2 * kMaxRows + r * kPartStride<D> + kVec * lane;
+            float v[kVec];  // this lane's kVec consecutive columns, in 16- (or 8-) byte loads
+            if constexpr (kVec % 4 == 0) {
+#pragma unroll
+                for (int e = 0; e < kVec; e += 4) *reinterpret_cast<float4*>(v + e) = *reinterpret_cast<const float4*>(a + e);
+            } else if constexpr (kVec == 2) {
+                *reinterpret_cast<float2*>(v) = *reinterpret_cast<const float2*>(a);
+            } else {
+                v[0] = a[0];
+            }
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) acc[e] += wk * v[e];
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        __nv_bfloat16* o = p.out + b * p.out_sb + (head0 + r) * p.out_sh + kVec * lane;
+        if constexpr (kVec == 1) {
+            o[0] = __float2bfloat16_rn(acc[0] * inv);
+        } else {
+#pragma unroll
+            for (int e = 0; e < kVec; e += 2)
+                *reinterpret_cast<uint32_t*>(o + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+        }
+    }
+}
+
+// SHARE (balanced mode with g > 16, so HB = ceil(g / 16) head blocks per kv head): the HB
+// warps of one kv head, which walk the same positions in one CTA, share one K/V ring, which
+// the first of them (the leader) fills.  Before refilling a stage the leader waits on that
+// stage's `empty` mbarrier, on which the other HB - 1 warps arrive once they have read the
+// tile.  Each warp loads its own Q rows into a Q ring of its own.  Shared-memory layout:
+// [K/V rings, one per kv head of the CTA][Q rings, one per warp], so a CTA of HB warps
+// holds one K/V ring instead of HB.
+template <int D, int STAGES, bool SHARE, bool LEAN>
+__global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
+    split_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
+                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
+    using G = Geometry<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int B = p.B;
+
+    // ---- shared-memory carve-up: mbarriers, lengths, prefix sums, stage ring
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empties = bars + p.warps * STAGES;  // SHARE: stage released by the followers
+    // raised by a warp that gave up on a wait: the CTA's other waits then give up too
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(empties + (SHARE ? p.warps * STAGES : 0));
+    int32_t* s_len = reinterpret_cast<int32_t*>(empties + (SHARE ? p.warps * STAGES : 0) + 1);
+    int32_t* s_cum = s_len + B;
+    const uint32_t meta_end = smem_u32(s_cum + B + 1);
+    const uint32_t ring = (meta_end + 1023u) & ~1023u;
+
+    if (tid == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+    }
+    // Launched with programmatic dependent launch: this CTA may start while the
+    // previous kernel in the stream is still running.  Nothing above touches
+    // global memory; from here on, that kernel has finished and its writes are
+    // visible.
+    pdl_wait_prior_grid();
+
+    // ---- per-sequence tile counts and their prefix sum (every CTA, from L2)
+    const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
+    uint32_t len_flags = 0;
+    for (int b = tid; b < B; b += blockDim.x) {
+        int L = __ldcg(p.seq_lens + b);
+        if (L < 0) {
+            L = 0;
+            len_flags |= kFlagLenNegative;
+        }
+        if (L > cap) {
+            L = static_cast<int>(cap);
+            len_flags |= kFlagLenClamped;
+        }
+        s_len[b] = L;
+        s_cum[b + 1] = (L + kTile - 1) / kTile;
+    }
+    if (tid == 0) {
+        s_cum[0] = 0;
+        *s_abort = 0u;
+    }
+    if (len_flags && blockIdx.x == 0) atomicOr(p.flags, len_flags);
+    __syncthreads();
+    if (SHARE && warp == 1) {
+        // every warp's ring barriers, before any warp waits on another warp's
+        for (int i = lane; i < p.warps * STAGES; i += 32) {
+            mbar_init(smem_u32(bars + i), 1);
+            mbar_init(smem_u32(empties + i), static_cast<uint32_t>(p.HB - 1));
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        const int per = (B + 31) / 32;
+        const int lo = 1 + lane * per;
+        const int hi = min(lo + per, B + 1);
+        int sum = 0;
+        for (int i = lo; i < hi; ++i) sum += s_cum[i];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int i = lo; i < hi; ++i) {
+            run += s_cum[i];
+            s_cum[i] = run;
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        for (int i = tid; i <= B; i += blockDim.x) p.cum_out[i] = s_cum[i];
+    }
+    // The combine kernel may start its launch now; it waits (griddepcontrol.wait)
+    // for this whole grid to finish before it reads anything.
+    pdl_launch_dependents();
+    // No CTA-wide barrier after this point: warps are independent workers.
+
+    const int units_per_seq = p.Hkv * p.HB;
+    const int w = blockIdx.x * p.warps + warp;
+    if (w >= p.num_workers) return;
+    if (p.zero_empty) {
+        // no combine kernel follows: the workers write the zero rows of empty sequences
+        for (int u = w; u < p.B * units_per_seq; u += p.num_workers) {
+            const int b = u / units_per_seq;
+            if (s_cum[b + 1] != s_cum[b]) continue;
+            const int ulz = u - b * units_per_seq, kvh = ulz / p.HB, hb = ulz - (ulz / p.HB) * p.HB;
+            write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
+        }
+    }
+
+    // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-
+    // sequence ul (kv head and head block).
+    int ws, we, ul;
+    int fixed_slot = -1;
+    if (p.mode == 0) {
+        // Workers form groups of units_per_seq warps, one per (kv head, head block);
+        // group grp owns an equal share of the positions of all sequences.  The warps
+        // of a group walk the same pages together, so the kv heads of a page are read
+        // at about the same time.
+        const int grp = w / units_per_seq;
+        ul = w - grp * units_per_seq;
+        ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
+        we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
+    } else {
+        // fixed splits: warp w takes split w % k of unit w / k
+        const int u = w / p.ksplit;
+        const int s = w - u * p.ksplit;
+        const int b = u / units_per_seq;
+        ul = u - b * units_per_seq;
+        const int n = s_cum[b + 1] - s_cum[b];
+        if (n == 0) {
+            if (s == 0) {
+                const int kvh = ul / p.HB, hb = ul - (ul / p.HB) * p.HB;
+                write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
+            }
+            return;
+        }
+        const int S = min(p.ksplit, n);
+        const int c = (n + S - 1) / S;
+        const int t0 = s * c;
+        if (t0 >= n) return;
+        const int t1 = min(t0 + c, n);
+        ws = s_cum[b] + t0;
+        we = s_cum[b] + t1;
+        fixed_slot = u * p.ksplit + s;
+    }
+    if (ws >= we) return;
+
+    const uint32_t bar0 = smem_u32(bars + warp * STAGES);
+    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;  // unshared layout
+    if constexpr (!SHARE) {
+        if (lane == 0) {
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+    }
+
+    const uint64_t pol_stream = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
+
+    const int kvh = ul / p.HB;
+    const int hb = ul - kvh * p.HB;
+    // Stage addresses.  Unshared: stage t of this warp is [K | V | Q] at wring + t * stage_bytes.
+    // SHARE: the K/V ring of this warp's kv head (its leader is hb warps lower in the same
+    // CTA: the host makes the warps per CTA a multiple of HB), and a Q ring of its own.
+    const bool follower = SHARE && hb > 0;
+    const uint32_t kv_step = SHARE ? 2 * G::kKVTileBytes : p.stage_bytes;
+    const uint32_t q_step = SHARE ? ((p.q_box_bytes + 1023u) & ~1023u) : p.stage_bytes;
+    const uint32_t kv_ring = SHARE ? ring + static_cast<uint32_t>(warp / p.HB) * STAGES * kv_step : wring;
+    const uint32_t q_ring = SHARE ? ring + static_cast<uint32_t>(p.warps / p.HB) * STAGES * kv_step +
+                                        static_cast<uint32_t>(warp) * STAGES * q_step
+                                  : wring + 2 * G::kKVTileBytes;
+    const uint32_t kv_bar0 = SHARE ? smem_u32(bars + (warp - hb) * STAGES) : bar0;
+    const uint32_t empty0 = smem_u32(empties + (warp - hb) * STAGES);
+    const int head0 = kvh * p.g + kMaxRows * hb;
+    const int rows = min(kMaxRows, p.g - kMaxRows * hb);
+
+    // LEAN: the lean per-tile form, which trims the instructions of a tile:
+    // - the row sums of the bf16 weights come from an mma against a B of ones;
+    // - 2^x is the SFU instruction;
+    // - full tiles skip the masking selects;
+    // - the rescale of the accumulators is skipped while no row's max grows;
+    // - the page slot is a running cursor.
+    // The plain form instead keeps:
+    // - per-thread row sums, with the quad's partial sums added at the unit's end;
+    // - exp2f;
+    // - masking and rescale on every tile.
+    // The host picks the form by measurement (B200, 268 MB of K/V, CUDA-graph replays):
+    // - lean: D = 32, 64 and 128 (7-15% faster where per-tile latency binds);
+    // - plain: D = 256, which sits at the 255-register cap (the lean form measured 2-3%
+    //   slower there).  unit_kernel takes the plain form at D = 128 too (the lean form
+    //   measured 1% slower on the llama8b shape with one CTA per unit).
+    constexpr bool kLean = LEAN;
+
+    // ---- producer state: next position to issue, its cursor, page-table window
+    int pi = ws;
+    int pb, pj, pn;
+    decode_pos(ws, s_cum, B, pb, pj, pn);
+    int pslot = (pj * kTile) % p.P;  // token slot of tile pj in its page (lean: stepped below)
+    int wbase = ws;
+    int32_t pg_cur = follower ? 0 : fetch_page(p, s_cum, ws + lane, we);
+    int32_t pg_nxt = follower ? 0 : fetch_page(p, s_cum, ws + 32 + lane, we);
+
+    bool stopped = false;  // the leader of a shared ring gave up on a release: no further issues
+    auto issue_next = [&](int stage) {
+        if (pi >= we || stopped) return;
+        if (follower) {
+            // this warp's Q rows only; an expect of 0 bytes keeps one phase per tile
+            const bool qload = (pj == 0) || (pi == ws);
+            if (lane == 0) {
+                const uint32_t bar = bar0 + 8 * stage;
+                const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
+                mbar_arrive_expect_tx(bar, qload ? p.q_box_bytes : 0u);
+                if (qload) {
+                    if constexpr (D == 32) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
+                    else tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
+                }
+            }
+            ++pi;
+            if (pi < we) advance_pos(s_cum, pb, pj, pn);
+            return;
+        }
+        if (SHARE && pi - ws >= STAGES) {
+            // the followers have read the tile this stage held, STAGES tiles back.  If they
+            // never release it (a follower gave up), issue nothing more: the stage may still
+            // be read, and the consumer loop below stops at the first tile not issued.
+            const int kk = pi - ws - STAGES;
+            if (!warp_wait(empty0 + 8 * stage, static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns, s_abort, p.flags)) {
+                stopped = true;
+                return;
+            }
+        }
+        int off = pi - wbase;
+        if (off >= 32) {
+            pg_cur = pg_nxt;
+            wbase += 32;
+            off -= 32;
+            pg_nxt = fetch_page(p, s_cum, wbase + 32 + lane, we);
+        }
+        const int32_t page = __shfl_sync(0xffffffffu, pg_cur, off);
+        const int slot = kLean ? pslot : (pj * kTile) % p.P;
+        const bool qload = (pj == 0) || (pi == ws);
+        if (lane == 0) {
+            if (page < 0 || page >= p.NP) atomicOr(p.flags, kFlagPageOOR);
+            const uint32_t bar = bar0 + 8 * stage;
+            const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;
+            const uint32_t qdst = q_ring + static_cast<uint32_t>(stage) * q_step;
+            mbar_arrive_expect_tx(bar, 2 * G::kKVTileBytes + (qload ? p.q_box_bytes : 0u));
+            if constexpr (D == 32) {
+                tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, page, pol_stream);
+                tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, pol_stream);
+                if (qload) tma_load_3d(qdst, &qmap, bar, 0, head0, pb, pol_keep);
+            } else {
+                tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, page, 0, pol_stream);
+                tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, page, 0, pol_stream);
+                if (qload) tma_load_4d(qdst, &qmap, bar, 0, head0, pb, 0, pol_keep);
+            }
+        }
+        ++pi;
+        if (pi < we) {
+            advance_pos(s_cum, pb, pj, pn);
+            if constexpr (kLean) pslot = (pj == 0 || pslot + kTile == p.P) ? 0 : pslot + kTile;
+        }
+    };
+
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) issue_next(s);
+
+    // ---- consumer state
+    int cb, cj, cn;
+    decode_pos(ws, s_cum, B, cb, cj, cn);
+    int seg_start = ws;
+    int j_start = cj;
+    TileAcc<D, LEAN> st;
+
+    for (int i = ws; i < we; ++i) {
+        const int k = i - ws;
+        const int stage = k % STAGES;
+        const uint32_t parity = static_cast<uint32_t>(k / STAGES) & 1u;
+        const uint32_t sbase = kv_ring + static_cast<uint32_t>(stage) * kv_step;  // K, V
+        const uint32_t qbase_t = q_ring + static_cast<uint32_t>(stage) * q_step;  // this warp's Q
+        const bool unit_start = (cj == 0) || (i == ws);
+
+        if (i >= pi || !warp_wait(kv_bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags) ||
+            (follower && !warp_wait(bar0 + 8 * stage, parity, p.wait_ns, s_abort, p.flags))) {
+            // Gave up (this warp timed out, another warp of the CTA did, or this warp, as the
+            // leader of a shared ring, stopped issuing): let this warp's own copies in flight
+            // land, each wait bounded, then stop.
+            *s_abort = 1u;
+            for (int s = 0; s < STAGES; ++s) {
+                const int t = i + s;
+                if (t < pi) {
+                    const int kk = t - ws;
+                    warp_wait(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns / 8,
+                              nullptr, nullptr);
+                }
+            }
+            return;
+        }
+
+        if (unit_start) {
+            seg_start = i;
+            j_start = cj;
+            st.reset();
+            st.load_q(qbase_t, p.rows_max, rows, lane);
+        }
+        st.step(sbase, min(kTile, s_len[cb] - kTile * cj), p.scale_log2, lane);
 
         // ---- the stage is consumed: refill it with tile i + STAGES.  Each lane
         // orders its own shared-memory accesses (the tail zeroing included)
@@ -785,62 +832,193 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         // ---- end of this unit's run in this worker: write output or a partial
         const bool unit_end = (cj == cn - 1) || (i == we - 1);
         if (unit_end) {
-            float ll = accl[0], lh = accl[2];
-            if constexpr (!kLean) {
-                ll += __shfl_xor_sync(0xffffffffu, ll, 1);
-                ll += __shfl_xor_sync(0xffffffffu, ll, 2);
-                lh += __shfl_xor_sync(0xffffffffu, lh, 1);
-                lh += __shfl_xor_sync(0xffffffffu, lh, 2);
-            }
             const bool direct = (j_start == 0) && (cj == cn - 1);
             if (direct) {
-                const float il = 1.f / ll, ih = 1.f / lh;
-                __nv_bfloat16* o_lo = p.out + cb * p.out_sb + (head0 + gq) * p.out_sh;
-                __nv_bfloat16* o_hi = o_lo + 8 * p.out_sh;
-#pragma unroll
-                for (int nd = 0; nd < G::kNTiles; ++nd) {
-                    const int d = 8 * nd + 2 * tq;
-                    if (gq < rows)
-                        *reinterpret_cast<uint32_t*>(o_lo + d) = pack_bf16x2(acc[nd][0] * il, acc[nd][1] * il);
-                    if (gq + 8 < rows)
-                        *reinterpret_cast<uint32_t*>(o_hi + d) = pack_bf16x2(acc[nd][2] * ih, acc[nd][3] * ih);
-                }
+                st.write_out(p.out + cb * p.out_sb + head0 * p.out_sh, p.out_sh, rows, lane);
             } else {
                 const int64_t slot =
                     (p.mode == 0) ? (2 * static_cast<int64_t>(w) + (seg_start == ws ? 0 : 1)) : fixed_slot;
-                // CTA-local mode: the part goes to this warp's (now idle) ring, as (m, l) rows
-                // then accumulator rows
-                float* const own = reinterpret_cast<float*>(smem + (wring - smem_u32(smem)));
-                float* op = (p.mode == 2) ? own + 2 * kMaxRows : p.o_part + slot * p.rows_max * D;
-                float* mp = (p.mode == 2) ? own : p.ml_part + slot * p.rows_max * 2;
-                const int ost = (p.mode == 2) ? kPartStride<D> : D;
-#pragma unroll
-                for (int nd = 0; nd < G::kNTiles; ++nd) {
-                    const int d = 8 * nd + 2 * tq;
-                    if (gq < rows)
-                        *reinterpret_cast<float2*>(op + gq * ost + d) = make_float2(acc[nd][0], acc[nd][1]);
-                    if (gq + 8 < rows)
-                        *reinterpret_cast<float2*>(op + (gq + 8) * ost + d) = make_float2(acc[nd][2], acc[nd][3]);
-                }
-                if (tq == 0) {
-                    if (gq < rows) *reinterpret_cast<float2*>(mp + 2 * gq) = make_float2(m_lo, ll);
-                    if (gq + 8 < rows) *reinterpret_cast<float2*>(mp + 2 * (gq + 8)) = make_float2(m_hi, lh);
-                }
+                st.write_part(p.o_part + slot * p.rows_max * D, D, p.ml_part + slot * p.rows_max * 2, rows, lane);
             }
         }
         if (i + 1 < we) advance_pos(s_cum, cb, cj, cn);
     }
-    // CTA-local mode: part `warp` of the CTA's unit (recomputed here rather than kept
-    // live through the loop)
-    const int nparts = (!SHARE && p.mode == 2) ? cta_local_parts(cta_local_tiles(p, s_cum, blockIdx.x), p.ksplit) : 1;
-    if (nparts >= 2) {
-        // every lane's part rows are written: arrive, wait (bounded) for the other parts,
-        // and merge this warp's share of the rows
-        mbar_arrive(smem_u32(merge_bar));
-        if (!warp_wait(smem_u32(merge_bar), 0u, p.wait_ns, s_abort, p.flags)) return;
-        cta_local_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, cb,
-                           head0, rows, warp, nparts, lane);
+}
+
+// One CTA per unit (sequence b = unit / (Hkv * HB), kv head, head block), for launches in
+// which every unit has an SM of its own; the call is this one kernel.
+//  * The mbarriers are set up before the wait on the previous grid.  After it, lane 0 of
+//    each warp loads the sequence's length and claims its first STAGES + 1 tiles, loading
+//    their page-table entries as the claims return.  (Deterministic first tiles, with all
+//    those loads issued at once, measured 8% slower on the llama8b shape: the kv heads of
+//    a sequence then read its pages in lockstep and whole sequences fell behind.)
+//  * The warps claim the unit's 32-token tiles one at a time from a counter in shared
+//    memory, each one tile ahead of its issue (the page-table entry of the claimed tile is
+//    loaded while the tile before it streams), so a warp that streams faster takes more
+//    tiles and the warps of the CTA end close together.
+//  * Each warp keeps a running (max, sum, accumulator) over its tiles, writes it into its own
+//    ring once its copies have landed, and the warps merge the parts through shared memory.
+// Shared-memory layout: [full mbarriers, warps x STAGES][merge mbarrier][abort word, tile
+// counter][claimed tile of each stage, warps x STAGES], then 1024-aligned rings of
+// [K | V | Q] stages, one ring per warp.
+template <int D, int STAGES, bool LEAN>
+__global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
+    unit_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
+                const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
+    using G = Geometry<D>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int W = p.warps;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* merge_bar = bars + W * STAGES;
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(merge_bar + 1);
+    uint32_t* s_next = reinterpret_cast<uint32_t*>(merge_bar + 1) + 1;
+    int32_t* s_tile = reinterpret_cast<int32_t*>(merge_bar + 2);
+    const uint32_t ring = (smem_u32(s_tile + W * STAGES) + 1023u) & ~1023u;
+    const uint32_t wring = ring + static_cast<uint32_t>(warp) * STAGES * p.stage_bytes;
+    const uint32_t bar0 = smem_u32(bars + warp * STAGES);
+    int32_t* my_tile = s_tile + warp * STAGES;
+
+    // ---- set-up that reads no global memory, overlapping the end of the previous kernel
+    if (tid == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+        *s_abort = 0u;
+        *s_next = 0u;
+        mbar_init(smem_u32(merge_bar), 32u * static_cast<uint32_t>(W));  // every lane of every warp arrives
     }
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+    }
+    if (lane == 0) fence_mbar_init();
+    __syncthreads();
+    int nxt_t = 0;  // lane 0: the claimed tile that is issued next
+    pdl_wait_prior_grid();
+    pdl_launch_dependents();
+
+    const int u = blockIdx.x;
+    const int ups = p.Hkv * p.HB;
+    const int b = u / ups;
+    const int ul = u - b * ups;
+    const int kvh = ul / p.HB;
+    const int hb = ul - kvh * p.HB;
+    const int head0 = kvh * p.g + kMaxRows * hb;
+    const int rows = min(kMaxRows, p.g - kMaxRows * hb);
+    // Contiguous KV (no page table): sequence b is "page" b of P = Lmax tokens, any length.
+    const bool contig = p.page_table == nullptr;
+    const int64_t cap = static_cast<int64_t>(p.MP) * p.P;  // tokens the page table can address
+    const int32_t* pt_row = contig ? nullptr : p.page_table + static_cast<int64_t>(b) * p.pt_s0;
+    const int tiles_per_page = contig ? 1 : p.P / kTile;
+    const uint64_t pol_stream = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
+
+    // ---- producer state (lane 0): the next claimed tile and its page (a load in flight)
+    auto page_of = [&](int t) -> int32_t {  // lane 0
+        if (contig) return b;
+        return (static_cast<int64_t>(t) * kTile < cap)
+                   ? __ldcg(pt_row + static_cast<int64_t>(t / tiles_per_page) * p.pt_s1) : 0;
+    };
+    int32_t nxt_pg = 0;
+    auto claim = [&]() {  // lane 0
+        nxt_t = static_cast<int>(atomicAdd(s_next, 1u));
+        nxt_pg = page_of(nxt_t);
+    };
+    // lane 0: the sequence's length, then this warp's first STAGES + 1 claims with their pages
+    int L = 0;
+    int t0[STAGES];
+    int32_t pg0[STAGES];
+    if (lane == 0) {
+        L = __ldcg(p.seq_lens + b);
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+            claim();
+            t0[s] = nxt_t;
+            pg0[s] = nxt_pg;
+        }
+        claim();
+        uint32_t len_flags = 0;
+        if (L < 0) {
+            L = 0;
+            len_flags |= kFlagLenNegative;
+        }
+        if (L > cap) {
+            L = static_cast<int>(cap);
+            len_flags |= kFlagLenClamped;
+        }
+        if (len_flags && warp == 0) atomicOr(p.flags, len_flags);
+    }
+    L = __shfl_sync(0xffffffffu, L, 0);
+    const int n = (L + kTile - 1) / kTile;
+
+    // Issue tile t (page pg) into stage `stage`, with the Q rows on this warp's first tile.
+    auto issue = [&](int stage, int t, int32_t pg, bool qload) {  // lane 0
+        if (pg < 0 || pg >= p.NP) atomicOr(p.flags, kFlagPageOOR);
+        my_tile[stage] = t;
+        const uint32_t bar = bar0 + 8 * stage;
+        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+        const int slot = contig ? t * kTile : (t % tiles_per_page) * kTile;
+        mbar_arrive_expect_tx(bar, 2 * G::kKVTileBytes + (qload ? p.q_box_bytes : 0u));
+        if constexpr (D == 32) {
+            tma_load_4d(sbase, &kmap, bar, 0, kvh, slot, pg, pol_stream);
+            tma_load_4d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, pg, pol_stream);
+            if (qload) tma_load_3d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, b, pol_keep);
+        } else {
+            tma_load_5d(sbase, &kmap, bar, 0, kvh, slot, pg, 0, pol_stream);
+            tma_load_5d(sbase + G::kKVTileBytes, &vmap, bar, 0, kvh, slot, pg, 0, pol_stream);
+            if (qload) tma_load_4d(sbase + 2 * G::kKVTileBytes, &qmap, bar, 0, head0, b, 0, pol_keep);
+        }
+    };
+    int issued = 0;  // stages issued so far (warp-uniform)
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+            if (t0[s] < n) {
+                issue(s, t0[s], pg0[s], s == 0);
+                ++issued;
+            }
+        }
+    }
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+
+    TileAcc<D, LEAN> st;
+    st.reset();
+    for (int k = 0; k < issued; ++k) {
+        const int stage = k % STAGES;
+        const uint32_t sbase = wring + static_cast<uint32_t>(stage) * p.stage_bytes;
+        if (!warp_wait(bar0 + 8 * stage, static_cast<uint32_t>(k / STAGES) & 1u, p.wait_ns, s_abort, p.flags)) {
+            // gave up: let this warp's other copies in flight land (bounded), then stop
+            *s_abort = 1u;
+            for (int kk = k + 1; kk < issued; ++kk)
+                warp_wait(bar0 + 8 * (kk % STAGES), static_cast<uint32_t>(kk / STAGES) & 1u, p.wait_ns / 8, nullptr,
+                          nullptr);
+            return;
+        }
+        const int t = my_tile[stage];
+        if (k == 0) st.load_q(sbase + 2 * G::kKVTileBytes, p.rows_max, rows, lane);
+        st.step(sbase, min(kTile, L - kTile * t), p.scale_log2, lane);
+        // the stage is consumed: refill it with the claimed tile, if any, and claim the next
+        fence_proxy_async_smem();
+        __syncwarp();
+        int more = 0;
+        if (lane == 0 && nxt_t < n) {
+            issue(stage, nxt_t, nxt_pg, false);
+            claim();
+            more = 1;
+        }
+        issued += __shfl_sync(0xffffffffu, more, 0);
+    }
+
+    // ---- this warp's part (empty when it got no tile) into its own ring, then the merge
+    float* const own = reinterpret_cast<float*>(smem + (wring - smem_u32(smem)));
+    st.write_part(own + 2 * kMaxRows, kPartStride<D>, own, rows, lane);
+    mbar_arrive(smem_u32(merge_bar));
+    if (!warp_wait(smem_u32(merge_bar), 0u, p.wait_ns, s_abort, p.flags)) return;
+    unit_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, b, head0,
+                       rows, warp, W, lane);
 }
 
 constexpr int kCombineBatch = 4;  // partial slots whose loads a warp issues together

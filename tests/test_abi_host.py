@@ -230,11 +230,11 @@ _SHARE_TRAITS = {32: None, 64: (4, 8), 128: (2, 8), 256: (2, 4)}
 
 def _smem(B, D, rows, warps, stages, hb, shared):
     """Dynamic shared memory of the split kernel: mbarriers (full, plus empty when the K/V
-    ring is shared), the merge barrier, the CTA's abort word (8 bytes), lengths and prefix
-    sums, 1 KB of alignment slack, then the rings: per warp [K | V | Q] stages, or, shared,
-    one K/V ring per kv head and one Q ring per warp (K and V tiles are 32 tokens x D bf16,
-    Q tiles 1 KB aligned)."""
-    meta = 8 * warps * stages * (2 if shared else 1) + 8 + 8 + 4 * (2 * B + 1)
+    ring is shared), the CTA's abort word (8 bytes), lengths and prefix sums, 1 KB of
+    alignment slack, then the rings: per warp [K | V | Q] stages, or, shared, one K/V ring
+    per kv head and one Q ring per warp (K and V tiles are 32 tokens x D bf16, Q tiles 1 KB
+    aligned)."""
+    meta = 8 * warps * stages * (2 if shared else 1) + 8 + 4 * (2 * B + 1)
     kv = 2 * 32 * D * 2
     q = -(-rows * D * 2 // 1024) * 1024
     rings = (warps // hb * stages * kv + warps * stages * q) if shared else warps * stages * (kv + q)
