@@ -51,6 +51,8 @@ GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes
 GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
 PREFILL_METRIC = "paged multi-query (prefill chunk) attention achieved TFLOP/s and HBM GB/s"
 PREFILL_WORKLOADS = ["prefill_llama8b_chunk"]
+SWEEP_WORKLOADS = ["sweep"]
+SWEEP_METRIC = "paged decode attention us/call with a cold L2, head-dim / GQA sweep (B=4, L ~ U{1..1024})"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "split_kernel_traffic.json")
 PREFILL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "prefill_tc2_kernel_traffic.json")
 GEMV_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemv_kernel_traffic.json")
@@ -62,7 +64,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=sorted(workloads.NAMED) + GEMV_WORKLOADS + PREFILL_WORKLOADS,
+    p.add_argument("--workload", choices=sorted(workloads.NAMED) + GEMV_WORKLOADS + PREFILL_WORKLOADS + SWEEP_WORKLOADS,
                    default="llama8b",
                    help="a decode-attention workload, or gemv_<layer>_m<M> for the decode projection")
     p.add_argument("--num-splits", type=int, default=0, help="0 = auto (the default launch configuration)")
@@ -1005,10 +1007,84 @@ def run_prefill(a):
     return 0
 
 
+def run_sweep(a):
+    """The head-dim / GQA sweep: every (D, heads, num_splits) case of the configuration, one
+    call at a time with the L2 flushed before each (a 512 MB write), timed with CUDA events
+    around the call.  The cases' footprints (2-17 MB) would otherwise stay in L2."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        print("no CUDA device", file=sys.stderr)
+        return 2
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_group(world, "nccl")
+    import decode_attention_paged_split_b200 as apd
+
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    samples = max(5, min(a.steps, 200))
+    clocks = ClockSampler(local, enabled=not a.no_clocks and rank == 0)
+    cases, total_us, total_bytes = [], 0.0, 0
+    for d, hq, hkv, s in workloads.sweep_cases():
+        w = workloads.sweep_case(d, hq, hkv, s, seed=2024 + 1000003 * rank)
+        q, k_, v_ = w.q.to(device), w.k_cache.contiguous().to(device), w.v_cache.contiguous().to(device)
+        pt, sl = w.page_table.to(device), w.seq_lens.to(device)
+        out = torch.empty_like(q)
+        ws = apd.alloc_workspace(w.batch, hq, hkv, d, s, device=device)
+        call = apd.DecodeCall(q, k_, v_, pt, sl, out, w.scale, s, ws)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(samples)]
+        with torch.cuda.stream(stream):
+            for i in range(a.warmup):
+                call(stream)
+            for i, (e0, e1) in enumerate(ev):
+                flush.fill_(i & 0xFF)
+                e0.record(stream)
+                call(stream)
+                e1.record(stream)
+            warm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(samples)]
+            for e0, e1 in warm:
+                e0.record(stream)
+                call(stream)
+                e1.record(stream)
+        stream.synchronize()
+        cold = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
+        hot = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in warm)
+        cold = max_over_ranks(cold, dist, device)
+        b = w.algorithmic_bytes()
+        pl = apd.query_plan(w.batch, hq, hkv, d, s)
+        cases.append({"case": w.name, "head_dim": d, "num_q_heads": hq, "num_kv_heads": hkv, "num_splits": s,
+                      "kv_tokens": w.kv_tokens(), "algorithmic_bytes": b, "cold_l2_us": cold, "warm_l2_us": hot,
+                      "cold_gbs": b / cold / 1e3, "launches": 1 + (1 if pl.combine_ctas > 0 else 0)})
+        total_us += cold
+        total_bytes += b
+    clock_info = clocks.stop()
+    if rank == 0:
+        peak, peak_src = peaks()
+        line = {"metric": SWEEP_METRIC, "value": total_us, "unit": "us (sum over the 16 cases)", "n_gpus": world,
+                "steps": samples, "warmup": a.warmup, "ms_per_step": total_us / 1e3, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "sweep_b4_d32-256_h8x8-32x8_s1-4",
+                           "l2": "512 MB written before each timed call (cold L2); warm_l2_us: the same call "
+                                 "repeated without the flush",
+                           "timing": f"CUDA events around each call, median of {samples}"},
+                "roofline": {"bound": "hbm", "achieved": total_bytes / total_us / 1e3, "peak": peak, "unit": UNIT,
+                             "frac": total_bytes / total_us / 1e3 / peak, "traffic": None,
+                             "peak_source": peak_src,
+                             "note": "latency-bound: 2-17 MB per call is a few microseconds at the HBM rate"},
+                "cases": cases, "clocks": clock_info,
+                "gpu_launches": sum(c["launches"] for c in cases) * (samples * 2 + a.warmup)}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     a = parse_args(argv)
+    if a.workload == "sweep" and a.impl != "reference":
+        return run_sweep(a)
     if a.impl == "reference":
-        if a.workload.startswith(("gemv_", "prefill_")):
+        if a.workload.startswith(("gemv_", "prefill_")) or a.workload == "sweep":
             print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the decode-attention "
                                                                   "workloads; use the gemv workloads' cpu_baseline"}))
             return 0

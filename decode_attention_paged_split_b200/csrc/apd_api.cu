@@ -201,11 +201,28 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
 // share of the groups, plus the one it starts in) and num_splits in the fixed mode.
 // Measured (llama8b-shaped, L = 4096, graph-timed): 8 warps at 4 partials per unit cost
 // llama8b 45.9 -> 48.2 us and ragged 332 -> 345-353 us, so 4 stays the floor.
+int64_t partials_per_unit(const Shape& s, const Plan& pl) {
+    return pl.mode == 0 ? pl.groups / std::max(1, s.B) + 1 : pl.ksplit;
+}
 int combine_warps(const Shape& s, const Plan& pl) {
-    const int64_t per_unit = pl.mode == 0 ? pl.groups / std::max(1, s.B) + 1 : pl.ksplit;
+    const int64_t per_unit = partials_per_unit(s, pl);
     int w = 4;
     while (w < 16 && static_cast<int64_t>(w) * apd::kCombineBatch < per_unit) w *= 2;
     return w;
+}
+
+// With at most one batch of partials per unit, a grid of a few CTAs per SM that walk the
+// units (each warp merging whole rows) beats one CTA per (unit, row): the large-batch plans
+// have about one partial per unit, and most of their units are covered by one warp, so most
+// row CTAs would only return.  Graph-timed on B200: ragged (B = 128, 64/8 heads) 414-419 ->
+// 409-410 us per call; the llama8b-shaped batch without host lengths (5 partials per unit)
+// went 46.0 -> 46.6 us, so it keeps one CTA per (unit, row).
+bool combine_per_unit(const Shape& s, const Plan& pl) {
+    return partials_per_unit(s, pl) <= apd::kCombineBatch;
+}
+constexpr int kCombineUnitCtasPerSm = 4;
+int64_t combine_unit_ctas(const Shape& s, int sm_count) {
+    return std::min<int64_t>(s.units, static_cast<int64_t>(sm_count) * kCombineUnitCtasPerSm);
 }
 
 // tiles_bound: an upper bound on the number of tiles (host-known), or -1.
@@ -256,7 +273,9 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         pl->slots = 2 * workers;
         // one group covers every position: no unit is split, every warp writes its
         // output directly, and the call is a single launch (the unsplit path)
-        pl->combine_ctas = groups > 1 ? static_cast<int>(s.units * s.rows_max) : 0;
+        pl->combine_ctas = groups > 1 ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
+                                                                                 : s.units * s.rows_max)
+                                      : 0;
         pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
         if (host_lens && pl->combine_ctas > 0 && cta_local_wins(s, *pl, sm_count, host_lens, len_cap))
             cta_local_plan(s, pl);
@@ -268,7 +287,9 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         if (workers > INT32_MAX / 2) return APD_ERR_TOO_LARGE;
         pl->workers = static_cast<int>(workers);
         pl->slots = num_splits >= 2 ? workers : 0;
-        pl->combine_ctas = num_splits >= 2 ? static_cast<int>(s.units * s.rows_max) : 0;
+        pl->combine_ctas = num_splits >= 2 ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
+                                                                                        : s.units * s.rows_max)
+                                           : 0;
     }
     if (pl->mode != 2) pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
     pl->ws_needed = ws_bytes_for(s, pl->slots);
@@ -602,17 +623,23 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
         cp.ksplit = pl.ksplit;
         cp.num_workers = pl.workers;
         cp.groups = pl.groups;
-        const int cw = combine_warps(s, pl);
+        const bool per_unit = combine_per_unit(s, pl);
+        const int cw = per_unit ? (s.rows_max >= 8 ? 8 : 4) : combine_warps(s, pl);
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
+        cfg.gridDim = per_unit ? dim3(static_cast<unsigned>(pl.combine_ctas))
+                               : dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
         cfg.blockDim = dim3(32 * cw);
-        cfg.dynamicSmemBytes = 0;
+        cfg.dynamicSmemBytes = per_unit ? 4u * (s.B + 1) : 0u;
         cfg.stream = stream;
         cfg.attrs = pdl_attr;
         cfg.numAttrs = (use_pdl && !(opts && opts->split_done_event)) ? 1 : 0;
-        e = cw == 16 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 16>, cp)
-            : cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 8>, cp)
-                      : cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 4>, cp);
+        if (per_unit)
+            e = cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 8>, cp)
+                        : cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 4>, cp);
+        else
+            e = cw == 16 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 16>, cp)
+                : cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 8>, cp)
+                          : cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 4>, cp);
         if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
     }
     return APD_OK;

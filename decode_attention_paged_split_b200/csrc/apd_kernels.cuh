@@ -1217,4 +1217,178 @@ __global__ void __launch_bounds__(32 * W) combine_kernel(const __grid_constant__
     }
 }
 
+// The unit's partial slots in the combine: which slots hold its parts, as the split kernel
+// wrote them (balanced groups, or fixed splits), and the unit's sequence facts.
+struct UnitSlots {
+    int n = 0;         // tiles of the unit's sequence (0: empty sequence)
+    int nk = 0;        // partial slots, numbered k = 0 .. nk-1 (<= 1: nothing to merge)
+    int g_first = 0;   // balanced: the first group meeting the sequence
+    int64_t total = 0, Sb = 0;
+    int64_t first_fixed = 0;
+};
+
+// Balanced mode: the groups whose shares of the sequence-tile positions meet sequence b
+// (cum_b = tiles before b, cum_B = all tiles); fixed mode: the unit's non-empty splits.
+__device__ __forceinline__ UnitSlots unit_slots(const CombineParams& p, int u, int n, int cum_b, int cum_B) {
+    UnitSlots s;
+    s.n = n;
+    if (n == 0) return s;
+    if (p.mode == 0) {
+        s.total = cum_B;
+        s.Sb = cum_b;
+        s.g_first = worker_of(s.Sb, s.total, p.groups);
+        const int g_last = worker_of(s.Sb + n - 1, s.total, p.groups);
+        s.nk = g_last - s.g_first + 1;  // 1: one warp covered it and wrote the output
+    } else {
+        const int S = min(p.ksplit, n);
+        const int c = (n + S - 1) / S;
+        s.nk = (n + c - 1) / c;
+        s.first_fixed = static_cast<int64_t>(u) * p.ksplit;
+    }
+    return s;
+}
+
+// Slot of partial k of unit-in-sequence ul, or -1 for a group whose share is empty.
+__device__ __forceinline__ int64_t slot_of(const CombineParams& p, const UnitSlots& s, int ul, int k) {
+    if (p.mode != 0) return s.first_fixed + k;
+    const int g = s.g_first + k;
+    const int64_t a = run_start(g, s.total, p.groups);
+    if (a == run_start(g + 1, s.total, p.groups)) return -1;
+    const int64_t w = static_cast<int64_t>(g) * p.Hkv * p.HB + ul;
+    return 2 * w + ((k == 0 && a != s.Sb) ? 1 : 0);
+}
+
+// Combine for plans with few partials per unit (large batches): a grid of at most a few
+// CTAs per SM, each taking units u = blockIdx.x, + gridDim.x, ...  Every CTA first turns
+// seq_lens into the tiles' prefix sums in shared memory (before the wait on the split grid:
+// seq_lens is not written by it), so a unit that one warp covered, or an empty one, costs no
+// global access after the wait.  A unit to merge has each warp merge whole rows on its own
+// (all of a row's partial slots, kCombineBatch loads in flight).  Same merge as
+// combine_kernel.  Dynamic shared memory: (B + 1) int32.
+template <int D, int W>
+__global__ void __launch_bounds__(32 * W) combine_unit_kernel(const __grid_constant__ CombineParams p) {
+    constexpr int kCols = D / 4;                 // float4 columns of a row
+    constexpr int kPerLane = (kCols + 31) / 32;  // float4 columns per lane
+    extern __shared__ int32_t s_cum[];           // [B + 1]: tiles of the sequences before b
+    __shared__ int s_wsum[W];
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int B = p.B;
+    {
+        // each thread takes `per` consecutive sequences; block-wide exclusive scan
+        const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
+        const int per = (B + 32 * W - 1) / (32 * W);
+        const int lo = tid * per, hi = min(lo + per, B);
+        int sum = 0;
+        for (int i = lo; i < hi; ++i) {
+            int L = __ldcg(p.seq_lens + i);
+            L = L < 0 ? 0 : (L > cap ? static_cast<int>(cap) : L);
+            const int t = (L + kTile - 1) / kTile;
+            s_cum[i + 1] = t;
+            sum += t;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int run = incl - sum;
+        for (int w = 0; w < warp; ++w) run += s_wsum[w];
+        for (int i = lo; i < hi; ++i) {
+            run += s_cum[i + 1];
+            s_cum[i + 1] = run;
+        }
+        if (tid == 0) s_cum[0] = 0;
+        __syncthreads();
+    }
+    pdl_wait_prior_grid();
+    const int ups = p.Hkv * p.HB;
+    const int units = B * ups;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int b = u / ups;
+        const int ul = u - b * ups;
+        const int kvh = ul / p.HB;
+        const int hb = ul - kvh * p.HB;
+        const int rows = min(kMaxRows, p.g - kMaxRows * hb);
+        const int head0 = kvh * p.g + kMaxRows * hb;
+        const UnitSlots us = unit_slots(p, u, s_cum[b + 1] - s_cum[b], s_cum[b], s_cum[B]);
+        if (us.n == 0) {
+            if (p.mode == 0)  // balanced mode: the combine writes the rows of empty sequences
+                for (int i = tid; i < rows * kCols; i += blockDim.x) {
+                    const int r = i / kCols, c = i - r * kCols;
+                    *reinterpret_cast<uint2*>(p.out + b * p.out_sb + (head0 + r) * p.out_sh + 4 * c) =
+                        make_uint2(0u, 0u);
+                }
+            continue;
+        }
+        if (us.nk <= 1) continue;
+
+        for (int r = warp; r < rows; r += W) {
+            float M = -INFINITY, den = 0.f;
+            float4 acc[kPerLane];
+#pragma unroll
+            for (int j = 0; j < kPerLane; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k0 = 0; k0 < us.nk; k0 += kCombineBatch) {
+                float2 ml[kCombineBatch];
+                float4 o[kCombineBatch][kPerLane];
+#pragma unroll
+                for (int t = 0; t < kCombineBatch; ++t) {
+                    const int kk = k0 + t;
+                    const int64_t slot = kk < us.nk ? slot_of(p, us, ul, kk) : -1;
+                    ml[t] = make_float2(-INFINITY, 0.f);
+                    if (slot >= 0) {
+                        ml[t] = *reinterpret_cast<const float2*>(p.ml_part + (slot * p.rows_max + r) * 2);
+                        const float4* src = reinterpret_cast<const float4*>(p.o_part + (slot * p.rows_max + r) * D);
+#pragma unroll
+                        for (int j = 0; j < kPerLane; ++j) {
+                            const int c = lane + 32 * j;
+                            o[t][j] = c < kCols ? src[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < kCombineBatch; ++t) {
+                    if (!(ml[t].y > 0.f)) continue;  // empty split or no slot
+                    if (ml[t].x > M) {
+                        const float sc = exp2f(M - ml[t].x);  // 0 while M is -inf (acc and den are 0 then)
+                        den *= sc;
+#pragma unroll
+                        for (int j = 0; j < kPerLane; ++j) {
+                            acc[j].x *= sc;
+                            acc[j].y *= sc;
+                            acc[j].z *= sc;
+                            acc[j].w *= sc;
+                        }
+                        M = ml[t].x;
+                    }
+                    const float wgt = exp2f(ml[t].x - M);
+                    den += wgt * ml[t].y;
+#pragma unroll
+                    for (int j = 0; j < kPerLane; ++j) {
+                        acc[j].x += wgt * o[t][j].x;
+                        acc[j].y += wgt * o[t][j].y;
+                        acc[j].z += wgt * o[t][j].z;
+                        acc[j].w += wgt * o[t][j].w;
+                    }
+                }
+            }
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            __nv_bfloat16* orow = p.out + b * p.out_sb + (head0 + r) * p.out_sh;
+#pragma unroll
+            for (int j = 0; j < kPerLane; ++j) {
+                const int c = lane + 32 * j;
+                if (c < kCols) {
+                    uint2 packed;
+                    packed.x = pack_bf16x2(acc[j].x * inv, acc[j].y * inv);
+                    packed.y = pack_bf16x2(acc[j].z * inv, acc[j].w * inv);
+                    *reinterpret_cast<uint2*>(orow + 4 * c) = packed;
+                }
+            }
+        }
+    }
+}
+
 }  // namespace apd

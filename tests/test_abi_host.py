@@ -216,7 +216,11 @@ def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     assert budget - pl.num_workers < ups
     assert pl.partial_slots == 2 * pl.num_workers
     assert pl.rows_per_unit == min(g, 16) and pl.head_blocks == -(-g // 16)
-    assert pl.combine_ctas == B * Hkv * pl.head_blocks * pl.rows_per_unit
+    # when a unit has at most one batch of 4 partials (about groups / B + 1): up to 4
+    # combine CTAs per SM walking the units; else one per (unit, row)
+    per_unit = pl.num_workers // ups // B + 1 <= 4
+    units = B * Hkv * pl.head_blocks
+    assert pl.combine_ctas == (min(units, 4 * 148) if per_unit else units * pl.rows_per_unit)
     assert pl.smem_bytes <= 232448
     assert pl.workspace_bytes % 256 == 0
     assert pl.workspace_bytes == apd.lib().apd_workspace_size(B, Hq, Hkv, D, 0)
@@ -268,7 +272,30 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     local = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=[4096] * B, max_seq_len=4096)
     if local.mode == 2:
         assert local.shared_kv_ring == 0 and local.stages == stages
-        assert local.smem_bytes == _smem(B, D, rows, local.warps_per_cta, stages, hb, False)
+        assert local.smem_bytes == _unit_smem(D, rows, local.warps_per_cta, stages)
+
+
+def _unit_smem(D, rows, warps, stages):
+    """Dynamic shared memory of the one-CTA-per-unit kernel: full mbarriers, the merge
+    mbarrier, the abort word and tile counter (8 bytes), the claimed tile of each stage,
+    1 KB of alignment slack, then one [K | V | Q] ring per warp."""
+    meta = 8 * warps * stages + 8 + 8 + 4 * warps * stages
+    q = -(-rows * D * 2 // 1024) * 1024
+    return -(-meta // 16) * 16 + 1024 + warps * stages * (2 * 32 * D * 2 + q)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,L", [(16, 32, 8, 128, 4096), (18, 16, 8, 64, 3000), (1, 4, 1, 64, 256),
+                                          (16, 8, 8, 32, 1024), (32, 16, 4, 256, 1024)])
+def test_plan_unit_kernel_smem(B, Hq, Hkv, D, L):
+    """With host lengths that give one CTA per unit: the most warps (up to the head dim's
+    maximum) whose rings fit, and the unit kernel's shared-memory layout."""
+    pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=[L] * B, max_seq_len=L)
+    assert pl.mode == 2
+    stages, max_warps = _TRAITS[D]
+    rows = min(Hq // Hkv, 16)
+    w = max(x for x in range(1, max_warps + 1) if _unit_smem(D, rows, x, stages) <= 232448)
+    assert pl.warps_per_cta == w and pl.stages == stages
+    assert pl.smem_bytes == _unit_smem(D, rows, w, stages)
 
 
 @pytest.mark.parametrize("splits", [1, 2, 4, 148])
@@ -280,7 +307,7 @@ def test_plan_fixed(splits):
     assert pl.num_workers == units * splits
     assert pl.grid_ctas == -(-pl.num_workers // pl.warps_per_cta)
     assert pl.partial_slots == (units * splits if splits > 1 else 0)
-    assert pl.combine_ctas == (units * pl.rows_per_unit if splits > 1 else 0)
+    assert pl.combine_ctas == ((min(units, 4 * 148) if splits <= 4 else units * pl.rows_per_unit) if splits > 1 else 0)
     assert pl.workspace_bytes == apd.workspace_size(B, Hq, Hkv, D, splits)
 
 

@@ -74,6 +74,23 @@ def test_ragged_and_empty_sequences(D, S):
     assert torch.all(out[0] == 0) and torch.all(out[8] == 0)
 
 
+@pytest.mark.parametrize("S", [0, 3])
+def test_large_batch_combine_walks_the_units(S):
+    """Batches with more units than the combine grid (at most 4 CTAs per SM): its CTAs walk
+    several units each, skipping the units one warp covered and writing the zero rows of
+    empty sequences (auto splits), or merging fixed splits."""
+    rng = np.random.default_rng(5)
+    lens = rng.integers(0, 400, size=700)
+    lens[::37] = 0
+    w = small(23, B=700, Hq=8, Hkv=1, D=64, lens=lens, pool=int(sum((lens + 31) // 32)) + 8, poison=True,
+              max_pages_per_seq=13)
+    pl = apd.query_plan(700, 8, 1, 64, S)
+    assert 0 < pl.combine_ctas < 700  # units per combine CTA > 1
+    out = DeviceProblem(w).run(S)
+    check_close(out, oracle.paged_decode(w), f"large batch S={S}")
+    assert torch.all(out[torch.from_numpy(lens == 0).to(out.device)] == 0)
+
+
 @pytest.mark.parametrize("S", [1, 0, 5])
 def test_all_sequences_empty(S):
     w = small(22, B=3, Hq=4, Hkv=1, D=64, lens=(0, 0, 0), pool=2, max_pages_per_seq=4)
