@@ -160,13 +160,18 @@ struct Plan {
 // One-CTA-per-unit plan (mode 2, unit_kernel): CTA u owns unit u, its warps claim the
 // unit's tiles from a shared counter and merge their parts in shared memory; a single
 // launch, no partials in the workspace.
-void cta_local_plan(const Shape& s, Plan* pl) {
-    pl->mode = 2;
+// The unit kernel's geometry: the most warps (up to the head dim's maximum) whose rings fit.
+void unit_geometry(const Shape& s, Plan* pl) {
     pl->share = false;
     pl->stages = traits_for(s.D).stages;
     pl->warps = traits_for(s.D).max_warps;
     while (pl->warps > 1 && unit_smem_bytes(s, pl->warps, pl->stages) > kSmemLimit) --pl->warps;
     pl->smem = unit_smem_bytes(s, pl->warps, pl->stages);
+}
+
+void cta_local_plan(const Shape& s, Plan* pl) {
+    pl->mode = 2;
+    unit_geometry(s, pl);
     pl->ksplit = pl->warps;
     pl->groups = 0;
     pl->workers = static_cast<int>(s.units * pl->warps);
@@ -280,18 +285,21 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
         if (host_lens && pl->combine_ctas > 0 && cta_local_wins(s, *pl, sm_count, host_lens, len_cap))
             cta_local_plan(s, pl);
     } else {
+        // fixed splits: one unit-kernel CTA per split of each unit
         pl->mode = 1;
         pl->ksplit = num_splits;
         pl->groups = 0;
-        const int64_t workers = s.units * num_splits;
-        if (workers > INT32_MAX / 2) return APD_ERR_TOO_LARGE;
-        pl->workers = static_cast<int>(workers);
-        pl->slots = num_splits >= 2 ? workers : 0;
+        unit_geometry(s, pl);
+        const int64_t ctas = s.units * num_splits;
+        if (ctas > INT32_MAX / 64) return APD_ERR_TOO_LARGE;
+        pl->ctas = static_cast<int>(ctas);
+        pl->workers = static_cast<int>(ctas * pl->warps);
+        pl->slots = num_splits >= 2 ? ctas : 0;
         pl->combine_ctas = num_splits >= 2 ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
                                                                                         : s.units * s.rows_max)
                                            : 0;
     }
-    if (pl->mode != 2) pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
+    if (pl->mode == 0) pl->ctas = (pl->workers + pl->warps - 1) / pl->warps;
     pl->ws_needed = ws_bytes_for(s, pl->slots);
     if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
     return APD_OK;
@@ -301,7 +309,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
-    bool smem_attr_set[12] = {};  // head dim x {split kernel, split kernel with shared rings, unit kernel}
+    bool smem_attr_set[16] = {};  // head dim x {split kernel, with shared rings, unit kernel, unit kernel with fixed splits}
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -515,11 +523,12 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
             variant = 1;
         }
     }
-    if (pl.mode == 2) {
-        // one CTA per unit: the lean per-tile form at D = 32 and 64 only (the plain form
-        // measured 1% faster for the llama8b shape at D = 128)
-        kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64)>;
-        variant = 2;
+    if (pl.mode != 0) {
+        // one CTA per unit (or per split of a unit): the lean per-tile form at D = 32 and 64
+        // only (the plain form measured 1% faster for the llama8b shape at D = 128)
+        if (pl.mode == 1) kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64), true>;
+        else kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64), false>;
+        variant = pl.mode == 1 ? 3 : 2;
     }
     const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + 4 * variant;
     {

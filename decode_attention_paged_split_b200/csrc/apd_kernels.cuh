@@ -12,13 +12,16 @@
 //    block).  All tiles of all units are laid out in one flattened index space
 //    (b-major, then kv head / head block, then tile), found on the device from
 //    a prefix sum of the per-sequence tile counts.
-//  * Every warp is an independent worker that owns a contiguous run of that
-//    space: in balanced mode (num_splits == 0) the runs are equal shares of the
-//    whole space, one per resident warp of a persistent, SM-count-sized grid;
-//    in fixed mode (num_splits == k) the runs are the k page-aligned chunks of
-//    each unit.  A warp that covers a whole unit writes the final bf16 output;
-//    otherwise it writes an unnormalised fp32 partial plus (m, l), and the
-//    combine kernel merges the partials of each unit.
+//  * split_kernel (auto splits, num_splits == 0): every warp is an independent
+//    worker that owns a contiguous run of that space, an equal share of it, one per
+//    resident warp of a persistent, SM-count-sized grid.  A warp that covers a
+//    whole unit writes the final bf16 output; otherwise it writes an unnormalised
+//    fp32 partial plus (m, l), and the combine kernel merges the partials of each
+//    unit.
+//  * unit_kernel: one CTA per unit when every unit gets an SM of its own (auto
+//    splits with host-known lengths), or one CTA per split of a unit with fixed
+//    splits (num_splits == k, the k page-aligned chunks of each unit).  The CTA's
+//    warps claim its tiles one at a time and merge their parts in shared memory.
 //  * Each warp runs its own STAGES-deep ring in shared memory.  Lane 0 issues
 //    TMA tiled loads (cp.async.bulk.tensor, 128-byte swizzle) of the K and V
 //    tiles [32 tokens x D] of the next tiles straight from the paged cache
@@ -104,8 +107,8 @@ struct SplitParams {
     int32_t zero_empty;  // balanced mode with no combine kernel: write the rows of empty sequences
     uint32_t* flags;
     int32_t B, Hq, Hkv, g, HB, rows_max, P, NP, MP;
-    int32_t mode;       // 0 balanced, 1 fixed (split_kernel); 2 one CTA per unit (unit_kernel)
-    int32_t ksplit;     // fixed mode: k
+    int32_t mode;       // 0 balanced (split_kernel); 1 fixed splits, 2 one CTA per unit (unit_kernel)
+    int32_t ksplit;     // fixed splits: k
     int32_t num_workers;
     int32_t groups;     // balanced mode: worker groups (num_workers = groups * Hkv * HB)
     int32_t warps;      // warps per CTA
@@ -469,9 +472,11 @@ constexpr int kPartStride = D + 8;
 // bytes later.
 // Warp `part` of `nparts` merges rows part, part + nparts, ...:
 //   M = max_k m_k over parts with l_k > 0, out = sum_k 2^(m_k - M) acc_k / sum_k 2^(m_k - M) l_k.
+// With `slot` >= 0 the merged part is written unnormalised to partial slot `slot` instead (the
+// accumulator sum_k 2^(m_k - M) acc_k and (M, sum_k 2^(m_k - M) l_k)), for the combine kernel.
 template <int D>
 __device__ __noinline__ void unit_merge(const SplitParams& p, const uint8_t* ring0, uint32_t warp_bytes,
-                                                int b, int head0, int rows, int part, int nparts, int lane) {
+                                        int b, int head0, int rows, int part, int nparts, int lane, int64_t slot) {
     constexpr int kVec = D / 32;  // consecutive columns per lane
     for (int r = part; r < rows; r += nparts) {
         float M = -INFINITY;
@@ -499,6 +504,13 @@ __device__ __noinline__ void unit_merge(const SplitParams& p, const uint8_t* rin
             }
 #pragma unroll
             for (int e = 0; e < kVec; ++e) acc[e] += wk * v[e];
+        }
+        if (slot >= 0) {
+            float* po = p.o_part + (slot * p.rows_max + r) * D + kVec * lane;
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) po[e] = acc[e];
+            if (lane == 0) *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + r) * 2) = make_float2(M, den);
+            continue;
         }
         const float inv = den > 0.f ? 1.f / den : 0.f;
         __nv_bfloat16* o = p.out + b * p.out_sb + (head0 + r) * p.out_sh + kVec * lane;
@@ -621,42 +633,15 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
         }
     }
 
-    // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-
-    // sequence ul (kv head and head block).
-    int ws, we, ul;
-    int fixed_slot = -1;
-    if (p.mode == 0) {
-        // Workers form groups of units_per_seq warps, one per (kv head, head block);
-        // group grp owns an equal share of the positions of all sequences.  The warps
-        // of a group walk the same pages together, so the kv heads of a page are read
-        // at about the same time.
-        const int grp = w / units_per_seq;
-        ul = w - grp * units_per_seq;
-        ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
-        we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
-    } else {
-        // fixed splits: warp w takes split w % k of unit w / k
-        const int u = w / p.ksplit;
-        const int s = w - u * p.ksplit;
-        const int b = u / units_per_seq;
-        ul = u - b * units_per_seq;
-        const int n = s_cum[b + 1] - s_cum[b];
-        if (n == 0) {
-            if (s == 0) {
-                const int kvh = ul / p.HB, hb = ul - (ul / p.HB) * p.HB;
-                write_zero_rows<D>(p, b, kvh * p.g + kMaxRows * hb, min(kMaxRows, p.g - kMaxRows * hb), lane);
-            }
-            return;
-        }
-        const int S = min(p.ksplit, n);
-        const int c = (n + S - 1) / S;
-        const int t0 = s * c;
-        if (t0 >= n) return;
-        const int t1 = min(t0 + c, n);
-        ws = s_cum[b] + t0;
-        we = s_cum[b] + t1;
-        fixed_slot = u * p.ksplit + s;
-    }
+    // This warp's run [ws, we) of sequence-tile positions, all for one unit-in-sequence ul
+    // (kv head and head block).  Workers form groups of units_per_seq warps, one per (kv
+    // head, head block); group grp owns an equal share of the positions of all sequences.
+    // The warps of a group walk the same pages together, so the kv heads of a page are read
+    // at about the same time.
+    const int grp = w / units_per_seq;
+    const int ul = w - grp * units_per_seq;
+    const int ws = static_cast<int>(run_start(grp, s_cum[B], p.groups));
+    const int we = static_cast<int>(run_start(grp + 1, s_cum[B], p.groups));
     if (ws >= we) return;
 
     const uint32_t bar0 = smem_u32(bars + warp * STAGES);
@@ -836,8 +821,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
             if (direct) {
                 st.write_out(p.out + cb * p.out_sb + head0 * p.out_sh, p.out_sh, rows, lane);
             } else {
-                const int64_t slot =
-                    (p.mode == 0) ? (2 * static_cast<int64_t>(w) + (seg_start == ws ? 0 : 1)) : fixed_slot;
+                const int64_t slot = 2 * static_cast<int64_t>(w) + (seg_start == ws ? 0 : 1);
                 st.write_part(p.o_part + slot * p.rows_max * D, D, p.ml_part + slot * p.rows_max * 2, rows, lane);
             }
         }
@@ -846,7 +830,12 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
 }
 
 // One CTA per unit (sequence b = unit / (Hkv * HB), kv head, head block), for launches in
-// which every unit has an SM of its own; the call is this one kernel.
+// which every unit has an SM of its own (mode 2; the call is this one kernel), or, FIXED, one
+// CTA per split of a unit with fixed splits (mode 1, k = ksplit: CTA u k + s takes split s,
+// the tiles [s c, min((s + 1) c, n)) with c = ceil(n / min(k, n)), and writes the output when
+// the unit has one non-empty split, else a partial for the combine kernel).  The two are
+// separate instantiations: code for fixed splits in the mode-2 kernel measured 8% slower on
+// the llama8b shape (47.3 against 43.9 us), with the mode-2 path itself unchanged.
 //  * The mbarriers are set up before the wait on the previous grid.  After it, lane 0 of
 //    each warp loads the sequence's length and claims its first STAGES + 1 tiles, loading
 //    their page-table entries as the claims return.  (Deterministic first tiles, with all
@@ -861,7 +850,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, SHARE>, 1)
 // Shared-memory layout: [full mbarriers, warps x STAGES][merge mbarrier][abort word, tile
 // counter][claimed tile of each stage, warps x STAGES], then 1024-aligned rings of
 // [K | V | Q] stages, one ring per warp.
-template <int D, int STAGES, bool LEAN>
+template <int D, int STAGES, bool LEAN, bool FIXED>
 __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
     unit_kernel(const __grid_constant__ SplitParams p, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
@@ -900,7 +889,9 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
     pdl_wait_prior_grid();
     pdl_launch_dependents();
 
-    const int u = blockIdx.x;
+    const int nsplit = FIXED ? p.ksplit : 1;
+    const int u = FIXED ? blockIdx.x / nsplit : blockIdx.x;
+    const int split = FIXED ? blockIdx.x - u * nsplit : 0;
     const int ups = p.Hkv * p.HB;
     const int b = u / ups;
     const int ul = u - b * ups;
@@ -923,9 +914,31 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
                    ? __ldcg(pt_row + static_cast<int64_t>(t / tiles_per_page) * p.pt_s1) : 0;
     };
     int32_t nxt_pg = 0;
+    // Fixed splits take their tiles in a fixed order, so that a call's result does not depend
+    // on timing: warp w streams the w-th contiguous share [w_lo, w_hi) of the split's tiles.
+    int w_lo = 0, w_hi = 0;
     auto claim = [&]() {  // lane 0
-        nxt_t = static_cast<int>(atomicAdd(s_next, 1u));
-        nxt_pg = page_of(nxt_t);
+        if constexpr (FIXED) {
+            nxt_t = w_lo < w_hi ? w_lo++ : (1 << 30);
+            nxt_pg = nxt_t < w_hi ? page_of(nxt_t) : 0;
+        } else {
+            nxt_t = static_cast<int>(atomicAdd(s_next, 1u));
+            nxt_pg = page_of(nxt_t);
+        }
+    };
+    // The split [t0, t1) of n tiles (fixed splits), and how many splits are not empty.
+    auto split_range = [&](int n, int& t0, int& t1, int& nk) {
+        if (!FIXED || n == 0) {
+            t0 = 0;
+            t1 = n;
+            nk = 1;
+            return;
+        }
+        const int S = max(1, min(nsplit, n));
+        const int c = (n + S - 1) / S;
+        t0 = min(split * c, n);
+        t1 = min(t0 + c, n);
+        nk = (n + c - 1) / c;
     };
     // lane 0: the sequence's length, then this warp's first STAGES + 1 claims with their pages
     int L = 0;
@@ -933,6 +946,27 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
     int32_t pg0[STAGES];
     if (lane == 0) {
         L = __ldcg(p.seq_lens + b);
+        auto clamp_len = [&]() {
+            uint32_t len_flags = 0;
+            if (L < 0) {
+                L = 0;
+                len_flags |= kFlagLenNegative;
+            }
+            if (L > cap) {
+                L = static_cast<int>(cap);
+                len_flags |= kFlagLenClamped;
+            }
+            if (len_flags && warp == 0 && split == 0) atomicOr(p.flags, len_flags);
+        };
+        if constexpr (FIXED) {
+            // fixed splits: the split's tiles depend on the length, so it comes first
+            clamp_len();
+            int s0, s1, nk_;
+            split_range((L + kTile - 1) / kTile, s0, s1, nk_);
+            const int cnt = s1 - s0, c = (cnt + W - 1) / W;
+            w_lo = s0 + min(cnt, warp * c);
+            w_hi = s0 + min(cnt, (warp + 1) * c);
+        }
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) {
             claim();
@@ -940,19 +974,15 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
             pg0[s] = nxt_pg;
         }
         claim();
-        uint32_t len_flags = 0;
-        if (L < 0) {
-            L = 0;
-            len_flags |= kFlagLenNegative;
-        }
-        if (L > cap) {
-            L = static_cast<int>(cap);
-            len_flags |= kFlagLenClamped;
-        }
-        if (len_flags && warp == 0) atomicOr(p.flags, len_flags);
+        if constexpr (!FIXED) clamp_len();
     }
     L = __shfl_sync(0xffffffffu, L, 0);
     const int n = (L + kTile - 1) / kTile;
+    int t_lo, t_hi, nk;  // this CTA's tiles [t_lo, t_hi) and the unit's non-empty splits
+    split_range(n, t_lo, t_hi, nk);
+    // an empty split writes nothing (the unit's output, zeros for an empty sequence, comes
+    // from split 0)
+    if (FIXED && t_lo >= t_hi && split > 0) return;
 
     // Issue tile t (page pg) into stage `stage`, with the Q rows on this warp's first tile.
     auto issue = [&](int stage, int t, int32_t pg, bool qload) {  // lane 0
@@ -976,7 +1006,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) {
-            if (t0[s] < n) {
+            if (t0[s] < t_hi) {
                 issue(s, t0[s], pg0[s], s == 0);
                 ++issued;
             }
@@ -1004,7 +1034,7 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
         fence_proxy_async_smem();
         __syncwarp();
         int more = 0;
-        if (lane == 0 && nxt_t < n) {
+        if (lane == 0 && nxt_t < t_hi) {
             issue(stage, nxt_t, nxt_pg, false);
             claim();
             more = 1;
@@ -1017,8 +1047,10 @@ __global__ void __launch_bounds__(32 * kMaxWarpsD<D, false>, 1)
     st.write_part(own + 2 * kMaxRows, kPartStride<D>, own, rows, lane);
     mbar_arrive(smem_u32(merge_bar));
     if (!warp_wait(smem_u32(merge_bar), 0u, p.wait_ns, s_abort, p.flags)) return;
-    unit_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, b, head0,
-                       rows, warp, W, lane);
+    // one non-empty split: the output; else this split's partial
+    const int64_t slot = (FIXED && nk > 1) ? static_cast<int64_t>(u) * nsplit + split : -1;
+    unit_merge<D>(p, smem + (ring - smem_u32(smem)), static_cast<uint32_t>(STAGES) * p.stage_bytes, b, head0, rows,
+                  warp, W, lane, slot);
 }
 
 constexpr int kCombineBatch = 4;  // partial slots whose loads a warp issues together

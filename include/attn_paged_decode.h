@@ -197,7 +197,14 @@ int apd_attn_paged_decode(const apd_tensor* q, const apd_tensor* k_cache, const 
  *                     (plan mode 2), with no partials and no combine kernel.
  *                     Otherwise the plan is the one without the hint.  The kernels
  *                     always read the lengths from the device seq_lens, so a hint
- *                     that differs from them changes the speed, never the result.
+ *                     that differs from them changes the speed, never the result
+ *                     beyond rounding.  Mode 2 is the one plan that is not bitwise
+ *                     reproducible: its warps take the unit's tiles in the order
+ *                     they become free (the fastest order measured), so the parts
+ *                     they merge, and the last bits of the output, can differ from
+ *                     call to call (always within the accuracy of the other plans).
+ *                     Without the hint, and with fixed splits, every call on the
+ *                     same inputs gives the same bits.
  */
 typedef struct apd_launch_options {
     void* split_done_event;       /* cudaEvent_t or NULL */

@@ -264,11 +264,12 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     assert pl.shared_kv_ring == int(shared)
     assert pl.warps_per_cta == ws[0] and pl.stages == stages
     assert pl.smem_bytes == _smem(B, D, rows, ws[0], stages, hb, shared)
-    # fixed splits and the one-CTA-per-unit plan keep one ring per warp
-    stages, ws = fits(False)
+    # fixed splits and the one-CTA-per-unit plan run the unit kernel: one ring per warp
+    stages, max_warps = _TRAITS[D]
+    uw = max(x for x in range(1, max_warps + 1) if _unit_smem(D, rows, x, stages) <= 232448)
     fixed = apd.query_plan(B, Hq, Hkv, D, 2, sm_count=148)
-    assert fixed.shared_kv_ring == 0 and fixed.stages == stages and fixed.warps_per_cta == ws[0]
-    assert fixed.smem_bytes == _smem(B, D, rows, ws[0], stages, hb, False)
+    assert fixed.shared_kv_ring == 0 and fixed.stages == stages and fixed.warps_per_cta == uw
+    assert fixed.smem_bytes == _unit_smem(D, rows, uw, stages)
     local = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=[4096] * B, max_seq_len=4096)
     if local.mode == 2:
         assert local.shared_kv_ring == 0 and local.stages == stages
@@ -304,8 +305,9 @@ def test_plan_fixed(splits):
     pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=148)
     units = B * Hkv
     assert pl.mode == 1
-    assert pl.num_workers == units * splits
-    assert pl.grid_ctas == -(-pl.num_workers // pl.warps_per_cta)
+    # one unit-kernel CTA per split of each unit
+    assert pl.grid_ctas == units * splits
+    assert pl.num_workers == pl.grid_ctas * pl.warps_per_cta
     assert pl.partial_slots == (units * splits if splits > 1 else 0)
     assert pl.combine_ctas == ((min(units, 4 * 148) if splits <= 4 else units * pl.rows_per_unit) if splits > 1 else 0)
     assert pl.workspace_bytes == apd.workspace_size(B, Hq, Hkv, D, splits)
@@ -589,7 +591,8 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
     - every CTA's warps are within the launch bound;
     - the grid covers the workers;
     - with a shared K/V ring, the head blocks of a kv head share a CTA;
-    - with the CTA-local plan, each unit gets its own SM and no combine runs."""
+    - with fixed splits, one unit-kernel CTA per split of each unit;
+    - with the one-CTA-per-unit plan, each unit gets its own SM and no combine runs."""
     Hq = Hkv * g
     hb = -(-g // 16)
     pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=sm, host_seq_lens=[L] * B, max_seq_len=70000)
@@ -608,7 +611,8 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
         assert splits == 0 and pl.num_workers % (Hkv * hb) == 0
         assert pl.grid_ctas <= max(sm, -(-(Hkv * hb) // pl.warps_per_cta))
     elif pl.mode == 1:
-        assert splits > 0 and pl.num_workers == units * splits
+        assert splits > 0 and pl.grid_ctas == units * splits
+        assert pl.num_workers == pl.grid_ctas * pl.warps_per_cta
     else:
         assert splits == 0 and pl.mode == 2 and units <= sm
         assert pl.grid_ctas == units and pl.combine_ctas == 0 and pl.partial_slots == 0
