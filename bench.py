@@ -141,7 +141,7 @@ def make_instances(name: str, rank: int, count: int = 2):
     table) and independent values; the seed of the values differs per rank and instance."""
     gen = workloads.NAMED[name]
     base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262, "llama8b_contig": 8,
-            "long_contig": 131072, "gqa32": 32}[name]
+            "long_contig": 131072, "gqa32": 32, "hd32": 77, "hd64": 77, "hd256": 77}[name]
     return [gen(seed=base, value_seed=base + 1000003 * rank + i) for i in range(count)]
 
 

@@ -444,6 +444,17 @@ def gqa32(seed: int = 32, **kw) -> Workload:
     return make(**args)
 
 
+def head_dim_scale(head_dim: int, seed: int = 77, **kw) -> Workload:
+    """The llama8b shape (B=16, 32 q heads / 8 kv heads) at another head dim, with the
+    sequence length that keeps 268 MB of K/V: L = 4096 * 128 / D, shuffled pool."""
+    L = 4096 * 128 // head_dim
+    args = dict(name=f"hd{head_dim}_b16_h32x8_d{head_dim}_l{L}", seed=seed, batch=16, num_q_heads=32,
+                num_kv_heads=8, head_dim=head_dim, page_size=32, seq_lens=[L] * 16, pool_pages=16 * L // 32,
+                num_splits=0)
+    args.update(kw)
+    return make(**args)
+
+
 NAMED = {
     "tiny": tiny,
     "llama8b": llama8b,
@@ -452,6 +463,9 @@ NAMED = {
     "gqa32": gqa32,
     "llama8b_contig": llama8b_contig,
     "long_contig": long_contig,
+    "hd32": lambda seed=77, **kw: head_dim_scale(32, seed, **kw),
+    "hd64": lambda seed=77, **kw: head_dim_scale(64, seed, **kw),
+    "hd256": lambda seed=77, **kw: head_dim_scale(256, seed, **kw),
 }
 
 
