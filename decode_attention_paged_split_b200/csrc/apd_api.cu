@@ -181,11 +181,16 @@ void cta_local_plan(const Shape& s, Plan* pl) {
 }
 
 // Whether the one-CTA-per-unit plan beats the balanced plan `pl` for these host-known lengths
-// (clamped to [0, len_cap] as the kernels clamp them).  Only when every unit gets a CTA
-// of its own on a distinct SM, and the longest unit is at most the balanced plan's
-// share per CTA plus about what the combine kernel costs: 3% and 1024 / D tiles.
+// (clamped to [0, len_cap] as the kernels clamp them).  Only when every unit gets a CTA of
+// its own on a distinct SM, a kv head has one head block (with more, each block's CTA would
+// stream the kv head's K/V again: g = 32 measured 187 against 62 us), and the longest unit
+// is at most the share per CTA of a launch on max(units, 7/8 of the SMs) CTAs (so that a
+// few long units, which would leave most SMs idle, do not qualify) plus about what the
+// combine kernel costs: 3% and 1024 / D tiles.  Measured on B200 at 268 MB of K/V, 128
+// equal units: D = 32 53.4 -> 49.7 us, D = 64 48.5 -> 43.9 us, D = 128 46.2 -> 43.9 us,
+// D = 256 49.2 -> 45.7 us against the balanced plan.
 bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t* host_lens, int64_t len_cap) {
-    if (s.units > sm_count || pl.ctas < 1) return false;
+    if (s.units > sm_count || pl.ctas < 1 || s.HB > 1) return false;
     // a part's (m, l) and accumulator rows go to its warp's ring once the stream ends
     if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(traits_for(s.D).stages) * stage_bytes(s))
         return false;
@@ -197,7 +202,8 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
         total += n * ups;
         longest = std::max(longest, n);
     }
-    const int64_t share = (total + pl.ctas - 1) / pl.ctas;
+    const int64_t ctas = std::max<int64_t>(s.units, static_cast<int64_t>(sm_count) * 7 / 8);
+    const int64_t share = (total + ctas - 1) / ctas;
     return 32 * longest <= 33 * share + 32 * (1024 / s.D);
 }
 

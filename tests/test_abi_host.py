@@ -322,14 +322,16 @@ def test_plan_small_workspace_uses_fewer_workers():
 
 
 def cta_local_expected(B, Hq, Hkv, D, lens, cap, sm=148):
-    """The CTA-local choice restated from its rule: every unit on its own SM, and the
-    longest unit within 3% plus 1024 / D tiles of the balanced plan's share per CTA."""
+    """The one-CTA-per-unit choice restated from its rule: every unit on its own SM, one
+    head block per kv head, and the longest unit within 3% plus 1024 / D tiles of the share
+    per CTA of a launch on max(units, 7/8 of the SMs) CTAs."""
     base = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
     units = B * Hkv * base.head_blocks
     tiles = [-(-min(max(L, 0), cap) // 32) for L in lens]
     total = sum(tiles) * Hkv * base.head_blocks
-    share = -(-total // base.grid_ctas)
-    return units <= sm and base.combine_ctas > 0 and 32 * max(tiles) <= 33 * share + 32 * (1024 // D)
+    share = -(-total // max(units, sm * 7 // 8))
+    return (units <= sm and base.head_blocks == 1 and base.combine_ctas > 0
+            and 32 * max(tiles) <= 33 * share + 32 * (1024 // D))
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,D,lens,cap,want", [
@@ -346,6 +348,10 @@ def cta_local_expected(B, Hq, Hkv, D, lens, cap, sm=148):
     (18, 16, 8, 64, [3000] * 18, 3008, 2),             # 144 units on 148 SMs (D = 64 uses every SM)
     (4, 40, 2, 64, [1500] * 4, 1536, 0),               # 16 units: balanced spreads them wider
     (1, 4, 1, 64, [256], 256, 2),                      # the tiny case: one unit, one launch
+    (16, 32, 8, 32, [16384] * 16, 16384, 2),           # other head dims at 128 equal units
+    (16, 32, 8, 64, [8192] * 16, 8192, 2),
+    (16, 32, 8, 256, [2048] * 16, 2048, 2),
+    (16, 64, 2, 128, [16384] * 16, 16384, 0),          # two head blocks per kv head: balanced, shared ring
 ])
 def test_plan_cta_local_from_host_lengths(B, Hq, Hkv, D, lens, cap, want):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=lens, max_seq_len=cap)

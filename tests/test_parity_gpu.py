@@ -472,14 +472,18 @@ HINT_LEN = {32: 1140, 64: 564, 128: 250, 256: 120}
 @pytest.mark.parametrize("D", workloads.SWEEP_HEAD_DIMS)
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (40, 2), (8, 8), (48, 1)])
 def test_host_hint_cta_local_matches_oracle(D, Hq, Hkv):
-    """Equal lengths: the hint selects the one-kernel plan (mode 2); g = 4, 20 (two head
-    blocks, the second partial), 1 and 48 (three)."""
+    """Equal lengths: the hint selects the one-kernel plan (mode 2) for g = 4 and 1; with
+    more than one head block per kv head (g = 20, the second block partial, and 48) each
+    block's CTA would stream the K/V again, so the balanced plan stays."""
     L = HINT_LEN[D]
     lens = [L] * 5
     mp = -(-L // 32)
     w = small(71, B=5, Hq=Hq, Hkv=Hkv, D=D, lens=lens, pool=5 * mp + 4, poison=True, max_pages_per_seq=mp)
     pl = apd.query_plan(5, Hq, Hkv, D, 0, host_seq_lens=lens, max_seq_len=mp * 32)
-    assert pl.mode == 2 and pl.combine_ctas == 0
+    if Hq // Hkv <= 16:
+        assert pl.mode == 2 and pl.combine_ctas == 0
+    else:
+        assert pl.mode == 0
     out, ws = run_hinted(w, lens)
     check_close(out, oracle.paged_decode(w), f"hint D={D} {Hq}/{Hkv}")
     assert apd.read_device_flags(ws) == 0
