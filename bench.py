@@ -251,6 +251,19 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- measurement legs
 DECODE_KERNEL_SOURCES = ("apd_kernels.cuh", "apd_ptx.cuh")  # the split and combine kernels' device code
+# the tensor-core multi-query decode kernel (plan mode 3) and the pieces it is built from
+DECODE_TC_KERNEL_SOURCES = ("apd_decode_tc.cuh", "apd_kernels.cuh", "apd_prefill_tc.cuh", "apd_ptx.cuh")
+PLAN_MODE_NAMES = {0: "balanced + combine", 1: "fixed splits", 2: "one CTA per unit, single kernel",
+                   3: "tensor-core multi-query"}
+
+
+def decode_kernel_of(plan) -> tuple:
+    """The dominant kernel of a decode plan and the headers its device code comes from."""
+    if plan.mode == 3:
+        return "decode_mq_tc_kernel", DECODE_TC_KERNEL_SOURCES
+    if plan.mode in (1, 2):
+        return "unit_kernel", DECODE_KERNEL_SOURCES
+    return "split_kernel", DECODE_KERNEL_SOURCES
 
 
 def _code_only(text: str) -> str:
@@ -603,6 +616,7 @@ def measure_decode(a, name, apd, device, dist, rank, local, min_seconds, want_cl
     plan = apd.query_plan(w0.batch, w0.num_q_heads, w0.num_kv_heads, w0.head_dim, a.num_splits,
                           host_seq_lens=insts[0].host_lens, max_seq_len=max_len)
     launches_per_step = 1 + (1 if plan.combine_ctas > 0 else 0)
+    kname, ksources = decode_kernel_of(plan)
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize(device)
 
@@ -630,7 +644,7 @@ def measure_decode(a, name, apd, device, dist, rank, local, min_seconds, want_cl
             print(f"graph split timing unavailable ({err}); using eager event pairs", file=sys.stderr)
             _, split_s = time_steps(insts, stream, a.steps, split_events=True)
         split_s = max_over_ranks(split_s, dist, device)
-        kernel_timing = ("CUDA events recorded around each split kernel inside replays of a "
+        kernel_timing = (f"CUDA events recorded around each {kname} launch inside replays of a "
                          f"{GRAPH_CHUNK}-call graph (event-record nodes)")
     peak, peak_src = peaks()
     mean_bytes = bytes_rank / a.steps
@@ -639,15 +653,14 @@ def measure_decode(a, name, apd, device, dist, rank, local, min_seconds, want_cl
         "workload": w0.name, "us_per_call": t_med / a.steps * 1e6, "value": bytes_all / t_med / 1e9,
         "timing": timing_summary(times, a.steps),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                     "traffic": committed_traffic(name), "peak_source": peak_src, "kernel": "split_kernel",
+                     "traffic": committed_traffic(name, sources=ksources), "peak_source": peak_src, "kernel": kname,
                      "kernel_us": split_s * 1e6, "kernel_timing": kernel_timing,
                      "call_frac_of_peak": bytes_all / t_med / 1e9 / max(1, (dist.get_world_size() if dist else 1))
                      / peak},
         "gpu_launches": launches_per_step * a.steps * len(times),
         "clocks": clock_info,
         "plan": {"mode": plan.mode,
-                 "mode_name": {0: "balanced + combine", 1: "fixed splits", 2: "one CTA per unit, single kernel"}
-                 [plan.mode],
+                 "mode_name": PLAN_MODE_NAMES.get(plan.mode, str(plan.mode)),
                  "workers": plan.num_workers, "ctas": plan.grid_ctas, "warps_per_cta": plan.warps_per_cta,
                  "stages": plan.stages, "smem": plan.smem_bytes, "shared_kv_ring": bool(plan.shared_kv_ring),
                  "combine_ctas": plan.combine_ctas},

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "../../include/attn_paged_decode.h"
+#include "apd_decode_tc.cuh"
 #include "apd_gemv.cuh"
 #include "apd_kernels.cuh"
 #include "apd_prefill_tc.cuh"
@@ -207,6 +208,36 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
     return 32 * longest <= 33 * share + 32 * (1024 / s.D);
 }
 
+// Tensor-core multi-query plan (mode 3, decode_mq_tc_kernel): kv heads with 32 query heads
+// at D = 128.  One CTA per split of each (sequence, kv head); its 128-token tiles meet all
+// 32 query heads in one tcgen05 MMA, where the split kernel needs two head blocks.  The
+// partials take the fixed-split slots (the head blocks' rows of each split), so the combine
+// is the fixed-split one.
+using McShape128 = apd::McShape<128, 32>;
+constexpr int kMcWarps = McShape128::kThreads / 32;
+bool mq_tc_eligible(const Shape& s) { return s.D == 128 && s.g == 32; }
+
+// Splits per unit with automatic splitting: the (sequence, kv head) units spread over 7/8
+// of the SMs (the rate at which D = 128 streams best, as in the balanced plan), at most one
+// split per 128-token tile the page table can address, and no more than the workspace
+// holds.  Returns 0 when the workspace holds no partials at all and the unit count needs
+// some.
+int64_t mq_tc_auto_splits(const Shape& s, int sm_count, size_t ws_bytes, int64_t tiles_bound) {
+    const int64_t u2 = static_cast<int64_t>(s.B) * s.Hkv;
+    int64_t k = std::max<int64_t>(1, static_cast<int64_t>(sm_count) * 7 / 8 / std::max<int64_t>(1, u2));
+    if (tiles_bound >= 0) {
+        const int64_t per_unit = tiles_bound / std::max<int64_t>(1, s.units);  // 32-token tiles
+        k = std::min<int64_t>(k, std::max<int64_t>(1, (per_unit + 3) / 4));
+    }
+    if (ws_bytes != SIZE_MAX && k > 1) {
+        const int64_t fit = slots_fitting(s, ws_bytes) / std::max<int64_t>(1, s.units);
+        k = std::max<int64_t>(1, std::min(k, fit));
+    }
+    return k;
+}
+
+void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, Plan* pl);
+
 // Warps of a combine CTA: enough for one batch of kCombineBatch partial slots per warp,
 // 4 to 16.  A unit has about groups / B partials in the balanced mode (each sequence's
 // share of the groups, plus the one it starts in) and num_splits in the fixed mode.
@@ -236,12 +267,38 @@ int64_t combine_unit_ctas(const Shape& s, int sm_count) {
     return std::min<int64_t>(s.units, static_cast<int64_t>(sm_count) * kCombineUnitCtasPerSm);
 }
 
+void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, Plan* pl) {
+    pl->mode = 3;
+    pl->share = false;
+    pl->ksplit = static_cast<int>(ksplit);
+    pl->groups = 0;
+    pl->warps = kMcWarps;
+    pl->stages = McShape128::kStages;
+    pl->smem = McShape128::kSmemBytes;
+    pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * ksplit);
+    pl->workers = pl->ctas;
+    pl->slots = ksplit >= 2 ? s.units * ksplit : 0;
+    pl->combine_ctas = ksplit >= 2 ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
+                                                                              : s.units * s.rows_max)
+                                   : 0;
+}
+
 // tiles_bound: an upper bound on the number of tiles (host-known), or -1.
 // host_lens: NULL, or the B sequence lengths as the host knows them (a planning hint;
 // the kernels read the device lengths), clamped to len_cap.
+// allow_tc: the tensor-core multi-query plan may be chosen (the shared-ring self-test turns
+// it off to reach the shared ring).
 int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl,
-              const int32_t* host_lens = nullptr, int64_t len_cap = 0) {
+              const int32_t* host_lens = nullptr, int64_t len_cap = 0, bool allow_tc = true) {
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
+    if (allow_tc && mq_tc_eligible(s)) {
+        const int64_t k = num_splits > 0 ? num_splits : mq_tc_auto_splits(s, sm_count, ws_bytes, tiles_bound);
+        if (static_cast<int64_t>(s.B) * s.Hkv * k > INT32_MAX / 64) return APD_ERR_TOO_LARGE;
+        mq_tc_plan(s, k, sm_count, pl);
+        pl->ws_needed = ws_bytes_for(s, pl->slots);
+        if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
+        return APD_OK;
+    }
     const Traits t = traits_for(s.D);
     pl->stages = t.stages;
     pl->warps = warps_for(s);
@@ -316,6 +373,7 @@ struct DeviceState {
     bool init = false;
     int sm_count = 0;
     bool smem_attr_set[16] = {};  // head dim x {split kernel, with shared rings, unit kernel, unit kernel with fixed splits}
+    bool mq_tc_attr_set = false;
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -512,11 +570,150 @@ struct SplitTestHooks {
     int skip_release = 0;
 };
 
+// The caller's split_done_event, recorded right after the first kernel of the call.
+int record_split_done(const apd_launch_options* opts, cudaStream_t stream) {
+    if (!(opts && opts->split_done_event)) return APD_OK;
+    // while the stream is being captured into a CUDA graph the record becomes an
+    // event-record node (external), so the event still times the replayed kernel
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(opts->split_done_event), stream,
+                                 cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(split_done_event)");
+    return APD_OK;
+}
+
+// The combine kernel of a call whose first kernel wrote partials (launched with PDL unless
+// PDL is off or an event separates the two kernels).
+template <int D>
+int launch_combine(const Shape& s, const Plan& pl, const apd::CombineParams& cp, cudaStream_t stream,
+                   const apd_launch_options* opts) {
+    const bool use_pdl = !(opts && opts->disable_pdl);
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const bool per_unit = combine_per_unit(s, pl);
+    const int cw = per_unit ? (s.rows_max >= 8 ? 8 : 4) : combine_warps(s, pl);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = per_unit ? dim3(static_cast<unsigned>(pl.combine_ctas))
+                           : dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
+    cfg.blockDim = dim3(32 * cw);
+    cfg.dynamicSmemBytes = per_unit ? 4u * (s.B + 1) : 0u;
+    cfg.stream = stream;
+    cfg.attrs = pdl_attr;
+    cfg.numAttrs = (use_pdl && !(opts && opts->split_done_event)) ? 1 : 0;
+    cudaError_t e;
+    if (per_unit)
+        e = cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 8>, cp)
+                    : cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 4>, cp);
+    else
+        e = cw == 16 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 16>, cp)
+            : cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 8>, cp)
+                      : cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 4>, cp);
+    if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+    return APD_OK;
+}
+
+// Mode 3: the tensor-core multi-query kernel, then the combine when units are split.
+int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
+                 const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
+                 void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
+    constexpr int D = 128;
+    auto kern = apd::decode_mq_tc_kernel<D, 32>;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!dev->mq_tc_attr_set) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(McShape128::kSmemBytes));
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mq_tc_kernel)");
+            dev->mq_tc_attr_set = true;
+        }
+    }
+    // K/V boxes of one 64-element block each, so that a tile's rows of one block are
+    // contiguous (the canonical operand layout)
+    CUtensorMap kmap, vmap;
+    int rc = encode_kv_map(&kmap, k, V.kst, D, 1);
+    if (!rc) rc = encode_kv_map(&vmap, v, V.vst, D, 1);
+    if (rc) return rc;
+
+    const Shape& s = V.s;
+    char* ws = static_cast<char*>(workspace);
+    apd::McParams mp;
+    mp.q = static_cast<const __nv_bfloat16*>(q->data);
+    mp.q_sb = V.qst[0];
+    mp.q_sh = V.qst[1];
+    mp.page_table = pt ? static_cast<const int32_t*>(pt->data) : nullptr;
+    mp.pt_s0 = V.pst[0];
+    mp.pt_s1 = V.pst[1];
+    mp.seq_lens = static_cast<const int32_t*>(sl->data);
+    mp.out = static_cast<__nv_bfloat16*>(out->data);
+    mp.out_sb = V.ost[0];
+    mp.out_sh = V.ost[1];
+    mp.o_part = reinterpret_cast<float*>(ws + ws_head_bytes(s));
+    mp.ml_part = reinterpret_cast<float*>(ws + ws_head_bytes(s) +
+                                          align_up(static_cast<size_t>(pl.slots) * s.rows_max * s.D * 4, kWsAlign));
+    mp.flags = reinterpret_cast<uint32_t*>(ws);
+    mp.B = s.B;
+    mp.Hkv = s.Hkv;
+    mp.g = s.g;
+    mp.HB = s.HB;
+    mp.rows_max = s.rows_max;
+    mp.P = V.P;
+    mp.NP = V.NP;
+    mp.MP = V.MP;
+    mp.ksplit = pl.ksplit;
+    mp.scale_log2 = scale * 1.4426950408889634f;
+
+    const bool use_pdl = !(opts && opts->disable_pdl);
+    cudaLaunchAttribute pdl_attr[1];
+    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.ctas));
+    cfg.blockDim = dim3(static_cast<unsigned>(McShape128::kThreads));
+    cfg.dynamicSmemBytes = McShape128::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = pdl_attr;
+    cfg.numAttrs = use_pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp, kmap, vmap);
+    if (e != cudaSuccess) return cuda_fail(e, "decode_mq_tc_kernel launch");
+    rc = record_split_done(opts, stream);
+    if (rc) return rc;
+    if (pl.combine_ctas > 0) {
+        apd::CombineParams cp;
+        cp.cum = reinterpret_cast<int32_t*>(ws + kWsAlign);
+        cp.seq_lens = mp.seq_lens;
+        cp.MP = mp.MP;
+        cp.P = mp.P;
+        cp.o_part = mp.o_part;
+        cp.ml_part = mp.ml_part;
+        cp.out = mp.out;
+        cp.out_sb = mp.out_sb;
+        cp.out_sh = mp.out_sh;
+        cp.B = s.B;
+        cp.Hkv = s.Hkv;
+        cp.g = s.g;
+        cp.HB = s.HB;
+        cp.rows_max = s.rows_max;
+        cp.mode = pl.mode;
+        cp.ksplit = pl.ksplit;
+        cp.num_workers = pl.workers;
+        cp.groups = pl.groups;
+        return launch_combine<D>(s, pl, cp, stream, opts);
+    }
+    return APD_OK;
+}
+
 template <int D>
 int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
            const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts,
            const SplitTestHooks& hooks = SplitTestHooks()) {
+    if constexpr (D == 128) {
+        if (pl.mode == 3) return launch_mq_tc(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts);
+    }
+    if (pl.mode == 3) return APD_ERR_ARGUMENT;  // planned only for D = 128
     constexpr int kStagesD = kStages<D>;
     // the lean per-tile form everywhere but D = 256 (the split kernel's LEAN parameter lists
     // the measurements)
@@ -606,18 +803,8 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
         cudaError_t e = cudaLaunchKernelEx(&cfg, kern, sp, kmap, vmap, qmap);
         if (e != cudaSuccess) return cuda_fail(e, "split_kernel launch");
     }
-    cudaError_t e = cudaSuccess;
-    if (opts && opts->split_done_event) {
-        // while the stream is being captured into a CUDA graph the record becomes an
-        // event-record node (external), so the event still times the replayed kernel
-        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-        e = cudaStreamIsCapturing(stream, &cap);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
-        e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(opts->split_done_event), stream,
-                                     cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0u);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord(split_done_event)");
-    }
-
+    int rc2 = record_split_done(opts, stream);
+    if (rc2) return rc2;
     if (pl.combine_ctas > 0) {
         apd::CombineParams cp;
         cp.cum = sp.cum_out;
@@ -638,24 +825,7 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
         cp.ksplit = pl.ksplit;
         cp.num_workers = pl.workers;
         cp.groups = pl.groups;
-        const bool per_unit = combine_per_unit(s, pl);
-        const int cw = per_unit ? (s.rows_max >= 8 ? 8 : 4) : combine_warps(s, pl);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = per_unit ? dim3(static_cast<unsigned>(pl.combine_ctas))
-                               : dim3(static_cast<unsigned>(s.units), static_cast<unsigned>(s.rows_max));
-        cfg.blockDim = dim3(32 * cw);
-        cfg.dynamicSmemBytes = per_unit ? 4u * (s.B + 1) : 0u;
-        cfg.stream = stream;
-        cfg.attrs = pdl_attr;
-        cfg.numAttrs = (use_pdl && !(opts && opts->split_done_event)) ? 1 : 0;
-        if (per_unit)
-            e = cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 8>, cp)
-                        : cudaLaunchKernelEx(&cfg, apd::combine_unit_kernel<D, 4>, cp);
-        else
-            e = cw == 16 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 16>, cp)
-                : cw == 8 ? cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 8>, cp)
-                          : cudaLaunchKernelEx(&cfg, apd::combine_kernel<D, 4>, cp);
-        if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+        return launch_combine<D>(s, pl, cp, stream, opts);
     }
     return APD_OK;
 }
@@ -1088,10 +1258,11 @@ int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl,
-                   options ? options->host_seq_lens : nullptr, static_cast<int64_t>(V.MP) * V.P);
-    if (rc) return rc;
     const SplitTestHooks h = hooks ? *hooks : SplitTestHooks();
+    rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl,
+                   options ? options->host_seq_lens : nullptr, static_cast<int64_t>(V.MP) * V.P,
+                   /*allow_tc=*/!h.skip_release);
+    if (rc) return rc;
     // the release self-test needs the shared K/V ring (auto splits, more than 16 q heads per kv head)
     if (h.skip_release && !pl.share) return APD_ERR_ARGUMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -1,0 +1,585 @@
+// apd_decode_tc.cuh -- decode attention for kv heads shared by 32 query heads, on the
+// sm_100a fifth-generation tensor cores (tcgen05 + TMEM).
+//
+// Same operation as the split kernel (AstrAI commit log of csrc/kernels/attn_paged_decode.cu:
+// one query token per sequence, paged bf16 K/V, split-KV partials o_part / ml_part merged by
+// one combine kernel); this is the design for kv heads whose query heads fill a tensor-core
+// tile.  With g = 32 query heads per kv head, every K/V tile meets 32 query rows, twice the
+// 16 of one mma.sync head block; here the tile goes to the tensor core once for all of them.
+//
+//  - A CTA owns one split of one (sequence b, kv head) unit: a contiguous run of the
+//    sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it (so its partials
+//    go to the same slots and the same combine kernel merges them).
+//  - Tokens are the M side of both products, query heads the N side:
+//      S^T[t][h]  = sum_d K[t][d] Q[h][d]        (M = 128 tokens, N = 32 heads, K = D;
+//                                                 A = the K tile, B = Q, both K-major)
+//      O^T[d][h] += sum_t V[t][d] P^T[t][h]      (M = D, N = 32 heads, K = 128 tokens;
+//                                                 A = the V tile read MN-major, B = P^T
+//                                                 MN-major: P stored [token][head])
+//    so the staged K and V tiles are used exactly as the TMA lands them and no query row of
+//    the MMA is padding.
+//  - Warps 4 and 6 (producers) resolve each tile's four pages and issue the TMA loads of
+//    its K boxes (warp 4) and V boxes (warp 6) into two rings, each refilled as soon as its
+//    own stage is free: a K stage right after its S^T product, a V stage after its P V.
+//    Warp 5 lane 0 issues the MMAs, each product as soon as its operands are ready (S^T_j
+//    does not wait for P_{j-1} V_{j-1}, nor that for the next K tile), and commits them to
+//    the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T and two
+//    P buffers let the softmax of tile j + 1 run while P_j V_j is on the tensor core.
+//  - Warps 0-3 (softmax): TMEM lane t is token t of the tile, so thread t reads its token's
+//    32 scores with one tcgen05.ld and owns that token's exponentials.  The reference
+//    maximum of each head is shared by all tokens; it moves only when some score exceeds it
+//    by more than 2^8 (one OR-vote per tile over a named barrier; the head maxima are then
+//    reduced across the 128 threads, O^T and the running sums rescaled).  Each thread keeps
+//    its own running sums of the bf16 weights it wrote; they are added across the threads
+//    once, at the end.
+//
+// Every mbarrier wait is bounded.  A wait that runs out raises a shared abort flag that every
+// role polls; the softmax warps decide to stop only through the result of a barrier
+// reduction, so they leave together, and all warps meet before the TMEM columns are freed.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "apd_kernels.cuh"
+#include "apd_prefill_tc.cuh"
+#include "apd_ptx.cuh"
+
+namespace apd {
+
+struct McParams {
+    const __nv_bfloat16* q;  // [B][Hq][D], head dim contiguous
+    int64_t q_sb, q_sh;
+    const int32_t* page_table;  // NULL: contiguous KV, sequence b is page b of P tokens
+    int64_t pt_s0, pt_s1;
+    const int32_t* seq_lens;
+    __nv_bfloat16* out;
+    int64_t out_sb, out_sh;
+    float* o_part;   // [slots][rows_max][D]
+    float* ml_part;  // [slots][rows_max][2]
+    uint32_t* flags;
+    int32_t B, Hkv, g, HB, rows_max, P, NP, MP;
+    int32_t ksplit;  // splits per (sequence, kv head)
+    float scale_log2;
+};
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D, each operand
+// K-major or MN-major (bits 15 and 16), shape M x N.
+constexpr uint32_t mc_idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// OR of `pred` over the `nthreads` threads that meet at named barrier `id` (every warp of
+// them arrives with all its lanes).
+__device__ __forceinline__ bool bar_any(int id, int nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0u;
+}
+__device__ __forceinline__ void bar_named(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Reduce-scatter of NH = 32 values over the warp: afterwards v[0] of lane t holds the
+// reduction over the 32 lanes of value t (recursive halving: at offset o, a lane keeps the
+// upper half of its values when bit o of its lane index is set and takes the partner's
+// copy of them).
+template <bool kMax>
+__device__ __forceinline__ void warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+            const float keep = upper ? v[i + o] : v[i];
+            const float send = upper ? v[i] : v[i + o];
+            const float got = __shfl_xor_sync(0xffffffffu, send, o);
+            v[i] = kMax ? fmaxf(keep, got) : keep + got;
+        }
+    }
+}
+
+template <int D, int NH>
+struct McShape {
+    static_assert(D == 128 && NH == 32, "the tensor-core decode kernel serves D = 128, 32 heads per kv head");
+    static constexpr int kTok = 128;  // tokens per tile (TMEM lanes of S^T)
+    static constexpr int kStages = 3;
+    static constexpr int kSoftmaxWarps = 4;
+    static constexpr int kProducerWarp = 4, kMmaWarp = 5, kVProducerWarp = 6;
+    static constexpr int kThreads = 32 * 7;
+    static constexpr uint32_t kQBytes = NH * D * 2;
+    static constexpr uint32_t kKVBytes = kTok * D * 2;  // one K (or V) tile
+    static constexpr uint32_t kPBytes = kTok * NH * 2;
+    static constexpr uint32_t kQOff = 0;
+    static constexpr uint32_t kKOff = kQBytes;
+    static constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;
+    static constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;
+    static constexpr uint32_t kTileBytes = kPOff + 2 * kPBytes;  // two P buffers
+    // 2 KB header (mbarriers, TMEM address, abort flag, the per-warp head maxima and sums),
+    // up to 1 KB to reach 1024-byte alignment, then the tiles
+    static constexpr uint32_t kHeaderBytes = 2048;
+    static constexpr uint32_t kRedOff = 512;
+    static constexpr uint32_t kSmemBytes = kHeaderBytes + 1024 + kTileBytes;
+    static constexpr uint32_t kTmemCols = 128;
+    static constexpr uint32_t kColS = 0;        // two S^T buffers: columns [0, 2 NH)
+    static constexpr uint32_t kColO = 2 * NH;   // O^T: columns [2 NH, 3 NH)
+    static_assert(kColO + NH <= kTmemCols, "TMEM columns");
+    static_assert(kRedOff + 2 * 4 * NH * 4 <= kHeaderBytes, "header");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the TMEM columns are always free");
+};
+
+template <int D, int NH>
+__global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
+    decode_mq_tc_kernel(const __grid_constant__ McParams p, const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap) {
+    using T = McShape<D, NH>;
+    using O = OperandGeom<D>;   // K, V and Q staging: D/64 blocks of [rows][64]
+    using PG = OperandGeom<NH>; // P staging: [tokens][NH] rows of 2 NH bytes
+    constexpr int TK = T::kTok, ST = T::kStages;
+    constexpr uint32_t kIdescQK = mc_idesc(TK, NH, false, false);
+    constexpr uint32_t kIdescPV = mc_idesc(D, NH, true, true);
+    // mbarriers; S, P and PVDone come in pairs, one per S / P buffer (tile parity)
+    constexpr int kQFull = 0, kKFull = 1, kKEmpty = 1 + ST, kVFull = 1 + 2 * ST, kVEmpty = 1 + 3 * ST;
+    constexpr int kSFull = 1 + 4 * ST, kSFree = 3 + 4 * ST, kPFull = 5 + 4 * ST, kPVDone = 7 + 4 * ST;
+    constexpr int kDrain = 9 + 4 * ST, kBars = 10 + 4 * ST;
+    constexpr int kSoftThreads = 32 * T::kSoftmaxWarps;
+    constexpr int kBarId = 1;  // named barrier of the softmax warps
+    static_assert(8 * kBars + 8 <= static_cast<int>(T::kRedOff), "barrier area");
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t bar0 = smem_u32(smem);
+    auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * kBars);
+    volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + 8 * kBars + 4);
+    float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [4 warps][NH] head maxima
+    float* s_sum = s_red + 4 * NH;                                // [4 warps][NH] head sums
+    const uint32_t tb = (bar0 + T::kHeaderBytes + 1023u) & ~1023u;
+    const uint32_t q_s = tb + T::kQOff, p_s = tb + T::kPOff;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- work item: split `split` of unit (sequence b, kv head kvh)
+    const int nsplit = p.ksplit;
+    const int u2 = blockIdx.x / nsplit;
+    const int split = blockIdx.x - u2 * nsplit;
+    const int b = u2 / p.Hkv;
+    const int kvh = u2 - b * p.Hkv;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(kQFull), kSoftThreads);
+#pragma unroll
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(bar(kKFull + s), 1);
+            mbar_init(bar(kKEmpty + s), 1);
+            mbar_init(bar(kVFull + s), 1);
+            mbar_init(bar(kVEmpty + s), 1);
+        }
+        mbar_init(bar(kSFull), 1);
+        mbar_init(bar(kSFull + 1), 1);
+        mbar_init(bar(kSFree), kSoftThreads);
+        mbar_init(bar(kSFree + 1), kSoftThreads);
+        mbar_init(bar(kPFull), kSoftThreads);
+        mbar_init(bar(kPFull + 1), kSoftThreads);
+        mbar_init(bar(kPVDone), 1);
+        mbar_init(bar(kPVDone + 1), 1);
+        mbar_init(bar(kDrain), 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+    __syncthreads();
+    // Launched with programmatic dependent launch: nothing above reads global memory.
+    pdl_wait_prior_grid();
+    pdl_launch_dependents();
+
+    // ---- the sequence's length and this split's boxes [c0, c1) of 32 tokens, cut as the
+    // fixed-split plan cuts them (the combine recomputes the same cut)
+    const bool contig = p.page_table == nullptr;
+    const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
+    int L = __ldcg(p.seq_lens + b);
+    if (L < 0 || L > cap) {
+        if (threadIdx.x == 0 && split == 0) atomicOr(p.flags, L < 0 ? kFlagLenNegative : kFlagLenClamped);
+        L = L < 0 ? 0 : static_cast<int>(cap);
+    }
+    const int n32 = (L + kTile - 1) / kTile;
+    int c0 = 0, c1 = 0, nk = 1;
+    if (n32 > 0) {
+        const int S = max(1, min(nsplit, n32));
+        const int c = (n32 + S - 1) / S;
+        c0 = min(split * c, n32);
+        c1 = min(c0 + c, n32);
+        nk = (n32 + c - 1) / c;
+    }
+    if (c0 >= c1) {
+        // an empty split writes nothing; split 0 of an empty sequence writes its zero rows
+        if (split == 0) {
+            for (int i = threadIdx.x; i < p.g * (D / 8); i += blockDim.x) {
+                const int h = i / (D / 8), ch = i - h * (D / 8);
+                *reinterpret_cast<uint4*>(p.out + b * p.out_sb + (kvh * p.g + h) * p.out_sh + 8 * ch) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        return;  // the whole CTA, before any TMEM allocation or copy
+    }
+    const int tok0 = kTile * c0;
+    const int tok1 = min(kTile * c1, L);
+    const int ntiles = (tok1 - tok0 + TK - 1) / TK;
+
+    if (warp == T::kMmaWarp) {
+        tc_alloc(smem_u32(tmem_slot), T::kTmemCols);
+        tc_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    bool ok = true;
+    if (warp == T::kProducerWarp || warp == T::kVProducerWarp) {
+        // ================= producers: TMA loads of the K tiles (warp 4) or the V tiles
+        // (warp 6), four 32-token boxes each
+        const int kv = warp == T::kVProducerWarp ? 1 : 0;
+        const CUtensorMap* map = kv ? &vmap : &kmap;
+        const int full0 = kv ? kVFull : kKFull, empty0 = kv ? kVEmpty : kKEmpty;
+        const uint32_t ring = tb + (kv ? T::kVOff : T::kKOff);
+        const uint64_t pol = l2_policy_evict_first();  // every K/V byte is read once
+        constexpr int kBoxes = TK / kTile;               // 4
+        constexpr int kTB = 32 / kBoxes;                 // tiles whose pages one warp-wide load resolves
+        int32_t pg = 0;
+        int issued = 0;
+        for (int j = 0; j < ntiles; ++j) {
+            if (j % kTB == 0) {
+                const int jj = j + lane / kBoxes;
+                const int t = tok0 + jj * TK + (lane % kBoxes) * kTile;
+                pg = 0;
+                if (jj < ntiles && t < tok1)
+                    pg = contig ? b
+                                : __ldcg(p.page_table + static_cast<int64_t>(b) * p.pt_s0 +
+                                         static_cast<int64_t>(t / p.P) * p.pt_s1);
+            }
+            int32_t pages[kBoxes];
+#pragma unroll
+            for (int q = 0; q < kBoxes; ++q) pages[q] = __shfl_sync(0xffffffffu, pg, (j % kTB) * kBoxes + q);
+            const int ng = min(kBoxes, (tok1 - (tok0 + j * TK) + kTile - 1) / kTile);  // boxes holding tokens
+            const uint32_t bytes = static_cast<uint32_t>(ng) * kTile * D * 2u;
+            const int stage = j % ST;
+            if (j >= ST) ok = tc_wait(bar(empty0 + stage), static_cast<uint32_t>((j / ST) - 1) & 1u, abort_flag, p.flags);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (lane == 0) {
+                const uint32_t full = bar(full0 + stage);
+                const uint32_t dst = ring + static_cast<uint32_t>(stage) * T::kKVBytes;
+                mbar_arrive_expect_tx(full, bytes);
+#pragma unroll
+                for (int q = 0; q < kBoxes; ++q) {
+                    if (q >= ng) break;
+                    const int page = pages[q];
+                    if (kv == 0 && (page < 0 || page >= p.NP)) atomicOr(p.flags, kFlagPageOOR);
+                    const int tok = tok0 + j * TK + kTile * q;
+                    const int slot = contig ? tok : tok % p.P;
+#pragma unroll
+                    for (int c = 0; c < O::kBlk; ++c)
+                        tma_load_5d(dst + static_cast<uint32_t>(c * TK * O::kRowBytes + q * kTile * O::kRowBytes), map,
+                                    full, 0, kvh, slot, page, c, pol);
+                }
+            }
+            __syncwarp();
+            issued = j + 1;
+        }
+        if (!ok && lane == 0) {
+            // wait (bounded) for the copies still in flight before the CTA can exit
+            for (int s = 0; s < ST; ++s) {
+                if (issued > s) {
+                    const int jl = s + ST * ((issued - 1 - s) / ST);
+                    mbar_wait_bounded(bar(full0 + s), static_cast<uint32_t>(jl / ST) & 1u, kWaitTimeoutNs);
+                }
+            }
+        }
+    } else if (warp == T::kMmaWarp) {
+        // ================= MMA issuer (one thread): S^T_jq as soon as K_jq is staged and its
+        // S buffer is free, P_jp V_jp as soon as P_jp and V_jp are; tcgen05 operations of one
+        // thread run in issue order, so the P V products accumulate into O^T in tile order
+        if (lane == 0) {
+            bool issued = false;
+            ok = tc_wait(bar(kQFull), 0, abort_flag, p.flags);
+            int jq = 0, jp = 0;
+            uint64_t t_idle = global_timer_ns();
+            for (uint32_t it = 1; ok && jp < ntiles; ++it) {
+                bool progress = false;
+                if (jq < ntiles && mbar_try_wait(bar(kKFull + jq % ST), static_cast<uint32_t>(jq / ST) & 1u) &&
+                    (jq < 2 || mbar_try_wait(bar(kSFree + (jq & 1)), static_cast<uint32_t>((jq - 2) >> 1) & 1u))) {
+                    tc_fence_after();
+                    // S^T_jq = K_jq Q^T, K = D in steps of 16
+                    const uint32_t kb = tb + T::kKOff + static_cast<uint32_t>(jq % ST) * T::kKVBytes;
+                    const uint32_t d = tmem + T::kColS + static_cast<uint32_t>((jq & 1) * NH);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        tc_mma_bf16(d, O::desc(kb + O::kstep(k, TK), 16), O::desc(q_s + O::kstep(k, NH), 16),
+                                    kIdescQK, k > 0 ? 1u : 0u);
+                    tc_commit(bar(kSFull + (jq & 1)));
+                    tc_commit(bar(kKEmpty + jq % ST));
+                    issued = true;
+                    progress = true;
+                    ++jq;
+                }
+                if (jp < jq && mbar_try_wait(bar(kPFull + (jp & 1)), static_cast<uint32_t>(jp >> 1) & 1u) &&
+                    mbar_try_wait(bar(kVFull + jp % ST), static_cast<uint32_t>(jp / ST) & 1u)) {
+                    tc_fence_after();
+                    // O^T += V_jp^T P_jp^T, K = TK tokens in steps of 16
+                    const uint32_t vb = tb + T::kVOff + static_cast<uint32_t>(jp % ST) * T::kKVBytes;
+                    const uint32_t pb = p_s + static_cast<uint32_t>((jp & 1) * T::kPBytes);
+#pragma unroll
+                    for (int k = 0; k < TK / 16; ++k)
+                        tc_mma_bf16(tmem + T::kColO,
+                                    O::desc(vb + static_cast<uint32_t>(k * 16 * O::kRowBytes), TK * O::kRowBytes),
+                                    PG::desc(pb + static_cast<uint32_t>(k * 16 * PG::kRowBytes), TK * PG::kRowBytes),
+                                    kIdescPV, (jp > 0 || k > 0) ? 1u : 0u);
+                    tc_commit(bar(kPVDone + (jp & 1)));
+                    tc_commit(bar(kVEmpty + jp % ST));
+                    progress = true;
+                    ++jp;
+                }
+                if (progress) {
+                    it = 0;
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if ((it & 63u) == 0) {
+                    const uint64_t now = global_timer_ns();
+                    if (it == 64) t_idle = now;  // the first check of an idle stretch starts its clock
+                    else if (now - t_idle > kWaitTimeoutNs) {
+                        *abort_flag = 1u;
+                        atomicOr(p.flags, kFlagTimeout);
+                        ok = false;
+                    }
+                }
+            }
+            if (!ok && issued) {
+                // wait (bounded) for the MMAs still in flight
+                tc_commit(bar(kDrain));
+                mbar_wait_bounded(bar(kDrain), 0, kWaitTimeoutNs);
+            }
+        }
+    } else {
+        // ================= softmax warps: thread r owns token r of each tile (TMEM lane r)
+        const int r = 32 * warp + lane;
+        const uint32_t t_lane = static_cast<uint32_t>(32 * warp) << 16;
+        // Q rows kvh * g + h (h < NH) in the K-major B layout [D/64][NH][64]
+        for (int idx = threadIdx.x; idx < NH * (D / 8); idx += kSoftThreads) {
+            const int h = idx / (D / 8), ch = idx - h * (D / 8);
+            const uint4 v =
+                __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + (kvh * p.g + h) * p.q_sh + 8 * ch));
+            st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (NH * O::kRowBytes) + h * O::kRowBytes +
+                                                     (O::swz(h, ch % O::kChunks) << 4)),
+                         v.x, v.y, v.z, v.w);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(kQFull));
+
+        float m[NH];  // reference maximum of each head (log2 domain), the same in every thread
+        float l[NH];  // this thread's sums of the bf16 weights, relative to m
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+        }
+        bool wok = true, stopped = false;
+        for (int j = 0; j < ntiles; ++j) {
+            const int sb = j & 1;
+            float x[NH];
+            wok = warp_wait(bar(kSFull + sb), static_cast<uint32_t>(j >> 1) & 1u, kWaitTimeoutNs, abort_flag,
+                            p.flags);
+            if (wok) {
+                uint32_t sr[NH];
+                tc_fence_after();
+                tc_ld32(tmem + t_lane + T::kColS + static_cast<uint32_t>(sb * NH), sr);
+                tc_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
+                const bool valid = tok0 + j * TK + r < tok1;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+            } else {
+#pragma unroll
+                for (int h = 0; h < NH; ++h) x[h] = -INFINITY;
+            }
+            bool need = false;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) need |= x[h] > m[h] + 8.f;
+            // one vote per tile: a new reference for some head, or some warp gave up
+            const bool gave_up = !wok || *abort_flag != 0u;
+            if (bar_any(kBarId, kSoftThreads, need || gave_up)) {
+                if (bar_any(kBarId, kSoftThreads, gave_up)) {
+                    stopped = true;
+                    break;
+                }
+                // ---- new reference: the tile's maximum of each head over the 128 tokens
+                float v[NH];
+#pragma unroll
+                for (int h = 0; h < NH; ++h) v[h] = x[h];
+                warp_reduce_scatter32<true>(v, lane);
+                s_red[warp * NH + lane] = v[0];
+                bar_named(kBarId, kSoftThreads);
+                float alpha[NH];
+#pragma unroll
+                for (int h = 0; h < NH; h += 4) {
+                    float4 a = *reinterpret_cast<const float4*>(s_red + h);
+#pragma unroll
+                    for (int w = 1; w < 4; ++w) {
+                        const float4 c = *reinterpret_cast<const float4*>(s_red + w * NH + h);
+                        a.x = fmaxf(a.x, c.x);
+                        a.y = fmaxf(a.y, c.y);
+                        a.z = fmaxf(a.z, c.z);
+                        a.w = fmaxf(a.w, c.w);
+                    }
+                    const float tm[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float mn = fmaxf(m[h + e], tm[e]);
+                        // 1 for a head whose maximum did not move; 0 while m is -inf
+                        alpha[h + e] = (mn == m[h + e]) ? 1.f : ex2_approx(m[h + e] - mn);
+                        m[h + e] = mn;
+                        l[h + e] *= alpha[h + e];
+                    }
+                }
+                if (j > 0) {
+                    // O^T holds P V of the earlier tiles: rescale this thread's row (head dim
+                    // r) column by column, once the last P V has landed (in issue order, so
+                    // every earlier one has too)
+                    wok = warp_wait(bar(kPVDone + ((j - 1) & 1)), static_cast<uint32_t>((j - 1) >> 1) & 1u,
+                                    kWaitTimeoutNs, abort_flag, p.flags);
+                    if (wok) {
+                        tc_fence_after();
+                        uint32_t o[NH];
+                        tc_ld32(tmem + t_lane + T::kColO, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                        tc_st32(tmem + t_lane + T::kColO, o);
+                        tc_wait_st();
+                    }
+                }
+            }
+            if (!wok) continue;  // gave up in this tile: the next vote stops every warp
+
+            // ---- P = 2^(x - m) as bf16 pairs, and the sums of exactly those weights
+            uint32_t pw[NH / 2];
+#pragma unroll
+            for (int i = 0; i < NH / 2; ++i) {
+                const float p0 = ex2_approx(x[2 * i] - m[2 * i]);
+                const float p1 = ex2_approx(x[2 * i + 1] - m[2 * i + 1]);
+                pw[i] = pack_bf16x2(p0, p1);
+                l[2 * i] += bf16_lo(pw[i]);
+                l[2 * i + 1] += bf16_hi(pw[i]);
+            }
+            // ---- P buffer j & 1 is free once P_{j-2} V_{j-2} has completed
+            if (j > 1) {
+                wok = warp_wait(bar(kPVDone + (j & 1)), static_cast<uint32_t>((j - 2) >> 1) & 1u, kWaitTimeoutNs,
+                                abort_flag, p.flags);
+                if (!wok) continue;
+                tc_fence_after();
+            }
+            // row r of P^T ([token][head], 2 NH bytes, swizzled as the MN-major B layout)
+            const uint32_t pb = p_s + static_cast<uint32_t>((j & 1) * T::kPBytes);
+#pragma unroll
+            for (int c = 0; c < NH / 8; ++c)
+                st_shared_v4(pb + static_cast<uint32_t>(r * PG::kRowBytes + (PG::swz(r, c) << 4)), pw[4 * c],
+                             pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            // ---- last tile: V rows past the split's last token hold anything (NaN included,
+            // or nothing loaded): zero them before they meet a zero weight
+            if (j == ntiles - 1 && tok0 + j * TK + TK > tok1) {
+                const int stage = j % ST;
+                wok = warp_wait(bar(kVFull + stage), static_cast<uint32_t>(j / ST) & 1u, kWaitTimeoutNs, abort_flag,
+                                p.flags);
+                if (!wok) continue;
+                zero_v_rows<D, TK>(tb + T::kVOff + static_cast<uint32_t>(stage) * T::kKVBytes, tok1 - (tok0 + j * TK),
+                                   threadIdx.x, kSoftThreads);
+            }
+            fence_proxy_async_smem();  // P (and the zeroed V rows) -> tensor core
+            tc_fence_before();
+            mbar_arrive(bar(kPFull + (j & 1)));
+        }
+        // ---- epilogue: the heads' sums over the CTA's tokens, then out (or the partial)
+        if (!stopped && wok)
+            wok = warp_wait(bar(kPVDone + ((ntiles - 1) & 1)), static_cast<uint32_t>((ntiles - 1) >> 1) & 1u,
+                            kWaitTimeoutNs, abort_flag, p.flags);
+        float v[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) v[h] = l[h];
+        warp_reduce_scatter32<false>(v, lane);
+        s_sum[warp * NH + lane] = v[0];
+        const bool gave_up = stopped || !wok || *abort_flag != 0u;
+        if (!bar_any(kBarId, kSoftThreads, gave_up)) {
+            tc_fence_after();
+            uint32_t o[NH];
+            tc_ld32(tmem + t_lane + T::kColO, o);
+            tc_wait_ld();
+            float lt[NH];
+#pragma unroll
+            for (int h = 0; h < NH; h += 4) {
+                float4 a = *reinterpret_cast<const float4*>(s_sum + h);
+#pragma unroll
+                for (int w = 1; w < 4; ++w) {
+                    const float4 c = *reinterpret_cast<const float4*>(s_sum + w * NH + h);
+                    a.x += c.x;
+                    a.y += c.y;
+                    a.z += c.z;
+                    a.w += c.w;
+                }
+                lt[h] = a.x;
+                lt[h + 1] = a.y;
+                lt[h + 2] = a.z;
+                lt[h + 3] = a.w;
+            }
+            const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
+            if (nk == 1) {
+                // the only non-empty split: normalised rows straight to out
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                        __float2bfloat16_rn(__uint_as_float(o[h]) / lt[h]);
+            } else {
+                // the partial of this split, for each head block of 16 heads: slot
+                // ((b * Hkv + kvh) * HB + hb) * ksplit + split, row h - 16 hb
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const int64_t slot =
+                        (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
+                    p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[h]);
+                }
+                if (warp == 0) {
+                    float mm = 0.f, ll = 0.f;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        if (lane == h) {
+                            mm = m[h];
+                            ll = lt[h];
+                        }
+                    }
+                    const int64_t slot = (static_cast<int64_t>(u2) * p.HB + lane / kMaxRows) * p.ksplit + split;
+                    *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + lane % kMaxRows) * 2) =
+                        make_float2(mm, ll);
+                }
+            }
+        }
+    }
+    // ---- all roles meet before the TMEM columns are freed
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == T::kMmaWarp) {
+        tc_fence_after();
+        tc_dealloc(tmem, T::kTmemCols);
+    }
+}
+
+}  // namespace apd

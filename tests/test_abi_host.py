@@ -202,7 +202,7 @@ def test_workspace_size_invalid_is_zero():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,D", [(16, 32, 8, 128), (2, 32, 8, 128), (128, 64, 8, 128), (4, 8, 8, 32),
-                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 128), (8, 96, 2, 128)])
+                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 64), (8, 96, 2, 128)])
 def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
     g = Hq // Hkv
@@ -245,7 +245,7 @@ def _smem(B, D, rows, warps, stages, hb, shared):
     return -(-meta // 16) * 16 + 1024 + rings
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 64, 2, 128), (4, 96, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 128, 2, 128), (4, 96, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
                                         (4, 64, 2, 256), (4, 32, 8, 128), (4, 16, 1, 64)])
 def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     # balanced mode with g > 16: the head blocks of a kv head share one K/V ring, so the
@@ -274,6 +274,37 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     if local.mode == 2:
         assert local.shared_kv_ring == 0 and local.stages == stages
         assert local.smem_bytes == _unit_smem(D, rows, local.warps_per_cta, stages)
+
+
+_MC_SMEM = 2048 + 1024 + 32 * 128 * 2 + 3 * 2 * 128 * 128 * 2 + 2 * 128 * 32 * 2
+
+
+@pytest.mark.parametrize("B,Hkv,sm", [(16, 2, 148), (1, 1, 148), (4, 8, 148), (200, 1, 148), (3, 2, 132), (16, 2, 8)])
+def test_plan_tensor_core_multi_query(B, Hkv, sm):
+    """32 q heads per kv head at D = 128: the tensor-core multi-query kernel, one CTA per
+    split of each (sequence, kv head), 7 warps (4 softmax, 2 producers, 1 MMA issuer), 3
+    K and 3 V stages of 128 tokens, Q and two P buffers in shared memory.  Auto splits
+    spread the units over 7/8 of the SMs; the partials take the fixed-split slots of both
+    head blocks, and the combine runs only when a unit is split."""
+    Hq, D = 32 * Hkv, 128
+    units = B * Hkv * 2
+    pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
+    k = max(1, sm * 7 // 8 // (B * Hkv))
+    assert pl.mode == 3 and pl.shared_kv_ring == 0
+    assert pl.grid_ctas == B * Hkv * k and pl.num_workers == pl.grid_ctas
+    assert pl.warps_per_cta == 7 and pl.stages == 3 and pl.smem_bytes == _MC_SMEM <= 232448
+    assert pl.rows_per_unit == 16 and pl.head_blocks == 2
+    assert pl.partial_slots == (units * k if k > 1 else 0)
+    assert pl.combine_ctas == (0 if k == 1 else min(units, 4 * sm) if k <= 4 else units * 16)
+    for S in (1, 3, 8):
+        f = apd.query_plan(B, Hq, Hkv, D, S, sm_count=sm)
+        assert f.mode == 3 and f.grid_ctas == B * Hkv * S and f.partial_slots == (units * S if S > 1 else 0)
+    # a workspace that holds fewer partials caps the splits; one with none gives one split
+    small = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm, workspace_bytes=4096)
+    assert small.mode == 3 and small.grid_ctas == B * Hkv and small.partial_slots == 0
+    # other head dims and group sizes keep the mma.sync kernels
+    for Hq2, D2 in ((32 * Hkv, 64), (48 * Hkv, 128), (16 * Hkv, 128)):
+        assert apd.query_plan(B, Hq2, Hkv, D2, 0, sm_count=sm).mode != 3
 
 
 def _unit_smem(D, rows, warps, stages):
@@ -351,7 +382,8 @@ def cta_local_expected(B, Hq, Hkv, D, lens, cap, sm=148):
     (16, 32, 8, 32, [16384] * 16, 16384, 2),           # other head dims at 128 equal units
     (16, 32, 8, 64, [8192] * 16, 8192, 2),
     (16, 32, 8, 256, [2048] * 16, 2048, 2),
-    (16, 64, 2, 128, [16384] * 16, 16384, 0),          # two head blocks per kv head: balanced, shared ring
+    (16, 64, 2, 128, [16384] * 16, 16384, 3),          # 32 q heads per kv head at D = 128: tensor cores
+    (16, 64, 2, 64, [16384] * 16, 16384, 0),           # two head blocks per kv head: balanced, shared ring
 ])
 def test_plan_cta_local_from_host_lengths(B, Hq, Hkv, D, lens, cap, want):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=lens, max_seq_len=cap)
@@ -619,6 +651,13 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
     elif pl.mode == 1:
         assert splits > 0 and pl.grid_ctas == units * splits
         assert pl.num_workers == pl.grid_ctas * pl.warps_per_cta
+    elif pl.mode == 3:
+        # the tensor-core multi-query kernel: one CTA per split of each (sequence, kv head)
+        assert D == 128 and g == 32 and pl.grid_ctas % (B * Hkv) == 0
+        k = pl.grid_ctas // (B * Hkv)
+        assert k == splits or splits == 0
+        assert pl.partial_slots == (units * k if k > 1 else 0)
+        assert (pl.combine_ctas == 0) == (k == 1)
     else:
         assert splits == 0 and pl.mode == 2 and units <= sm
         assert pl.grid_ctas == units and pl.combine_ctas == 0 and pl.partial_slots == 0
