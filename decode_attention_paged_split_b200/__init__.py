@@ -82,7 +82,7 @@ class _Plan(ctypes.Structure):
         ("partial_slots", ctypes.c_int64),
         ("workspace_bytes", ctypes.c_int64),
         ("shared_kv_ring", ctypes.c_int32),
-        ("reserved0", ctypes.c_int32),
+        ("cluster_size", ctypes.c_int32),
     ]
 
 
@@ -497,6 +497,7 @@ class Plan:
     partial_slots: int
     workspace_bytes: int
     shared_kv_ring: int  # 1: a kv head's head-block warps read one K/V ring (balanced, g > 16)
+    cluster_size: int = 0  # mode 3: CTAs per cluster that merge a unit's splits in the kernel
 
 
 def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,

@@ -152,6 +152,7 @@ int64_t slots_fitting(const Shape& s, size_t bytes) {
 
 struct Plan {
     int mode, ksplit, workers, groups, ctas, warps, stages, combine_ctas;
+    int cluster = 0;  // mode 3: CTAs per cluster (the splits of a unit, merged over DSMEM), or 0
     bool share;  // balanced mode, g > 16: a kv head's HB warps share one K/V ring
     size_t smem;
     int64_t slots;
@@ -236,7 +237,18 @@ int64_t mq_tc_auto_splits(const Shape& s, int sm_count, size_t ws_bytes, int64_t
     return k;
 }
 
-void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, Plan* pl);
+void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan* pl);
+
+// Whether the splits of every unit can be one cluster of `k` CTAs that the device runs all
+// at once (cluster_caps[k]: clusters of k of the kernel's CTAs that fit the device at the
+// same time; without it, every k SMs are assumed to hold one).  Then the splits merge over
+// DSMEM in the kernel: measured on B200 (gqa32), the separate combine kernel costs 4.5 of
+// 49.6 us per call.
+int mq_tc_cluster(const Shape& s, int64_t k, int sm_count, const int* cluster_caps) {
+    if (k < 2 || k > apd::kMcMaxCluster) return 0;
+    const int64_t cap = cluster_caps ? cluster_caps[k] : sm_count / k;
+    return static_cast<int64_t>(s.B) * s.Hkv <= cap ? static_cast<int>(k) : 0;
+}
 
 // Warps of a combine CTA: enough for one batch of kCombineBatch partial slots per warp,
 // 4 to 16.  A unit has about groups / B partials in the balanced mode (each sequence's
@@ -267,20 +279,24 @@ int64_t combine_unit_ctas(const Shape& s, int sm_count) {
     return std::min<int64_t>(s.units, static_cast<int64_t>(sm_count) * kCombineUnitCtasPerSm);
 }
 
-void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, Plan* pl) {
+void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan* pl) {
     pl->mode = 3;
+    pl->cluster = cluster;
     pl->share = false;
     pl->ksplit = static_cast<int>(ksplit);
     pl->groups = 0;
     pl->warps = kMcWarps;
-    pl->stages = McShape128::kStages;
+    pl->stages = McShape128::kVStages;
     pl->smem = McShape128::kSmemBytes;
     pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * ksplit);
     pl->workers = pl->ctas;
+    // the partial slots are reserved whether or not the merge runs over DSMEM, so that the
+    // workspace a split count needs does not depend on the device's cluster placement
     pl->slots = ksplit >= 2 ? s.units * ksplit : 0;
-    pl->combine_ctas = ksplit >= 2 ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
-                                                                              : s.units * s.rows_max)
-                                   : 0;
+    pl->combine_ctas = ksplit >= 2 && cluster == 0
+                           ? static_cast<int>(combine_per_unit(s, *pl) ? combine_unit_ctas(s, sm_count)
+                                                                      : s.units * s.rows_max)
+                           : 0;
 }
 
 // tiles_bound: an upper bound on the number of tiles (host-known), or -1.
@@ -289,12 +305,13 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, Plan* pl) {
 // allow_tc: the tensor-core multi-query plan may be chosen (the shared-ring self-test turns
 // it off to reach the shared ring).
 int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl,
-              const int32_t* host_lens = nullptr, int64_t len_cap = 0, bool allow_tc = true) {
+              const int32_t* host_lens = nullptr, int64_t len_cap = 0, bool allow_tc = true,
+              const int* cluster_caps = nullptr) {
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
     if (allow_tc && mq_tc_eligible(s)) {
         const int64_t k = num_splits > 0 ? num_splits : mq_tc_auto_splits(s, sm_count, ws_bytes, tiles_bound);
         if (static_cast<int64_t>(s.B) * s.Hkv * k > INT32_MAX / 64) return APD_ERR_TOO_LARGE;
-        mq_tc_plan(s, k, sm_count, pl);
+        mq_tc_plan(s, k, sm_count, mq_tc_cluster(s, k, sm_count, cluster_caps), pl);
         pl->ws_needed = ws_bytes_for(s, pl->slots);
         if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
         return APD_OK;
@@ -374,6 +391,8 @@ struct DeviceState {
     int sm_count = 0;
     bool smem_attr_set[16] = {};  // head dim x {split kernel, with shared rings, unit kernel, unit kernel with fixed splits}
     bool mq_tc_attr_set = false;
+    bool mq_caps_init = false;
+    int mq_cluster_caps[apd::kMcMaxCluster + 1] = {};  // co-resident clusters of k tensor-core decode CTAs
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -396,6 +415,38 @@ int device_state(DeviceState** out) {
     }
     *out = &d;
     return APD_OK;
+}
+
+// Clusters of k tensor-core decode CTAs that the device runs at the same time, k = 2..8
+// (cudaOccupancyMaxActiveClusters; 0 where the query fails).  Computed once per device.
+const int* mq_cluster_caps(DeviceState* d) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (d->mq_caps_init) return d->mq_cluster_caps;
+    auto kern = apd::decode_mq_tc_kernel<128, 32>;
+    if (!d->mq_tc_attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(McShape128::kSmemBytes)) == cudaSuccess)
+            d->mq_tc_attr_set = true;
+    }
+    for (int c = 2; c <= apd::kMcMaxCluster; ++c) {
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = static_cast<unsigned>(c);
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(c * d->sm_count));
+        cfg.blockDim = dim3(static_cast<unsigned>(McShape128::kThreads));
+        cfg.dynamicSmemBytes = McShape128::kSmemBytes;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (!d->mq_tc_attr_set || cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        d->mq_cluster_caps[c] = n;
+    }
+    cudaGetLastError();  // a failed query only turns the cluster merge off
+    d->mq_caps_init = true;
+    return d->mq_cluster_caps;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -663,19 +714,31 @@ int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, c
     mp.NP = V.NP;
     mp.MP = V.MP;
     mp.ksplit = pl.ksplit;
+    mp.cluster = pl.cluster > 0 ? 1 : 0;
     mp.scale_log2 = scale * 1.4426950408889634f;
 
     const bool use_pdl = !(opts && opts->disable_pdl);
-    cudaLaunchAttribute pdl_attr[1];
-    pdl_attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl_attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attrs[2];
+    int na = 0;
+    if (pl.cluster > 0) {
+        attrs[na].id = cudaLaunchAttributeClusterDimension;
+        attrs[na].val.clusterDim.x = static_cast<unsigned>(pl.cluster);
+        attrs[na].val.clusterDim.y = 1;
+        attrs[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (use_pdl) {
+        attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attrs[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(pl.ctas));
     cfg.blockDim = dim3(static_cast<unsigned>(McShape128::kThreads));
     cfg.dynamicSmemBytes = McShape128::kSmemBytes;
     cfg.stream = stream;
-    cfg.attrs = pdl_attr;
-    cfg.numAttrs = use_pdl ? 1 : 0;
+    cfg.attrs = attrs;
+    cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mp, kmap, vmap);
     if (e != cudaSuccess) return cuda_fail(e, "decode_mq_tc_kernel launch");
     rc = record_split_done(opts, stream);
@@ -1261,7 +1324,7 @@ int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor
     const SplitTestHooks h = hooks ? *hooks : SplitTestHooks();
     rc = make_plan(V.s, num_splits, dev->sm_count, workspace_bytes, tiles_bound, &pl,
                    options ? options->host_seq_lens : nullptr, static_cast<int64_t>(V.MP) * V.P,
-                   /*allow_tc=*/!h.skip_release);
+                   /*allow_tc=*/!h.skip_release, mq_cluster_caps(dev));
     if (rc) return rc;
     // the release self-test needs the shared K/V ring (auto splits, more than 16 q heads per kv head)
     if (h.skip_release && !pl.share) return APD_ERR_ARGUMENT;
@@ -1330,7 +1393,8 @@ int apd_attn_paged_decode_noalloc(const apd_tensor* q, const apd_tensor* k_cache
     DeviceState* dev = nullptr;
     rc = device_state(&dev);
     if (rc) return rc;
-    rc = make_plan(V.s, num_splits, dev->sm_count, kScratch, tiles_bound, &pl);
+    rc = make_plan(V.s, num_splits, dev->sm_count, kScratch, tiles_bound, &pl, nullptr, 0, true,
+                   mq_cluster_caps(dev));
     if (rc == APD_ERR_WORKSPACE) return APD_ERR_SCRATCH_LIMIT;
     if (rc) return rc;
     void* scratch = nullptr;
@@ -1527,14 +1591,16 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
     Shape s;
     int rc = make_shape(batch, num_q_heads, num_kv_heads, head_dim, &s);
     if (rc) return rc;
+    const int* caps = nullptr;
     if (sm_count <= 0) {
         DeviceState* dev = nullptr;
         rc = device_state(&dev);
         if (rc) return rc;
         sm_count = dev->sm_count;
+        caps = mq_cluster_caps(dev);
     }
     Plan pl;
-    rc = make_plan(s, num_splits, sm_count, workspace_bytes, -1, &pl, host_seq_lens, max_seq_len);
+    rc = make_plan(s, num_splits, sm_count, workspace_bytes, -1, &pl, host_seq_lens, max_seq_len, true, caps);
     if (rc) return rc;
     plan->mode = pl.mode;
     plan->num_workers = pl.workers;
@@ -1548,7 +1614,7 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
     plan->partial_slots = pl.slots;
     plan->workspace_bytes = static_cast<int64_t>(pl.ws_needed);
     plan->shared_kv_ring = pl.share ? 1 : 0;
-    plan->reserved0 = 0;
+    plan->cluster_size = pl.cluster;
     return APD_OK;
 }
 

@@ -8,8 +8,12 @@
 // 16 of one mma.sync head block; here the tile goes to the tensor core once for all of them.
 //
 //  - A CTA owns one split of one (sequence b, kv head) unit: a contiguous run of the
-//    sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it (so its partials
-//    go to the same slots and the same combine kernel merges them).
+//    sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it.  With at most
+//    8 splits per unit the splits of a unit form one thread-block cluster: each split leaves
+//    its unnormalised part in its own shared memory, and split c then merges heads c, c + nk,
+//    c + 2 nk, ... of all nk parts over distributed shared memory and writes them out (one
+//    kernel, no partials in global memory).  With more splits the parts go to the
+//    fixed-split slots of o_part / ml_part and the combine kernel merges them.
 //  - Tokens are the M side of both products, query heads the N side:
 //      S^T[t][h]  = sum_d K[t][d] Q[h][d]        (M = 128 tokens, N = 32 heads, K = D;
 //                                                 A = the K tile, B = Q, both K-major)
@@ -60,7 +64,8 @@ struct McParams {
     float* ml_part;  // [slots][rows_max][2]
     uint32_t* flags;
     int32_t B, Hkv, g, HB, rows_max, P, NP, MP;
-    int32_t ksplit;  // splits per (sequence, kv head)
+    int32_t ksplit;   // splits per (sequence, kv head)
+    int32_t cluster;  // 1: the ksplit CTAs of a unit are one cluster and merge over DSMEM
     float scale_log2;
 };
 
@@ -108,11 +113,75 @@ __device__ __forceinline__ void warp_reduce_scatter32(float (&v)[32], int lane) 
     }
 }
 
+// ---- thread-block cluster pieces: the cluster barrier, DSMEM addressing and loads, and
+// mbarrier arrivals and waits across the cluster
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// The address in CTA `rank` of the cluster of this CTA's shared-memory address `addr`.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// The generic address of the same variable in CTA `rank` of the cluster (plain loads
+// through it read that CTA's shared memory).
+template <typename T>
+__device__ __forceinline__ const T* dsmem_ptr(const T* p, uint32_t rank) {
+    uint64_t r;
+    asm("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+    return reinterpret_cast<const T*>(r);
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// Arrive on an mbarrier of another CTA of the cluster (address from dsmem_addr), releasing
+// this thread's earlier writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// warp_wait with acquire at cluster scope (for arrivals from other CTAs of the cluster).
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                                  volatile uint32_t* abort_word, uint32_t* flags) {
+    bool done = mbar_try_wait_acq_cluster(bar, parity);
+    if (__all_sync(0xffffffffu, done)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (!done) done = mbar_try_wait_acq_cluster(bar, parity);
+        if (__all_sync(0xffffffffu, done)) return true;
+        if ((it & 15u) == 0) {
+            int give_up = 0;
+            if ((threadIdx.x & 31) == 0 && global_timer_ns() - t0 > timeout_ns) give_up = 1;
+            give_up = __shfl_sync(0xffffffffu, give_up, 0);
+            if (give_up) {
+                if ((threadIdx.x & 31) == 0) {
+                    *abort_word = 1u;
+                    atomicOr(flags, kFlagTimeout);
+                }
+                return false;
+            }
+        }
+    }
+}
+
+constexpr int kMcMaxCluster = 8;  // splits per unit merged over DSMEM (the portable cluster size)
+
 template <int D, int NH>
 struct McShape {
     static_assert(D == 128 && NH == 32, "the tensor-core decode kernel serves D = 128, 32 heads per kv head");
     static constexpr int kTok = 128;  // tokens per tile (TMEM lanes of S^T)
-    static constexpr int kStages = 3;
+    static constexpr int kKStages = 3, kVStages = 3;  // K and V ring depths
     static constexpr int kSoftmaxWarps = 4;
     static constexpr int kProducerWarp = 4, kMmaWarp = 5, kVProducerWarp = 6;
     static constexpr int kThreads = 32 * 7;
@@ -121,8 +190,8 @@ struct McShape {
     static constexpr uint32_t kPBytes = kTok * NH * 2;
     static constexpr uint32_t kQOff = 0;
     static constexpr uint32_t kKOff = kQBytes;
-    static constexpr uint32_t kVOff = kKOff + kStages * kKVBytes;
-    static constexpr uint32_t kPOff = kVOff + kStages * kKVBytes;
+    static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
+    static constexpr uint32_t kPOff = kVOff + kVStages * kKVBytes;
     static constexpr uint32_t kTileBytes = kPOff + 2 * kPBytes;  // two P buffers
     // 2 KB header (mbarriers, TMEM address, abort flag, the per-warp head maxima and sums),
     // up to 1 KB to reach 1024-byte alignment, then the tiles
@@ -133,6 +202,10 @@ struct McShape {
     static constexpr uint32_t kColS = 0;        // two S^T buffers: columns [0, 2 NH)
     static constexpr uint32_t kColO = 2 * NH;   // O^T: columns [2 NH, 3 NH)
     static_assert(kColO + NH <= kTmemCols, "TMEM columns");
+    // cluster merge: a split's part [NH][D] fp32 + [NH][2] in its K ring, its merge weights
+    // [kMcMaxCluster + 1][NH] in its Q buffer
+    static_assert(NH * D * 4 + NH * 8 <= kKStages * kKVBytes, "part in the K ring");
+    static_assert((kMcMaxCluster + 1) * NH * 4 <= kQBytes, "merge weights in the Q buffer");
     static_assert(kRedOff + 2 * 4 * NH * 4 <= kHeaderBytes, "header");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the TMEM columns are always free");
@@ -145,13 +218,13 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     using T = McShape<D, NH>;
     using O = OperandGeom<D>;   // K, V and Q staging: D/64 blocks of [rows][64]
     using PG = OperandGeom<NH>; // P staging: [tokens][NH] rows of 2 NH bytes
-    constexpr int TK = T::kTok, ST = T::kStages;
+    constexpr int TK = T::kTok, KST = T::kKStages, VST = T::kVStages;
     constexpr uint32_t kIdescQK = mc_idesc(TK, NH, false, false);
     constexpr uint32_t kIdescPV = mc_idesc(D, NH, true, true);
     // mbarriers; S, P and PVDone come in pairs, one per S / P buffer (tile parity)
-    constexpr int kQFull = 0, kKFull = 1, kKEmpty = 1 + ST, kVFull = 1 + 2 * ST, kVEmpty = 1 + 3 * ST;
-    constexpr int kSFull = 1 + 4 * ST, kSFree = 3 + 4 * ST, kPFull = 5 + 4 * ST, kPVDone = 7 + 4 * ST;
-    constexpr int kDrain = 9 + 4 * ST, kBars = 10 + 4 * ST;
+    constexpr int kQFull = 0, kKFull = 1, kKEmpty = 1 + KST, kVFull = 1 + 2 * KST, kVEmpty = 1 + 2 * KST + VST;
+    constexpr int kSFull = 1 + 2 * (KST + VST), kSFree = kSFull + 2, kPFull = kSFull + 4, kPVDone = kSFull + 6;
+    constexpr int kDrain = kSFull + 8, kParts = kSFull + 9, kBars = kSFull + 10;
     constexpr int kSoftThreads = 32 * T::kSoftmaxWarps;
     constexpr int kBarId = 1;  // named barrier of the softmax warps
     static_assert(8 * kBars + 8 <= static_cast<int>(T::kRedOff), "barrier area");
@@ -177,9 +250,12 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(kQFull), kSoftThreads);
 #pragma unroll
-        for (int s = 0; s < ST; ++s) {
+        for (int s = 0; s < KST; ++s) {
             mbar_init(bar(kKFull + s), 1);
             mbar_init(bar(kKEmpty + s), 1);
+        }
+#pragma unroll
+        for (int s = 0; s < VST; ++s) {
             mbar_init(bar(kVFull + s), 1);
             mbar_init(bar(kVEmpty + s), 1);
         }
@@ -192,12 +268,15 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         mbar_init(bar(kPVDone), 1);
         mbar_init(bar(kPVDone + 1), 1);
         mbar_init(bar(kDrain), 1);
+        mbar_init(bar(kParts), static_cast<uint32_t>(max(1, nsplit - 1)));  // one arrival per other split
         *abort_flag = 0u;
         fence_mbar_init();
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
     __syncthreads();
+    // cluster phase 0 (waited before any DSMEM access): every CTA has initialised its mbarriers
+    if (p.cluster) cluster_arrive_relaxed();
     // Launched with programmatic dependent launch: nothing above reads global memory.
     pdl_wait_prior_grid();
     pdl_launch_dependents();
@@ -229,6 +308,12 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                     make_uint4(0u, 0u, 0u, 0u);
             }
         }
+        if (p.cluster) {
+            cluster_wait();
+            if (threadIdx.x < nsplit && threadIdx.x != split) mbar_arrive_remote(dsmem_addr(bar(kParts), threadIdx.x));
+            cluster_arrive();
+            cluster_wait();
+        }
         return;  // the whole CTA, before any TMEM allocation or copy
     }
     const int tok0 = kTile * c0;
@@ -245,12 +330,14 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     bool ok = true;
+    bool cluster_waited = false;  // this thread has waited for cluster phase 0
     if (warp == T::kProducerWarp || warp == T::kVProducerWarp) {
         // ================= producers: TMA loads of the K tiles (warp 4) or the V tiles
         // (warp 6), four 32-token boxes each
         const int kv = warp == T::kVProducerWarp ? 1 : 0;
         const CUtensorMap* map = kv ? &vmap : &kmap;
         const int full0 = kv ? kVFull : kKFull, empty0 = kv ? kVEmpty : kKEmpty;
+        const int ST = kv ? VST : KST;
         const uint32_t ring = tb + (kv ? T::kVOff : T::kKOff);
         const uint64_t pol = l2_policy_evict_first();  // every K/V byte is read once
         constexpr int kBoxes = TK / kTile;               // 4
@@ -316,27 +403,27 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             uint64_t t_idle = global_timer_ns();
             for (uint32_t it = 1; ok && jp < ntiles; ++it) {
                 bool progress = false;
-                if (jq < ntiles && mbar_try_wait(bar(kKFull + jq % ST), static_cast<uint32_t>(jq / ST) & 1u) &&
+                if (jq < ntiles && mbar_try_wait(bar(kKFull + jq % KST), static_cast<uint32_t>(jq / KST) & 1u) &&
                     (jq < 2 || mbar_try_wait(bar(kSFree + (jq & 1)), static_cast<uint32_t>((jq - 2) >> 1) & 1u))) {
                     tc_fence_after();
                     // S^T_jq = K_jq Q^T, K = D in steps of 16
-                    const uint32_t kb = tb + T::kKOff + static_cast<uint32_t>(jq % ST) * T::kKVBytes;
+                    const uint32_t kb = tb + T::kKOff + static_cast<uint32_t>(jq % KST) * T::kKVBytes;
                     const uint32_t d = tmem + T::kColS + static_cast<uint32_t>((jq & 1) * NH);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
                         tc_mma_bf16(d, O::desc(kb + O::kstep(k, TK), 16), O::desc(q_s + O::kstep(k, NH), 16),
                                     kIdescQK, k > 0 ? 1u : 0u);
                     tc_commit(bar(kSFull + (jq & 1)));
-                    tc_commit(bar(kKEmpty + jq % ST));
+                    tc_commit(bar(kKEmpty + jq % KST));
                     issued = true;
                     progress = true;
                     ++jq;
                 }
                 if (jp < jq && mbar_try_wait(bar(kPFull + (jp & 1)), static_cast<uint32_t>(jp >> 1) & 1u) &&
-                    mbar_try_wait(bar(kVFull + jp % ST), static_cast<uint32_t>(jp / ST) & 1u)) {
+                    mbar_try_wait(bar(kVFull + jp % VST), static_cast<uint32_t>(jp / VST) & 1u)) {
                     tc_fence_after();
                     // O^T += V_jp^T P_jp^T, K = TK tokens in steps of 16
-                    const uint32_t vb = tb + T::kVOff + static_cast<uint32_t>(jp % ST) * T::kKVBytes;
+                    const uint32_t vb = tb + T::kVOff + static_cast<uint32_t>(jp % VST) * T::kKVBytes;
                     const uint32_t pb = p_s + static_cast<uint32_t>((jp & 1) * T::kPBytes);
 #pragma unroll
                     for (int k = 0; k < TK / 16; ++k)
@@ -345,7 +432,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                                     PG::desc(pb + static_cast<uint32_t>(k * 16 * PG::kRowBytes), TK * PG::kRowBytes),
                                     kIdescPV, (jp > 0 || k > 0) ? 1u : 0u);
                     tc_commit(bar(kPVDone + (jp & 1)));
-                    tc_commit(bar(kVEmpty + jp % ST));
+                    tc_commit(bar(kVEmpty + jp % VST));
                     progress = true;
                     ++jp;
                 }
@@ -497,8 +584,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             // ---- last tile: V rows past the split's last token hold anything (NaN included,
             // or nothing loaded): zero them before they meet a zero weight
             if (j == ntiles - 1 && tok0 + j * TK + TK > tok1) {
-                const int stage = j % ST;
-                wok = warp_wait(bar(kVFull + stage), static_cast<uint32_t>(j / ST) & 1u, kWaitTimeoutNs, abort_flag,
+                const int stage = j % VST;
+                wok = warp_wait(bar(kVFull + stage), static_cast<uint32_t>(j / VST) & 1u, kWaitTimeoutNs, abort_flag,
                                 p.flags);
                 if (!wok) continue;
                 zero_v_rows<D, TK>(tb + T::kVOff + static_cast<uint32_t>(stage) * T::kKVBytes, tok1 - (tok0 + j * TK),
@@ -518,12 +605,18 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         warp_reduce_scatter32<false>(v, lane);
         s_sum[warp * NH + lane] = v[0];
         const bool gave_up = stopped || !wok || *abort_flag != 0u;
-        if (!bar_any(kBarId, kSoftThreads, gave_up)) {
+        const bool any_gave_up = bar_any(kBarId, kSoftThreads, gave_up);
+        uint32_t o[NH];
+        float lt[NH];
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            o[h] = 0u;
+            lt[h] = 0.f;
+        }
+        if (!any_gave_up) {
             tc_fence_after();
-            uint32_t o[NH];
             tc_ld32(tmem + t_lane + T::kColO, o);
             tc_wait_ld();
-            float lt[NH];
 #pragma unroll
             for (int h = 0; h < NH; h += 4) {
                 float4 a = *reinterpret_cast<const float4*>(s_sum + h);
@@ -540,20 +633,23 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                 lt[h + 2] = a.z;
                 lt[h + 3] = a.w;
             }
-            const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
-            if (nk == 1) {
-                // the only non-empty split: normalised rows straight to out
+        }
+        const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
+        if (nk == 1) {
+            // the only non-empty split: normalised rows straight to out
+            if (!any_gave_up) {
 #pragma unroll
                 for (int h = 0; h < NH; ++h)
                     p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
                         __float2bfloat16_rn(__uint_as_float(o[h]) / lt[h]);
-            } else {
+            }
+        } else if (!p.cluster) {
+            if (!any_gave_up) {
                 // the partial of this split, for each head block of 16 heads: slot
                 // ((b * Hkv + kvh) * HB + hb) * ksplit + split, row h - 16 hb
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
-                    const int64_t slot =
-                        (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
+                    const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
                     p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[h]);
                 }
                 if (warp == 0) {
@@ -570,6 +666,84 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                         make_float2(mm, ll);
                 }
             }
+        } else {
+            // ---- merge over the cluster.  Part of split s: [NH][D] fp32 (O^T unnormalised),
+            // then [NH] (m, l) pairs, at the start of its K ring (free once its last S^T is done)
+            float* const part_p = reinterpret_cast<float*>(smem + (tb + T::kKOff - bar0));
+            cluster_wait();  // phase 0: every CTA of the cluster has its mbarriers initialised
+            cluster_waited = true;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) part_p[h * D + dd] = __uint_as_float(o[h]);
+            if (warp == 0) {
+                float mm = 0.f, ll = 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    if (lane == h) {
+                        mm = m[h];
+                        ll = lt[h];
+                    }
+                }
+                part_p[NH * D + 2 * lane] = mm;
+                part_p[NH * D + 2 * lane + 1] = ll;
+            }
+            fence_acq_rel_cluster();
+            bar_named(kBarId, kSoftThreads);
+            // tell every other CTA of the cluster that this part is ready
+            if (threadIdx.x < nsplit && threadIdx.x != split) mbar_arrive_remote(dsmem_addr(bar(kParts), threadIdx.x));
+            // this split merges heads h = split + j nk (j < nh) of every part:
+            // w_s = 2^(m_s - M) over the non-empty parts, out = sum_s w_s O_s / sum_s w_s l_s
+            const int nh = (NH - split + nk - 1) / nk;
+            const bool pok = warp_wait_cluster(bar(kParts), 0u, kWaitTimeoutNs, abort_flag, p.flags);
+            float* const wts = reinterpret_cast<float*>(smem + (q_s - bar0));  // [kMcMaxCluster + 1][NH]
+            if (warp == 0 && pok && lane < nh) {
+                const int h = split + lane * nk;
+                float ms[kMcMaxCluster], ls[kMcMaxCluster];
+#pragma unroll
+                for (int s = 0; s < kMcMaxCluster; ++s) {
+                    ms[s] = -INFINITY;
+                    ls[s] = 0.f;
+                    if (s < nk) {
+                        const float* q = dsmem_ptr(part_p + NH * D + 2 * h, static_cast<uint32_t>(s));
+                        ms[s] = q[0];
+                        ls[s] = q[1];
+                    }
+                }
+                float M = -INFINITY;
+#pragma unroll
+                for (int s = 0; s < kMcMaxCluster; ++s)
+                    if (ls[s] > 0.f) M = fmaxf(M, ms[s]);
+                float den = 0.f;
+#pragma unroll
+                for (int s = 0; s < kMcMaxCluster; ++s) {
+                    const float w = ls[s] > 0.f ? exp2f(ms[s] - M) : 0.f;
+                    wts[s * NH + lane] = w;
+                    den += w * ls[s];
+                }
+                wts[kMcMaxCluster * NH + lane] = den > 0.f ? 1.f / den : 0.f;
+            }
+            if (!bar_any(kBarId, kSoftThreads, !pok || any_gave_up)) {
+                constexpr int kMaxH = NH / 2;  // heads per split when nk = 2
+                float acc[kMaxH];
+#pragma unroll
+                for (int j = 0; j < kMaxH; ++j) acc[j] = 0.f;
+#pragma unroll
+                for (int s = 0; s < kMcMaxCluster; ++s) {
+                    if (s < nk) {  // the loads of all parts can be in flight together
+                        const float* src = dsmem_ptr(part_p + dd, static_cast<uint32_t>(s));
+                        float v[kMaxH];
+#pragma unroll
+                        for (int j = 0; j < kMaxH; ++j) v[j] = j < nh ? src[(split + j * nk) * D] : 0.f;
+#pragma unroll
+                        for (int j = 0; j < kMaxH; ++j) acc[j] += wts[s * NH + j] * v[j];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kMaxH; ++j) {
+                    if (j < nh)
+                        p.out[b * p.out_sb + (kvh * p.g + split + j * nk) * p.out_sh + dd] =
+                            __float2bfloat16_rn(acc[j] * wts[kMcMaxCluster * NH + j]);
+                }
+            }
         }
     }
     // ---- all roles meet before the TMEM columns are freed
@@ -579,6 +753,12 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     if (warp == T::kMmaWarp) {
         tc_fence_after();
         tc_dealloc(tmem, T::kTmemCols);
+    }
+    if (p.cluster) {
+        if (!cluster_waited) cluster_wait();  // phase 0, for the warps that did not merge
+        // phase 1: no CTA of the cluster leaves while split 0 may still read its part
+        cluster_arrive();
+        cluster_wait();
     }
 }
 

@@ -437,7 +437,10 @@ typedef struct apd_plan {
     int32_t mode;              /* 0 = balanced (num_splits == 0), 1 = fixed splits,
                                   2 = one CTA per unit, parts merged in shared memory
                                   (num_splits == 0 with host lengths, see
-                                  apd_launch_options.host_seq_lens) */
+                                  apd_launch_options.host_seq_lens),
+                                  3 = tensor-core multi-query kernel (32 q heads per
+                                  kv head at head_dim 128, any num_splits): one CTA per
+                                  split of each (sequence, kv head)             */
     int32_t num_workers;       /* warps that each own a run of tiles             */
     int32_t grid_ctas;         /* CTAs of the split kernel                       */
     int32_t warps_per_cta;
@@ -454,7 +457,9 @@ typedef struct apd_plan {
                                   from one ring that the first of them fills, so
                                   each K/V tile leaves HBM once (warps_per_cta is
                                   then a multiple of head_blocks)               */
-    int32_t reserved0;
+    int32_t cluster_size;      /* mode 3: the splits of a unit run as one thread-block
+                                  cluster of this many CTAs and merge in the kernel
+                                  (no combine kernel); 0 otherwise               */
 } apd_plan;
 
 /* apd_query_plan -- fills *plan.  workspace_bytes: the size that will be passed

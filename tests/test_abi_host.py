@@ -284,8 +284,10 @@ def test_plan_tensor_core_multi_query(B, Hkv, sm):
     """32 q heads per kv head at D = 128: the tensor-core multi-query kernel, one CTA per
     split of each (sequence, kv head), 7 warps (4 softmax, 2 producers, 1 MMA issuer), 3
     K and 3 V stages of 128 tokens, Q and two P buffers in shared memory.  Auto splits
-    spread the units over 7/8 of the SMs; the partials take the fixed-split slots of both
-    head blocks, and the combine runs only when a unit is split."""
+    spread the units over 7/8 of the SMs.  A unit's splits (up to 8) that the device can run
+    as one cluster merge over DSMEM in the kernel; otherwise their partials take the
+    fixed-split slots of both head blocks and the combine kernel merges them.  The slots are
+    reserved either way."""
     Hq, D = 32 * Hkv, 128
     units = B * Hkv * 2
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
@@ -295,10 +297,15 @@ def test_plan_tensor_core_multi_query(B, Hkv, sm):
     assert pl.warps_per_cta == 7 and pl.stages == 3 and pl.smem_bytes == _MC_SMEM <= 232448
     assert pl.rows_per_unit == 16 and pl.head_blocks == 2
     assert pl.partial_slots == (units * k if k > 1 else 0)
-    assert pl.combine_ctas == (0 if k == 1 else min(units, 4 * sm) if k <= 4 else units * 16)
-    for S in (1, 3, 8):
+    # up to 8 splits of a unit that fit the device as one cluster each merge in the kernel
+    # (with an SM count given, every k SMs are taken to hold a cluster of k)
+    cl = k if 2 <= k <= 8 and B * Hkv <= sm // k else 0
+    assert pl.cluster_size == cl
+    assert pl.combine_ctas == (0 if k == 1 or cl else min(units, 4 * sm) if k <= 4 else units * 16)
+    for S in (1, 3, 8, 12):
         f = apd.query_plan(B, Hq, Hkv, D, S, sm_count=sm)
         assert f.mode == 3 and f.grid_ctas == B * Hkv * S and f.partial_slots == (units * S if S > 1 else 0)
+        assert f.cluster_size == (S if 2 <= S <= 8 and B * Hkv <= sm // S else 0)
     # a workspace that holds fewer partials caps the splits; one with none gives one split
     small = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm, workspace_bytes=4096)
     assert small.mode == 3 and small.grid_ctas == B * Hkv and small.partial_slots == 0
@@ -657,7 +664,8 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
         k = pl.grid_ctas // (B * Hkv)
         assert k == splits or splits == 0
         assert pl.partial_slots == (units * k if k > 1 else 0)
-        assert (pl.combine_ctas == 0) == (k == 1)
+        assert pl.cluster_size in (0, k) and (pl.cluster_size == 0 or 2 <= k <= 8)
+        assert (pl.combine_ctas == 0) == (k == 1 or pl.cluster_size > 0)
     else:
         assert splits == 0 and pl.mode == 2 and units <= sm
         assert pl.grid_ctas == units and pl.combine_ctas == 0 and pl.partial_slots == 0
