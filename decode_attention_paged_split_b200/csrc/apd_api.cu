@@ -209,14 +209,22 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
     return 32 * longest <= 33 * share + 32 * (1024 / s.D);
 }
 
-// Tensor-core multi-query plan (mode 3, decode_mq_tc_kernel): kv heads with 32 query heads
-// at D = 128.  One CTA per split of each (sequence, kv head); its 128-token tiles meet all
-// 32 query heads in one tcgen05 MMA, where the split kernel needs two head blocks.  The
-// partials take the fixed-split slots (the head blocks' rows of each split), so the combine
-// is the fixed-split one.
-using McShape128 = apd::McShape<128, 32>;
-constexpr int kMcWarps = McShape128::kThreads / 32;
-bool mq_tc_eligible(const Shape& s) { return s.D == 128 && s.g == 32; }
+// Tensor-core multi-query plan (mode 3, decode_mq_tc_kernel): kv heads with 17 to 64 query
+// heads at D = 128.  One CTA per split of each (sequence, kv head); its 128-token tiles meet
+// all the query heads (padded to NH = 32 or 64) in one tcgen05 MMA, where the split kernel
+// needs a head block of 16 per warp.  The partials take the fixed-split slots (the head
+// blocks' rows of each split), so the combine is the fixed-split one.
+template <int NH>
+using McShapeT = apd::McShape<128, NH>;
+constexpr int kMcWarps = McShapeT<32>::kThreads / 32;
+static_assert(McShapeT<64>::kThreads == McShapeT<32>::kThreads, "one warp layout");
+// NH of the tensor-core kernel for this shape, or 0 when the shape does not take it
+int mq_tc_heads(const Shape& s) { return s.D == 128 && s.g > 16 && s.g <= 64 ? (s.g <= 32 ? 32 : 64) : 0; }
+bool mq_tc_eligible(const Shape& s) { return mq_tc_heads(s) > 0; }
+// Co-resident clusters of k tensor-core decode CTAs, per NH (index 0: 32 heads, 1: 64).
+struct McCaps {
+    int c[2][apd::kMcMaxCluster + 1];
+};
 
 // Splits per unit with automatic splitting: the (sequence, kv head) units spread over 7/8
 // of the SMs (the rate at which D = 128 streams best, as in the balanced plan), at most one
@@ -244,9 +252,9 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
 // same time; without it, every k SMs are assumed to hold one).  Then the splits merge over
 // DSMEM in the kernel: measured on B200 (gqa32), the separate combine kernel costs 4.5 of
 // 49.6 us per call.
-int mq_tc_cluster(const Shape& s, int64_t k, int sm_count, const int* cluster_caps) {
+int mq_tc_cluster(const Shape& s, int64_t k, int sm_count, const McCaps* caps) {
     if (k < 2 || k > apd::kMcMaxCluster) return 0;
-    const int64_t cap = cluster_caps ? cluster_caps[k] : sm_count / k;
+    const int64_t cap = caps ? caps->c[mq_tc_heads(s) == 64 ? 1 : 0][k] : sm_count / k;
     return static_cast<int64_t>(s.B) * s.Hkv <= cap ? static_cast<int>(k) : 0;
 }
 
@@ -286,8 +294,9 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
     pl->ksplit = static_cast<int>(ksplit);
     pl->groups = 0;
     pl->warps = kMcWarps;
-    pl->stages = McShape128::kVStages;
-    pl->smem = McShape128::kSmemBytes;
+    const bool h64 = mq_tc_heads(s) == 64;
+    pl->stages = h64 ? McShapeT<64>::kVStages : McShapeT<32>::kVStages;
+    pl->smem = h64 ? McShapeT<64>::kSmemBytes : McShapeT<32>::kSmemBytes;
     pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * ksplit);
     pl->workers = pl->ctas;
     // the partial slots are reserved whether or not the merge runs over DSMEM, so that the
@@ -306,7 +315,7 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
 // it off to reach the shared ring).
 int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int64_t tiles_bound, Plan* pl,
               const int32_t* host_lens = nullptr, int64_t len_cap = 0, bool allow_tc = true,
-              const int* cluster_caps = nullptr) {
+              const McCaps* cluster_caps = nullptr) {
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
     if (allow_tc && mq_tc_eligible(s)) {
         const int64_t k = num_splits > 0 ? num_splits : mq_tc_auto_splits(s, sm_count, ws_bytes, tiles_bound);
@@ -390,9 +399,9 @@ struct DeviceState {
     bool init = false;
     int sm_count = 0;
     bool smem_attr_set[16] = {};  // head dim x {split kernel, with shared rings, unit kernel, unit kernel with fixed splits}
-    bool mq_tc_attr_set = false;
+    bool mq_tc_attr_set[2] = {false, false};  // NH = 32, 64
     bool mq_caps_init = false;
-    int mq_cluster_caps[apd::kMcMaxCluster + 1] = {};  // co-resident clusters of k tensor-core decode CTAs
+    McCaps mq_caps = {};  // co-resident clusters of k tensor-core decode CTAs
     bool gemv_attr_set = false;
     bool prefill_attr_set[4] = {false, false, false, false};
     bool prefill_tc_attr_set[4] = {false, false, false, false};
@@ -419,14 +428,14 @@ int device_state(DeviceState** out) {
 
 // Clusters of k tensor-core decode CTAs that the device runs at the same time, k = 2..8
 // (cudaOccupancyMaxActiveClusters; 0 where the query fails).  Computed once per device.
-const int* mq_cluster_caps(DeviceState* d) {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (d->mq_caps_init) return d->mq_cluster_caps;
-    auto kern = apd::decode_mq_tc_kernel<128, 32>;
-    if (!d->mq_tc_attr_set) {
+template <int NH>
+void mq_query_caps(DeviceState* d, int* caps) {
+    auto kern = apd::decode_mq_tc_kernel<128, NH>;
+    const int hi = NH == 64 ? 1 : 0;
+    if (!d->mq_tc_attr_set[hi]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(McShape128::kSmemBytes)) == cudaSuccess)
-            d->mq_tc_attr_set = true;
+                                 static_cast<int>(McShapeT<NH>::kSmemBytes)) == cudaSuccess)
+            d->mq_tc_attr_set[hi] = true;
     }
     for (int c = 2; c <= apd::kMcMaxCluster; ++c) {
         cudaLaunchAttribute attr;
@@ -436,17 +445,24 @@ const int* mq_cluster_caps(DeviceState* d) {
         attr.val.clusterDim.z = 1;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(c * d->sm_count));
-        cfg.blockDim = dim3(static_cast<unsigned>(McShape128::kThreads));
-        cfg.dynamicSmemBytes = McShape128::kSmemBytes;
+        cfg.blockDim = dim3(static_cast<unsigned>(McShapeT<NH>::kThreads));
+        cfg.dynamicSmemBytes = McShapeT<NH>::kSmemBytes;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (!d->mq_tc_attr_set || cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
-        d->mq_cluster_caps[c] = n;
+        if (!d->mq_tc_attr_set[hi] || cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        caps[c] = n;
     }
-    cudaGetLastError();  // a failed query only turns the cluster merge off
-    d->mq_caps_init = true;
-    return d->mq_cluster_caps;
+}
+const McCaps* mq_cluster_caps(DeviceState* d) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d->mq_caps_init) {
+        mq_query_caps<32>(d, d->mq_caps.c[0]);
+        mq_query_caps<64>(d, d->mq_caps.c[1]);
+        cudaGetLastError();  // a failed query only turns the cluster merge off
+        d->mq_caps_init = true;
+    }
+    return &d->mq_caps;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -666,19 +682,23 @@ int launch_combine(const Shape& s, const Plan& pl, const apd::CombineParams& cp,
     return APD_OK;
 }
 
-// Mode 3: the tensor-core multi-query kernel, then the combine when units are split.
+// Mode 3: the tensor-core multi-query kernel, then the combine when units are split and
+// not merged in a cluster.
+template <int NH>
 int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
                  const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
                  void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
     constexpr int D = 128;
-    auto kern = apd::decode_mq_tc_kernel<D, 32>;
+    using McShape128 = McShapeT<NH>;
+    auto kern = apd::decode_mq_tc_kernel<D, NH>;
     {
         std::lock_guard<std::mutex> lock(g_mu);
-        if (!dev->mq_tc_attr_set) {
+        const int hi = NH == 64 ? 1 : 0;
+        if (!dev->mq_tc_attr_set[hi]) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  static_cast<int>(McShape128::kSmemBytes));
             if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode_mq_tc_kernel)");
-            dev->mq_tc_attr_set = true;
+            dev->mq_tc_attr_set[hi] = true;
         }
     }
     // K/V boxes of one 64-element block each, so that a tile's rows of one block are
@@ -774,7 +794,10 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
            void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts,
            const SplitTestHooks& hooks = SplitTestHooks()) {
     if constexpr (D == 128) {
-        if (pl.mode == 3) return launch_mq_tc(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts);
+        if (pl.mode == 3)
+            return mq_tc_heads(V.s) == 64
+                       ? launch_mq_tc<64>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts)
+                       : launch_mq_tc<32>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts);
     }
     if (pl.mode == 3) return APD_ERR_ARGUMENT;  // planned only for D = 128
     constexpr int kStagesD = kStages<D>;
@@ -1591,7 +1614,7 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
     Shape s;
     int rc = make_shape(batch, num_q_heads, num_kv_heads, head_dim, &s);
     if (rc) return rc;
-    const int* caps = nullptr;
+    const McCaps* caps = nullptr;
     if (sm_count <= 0) {
         DeviceState* dev = nullptr;
         rc = device_state(&dev);

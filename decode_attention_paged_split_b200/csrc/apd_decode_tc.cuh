@@ -179,9 +179,12 @@ constexpr int kMcMaxCluster = 8;  // splits per unit merged over DSMEM (the port
 
 template <int D, int NH>
 struct McShape {
-    static_assert(D == 128 && NH == 32, "the tensor-core decode kernel serves D = 128, 32 heads per kv head");
+    static_assert(D == 128 && (NH == 32 || NH == 64), "the tensor-core decode kernel: D = 128, 32 or 64 heads");
     static constexpr int kTok = 128;  // tokens per tile (TMEM lanes of S^T)
-    static constexpr int kKStages = 3, kVStages = 3;  // K and V ring depths
+    static constexpr int kChunks = NH / 32;  // softmax passes of 32 heads
+    // K and V ring depths: 3 + 3 stages of 32 KB; at 64 heads the Q and P buffers double and
+    // the K ring keeps 2 (gqa48: K 2 + V 3 measured 61.6-62.1 us, K 3 + V 2 62.4-62.7 us)
+    static constexpr int kKStages = NH == 32 ? 3 : 2, kVStages = 3;
     static constexpr int kSoftmaxWarps = 4;
     static constexpr int kProducerWarp = 4, kMmaWarp = 5, kVProducerWarp = 6;
     static constexpr int kThreads = 32 * 7;
@@ -198,7 +201,7 @@ struct McShape {
     static constexpr uint32_t kHeaderBytes = 2048;
     static constexpr uint32_t kRedOff = 512;
     static constexpr uint32_t kSmemBytes = kHeaderBytes + 1024 + kTileBytes;
-    static constexpr uint32_t kTmemCols = 128;
+    static constexpr uint32_t kTmemCols = NH == 32 ? 128 : 256;
     static constexpr uint32_t kColS = 0;        // two S^T buffers: columns [0, 2 NH)
     static constexpr uint32_t kColO = 2 * NH;   // O^T: columns [2 NH, 3 NH)
     static_assert(kColO + NH <= kTmemCols, "TMEM columns");
@@ -206,7 +209,7 @@ struct McShape {
     // [kMcMaxCluster + 1][NH] in its Q buffer
     static_assert(NH * D * 4 + NH * 8 <= kKStages * kKVBytes, "part in the K ring");
     static_assert((kMcMaxCluster + 1) * NH * 4 <= kQBytes, "merge weights in the Q buffer");
-    static_assert(kRedOff + 2 * 4 * NH * 4 <= kHeaderBytes, "header");
+    static_assert(kRedOff + 4 * 32 * 4 + 4 * NH * 4 <= kHeaderBytes, "header");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the TMEM columns are always free");
 };
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     using T = McShape<D, NH>;
     using O = OperandGeom<D>;   // K, V and Q staging: D/64 blocks of [rows][64]
     using PG = OperandGeom<NH>; // P staging: [tokens][NH] rows of 2 NH bytes
-    constexpr int TK = T::kTok, KST = T::kKStages, VST = T::kVStages;
+    constexpr int TK = T::kTok, KST = T::kKStages, VST = T::kVStages, NC = T::kChunks;
     constexpr uint32_t kIdescQK = mc_idesc(TK, NH, false, false);
     constexpr uint32_t kIdescPV = mc_idesc(D, NH, true, true);
     // mbarriers; S, P and PVDone come in pairs, one per S / P buffer (tile parity)
@@ -234,8 +237,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * kBars);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + 8 * kBars + 4);
-    float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [4 warps][NH] head maxima
-    float* s_sum = s_red + 4 * NH;                                // [4 warps][NH] head sums
+    float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [4 warps][32] head maxima
+    float* s_sum = s_red + 4 * 32;                                // [4 warps][NH] head sums
     const uint32_t tb = (bar0 + T::kHeaderBytes + 1023u) & ~1023u;
     const uint32_t q_s = tb + T::kQOff, p_s = tb + T::kPOff;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -460,14 +463,28 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         // ================= softmax warps: thread r owns token r of each tile (TMEM lane r)
         const int r = 32 * warp + lane;
         const uint32_t t_lane = static_cast<uint32_t>(32 * warp) << 16;
-        // Q rows kvh * g + h (h < NH) in the K-major B layout [D/64][NH][64]
-        for (int idx = threadIdx.x; idx < NH * (D / 8); idx += kSoftThreads) {
-            const int h = idx / (D / 8), ch = idx - h * (D / 8);
-            const uint4 v =
-                __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + (kvh * p.g + h) * p.q_sh + 8 * ch));
-            st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (NH * O::kRowBytes) + h * O::kRowBytes +
-                                                     (O::swz(h, ch % O::kChunks) << 4)),
-                         v.x, v.y, v.z, v.w);
+        // Q rows kvh * g + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at and past
+        // g (padding up to NH) are zeros.  A thread's loads are all issued before its stores.
+        {
+            constexpr int kPer = NH * (D / 8) / kSoftThreads;  // 16-byte chunks per thread
+            static_assert(NH * (D / 8) % kSoftThreads == 0, "Q chunks per thread");
+            uint4 v[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int idx = threadIdx.x + u * kSoftThreads;
+                const int h = idx / (D / 8), ch = idx - h * (D / 8);
+                v[u] = h < p.g ? __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + (kvh * p.g + h) * p.q_sh +
+                                                                      8 * ch))
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int idx = threadIdx.x + u * kSoftThreads;
+                const int h = idx / (D / 8), ch = idx - h * (D / 8);
+                st_shared_v4(q_s + static_cast<uint32_t>((ch / O::kChunks) * (NH * O::kRowBytes) + h * O::kRowBytes +
+                                                         (O::swz(h, ch % O::kChunks) << 4)),
+                             v[u].x, v[u].y, v[u].z, v[u].w);
+            }
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(kQFull));
@@ -479,29 +496,41 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             m[h] = -INFINITY;
             l[h] = 0.f;
         }
+        // scores of heads [32 c, 32 c + 32) of this thread's token in S buffer sb, scaled to the
+        // log2 domain; -inf past the split's last token
+        auto load_x = [&](int c, int sb, bool valid, float (&x)[32]) {
+            uint32_t sr[32];
+            tc_ld32(tmem + t_lane + T::kColS + static_cast<uint32_t>(sb * NH + 32 * c), sr);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+        };
         bool wok = true, stopped = false;
         for (int j = 0; j < ntiles; ++j) {
             const int sb = j & 1;
-            float x[NH];
+            const bool valid = tok0 + j * TK + r < tok1;
+            float x0[32];  // the scores of chunk 0, kept when there is only one chunk
+            bool need = false;
             wok = warp_wait(bar(kSFull + sb), static_cast<uint32_t>(j >> 1) & 1u, kWaitTimeoutNs, abort_flag,
                             p.flags);
             if (wok) {
-                uint32_t sr[NH];
                 tc_fence_after();
-                tc_ld32(tmem + t_lane + T::kColS + static_cast<uint32_t>(sb * NH), sr);
-                tc_wait_ld();
-                tc_fence_before();
-                mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
-                const bool valid = tok0 + j * TK + r < tok1;
 #pragma unroll
-                for (int h = 0; h < NH; ++h) x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
-            } else {
+                for (int c = 0; c < NC; ++c) {
+                    float x[32];
+                    load_x(c, sb, valid, x);
 #pragma unroll
-                for (int h = 0; h < NH; ++h) x[h] = -INFINITY;
+                    for (int i = 0; i < 32; ++i) need |= x[i] > m[32 * c + i] + 8.f;
+                    if constexpr (NC == 1) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) x0[i] = x[i];
+                    }
+                }
+                if constexpr (NC == 1) {
+                    tc_fence_before();
+                    mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
+                }
             }
-            bool need = false;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) need |= x[h] > m[h] + 8.f;
             // one vote per tile: a new reference for some head, or some warp gave up
             const bool gave_up = !wok || *abort_flag != 0u;
             if (bar_any(kBarId, kSoftThreads, need || gave_up)) {
@@ -509,64 +538,89 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                     stopped = true;
                     break;
                 }
-                // ---- new reference: the tile's maximum of each head over the 128 tokens
-                float v[NH];
-#pragma unroll
-                for (int h = 0; h < NH; ++h) v[h] = x[h];
-                warp_reduce_scatter32<true>(v, lane);
-                s_red[warp * NH + lane] = v[0];
-                bar_named(kBarId, kSoftThreads);
-                float alpha[NH];
-#pragma unroll
-                for (int h = 0; h < NH; h += 4) {
-                    float4 a = *reinterpret_cast<const float4*>(s_red + h);
-#pragma unroll
-                    for (int w = 1; w < 4; ++w) {
-                        const float4 c = *reinterpret_cast<const float4*>(s_red + w * NH + h);
-                        a.x = fmaxf(a.x, c.x);
-                        a.y = fmaxf(a.y, c.y);
-                        a.z = fmaxf(a.z, c.z);
-                        a.w = fmaxf(a.w, c.w);
-                    }
-                    const float tm[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float mn = fmaxf(m[h + e], tm[e]);
-                        // 1 for a head whose maximum did not move; 0 while m is -inf
-                        alpha[h + e] = (mn == m[h + e]) ? 1.f : ex2_approx(m[h + e] - mn);
-                        m[h + e] = mn;
-                        l[h + e] *= alpha[h + e];
-                    }
-                }
+                // ---- new reference: the tile's maximum of each head over the 128 tokens,
+                // 32 heads at a time; O^T columns of the heads whose reference moved rescaled
                 if (j > 0) {
-                    // O^T holds P V of the earlier tiles: rescale this thread's row (head dim
-                    // r) column by column, once the last P V has landed (in issue order, so
-                    // every earlier one has too)
+                    // O^T holds P V of the earlier tiles: rescale once the last P V has landed
+                    // (in issue order, so every earlier one has too)
                     wok = warp_wait(bar(kPVDone + ((j - 1) & 1)), static_cast<uint32_t>((j - 1) >> 1) & 1u,
                                     kWaitTimeoutNs, abort_flag, p.flags);
-                    if (wok) {
+                }
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    float v[32];
+                    if constexpr (NC == 1) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = x0[i];
+                    } else {
+                        load_x(c, sb, valid, v);
+                    }
+                    warp_reduce_scatter32<true>(v, lane);
+                    s_red[warp * 32 + lane] = v[0];
+                    bar_named(kBarId, kSoftThreads);
+                    float alpha[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        float4 a = *reinterpret_cast<const float4*>(s_red + i);
+#pragma unroll
+                        for (int w = 1; w < 4; ++w) {
+                            const float4 q = *reinterpret_cast<const float4*>(s_red + w * 32 + i);
+                            a.x = fmaxf(a.x, q.x);
+                            a.y = fmaxf(a.y, q.y);
+                            a.z = fmaxf(a.z, q.z);
+                            a.w = fmaxf(a.w, q.w);
+                        }
+                        const float tm[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int h = 32 * c + i + e;
+                            const float mn = fmaxf(m[h], tm[e]);
+                            // 1 for a head whose maximum did not move; 0 while m is -inf
+                            alpha[i + e] = (mn == m[h]) ? 1.f : ex2_approx(m[h] - mn);
+                            m[h] = mn;
+                            l[h] *= alpha[i + e];
+                        }
+                    }
+                    if (j > 0 && wok) {
                         tc_fence_after();
-                        uint32_t o[NH];
-                        tc_ld32(tmem + t_lane + T::kColO, o);
+                        uint32_t o[32];
+                        const uint32_t oa = tmem + t_lane + T::kColO + static_cast<uint32_t>(32 * c);
+                        tc_ld32(oa, o);
                         tc_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < NH; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                        tc_st32(tmem + t_lane + T::kColO, o);
-                        tc_wait_st();
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[i]);
+                        tc_st32(oa, o);
                     }
+                    bar_named(kBarId, kSoftThreads);  // s_red is read by every thread before its next use
                 }
+                if (j > 0 && wok) tc_wait_st();
             }
             if (!wok) continue;  // gave up in this tile: the next vote stops every warp
 
             // ---- P = 2^(x - m) as bf16 pairs, and the sums of exactly those weights
             uint32_t pw[NH / 2];
 #pragma unroll
-            for (int i = 0; i < NH / 2; ++i) {
-                const float p0 = ex2_approx(x[2 * i] - m[2 * i]);
-                const float p1 = ex2_approx(x[2 * i + 1] - m[2 * i + 1]);
-                pw[i] = pack_bf16x2(p0, p1);
-                l[2 * i] += bf16_lo(pw[i]);
-                l[2 * i + 1] += bf16_hi(pw[i]);
+            for (int c = 0; c < NC; ++c) {
+                float x[32];
+                if constexpr (NC == 1) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = x0[i];
+                } else {
+                    load_x(c, sb, valid, x);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int h = 32 * c + 2 * i;
+                    const float p0 = ex2_approx(x[2 * i] - m[h]);
+                    const float p1 = ex2_approx(x[2 * i + 1] - m[h + 1]);
+                    pw[16 * c + i] = pack_bf16x2(p0, p1);
+                    l[h] += bf16_lo(pw[16 * c + i]);
+                    l[h + 1] += bf16_hi(pw[16 * c + i]);
+                }
+            }
+            if constexpr (NC > 1) {
+                tc_fence_before();
+                mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
             }
             // ---- P buffer j & 1 is free once P_{j-2} V_{j-2} has completed
             if (j > 1) {
@@ -595,75 +649,103 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             tc_fence_before();
             mbar_arrive(bar(kPFull + (j & 1)));
         }
-        // ---- epilogue: the heads' sums over the CTA's tokens, then out (or the partial)
+        // ---- epilogue: the heads' sums over the CTA's tokens, then out (or the partial, or the
+        // cluster part).  Heads at and past g are padding (zero Q rows): never written.
         if (!stopped && wok)
             wok = warp_wait(bar(kPVDone + ((ntiles - 1) & 1)), static_cast<uint32_t>((ntiles - 1) >> 1) & 1u,
                             kWaitTimeoutNs, abort_flag, p.flags);
-        float v[NH];
 #pragma unroll
-        for (int h = 0; h < NH; ++h) v[h] = l[h];
-        warp_reduce_scatter32<false>(v, lane);
-        s_sum[warp * NH + lane] = v[0];
+        for (int c = 0; c < NC; ++c) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = l[32 * c + i];
+            warp_reduce_scatter32<false>(v, lane);
+            s_sum[warp * NH + 32 * c + lane] = v[0];
+        }
         const bool gave_up = stopped || !wok || *abort_flag != 0u;
         const bool any_gave_up = bar_any(kBarId, kSoftThreads, gave_up);
-        uint32_t o[NH];
-        float lt[NH];
+        const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
+        // sum over the four softmax warps of the heads' sums, heads [32 c, 32 c + 32)
+        auto sums = [&](int c, float (&lt)[32]) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            o[h] = 0u;
-            lt[h] = 0.f;
-        }
-        if (!any_gave_up) {
-            tc_fence_after();
-            tc_ld32(tmem + t_lane + T::kColO, o);
-            tc_wait_ld();
-#pragma unroll
-            for (int h = 0; h < NH; h += 4) {
-                float4 a = *reinterpret_cast<const float4*>(s_sum + h);
+            for (int i = 0; i < 32; i += 4) {
+                float4 a = *reinterpret_cast<const float4*>(s_sum + 32 * c + i);
 #pragma unroll
                 for (int w = 1; w < 4; ++w) {
-                    const float4 c = *reinterpret_cast<const float4*>(s_sum + w * NH + h);
-                    a.x += c.x;
-                    a.y += c.y;
-                    a.z += c.z;
-                    a.w += c.w;
+                    const float4 q = *reinterpret_cast<const float4*>(s_sum + w * NH + 32 * c + i);
+                    a.x += q.x;
+                    a.y += q.y;
+                    a.z += q.z;
+                    a.w += q.w;
                 }
-                lt[h] = a.x;
-                lt[h + 1] = a.y;
-                lt[h + 2] = a.z;
-                lt[h + 3] = a.w;
+                lt[i] = a.x;
+                lt[i + 1] = a.y;
+                lt[i + 2] = a.z;
+                lt[i + 3] = a.w;
             }
-        }
-        const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
+        };
+        auto load_o = [&](int c, uint32_t (&o)[32]) {
+            tc_ld32(tmem + t_lane + T::kColO + static_cast<uint32_t>(32 * c), o);
+            tc_wait_ld();
+        };
+        // m and l of head 32 c + lane, for warp 0's writes of (m, l) pairs
+        auto head_ml = [&](int c, const float (&lt)[32], float& mm, float& ll) {
+            mm = 0.f;
+            ll = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if (lane == i) {
+                    mm = m[32 * c + i];
+                    ll = lt[i];
+                }
+            }
+        };
         if (nk == 1) {
             // the only non-empty split: normalised rows straight to out
             if (!any_gave_up) {
+                tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < NH; ++h)
-                    p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
-                        __float2bfloat16_rn(__uint_as_float(o[h]) / lt[h]);
+                for (int c = 0; c < NC; ++c) {
+                    uint32_t o[32];
+                    float lt[32];
+                    load_o(c, o);
+                    sums(c, lt);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int h = 32 * c + i;
+                        if (h < p.g)
+                            p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                                __float2bfloat16_rn(__uint_as_float(o[i]) / lt[i]);
+                    }
+                }
             }
         } else if (!p.cluster) {
             if (!any_gave_up) {
                 // the partial of this split, for each head block of 16 heads: slot
                 // ((b * Hkv + kvh) * HB + hb) * ksplit + split, row h - 16 hb
+                tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
-                    p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[h]);
-                }
-                if (warp == 0) {
-                    float mm = 0.f, ll = 0.f;
+                for (int c = 0; c < NC; ++c) {
+                    uint32_t o[32];
+                    float lt[32];
+                    load_o(c, o);
+                    sums(c, lt);
 #pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        if (lane == h) {
-                            mm = m[h];
-                            ll = lt[h];
+                    for (int i = 0; i < 32; ++i) {
+                        const int h = 32 * c + i;
+                        if (h < p.g) {
+                            const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
+                            p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[i]);
                         }
                     }
-                    const int64_t slot = (static_cast<int64_t>(u2) * p.HB + lane / kMaxRows) * p.ksplit + split;
-                    *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + lane % kMaxRows) * 2) =
-                        make_float2(mm, ll);
+                    if (warp == 0 && 32 * c + lane < p.g) {
+                        float mm, ll;
+                        head_ml(c, lt, mm, ll);
+                        const int h = 32 * c + lane;
+                        const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
+                        *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + h % kMaxRows) * 2) =
+                            make_float2(mm, ll);
+                    }
                 }
             }
         } else {
@@ -672,19 +754,29 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             float* const part_p = reinterpret_cast<float*>(smem + (tb + T::kKOff - bar0));
             cluster_wait();  // phase 0: every CTA of the cluster has its mbarriers initialised
             cluster_waited = true;
+            if (!any_gave_up) tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < NH; ++h) part_p[h * D + dd] = __uint_as_float(o[h]);
-            if (warp == 0) {
-                float mm = 0.f, ll = 0.f;
+            for (int c = 0; c < NC; ++c) {
+                uint32_t o[32];
+                float lt[32];
+                if (!any_gave_up) {
+                    load_o(c, o);
+                    sums(c, lt);
+                } else {
 #pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    if (lane == h) {
-                        mm = m[h];
-                        ll = lt[h];
+                    for (int i = 0; i < 32; ++i) {
+                        o[i] = 0u;
+                        lt[i] = 0.f;
                     }
                 }
-                part_p[NH * D + 2 * lane] = mm;
-                part_p[NH * D + 2 * lane + 1] = ll;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) part_p[(32 * c + i) * D + dd] = __uint_as_float(o[i]);
+                if (warp == 0) {
+                    float mm, ll;
+                    head_ml(c, lt, mm, ll);
+                    part_p[NH * D + 2 * (32 * c + lane)] = mm;
+                    part_p[NH * D + 2 * (32 * c + lane) + 1] = ll;
+                }
             }
             fence_acq_rel_cluster();
             bar_named(kBarId, kSoftThreads);
@@ -739,8 +831,9 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                 }
 #pragma unroll
                 for (int j = 0; j < kMaxH; ++j) {
-                    if (j < nh)
-                        p.out[b * p.out_sb + (kvh * p.g + split + j * nk) * p.out_sh + dd] =
+                    const int h = split + j * nk;
+                    if (j < nh && h < p.g)
+                        p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
                             __float2bfloat16_rn(acc[j] * wts[kMcMaxCluster * NH + j]);
                 }
             }

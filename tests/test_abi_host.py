@@ -202,7 +202,7 @@ def test_workspace_size_invalid_is_zero():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,D", [(16, 32, 8, 128), (2, 32, 8, 128), (128, 64, 8, 128), (4, 8, 8, 32),
-                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 64), (8, 96, 2, 128)])
+                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 64), (8, 160, 2, 128)])
 def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
     g = Hq // Hkv
@@ -245,7 +245,7 @@ def _smem(B, D, rows, warps, stages, hb, shared):
     return -(-meta // 16) * 16 + 1024 + rings
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 128, 2, 128), (4, 96, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 160, 2, 128), (4, 192, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
                                         (4, 64, 2, 256), (4, 32, 8, 128), (4, 16, 1, 64)])
 def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     # balanced mode with g > 16: the head blocks of a kv head share one K/V ring, so the
@@ -276,26 +276,35 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
         assert local.smem_bytes == _unit_smem(D, rows, local.warps_per_cta, stages)
 
 
-_MC_SMEM = 2048 + 1024 + 32 * 128 * 2 + 3 * 2 * 128 * 128 * 2 + 2 * 128 * 32 * 2
+def _mc_smem(nh):
+    """Shared memory of the tensor-core multi-query kernel: 2 KB header, 1 KB of alignment
+    slack, Q [nh][128], 3 (nh = 32) or 2 (nh = 64) K stages and 3 V stages of 128 tokens x
+    128, two P buffers [128][nh] (bf16)."""
+    k_stages = 3 if nh == 32 else 2
+    return 2048 + 1024 + nh * 128 * 2 + (k_stages + 3) * 128 * 128 * 2 + 2 * 128 * nh * 2
 
 
+@pytest.mark.parametrize("g", [32, 20, 48, 64])
 @pytest.mark.parametrize("B,Hkv,sm", [(16, 2, 148), (1, 1, 148), (4, 8, 148), (200, 1, 148), (3, 2, 132), (16, 2, 8)])
-def test_plan_tensor_core_multi_query(B, Hkv, sm):
-    """32 q heads per kv head at D = 128: the tensor-core multi-query kernel, one CTA per
-    split of each (sequence, kv head), 7 warps (4 softmax, 2 producers, 1 MMA issuer), 3
-    K and 3 V stages of 128 tokens, Q and two P buffers in shared memory.  Auto splits
+def test_plan_tensor_core_multi_query(B, Hkv, sm, g):
+    """17 to 64 q heads per kv head at D = 128: the tensor-core multi-query kernel (heads
+    padded to 32 or 64), one CTA per split of each (sequence, kv head), 7 warps (4 softmax,
+    2 producers, 1 MMA issuer), K and V rings of 128-token stages, Q and two P buffers in
+    shared memory.  Auto splits
     spread the units over 7/8 of the SMs.  A unit's splits (up to 8) that the device can run
     as one cluster merge over DSMEM in the kernel; otherwise their partials take the
     fixed-split slots of both head blocks and the combine kernel merges them.  The slots are
     reserved either way."""
-    Hq, D = 32 * Hkv, 128
-    units = B * Hkv * 2
+    Hq, D = g * Hkv, 128
+    nh = 32 if g <= 32 else 64
+    units = B * Hkv * -(-g // 16)
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
     k = max(1, sm * 7 // 8 // (B * Hkv))
     assert pl.mode == 3 and pl.shared_kv_ring == 0
     assert pl.grid_ctas == B * Hkv * k and pl.num_workers == pl.grid_ctas
-    assert pl.warps_per_cta == 7 and pl.stages == 3 and pl.smem_bytes == _MC_SMEM <= 232448
-    assert pl.rows_per_unit == 16 and pl.head_blocks == 2
+    assert pl.warps_per_cta == 7 and pl.stages == 3
+    assert pl.smem_bytes == _mc_smem(nh) <= 232448
+    assert pl.rows_per_unit == 16 and pl.head_blocks == -(-g // 16)
     assert pl.partial_slots == (units * k if k > 1 else 0)
     # up to 8 splits of a unit that fit the device as one cluster each merge in the kernel
     # (with an SM count given, every k SMs are taken to hold a cluster of k)
@@ -310,7 +319,7 @@ def test_plan_tensor_core_multi_query(B, Hkv, sm):
     small = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm, workspace_bytes=4096)
     assert small.mode == 3 and small.grid_ctas == B * Hkv and small.partial_slots == 0
     # other head dims and group sizes keep the mma.sync kernels
-    for Hq2, D2 in ((32 * Hkv, 64), (48 * Hkv, 128), (16 * Hkv, 128)):
+    for Hq2, D2 in ((g * Hkv, 64), (80 * Hkv, 128), (16 * Hkv, 128)):
         assert apd.query_plan(B, Hq2, Hkv, D2, 0, sm_count=sm).mode != 3
 
 
@@ -660,7 +669,7 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
         assert pl.num_workers == pl.grid_ctas * pl.warps_per_cta
     elif pl.mode == 3:
         # the tensor-core multi-query kernel: one CTA per split of each (sequence, kv head)
-        assert D == 128 and g == 32 and pl.grid_ctas % (B * Hkv) == 0
+        assert D == 128 and 16 < g <= 64 and pl.grid_ctas % (B * Hkv) == 0
         k = pl.grid_ctas // (B * Hkv)
         assert k == splits or splits == 0
         assert pl.partial_slots == (units * k if k > 1 else 0)

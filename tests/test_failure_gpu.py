@@ -31,18 +31,18 @@ def test_context_is_usable_after_a_wait_gave_up():
 
 
 def test_shared_ring_leader_stops_when_a_release_never_comes():
-    """The shared K/V ring's error path (48 q heads per kv head, auto splits): the
+    """The shared K/V ring's error path (80 q heads per kv head, auto splits): the
     self-test runs the real decode with followers that never release a stage and a 1 ms
     limit per wait.  Each ring's leader must give up at its first refill, stop issuing and
     return, and its followers must stop through the CTA's abort word, so the call ends
     within a few limits (a leader that kept refilling would wait out one limit per tile:
     over 100 ms here) with APD_FLAG_WAIT_TIMEOUT set.  A normal call afterwards is correct."""
-    w = workloads.make(name="ring_release", seed=83, batch=4, num_q_heads=96, num_kv_heads=2, head_dim=128,
+    w = workloads.make(name="ring_release", seed=83, batch=4, num_q_heads=160, num_kv_heads=2, head_dim=128,
                        seq_lens=[16384, 16000, 12000, 16384], page_size=32)
     dp = DeviceProblem(w)
-    default = apd.workspace_size(4, 96, 2, 128, 0)
+    default = apd.workspace_size(4, 160, 2, 128, 0)
     ws = torch.zeros(default // 16 // 256 * 256, dtype=torch.uint8, device="cuda")  # long runs per warp
-    plan = apd.query_plan(4, 96, 2, 128, 0, workspace_bytes=ws.numel())
+    plan = apd.query_plan(4, 160, 2, 128, 0, workspace_bytes=ws.numel())
     assert plan.shared_kv_ring == 1 and plan.mode == 0
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -1,5 +1,6 @@
-"""GPU parity of the tensor-core multi-query decode (plan mode 3: 32 q heads per kv head at
-D = 128, decode_mq_tc_kernel + the fixed-split combine) against the fp64 CPU oracle.
+"""GPU parity of the tensor-core multi-query decode (plan mode 3: 17 to 64 q heads per kv head
+at D = 128, decode_mq_tc_kernel with the heads padded to 32 or 64, merged in a cluster or by
+the fixed-split combine) against the fp64 CPU oracle.
 
 Per output element |gpu - ref| <= 1e-2 + 1e-2 |ref| (ref = fp64 oracle value), as for every
 decode path.  Covered: automatic and fixed split counts (one split per unit, partial 128-token
@@ -139,6 +140,20 @@ def test_contract_flags():
     assert np.isfinite(out).all()
     assert np.all(out[2] == 0)
     check_close(dp.out[[0]], ref[[0]], "untouched sequence")
+
+
+@pytest.mark.parametrize("g", [20, 48, 64])
+@pytest.mark.parametrize("S", [0, 1, 3, 16])
+def test_other_group_sizes(g, S):
+    """Group sizes padded to the kernel's 32 or 64 heads (20 -> 32; 48, 64 -> 64: the softmax
+    in two passes of 32 heads): ragged lengths with an empty sequence, poisoned slots, and
+    score outliers that move the reference maximum of some heads."""
+    w = small(13, 4, 2 * g, 2, (1900, 0, 77, 640), pool=120, poison=True, k_outlier_frac=0.02,
+              k_outlier_mult=20.0)
+    dp, out = run_mode3(w, S)
+    check_close(out, oracle.paged_decode(w), f"g={g} S={S}")
+    assert torch.all(out[1] == 0)
+    assert apd.read_device_flags(dp.workspace) == 0
 
 
 def test_gqa32_full_size():
