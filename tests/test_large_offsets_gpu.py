@@ -2,7 +2,8 @@
 
 Every K/V access goes through TMA tensor maps (64-bit byte strides, 32-bit
 coordinates), and q / out / mask through 64-bit strides; these cases pin that on
-caches of 4.5-7 GB each.  Only the pages (or rows) a call references are filled
+caches of 4.5-7 GB each, for the split, unit and tensor-core decode kernels and both
+prefill kernels.  Only the pages (or rows) a call references are filled
 with the workload's seeded values, placed at the far end of a large allocation whose
 other contents are never written and must never be read; the oracle sees the
 compact workload.  Per element |gpu - ref| <= 1e-2 + 1e-2 |ref|, as everywhere."""
@@ -49,6 +50,24 @@ def test_paged_decode_pages_past_2_31_elements(S):
     ws = apd.alloc_workspace(3, 16, 2, 128, S)
     apd.attn_paged_decode(dp.q, k, v, pt, dp.seq_lens, dp.out, w.scale, S, ws)
     check_close(dp.out, ref, f"pages past 2^31 S={S}")
+    assert apd.read_device_flags(ws) == 0
+
+
+@pytest.mark.parametrize("Hq,S", [(64, 0), (64, 3), (64, 16), (96, 0)])
+def test_tensor_core_decode_pages_past_2_31_elements(Hq, S):
+    """The tensor-core multi-query kernel (32 and 48 q heads per kv head at D = 128), with
+    its splits merged in a cluster (auto, 3) or by the combine (16)."""
+    w = workloads.make(name="far", seed=64, batch=3, num_q_heads=Hq, num_kv_heads=2, head_dim=128, page_size=32,
+                       seq_lens=[1000, 700, 33], pool_pages=64)
+    assert apd.query_plan(3, Hq, 2, 128, S).mode == 3
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    k, base = far_pool(dp.k, dp.k.shape[0])
+    v, _ = far_pool(dp.v, dp.v.shape[0])
+    pt = dp.page_table + base
+    ws = apd.alloc_workspace(3, Hq, 2, 128, S)
+    apd.attn_paged_decode(dp.q, k, v, pt, dp.seq_lens, dp.out, w.scale, S, ws)
+    check_close(dp.out, ref, f"tensor-core pages past 2^31 {Hq}/2 S={S}")
     assert apd.read_device_flags(ws) == 0
 
 
