@@ -25,6 +25,7 @@ __all__ = [
     "attn_paged_prefill",
     "selftest_bounded_wait",
     "selftest_shared_ring_release",
+    "selftest_mq_tc_stall",
     "gemv",
     "gemv_workspace_size",
     "DecodeCall",
@@ -173,6 +174,9 @@ def _load():
     L.apd_selftest_shared_ring_release.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
                                                    ctypes.c_uint64, ctypes.c_void_p]
     L.apd_selftest_shared_ring_release.restype = ctypes.c_int
+    L.apd_selftest_mq_tc_stall.argtypes = [T, T, T, T, T, T, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_size_t, ctypes.c_uint64, ctypes.c_void_p]
+    L.apd_selftest_mq_tc_stall.restype = ctypes.c_int
     L.apd_gemv_workspace_size.argtypes = [ctypes.c_int] * 3
     L.apd_gemv_workspace_size.restype = ctypes.c_size_t
     L.apd_gemv_query_plan.argtypes = [ctypes.c_int] * 4 + [ctypes.POINTER(_GemvPlan)]
@@ -352,6 +356,20 @@ def selftest_shared_ring_release(q, k_cache, v_cache, page_table, seq_lens, out,
                                                   int(short_timeout_ns), _stream_handle(stream, q.device))
     if rc:
         raise APDError(rc, "apd_selftest_shared_ring_release")
+
+
+def selftest_mq_tc_stall(q, k_cache, v_cache, page_table, seq_lens, out, scale: float, num_splits: int,
+                         workspace: torch.Tensor, short_timeout_ns: int = 1_000_000, stream=None) -> None:
+    """Enqueues the tensor-core multi-query kernel's stall self-test (apd_selftest_mq_tc_stall)
+    on a problem that takes that kernel: the softmax warps never hand over the weights of their
+    second tile and every wait gives up after short_timeout_ns.  Read the outcome with
+    read_device_flags(workspace)."""
+    descs = [_desc(t) for t in (q, k_cache, v_cache, page_table, seq_lens, out)]
+    rc = _load().apd_selftest_mq_tc_stall(*[ctypes.byref(d) for d in descs], ctypes.c_float(scale), int(num_splits),
+                                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                          int(short_timeout_ns), _stream_handle(stream, q.device))
+    if rc:
+        raise APDError(rc, "apd_selftest_mq_tc_stall")
 
 
 def prefill_auto_kernel(head_dim: int) -> str:

@@ -634,7 +634,8 @@ int encode_q_map(CUtensorMap* map, const apd_tensor* t, const int64_t* st, int D
 // Self-test settings of the split kernel (the defaults are the product's).
 struct SplitTestHooks {
     uint64_t wait_ns = apd::kWaitTimeoutNs;
-    int skip_release = 0;
+    int skip_release = 0;  // shared-ring followers never release a stage
+    int skip_pfull = 0;    // tensor-core kernel: the softmax warps never hand over P of tile 1
 };
 
 // The caller's split_done_event, recorded right after the first kernel of the call.
@@ -687,7 +688,8 @@ int launch_combine(const Shape& s, const Plan& pl, const apd::CombineParams& cp,
 template <int NH>
 int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, const apd_tensor* v,
                  const apd_tensor* pt, const apd_tensor* sl, const apd_tensor* out, float scale, const Plan& pl,
-                 void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts) {
+                 void* workspace, DeviceState* dev, cudaStream_t stream, const apd_launch_options* opts,
+                 const SplitTestHooks& hooks) {
     constexpr int D = 128;
     using McShape128 = McShapeT<NH>;
     auto kern = apd::decode_mq_tc_kernel<D, NH>;
@@ -736,6 +738,8 @@ int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, c
     mp.ksplit = pl.ksplit;
     mp.cluster = pl.cluster > 0 ? 1 : 0;
     mp.scale_log2 = scale * 1.4426950408889634f;
+    mp.wait_ns = hooks.wait_ns;
+    mp.test_skip_pfull = hooks.skip_pfull;
 
     const bool use_pdl = !(opts && opts->disable_pdl);
     cudaLaunchAttribute attrs[2];
@@ -796,8 +800,8 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     if constexpr (D == 128) {
         if (pl.mode == 3)
             return mq_tc_heads(V.s) == 64
-                       ? launch_mq_tc<64>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts)
-                       : launch_mq_tc<32>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts);
+                       ? launch_mq_tc<64>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts, hooks)
+                       : launch_mq_tc<32>(V, q, k, v, pt, sl, out, scale, pl, workspace, dev, stream, opts, hooks);
     }
     if (pl.mode == 3) return APD_ERR_ARGUMENT;  // planned only for D = 128
     constexpr int kStagesD = kStages<D>;
@@ -1351,6 +1355,8 @@ int decode_impl(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor
     if (rc) return rc;
     // the release self-test needs the shared K/V ring (auto splits, more than 16 q heads per kv head)
     if (h.skip_release && !pl.share) return APD_ERR_ARGUMENT;
+    // the stall self-test needs the tensor-core multi-query kernel
+    if (h.skip_pfull && pl.mode != 3) return APD_ERR_ARGUMENT;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     switch (V.s.D) {
         case 32: return launch<32>(V, q, k_cache, v_cache, page_table, seq_lens, out, scale, pl, workspace, dev, st, options, h);
@@ -1680,6 +1686,19 @@ int apd_selftest_shared_ring_release(const apd_tensor* q, const apd_tensor* k_ca
     h.skip_release = 1;
     return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, scale, 0, workspace, workspace_bytes, stream,
                        nullptr, &h);
+}
+
+int apd_selftest_mq_tc_stall(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                             uint64_t short_timeout_ns, apd_stream_t stream) {
+    if (!page_table) return APD_ERR_NULL_POINTER;
+    if (short_timeout_ns == 0 || short_timeout_ns > 1000000000ull) return APD_ERR_ARGUMENT;
+    SplitTestHooks h;
+    h.wait_ns = short_timeout_ns;
+    h.skip_pfull = 1;
+    return decode_impl(q, k_cache, v_cache, page_table, seq_lens, out, scale, num_splits, workspace, workspace_bytes,
+                       stream, nullptr, &h);
 }
 
 int apd_selftest_bounded_wait(uint32_t* out, uint64_t short_timeout_ns, apd_stream_t stream) {

@@ -67,6 +67,8 @@ struct McParams {
     int32_t ksplit;   // splits per (sequence, kv head)
     int32_t cluster;  // 1: the ksplit CTAs of a unit are one cluster and merge over DSMEM
     float scale_log2;
+    uint64_t wait_ns;         // limit of each wait (kWaitTimeoutNs; shorter in the self-test)
+    int32_t test_skip_pfull;  // self-test only: the softmax warps never hand over P of tile 1
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B, fp32 D, each operand
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             const int ng = min(kBoxes, (tok1 - (tok0 + j * TK) + kTile - 1) / kTile);  // boxes holding tokens
             const uint32_t bytes = static_cast<uint32_t>(ng) * kTile * D * 2u;
             const int stage = j % ST;
-            if (j >= ST) ok = tc_wait(bar(empty0 + stage), static_cast<uint32_t>((j / ST) - 1) & 1u, abort_flag, p.flags);
+            if (j >= ST) ok = tc_wait(bar(empty0 + stage), static_cast<uint32_t>((j / ST) - 1) & 1u, abort_flag, p.flags, p.wait_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             if (lane == 0) {
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             for (int s = 0; s < ST; ++s) {
                 if (issued > s) {
                     const int jl = s + ST * ((issued - 1 - s) / ST);
-                    mbar_wait_bounded(bar(full0 + s), static_cast<uint32_t>(jl / ST) & 1u, kWaitTimeoutNs);
+                    mbar_wait_bounded(bar(full0 + s), static_cast<uint32_t>(jl / ST) & 1u, p.wait_ns);
                 }
             }
         }
@@ -401,7 +403,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         // thread run in issue order, so the P V products accumulate into O^T in tile order
         if (lane == 0) {
             bool issued = false;
-            ok = tc_wait(bar(kQFull), 0, abort_flag, p.flags);
+            ok = tc_wait(bar(kQFull), 0, abort_flag, p.flags, p.wait_ns);
             int jq = 0, jp = 0;
             uint64_t t_idle = global_timer_ns();
             for (uint32_t it = 1; ok && jp < ntiles; ++it) {
@@ -446,7 +448,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                 } else if ((it & 63u) == 0) {
                     const uint64_t now = global_timer_ns();
                     if (it == 64) t_idle = now;  // the first check of an idle stretch starts its clock
-                    else if (now - t_idle > kWaitTimeoutNs) {
+                    else if (now - t_idle > p.wait_ns) {
                         *abort_flag = 1u;
                         atomicOr(p.flags, kFlagTimeout);
                         ok = false;
@@ -456,7 +458,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             if (!ok && issued) {
                 // wait (bounded) for the MMAs still in flight
                 tc_commit(bar(kDrain));
-                mbar_wait_bounded(bar(kDrain), 0, kWaitTimeoutNs);
+                mbar_wait_bounded(bar(kDrain), 0, p.wait_ns);
             }
         }
     } else {
@@ -511,7 +513,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             const bool valid = tok0 + j * TK + r < tok1;
             float x0[32];  // the scores of chunk 0, kept when there is only one chunk
             bool need = false;
-            wok = warp_wait(bar(kSFull + sb), static_cast<uint32_t>(j >> 1) & 1u, kWaitTimeoutNs, abort_flag,
+            wok = warp_wait(bar(kSFull + sb), static_cast<uint32_t>(j >> 1) & 1u, p.wait_ns, abort_flag,
                             p.flags);
             if (wok) {
                 tc_fence_after();
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                     // O^T holds P V of the earlier tiles: rescale once the last P V has landed
                     // (in issue order, so every earlier one has too)
                     wok = warp_wait(bar(kPVDone + ((j - 1) & 1)), static_cast<uint32_t>((j - 1) >> 1) & 1u,
-                                    kWaitTimeoutNs, abort_flag, p.flags);
+                                    p.wait_ns, abort_flag, p.flags);
                 }
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
@@ -624,7 +626,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             }
             // ---- P buffer j & 1 is free once P_{j-2} V_{j-2} has completed
             if (j > 1) {
-                wok = warp_wait(bar(kPVDone + (j & 1)), static_cast<uint32_t>((j - 2) >> 1) & 1u, kWaitTimeoutNs,
+                wok = warp_wait(bar(kPVDone + (j & 1)), static_cast<uint32_t>((j - 2) >> 1) & 1u, p.wait_ns,
                                 abort_flag, p.flags);
                 if (!wok) continue;
                 tc_fence_after();
@@ -639,7 +641,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             // or nothing loaded): zero them before they meet a zero weight
             if (j == ntiles - 1 && tok0 + j * TK + TK > tok1) {
                 const int stage = j % VST;
-                wok = warp_wait(bar(kVFull + stage), static_cast<uint32_t>(j / VST) & 1u, kWaitTimeoutNs, abort_flag,
+                wok = warp_wait(bar(kVFull + stage), static_cast<uint32_t>(j / VST) & 1u, p.wait_ns, abort_flag,
                                 p.flags);
                 if (!wok) continue;
                 zero_v_rows<D, TK>(tb + T::kVOff + static_cast<uint32_t>(stage) * T::kKVBytes, tok1 - (tok0 + j * TK),
@@ -647,13 +649,13 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             }
             fence_proxy_async_smem();  // P (and the zeroed V rows) -> tensor core
             tc_fence_before();
-            mbar_arrive(bar(kPFull + (j & 1)));
+            if (!(p.test_skip_pfull && j == 1)) mbar_arrive(bar(kPFull + (j & 1)));
         }
         // ---- epilogue: the heads' sums over the CTA's tokens, then out (or the partial, or the
         // cluster part).  Heads at and past g are padding (zero Q rows): never written.
         if (!stopped && wok)
             wok = warp_wait(bar(kPVDone + ((ntiles - 1) & 1)), static_cast<uint32_t>((ntiles - 1) >> 1) & 1u,
-                            kWaitTimeoutNs, abort_flag, p.flags);
+                            p.wait_ns, abort_flag, p.flags);
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             float v[32];
@@ -785,7 +787,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             // this split merges heads h = split + j nk (j < nh) of every part:
             // w_s = 2^(m_s - M) over the non-empty parts, out = sum_s w_s O_s / sum_s w_s l_s
             const int nh = (NH - split + nk - 1) / nk;
-            const bool pok = warp_wait_cluster(bar(kParts), 0u, kWaitTimeoutNs, abort_flag, p.flags);
+            const bool pok = warp_wait_cluster(bar(kParts), 0u, p.wait_ns, abort_flag, p.flags);
             float* const wts = reinterpret_cast<float*>(smem + (q_s - bar0));  // [kMcMaxCluster + 1][NH]
             if (warp == 0 && pok && lane < nh) {
                 const int h = split + lane * nk;

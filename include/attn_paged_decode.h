@@ -431,6 +431,27 @@ int apd_selftest_shared_ring_release(const apd_tensor* q, const apd_tensor* k_ca
                                      float scale, void* workspace, size_t workspace_bytes,
                                      uint64_t short_timeout_ns, apd_stream_t stream);
 
+/*
+ * apd_selftest_mq_tc_stall -- exercises, on the GPU and without any fault, the error path
+ * of the tensor-core multi-query kernel (apd_plan.mode 3: 17 to 64 q heads per kv head at
+ * head_dim 128).  It runs apd_attn_paged_decode(num_splits) on the given problem with two
+ * differences: the softmax warps never hand over the weights P of their second tile, and
+ * every wait gives up after `short_timeout_ns` (1 .. 1e9 ns) instead of 2 s.  The MMA
+ * issuer and the softmax warps must then give up, raise the CTA's abort flag, leave their
+ * loops together (the softmax warps through a barrier vote), wait (bounded) for their
+ * copies and MMAs in flight and meet before the TMEM columns are freed and, with the
+ * cluster merge, at the cluster barrier.  The call ends within a few limits, the flag word
+ * in the workspace gets APD_FLAG_WAIT_TIMEOUT, and `out` is undefined.
+ *
+ *   Arguments as apd_attn_paged_decode.  Returns APD_ERR_ARGUMENT before any launch when
+ *   the problem does not take the tensor-core kernel or the limit is out of range;
+ *   otherwise as that call.
+ */
+int apd_selftest_mq_tc_stall(const apd_tensor* q, const apd_tensor* k_cache, const apd_tensor* v_cache,
+                             const apd_tensor* page_table, const apd_tensor* seq_lens, const apd_tensor* out,
+                             float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                             uint64_t short_timeout_ns, apd_stream_t stream);
+
 /* apd_plan -- how a call with these arguments would be launched (for tests,
  * benchmarks and profiling). */
 typedef struct apd_plan {
@@ -438,9 +459,10 @@ typedef struct apd_plan {
                                   2 = one CTA per unit, parts merged in shared memory
                                   (num_splits == 0 with host lengths, see
                                   apd_launch_options.host_seq_lens),
-                                  3 = tensor-core multi-query kernel (32 q heads per
-                                  kv head at head_dim 128, any num_splits): one CTA per
-                                  split of each (sequence, kv head)             */
+                                  3 = tensor-core multi-query kernel (17 to 64 q
+                                  heads per kv head at head_dim 128, any
+                                  num_splits): one CTA per split of each
+                                  (sequence, kv head)                           */
     int32_t num_workers;       /* warps that each own a run of tiles             */
     int32_t grid_ctas;         /* CTAs of the split kernel                       */
     int32_t warps_per_cta;

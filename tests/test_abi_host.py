@@ -579,6 +579,25 @@ def test_release_selftest_arguments_are_checked_before_any_launch():
     assert call(g4) in (ARG, CUDA)  # ARG once the plan is made (it needs the device's SM count)
 
 
+def test_stall_selftest_arguments_are_checked_before_any_launch():
+    """The tensor-core kernel's stall self-test: a NULL page table, a limit outside 1 ns ..
+    1 s, and a problem that does not take that kernel (g = 4) are refused without a launch."""
+    L = apd.lib()
+
+    def call(p, limit=1_000_000, pt=True):
+        a = [ctypes.byref(p[n]) for n in ("q", "k", "v")] + [ctypes.byref(p["pt"]) if pt else None] + \
+            [ctypes.byref(p[n]) for n in ("sl", "out")]
+        return L.apd_selftest_mq_tc_stall(*a, ctypes.c_float(0.1), 0, FAKE, 1 << 30, limit, None)
+
+    g32 = dict(q=T([2, 64, 128]), out=T([2, 64, 128]), k=T([16, 32, 2, 128]), v=T([16, 32, 2, 128]),
+               pt=T([2, 4], apd.DTYPE_INT32), sl=T([2], apd.DTYPE_INT32))
+    assert call(g32, pt=False) == NULLP
+    assert call(g32, limit=0) == ARG
+    assert call(g32, limit=2_000_000_000) == ARG
+    g4 = dict(g32, q=T([2, 8, 128]), out=T([2, 8, 128]))
+    assert call(g4) in (ARG, CUDA)  # ARG once the plan is made (it needs the device's SM count)
+
+
 # ---------------------------------------------------------------- GEMV planning
 @pytest.mark.parametrize("M,N,K", [(1, 100000, 1536), (8, 100000, 1536), (1, 6912, 1536), (3, 1536, 1536),
                                    (1, 256, 1536), (8, 1536, 6912), (5, 50, 1040), (2, 3000, 1000), (1, 64, 200),

@@ -64,3 +64,32 @@ def test_release_selftest_needs_the_shared_ring():
     ws = apd.alloc_workspace(2, 32, 8, 128, 0)
     with pytest.raises(apd.APDError):
         apd.selftest_shared_ring_release(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, ws)
+
+
+@pytest.mark.parametrize("B,S", [(16, 0), (4, 0), (16, 16)])
+def test_tensor_core_kernel_stops_when_a_hand_over_never_comes(B, S):
+    """The tensor-core multi-query kernel's error path (32 q heads per kv head at D = 128),
+    with the splits merged in a cluster (B = 16, auto: 4 splits) or by the combine (B = 4,
+    auto: 16 splits; B = 16 with 16 fixed splits).  The self-test runs the real decode with
+    softmax warps that never hand over the weights of their second tile and a 1 ms limit
+    per wait: the MMA issuer and the softmax warps must give up, leave their loops together,
+    wait for their copies and MMAs in flight, free TMEM and meet at the cluster barrier, so
+    the call ends within a few limits with APD_FLAG_WAIT_TIMEOUT set.  A normal call
+    afterwards is correct."""
+    w = workloads.make(name="mq_stall", seed=85, batch=B, num_q_heads=64, num_kv_heads=2, head_dim=128,
+                       seq_lens=[16384] * B, page_size=32)
+    dp = DeviceProblem(w)
+    ws = apd.alloc_workspace(B, 64, 2, 128, S)
+    plan = apd.query_plan(B, 64, 2, 128, S)
+    assert plan.mode == 3 and (plan.cluster_size > 0) == (B == 16 and S == 0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    apd.selftest_mq_tc_stall(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, S, ws, 1_000_000)
+    e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert apd.read_device_flags(ws) & apd.FLAG_WAIT_TIMEOUT
+    assert ms < 30.0, f"the self-test call took {ms:.1f} ms"
+    check_close(dp.run(S, workspace=ws), oracle.paged_decode(w), "decode after the stall self-test")
+    assert apd.read_device_flags(ws) == 0
