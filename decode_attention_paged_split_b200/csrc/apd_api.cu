@@ -216,8 +216,7 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
 // blocks' rows of each split), so the combine is the fixed-split one.
 template <int NH>
 using McShapeT = apd::McShape<128, NH>;
-constexpr int kMcWarps = McShapeT<32>::kThreads / 32;
-static_assert(McShapeT<64>::kThreads == McShapeT<32>::kThreads, "one warp layout");
+
 // NH of the tensor-core kernel for this shape, or 0 when the shape does not take it
 int mq_tc_heads(const Shape& s) { return s.D == 128 && s.g > 16 && s.g <= 64 ? (s.g <= 32 ? 32 : 64) : 0; }
 bool mq_tc_eligible(const Shape& s) { return mq_tc_heads(s) > 0; }
@@ -293,8 +292,8 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
     pl->share = false;
     pl->ksplit = static_cast<int>(ksplit);
     pl->groups = 0;
-    pl->warps = kMcWarps;
     const bool h64 = mq_tc_heads(s) == 64;
+    pl->warps = (h64 ? McShapeT<64>::kThreads : McShapeT<32>::kThreads) / 32;
     pl->stages = h64 ? McShapeT<64>::kVStages : McShapeT<32>::kVStages;
     pl->smem = h64 ? McShapeT<64>::kSmemBytes : McShapeT<32>::kSmemBytes;
     pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * ksplit);

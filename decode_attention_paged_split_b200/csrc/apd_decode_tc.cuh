@@ -22,18 +22,20 @@
 //                                                 MN-major: P stored [token][head])
 //    so the staged K and V tiles are used exactly as the TMA lands them and no query row of
 //    the MMA is padding.
-//  - Warps 4 and 6 (producers) resolve each tile's four pages and issue the TMA loads of
-//    its K boxes (warp 4) and V boxes (warp 6) into two rings, each refilled as soon as its
+//  - Two producer warps (after the softmax warps) resolve each tile's four pages and issue
+//    the TMA loads of its K boxes and its V boxes into two rings, each refilled as soon as its
 //    own stage is free: a K stage right after its S^T product, a V stage after its P V.
-//    Warp 5 lane 0 issues the MMAs, each product as soon as its operands are ready (S^T_j
-//    does not wait for P_{j-1} V_{j-1}, nor that for the next K tile), and commits them to
-//    the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T and two
+//    One lane of the warp between them issues the MMAs, each product as soon as its operands
+//    are ready (S^T_j does not wait for P_{j-1} V_{j-1}, nor that for the next K tile), and
+//    commits them to the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T and two
 //    P buffers let the softmax of tile j + 1 run while P_j V_j is on the tensor core.
-//  - Warps 0-3 (softmax): TMEM lane t is token t of the tile, so thread t reads its token's
-//    32 scores with one tcgen05.ld and owns that token's exponentials.  The reference
+//  - Softmax warps, one group of 4 per 32 heads (warps 0-3, and 4-7 at 64 heads): TMEM lane t
+//    is token t of the tile, so thread t of a group reads its token's 32 scores of the
+//    group's heads with one tcgen05.ld and owns those exponentials.  The reference
 //    maximum of each head is shared by all tokens; it moves only when some score exceeds it
-//    by more than 2^8 (one OR-vote per tile over a named barrier; the head maxima are then
-//    reduced across the 128 threads, O^T and the running sums rescaled).  Each thread keeps
+//    by more than 2^8 (one OR-vote per tile and group over the group's named barrier; the
+//    head maxima are then reduced across its 128 threads, O^T and the running sums
+//    rescaled).  Each thread keeps
 //    its own running sums of the bf16 weights it wrote; they are added across the threads
 //    once, at the end.
 //
@@ -183,13 +185,14 @@ template <int D, int NH>
 struct McShape {
     static_assert(D == 128 && (NH == 32 || NH == 64), "the tensor-core decode kernel: D = 128, 32 or 64 heads");
     static constexpr int kTok = 128;  // tokens per tile (TMEM lanes of S^T)
-    static constexpr int kChunks = NH / 32;  // softmax passes of 32 heads
+    static constexpr int kGroups = NH / 32;  // softmax groups of 4 warps, 32 heads each
     // K and V ring depths: 3 + 3 stages of 32 KB; at 64 heads the Q and P buffers double and
     // the K ring keeps 2 (gqa48: K 2 + V 3 measured 61.6-62.1 us, K 3 + V 2 62.4-62.7 us)
     static constexpr int kKStages = NH == 32 ? 3 : 2, kVStages = 3;
-    static constexpr int kSoftmaxWarps = 4;
-    static constexpr int kProducerWarp = 4, kMmaWarp = 5, kVProducerWarp = 6;
-    static constexpr int kThreads = 32 * 7;
+    static constexpr int kSoftmaxWarps = 4 * kGroups;
+    static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1,
+                         kVProducerWarp = kSoftmaxWarps + 2;
+    static constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
     static constexpr uint32_t kQBytes = NH * D * 2;
     static constexpr uint32_t kKVBytes = kTok * D * 2;  // one K (or V) tile
     static constexpr uint32_t kPBytes = kTok * NH * 2;
@@ -198,9 +201,9 @@ struct McShape {
     static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
     static constexpr uint32_t kPOff = kVOff + kVStages * kKVBytes;
     static constexpr uint32_t kTileBytes = kPOff + 2 * kPBytes;  // two P buffers
-    // 2 KB header (mbarriers, TMEM address, abort flag, the per-warp head maxima and sums),
+    // 3 KB header (mbarriers, TMEM address, abort flag, the per-warp head maxima and sums),
     // up to 1 KB to reach 1024-byte alignment, then the tiles
-    static constexpr uint32_t kHeaderBytes = 2048;
+    static constexpr uint32_t kHeaderBytes = 3072;
     static constexpr uint32_t kRedOff = 512;
     static constexpr uint32_t kSmemBytes = kHeaderBytes + 1024 + kTileBytes;
     static constexpr uint32_t kTmemCols = NH == 32 ? 128 : 256;
@@ -211,7 +214,7 @@ struct McShape {
     // [kMcMaxCluster + 1][NH] in its Q buffer
     static_assert(NH * D * 4 + NH * 8 <= kKStages * kKVBytes, "part in the K ring");
     static_assert((kMcMaxCluster + 1) * NH * 4 <= kQBytes, "merge weights in the Q buffer");
-    static_assert(kRedOff + 4 * 32 * 4 + 4 * NH * 4 <= kHeaderBytes, "header");
+    static_assert(kRedOff + kGroups * 4 * 32 * 4 + 4 * NH * 4 + NH * 4 <= kHeaderBytes, "header");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the TMEM columns are always free");
 };
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     using T = McShape<D, NH>;
     using O = OperandGeom<D>;   // K, V and Q staging: D/64 blocks of [rows][64]
     using PG = OperandGeom<NH>; // P staging: [tokens][NH] rows of 2 NH bytes
-    constexpr int TK = T::kTok, KST = T::kKStages, VST = T::kVStages, NC = T::kChunks;
+    constexpr int TK = T::kTok, KST = T::kKStages, VST = T::kVStages, NG = T::kGroups;
     constexpr uint32_t kIdescQK = mc_idesc(TK, NH, false, false);
     constexpr uint32_t kIdescPV = mc_idesc(D, NH, true, true);
     // mbarriers; S, P and PVDone come in pairs, one per S / P buffer (tile parity)
@@ -231,7 +234,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     constexpr int kSFull = 1 + 2 * (KST + VST), kSFree = kSFull + 2, kPFull = kSFull + 4, kPVDone = kSFull + 6;
     constexpr int kDrain = kSFull + 8, kParts = kSFull + 9, kBars = kSFull + 10;
     constexpr int kSoftThreads = 32 * T::kSoftmaxWarps;
-    constexpr int kBarId = 1;  // named barrier of the softmax warps
+    // named barriers: 1 + g for the 4 warps of softmax group g, kAllBarId for all of them
+    constexpr int kAllBarId = 1 + NG;
     static_assert(8 * kBars + 8 <= static_cast<int>(T::kRedOff), "barrier area");
 
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -239,8 +243,9 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * kBars);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + 8 * kBars + 4);
-    float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [4 warps][32] head maxima
-    float* s_sum = s_red + 4 * 32;                                // [4 warps][NH] head sums
+    float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [group][4 warps][32] head maxima
+    float* s_sum = s_red + NG * 4 * 32;                           // [4 warps][NH] head sums
+    float* s_m = s_sum + 4 * NH;                                  // [NH] the heads' reference maxima
     const uint32_t tb = (bar0 + T::kHeaderBytes + 1023u) & ~1023u;
     const uint32_t q_s = tb + T::kQOff, p_s = tb + T::kPOff;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -337,8 +342,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     bool ok = true;
     bool cluster_waited = false;  // this thread has waited for cluster phase 0
     if (warp == T::kProducerWarp || warp == T::kVProducerWarp) {
-        // ================= producers: TMA loads of the K tiles (warp 4) or the V tiles
-        // (warp 6), four 32-token boxes each
+        // ================= producers: TMA loads of the K tiles or the V tiles, four 32-token
+        // boxes each
         const int kv = warp == T::kVProducerWarp ? 1 : 0;
         const CUtensorMap* map = kv ? &vmap : &kmap;
         const int full0 = kv ? kVFull : kKFull, empty0 = kv ? kVEmpty : kKEmpty;
@@ -462,9 +467,13 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             }
         }
     } else {
-        // ================= softmax warps: thread r owns token r of each tile (TMEM lane r)
-        const int r = 32 * warp + lane;
-        const uint32_t t_lane = static_cast<uint32_t>(32 * warp) << 16;
+        // ================= softmax warps: group grp (warps 4 grp .. 4 grp + 3) owns heads
+        // [32 grp, 32 grp + 32); thread r of a group owns token r of each tile (TMEM lane r)
+        const int grp = warp >> 2, wq = warp & 3;
+        const int r = 32 * wq + lane;
+        const int hoff = 32 * grp;
+        const int gbar = 1 + grp;  // this group's named barrier
+        const uint32_t t_lane = static_cast<uint32_t>(32 * wq) << 16;
         // Q rows kvh * g + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at and past
         // g (padding up to NH) are zeros.  A thread's loads are all issued before its stores.
         {
@@ -491,82 +500,77 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(bar(kQFull));
 
-        float m[NH];  // reference maximum of each head (log2 domain), the same in every thread
-        float l[NH];  // this thread's sums of the bf16 weights, relative to m
+        // the reference maximum of each of the group's heads (log2 domain) lives in shared
+        // memory (the same for every thread of the group; written only when it moves)
+        float* const g_m = s_m + hoff;
+        if (wq == 0) g_m[lane] = -INFINITY;
+        bar_named(gbar, 128);
+        auto load_m = [&](float (&mv)[32]) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            m[h] = -INFINITY;
-            l[h] = 0.f;
-        }
-        // scores of heads [32 c, 32 c + 32) of this thread's token in S buffer sb, scaled to the
-        // log2 domain; -inf past the split's last token
-        auto load_x = [&](int c, int sb, bool valid, float (&x)[32]) {
-            uint32_t sr[32];
-            tc_ld32(tmem + t_lane + T::kColS + static_cast<uint32_t>(sb * NH + 32 * c), sr);
-            tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+            for (int i = 0; i < 32; i += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(g_m + i);
+                mv[i] = a.x;
+                mv[i + 1] = a.y;
+                mv[i + 2] = a.z;
+                mv[i + 3] = a.w;
+            }
         };
+        float l[32];  // this thread's sums of the bf16 weights, relative to the reference
+#pragma unroll
+        for (int i = 0; i < 32; ++i) l[i] = 0.f;
+        float* const g_red = s_red + grp * 4 * 32;  // this group's [4 warps][32] maxima
         bool wok = true, stopped = false;
         for (int j = 0; j < ntiles; ++j) {
             const int sb = j & 1;
-            const bool valid = tok0 + j * TK + r < tok1;
-            float x0[32];  // the scores of chunk 0, kept when there is only one chunk
-            bool need = false;
+            float x[32];
             wok = warp_wait(bar(kSFull + sb), static_cast<uint32_t>(j >> 1) & 1u, p.wait_ns, abort_flag,
                             p.flags);
             if (wok) {
+                uint32_t sr[32];
                 tc_fence_after();
+                tc_ld32(tmem + t_lane + T::kColS + static_cast<uint32_t>(sb * NH + hoff), sr);
+                tc_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
+                const bool valid = tok0 + j * TK + r < tok1;
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    float x[32];
-                    load_x(c, sb, valid, x);
+                for (int i = 0; i < 32; ++i) x[i] = valid ? __uint_as_float(sr[i]) * p.scale_log2 : -INFINITY;
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) need |= x[i] > m[32 * c + i] + 8.f;
-                    if constexpr (NC == 1) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) x0[i] = x[i];
-                    }
-                }
-                if constexpr (NC == 1) {
-                    tc_fence_before();
-                    mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
-                }
+                for (int i = 0; i < 32; ++i) x[i] = -INFINITY;
             }
-            // one vote per tile: a new reference for some head, or some warp gave up
+            bool need = false;
+            {
+                float m[32];
+                load_m(m);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) need |= x[i] > m[i] + 8.f;
+            }
+            // one vote per tile and group: a new reference for some head, or some warp gave up
             const bool gave_up = !wok || *abort_flag != 0u;
-            if (bar_any(kBarId, kSoftThreads, need || gave_up)) {
-                if (bar_any(kBarId, kSoftThreads, gave_up)) {
+            if (bar_any(gbar, 128, need || gave_up)) {
+                if (bar_any(gbar, 128, gave_up)) {
                     stopped = true;
                     break;
                 }
-                // ---- new reference: the tile's maximum of each head over the 128 tokens,
-                // 32 heads at a time; O^T columns of the heads whose reference moved rescaled
-                if (j > 0) {
-                    // O^T holds P V of the earlier tiles: rescale once the last P V has landed
-                    // (in issue order, so every earlier one has too)
-                    wok = warp_wait(bar(kPVDone + ((j - 1) & 1)), static_cast<uint32_t>((j - 1) >> 1) & 1u,
-                                    p.wait_ns, abort_flag, p.flags);
-                }
+                // ---- new reference: the tile's maximum of each head over the 128 tokens
+                float v[32];
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    float v[32];
-                    if constexpr (NC == 1) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = x0[i];
-                    } else {
-                        load_x(c, sb, valid, v);
-                    }
-                    warp_reduce_scatter32<true>(v, lane);
-                    s_red[warp * 32 + lane] = v[0];
-                    bar_named(kBarId, kSoftThreads);
-                    float alpha[32];
+                for (int i = 0; i < 32; ++i) v[i] = x[i];
+                warp_reduce_scatter32<true>(v, lane);
+                g_red[wq * 32 + lane] = v[0];
+                bar_named(gbar, 128);
+                float alpha[32];
+                float mnew = 0.f;  // lane i: the new reference of head i
+                {
+                    float m[32];
+                    load_m(m);
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
-                        float4 a = *reinterpret_cast<const float4*>(s_red + i);
+                        float4 a = *reinterpret_cast<const float4*>(g_red + i);
 #pragma unroll
                         for (int w = 1; w < 4; ++w) {
-                            const float4 q = *reinterpret_cast<const float4*>(s_red + w * 32 + i);
+                            const float4 q = *reinterpret_cast<const float4*>(g_red + w * 32 + i);
                             a.x = fmaxf(a.x, q.x);
                             a.y = fmaxf(a.y, q.y);
                             a.z = fmaxf(a.z, q.z);
@@ -575,54 +579,52 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                         const float tm[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            const int h = 32 * c + i + e;
-                            const float mn = fmaxf(m[h], tm[e]);
+                            const float mn = fmaxf(m[i + e], tm[e]);
                             // 1 for a head whose maximum did not move; 0 while m is -inf
-                            alpha[i + e] = (mn == m[h]) ? 1.f : ex2_approx(m[h] - mn);
-                            m[h] = mn;
-                            l[h] *= alpha[i + e];
+                            alpha[i + e] = (mn == m[i + e]) ? 1.f : ex2_approx(m[i + e] - mn);
+                            if (lane == i + e) mnew = mn;
+                            l[i + e] *= alpha[i + e];
                         }
                     }
-                    if (j > 0 && wok) {
+                }
+                bar_named(gbar, 128);  // every thread has read the old references
+                if (wq == 0) g_m[lane] = mnew;
+                bar_named(gbar, 128);  // the new references are visible to the group
+                if (j > 0) {
+                    // O^T holds P V of the earlier tiles: rescale this thread's row (head dim
+                    // r) in the group's columns once the last P V has landed (in issue order,
+                    // so every earlier one has too)
+                    wok = warp_wait(bar(kPVDone + ((j - 1) & 1)), static_cast<uint32_t>((j - 1) >> 1) & 1u,
+                                    p.wait_ns, abort_flag, p.flags);
+                    if (wok) {
                         tc_fence_after();
                         uint32_t o[32];
-                        const uint32_t oa = tmem + t_lane + T::kColO + static_cast<uint32_t>(32 * c);
+                        const uint32_t oa = tmem + t_lane + T::kColO + static_cast<uint32_t>(hoff);
                         tc_ld32(oa, o);
                         tc_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[i]);
                         tc_st32(oa, o);
+                        tc_wait_st();
                     }
-                    bar_named(kBarId, kSoftThreads);  // s_red is read by every thread before its next use
                 }
-                if (j > 0 && wok) tc_wait_st();
             }
-            if (!wok) continue;  // gave up in this tile: the next vote stops every warp
+            if (!wok) continue;  // gave up in this tile: the next vote stops every warp of the group
 
             // ---- P = 2^(x - m) as bf16 pairs, and the sums of exactly those weights
-            uint32_t pw[NH / 2];
+            uint32_t pw[16];
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                float x[32];
-                if constexpr (NC == 1) {
+            for (int i = 0; i < 16; i += 2) {
+                const float4 mv = *reinterpret_cast<const float4*>(g_m + 2 * i);
+                const float m4[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = x0[i];
-                } else {
-                    load_x(c, sb, valid, x);
+                for (int e = 0; e < 2; ++e) {
+                    const float p0 = ex2_approx(x[2 * (i + e)] - m4[2 * e]);
+                    const float p1 = ex2_approx(x[2 * (i + e) + 1] - m4[2 * e + 1]);
+                    pw[i + e] = pack_bf16x2(p0, p1);
+                    l[2 * (i + e)] += bf16_lo(pw[i + e]);
+                    l[2 * (i + e) + 1] += bf16_hi(pw[i + e]);
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int h = 32 * c + 2 * i;
-                    const float p0 = ex2_approx(x[2 * i] - m[h]);
-                    const float p1 = ex2_approx(x[2 * i + 1] - m[h + 1]);
-                    pw[16 * c + i] = pack_bf16x2(p0, p1);
-                    l[h] += bf16_lo(pw[16 * c + i]);
-                    l[h + 1] += bf16_hi(pw[16 * c + i]);
-                }
-            }
-            if constexpr (NC > 1) {
-                tc_fence_before();
-                mbar_arrive(bar(kSFree + sb));  // the S buffer may take tile j + 2
             }
             // ---- P buffer j & 1 is free once P_{j-2} V_{j-2} has completed
             if (j > 1) {
@@ -631,12 +633,13 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                 if (!wok) continue;
                 tc_fence_after();
             }
-            // row r of P^T ([token][head], 2 NH bytes, swizzled as the MN-major B layout)
+            // the group's 64 bytes of row r of P^T ([token][head], 2 NH bytes, swizzled as the
+            // MN-major B layout)
             const uint32_t pb = p_s + static_cast<uint32_t>((j & 1) * T::kPBytes);
 #pragma unroll
-            for (int c = 0; c < NH / 8; ++c)
-                st_shared_v4(pb + static_cast<uint32_t>(r * PG::kRowBytes + (PG::swz(r, c) << 4)), pw[4 * c],
-                             pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            for (int q = 0; q < 4; ++q)
+                st_shared_v4(pb + static_cast<uint32_t>(r * PG::kRowBytes + (PG::swz(r, 4 * grp + q) << 4)),
+                             pw[4 * q], pw[4 * q + 1], pw[4 * q + 2], pw[4 * q + 3]);
             // ---- last tile: V rows past the split's last token hold anything (NaN included,
             // or nothing loaded): zero them before they meet a zero weight
             if (j == ntiles - 1 && tok0 + j * TK + TK > tok1) {
@@ -656,25 +659,33 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         if (!stopped && wok)
             wok = warp_wait(bar(kPVDone + ((ntiles - 1) & 1)), static_cast<uint32_t>((ntiles - 1) >> 1) & 1u,
                             p.wait_ns, abort_flag, p.flags);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
+        {
             float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = l[32 * c + i];
+            for (int i = 0; i < 32; ++i) v[i] = l[i];
             warp_reduce_scatter32<false>(v, lane);
-            s_sum[warp * NH + 32 * c + lane] = v[0];
+            s_sum[wq * NH + hoff + lane] = v[0];
         }
         const bool gave_up = stopped || !wok || *abort_flag != 0u;
-        const bool any_gave_up = bar_any(kBarId, kSoftThreads, gave_up);
+        const bool any_gave_up = bar_any(gbar, 128, gave_up);
         const int dd = r;  // this thread's head-dim column of O (TMEM lane of O^T)
-        // sum over the four softmax warps of the heads' sums, heads [32 c, 32 c + 32)
-        auto sums = [&](int c, float (&lt)[32]) {
+        uint32_t o[32];
+        float lt[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            o[i] = 0u;
+            lt[i] = 0.f;
+        }
+        if (!any_gave_up) {
+            tc_fence_after();
+            tc_ld32(tmem + t_lane + T::kColO + static_cast<uint32_t>(hoff), o);
+            tc_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
-                float4 a = *reinterpret_cast<const float4*>(s_sum + 32 * c + i);
+                float4 a = *reinterpret_cast<const float4*>(s_sum + hoff + i);
 #pragma unroll
                 for (int w = 1; w < 4; ++w) {
-                    const float4 q = *reinterpret_cast<const float4*>(s_sum + w * NH + 32 * c + i);
+                    const float4 q = *reinterpret_cast<const float4*>(s_sum + w * NH + hoff + i);
                     a.x += q.x;
                     a.y += q.y;
                     a.z += q.z;
@@ -685,69 +696,41 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                 lt[i + 2] = a.z;
                 lt[i + 3] = a.w;
             }
-        };
-        auto load_o = [&](int c, uint32_t (&o)[32]) {
-            tc_ld32(tmem + t_lane + T::kColO + static_cast<uint32_t>(32 * c), o);
-            tc_wait_ld();
-        };
-        // m and l of head 32 c + lane, for warp 0's writes of (m, l) pairs
-        auto head_ml = [&](int c, const float (&lt)[32], float& mm, float& ll) {
-            mm = 0.f;
-            ll = 0.f;
+        }
+        // m and l of the group's head `lane`, for the writes of (m, l) pairs
+        const float mm = g_m[lane];
+        float ll = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                if (lane == i) {
-                    mm = m[32 * c + i];
-                    ll = lt[i];
-                }
-            }
-        };
+        for (int i = 0; i < 32; ++i)
+            if (lane == i) ll = lt[i];
         if (nk == 1) {
             // the only non-empty split: normalised rows straight to out
             if (!any_gave_up) {
-                tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    uint32_t o[32];
-                    float lt[32];
-                    load_o(c, o);
-                    sums(c, lt);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int h = 32 * c + i;
-                        if (h < p.g)
-                            p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
-                                __float2bfloat16_rn(__uint_as_float(o[i]) / lt[i]);
-                    }
+                for (int i = 0; i < 32; ++i) {
+                    const int h = hoff + i;
+                    if (h < p.g)
+                        p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                            __float2bfloat16_rn(__uint_as_float(o[i]) / lt[i]);
                 }
             }
         } else if (!p.cluster) {
             if (!any_gave_up) {
                 // the partial of this split, for each head block of 16 heads: slot
                 // ((b * Hkv + kvh) * HB + hb) * ksplit + split, row h - 16 hb
-                tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < NC; ++c) {
-                    uint32_t o[32];
-                    float lt[32];
-                    load_o(c, o);
-                    sums(c, lt);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int h = 32 * c + i;
-                        if (h < p.g) {
-                            const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
-                            p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[i]);
-                        }
-                    }
-                    if (warp == 0 && 32 * c + lane < p.g) {
-                        float mm, ll;
-                        head_ml(c, lt, mm, ll);
-                        const int h = 32 * c + lane;
+                for (int i = 0; i < 32; ++i) {
+                    const int h = hoff + i;
+                    if (h < p.g) {
                         const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
-                        *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + h % kMaxRows) * 2) =
-                            make_float2(mm, ll);
+                        p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[i]);
                     }
+                }
+                if (wq == 0 && hoff + lane < p.g) {
+                    const int h = hoff + lane;
+                    const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
+                    *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + h % kMaxRows) * 2) =
+                        make_float2(mm, ll);
                 }
             }
         } else {
@@ -756,87 +739,71 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             float* const part_p = reinterpret_cast<float*>(smem + (tb + T::kKOff - bar0));
             cluster_wait();  // phase 0: every CTA of the cluster has its mbarriers initialised
             cluster_waited = true;
-            if (!any_gave_up) tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < NC; ++c) {
-                uint32_t o[32];
-                float lt[32];
-                if (!any_gave_up) {
-                    load_o(c, o);
-                    sums(c, lt);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        o[i] = 0u;
-                        lt[i] = 0.f;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) part_p[(32 * c + i) * D + dd] = __uint_as_float(o[i]);
-                if (warp == 0) {
-                    float mm, ll;
-                    head_ml(c, lt, mm, ll);
-                    part_p[NH * D + 2 * (32 * c + lane)] = mm;
-                    part_p[NH * D + 2 * (32 * c + lane) + 1] = ll;
-                }
+            for (int i = 0; i < 32; ++i) part_p[(hoff + i) * D + dd] = __uint_as_float(o[i]);
+            if (wq == 0) {
+                part_p[NH * D + 2 * (hoff + lane)] = mm;
+                part_p[NH * D + 2 * (hoff + lane) + 1] = ll;
             }
             fence_acq_rel_cluster();
-            bar_named(kBarId, kSoftThreads);
+            bar_named(kAllBarId, kSoftThreads);  // both groups' halves of the part are written
             // tell every other CTA of the cluster that this part is ready
             if (threadIdx.x < nsplit && threadIdx.x != split) mbar_arrive_remote(dsmem_addr(bar(kParts), threadIdx.x));
-            // this split merges heads h = split + j nk (j < nh) of every part:
-            // w_s = 2^(m_s - M) over the non-empty parts, out = sum_s w_s O_s / sum_s w_s l_s
-            const int nh = (NH - split + nk - 1) / nk;
-            const bool pok = warp_wait_cluster(bar(kParts), 0u, p.wait_ns, abort_flag, p.flags);
-            float* const wts = reinterpret_cast<float*>(smem + (q_s - bar0));  // [kMcMaxCluster + 1][NH]
-            if (warp == 0 && pok && lane < nh) {
-                const int h = split + lane * nk;
-                float ms[kMcMaxCluster], ls[kMcMaxCluster];
+            if (grp == 0) {
+                // group 0 merges heads h = split + j nk (j < nh) of every part:
+                // w_s = 2^(m_s - M) over the non-empty parts, out = sum_s w_s O_s / sum_s w_s l_s
+                const int nh = (NH - split + nk - 1) / nk;
+                const bool pok = warp_wait_cluster(bar(kParts), 0u, p.wait_ns, abort_flag, p.flags);
+                float* const wts = reinterpret_cast<float*>(smem + (q_s - bar0));  // [kMcMaxCluster + 1][NH]
+                if (wq == 0 && pok && lane < nh) {
+                    const int h = split + lane * nk;
+                    float ms[kMcMaxCluster], ls[kMcMaxCluster];
 #pragma unroll
-                for (int s = 0; s < kMcMaxCluster; ++s) {
-                    ms[s] = -INFINITY;
-                    ls[s] = 0.f;
-                    if (s < nk) {
-                        const float* q = dsmem_ptr(part_p + NH * D + 2 * h, static_cast<uint32_t>(s));
-                        ms[s] = q[0];
-                        ls[s] = q[1];
+                    for (int s = 0; s < kMcMaxCluster; ++s) {
+                        ms[s] = -INFINITY;
+                        ls[s] = 0.f;
+                        if (s < nk) {
+                            const float* q = dsmem_ptr(part_p + NH * D + 2 * h, static_cast<uint32_t>(s));
+                            ms[s] = q[0];
+                            ls[s] = q[1];
+                        }
                     }
-                }
-                float M = -INFINITY;
+                    float M = -INFINITY;
 #pragma unroll
-                for (int s = 0; s < kMcMaxCluster; ++s)
-                    if (ls[s] > 0.f) M = fmaxf(M, ms[s]);
-                float den = 0.f;
+                    for (int s = 0; s < kMcMaxCluster; ++s)
+                        if (ls[s] > 0.f) M = fmaxf(M, ms[s]);
+                    float den = 0.f;
 #pragma unroll
-                for (int s = 0; s < kMcMaxCluster; ++s) {
-                    const float w = ls[s] > 0.f ? exp2f(ms[s] - M) : 0.f;
-                    wts[s * NH + lane] = w;
-                    den += w * ls[s];
-                }
-                wts[kMcMaxCluster * NH + lane] = den > 0.f ? 1.f / den : 0.f;
-            }
-            if (!bar_any(kBarId, kSoftThreads, !pok || any_gave_up)) {
-                constexpr int kMaxH = NH / 2;  // heads per split when nk = 2
-                float acc[kMaxH];
-#pragma unroll
-                for (int j = 0; j < kMaxH; ++j) acc[j] = 0.f;
-#pragma unroll
-                for (int s = 0; s < kMcMaxCluster; ++s) {
-                    if (s < nk) {  // the loads of all parts can be in flight together
-                        const float* src = dsmem_ptr(part_p + dd, static_cast<uint32_t>(s));
-                        float v[kMaxH];
-#pragma unroll
-                        for (int j = 0; j < kMaxH; ++j) v[j] = j < nh ? src[(split + j * nk) * D] : 0.f;
-#pragma unroll
-                        for (int j = 0; j < kMaxH; ++j) acc[j] += wts[s * NH + j] * v[j];
+                    for (int s = 0; s < kMcMaxCluster; ++s) {
+                        const float w = ls[s] > 0.f ? exp2f(ms[s] - M) : 0.f;
+                        wts[s * NH + lane] = w;
+                        den += w * ls[s];
                     }
+                    wts[kMcMaxCluster * NH + lane] = den > 0.f ? 1.f / den : 0.f;
                 }
+                if (!bar_any(gbar, 128, !pok || any_gave_up)) {
+                    constexpr int kMaxH = NH / 2;  // heads per split when nk = 2
+                    float acc[kMaxH];
 #pragma unroll
-                for (int j = 0; j < kMaxH; ++j) {
-                    const int h = split + j * nk;
-                    if (j < nh && h < p.g)
-                        p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
-                            __float2bfloat16_rn(acc[j] * wts[kMcMaxCluster * NH + j]);
+                    for (int jj = 0; jj < kMaxH; ++jj) acc[jj] = 0.f;
+#pragma unroll
+                    for (int s = 0; s < kMcMaxCluster; ++s) {
+                        if (s < nk) {  // the loads of all parts can be in flight together
+                            const float* src = dsmem_ptr(part_p + dd, static_cast<uint32_t>(s));
+                            float v[kMaxH];
+#pragma unroll
+                            for (int jj = 0; jj < kMaxH; ++jj) v[jj] = jj < nh ? src[(split + jj * nk) * D] : 0.f;
+#pragma unroll
+                            for (int jj = 0; jj < kMaxH; ++jj) acc[jj] += wts[s * NH + jj] * v[jj];
+                        }
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < kMaxH; ++jj) {
+                        const int h = split + jj * nk;
+                        if (jj < nh && h < p.g)
+                            p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                                __float2bfloat16_rn(acc[jj] * wts[kMcMaxCluster * NH + jj]);
+                    }
                 }
             }
         }

@@ -277,20 +277,20 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
 
 
 def _mc_smem(nh):
-    """Shared memory of the tensor-core multi-query kernel: 2 KB header, 1 KB of alignment
+    """Shared memory of the tensor-core multi-query kernel: 3 KB header, 1 KB of alignment
     slack, Q [nh][128], 3 (nh = 32) or 2 (nh = 64) K stages and 3 V stages of 128 tokens x
     128, two P buffers [128][nh] (bf16)."""
     k_stages = 3 if nh == 32 else 2
-    return 2048 + 1024 + nh * 128 * 2 + (k_stages + 3) * 128 * 128 * 2 + 2 * 128 * nh * 2
+    return 3072 + 1024 + nh * 128 * 2 + (k_stages + 3) * 128 * 128 * 2 + 2 * 128 * nh * 2
 
 
 @pytest.mark.parametrize("g", [32, 20, 48, 64])
 @pytest.mark.parametrize("B,Hkv,sm", [(16, 2, 148), (1, 1, 148), (4, 8, 148), (200, 1, 148), (3, 2, 132), (16, 2, 8)])
 def test_plan_tensor_core_multi_query(B, Hkv, sm, g):
     """17 to 64 q heads per kv head at D = 128: the tensor-core multi-query kernel (heads
-    padded to 32 or 64), one CTA per split of each (sequence, kv head), 7 warps (4 softmax,
-    2 producers, 1 MMA issuer), K and V rings of 128-token stages, Q and two P buffers in
-    shared memory.  Auto splits
+    padded to 32 or 64), one CTA per split of each (sequence, kv head), 7 or 11 warps (4
+    softmax warps per 32 heads, 2 producers, 1 MMA issuer), K and V rings of 128-token
+    stages, Q and two P buffers in shared memory.  Auto splits
     spread the units over 7/8 of the SMs.  A unit's splits (up to 8) that the device can run
     as one cluster merge over DSMEM in the kernel; otherwise their partials take the
     fixed-split slots of both head blocks and the combine kernel merges them.  The slots are
@@ -302,7 +302,8 @@ def test_plan_tensor_core_multi_query(B, Hkv, sm, g):
     k = max(1, sm * 7 // 8 // (B * Hkv))
     assert pl.mode == 3 and pl.shared_kv_ring == 0
     assert pl.grid_ctas == B * Hkv * k and pl.num_workers == pl.grid_ctas
-    assert pl.warps_per_cta == 7 and pl.stages == 3
+    # a softmax group of 4 warps per 32 heads, 2 producer warps and the MMA issuer's warp
+    assert pl.warps_per_cta == 4 * (nh // 32) + 3 and pl.stages == 3
     assert pl.smem_bytes == _mc_smem(nh) <= 232448
     assert pl.rows_per_unit == 16 and pl.head_blocks == -(-g // 16)
     assert pl.partial_slots == (units * k if k > 1 else 0)
@@ -670,6 +671,8 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
     hb = -(-g // 16)
     pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=sm, host_seq_lens=[L] * B, max_seq_len=70000)
     bound = {32: 12, 64: 10}.get(D, 8) if not pl.shared_kv_ring else 8
+    if pl.mode == 3:
+        bound = 11  # the tensor-core kernel at 64 heads: 2 softmax groups + 3 warps
     assert pl.smem_bytes <= 232448
     assert 1 <= pl.warps_per_cta <= bound
     assert pl.grid_ctas * pl.warps_per_cta >= pl.num_workers > 0
