@@ -27,8 +27,9 @@
 //    own stage is free: a K stage right after its S^T product, a V stage after its P V.
 //    One lane of the warp between them issues the MMAs, each product as soon as its operands
 //    are ready (S^T_j does not wait for P_{j-1} V_{j-1}, nor that for the next K tile), and
-//    commits them to the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T and two
-//    P buffers let the softmax of tile j + 1 run while P_j V_j is on the tensor core.
+//    commits them to the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T
+//    buffers (and at 32 heads two P buffers) let the softmax of tile j + 1 run while P_j V_j
+//    is on the tensor core.
 //  - Softmax warps, one group of 4 per 32 heads (warps 0-3, and 4-7 at 64 heads): TMEM lane t
 //    is token t of the tile, so thread t of a group reads its token's 32 scores of the
 //    group's heads with one tcgen05.ld and owns those exponentials.  The reference
@@ -186,9 +187,11 @@ struct McShape {
     static_assert(D == 128 && (NH == 32 || NH == 64), "the tensor-core decode kernel: D = 128, 32 or 64 heads");
     static constexpr int kTok = 128;  // tokens per tile (TMEM lanes of S^T)
     static constexpr int kGroups = NH / 32;  // softmax groups of 4 warps, 32 heads each
-    // K and V ring depths: 3 + 3 stages of 32 KB; at 64 heads the Q and P buffers double and
-    // the K ring keeps 2 (gqa48: K 2 + V 3 measured 61.6-62.1 us, K 3 + V 2 62.4-62.7 us)
-    static constexpr int kKStages = NH == 32 ? 3 : 2, kVStages = 3;
+    // K and V ring depths: 3 + 3 stages of 32 KB.  At 64 heads Q and P double, and the third
+    // K stage fits only with one P buffer (the 2-stage K ring bounded the tile period there:
+    // traced 1.38 us against 1.18 us at 32 heads)
+    static constexpr int kKStages = 3, kVStages = 3;
+    static constexpr int kPBuffers = NH == 32 ? 2 : 1;
     static constexpr int kSoftmaxWarps = 4 * kGroups;
     static constexpr int kProducerWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1,
                          kVProducerWarp = kSoftmaxWarps + 2;
@@ -200,10 +203,11 @@ struct McShape {
     static constexpr uint32_t kKOff = kQBytes;
     static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
     static constexpr uint32_t kPOff = kVOff + kVStages * kKVBytes;
-    static constexpr uint32_t kTileBytes = kPOff + 2 * kPBytes;  // two P buffers
-    // 3 KB header (mbarriers, TMEM address, abort flag, the per-warp head maxima and sums),
-    // up to 1 KB to reach 1024-byte alignment, then the tiles
-    static constexpr uint32_t kHeaderBytes = 3072;
+    static constexpr uint32_t kTileBytes = kPOff + kPBuffers * kPBytes;
+    // header (mbarriers, TMEM address, abort flag, the per-warp head maxima and the reference
+    // maxima), up to 1 KB to reach 1024-byte alignment, then the tiles.  The per-warp head
+    // sums of the epilogue go to the second half of the Q buffer, idle by then.
+    static constexpr uint32_t kHeaderBytes = NH == 32 ? 2048 : 1792;
     static constexpr uint32_t kRedOff = 512;
     static constexpr uint32_t kSmemBytes = kHeaderBytes + 1024 + kTileBytes;
     static constexpr uint32_t kTmemCols = NH == 32 ? 128 : 256;
@@ -214,7 +218,9 @@ struct McShape {
     // [kMcMaxCluster + 1][NH] in its Q buffer
     static_assert(NH * D * 4 + NH * 8 <= kKStages * kKVBytes, "part in the K ring");
     static_assert((kMcMaxCluster + 1) * NH * 4 <= kQBytes, "merge weights in the Q buffer");
-    static_assert(kRedOff + kGroups * 4 * 32 * 4 + 4 * NH * 4 + NH * 4 <= kHeaderBytes, "header");
+    static_assert(kRedOff + kGroups * 4 * 32 * 4 + NH * 4 <= kHeaderBytes, "header");
+    static_assert(4 * NH * 4 <= kQBytes / 2 && (kMcMaxCluster + 1) * NH * 4 <= kQBytes / 2,
+                  "epilogue sums and merge weights in the two halves of the Q buffer");
     static_assert(kSmemBytes <= 232448, "shared memory per CTA");
     static_assert(kSmemBytes > 232448 / 2, "one CTA per SM, so the TMEM columns are always free");
 };
@@ -244,9 +250,10 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + 8 * kBars);
     volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + 8 * kBars + 4);
     float* s_red = reinterpret_cast<float*>(smem + T::kRedOff);  // [group][4 warps][32] head maxima
-    float* s_sum = s_red + NG * 4 * 32;                           // [4 warps][NH] head sums
-    float* s_m = s_sum + 4 * NH;                                  // [NH] the heads' reference maxima
+    float* s_m = s_red + NG * 4 * 32;                             // [NH] the heads' reference maxima
     const uint32_t tb = (bar0 + T::kHeaderBytes + 1023u) & ~1023u;
+    // [4 warps][NH] head sums, written in the epilogue once every S^T product is done
+    float* s_sum = reinterpret_cast<float*>(smem + (tb + T::kQOff + T::kQBytes / 2 - bar0));
     const uint32_t q_s = tb + T::kQOff, p_s = tb + T::kPOff;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -434,7 +441,7 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                     tc_fence_after();
                     // O^T += V_jp^T P_jp^T, K = TK tokens in steps of 16
                     const uint32_t vb = tb + T::kVOff + static_cast<uint32_t>(jp % VST) * T::kKVBytes;
-                    const uint32_t pb = p_s + static_cast<uint32_t>((jp & 1) * T::kPBytes);
+                    const uint32_t pb = p_s + static_cast<uint32_t>((jp % T::kPBuffers) * T::kPBytes);
 #pragma unroll
                     for (int k = 0; k < TK / 16; ++k)
                         tc_mma_bf16(tmem + T::kColO,
@@ -626,16 +633,21 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
                     l[2 * (i + e) + 1] += bf16_hi(pw[i + e]);
                 }
             }
-            // ---- P buffer j & 1 is free once P_{j-2} V_{j-2} has completed
-            if (j > 1) {
-                wok = warp_wait(bar(kPVDone + (j & 1)), static_cast<uint32_t>((j - 2) >> 1) & 1u, p.wait_ns,
-                                abort_flag, p.flags);
-                if (!wok) continue;
-                tc_fence_after();
+            // ---- the P buffer of tile j is free once P V of the tile before that used it has
+            // completed: j - 2 with two buffers, j - 1 with one
+            {
+                constexpr int kBack = T::kPBuffers;
+                if (j >= kBack) {
+                    const int jb = j - kBack;
+                    wok = warp_wait(bar(kPVDone + (jb & 1)), static_cast<uint32_t>(jb >> 1) & 1u, p.wait_ns,
+                                    abort_flag, p.flags);
+                    if (!wok) continue;
+                    tc_fence_after();
+                }
             }
             // the group's 64 bytes of row r of P^T ([token][head], 2 NH bytes, swizzled as the
             // MN-major B layout)
-            const uint32_t pb = p_s + static_cast<uint32_t>((j & 1) * T::kPBytes);
+            const uint32_t pb = p_s + static_cast<uint32_t>((j % T::kPBuffers) * T::kPBytes);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 st_shared_v4(pb + static_cast<uint32_t>(r * PG::kRowBytes + (PG::swz(r, 4 * grp + q) << 4)),

@@ -277,11 +277,11 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
 
 
 def _mc_smem(nh):
-    """Shared memory of the tensor-core multi-query kernel: 3 KB header, 1 KB of alignment
-    slack, Q [nh][128], 3 (nh = 32) or 2 (nh = 64) K stages and 3 V stages of 128 tokens x
-    128, two P buffers [128][nh] (bf16)."""
-    k_stages = 3 if nh == 32 else 2
-    return 3072 + 1024 + nh * 128 * 2 + (k_stages + 3) * 128 * 128 * 2 + 2 * 128 * nh * 2
+    """Shared memory of the tensor-core multi-query kernel: the header (2 KB at 32 heads,
+    1.75 KB at 64), 1 KB of alignment slack, Q [nh][128], 3 K and 3 V stages of 128 tokens x
+    128, and two P buffers [128][nh] (bf16) at 32 heads, one at 64."""
+    header, p_buffers = (2048, 2) if nh == 32 else (1792, 1)
+    return header + 1024 + nh * 128 * 2 + 6 * 128 * 128 * 2 + p_buffers * 128 * nh * 2
 
 
 @pytest.mark.parametrize("g", [32, 20, 48, 64])
