@@ -68,6 +68,13 @@ constexpr Traits share_traits_for(int D) {
 }
 template <int D>
 constexpr int kStages = traits_for(D).stages;
+
+// The unit kernel (one CTA per unit, or per split with fixed splits) at D = 32 takes 16 warps
+// x 2 stages: B = 16 at 268 MB of K/V, one CTA per unit, 46.7 -> 44.0 us against 12 x 3 (14 x 3
+// 46.1, 11 x 4 49.5).  The balanced split kernel keeps 12 x 3 (16 x 2 took 50.9 -> 52.0 us).
+constexpr Traits unit_traits_for(int D) { return D == 32 ? Traits{2, 16} : traits_for(D); }
+template <int D>
+constexpr int kUnitStages = unit_traits_for(D).stages;
 template <int D>
 constexpr int kShareStages = share_traits_for(D).stages;
 
@@ -77,6 +84,8 @@ static_assert(traits_for(32).max_warps <= apd::kMaxWarpsD<32, false> &&
                   traits_for(128).max_warps <= apd::kMaxWarpsD<128, false> &&
                   traits_for(256).max_warps <= apd::kMaxWarpsD<256, false>,
               "warps per CTA above the split kernel's launch bound");
+static_assert(unit_traits_for(32).max_warps <= apd::kMaxWarpsD<32, false>,
+              "warps per CTA above the unit kernel's launch bound");
 static_assert(share_traits_for(64).max_warps <= apd::kMaxWarpsD<64, true> &&
                   share_traits_for(128).max_warps <= apd::kMaxWarpsD<128, true> &&
                   share_traits_for(256).max_warps <= apd::kMaxWarpsD<256, true>,
@@ -165,8 +174,8 @@ struct Plan {
 // The unit kernel's geometry: the most warps (up to the head dim's maximum) whose rings fit.
 void unit_geometry(const Shape& s, Plan* pl) {
     pl->share = false;
-    pl->stages = traits_for(s.D).stages;
-    pl->warps = traits_for(s.D).max_warps;
+    pl->stages = unit_traits_for(s.D).stages;
+    pl->warps = unit_traits_for(s.D).max_warps;
     while (pl->warps > 1 && unit_smem_bytes(s, pl->warps, pl->stages) > kSmemLimit) --pl->warps;
     pl->smem = unit_smem_bytes(s, pl->warps, pl->stages);
 }
@@ -194,7 +203,7 @@ void cta_local_plan(const Shape& s, Plan* pl) {
 bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t* host_lens, int64_t len_cap) {
     if (s.units > sm_count || pl.ctas < 1 || s.HB > 1) return false;
     // a part's (m, l) and accumulator rows go to its warp's ring once the stream ends
-    if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(traits_for(s.D).stages) * stage_bytes(s))
+    if (128ull + 4ull * s.rows_max * (s.D + 8) > static_cast<size_t>(unit_traits_for(s.D).stages) * stage_bytes(s))
         return false;
     const int64_t ups = static_cast<int64_t>(s.Hkv) * s.HB;
     int64_t total = 0, longest = 0;
@@ -818,8 +827,8 @@ int launch(const Validated& V, const apd_tensor* q, const apd_tensor* k, const a
     if (pl.mode != 0) {
         // one CTA per unit (or per split of a unit): the lean per-tile form at D = 32 and 64
         // only (the plain form measured 1% faster for the llama8b shape at D = 128)
-        if (pl.mode == 1) kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64), true>;
-        else kern = apd::unit_kernel<D, kStagesD, (D == 32 || D == 64), false>;
+        if (pl.mode == 1) kern = apd::unit_kernel<D, kUnitStages<D>, (D == 32 || D == 64), true>;
+        else kern = apd::unit_kernel<D, kUnitStages<D>, (D == 32 || D == 64), false>;
         variant = pl.mode == 1 ? 3 : 2;
     }
     const int kSlot = ((D == 32) ? 0 : (D == 64) ? 1 : (D == 128) ? 2 : 3) + 4 * variant;

@@ -57,7 +57,7 @@ constexpr int kMaxWarps = 8;       // warps per CTA, upper bound (D >= 128, shar
 // and their register footprint leaves room for more warps: 12 at D = 32 and 10 at D = 64
 // with one ring per warp (the launch bound caps registers at 170 and 204).
 template <int D, bool SHARE>
-constexpr int kMaxWarpsD = SHARE ? kMaxWarps : (D == 32 ? 12 : (D == 64 ? 10 : kMaxWarps));
+constexpr int kMaxWarpsD = SHARE ? kMaxWarps : (D == 32 ? 16 : (D == 64 ? 10 : kMaxWarps));
 constexpr uint32_t kFlagPageOOR = 0x1u;
 constexpr uint32_t kFlagLenClamped = 0x2u;
 constexpr uint32_t kFlagLenNegative = 0x4u;

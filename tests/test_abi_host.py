@@ -229,6 +229,8 @@ def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
 # per head dim: async-copy stages and the most warps a CTA may have, with one ring per
 # warp and with a K/V ring shared by the head blocks of a kv head (None: not shared)
 _TRAITS = {32: (3, 12), 64: (2, 10), 128: (3, 6), 256: (2, 4)}
+# the unit kernel (one CTA per unit, or per fixed split): 16 warps x 2 stages at D = 32
+_UNIT_TRAITS = {**_TRAITS, 32: (2, 16)}
 _SHARE_TRAITS = {32: None, 64: (4, 8), 128: (2, 8), 256: (2, 4)}
 
 
@@ -265,7 +267,7 @@ def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     assert pl.warps_per_cta == ws[0] and pl.stages == stages
     assert pl.smem_bytes == _smem(B, D, rows, ws[0], stages, hb, shared)
     # fixed splits and the one-CTA-per-unit plan run the unit kernel: one ring per warp
-    stages, max_warps = _TRAITS[D]
+    stages, max_warps = _UNIT_TRAITS[D]
     uw = max(x for x in range(1, max_warps + 1) if _unit_smem(D, rows, x, stages) <= 232448)
     fixed = apd.query_plan(B, Hq, Hkv, D, 2, sm_count=148)
     assert fixed.shared_kv_ring == 0 and fixed.stages == stages and fixed.warps_per_cta == uw
@@ -340,7 +342,7 @@ def test_plan_unit_kernel_smem(B, Hq, Hkv, D, L):
     maximum) whose rings fit, and the unit kernel's shared-memory layout."""
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148, host_seq_lens=[L] * B, max_seq_len=L)
     assert pl.mode == 2
-    stages, max_warps = _TRAITS[D]
+    stages, max_warps = _UNIT_TRAITS[D]
     rows = min(Hq // Hkv, 16)
     w = max(x for x in range(1, max_warps + 1) if _unit_smem(D, rows, x, stages) <= 232448)
     assert pl.warps_per_cta == w and pl.stages == stages
@@ -670,7 +672,7 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
     Hq = Hkv * g
     hb = -(-g // 16)
     pl = apd.query_plan(B, Hq, Hkv, D, splits, sm_count=sm, host_seq_lens=[L] * B, max_seq_len=70000)
-    bound = {32: 12, 64: 10}.get(D, 8) if not pl.shared_kv_ring else 8
+    bound = {32: 16, 64: 10}.get(D, 8) if not pl.shared_kv_ring else 8
     if pl.mode == 3:
         bound = 11  # the tensor-core kernel at 64 heads: 2 softmax groups + 3 warps
     assert pl.smem_bytes <= 232448
