@@ -1,4 +1,4 @@
-// apd_decode_tc.cuh -- decode attention for kv heads shared by 32 query heads, on the
+// apd_decode_tc.cuh -- decode attention for kv heads shared by 17 to 64 query heads, on the
 // sm_100a fifth-generation tensor cores (tcgen05 + TMEM).
 //
 // Same operation as the split kernel (AstrAI commit log of csrc/kernels/attn_paged_decode.cu:
@@ -6,6 +6,7 @@
 // one combine kernel); this is the design for kv heads whose query heads fill a tensor-core
 // tile.  With g = 32 query heads per kv head, every K/V tile meets 32 query rows, twice the
 // 16 of one mma.sync head block; here the tile goes to the tensor core once for all of them.
+// The heads are padded to NH = 32 or 64 with zero Q rows, whose outputs are never written.
 //
 //  - A CTA owns one split of one (sequence b, kv head) unit: a contiguous run of the
 //    sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it.  With at most
@@ -15,34 +16,33 @@
 //    kernel, no partials in global memory).  With more splits the parts go to the
 //    fixed-split slots of o_part / ml_part and the combine kernel merges them.
 //  - Tokens are the M side of both products, query heads the N side:
-//      S^T[t][h]  = sum_d K[t][d] Q[h][d]        (M = 128 tokens, N = 32 heads, K = D;
+//      S^T[t][h]  = sum_d K[t][d] Q[h][d]        (M = 128 tokens, N = NH heads, K = D;
 //                                                 A = the K tile, B = Q, both K-major)
-//      O^T[d][h] += sum_t V[t][d] P^T[t][h]      (M = D, N = 32 heads, K = 128 tokens;
+//      O^T[d][h] += sum_t V[t][d] P^T[t][h]      (M = D, N = NH heads, K = 128 tokens;
 //                                                 A = the V tile read MN-major, B = P^T
 //                                                 MN-major: P stored [token][head])
-//    so the staged K and V tiles are used exactly as the TMA lands them and no query row of
-//    the MMA is padding.
+//    so the staged K and V tiles are used exactly as the TMA lands them.
 //  - Two producer warps (after the softmax warps) resolve each tile's four pages and issue
-//    the TMA loads of its K boxes and its V boxes into two rings, each refilled as soon as its
-//    own stage is free: a K stage right after its S^T product, a V stage after its P V.
+//    the TMA loads of its K boxes and its V boxes into two rings, each refilled as soon as
+//    its own stage is free: a K stage right after its S^T product, a V stage after its P V.
 //    One lane of the warp between them issues the MMAs, each product as soon as its operands
 //    are ready (S^T_j does not wait for P_{j-1} V_{j-1}, nor that for the next K tile), and
-//    commits them to the mbarriers that free the stages and hand S^T to the softmax warps.  Two S^T
-//    buffers (and at 32 heads two P buffers) let the softmax of tile j + 1 run while P_j V_j
-//    is on the tensor core.
+//    commits them to the mbarriers that free the stages and hand S^T to the softmax warps.
+//    Two S^T buffers (and at 32 heads two P buffers) let the softmax of tile j + 1 run while
+//    P_j V_j is on the tensor core.
 //  - Softmax warps, one group of 4 per 32 heads (warps 0-3, and 4-7 at 64 heads): TMEM lane t
 //    is token t of the tile, so thread t of a group reads its token's 32 scores of the
-//    group's heads with one tcgen05.ld and owns those exponentials.  The reference
-//    maximum of each head is shared by all tokens; it moves only when some score exceeds it
-//    by more than 2^8 (one OR-vote per tile and group over the group's named barrier; the
-//    head maxima are then reduced across its 128 threads, O^T and the running sums
-//    rescaled).  Each thread keeps
-//    its own running sums of the bf16 weights it wrote; they are added across the threads
-//    once, at the end.
+//    group's heads with one tcgen05.ld and owns those exponentials.  The reference maximum
+//    of each head is shared by all tokens (in shared memory); it moves only when some score
+//    exceeds it by more than 2^8 (one OR-vote per tile and group over the group's named
+//    barrier; the head maxima are then reduced across its 128 threads, O^T and the running
+//    sums rescaled).  Each thread keeps its own running sums of the bf16 weights it wrote;
+//    they are added across the threads once, at the end.
 //
 // Every mbarrier wait is bounded.  A wait that runs out raises a shared abort flag that every
 // role polls; the softmax warps decide to stop only through the result of a barrier
-// reduction, so they leave together, and all warps meet before the TMEM columns are freed.
+// reduction, so the warps of a group leave together, and all warps meet before the TMEM
+// columns are freed and, with the cluster merge, at the cluster barrier.
 #pragma once
 
 #include <cuda.h>
@@ -99,7 +99,7 @@ __device__ __forceinline__ void bar_named(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Reduce-scatter of NH = 32 values over the warp: afterwards v[0] of lane t holds the
+// Reduce-scatter of 32 values over the warp: afterwards v[0] of lane t holds the
 // reduction over the 32 lanes of value t (recursive halving: at offset o, a lane keeps the
 // upper half of its values when bit o of its lane index is set and takes the partner's
 // copy of them).
