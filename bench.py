@@ -4,7 +4,7 @@ One step = one decode-attention call (split kernel + combine kernel) over one
 batch of synthetic decode queries against a paged bf16 KV cache, through the
 C-ABI library.  Prints ONE JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|long|ragged|gqa32|tiny|...]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b|long|ragged|gqa32|gqa80|tiny|...]
     python bench.py --impl reference ...      # the fp64 CPU oracle, timed on the host cores
 
 Metric: achieved HBM bandwidth over algorithmic bytes (KV bytes that must be read
@@ -41,7 +41,7 @@ import workloads  # noqa: E402
 METRIC = "paged decode attention achieved HBM GB/s (algorithmic KV+q+out bytes per call / time)"
 UNIT = "GB/s"
 DEFAULT_STEPS = {"llama8b": 200, "long": 100, "ragged": 50, "tiny": 200, "llama8b_contig": 200,
-                 "long_contig": 100, "gqa32": 200}
+                 "long_contig": 100, "gqa32": 200, "gqa80": 100}
 DEFAULT_REFERENCE_STEPS = 20
 # measured beside the headline decode workload, in the same run (the other configurations with a
 # 70% target or a reported number)
@@ -141,7 +141,7 @@ def make_instances(name: str, rank: int, count: int = 2):
     table) and independent values; the seed of the values differs per rank and instance."""
     gen = workloads.NAMED[name]
     base = {"tiny": 1234, "llama8b": 8, "long": 131072, "ragged": 4262, "llama8b_contig": 8,
-            "long_contig": 131072, "gqa32": 32, "hd32": 77, "hd64": 77, "hd256": 77}[name]
+            "long_contig": 131072, "gqa32": 32, "gqa80": 80, "hd32": 77, "hd64": 77, "hd256": 77}[name]
     return [gen(seed=base, value_seed=base + 1000003 * rank + i) for i in range(count)]
 
 

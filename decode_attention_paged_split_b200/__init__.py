@@ -84,6 +84,8 @@ class _Plan(ctypes.Structure):
         ("workspace_bytes", ctypes.c_int64),
         ("shared_kv_ring", ctypes.c_int32),
         ("cluster_size", ctypes.c_int32),
+        ("q_head_blocks", ctypes.c_int32),
+        ("q_heads_per_block", ctypes.c_int32),
     ]
 
 
@@ -516,6 +518,8 @@ class Plan:
     workspace_bytes: int
     shared_kv_ring: int  # 1: a kv head's head-block warps read one K/V ring (balanced, g > 16)
     cluster_size: int = 0  # mode 3: CTAs per cluster that merge a unit's splits in the kernel
+    q_head_blocks: int = 1  # mode 3: CTAs per split of a (sequence, kv head), one per block of q heads
+    q_heads_per_block: int = 0  # mode 3: q heads of each block but the last (a multiple of 16)
 
 
 def query_plan(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_splits: int = 0,

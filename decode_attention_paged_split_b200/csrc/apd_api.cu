@@ -12,6 +12,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -93,6 +94,9 @@ static_assert(share_traits_for(64).max_warps <= apd::kMaxWarpsD<64, true> &&
 
 bool head_dim_ok(int D) { return D == 32 || D == 64 || D == 128 || D == 256; }
 
+// the binding mirrors apd_plan field by field
+static_assert(sizeof(apd_plan) == 72 && offsetof(apd_plan, q_heads_per_block) == 68, "apd_plan layout");
+
 struct Shape {
     int B, Hq, Hkv, D, g, HB, rows_max;
     int64_t units;  // B * Hkv * HB
@@ -162,6 +166,8 @@ int64_t slots_fitting(const Shape& s, size_t bytes) {
 struct Plan {
     int mode, ksplit, workers, groups, ctas, warps, stages, combine_ctas;
     int cluster = 0;  // mode 3: CTAs per cluster (the splits of a unit, merged over DSMEM), or 0
+    int hblocks = 1;  // mode 3: q-head blocks per kv head (CTAs per split of a (sequence, kv head))
+    int hb_heads = 0; // mode 3: q heads per block (a multiple of 16, at most 64)
     bool share;  // balanced mode, g > 16: a kv head's HB warps share one K/V ring
     size_t smem;
     int64_t slots;
@@ -218,29 +224,40 @@ bool cta_local_wins(const Shape& s, const Plan& pl, int sm_count, const int32_t*
     return 32 * longest <= 33 * share + 32 * (1024 / s.D);
 }
 
-// Tensor-core multi-query plan (mode 3, decode_mq_tc_kernel): kv heads with 17 to 64 query
-// heads at D = 128.  One CTA per split of each (sequence, kv head); its 128-token tiles meet
-// all the query heads (padded to NH = 32 or 64) in one tcgen05 MMA, where the split kernel
-// needs a head block of 16 per warp.  The partials take the fixed-split slots (the head
-// blocks' rows of each split), so the combine is the fixed-split one.
+// Tensor-core multi-query plan (mode 3, decode_mq_tc_kernel): kv heads with more than 16
+// query heads at D = 128.  One CTA per split of each (sequence, kv head, q-head block); its
+// 128-token tiles meet all the block's query heads (padded to NH = 32 or 64) in one tcgen05
+// MMA, where the split kernel needs a head block of 16 per warp.  Up to 64 query heads are
+// one block; above that, ceil(g / 64) blocks of ceil(g / blocks) heads rounded up to 16, so
+// that every block starts on a 16-row boundary of the partial slots.  The partials take the
+// fixed-split slots (the 16-row head blocks' rows of each split), so the combine is the
+// fixed-split one.
 template <int NH>
 using McShapeT = apd::McShape<128, NH>;
 
+constexpr int kMcBlockHeads = 64;  // most q heads of one tensor-core decode CTA
+int mq_tc_hblocks(const Shape& s) { return (s.g + kMcBlockHeads - 1) / kMcBlockHeads; }
+int mq_tc_block_heads(const Shape& s) {
+    const int nb = mq_tc_hblocks(s);
+    return ((s.g + nb - 1) / nb + apd::kMaxRows - 1) / apd::kMaxRows * apd::kMaxRows;
+}
 // NH of the tensor-core kernel for this shape, or 0 when the shape does not take it
-int mq_tc_heads(const Shape& s) { return s.D == 128 && s.g > 16 && s.g <= 64 ? (s.g <= 32 ? 32 : 64) : 0; }
+int mq_tc_heads(const Shape& s) {
+    return s.D == 128 && s.g > 16 ? (mq_tc_block_heads(s) <= 32 ? 32 : 64) : 0;
+}
 bool mq_tc_eligible(const Shape& s) { return mq_tc_heads(s) > 0; }
 // Co-resident clusters of k tensor-core decode CTAs, per NH (index 0: 32 heads, 1: 64).
 struct McCaps {
     int c[2][apd::kMcMaxCluster + 1];
 };
 
-// Splits per unit with automatic splitting: the (sequence, kv head) units spread over 7/8
-// of the SMs (the rate at which D = 128 streams best, as in the balanced plan), at most one
-// split per 128-token tile the page table can address, and no more than the workspace
-// holds.  Returns 0 when the workspace holds no partials at all and the unit count needs
-// some.
+// Splits per unit with automatic splitting: the (sequence, kv head, q-head block) units
+// spread over 7/8 of the SMs (the rate at which D = 128 streams best, as in the balanced
+// plan), at most one split per 128-token tile the page table can address, and no more than
+// the workspace holds.  Returns 0 when the workspace holds no partials at all and the unit
+// count needs some.
 int64_t mq_tc_auto_splits(const Shape& s, int sm_count, size_t ws_bytes, int64_t tiles_bound) {
-    const int64_t u2 = static_cast<int64_t>(s.B) * s.Hkv;
+    const int64_t u2 = static_cast<int64_t>(s.B) * s.Hkv * mq_tc_hblocks(s);
     int64_t k = std::max<int64_t>(1, static_cast<int64_t>(sm_count) * 7 / 8 / std::max<int64_t>(1, u2));
     if (tiles_bound >= 0) {
         const int64_t per_unit = tiles_bound / std::max<int64_t>(1, s.units);  // 32-token tiles
@@ -263,7 +280,7 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
 int mq_tc_cluster(const Shape& s, int64_t k, int sm_count, const McCaps* caps) {
     if (k < 2 || k > apd::kMcMaxCluster) return 0;
     const int64_t cap = caps ? caps->c[mq_tc_heads(s) == 64 ? 1 : 0][k] : sm_count / k;
-    return static_cast<int64_t>(s.B) * s.Hkv <= cap ? static_cast<int>(k) : 0;
+    return static_cast<int64_t>(s.B) * s.Hkv * mq_tc_hblocks(s) <= cap ? static_cast<int>(k) : 0;
 }
 
 // Warps of a combine CTA: enough for one batch of kCombineBatch partial slots per warp,
@@ -305,7 +322,9 @@ void mq_tc_plan(const Shape& s, int64_t ksplit, int sm_count, int cluster, Plan*
     pl->warps = (h64 ? McShapeT<64>::kThreads : McShapeT<32>::kThreads) / 32;
     pl->stages = h64 ? McShapeT<64>::kVStages : McShapeT<32>::kVStages;
     pl->smem = h64 ? McShapeT<64>::kSmemBytes : McShapeT<32>::kSmemBytes;
-    pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * ksplit);
+    pl->hblocks = mq_tc_hblocks(s);
+    pl->hb_heads = mq_tc_block_heads(s);
+    pl->ctas = static_cast<int>(static_cast<int64_t>(s.B) * s.Hkv * pl->hblocks * ksplit);
     pl->workers = pl->ctas;
     // the partial slots are reserved whether or not the merge runs over DSMEM, so that the
     // workspace a split count needs does not depend on the device's cluster placement
@@ -327,7 +346,7 @@ int make_plan(const Shape& s, int num_splits, int sm_count, size_t ws_bytes, int
     if (num_splits < 0) return APD_ERR_NUM_SPLITS;
     if (allow_tc && mq_tc_eligible(s)) {
         const int64_t k = num_splits > 0 ? num_splits : mq_tc_auto_splits(s, sm_count, ws_bytes, tiles_bound);
-        if (static_cast<int64_t>(s.B) * s.Hkv * k > INT32_MAX / 64) return APD_ERR_TOO_LARGE;
+        if (static_cast<int64_t>(s.B) * s.Hkv * mq_tc_hblocks(s) * k > INT32_MAX / 64) return APD_ERR_TOO_LARGE;
         mq_tc_plan(s, k, sm_count, mq_tc_cluster(s, k, sm_count, cluster_caps), pl);
         pl->ws_needed = ws_bytes_for(s, pl->slots);
         if (ws_bytes != SIZE_MAX && ws_bytes < pl->ws_needed) return APD_ERR_WORKSPACE;
@@ -743,6 +762,8 @@ int launch_mq_tc(const Validated& V, const apd_tensor* q, const apd_tensor* k, c
     mp.P = V.P;
     mp.NP = V.NP;
     mp.MP = V.MP;
+    mp.nhb = pl.hblocks;
+    mp.hbh = pl.hb_heads;
     mp.ksplit = pl.ksplit;
     mp.cluster = pl.cluster > 0 ? 1 : 0;
     mp.scale_log2 = scale * 1.4426950408889634f;
@@ -1652,6 +1673,8 @@ int apd_query_plan_ex(int batch, int num_q_heads, int num_kv_heads, int head_dim
     plan->workspace_bytes = static_cast<int64_t>(pl.ws_needed);
     plan->shared_kv_ring = pl.share ? 1 : 0;
     plan->cluster_size = pl.cluster;
+    plan->q_head_blocks = pl.mode == 3 ? pl.hblocks : 1;
+    plan->q_heads_per_block = pl.mode == 3 ? pl.hb_heads : 0;
     return APD_OK;
 }
 

@@ -1,5 +1,5 @@
-// apd_decode_tc.cuh -- decode attention for kv heads shared by 17 to 64 query heads, on the
-// sm_100a fifth-generation tensor cores (tcgen05 + TMEM).
+// apd_decode_tc.cuh -- decode attention for kv heads shared by more than 16 query heads, on
+// the sm_100a fifth-generation tensor cores (tcgen05 + TMEM).
 //
 // Same operation as the split kernel (AstrAI commit log of csrc/kernels/attn_paged_decode.cu:
 // one query token per sequence, paged bf16 K/V, split-KV partials o_part / ml_part merged by
@@ -7,9 +7,13 @@
 // tile.  With g = 32 query heads per kv head, every K/V tile meets 32 query rows, twice the
 // 16 of one mma.sync head block; here the tile goes to the tensor core once for all of them.
 // The heads are padded to NH = 32 or 64 with zero Q rows, whose outputs are never written.
+// Above 64 query heads per kv head the heads are cut into nhb = ceil(g / 64) blocks of
+// equal size rounded up to 16 heads (g = 80: 48 + 32), one CTA per block and split.  The
+// blocks' CTAs of one split read the same K/V tiles; when they run at the same time (the
+// automatic split count keeps every CTA in one wave) the later reads are L2 hits.
 //
-//  - A CTA owns one split of one (sequence b, kv head) unit: a contiguous run of the
-//    sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it.  With at most
+//  - A CTA owns one split of one (sequence b, kv head, q-head block) unit: a contiguous run
+//    of the sequence's 32-token boxes, cut exactly as the fixed-split plan cuts it.  With at most
 //    8 splits per unit the splits of a unit form one thread-block cluster: each split leaves
 //    its unnormalised part in its own shared memory, and split c then merges heads c, c + nk,
 //    c + 2 nk, ... of all nk parts over distributed shared memory and writes them out (one
@@ -67,7 +71,8 @@ struct McParams {
     float* ml_part;  // [slots][rows_max][2]
     uint32_t* flags;
     int32_t B, Hkv, g, HB, rows_max, P, NP, MP;
-    int32_t ksplit;   // splits per (sequence, kv head)
+    int32_t nhb, hbh; // q-head blocks per kv head, q heads per block (a multiple of 16, <= NH)
+    int32_t ksplit;   // splits per (sequence, kv head, q-head block)
     int32_t cluster;  // 1: the ksplit CTAs of a unit are one cluster and merge over DSMEM
     float scale_log2;
     uint64_t wait_ns;         // limit of each wait (kWaitTimeoutNs; shorter in the self-test)
@@ -257,12 +262,18 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     const uint32_t q_s = tb + T::kQOff, p_s = tb + T::kPOff;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- work item: split `split` of unit (sequence b, kv head kvh)
+    // ---- work item: split `split` of q-head block hb of unit (sequence b, kv head kvh); the
+    // block holds q heads h0 .. h0 + gh - 1 of the kv head's g
     const int nsplit = p.ksplit;
-    const int u2 = blockIdx.x / nsplit;
-    const int split = blockIdx.x - u2 * nsplit;
+    const int ub = blockIdx.x / nsplit;
+    const int split = blockIdx.x - ub * nsplit;
+    const int u2 = ub / p.nhb;
+    const int hb = ub - u2 * p.nhb;
     const int b = u2 / p.Hkv;
     const int kvh = u2 - b * p.Hkv;
+    const int h0 = hb * p.hbh;
+    const int gh = min(p.hbh, p.g - h0);
+    const int qh0 = kvh * p.g + h0;  // first q head of the block
 
     if (threadIdx.x == 0) {
         mbar_init(bar(kQFull), kSoftThreads);
@@ -304,7 +315,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     const int64_t cap = static_cast<int64_t>(p.MP) * p.P;
     int L = __ldcg(p.seq_lens + b);
     if (L < 0 || L > cap) {
-        if (threadIdx.x == 0 && split == 0) atomicOr(p.flags, L < 0 ? kFlagLenNegative : kFlagLenClamped);
+        if (threadIdx.x == 0 && split == 0 && hb == 0)
+            atomicOr(p.flags, L < 0 ? kFlagLenNegative : kFlagLenClamped);
         L = L < 0 ? 0 : static_cast<int>(cap);
     }
     const int n32 = (L + kTile - 1) / kTile;
@@ -319,10 +331,10 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
     if (c0 >= c1) {
         // an empty split writes nothing; split 0 of an empty sequence writes its zero rows
         if (split == 0) {
-            for (int i = threadIdx.x; i < p.g * (D / 8); i += blockDim.x) {
+            for (int i = threadIdx.x; i < gh * (D / 8); i += blockDim.x) {
                 const int h = i / (D / 8), ch = i - h * (D / 8);
-                *reinterpret_cast<uint4*>(p.out + b * p.out_sb + (kvh * p.g + h) * p.out_sh + 8 * ch) =
-                    make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(p.out + b * p.out_sb + static_cast<int64_t>(qh0 + h) * p.out_sh +
+                                          8 * ch) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
         if (p.cluster) {
@@ -481,8 +493,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         const int hoff = 32 * grp;
         const int gbar = 1 + grp;  // this group's named barrier
         const uint32_t t_lane = static_cast<uint32_t>(32 * wq) << 16;
-        // Q rows kvh * g + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at and past
-        // g (padding up to NH) are zeros.  A thread's loads are all issued before its stores.
+        // Q rows kvh * g + h0 + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at and
+        // past gh (padding up to NH) are zeros.  A thread's loads are all issued before its stores.
         {
             constexpr int kPer = NH * (D / 8) / kSoftThreads;  // 16-byte chunks per thread
             static_assert(NH * (D / 8) % kSoftThreads == 0, "Q chunks per thread");
@@ -491,9 +503,9 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
             for (int u = 0; u < kPer; ++u) {
                 const int idx = threadIdx.x + u * kSoftThreads;
                 const int h = idx / (D / 8), ch = idx - h * (D / 8);
-                v[u] = h < p.g ? __ldg(reinterpret_cast<const uint4*>(p.q + b * p.q_sb + (kvh * p.g + h) * p.q_sh +
-                                                                      8 * ch))
-                               : make_uint4(0u, 0u, 0u, 0u);
+                v[u] = h < gh ? __ldg(reinterpret_cast<const uint4*>(
+                                    p.q + b * p.q_sb + static_cast<int64_t>(qh0 + h) * p.q_sh + 8 * ch))
+                              : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
@@ -721,25 +733,26 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int h = hoff + i;
-                    if (h < p.g)
-                        p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                    if (h < gh)
+                        p.out[b * p.out_sb + static_cast<int64_t>(qh0 + h) * p.out_sh + dd] =
                             __float2bfloat16_rn(__uint_as_float(o[i]) / lt[i]);
                 }
             }
         } else if (!p.cluster) {
             if (!any_gave_up) {
-                // the partial of this split, for each head block of 16 heads: slot
-                // ((b * Hkv + kvh) * HB + hb) * ksplit + split, row h - 16 hb
+                // the partial of this split, for each block of 16 q heads (h0 is a multiple of
+                // 16): slot ((b * Hkv + kvh) * HB + hh / 16) * ksplit + split, row hh % 16 of
+                // q head hh = h0 + h of the kv head
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int h = hoff + i;
-                    if (h < p.g) {
+                    const int h = h0 + hoff + i;
+                    if (hoff + i < gh) {
                         const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
                         p.o_part[(slot * p.rows_max + h % kMaxRows) * D + dd] = __uint_as_float(o[i]);
                     }
                 }
-                if (wq == 0 && hoff + lane < p.g) {
-                    const int h = hoff + lane;
+                if (wq == 0 && hoff + lane < gh) {
+                    const int h = h0 + hoff + lane;
                     const int64_t slot = (static_cast<int64_t>(u2) * p.HB + h / kMaxRows) * p.ksplit + split;
                     *reinterpret_cast<float2*>(p.ml_part + (slot * p.rows_max + h % kMaxRows) * 2) =
                         make_float2(mm, ll);
@@ -812,8 +825,8 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
 #pragma unroll
                     for (int jj = 0; jj < kMaxH; ++jj) {
                         const int h = split + jj * nk;
-                        if (jj < nh && h < p.g)
-                            p.out[b * p.out_sb + (kvh * p.g + h) * p.out_sh + dd] =
+                        if (jj < nh && h < gh)
+                            p.out[b * p.out_sb + static_cast<int64_t>(qh0 + h) * p.out_sh + dd] =
                                 __float2bfloat16_rn(acc[jj] * wts[kMcMaxCluster * NH + jj]);
                     }
                 }

@@ -433,8 +433,8 @@ int apd_selftest_shared_ring_release(const apd_tensor* q, const apd_tensor* k_ca
 
 /*
  * apd_selftest_mq_tc_stall -- exercises, on the GPU and without any fault, the error path
- * of the tensor-core multi-query kernel (apd_plan.mode 3: 17 to 64 q heads per kv head at
- * head_dim 128).  It runs apd_attn_paged_decode(num_splits) on the given problem with two
+ * of the tensor-core multi-query kernel (apd_plan.mode 3: more than 16 q heads per kv head
+ * at head_dim 128).  It runs apd_attn_paged_decode(num_splits) on the given problem with two
  * differences: the softmax warps never hand over the weights P of their second tile, and
  * every wait gives up after `short_timeout_ns` (1 .. 1e9 ns) instead of 2 s.  The MMA
  * issuer and the softmax warps must then give up, raise the CTA's abort flag, leave their
@@ -459,10 +459,10 @@ typedef struct apd_plan {
                                   2 = one CTA per unit, parts merged in shared memory
                                   (num_splits == 0 with host lengths, see
                                   apd_launch_options.host_seq_lens),
-                                  3 = tensor-core multi-query kernel (17 to 64 q
-                                  heads per kv head at head_dim 128, any
+                                  3 = tensor-core multi-query kernel (more than
+                                  16 q heads per kv head at head_dim 128, any
                                   num_splits): one CTA per split of each
-                                  (sequence, kv head)                           */
+                                  (sequence, kv head, q-head block)             */
     int32_t num_workers;       /* warps that each own a run of tiles             */
     int32_t grid_ctas;         /* CTAs of the split kernel                       */
     int32_t warps_per_cta;
@@ -482,6 +482,12 @@ typedef struct apd_plan {
     int32_t cluster_size;      /* mode 3: the splits of a unit run as one thread-block
                                   cluster of this many CTAs and merge in the kernel
                                   (no combine kernel); 0 otherwise               */
+    int32_t q_head_blocks;     /* mode 3: CTAs per split of a (sequence, kv head),
+                                  each owning one block of its query heads:
+                                  ceil(g / 64); 1 otherwise                      */
+    int32_t q_heads_per_block; /* mode 3: query heads of a block but the last,
+                                  ceil(g / q_head_blocks) rounded up to 16; 0
+                                  otherwise                                      */
 } apd_plan;
 
 /* apd_query_plan -- fills *plan.  workspace_bytes: the size that will be passed

@@ -201,8 +201,13 @@ def test_workspace_size_invalid_is_zero():
         apd.workspace_size(2, 6, 4, 64)
 
 
+def test_plan_struct_layout():
+    # the C struct apd_plan and its ctypes mirror: 8 int32, 3 int64, 4 int32
+    assert ctypes.sizeof(apd._Plan) == 72 and apd._Plan.q_heads_per_block.offset == 68
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,D", [(16, 32, 8, 128), (2, 32, 8, 128), (128, 64, 8, 128), (4, 8, 8, 32),
-                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 64), (8, 160, 2, 128)])
+                                        (4, 32, 8, 256), (3, 40, 2, 64), (16, 64, 2, 64), (8, 160, 2, 64)])
 def test_plan_balanced_fills_the_device(B, Hq, Hkv, D):
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=148)
     g = Hq // Hkv
@@ -247,7 +252,7 @@ def _smem(B, D, rows, warps, stages, hb, shared):
     return -(-meta // 16) * 16 + 1024 + rings
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 160, 2, 128), (4, 192, 2, 128), (4, 64, 1, 64), (4, 80, 1, 32),
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(4, 160, 2, 64), (4, 192, 2, 256), (4, 64, 1, 64), (4, 80, 1, 32),
                                         (4, 64, 2, 256), (4, 32, 8, 128), (4, 16, 1, 64)])
 def test_plan_shared_kv_ring(B, Hq, Hkv, D):
     # balanced mode with g > 16: the head blocks of a kv head share one K/V ring, so the
@@ -286,24 +291,29 @@ def _mc_smem(nh):
     return header + 1024 + nh * 128 * 2 + 6 * 128 * 128 * 2 + p_buffers * 128 * nh * 2
 
 
-@pytest.mark.parametrize("g", [32, 20, 48, 64])
+@pytest.mark.parametrize("g", [32, 20, 48, 64, 65, 80, 96, 128, 200])
 @pytest.mark.parametrize("B,Hkv,sm", [(16, 2, 148), (1, 1, 148), (4, 8, 148), (200, 1, 148), (3, 2, 132), (16, 2, 8)])
 def test_plan_tensor_core_multi_query(B, Hkv, sm, g):
-    """17 to 64 q heads per kv head at D = 128: the tensor-core multi-query kernel (heads
-    padded to 32 or 64), one CTA per split of each (sequence, kv head), 7 or 11 warps (4
-    softmax warps per 32 heads, 2 producers, 1 MMA issuer), K and V rings of 128-token
-    stages, Q and two P buffers in shared memory.  Auto splits
-    spread the units over 7/8 of the SMs.  A unit's splits (up to 8) that the device can run
-    as one cluster merge over DSMEM in the kernel; otherwise their partials take the
-    fixed-split slots of both head blocks and the combine kernel merges them.  The slots are
-    reserved either way."""
+    """More than 16 q heads per kv head at D = 128: the tensor-core multi-query kernel.
+    The q heads of a kv head form nb = ceil(g / 64) blocks of ceil(g / nb) heads rounded
+    up to 16 (the last block takes the rest), each padded to 32 or 64; one CTA per split of
+    each (sequence, kv head, block), 7 or 11 warps (4 softmax warps per 32 heads, 2
+    producers, 1 MMA issuer), K and V rings of 128-token stages, Q and two P buffers in
+    shared memory.  Auto splits spread the (sequence, kv head, block) units over 7/8 of the
+    SMs.  A unit's splits (up to 8) that the device can run as one cluster merge over DSMEM
+    in the kernel; otherwise their partials take the fixed-split slots of the 16-row head
+    blocks and the combine kernel merges them.  The slots are reserved either way."""
     Hq, D = g * Hkv, 128
-    nh = 32 if g <= 32 else 64
+    nb = -(-g // 64)
+    per_block = -(-(-(-g // nb)) // 16) * 16
+    assert per_block <= 64 and (nb - 1) * per_block < g
+    nh = 32 if per_block <= 32 else 64
     units = B * Hkv * -(-g // 16)
     pl = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm)
-    k = max(1, sm * 7 // 8 // (B * Hkv))
+    k = max(1, sm * 7 // 8 // (B * Hkv * nb))
     assert pl.mode == 3 and pl.shared_kv_ring == 0
-    assert pl.grid_ctas == B * Hkv * k and pl.num_workers == pl.grid_ctas
+    assert pl.q_head_blocks == nb and pl.q_heads_per_block == per_block
+    assert pl.grid_ctas == B * Hkv * nb * k and pl.num_workers == pl.grid_ctas
     # a softmax group of 4 warps per 32 heads, 2 producer warps and the MMA issuer's warp
     assert pl.warps_per_cta == 4 * (nh // 32) + 3 and pl.stages == 3
     assert pl.smem_bytes == _mc_smem(nh) <= 232448
@@ -311,18 +321,18 @@ def test_plan_tensor_core_multi_query(B, Hkv, sm, g):
     assert pl.partial_slots == (units * k if k > 1 else 0)
     # up to 8 splits of a unit that fit the device as one cluster each merge in the kernel
     # (with an SM count given, every k SMs are taken to hold a cluster of k)
-    cl = k if 2 <= k <= 8 and B * Hkv <= sm // k else 0
+    cl = k if 2 <= k <= 8 and B * Hkv * nb <= sm // k else 0
     assert pl.cluster_size == cl
     assert pl.combine_ctas == (0 if k == 1 or cl else min(units, 4 * sm) if k <= 4 else units * 16)
     for S in (1, 3, 8, 12):
         f = apd.query_plan(B, Hq, Hkv, D, S, sm_count=sm)
-        assert f.mode == 3 and f.grid_ctas == B * Hkv * S and f.partial_slots == (units * S if S > 1 else 0)
-        assert f.cluster_size == (S if 2 <= S <= 8 and B * Hkv <= sm // S else 0)
+        assert f.mode == 3 and f.grid_ctas == B * Hkv * nb * S and f.partial_slots == (units * S if S > 1 else 0)
+        assert f.cluster_size == (S if 2 <= S <= 8 and B * Hkv * nb <= sm // S else 0)
     # a workspace that holds fewer partials caps the splits; one with none gives one split
     small = apd.query_plan(B, Hq, Hkv, D, 0, sm_count=sm, workspace_bytes=4096)
-    assert small.mode == 3 and small.grid_ctas == B * Hkv and small.partial_slots == 0
+    assert small.mode == 3 and small.grid_ctas == B * Hkv * nb and small.partial_slots == 0
     # other head dims and group sizes keep the mma.sync kernels
-    for Hq2, D2 in ((g * Hkv, 64), (80 * Hkv, 128), (16 * Hkv, 128)):
+    for Hq2, D2 in ((g * Hkv, 64), (g * Hkv, 256), (16 * Hkv, 128)):
         assert apd.query_plan(B, Hq2, Hkv, D2, 0, sm_count=sm).mode != 3
 
 
@@ -658,7 +668,7 @@ def test_gemv_plan_rejects_bad_shapes():
 
 
 @settings(max_examples=300, deadline=None)
-@given(B=st.integers(1, 300), Hkv=st.sampled_from([1, 2, 4, 8, 16]), g=st.integers(1, 80),
+@given(B=st.integers(1, 300), Hkv=st.sampled_from([1, 2, 4, 8, 16]), g=st.integers(1, 200),
        D=st.sampled_from([32, 64, 128, 256]), sm=st.sampled_from([1, 8, 132, 148]),
        splits=st.sampled_from([0, 0, 1, 3]), L=st.integers(0, 70000))
 def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
@@ -692,9 +702,13 @@ def test_plan_invariants(B, Hkv, g, D, sm, splits, L):
         assert splits > 0 and pl.grid_ctas == units * splits
         assert pl.num_workers == pl.grid_ctas * pl.warps_per_cta
     elif pl.mode == 3:
-        # the tensor-core multi-query kernel: one CTA per split of each (sequence, kv head)
-        assert D == 128 and 16 < g <= 64 and pl.grid_ctas % (B * Hkv) == 0
-        k = pl.grid_ctas // (B * Hkv)
+        # the tensor-core multi-query kernel: one CTA per split of each (sequence, kv head,
+        # block of at most 64 q heads)
+        nb = -(-g // 64)
+        assert D == 128 and g > 16 and pl.q_head_blocks == nb and pl.grid_ctas % (B * Hkv * nb) == 0
+        assert pl.q_heads_per_block % 16 == 0 and pl.q_heads_per_block <= 64
+        assert (nb - 1) * pl.q_heads_per_block < g <= nb * pl.q_heads_per_block
+        k = pl.grid_ctas // (B * Hkv * nb)
         assert k == splits or splits == 0
         assert pl.partial_slots == (units * k if k > 1 else 0)
         assert pl.cluster_size in (0, k) and (pl.cluster_size == 0 or 2 <= k <= 8)

@@ -1,6 +1,7 @@
-"""GPU parity of the tensor-core multi-query decode (plan mode 3: 17 to 64 q heads per kv head
-at D = 128, decode_mq_tc_kernel with the heads padded to 32 or 64, merged in a cluster or by
-the fixed-split combine) against the fp64 CPU oracle.
+"""GPU parity of the tensor-core multi-query decode (plan mode 3: more than 16 q heads per kv
+head at D = 128, decode_mq_tc_kernel with the heads padded to 32 or 64, above 64 cut into
+blocks of q heads, merged in a cluster or by the fixed-split combine) against the fp64 CPU
+oracle.
 
 Per output element |gpu - ref| <= 1e-2 + 1e-2 |ref| (ref = fp64 oracle value), as for every
 decode path.  Covered: automatic and fixed split counts (one split per unit, partial 128-token
@@ -8,8 +9,9 @@ tiles at the ends of splits, splits that get no token), lengths around the 32- a
 tile edges with empty sequences, NaN-poisoned unused slots, pages of 64 tokens, HND storage,
 the contiguous cache (bit-identical to the same tokens paged), scores with large outliers
 and a large scale (the reference maximum moves mid-stream and O is rescaled), determinism,
-CUDA-graph replay, the device-side contract flags, and the full-size 32-heads-per-kv-head
-workload in the launch configuration the benchmark times.
+CUDA-graph replay, the device-side contract flags, group sizes from 20 to 200 q heads per kv
+head, and the full-size 32- and 80-heads-per-kv-head workloads in the launch configuration
+the benchmark times.
 """
 import numpy as np
 import pytest
@@ -164,4 +166,51 @@ def test_gqa32_full_size():
     dp = DeviceProblem(w)
     check_close(dp.run(0), ref, "gqa32 auto")
     check_close(dp.run(16), ref, "gqa32 S=16")
+    assert apd.read_device_flags(dp.workspace) == 0
+
+
+@pytest.mark.parametrize("g,Hkv", [(65, 2), (80, 2), (128, 1), (200, 1)])
+@pytest.mark.parametrize("S", [0, 1, 3, 16])
+def test_q_head_blocks(g, Hkv, S):
+    """More than 64 q heads per kv head: ceil(g / 64) blocks of q heads, one CTA per block
+    and split (65 -> 48 + 17, 80 -> 48 + 32, 128 -> 64 + 64, 200 -> 64 + 64 + 64 + 8), the
+    blocks after the first starting inside the 16-row slot layout of the partials.  Ragged
+    lengths with an empty sequence, poisoned slots, score outliers."""
+    w = small(14, 4, g * Hkv, Hkv, (1900, 0, 77, 640), pool=120, poison=True, k_outlier_frac=0.02,
+              k_outlier_mult=20.0)
+    pl = apd.query_plan(4, g * Hkv, Hkv, 128, S)
+    nb = -(-g // 64)
+    assert pl.q_head_blocks == nb and pl.grid_ctas % (4 * Hkv * nb) == 0
+    dp, out = run_mode3(w, S)
+    check_close(out, oracle.paged_decode(w), f"g={g} S={S}")
+    assert torch.all(out[1] == 0)
+    assert apd.read_device_flags(dp.workspace) == 0
+
+
+def test_q_head_blocks_contract_flags():
+    """Page-table and length violations seen by the CTA of every block of q heads are
+    flagged once in the shared flag word, and the other sequences stay exact."""
+    w = small(15, 3, 160, 2, (300, 64, 100), pool=20, max_pages_per_seq=10)
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    dp.page_table[1, 0] = w.num_pages + 3
+    dp.seq_lens[2] = -7
+    ws = apd.alloc_workspace(3, 160, 2, 128, 0)
+    apd.workspace_init(ws)
+    apd.attn_paged_decode(dp.q, dp.k, dp.v, dp.page_table, dp.seq_lens, dp.out, w.scale, 0, ws)
+    flags = apd.read_device_flags(ws)
+    assert flags & apd.FLAG_PAGE_OUT_OF_RANGE and flags & apd.FLAG_SEQ_LEN_NEGATIVE
+    out = dp.out.to(torch.float64).cpu().numpy()
+    assert np.isfinite(out).all() and np.all(out[2] == 0)
+    check_close(dp.out[[0]], ref[[0]], "untouched sequence")
+
+
+def test_gqa80_full_size():
+    w = workloads.gqa80()
+    pl = apd.query_plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, 0)
+    assert pl.mode == 3 and pl.q_head_blocks == 2 and pl.q_heads_per_block == 48
+    ref = oracle.paged_decode(w)
+    dp = DeviceProblem(w)
+    check_close(dp.run(0), ref, "gqa80 auto")
+    check_close(dp.run(16), ref, "gqa80 S=16")
     assert apd.read_device_flags(dp.workspace) == 0

@@ -152,8 +152,8 @@ def test_gqa_groups(Hq, Hkv, S):
 def test_shared_kv_ring(D, Hq, Hkv, ws_div):
     """Balanced mode with g = 20, 32, 48, 80 (2 to 5 head blocks per kv head): the head
     blocks of a kv head read one K/V ring (except D = 32, D = 256 with 5 head blocks, and
-    g <= 64 at D = 128, which takes the tensor-core multi-query kernel).  Ragged lengths with an empty sequence and a
-    partial last tile, NaN-poisoned unused slots; ws_div = 16 gives a workspace a sixteenth
+    D = 128, which takes the tensor-core multi-query kernel).  Ragged lengths with an empty
+    sequence and a partial last tile, NaN-poisoned unused slots; ws_div = 16 gives a workspace a sixteenth
     of the default, so fewer groups and runs of many tiles per warp (every stage's release
     barrier goes through many phases)."""
     lens = (1500, 0, 33, 777)
@@ -165,7 +165,7 @@ def test_shared_kv_ring(D, Hq, Hkv, ws_div):
     # D = 32 keeps one ring per warp; D = 256 takes at most 4 warps per CTA, so 5 head
     # blocks keep one ring per warp too
     shared = D != 32 and not (D == 256 and pl.head_blocks > 4)
-    if D == 128 and Hq // Hkv <= 64:
+    if D == 128:
         assert pl.mode == 3  # the tensor-core multi-query kernel (tests/test_mq_tc_gpu.py)
     else:
         assert pl.mode == 0 and pl.shared_kv_ring == int(shared)
@@ -174,7 +174,7 @@ def test_shared_kv_ring(D, Hq, Hkv, ws_div):
     assert apd.read_device_flags(ws) == 0
 
 
-@pytest.mark.parametrize("D,Hq,Hkv", [(128, 160, 2), (64, 48, 1)])
+@pytest.mark.parametrize("D,Hq,Hkv", [(64, 160, 2), (64, 48, 1), (256, 96, 2)])
 def test_shared_kv_ring_one_group(D, Hq, Hkv):
     """The shared K/V ring with a workspace that holds one worker group only: every warp
     streams all positions, units are written directly (no combine kernel), and the
@@ -488,7 +488,7 @@ def test_host_hint_cta_local_matches_oracle(D, Hq, Hkv):
     if Hq // Hkv <= 16:
         assert pl.mode == 2 and pl.combine_ctas == 0
     else:
-        assert pl.mode == (3 if D == 128 and Hq // Hkv <= 64 else 0)
+        assert pl.mode == (3 if D == 128 else 0)
     out, ws = run_hinted(w, lens)
     check_close(out, oracle.paged_decode(w), f"hint D={D} {Hq}/{Hkv}")
     assert apd.read_device_flags(ws) == 0

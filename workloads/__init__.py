@@ -444,6 +444,16 @@ def gqa32(seed: int = 32, **kw) -> Workload:
     return make(**args)
 
 
+def gqa80(seed: int = 80, **kw) -> Workload:
+    """B=16, 80 q heads / 1 kv head (two blocks of q heads for the tensor-core decode), D=128,
+    L=32768 each (268 MB of K/V, the llama8b byte count), shuffled pool."""
+    args = dict(name="gqa80_b16_h80x1_d128_l32768", seed=seed, batch=16, num_q_heads=80,
+                num_kv_heads=1, head_dim=128, page_size=32, seq_lens=[32768] * 16, pool_pages=16384,
+                num_splits=0)
+    args.update(kw)
+    return make(**args)
+
+
 def head_dim_scale(head_dim: int, seed: int = 77, **kw) -> Workload:
     """The llama8b shape (B=16, 32 q heads / 8 kv heads) at another head dim, with the
     sequence length that keeps 268 MB of K/V: L = 4096 * 128 / D, shuffled pool."""
@@ -461,6 +471,7 @@ NAMED = {
     "long": long_context,
     "ragged": ragged,
     "gqa32": gqa32,
+    "gqa80": gqa80,
     "llama8b_contig": llama8b_contig,
     "long_contig": long_contig,
     "hd32": lambda seed=77, **kw: head_dim_scale(32, seed, **kw),
