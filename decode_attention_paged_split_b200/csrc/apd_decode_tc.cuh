@@ -368,7 +368,9 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         const int full0 = kv ? kVFull : kKFull, empty0 = kv ? kVEmpty : kKEmpty;
         const int ST = kv ? VST : KST;
         const uint32_t ring = tb + (kv ? T::kVOff : T::kKOff);
-        const uint64_t pol = l2_policy_evict_first();  // every K/V byte is read once
+        // every K/V byte leaves HBM once: one CTA reads it, or the blocks' CTAs of one split
+        // read it about together (measured at g = 80: DRAM reads = the algorithmic bytes)
+        const uint64_t pol = l2_policy_evict_first();
         constexpr int kBoxes = TK / kTile;               // 4
         constexpr int kTB = 32 / kBoxes;                 // tiles whose pages one warp-wide load resolves
         int32_t pg = 0;
@@ -493,8 +495,9 @@ __global__ void __launch_bounds__(McShape<D, NH>::kThreads, 1)
         const int hoff = 32 * grp;
         const int gbar = 1 + grp;  // this group's named barrier
         const uint32_t t_lane = static_cast<uint32_t>(32 * wq) << 16;
-        // Q rows kvh * g + h0 + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at and
-        // past gh (padding up to NH) are zeros.  A thread's loads are all issued before its stores.
+        // Q rows kvh * g + h0 + h (h < NH) in the K-major B layout [D/64][NH][64]; rows at
+        // and past gh (padding up to NH) are zeros.  A thread's loads are all issued before
+        // its stores.
         {
             constexpr int kPer = NH * (D / 8) / kSoftThreads;  // 16-byte chunks per thread
             static_assert(NH * (D / 8) % kSoftThreads == 0, "Q chunks per thread");
