@@ -16,7 +16,9 @@
  *   stored positions.  The KV range of each (sequence, kv head) is split across
  *   workers (split-KV); each split leaves a partial output with its running max
  *   and sum, and one combine kernel merges them.  Query heads that share a kv
- *   head are processed together, so K/V are read once per kv head.
+ *   head are processed together, so K/V leave HBM once per kv head (above 64
+ *   query heads per kv head at head_dim 128, blocks of at most 64 of them read
+ *   the same tiles at about the same time, the repeats from L2).
  *
  * Ownership and threading.  The caller owns every buffer, including the
  * workspace.  The library allocates nothing, never synchronises the stream and
