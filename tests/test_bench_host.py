@@ -117,6 +117,26 @@ def test_instances_differ_per_rank_and_instance():
     assert r0.algorithmic_bytes() == r1.algorithmic_bytes() and not torch.equal(r0.q, r1.q)
 
 
+def test_every_named_workload_has_a_bench_seed_and_a_parser_choice():
+    # make_instances looks the workload's seed up before generating anything
+    for name in bench.workloads.NAMED:
+        assert bench.make_instances(name, 0, 0) == []
+        assert bench.parse_args(["--workload", name]).workload == name
+
+
+def test_committed_traffic_records_are_well_formed():
+    # one record per decode workload, each naming its kernel and command, with read + write
+    # bytes that add up; a stale record (older device code) is reported as null by the bench
+    with open(bench.TRAFFIC_FILE) as f:
+        recs = json.load(f)
+    names = [r["workload"] for r in recs]
+    assert len(names) == len(set(names)) and set(names) <= set(bench.workloads.NAMED)
+    for r in recs:
+        assert r["dram_bytes_per_launch"] == r["dram_bytes_read"] + r["dram_bytes_write"]
+        assert r["command"].startswith("ncu ") and "--clock-control none" in r["command"]
+        assert r["kernel"].startswith("apd::") and len(r["kernel_source_sha"]) == 16
+
+
 def test_reference_arm_prints_one_json_line():
     env = dict(os.environ)
     env.pop("WORLD_SIZE", None)
