@@ -43,9 +43,9 @@ UNIT = "GB/s"
 DEFAULT_STEPS = {"llama8b": 200, "long": 100, "ragged": 50, "tiny": 200, "llama8b_contig": 200,
                  "long_contig": 100, "gqa32": 200, "gqa80": 100}
 DEFAULT_REFERENCE_STEPS = 20
-# measured beside the headline decode workload, in the same run (the other configurations with a
-# 70% target or a reported number)
-PER_CONFIG = ("long", "ragged")
+# measured beside the headline decode workload, in the same run: the other configurations with a
+# 70% target or a reported number, and the multi-query shapes of the tensor-core decode kernel
+PER_CONFIG = ("long", "ragged", "gqa32", "gqa80")
 CSRC = os.path.join(ROOT, "decode_attention_paged_split_b200", "csrc")
 GEMV_METRIC = "decode projection GEMV achieved HBM GB/s (algorithmic W+x+y bytes per call / time)"
 GEMV_WORKLOADS = [f"gemv_{layer}_m{m}" for layer in workloads.GEMV_SHAPES for m in (1, 3, 8)]
